@@ -1,0 +1,376 @@
+"""CPU oracle for group-wise weight-only quantization (W4A16 / W3A16) and AWQ.
+
+TEST INFRASTRUCTURE ONLY. This is a plain, slow, obviously-correct numpy
+restatement of what the CUDA library computes. Only ``tests/``,
+``__graft_entry__.smoke()`` and the ``cpu_baseline`` / ``--impl reference``
+legs of ``bench.py`` may import it. It shares no code with the CUDA path:
+neither side imports the other; both take their inputs from ``synth``.
+
+Every function cites the web page (by title) and the section it restates.
+Pages cited:
+
+* [MIT-Lab4/5] "MIT 6.5940 Lab 4 + Lab 5: Quantizing an LLM with AWQ, Then
+  Running LLaMA2-7B on Your Own Laptop"
+* [CMU-L19/20] "CMU 11-868 L19-L20 Model Quantization: GPTQ Saves Memory, and
+  the Speedup Comes Along for the Ride"
+* [Quantising-LLMs] "Quantising Large Language Models for Efficient Inference"
+* [TinyChat] "TinyChat (AWQ on-device runtime)"
+* [160GB-Laptop] "LLM Quantization: 160GB Model on a Laptop"
+
+Floating-point contract (the pages fix none of it; these are this library's
+readings, identical on the GPU):
+
+* fp16 inputs are widened exactly to fp32. With AWQ scaling, w' = w * s_k in
+  fp32 (exact: an 11-bit by 11-bit significand product fits in 24 bits).
+* Every quantization decision (range, step, zero point, code) is taken in
+  IEEE fp32 with round-to-nearest-even: fp32 division, ``rint`` (ties to
+  even), integer add, clamp.
+* The per-group step is stored in fp16 rounded toward +inf, so the clamped
+  range never cuts off the group's extreme values.
+* Dequantized weights, matmul references and AWQ losses are computed in fp64.
+
+Pins: every function here is checked in ``tests/test_oracle_pins.py`` against
+values the pages print, closed forms, invariants or brute force; none is
+"parity unpinned".
+"""
+from __future__ import annotations
+
+
+import numpy as np
+
+__all__ = [
+    "f16_round_up",
+    "quantize_groups",
+    "dequantize",
+    "pack_codes",
+    "unpack_codes",
+    "packed_words_per_row",
+    "gemm_ref",
+    "absmax_quantize_int8",
+    "zeropoint_quantize_int8",
+    "activation_absmean",
+    "awq_alpha_grid",
+    "awq_candidates",
+    "awq_error_matrix",
+    "awq_loss",
+    "awq_search",
+    "MU_FLOOR",
+]
+
+
+# ---------------------------------------------------------------------------
+# fp16 rounding helper
+# ---------------------------------------------------------------------------
+
+def f16_round_up(v32: np.ndarray) -> np.ndarray:
+    """Smallest fp16 value >= each fp32 value (round toward +inf).
+
+    numpy's fp32->fp16 cast rounds to nearest-even; where that result lies
+    below the input, step to the next fp16 value upward.
+    """
+    v32 = np.asarray(v32, dtype=np.float32)
+    h = v32.astype(np.float16)
+    below = h.astype(np.float32) < v32
+    if np.any(below):
+        h = h.copy()
+        h[below] = np.nextafter(h[below], np.float16(np.inf))
+    return h
+
+
+# ---------------------------------------------------------------------------
+# Group-wise quantizer
+# ---------------------------------------------------------------------------
+
+def quantize_groups(W16: np.ndarray, bits: int, group: int, symmetric: bool,
+                    s16: np.ndarray | None = None):
+    """Round-to-nearest group-wise quantization of an [N][K] fp16 weight.
+
+    A group is ``group`` consecutive input channels (along K) of one output
+    row: [Quantising-LLMs] "Post-training methods for 4-bit weights" puts one
+    scale (and zero point) on each group of 64-128 weights within a row, and
+    its numpy routine reshapes each row into groups of that many entries.
+
+    Symmetric (absmax) branch -- [160GB-Laptop] "Symmetric Quantization" and
+    the [Quantising-LLMs] routine: qmax = 2^(b-1) - 1, step = max|w| / qmax,
+    code = clip(round(w / step), -qmax - 1, qmax), value = code * step.
+    Stored as unsigned code + 2^(b-1) with zero point 2^(b-1), so both
+    branches dequantize as (q - zero) * step.
+
+    Asymmetric branch -- [160GB-Laptop] "Asymmetric Quantization" maps
+    [min, max] onto [qmin, qmax] with step = (max - min) / (qmax - qmin);
+    [CMU-L19/20] "absmax and zero-point" writes the offset as a rounded
+    integer zero point and uses range := 1 when the range is 0. With
+    Q = 2^b - 1: mn = min(min w', 0), mx = max(max w', 0), r = mx - mn,
+    step = fp16_up(r / Q) (or 1 when r == 0), zero = clamp(rint(-mn/step), 0, Q),
+    q = clamp(rint(w'/step) + zero, 0, Q).
+
+    ``s16`` ([K] fp16, optional) applies AWQ's per-input-channel scaling
+    W * diag(s) before quantization ([MIT-Lab4/5] "Question 2").
+
+    Returns (codes uint8 [N][K], steps fp16 [N][K/group], zeros fp16 [N][K/group]).
+    """
+    W16 = np.asarray(W16)
+    assert W16.dtype == np.float16 and W16.ndim == 2
+    N, K = W16.shape
+    assert K % group == 0, "K must be a multiple of the group size"
+    assert 2 <= bits <= 8
+    w = W16.astype(np.float32)
+    if s16 is not None:
+        s16 = np.asarray(s16)
+        assert s16.dtype == np.float16 and s16.shape == (K,)
+        w = w * s16.astype(np.float32)[None, :]
+    G = K // group
+    wg = w.reshape(N, G, group)
+
+    if symmetric:
+        qmax = (1 << (bits - 1)) - 1
+        amax = np.abs(wg).max(axis=2)                      # fp32, exact
+        step_h = f16_round_up(amax / np.float32(qmax))
+        step_h = np.where(amax == 0, np.float16(1.0), step_h)
+        if not np.all(np.isfinite(step_h)):
+            raise OverflowError("group step does not fit fp16")
+        sf = step_h.astype(np.float32)[:, :, None]
+        qs = np.clip(np.rint(wg / sf), -qmax - 1, qmax).astype(np.int32)
+        codes = (qs + (1 << (bits - 1))).astype(np.uint8)
+        zeros = np.full((N, G), float(1 << (bits - 1)), dtype=np.float16)
+    else:
+        Q = (1 << bits) - 1
+        mn = np.minimum(wg.min(axis=2), np.float32(0))
+        mx = np.maximum(wg.max(axis=2), np.float32(0))
+        r = (mx - mn).astype(np.float32)                    # fp32 subtraction
+        step_h = f16_round_up(r / np.float32(Q))
+        step_h = np.where(r == 0, np.float16(1.0), step_h)
+        if not np.all(np.isfinite(step_h)):
+            raise OverflowError("group step does not fit fp16")
+        sf32 = step_h.astype(np.float32)
+        zero = np.clip(np.rint(-mn / sf32), 0, Q).astype(np.int32)
+        q = np.rint(wg / sf32[:, :, None]).astype(np.int32) + zero[:, :, None]
+        codes = np.clip(q, 0, Q).astype(np.uint8)
+        zeros = zero.astype(np.float16)
+    return codes.reshape(N, K), step_h.astype(np.float16), zeros
+
+
+def dequantize(codes: np.ndarray, steps: np.ndarray, zeros: np.ndarray, group: int) -> np.ndarray:
+    """fp64 weight (q - zero) * step for each element ([160GB-Laptop]
+    "Symmetric Quantization": dequantize = code * scale; the zero-point form of
+    [CMU-L19/20] "absmax and zero-point": (q - zp) / scale with scale a multiplier)."""
+    N, K = codes.shape
+    G = K // group
+    q = codes.astype(np.float64).reshape(N, G, group)
+    z = zeros.astype(np.float64)[:, :, None]
+    s = steps.astype(np.float64)[:, :, None]
+    return ((q - z) * s).reshape(N, K)
+
+
+# ---------------------------------------------------------------------------
+# Packed layouts
+# ---------------------------------------------------------------------------
+#
+# 4-bit: row-major [N][K/8] uint32. Word c of a row holds k = 8c..8c+7.
+#   Nibble slot j (bits 4j..4j+3) holds k = 8c + 2j for j < 4 and
+#   k = 8c + 2(j-4) + 1 for j >= 4, i.e. slot order [k0,k2,k4,k6,k1,k3,k5,k7].
+#   A mask of 0x000F000F over (word >> 4j) therefore yields the consecutive
+#   pair (k_2j, k_2j+1) in the two 16-bit halves. This is the same idea as
+#   TinyChatEngine's offline reordering ([MIT-Lab4/5] "Background: why the
+#   4-bit weights get reordered first"), redone for 16-bit GPU lanes.
+#
+# 3-bit: row-major [N][3K/32] uint32. Three words (t = 0, 1, 2) per 32 k:
+#   word t, pair j (0..4): bits 3j..3j+2 hold k = 32c + 10t + 2j, bits
+#   16+3j..18+3j hold k = 32c + 10t + 2j + 1; k = 32c+30 keeps its bit b in
+#   bit 15 of word b and k = 32c+31 keeps its bit b in bit 31 of word b.
+#   Exactly 3 bits per weight.
+
+def packed_words_per_row(K: int, bits: int) -> int:
+    if bits == 4:
+        assert K % 8 == 0
+        return K // 8
+    if bits == 3:
+        assert K % 32 == 0
+        return 3 * K // 32
+    raise ValueError("bits must be 3 or 4")
+
+
+def _pack4(codes: np.ndarray) -> np.ndarray:
+    N, K = codes.shape
+    c = codes.astype(np.uint32).reshape(N, K // 8, 8)
+    words = np.zeros((N, K // 8), dtype=np.uint32)
+    for j in range(4):
+        words |= c[:, :, 2 * j] << np.uint32(4 * j)
+        words |= c[:, :, 2 * j + 1] << np.uint32(4 * (j + 4))
+    return words
+
+
+def _unpack4(words: np.ndarray, K: int) -> np.ndarray:
+    N = words.shape[0]
+    w = words.reshape(N, K // 8)
+    out = np.zeros((N, K // 8, 8), dtype=np.uint8)
+    for j in range(4):
+        out[:, :, 2 * j] = (w >> np.uint32(4 * j)) & 0xF
+        out[:, :, 2 * j + 1] = (w >> np.uint32(4 * (j + 4))) & 0xF
+    return out.reshape(N, K)
+
+
+def _pack3(codes: np.ndarray) -> np.ndarray:
+    N, K = codes.shape
+    c = codes.astype(np.uint32).reshape(N, K // 32, 32)
+    words = np.zeros((N, K // 32, 3), dtype=np.uint32)
+    for t in range(3):
+        for j in range(5):
+            words[:, :, t] |= c[:, :, 10 * t + 2 * j] << np.uint32(3 * j)
+            words[:, :, t] |= c[:, :, 10 * t + 2 * j + 1] << np.uint32(16 + 3 * j)
+        words[:, :, t] |= ((c[:, :, 30] >> np.uint32(t)) & 1) << np.uint32(15)
+        words[:, :, t] |= ((c[:, :, 31] >> np.uint32(t)) & 1) << np.uint32(31)
+    return words.reshape(N, 3 * K // 32)
+
+
+def _unpack3(words: np.ndarray, K: int) -> np.ndarray:
+    N = words.shape[0]
+    w = words.reshape(N, K // 32, 3)
+    out = np.zeros((N, K // 32, 32), dtype=np.uint8)
+    for t in range(3):
+        for j in range(5):
+            out[:, :, 10 * t + 2 * j] = (w[:, :, t] >> np.uint32(3 * j)) & 7
+            out[:, :, 10 * t + 2 * j + 1] = (w[:, :, t] >> np.uint32(16 + 3 * j)) & 7
+        out[:, :, 30] |= (((w[:, :, t] >> np.uint32(15)) & 1) << np.uint32(t)).astype(np.uint8)
+        out[:, :, 31] |= (((w[:, :, t] >> np.uint32(31)) & 1) << np.uint32(t)).astype(np.uint8)
+    return out.reshape(N, K)
+
+
+def pack_codes(codes: np.ndarray, bits: int) -> np.ndarray:
+    """Pack b-bit codes [N][K] into the documented uint32 layout."""
+    assert codes.dtype == np.uint8
+    assert int(codes.max(initial=0)) < (1 << bits)
+    return _pack4(codes) if bits == 4 else _pack3(codes)
+
+
+def unpack_codes(words: np.ndarray, bits: int, K: int) -> np.ndarray:
+    return _unpack4(words, K) if bits == 4 else _unpack3(words, K)
+
+
+# ---------------------------------------------------------------------------
+# W4A16 / W3A16 matmul reference
+# ---------------------------------------------------------------------------
+
+def gemm_ref(X16: np.ndarray, codes: np.ndarray, steps: np.ndarray, zeros: np.ndarray,
+             group: int) -> np.ndarray:
+    """Y[m][n] = sum_k x[m][k] * (q[n][k] - zero) * step, in fp64.
+
+    This is the weight-only matmul of [Quantising-LLMs] "Weight-only vs
+    weight-and-activation quantisation" (16-bit activations, weights
+    dequantized inside the matmul), written as a plain fp64 matmul of the
+    dequantized weight; one library matmul is the only step.
+    """
+    D = dequantize(codes, steps, zeros, group)
+    return np.asarray(X16, dtype=np.float64) @ D.T
+
+
+# ---------------------------------------------------------------------------
+# int8 absmax / zero-point ([CMU-L19/20] "absmax and zero-point")
+# ---------------------------------------------------------------------------
+
+def absmax_quantize_int8(X: np.ndarray):
+    """Per-tensor int8 absmax: multiplier 127/max|X|, code = round(multiplier*X)
+    (round half to even), dequant = code / multiplier."""
+    X = np.asarray(X, dtype=np.float64)
+    mult = 127.0 / np.max(np.abs(X))
+    q = np.rint(mult * X)
+    return q.astype(np.int8), q / mult
+
+
+def zeropoint_quantize_int8(X: np.ndarray):
+    """Per-tensor int8 zero-point: range (1 if zero), multiplier 255/range,
+    zp = round(-multiplier*min - 128), code = clip(round(X*multiplier + zp), -128, 127),
+    dequant = (code - zp) / multiplier."""
+    X = np.asarray(X, dtype=np.float64)
+    rng_ = float(np.max(X) - np.min(X))
+    rng_ = 1.0 if rng_ == 0 else rng_
+    mult = 255.0 / rng_
+    zp = np.rint(-mult * np.min(X) - 128.0)
+    q = np.clip(np.rint(X * mult + zp), -128, 127)
+    return q.astype(np.int8), (q - zp) / mult
+
+
+# ---------------------------------------------------------------------------
+# AWQ: activation statistics, candidate scales, reconstruction loss, search
+# ---------------------------------------------------------------------------
+
+MU_FLOOR = 2.0 ** -14
+
+
+def activation_absmean(X16: np.ndarray) -> np.ndarray:
+    """mu_k = mean over calibration tokens of |x_tk|, in fp64.
+
+    [MIT-Lab4/5] "Starting point and setup": forward hooks record the mean
+    absolute value of each linear layer's input. Each fp16 value is a
+    multiple of 2^-24 below 2^16, so the fp64 sum of up to 2^13 of them is
+    exact in any order; one fp64 division by T follows.
+    """
+    X = np.asarray(X16)
+    assert X.dtype == np.float16
+    T = X.shape[0]
+    return np.abs(X.astype(np.float64)).sum(axis=0) / float(T)
+
+
+def awq_alpha_grid(n_alpha: int = 20) -> np.ndarray:
+    """alpha_j = j / n_alpha in fp64 (0, 0.05, ..., 0.95 for 20)."""
+    return np.arange(n_alpha, dtype=np.float64) / float(n_alpha)
+
+
+def awq_candidates(mu: np.ndarray, alphas: np.ndarray) -> np.ndarray:
+    """s_alpha,k = fp16_RN(max(mu_k, 2^-14) ** alpha), fp64 pow.
+
+    [MIT-Lab4/5] "Question 2": scale the salient (large-activation) input
+    channels up by s, computed from the activation statistic, and search over
+    the scale. The floor on mu keeps s > 0 on all-zero channels.
+    """
+    m = np.maximum(np.asarray(mu, dtype=np.float64), MU_FLOOR)
+    out = np.empty((len(alphas), m.shape[0]), dtype=np.float16)
+    for j, a in enumerate(alphas):
+        out[j] = np.power(m, float(a)).astype(np.float16)
+    return out
+
+
+def awq_error_matrix(W16: np.ndarray, s16: np.ndarray, bits: int, group: int,
+                     symmetric: bool) -> np.ndarray:
+    """E = W - Q(W diag(s)) diag(s)^-1 in fp64 ("scale up, quantize, scale
+    down" of [MIT-Lab4/5] "Question 2"; Q is quantize-then-dequantize, the
+    pseudo quantization of "Starting point and setup")."""
+    codes, steps, zeros = quantize_groups(W16, bits, group, symmetric, s16=s16)
+    Dq = dequantize(codes, steps, zeros, group)
+    return W16.astype(np.float64) - Dq / s16.astype(np.float64)[None, :]
+
+
+def awq_loss(X16: np.ndarray, Ws, s16: np.ndarray, bits: int, group: int,
+             symmetric: bool) -> float:
+    """L = sum over linears of || X E^T ||_F^2 in fp64.
+
+    The layer-wise reconstruction objective ||WX - W^X||^2 of [CMU-L19/20]
+    "Quantizing during training vs. after it", restricted to W^ =
+    Q(W diag s) diag(s)^-1; linears fed by the same input are summed.
+    """
+    X = np.asarray(X16, dtype=np.float64)
+    total = 0.0
+    for W in Ws:
+        E = awq_error_matrix(W, s16, bits, group, symmetric)
+        P = X @ E.T
+        total += float(np.sum(P * P))
+    return total
+
+
+def awq_search(X16: np.ndarray, Ws, bits: int, group: int, symmetric: bool,
+               alphas: np.ndarray | None = None) -> dict:
+    """Grid search over alpha; picks the lowest loss (first index on ties).
+
+    Steps, in the order [MIT-Lab4/5] "Question 2" gives them: compute the
+    scale from the activation statistic, scale the weight up, quantize,
+    scale down, measure the error, keep the best.
+    """
+    if alphas is None:
+        alphas = awq_alpha_grid(20)
+    mu = activation_absmean(X16)
+    S = awq_candidates(mu, alphas)
+    losses = np.array([awq_loss(X16, Ws, S[j], bits, group, symmetric)
+                       for j in range(len(alphas))], dtype=np.float64)
+    best = int(np.argmin(losses))
+    return {"mu": mu, "candidates": S, "losses": losses, "best": best, "s": S[best].copy(),
+            "alphas": np.asarray(alphas, dtype=np.float64)}

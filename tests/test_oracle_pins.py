@@ -1,0 +1,389 @@
+"""Pins for the CPU oracle: values the pages print, closed forms, invariants and
+brute force. Each test would fail on a plausible slip in the oracle (a dropped
+term, a wrong sign or index, a transposed operand, the wrong rounding)."""
+import json
+import os
+from fractions import Fraction
+
+import numpy as np
+import pytest
+
+import oracle as O
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+
+
+def _load(name):
+    with open(os.path.join(GOLDEN, name)) as f:
+        return json.load(f)
+
+
+# ---------------------------------------------------------------------------
+# "LLM Quantization: 160GB Model on a Laptop" -- Symmetric Quantization example
+# ---------------------------------------------------------------------------
+
+def test_worked_example_symmetric_4bit():
+    g = _load("p5_symmetric_worked_example.json")
+    v = np.array(g["values"], dtype=np.float16)[None, :]
+    codes, steps, zeros = O.quantize_groups(v, g["bits"], len(g["values"]), symmetric=True)
+    q = codes.astype(int)[0] - int(zeros[0, 0])
+    assert q.tolist() == g["quantized"]
+    step = float(steps[0, 0])
+    assert abs(step - g["scale_approx"]) < 5e-4
+    assert step == 0.127197265625  # smallest fp16 >= 0.8901367/7
+    deq = O.dequantize(codes, steps, zeros, len(g["values"]))[0]
+    assert np.allclose(deq, g["dequantized_printed"], atol=6e-4)
+    rel = np.mean(np.abs(deq - v[0].astype(np.float64)) / np.abs(v[0].astype(np.float64)))
+    assert abs(rel - g["average_error_printed"]) < 5e-3
+
+
+# ---------------------------------------------------------------------------
+# "CMU 11-868 L19-L20" -- absmax and zero-point (int8)
+# ---------------------------------------------------------------------------
+
+def test_int8_absmax_hand_cases():
+    for c in _load("p2_int8_hand_cases.json")["absmax"]:
+        q, deq = O.absmax_quantize_int8(np.array(c["X"]))
+        assert q.tolist() == c["q"], c["note"]
+        mult = 127.0 / np.max(np.abs(c["X"]))
+        assert np.allclose(deq, np.array(c["q"]) / mult)
+
+
+def test_int8_zeropoint_hand_cases():
+    for c in _load("p2_int8_hand_cases.json")["zeropoint"]:
+        q, deq = O.zeropoint_quantize_int8(np.array(c["X"]))
+        assert q.tolist() == c["q"], c["note"]
+        if "dequant" in c:
+            assert np.allclose(deq, c["dequant"])
+
+
+def test_asym_8bit_equals_int8_zeropoint_when_step_is_exact():
+    """With range 255/256 the step 2^-8 is exact in fp16 and the page's
+    multiplier is exactly 256: our unsigned 8-bit codes minus 128 must equal
+    the page's int8 codes (including ties, which both round to even)."""
+    g = np.random.default_rng(11)
+    ks = g.integers(-256, 255, size=126)                 # odd/even halves -> ties
+    x = np.concatenate([[-0.5, 127 / 256], ks / 512.0]).astype(np.float16)
+    codes, steps, zeros = O.quantize_groups(x[None, :], 8, x.size, symmetric=False)
+    assert float(steps[0, 0]) == 2.0 ** -8 and float(zeros[0, 0]) == 128
+    q_page, _ = O.zeropoint_quantize_int8(x.astype(np.float64))
+    assert (codes[0].astype(int) - 128).tolist() == q_page.astype(int).tolist()
+
+
+# ---------------------------------------------------------------------------
+# "Quantising Large Language Models" -- the group-wise symmetric routine
+# ---------------------------------------------------------------------------
+
+def test_symmetric_equals_page_routine_when_step_is_exact():
+    """Groups whose max |w| is 7 * 2^-7: the step 2^-7 is exact, so the fp16
+    round-up is a no-op and the page's float64 routine must agree exactly."""
+    g = np.random.default_rng(3)
+    N, K, grp = 4, 512, 128
+    w = (g.uniform(-0.05, 0.05, size=(N, K))).astype(np.float16)
+    for n in range(N):
+        for gi in range(K // grp):
+            j = gi * grp + int(g.integers(0, grp))
+            w[n, j] = np.float16(7 * 2.0 ** -7) * (1 if (n + gi) % 2 else -1)
+    codes, steps, zeros = O.quantize_groups(w, 4, grp, symmetric=True)
+    assert np.all(steps == np.float16(2.0 ** -7))
+    ours = O.dequantize(codes, steps, zeros, grp)
+    # the page's routine: scale = max|w|/qmax, clip(round(w/scale), -qmax-1, qmax) * scale
+    wr = w.astype(np.float64).reshape(N, K // grp, grp)
+    scale = np.abs(wr).max(axis=2, keepdims=True) / 7
+    page = (np.clip(np.round(wr / scale), -8, 7) * scale).reshape(N, K)
+    assert np.array_equal(ours, page)
+
+
+def test_group_size_sweep_error_is_monotone():
+    """The page's experiment: a N(0, 0.02) row of 4096 with two 0.8 outliers,
+    4-bit symmetric; mean abs error must fall as the group shrinks."""
+    g = np.random.default_rng(0)
+    row = g.normal(0, 0.02, 4096)
+    row[[10, 500]] = 0.8
+    w = row.astype(np.float16)[None, :]
+    errs = []
+    for grp in (4096, 128, 32):
+        c, s, z = O.quantize_groups(w, 4, grp, symmetric=True)
+        errs.append(np.abs(O.dequantize(c, s, z, grp) - w.astype(np.float64)).mean())
+    assert errs[0] > errs[1] > errs[2]
+
+
+# ---------------------------------------------------------------------------
+# fp16 round-up and the asymmetric quantizer
+# ---------------------------------------------------------------------------
+
+_F16_ALL = np.arange(1 << 16, dtype=np.uint16).view(np.float16)
+_F16_SORTED = np.sort(_F16_ALL[np.isfinite(_F16_ALL)].astype(np.float64))
+
+
+def test_f16_round_up_brute_force():
+    g = np.random.default_rng(5)
+    v = np.concatenate([
+        g.uniform(0, 1, 3000), 10.0 ** g.uniform(-9, 4.8, 3000),
+        _F16_SORTED[_F16_SORTED > 0][:2000],            # exact fp16 values map to themselves
+    ]).astype(np.float32)
+    got = O.f16_round_up(v).astype(np.float64)
+    idx = np.searchsorted(_F16_SORTED, v.astype(np.float64), side="left")
+    want = _F16_SORTED[idx]
+    assert np.array_equal(got, want)
+
+
+def _rand_groups(seed, N=64, K=512):
+    g = np.random.default_rng(seed)
+    w = g.normal(0, 0.02, (N, K))
+    w[: N // 4] = np.abs(w[: N // 4]) * -1.0 + 0.004           # skewed negative rows
+    w[N // 4: N // 2] *= np.where(g.random((N // 4, K)) < 0.01, 30.0, 1.0)  # outliers
+    w[-1, :128] = 0.0                                            # an all-zero group
+    w[-2, :128] = 0.01                                           # a constant group
+    w[-3, :128] = g.uniform(0.01, 0.03, 128)                     # a group that does not straddle 0
+    w[-4, 128:256] = -g.uniform(0.01, 0.03, 128)
+    return w.astype(np.float16)
+
+
+@pytest.mark.parametrize("bits", [3, 4])
+@pytest.mark.parametrize("symmetric", [False, True])
+def test_quantizer_error_bound_and_code_range(bits, symmetric):
+    w = _rand_groups(7)
+    codes, steps, zeros = O.quantize_groups(w, bits, 128, symmetric)
+    assert codes.max() < (1 << bits)
+    z = zeros.astype(np.float64)
+    assert np.all((z >= 0) & (z <= (1 << bits) - 1) & (z == np.round(z)))
+    deq = O.dequantize(codes, steps, zeros, 128)
+    stepk = np.repeat(steps.astype(np.float64), 128, axis=1)
+    err = np.abs(deq - w.astype(np.float64))
+    assert np.all(err <= stepk * (0.5 + 2.0 ** -20))
+    assert np.all(deq[-1, :128] == 0)
+
+
+@pytest.mark.parametrize("symmetric", [False, True])
+def test_step_is_smallest_fp16_at_or_above_quotient(symmetric):
+    bits = 4
+    w = _rand_groups(8)
+    codes, steps, zeros = O.quantize_groups(w, bits, 128, symmetric)
+    wg = w.astype(np.float32).reshape(w.shape[0], -1, 128)
+    for n in range(0, w.shape[0], 5):
+        for gi in range(wg.shape[1]):
+            grp = wg[n, gi]
+            if symmetric:
+                num, den = Fraction(float(np.abs(grp).max())), (1 << (bits - 1)) - 1
+            else:
+                num = Fraction(float(max(grp.max(), 0))) - Fraction(float(min(grp.min(), 0)))
+                den = (1 << bits) - 1
+            if num == 0:
+                assert float(steps[n, gi]) == 1.0
+                continue
+            quot = num / den
+            s = Fraction(float(steps[n, gi]))
+            i = np.searchsorted(_F16_SORTED, float(steps[n, gi]))
+            below = Fraction(float(_F16_SORTED[i - 1]))
+            slack = Fraction(1, 1 << 23)  # the fp32 quotient and range are rounded
+            assert s >= quot * (1 - slack)
+            assert below < quot * (1 + slack)
+
+
+@pytest.mark.parametrize("bits", [3, 4])
+def test_codes_are_nearest_with_ties_to_even_brute_force(bits):
+    """For the chosen (step, zero), every code is the nearest of all 2^b codes
+    to the fp32 quotient w/step; equidistant pairs resolve to an even (q - zero)."""
+    g = np.random.default_rng(9)
+    w = g.normal(0, 1, (6, 8)).astype(np.float16)
+    w[0, :4] = [0.5, -0.5, 1.5, 2.5]                             # exact ties at step 1
+    w[0, 4:] = [0.0, 0.0, 0.0, 0.0]
+    codes, steps, zeros = O.quantize_groups(w, bits, 8, symmetric=False)
+    Q = (1 << bits) - 1
+    for n in range(w.shape[0]):
+        for gi in range(w.shape[1] // 8):
+            sf = np.float32(steps[n, gi])
+            z = int(zeros[n, gi])
+            for j in range(8):
+                k = gi * 8 + j
+                quot = float(np.float32(w[n, k]) / sf)
+                best = None
+                for c in range(Q + 1):
+                    d = abs(quot - (c - z))
+                    key = (d, (c - z) % 2)
+                    if best is None or key < best[0]:
+                        best = (key, c)
+                assert codes[n, k] == best[1], (n, k, quot, z)
+
+
+def test_asymmetric_beats_symmetric_on_skewed_groups():
+    """"LLM Quantization: 160GB Model on a Laptop", Asymmetric Quantization:
+    handling min and max separately lowers the error on skewed data."""
+    g = np.random.default_rng(10)
+    w = (-np.abs(g.normal(0, 0.02, (32, 1024))) + 0.002).astype(np.float16)
+    e = {}
+    for sym in (False, True):
+        c, s, z = O.quantize_groups(w, 4, 128, sym)
+        e[sym] = np.abs(O.dequantize(c, s, z, 128) - w.astype(np.float64)).mean()
+    assert e[False] < 0.75 * e[True]
+
+
+# ---------------------------------------------------------------------------
+# Packed layouts
+# ---------------------------------------------------------------------------
+
+def test_pack4_hand_words():
+    codes = np.array([list(range(8)), list(range(8, 16))], dtype=np.uint8)
+    words = O.pack_codes(codes, 4)
+    # slot order [k0, k2, k4, k6, k1, k3, k5, k7] from nibble 0 upward
+    assert words[0, 0] == 0x75316420
+    assert words[1, 0] == 0xFDB9ECA8
+
+
+def test_pack3_hand_words():
+    codes = (np.arange(32) % 8).astype(np.uint8)[None, :]
+    words = O.pack_codes(codes, 3)
+    # word 0: k0..k9 = 0,1,2,3,4,5,6,7,0,1 in pairs (low field, high field);
+    # k30 = 6 (bit 0 = 0), k31 = 7 (bit 0 = 1) -> bit 15 clear, bit 31 set.
+    w0 = (0 << 0) | (2 << 3) | (4 << 6) | (6 << 9) | (0 << 12) \
+        | (1 << 16) | (3 << 19) | (5 << 22) | (7 << 25) | (1 << 28) | (1 << 31)
+    assert w0 == 0x9F590D10
+    assert words[0, 0] == w0
+    # word 2: k20..k29 = 4,5,6,7,0,1,2,3,4,5; bit 2 of k30 (=1) and of k31 (=1)
+    w2 = (4 << 0) | (6 << 3) | (0 << 6) | (2 << 9) | (4 << 12) \
+        | (5 << 16) | (7 << 19) | (1 << 22) | (3 << 25) | (5 << 28) | (1 << 15) | (1 << 31)
+    assert words[0, 2] == w2
+
+
+@pytest.mark.parametrize("bits", [3, 4])
+def test_pack_roundtrip(bits):
+    g = np.random.default_rng(12)
+    codes = g.integers(0, 1 << bits, size=(17, 256)).astype(np.uint8)
+    words = O.pack_codes(codes, bits)
+    assert words.shape == (17, O.packed_words_per_row(256, bits))
+    assert np.array_equal(O.unpack_codes(words, bits, 256), codes)
+
+
+# ---------------------------------------------------------------------------
+# Matmul reference
+# ---------------------------------------------------------------------------
+
+def test_gemm_ref_closed_forms():
+    N, K, M = 5, 256, 3
+    g = np.random.default_rng(13)
+    X = g.normal(0, 1, (M, K)).astype(np.float16)
+    steps = g.uniform(0.001, 0.1, (N, K // 128)).astype(np.float16)
+    zeros = g.integers(0, 16, (N, K // 128)).astype(np.float16)
+    codes = np.repeat(zeros.astype(np.uint8), 128, axis=1)       # every code == zero
+    assert np.all(O.gemm_ref(X, codes, steps, zeros, 128) == 0)
+    n, k, q = 3, 200, 15
+    codes[n, k] = q
+    Y = O.gemm_ref(X, codes, steps, zeros, 128)
+    expect = X[:, k].astype(np.float64) * (q - float(zeros[n, k // 128])) * float(steps[n, k // 128])
+    assert np.allclose(Y[:, n], expect, rtol=1e-15, atol=0)
+    assert np.all(np.delete(Y, n, axis=1) == 0)
+
+
+def test_gemm_ref_brute_force_loops():
+    g = np.random.default_rng(14)
+    M, N, K, grp = 2, 3, 64, 32
+    X = g.normal(0, 1, (M, K)).astype(np.float16)
+    codes = g.integers(0, 16, (N, K)).astype(np.uint8)
+    steps = g.uniform(0.001, 0.1, (N, K // grp)).astype(np.float16)
+    zeros = g.integers(0, 16, (N, K // grp)).astype(np.float16)
+    Y = O.gemm_ref(X, codes, steps, zeros, grp)
+    for m in range(M):
+        for n in range(N):
+            acc = Fraction(0)
+            for k in range(K):
+                acc += Fraction(float(X[m, k])) * (int(codes[n, k]) - Fraction(float(zeros[n, k // grp]))) \
+                    * Fraction(float(steps[n, k // grp]))
+            assert abs(Y[m, n] - float(acc)) <= 1e-13 * max(1.0, abs(float(acc)))
+
+
+# ---------------------------------------------------------------------------
+# AWQ pieces
+# ---------------------------------------------------------------------------
+
+def test_smoothquant_identity_fp64():
+    """"Quantising Large Language Models", outlier features: Y = (X diag(s)^-1)(diag(s) W)."""
+    g = np.random.default_rng(15)
+    X = g.normal(0, 1, (16, 256))
+    W = g.normal(0, 0.02, (64, 256))
+    s = np.exp(g.normal(0, 1, 256))
+    Y = X @ W.T
+    Y2 = (X / s[None, :]) @ (W * s[None, :]).T
+    assert np.max(np.abs(Y - Y2)) <= 1e-13 * np.max(np.abs(Y))
+
+
+def test_absmean_exact_and_order_independent():
+    g = np.random.default_rng(16)
+    X = (g.normal(0, 1, (48, 16)) * np.where(g.random(16) < 0.2, 20, 1)).astype(np.float16)
+    mu = O.activation_absmean(X)
+    perm = g.permutation(48)
+    assert np.array_equal(mu, O.activation_absmean(X[perm]))
+    for k in range(16):
+        exact = sum(Fraction(abs(float(v))) for v in X[:, k]) / 48
+        assert mu[k] == float(exact)
+
+
+def test_awq_candidates_endpoints():
+    mu = np.array([0.0, 1e-9, 0.3, 1.0, 7.25, 300.0])
+    S = O.awq_candidates(mu, O.awq_alpha_grid(20))
+    assert np.all(S[0] == 1.0)                                    # alpha = 0
+    assert O.awq_alpha_grid(20)[10] == 0.5
+    assert np.array_equal(S[10], np.sqrt(np.maximum(mu, 2.0 ** -14)).astype(np.float16))
+    assert np.all(S > 0)
+
+
+def test_awq_alpha0_is_plain_rtn():
+    g = np.random.default_rng(17)
+    W = g.normal(0, 0.02, (32, 256)).astype(np.float16)
+    E = O.awq_error_matrix(W, np.ones(256, np.float16), 4, 128, False)
+    c, s, z = O.quantize_groups(W, 4, 128, False)
+    assert np.array_equal(E, W.astype(np.float64) - O.dequantize(c, s, z, 128))
+
+
+def test_awq_loss_brute_force_loops():
+    g = np.random.default_rng(18)
+    T, K, grp = 3, 16, 8
+    X = g.normal(0, 1, (T, K)).astype(np.float16)
+    Ws = [g.normal(0, 0.1, (2, K)).astype(np.float16), g.normal(0, 0.1, (1, K)).astype(np.float16)]
+    s = np.exp(g.normal(0, 0.5, K)).astype(np.float16)
+    L = O.awq_loss(X, Ws, s, 4, grp, False)
+    total = 0.0
+    for W in Ws:
+        c, st, z = O.quantize_groups(W, 4, grp, False, s16=s)
+        for t in range(T):
+            for n in range(W.shape[0]):
+                d = 0.0
+                for k in range(K):
+                    deq = (int(c[n, k]) - float(z[n, k // grp])) * float(st[n, k // grp])
+                    d += float(X[t, k]) * (float(W[n, k]) - deq / float(s[k]))
+                total += d * d
+    assert abs(L - total) <= 1e-12 * total
+
+
+def test_salient_channel_error_shrinks_with_scale():
+    """"MIT 6.5940 Lab 4 + Lab 5", Question 2: scaling one channel by s while the
+    group max is unchanged shrinks that channel's error by about s."""
+    g = np.random.default_rng(19)
+    errs = {1.0: [], 2.0: []}
+    for _ in range(400):
+        w = g.normal(0, 0.02, 128)
+        w[0] = 0.1                                                # keeps the group max fixed
+        w = w.astype(np.float16)
+        for sc in (1.0, 2.0):
+            s = np.ones(128, np.float16)
+            s[5] = sc                                             # w[5] * 2 stays below w[0]
+            if abs(float(w[5])) * sc >= 0.1:
+                continue
+            E = O.awq_error_matrix(w[None, :], s, 3, 128, True)
+            errs[sc].append(abs(E[0, 5]))
+    ratio = np.mean(errs[2.0]) / np.mean(errs[1.0])
+    assert 0.35 < ratio < 0.65
+
+
+def test_awq_search_picks_minimum_and_beats_rtn():
+    import synth
+    g = synth.rng(20)
+    X = synth.activations(g, 64, 256, channel_frac=0.02, channel_mult=20.0)
+    Ws = [synth.weight(g, 48, 256, 0.02), synth.weight(g, 16, 256, 0.02)]
+    r = O.awq_search(X, Ws, 4, 128, False)
+    assert r["best"] == int(np.argmin(r["losses"]))
+    assert r["losses"][r["best"]] <= r["losses"][0]
+    assert r["losses"][r["best"]] < 0.9 * r["losses"][0]          # outlier channels make AWQ pay
+    assert np.array_equal(r["s"], r["candidates"][r["best"]])
+    # the loss at the chosen alpha is what awq_loss reports for that scale
+    assert r["losses"][r["best"]] == O.awq_loss(X, Ws, r["s"], 4, 128, False)
