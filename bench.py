@@ -1,0 +1,615 @@
+#!/usr/bin/env python
+"""Benchmark of the W4A16 decode path on B200.
+
+A step is one decode pass (M = 1 token) through the seven linears of a
+LLaMA-2-7B-shaped block (q/k/v/o 4096x4096, gate/up 4096->11008, down
+11008->4096), 4-bit asymmetric, group 128, packed by this library. Steps
+rotate over copies of the block whose packed weights together exceed the L2
+cache, so every step streams its weights from HBM. Each block copy's seven
+launches are one CUDA graph.
+
+The headline `value` is the effective bandwidth of the step: algorithmic bytes
+(packed weights + fp16 steps + fp16 zeros + X + Y) / device time. `rows`
+carries the other hot-path rows measured in the same run (quantize + pack,
+single-shape GEMVs incl. the 3-bit and 8192x28672 cases, the small-M sweep,
+the AWQ search). `roofline` divides by the measured HBM copy bandwidth.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Multi-GPU (torchrun): every rank runs its own replicas (weak scaling, no
+collective on the data path); rank 0 prints the max-over-ranks timing.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "W4A16 GEMV effective GB/s & % of B200 HBM peak; small-M GEMM TFLOP/s"
+WORKLOAD = "llama2_7b_block_decode_M1_w4_asym_g128"
+L2_BYTES = 126 * 1024 * 1024
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+
+
+# ---------------------------------------------------------------------------
+# helpers
+# ---------------------------------------------------------------------------
+
+def gemm_bytes(M: int, N: int, K: int, bits: int) -> int:
+    """Algorithmic bytes of one W{bits}A16 matmul: packed weight, fp16 steps and
+    zeros (one each per 128 input channels of a row), X and Y."""
+    return N * K * bits // 8 + N * (K // 128) * 4 + M * K * 2 + M * N * 2
+
+
+def quantize_bytes(N: int, K: int, bits: int) -> int:
+    return N * K * 2 + N * K * bits // 8 + N * (K // 128) * 4
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                "source": "measured"}
+    return {"hbm_gbs": FALLBACK_HBM_GBS, "bf16_tflops": FALLBACK_BF16_TFLOPS,
+            "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    d = os.path.join(ROOT, "weight_only_quantization_group_b200", "csrc")
+    for name in sorted(os.listdir(d)):
+        if name.endswith((".cu", ".cuh")):
+            with open(os.path.join(d, name), "rb") as f:
+                h.update(name.encode())
+                h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(kernel: str):
+    """Per-launch DRAM bytes of `kernel` from the committed ncu summary, if the
+    kernel sources have not changed since it was captured."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    e = d.get(kernel)
+    if not e or e.get("source_hash") != kernel_source_hash():
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+        return False
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for nm, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+
+def run_ours(args, rank: int, world: int, local_rank: int):
+    import torch
+    import torch.distributed as dist
+
+    from weight_only_quantization_group_b200 import build
+    build.build()
+    import weight_only_quantization_group_b200 as wq
+    import synth
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    peaks = load_peaks()
+
+    def barrier():
+        if world > 1:
+            dist.barrier(device_ids=[local_rank])
+
+    def dt(t):
+        return torch.from_numpy(np.ascontiguousarray(t)).to(dev)
+
+    # -- the block: quantize + pack each linear on the GPU -------------------
+    cases = synth.config_llama7b_decode(1)
+    block = []
+    for c in cases:
+        N, K = c.W.shape
+        Wd = dt(c.W)
+        packed, steps, zeros = wq.wq_quantize_pack(Wd, bits=4)
+        block.append({"name": c.name, "N": N, "K": K, "X": dt(c.X), "W": Wd, "q": (packed, steps, zeros),
+                      "Xh": c.X})
+    assert wq.wq_get_last_device_error() == 0
+    step_bytes = sum(gemm_bytes(1, b["N"], b["K"], 4) for b in block)
+    block_w_bytes = sum(b["N"] * b["K"] // 2 for b in block)
+    n_copies = max(2, math.ceil(4 * L2_BYTES / block_w_bytes))
+
+    # -- rotating block copies and one graph per copy -------------------------
+    copies = [block]
+    for _ in range(n_copies - 1):
+        copies.append([{**b, "q": tuple(t.clone() for t in b["q"])} for b in block])
+    Ys = [[torch.empty((1, b["N"]), dtype=torch.float16, device=dev) for b in block] for _ in copies]
+    s_cap = torch.cuda.Stream(device=dev)
+    graphs = []
+    for ci, blk in enumerate(copies):
+        # warm the launch path (function attributes) before capture
+        for b, y in zip(blk, Ys[ci]):
+            wq.wq_w4a16_gemm(b["X"], *b["q"], b["N"], bits=4, out=y)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=s_cap):
+            for b, y in zip(blk, Ys[ci]):
+                wq.wq_w4a16_gemm(b["X"], *b["q"], b["N"], bits=4, out=y)
+        graphs.append(g)
+    torch.cuda.synchronize()
+
+    stream = torch.cuda.current_stream()
+    for i in range(args.warmup):
+        graphs[i % n_copies].replay()
+    torch.cuda.synchronize()
+    barrier()
+    torch.cuda.synchronize()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local_rank) as clk:
+        ev0.record(stream)
+        for i in range(args.steps):
+            graphs[i % n_copies].replay()
+        ev1.record(stream)
+        torch.cuda.synchronize()
+    barrier()
+    torch.cuda.synchronize()
+    ms = ev0.elapsed_time(ev1)
+    if world > 1:
+        t = torch.tensor([ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    assert wq.wq_get_last_device_error() == 0
+    ms_per_step = ms / args.steps
+    value = world * step_bytes * args.steps / (ms * 1e-3) / 1e9  # GB/s, all ranks
+
+    # -- e2e: the public call with host buffers, copies inside the timed region
+    xh = [torch.from_numpy(b["Xh"]).pin_memory() for b in block]
+    yh = [torch.empty((1, b["N"]), dtype=torch.float16).pin_memory() for b in block]
+    e2e_steps = max(20, min(2000, args.steps // 10))
+    h2d = sum(x.numel() * 2 for x in xh)
+    d2h = sum(y.numel() * 2 for y in yh)
+
+    def e2e_step(blk):
+        for b, x, y in zip(blk, xh, yh):
+            b["X"].copy_(x, non_blocking=True)
+            out = wq.wq_w4a16_gemm(b["X"], *b["q"], b["N"], bits=4)
+            y.copy_(out, non_blocking=True)
+        torch.cuda.current_stream().synchronize()
+
+    for i in range(3):
+        e2e_step(copies[i % n_copies])
+    barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for i in range(e2e_steps):
+        e2e_step(copies[i % n_copies])
+    e1.record()
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    e2e_value = world * step_bytes * e2e_steps / (e2e_ms * 1e-3) / 1e9
+
+    rows = {}
+    if rank == 0 and not args.no_rows:
+        rows = measure_rows(wq, torch, synth, dev, block, peaks)
+
+    del graphs
+    if rank != 0:
+        return None
+
+    clocks = clk.summary()
+    traffic = profiled_traffic("gemv_kernel<4,1,2>")
+    achieved = step_bytes / (ms_per_step * 1e-3) / 1e9
+    line = {
+        "metric": METRIC,
+        "value": round(value, 2),
+        "unit": "GB/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms_per_step,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f16",
+        "data": "synthetic",
+        "config": {
+            "workload": WORKLOAD,
+            "linears": [f"{b['name']}" for b in block],
+            "bytes_per_step": step_bytes,
+            "block_copies": n_copies,
+            "l2": f"inputs larger than L2: {n_copies} block copies, {n_copies * block_w_bytes / 1e6:.0f} MB of packed weight rotate",
+            "graph": "one CUDA graph of 7 launches per block copy",
+            "parallelism": f"replicas x{world}",
+        },
+        "roofline": {
+            "bound": "hbm",
+            "kernel": "gemv_kernel<4,1,2>",
+            "achieved": round(achieved, 2),
+            "peak": peaks["hbm_gbs"],
+            "peak_source": f"{peaks['source']} HBM copy bandwidth",
+            "unit": "GB/s",
+            "frac": round(achieved / peaks["hbm_gbs"], 4),
+            "traffic": traffic,
+            "note": "achieved = algorithmic bytes of the 7 launches / device time of the step (graph gaps included)",
+        },
+        "e2e": {"value": round(e2e_value, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "steps": e2e_steps, "ms_per_step": e2e_ms / e2e_steps,
+                "path": "wq_w4a16_gemm per linear, pinned host X in, Y out, stream sync per step"},
+        "gpu_launches": 7 * args.steps,
+        "clocks": clocks,
+        "rows": rows,
+    }
+    if not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(cases, args.cpu_seconds)
+    return line
+
+
+def _time_graph(torch, fn_list, reps: int = 5, inner: int = 1):
+    """Median ms of one pass over fn_list, captured as one graph and replayed."""
+    s = torch.cuda.Stream()
+    for f in fn_list:
+        f()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        for _ in range(inner):
+            for f in fn_list:
+                f()
+    g.replay()
+    torch.cuda.synchronize()
+    out = []
+    for _ in range(reps):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        g.replay()
+        b.record()
+        torch.cuda.synchronize()
+        out.append(a.elapsed_time(b) / inner)
+    del g
+    return statistics.median(out)
+
+
+def measure_rows(wq, torch, synth, dev, block, peaks):
+    rows = {}
+
+    def dt(t):
+        return torch.from_numpy(np.ascontiguousarray(t)).to(dev)
+
+    # S3 quantize + pack over the block (W fp16 read 404 MB > L2)
+    fns = [lambda b=b: wq.wq_quantize_pack(b["W"], bits=4, out=b["q"]) for b in block]
+    ms = _time_graph(torch, fns)
+    qb = sum(quantize_bytes(b["N"], b["K"], 4) for b in block)
+    rows["quantize_pack_block_w4"] = {"ms": ms, "GB/s": qb / (ms * 1e-3) / 1e9,
+                                      "frac_hbm": qb / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                                      "weights": sum(b["N"] * b["K"] for b in block)}
+
+    # single-shape GEMVs, rotating copies >= 4x L2
+    def gemv_row(name, N, K, bits, W16, X16, M=1):
+        packed, steps, zeros = wq.wq_quantize_pack(dt(W16), bits=bits)
+        wbytes = N * K * bits // 8
+        nc = max(2, math.ceil(4 * L2_BYTES / wbytes))
+        qs = [(packed, steps, zeros)] + [tuple(t.clone() for t in (packed, steps, zeros)) for _ in range(nc - 1)]
+        X = dt(X16)
+        Y = torch.empty((M, N), dtype=torch.float16, device=dev)
+        fns = [lambda q=q: wq.wq_w4a16_gemm(X, *q, N, bits=bits, out=Y) for q in qs]
+        ms = _time_graph(torch, fns) / nc
+        by = gemm_bytes(M, N, K, bits)
+        fl = 2.0 * M * N * K
+        rows[name] = {"M": M, "N": N, "K": K, "bits": bits, "us": ms * 1e3, "GB/s": by / (ms * 1e-3) / 1e9,
+                      "frac_hbm": by / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"], "TFLOP/s": fl / (ms * 1e-3) / 1e12}
+        del qs
+
+    for b in block[:1] + block[4:5] + block[6:7]:
+        gemv_row(f"gemv_{b['name']}", b["N"], b["K"], 4, b["W"].cpu().numpy(), b["Xh"])
+    for bits in (4, 3):
+        c = synth.config_llama65b_decode(bits)
+        gemv_row(f"gemv_llama65b_8192x8192_w{bits}", 8192, 8192, bits, c.W, c.X)
+        wq.wq_set_option(wq.WQ_OPT_GEMV_VARIANT, wq.WQ_GEMV_EXACT)
+        try:
+            gemv_row(f"gemv_llama65b_8192x8192_w{bits}_exact", 8192, 8192, bits, c.W, c.X)
+        finally:
+            wq.wq_set_option(wq.WQ_OPT_GEMV_VARIANT, wq.WQ_GEMV_OFFSET_SUMS)
+    big = synth.config_smallm_sweep(1)
+    for M in synth.SMALLM_SWEEP:
+        gemv_row(f"smallm_M{M}_8192x28672_w4", 28672, 8192, 4, big.W, synth.smallm_activations(M), M=M)
+    # the other kernel on each side of the crossover, for the record
+    for M in (4, 8, 16, 32):
+        path = wq.WQ_PATH_TENSOR_CORE if M < 16 else wq.WQ_PATH_GEMV
+        wq.wq_set_option(wq.WQ_OPT_GEMM_PATH, path)
+        try:
+            tag = "tc" if path == wq.WQ_PATH_TENSOR_CORE else "gemv"
+            gemv_row(f"smallm_M{M}_8192x28672_w4_{tag}", 28672, 8192, 4, big.W, synth.smallm_activations(M), M=M)
+        finally:
+            wq.wq_set_option(wq.WQ_OPT_GEMM_PATH, wq.WQ_PATH_AUTO)
+    wq.wq_set_option(wq.WQ_OPT_TC_A_OPERAND, wq.WQ_TC_A_SMEM)
+    try:
+        for M in (16, 64, 128):
+            gemv_row(f"smallm_M{M}_8192x28672_w4_tc_smemA", 28672, 8192, 4, big.W, synth.smallm_activations(M), M=M)
+    finally:
+        wq.wq_set_option(wq.WQ_OPT_TC_A_OPERAND, wq.WQ_TC_A_TMEM)
+    return rows
+
+
+def cpu_baseline(cases, seconds: float):
+    """The oracle (numpy, fp64 dequantize + matmul), as it stands, on a sample of
+    each linear's output rows, repeated until about `seconds` of CPU time."""
+    import oracle as O
+    try:
+        from threadpoolctl import threadpool_limits
+    except ImportError:  # pragma: no cover
+        threadpool_limits = None
+    prepared = []
+    frac = 16
+    for c in cases:
+        N, K = c.W.shape
+        rows = N // frac
+        codes, st, z = O.quantize_groups(c.W[:rows], 4, 128, False)
+        words = O.pack_codes(codes, 4)
+        prepared.append((c.X, words, st, z, rows, K))
+    ctx = threadpool_limits(limits=1) if threadpool_limits else None
+    t0 = time.perf_counter()
+    done_bytes, reps = 0, 0
+    if ctx:
+        ctx.__enter__()
+    try:
+        while True:
+            for X, words, st, z, rows, K in prepared:
+                codes = O.unpack_codes(words, 4, K)
+                O.gemm_ref(X, codes, st, z, 128)
+                done_bytes += gemm_bytes(1, rows, K, 4)
+            reps += 1
+            if time.perf_counter() - t0 >= seconds:
+                break
+    finally:
+        if ctx:
+            ctx.__exit__(None, None, None)
+    el = time.perf_counter() - t0
+    return {"value": round(done_bytes / el / 1e9, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "sample": f"1/{frac} of the output rows of each of the 7 linears (unpack + fp64 dequantize + fp64 "
+                      f"matmul), {reps} passes in {el:.1f} s, one thread"}
+
+
+# ---------------------------------------------------------------------------
+# reference arm: the oracle on the host cores
+# ---------------------------------------------------------------------------
+
+def run_reference(args, rank: int, world: int):
+    if rank != 0:
+        return None
+    import oracle as O
+    import synth
+    try:
+        from threadpoolctl import threadpool_limits
+        lim = threadpool_limits(limits=1)
+    except ImportError:  # pragma: no cover
+        lim = None
+    cases = synth.config_llama7b_decode(1)
+    budget = float(args.ref_seconds)
+    # calibrate rows per step so the whole run fits the budget
+    c0 = cases[0]
+    codes, st, z = O.quantize_groups(c0.W[:64], 4, 128, False)
+    words = O.pack_codes(codes, 4)
+    t0 = time.perf_counter()
+    O.gemm_ref(c0.X, O.unpack_codes(words, 4, c0.K if hasattr(c0, "K") else c0.W.shape[1]), st, z, 128)
+    per_row = (time.perf_counter() - t0) / 64
+    total_rows_per_step = sum(c.W.shape[0] for c in cases)
+    steps_total = args.steps + args.warmup
+    frac = min(1.0, budget / max(steps_total * per_row * total_rows_per_step, 1e-9))
+    prepared = []
+    for c in cases:
+        N, K = c.W.shape
+        rows = max(1, int(N * frac))
+        codes, st, z = O.quantize_groups(c.W[:rows], 4, 128, False)
+        prepared.append((c.X, O.pack_codes(codes, 4), st, z, rows, K))
+
+    def step():
+        b = 0
+        for X, words, st, z, rows, K in prepared:
+            O.gemm_ref(X, O.unpack_codes(words, 4, K), st, z, 128)
+            b += gemm_bytes(1, rows, K, 4)
+        return b
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    by = 0
+    for _ in range(args.steps):
+        by += step()
+    el = time.perf_counter() - t0
+    if lim is not None:
+        lim.__exit__(None, None, None)
+    value = by / el / 1e9
+    sample = (f"{frac:.5f} of the output rows of each of the 7 linears per step "
+              f"(unpack + fp64 dequantize + fp64 matmul), one thread")
+    return {
+        "impl": "reference",
+        "metric": METRIC,
+        "value": round(value, 5),
+        "unit": "GB/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": el * 1e3 / args.steps,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": WORKLOAD, "parallelism": "host cores (rank 0 only)"},
+        "cpu_baseline": {"value": round(value, 5), "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(value, 5), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+# ---------------------------------------------------------------------------
+# single-case mode (a small, bounded run of one kernel, e.g. under ncu)
+# ---------------------------------------------------------------------------
+
+def run_case(args):
+    import torch
+
+    from weight_only_quantization_group_b200 import build
+    build.build()
+    import weight_only_quantization_group_b200 as wq
+    import synth
+
+    dev = torch.device("cuda", 0)
+    g = synth.rng(77)
+    W = torch.from_numpy(synth.weight(g, args.N, args.K, 0.02)).to(dev)
+    X = torch.from_numpy(synth.activations(g, args.M, args.K)).to(dev)
+    opts = {"auto": wq.WQ_PATH_AUTO, "gemv": wq.WQ_PATH_GEMV, "tc": wq.WQ_PATH_TENSOR_CORE}
+    wq.wq_set_option(wq.WQ_OPT_GEMM_PATH, opts[args.path])
+    wq.wq_set_option(wq.WQ_OPT_GEMV_VARIANT, wq.WQ_GEMV_EXACT if args.gemv_variant == "exact"
+                     else wq.WQ_GEMV_OFFSET_SUMS)
+    wq.wq_set_option(wq.WQ_OPT_TC_A_OPERAND, wq.WQ_TC_A_SMEM if args.tc_a == "smem" else wq.WQ_TC_A_TMEM)
+    q = wq.wq_quantize_pack(W, bits=args.bits)
+    Y = torch.empty((args.M, args.N), dtype=torch.float16, device=dev)
+    torch.cuda.synchronize()
+    times = []
+    for _ in range(args.reps):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        if args.case == "gemm":
+            wq.wq_w4a16_gemm(X, *q, args.N, bits=args.bits, out=Y)
+        else:
+            wq.wq_quantize_pack(W, bits=args.bits, out=q)
+        b.record()
+        torch.cuda.synchronize()
+        times.append(a.elapsed_time(b) * 1e3)
+    st = wq.wq_get_last_device_error()
+    print(json.dumps({"case": args.case, "M": args.M, "N": args.N, "K": args.K, "bits": args.bits,
+                      "path": args.path, "us": times, "device_status": st}))
+    if st != 0:
+        sys.exit(1)
+
+
+# ---------------------------------------------------------------------------
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20000)
+    ap.add_argument("--warmup", type=int, default=200)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-rows", action="store_true", help="skip the per-row measurements")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--ref-seconds", type=float, default=60.0)
+    ap.add_argument("--case", choices=["gemm", "quantize"], default=None,
+                    help="run one small kernel configuration --reps times (for profiling)")
+    ap.add_argument("--M", type=int, default=1)
+    ap.add_argument("--N", type=int, default=8192)
+    ap.add_argument("--K", type=int, default=8192)
+    ap.add_argument("--bits", type=int, default=4)
+    ap.add_argument("--reps", type=int, default=3)
+    ap.add_argument("--path", choices=["auto", "gemv", "tc"], default="auto")
+    ap.add_argument("--gemv-variant", choices=["offset", "exact"], default="offset")
+    ap.add_argument("--tc-a", choices=["tmem", "smem"], default="tmem")
+    args = ap.parse_args()
+    if args.case:
+        run_case(args)
+        return
+    if args.warmup < 3:
+        args.warmup = 3
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        line = run_reference(args, rank, world)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return
+
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        line = run_ours(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+    if line is not None:
+        print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

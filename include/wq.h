@@ -1,0 +1,183 @@
+/*
+ * wq.h -- C ABI of the B200 (sm_100a) group-wise weight-only quantization
+ * library (libwq.so).
+ *
+ * The library quantizes fp16 weights group-wise to 3 or 4 bits, packs them in
+ * the layout documented below, searches AWQ per-input-channel scales, and
+ * runs the W4A16 / W3A16 matmul Y = X * W^T that dequantizes the packed
+ * weights on the fly (fp16 activations, fp32 accumulation, fp16 output).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - W is an nn.Linear weight: [N][K] row-major fp16 (N output channels, K
+ *    input channels). X is [M][K] row-major fp16, Y is [M][N] row-major fp16.
+ *  - A group is `group_size` (= 128) consecutive input channels of one
+ *    output row ("Quantising Large Language Models for Efficient Inference",
+ *    section "Post-training methods for 4-bit weights": one scale and zero
+ *    point per group of 64-128 weights within a row).
+ *  - Pointers named *_dev are device pointers the caller allocated (e.g. torch
+ *    tensors' data_ptr()). The library never frees or retains them.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *    stream). All device work is enqueued asynchronously on it; the host side
+ *    validates arguments synchronously and returns before the work runs.
+ *  - Argument errors are reported by the return value and enqueue nothing.
+ *    Launch failures return WQ_ERR_CUDA. Conditions found on the device (a
+ *    step that overflows fp16, a bounded wait that ran out) are latched in a
+ *    per-device flag read by wq_get_last_device_error().
+ *  - No entry point allocates device memory, except that the first call on a
+ *    device looks up the address of the library's device error flag.
+ *
+ * Quantization contract (bit-exact; identical in the CPU oracle)
+ * --------------------------------------------------------------
+ *  fp16 inputs are widened exactly to fp32; with AWQ scales s, w' = w * s_k
+ *  (exact). Asymmetric, Q = 2^b - 1 ("LLM Quantization: 160GB Model on a
+ *  Laptop", section "Asymmetric Quantization", in the integer zero-point form
+ *  of "CMU 11-868 L19-L20 Model Quantization", section "absmax and
+ *  zero-point"):
+ *     mn = min(min_g w', 0), mx = max(max_g w', 0), r = mx - mn      (fp32)
+ *     step = (r == 0) ? 1 : fp16_round_toward_+inf(r / Q)          (fp32 div)
+ *     zero = clamp(rint(-mn / step), 0, Q)
+ *     q    = clamp(rint(w' / step) + zero, 0, Q)       rint: ties to even
+ *  Symmetric, qmax = 2^(b-1) - 1 ("LLM Quantization: 160GB Model on a
+ *  Laptop", section "Symmetric Quantization"):
+ *     step = (max|w'| == 0) ? 1 : fp16_round_toward_+inf(max|w'| / qmax)
+ *     q    = clamp(rint(w' / step), -qmax - 1, qmax) + 2^(b-1); zero = 2^(b-1)
+ *  Both dequantize as (q - zero) * step. Steps and zeros are stored as fp16.
+ *
+ * Packed layouts (row-major over output rows; no padding between rows)
+ * --------------------------------------------------------------------
+ *  4-bit: uint32 [N][K/8]. Word c of a row holds k = 8c .. 8c+7; nibble slot
+ *         j (bits 4j..4j+3) holds k = 8c+2j for j < 4 and k = 8c+2(j-4)+1
+ *         for j >= 4 (slot order k0,k2,k4,k6,k1,k3,k5,k7), so that
+ *         (word >> 4j) & 0x000F000F is the pair (k_2j, k_2j+1) in two 16-bit
+ *         lanes. This is the GPU counterpart of the offline nibble reordering
+ *         in "MIT 6.5940 Lab 4 + Lab 5", section "Background: why the 4-bit
+ *         weights get reordered first".
+ *  3-bit: uint32 [N][3K/32]. Three words t = 0,1,2 per 32 consecutive k:
+ *         word t, pair j = 0..4: bits 3j..3j+2 hold k = 10t+2j, bits
+ *         16+3j..18+3j hold k = 10t+2j+1; bit b of k = 30 is bit 15 of word b
+ *         and bit b of k = 31 is bit 31 of word b. Exactly 3 bits per weight.
+ *  steps, zeros: fp16 [N][K/group_size] row-major.
+ *
+ * Supported: bits in {3, 4}; group_size == 128; K % 128 == 0; N >= 1;
+ * M >= 1. Device pointers must be 16-byte aligned (weights, X, packed words)
+ * or 4-byte aligned (steps, zeros, Y, s, mu). Inputs must be finite.
+ */
+#ifndef WQ_H_
+#define WQ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define WQ_ABI_VERSION 1
+
+typedef enum wq_status {
+  WQ_OK = 0,
+  WQ_ERR_INVALID_ARG = 1,  /* null pointer, non-positive size, bad config  */
+  WQ_ERR_UNSUPPORTED = 2,  /* valid but not implemented (e.g. group != 128) */
+  WQ_ERR_ALIGNMENT = 3,    /* a pointer is not aligned as required          */
+  WQ_ERR_CUDA = 4,         /* a CUDA runtime call or launch failed          */
+  WQ_ERR_TIMEOUT = 5,      /* device: a bounded wait gave up                */
+  WQ_ERR_WORKSPACE = 6,    /* workspace pointer null or smaller than needed */
+  WQ_ERR_RANGE = 7         /* device: a step or scale is not finite in fp16 */
+} wq_status;
+
+typedef struct wq_quant_cfg {
+  int32_t bits;        /* 3 or 4                                   */
+  int32_t group_size;  /* 128                                      */
+  int32_t symmetric;   /* 0: asymmetric zero point, 1: symmetric   */
+} wq_quant_cfg;
+
+/* ABI version of the loaded library (WQ_ABI_VERSION). */
+int32_t wq_abi_version(void);
+
+/* Static string for a status code. Never NULL. */
+const char* wq_status_string(int32_t status);
+
+/* Number of uint32 words of the packed weight for an [N][K] matrix
+ * (N*K/8 for 4-bit, 3*N*K/32 for 3-bit); 0 if the config is invalid. */
+size_t wq_packed_words(int64_t N, int64_t K, const wq_quant_cfg* cfg);
+
+/* S3 -- quantize + pack.
+ * Quantizes W_dev (fp16 [N][K]) group-wise per the contract above, after the
+ * optional AWQ scaling W * diag(s) (s_dev: fp16 [K], or NULL for none;
+ * "MIT 6.5940 Lab 4 + Lab 5", section "Question 2"), and writes packed_dev
+ * (uint32, wq_packed_words(N,K,cfg) words), steps_dev and zeros_dev (fp16
+ * [N][K/128] each). One kernel launch. A step that is not finite in fp16
+ * latches WQ_ERR_RANGE in the device flag. */
+int32_t wq_quantize_pack(const void* W_dev, const void* s_dev, int64_t N, int64_t K,
+                         const wq_quant_cfg* cfg, uint32_t* packed_dev, void* steps_dev,
+                         void* zeros_dev, void* stream);
+
+/* Inverse of the packing: W_out_dev (fp16 [N][K]) = fp16_rn((q - zero) * step)
+ * for every element. A check/test helper, not on the decode path. */
+int32_t wq_unpack_dequant(const uint32_t* packed_dev, const void* steps_dev,
+                          const void* zeros_dev, int64_t N, int64_t K,
+                          const wq_quant_cfg* cfg, void* W_out_dev, void* stream);
+
+/* Workspace the matmul needs for (M, N, K, cfg), in bytes (currently 0:
+ * split-K partial sums are reduced on chip through thread-block-cluster
+ * shared memory). */
+size_t wq_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, const wq_quant_cfg* cfg);
+
+/* S5/S6 -- weight-only matmul Y = X * deq(W)^T.
+ * X_dev fp16 [M][K]; packed_dev/steps_dev/zeros_dev as written by
+ * wq_quantize_pack; Y_dev fp16 [M][N] (overwritten). Products are exact in
+ * fp32 and accumulated in fp32 ("Quantising Large Language Models",
+ * section "Weight-only vs weight-and-activation quantisation": weights are
+ * dequantized on the fly inside the matmul; "TinyChat (AWQ on-device
+ * runtime)", "Notable features": fused dequant + GEMM). Small M runs a
+ * bandwidth-bound GEMV kernel that streams the packed weights once; larger M
+ * (4-bit) runs a tcgen05 tensor-core kernel. workspace_dev may be NULL when
+ * wq_gemm_workspace_bytes() is 0. X must already be multiplied by
+ * diag(s)^-1 when the weight was packed with AWQ scales s. */
+int32_t wq_w4a16_gemm(const void* X_dev, const uint32_t* packed_dev, const void* steps_dev,
+                      const void* zeros_dev, int64_t M, int64_t N, int64_t K,
+                      const wq_quant_cfg* cfg, void* Y_dev, void* workspace_dev,
+                      size_t workspace_bytes, void* stream);
+
+/* Process-wide tuning options (not thread-safe against concurrent calls).
+ *  WQ_OPT_GEMM_PATH     WQ_PATH_AUTO (default): GEMV kernel below the
+ *                       crossover M, tensor-core kernel at or above it (4-bit);
+ *                       WQ_PATH_GEMV / WQ_PATH_TENSOR_CORE force one kernel
+ *                       (the tensor-core kernel is 4-bit only).
+ *  WQ_OPT_CROSSOVER_M   smallest M sent to the tensor-core kernel (default 16).
+ *  WQ_OPT_TC_A_OPERAND  where the tensor-core kernel stages the dequantized
+ *                       weight tile: WQ_TC_A_TMEM (tensor memory, default) or
+ *                       WQ_TC_A_SMEM (128-byte swizzled shared memory).
+ *  WQ_OPT_GEMV_VARIANT  how the GEMV kernel forms sum_k x_k (q_k - zero):
+ *                       WQ_GEMV_OFFSET_SUMS (default) multiplies x by the
+ *                       unpacked (1024 + q) and removes the offset with
+ *                       per-chunk activation sums (fewer instructions);
+ *                       WQ_GEMV_EXACT subtracts the zero point in fp16 first,
+ *                       so every product is exact.
+ * wq_set_option returns WQ_ERR_INVALID_ARG for an unknown option or value;
+ * wq_get_option returns the current value, or -1 for an unknown option. */
+#define WQ_OPT_GEMM_PATH 1
+#define WQ_OPT_CROSSOVER_M 2
+#define WQ_OPT_TC_A_OPERAND 3
+#define WQ_PATH_AUTO 0
+#define WQ_PATH_GEMV 1
+#define WQ_PATH_TENSOR_CORE 2
+#define WQ_TC_A_TMEM 0
+#define WQ_TC_A_SMEM 1
+#define WQ_OPT_GEMV_VARIANT 4
+#define WQ_GEMV_OFFSET_SUMS 0
+#define WQ_GEMV_EXACT 1
+int32_t wq_set_option(int32_t option, int64_t value);
+int64_t wq_get_option(int32_t option);
+
+/* Synchronizes `stream`, then returns and clears the device flag of the
+ * current device (WQ_OK if nothing was latched). Returns WQ_ERR_CUDA if the
+ * synchronization itself fails. */
+int32_t wq_get_last_device_error(void* stream);
+
+#ifdef __cplusplus
+}  /* extern "C" */
+#endif
+
+#endif  /* WQ_H_ */

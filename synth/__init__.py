@@ -35,6 +35,8 @@ __all__ = [
     "config_llama7b_decode",
     "config_llama65b_decode",
     "config_smallm_sweep",
+    "smallm_activations",
+    "SMALLM_SWEEP",
     "config_awq_block",
 ]
 
@@ -144,12 +146,16 @@ def config_llama65b_decode(bits: int, seed: int = 2, M: int = 1, K: int = 8192, 
 SMALLM_SWEEP = (1, 2, 4, 8, 16, 32, 64, 128)
 
 
+def smallm_activations(M: int, seed: int = 4, K: int = 8192) -> np.ndarray:
+    """The M fp16 rows ~ N(0, 1) of the small-M sweep (independent of the weight)."""
+    return activations(rng(seed * 1000 + M), M, K)
+
+
 def config_smallm_sweep(M: int, seed: int = 4, K: int = 8192, N: int = 28672) -> GemmCase:
     """K=8192, N=28672 weight (W ~ N(0, 0.01)) against M fp16 rows ~ N(0, 1)."""
     g = rng(seed)
     W = weight(g, N, K, 0.01)
-    X = activations(rng(seed * 1000 + M), M, K)
-    return GemmCase(f"smallm_K{K}_N{N}_M{M}", X, W)
+    return GemmCase(f"smallm_K{K}_N{N}_M{M}", smallm_activations(M, seed, K), W)
 
 
 def config_awq_block(seed: int = 5, T: int = 512, shapes=LLAMA2_7B_BLOCK,

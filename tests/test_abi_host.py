@@ -1,0 +1,83 @@
+"""Host-side checks of the C-ABI library: it loads without a GPU, exports every
+symbol the header declares, and rejects bad arguments before touching CUDA."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "wq.h")
+
+
+@pytest.fixture(scope="session")
+def wq():
+    from weight_only_quantization_group_b200 import build
+    build.build()
+    import weight_only_quantization_group_b200 as m
+    return m
+
+
+def _declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(wq_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_header_declares_the_boundary():
+    names = _declared_functions()
+    for required in ("wq_quantize_pack", "wq_w4a16_gemm", "wq_unpack_dequant", "wq_get_last_device_error"):
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol(wq):
+    L = ctypes.CDLL(wq.library_path)
+    missing = [n for n in _declared_functions() if not hasattr(L, n)]
+    assert not missing, missing
+    assert set(_declared_functions()) == set(wq.EXPORTED_SYMBOLS)
+
+
+def test_abi_version_and_status_strings(wq):
+    assert wq.wq_abi_version() == 1
+    for code in range(8):
+        assert wq.wq_status_string(code).startswith("WQ_")
+    assert wq.wq_status_string(99) == "unknown wq status"
+
+
+def test_packed_word_counts(wq):
+    assert wq.wq_packed_words(4096, 4096, bits=4) == 4096 * 4096 // 8
+    assert wq.wq_packed_words(8192, 8192, bits=3) == 8192 * 8192 * 3 // 32
+    assert wq.wq_packed_words(7, 11008, bits=4) == 7 * 11008 // 8
+    assert wq.wq_packed_words(128, 200, bits=4) == 0      # K not a multiple of 128
+    assert wq.wq_packed_words(128, 256, bits=5) == 0      # unsupported width
+    assert wq.wq_packed_words(0, 256, bits=4) == 0
+
+
+def _cfg(wq, bits=4, group=128, sym=0):
+    return wq._Cfg(bits, group, sym)
+
+
+def test_argument_validation_without_gpu(wq):
+    L = wq.lib()
+    good = 0x10000  # a fake, 16-byte aligned address; validation fails before any use
+    c = _cfg(wq)
+    by = ctypes.byref
+    # unsupported / invalid configs
+    assert L.wq_quantize_pack(good, None, 8, 256, by(_cfg(wq, bits=5)), good, good, good, None) == wq.WQ_ERR_UNSUPPORTED
+    assert L.wq_quantize_pack(good, None, 8, 256, by(_cfg(wq, bits=1)), good, good, good, None) == wq.WQ_ERR_INVALID_ARG
+    assert L.wq_quantize_pack(good, None, 8, 256, by(_cfg(wq, group=64)), good, good, good, None) == wq.WQ_ERR_UNSUPPORTED
+    assert L.wq_quantize_pack(good, None, 8, 256, by(_cfg(wq, sym=2)), good, good, good, None) == wq.WQ_ERR_INVALID_ARG
+    assert L.wq_quantize_pack(good, None, 8, 256, None, good, good, good, None) == wq.WQ_ERR_INVALID_ARG
+    # shapes
+    assert L.wq_quantize_pack(good, None, 0, 256, by(c), good, good, good, None) == wq.WQ_ERR_INVALID_ARG
+    assert L.wq_quantize_pack(good, None, 8, 200, by(c), good, good, good, None) == wq.WQ_ERR_INVALID_ARG
+    # null and misaligned pointers
+    assert L.wq_quantize_pack(None, None, 8, 256, by(c), good, good, good, None) == wq.WQ_ERR_INVALID_ARG
+    assert L.wq_quantize_pack(good + 8, None, 8, 256, by(c), good, good, good, None) == wq.WQ_ERR_ALIGNMENT
+    assert L.wq_quantize_pack(good, good + 2, 8, 256, by(c), good, good, good, None) == wq.WQ_ERR_ALIGNMENT
+    # matmul
+    assert L.wq_w4a16_gemm(good, good, good, good, 0, 8, 256, by(c), good, None, 0, None) == wq.WQ_ERR_INVALID_ARG
+    assert L.wq_w4a16_gemm(good + 4, good, good, good, 1, 8, 256, by(c), good, None, 0, None) == wq.WQ_ERR_ALIGNMENT
+    assert L.wq_w4a16_gemm(good, good, good, good, 1, 8, 256, by(c), None, None, 0, None) == wq.WQ_ERR_INVALID_ARG
+    assert L.wq_unpack_dequant(good, good, good, 8, 256, by(_cfg(wq, bits=6)), good, None) == wq.WQ_ERR_UNSUPPORTED
+    assert wq.wq_gemm_workspace_bytes(1, 4096, 4096) == 0

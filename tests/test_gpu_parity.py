@@ -1,0 +1,276 @@
+"""CUDA path vs the CPU oracle, element by element, through the C ABI.
+
+Integer outputs (codes, packed words, steps, zeros) must match bit for bit;
+matmul outputs must meet relative L2 error <= 1e-3 and max abs error <=
+1e-2 * max|y| against the oracle's fp64 matmul of the dequantized weight.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+import synth
+
+pytestmark = pytest.mark.gpu
+
+REL_L2 = 1e-3
+MAX_ABS = 1e-2
+
+
+@pytest.fixture(scope="module")
+def wq():
+    from weight_only_quantization_group_b200 import build
+    build.build()
+    import weight_only_quantization_group_b200 as m
+    assert torch.cuda.is_available()
+    return m
+
+
+def dev(a):
+    return torch.from_numpy(np.ascontiguousarray(a)).cuda()
+
+
+def gpu_quantize(wq, W, s, bits, sym):
+    packed, steps, zeros = wq.wq_quantize_pack(dev(W), None if s is None else dev(s), bits=bits, symmetric=sym)
+    assert wq.wq_get_last_device_error() == 0
+    return packed, steps, zeros
+
+
+def assert_quant_parity(wq, W, s, bits, sym):
+    codes, st, z = O.quantize_groups(W, bits, 128, sym, s16=s)
+    words = O.pack_codes(codes, bits).reshape(-1)
+    packed, steps, zeros = gpu_quantize(wq, W, s, bits, sym)
+    gs, gz = steps.cpu().numpy(), zeros.cpu().numpy()
+    assert np.array_equal(gs.view(np.uint16), st.view(np.uint16)), "steps differ"
+    assert np.array_equal(gz.view(np.uint16), z.view(np.uint16)), "zeros differ"
+    gp = packed.cpu().numpy().view(np.uint32)
+    assert gp.size == words.size
+    bad = np.flatnonzero(gp != words)
+    assert bad.size == 0, f"{bad.size} packed words differ, first at {bad[:5]}"
+    return (codes, st, z), (packed, steps, zeros)
+
+
+def assert_close(y, yref):
+    y = np.asarray(y, dtype=np.float64)
+    rel = np.linalg.norm(y - yref) / max(np.linalg.norm(yref), 1e-300)
+    mab = np.max(np.abs(y - yref)) / max(np.max(np.abs(yref)), 1e-300)
+    assert rel <= REL_L2 and mab <= MAX_ABS, (rel, mab)
+    return rel, mab
+
+
+def _awq_scale(K, seed):
+    g = np.random.default_rng(seed)
+    return np.exp(g.normal(0, 0.7, K)).astype(np.float16)
+
+
+# ---------------------------------------------------------------------------
+# S3 quantize + pack
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("bits", [3, 4])
+@pytest.mark.parametrize("sym", [False, True])
+@pytest.mark.parametrize("awq", [False, True])
+def test_quantize_pack_parity_ragged(wq, bits, sym, awq):
+    g = synth.rng(100 + bits)
+    W = synth.weight(g, 333, 1152, 0.02, channel_frac=0.01, channel_mult=10.0, heavy_frac=0.01)
+    s = _awq_scale(1152, 7) if awq else None
+    assert_quant_parity(wq, W, s, bits, sym)
+
+
+def test_quantize_pack_edge_groups(wq):
+    g = np.random.default_rng(1)
+    W = g.normal(0, 0.02, (24, 512))
+    W[0] = 0.0                                   # all-zero groups -> step 1, zero 0
+    W[1, :128] = 0.01                            # constant group
+    W[2, :128] = np.abs(W[2, :128]) + 0.001      # group above 0
+    W[3, 128:256] = -np.abs(W[3, 128:256]) - 1e-3
+    W[4] *= 1e-5                                 # tiny values -> subnormal fp16 steps
+    W[5] *= 500.0                                # large values
+    W[6, ::2] = 0.0
+    W16 = W.astype(np.float16)
+    for bits in (3, 4):
+        for sym in (False, True):
+            assert_quant_parity(wq, W16, None, bits, sym)
+
+
+def test_quantize_pack_small_linear(wq):
+    c = synth.config_small_linear(0)
+    assert_quant_parity(wq, c.W, None, 4, False)
+
+
+def test_quantize_pack_llama7b_full(wq):
+    for c in synth.config_llama7b_decode(1):
+        assert_quant_parity(wq, c.W, None, 4, False)
+
+
+@pytest.mark.parametrize("bits", [3, 4])
+def test_quantize_pack_llama65b_full(wq, bits):
+    c = synth.config_llama65b_decode(bits)
+    assert_quant_parity(wq, c.W, None, bits, False)
+
+
+@pytest.mark.parametrize("bits", [3, 4])
+def test_unpack_dequant_bit_exact(wq, bits):
+    g = synth.rng(200)
+    W = synth.weight(g, 77, 768, 0.02, channel_frac=0.02, channel_mult=8.0)
+    (codes, st, z), (packed, steps, zeros) = assert_quant_parity(wq, W, None, bits, False)
+    out = wq.wq_unpack_dequant(packed, steps, zeros, 77, 768, bits=bits).cpu().numpy()
+    ref = O.dequantize(codes, st, z, 128).astype(np.float16)
+    assert np.array_equal(out.view(np.uint16), ref.view(np.uint16))
+
+
+# ---------------------------------------------------------------------------
+# S5 GEMV (small M)
+# ---------------------------------------------------------------------------
+
+def run_gemm(wq, X, quant_gpu, N, bits, sym=False):
+    packed, steps, zeros = quant_gpu
+    Y = wq.wq_w4a16_gemm(dev(X), packed, steps, zeros, N, bits=bits, symmetric=sym)
+    assert wq.wq_get_last_device_error() == 0
+    return Y.cpu().numpy()
+
+
+@pytest.mark.parametrize("bits", [3, 4])
+@pytest.mark.parametrize("M", [1, 2, 3, 5, 8, 11])
+@pytest.mark.parametrize("NK", [(333, 1152), (64, 128), (1000, 4096), (17, 11008)])
+def test_gemv_parity_ragged(wq, bits, M, NK):
+    N, K = NK
+    g = synth.rng(300 + M + bits)
+    W = synth.weight(g, N, K, 0.02, channel_frac=0.01, channel_mult=10.0)
+    X = synth.activations(g, M, K, channel_frac=0.01, channel_mult=20.0)
+    (codes, st, z), qg = assert_quant_parity(wq, W, None, bits, False)
+    Y = run_gemm(wq, X, qg, N, bits)
+    assert_close(Y, O.gemm_ref(X, codes, st, z, 128))
+
+
+@pytest.mark.parametrize("bits", [3, 4])
+def test_gemv_symmetric(wq, bits):
+    g = synth.rng(400)
+    W = synth.weight(g, 256, 2048, 0.02)
+    X = synth.activations(g, 2, 2048)
+    (codes, st, z), qg = assert_quant_parity(wq, W, None, bits, True)
+    assert_close(run_gemm(wq, X, qg, 256, bits, sym=True), O.gemm_ref(X, codes, st, z, 128))
+
+
+def _gemv_error_bound(X, steps):
+    """Bound on the GEMV's rounding error per output: the kernel forms
+    sum_k x_k (q_k - z) from fp32 accumulators that carry a 1024 offset per
+    product (16 products per accumulator, each sum rounded at 2^-24), so the
+    error is below 3 * 16 * 1100 * 2^-24 * step * sum|x| per 32-channel chunk."""
+    K = X.shape[1]
+    ax = np.abs(X.astype(np.float64)).reshape(X.shape[0], K // 128, 128).sum(axis=2)   # [M][G]
+    return (3 * 16 * 1100 * 2.0 ** -24) * (ax @ steps.astype(np.float64).T) + 2.0 ** -24
+
+
+def test_gemv_closed_forms(wq):
+    """All codes equal to the zero point -> Y == 0 up to the kernel's rounding
+    bound; one nonzero code -> Y = x_k (q - zero) step."""
+    N, K = 48, 1024
+    g = np.random.default_rng(2)
+    X = synth.activations(synth.rng(3), 1, K)
+    zeros = g.integers(0, 16, (N, K // 128)).astype(np.float16)
+    steps = g.uniform(0.001, 0.1, (N, K // 128)).astype(np.float16)
+    bound = _gemv_error_bound(X, steps)
+    codes = np.repeat(zeros.astype(np.uint8), 128, axis=1)
+    packed = dev(O.pack_codes(codes, 4).reshape(-1).view(np.int32))
+    Y = run_gemm(wq, X, (packed, dev(steps), dev(zeros)), N, 4)
+    assert np.all(np.abs(Y.astype(np.float64)) <= bound)
+    n, k = 21, 517
+    codes[n, k] = (int(zeros[n, k // 128]) + 5) % 16
+    packed = dev(O.pack_codes(codes, 4).reshape(-1).view(np.int32))
+    Y = run_gemm(wq, X, (packed, dev(steps), dev(zeros)), N, 4).astype(np.float64)
+    ref = O.gemm_ref(X, codes, steps, zeros, 128)
+    others = np.delete(np.arange(N), n)
+    assert np.all(np.abs(Y[:, others]) <= bound[:, others])
+    assert abs(Y[0, n] - ref[0, n]) <= bound[0, n] + 2 ** -11 * abs(ref[0, n])
+
+
+def test_gemv_small_linear(wq):
+    c = synth.config_small_linear(0)
+    (codes, st, z), qg = assert_quant_parity(wq, c.W, None, 4, False)
+    assert_close(run_gemm(wq, c.X, qg, 128, 4), O.gemm_ref(c.X, codes, st, z, 128))
+
+
+def test_gemv_llama7b_block_full(wq):
+    for c in synth.config_llama7b_decode(1):
+        N = c.W.shape[0]
+        (codes, st, z), qg = assert_quant_parity(wq, c.W, None, 4, False)
+        assert_close(run_gemm(wq, c.X, qg, N, 4), O.gemm_ref(c.X, codes, st, z, 128))
+
+
+@pytest.mark.parametrize("bits", [3, 4])
+def test_gemv_llama65b_full(wq, bits):
+    c = synth.config_llama65b_decode(bits)
+    (codes, st, z), qg = assert_quant_parity(wq, c.W, None, bits, False)
+    assert_close(run_gemm(wq, c.X, qg, 8192, bits), O.gemm_ref(c.X, codes, st, z, 128))
+
+
+def test_smallm_sweep_full_weight(wq):
+    """K=8192, N=28672 at every M of the sweep, against the fp64 oracle."""
+    c = synth.config_smallm_sweep(1)
+    (codes, st, z), qg = assert_quant_parity(wq, c.W, None, 4, False)
+    D = O.dequantize(codes, st, z, 128)
+    for M in synth.SMALLM_SWEEP:
+        X = synth.smallm_activations(M)
+        Y = run_gemm(wq, X, qg, 28672, 4)
+        assert_close(Y, X.astype(np.float64) @ D.T)
+
+
+# ---------------------------------------------------------------------------
+# S6 tensor-core path (tcgen05), forced, both placements of the A operand
+# ---------------------------------------------------------------------------
+
+@pytest.fixture
+def tc_path(wq, request):
+    placement = request.param
+    wq.wq_set_option(wq.WQ_OPT_GEMM_PATH, wq.WQ_PATH_TENSOR_CORE)
+    wq.wq_set_option(wq.WQ_OPT_TC_A_OPERAND, wq.WQ_TC_A_TMEM if placement == "tmem" else wq.WQ_TC_A_SMEM)
+    yield placement
+    wq.wq_set_option(wq.WQ_OPT_GEMM_PATH, wq.WQ_PATH_AUTO)
+    wq.wq_set_option(wq.WQ_OPT_TC_A_OPERAND, wq.WQ_TC_A_TMEM)
+
+
+@pytest.mark.parametrize("tc_path", ["tmem", "smem"], indirect=True)
+@pytest.mark.parametrize("M", [1, 16, 17, 48, 64, 100, 128, 200, 256, 300])
+@pytest.mark.parametrize("NK", [(333, 1152), (1000, 4096)])
+def test_tc_gemm_parity(wq, tc_path, M, NK):
+    N, K = NK
+    g = synth.rng(500 + M)
+    W = synth.weight(g, N, K, 0.02, channel_frac=0.01, channel_mult=10.0)
+    X = synth.activations(g, M, K, channel_frac=0.01, channel_mult=20.0)
+    (codes, st, z), qg = assert_quant_parity(wq, W, None, 4, False)
+    assert_close(run_gemm(wq, X, qg, N, 4), O.gemm_ref(X, codes, st, z, 128))
+
+
+@pytest.mark.parametrize("tc_path", ["tmem", "smem"], indirect=True)
+def test_tc_gemm_symmetric_and_closed_form(wq, tc_path):
+    N, K, M = 256, 1024, 32
+    g = np.random.default_rng(21)
+    X = synth.activations(synth.rng(22), M, K)
+    zeros = np.full((N, K // 128), 8, np.float16)
+    steps = g.uniform(0.001, 0.1, (N, K // 128)).astype(np.float16)
+    codes = np.full((N, K), 8, np.uint8)
+    packed = dev(O.pack_codes(codes, 4).reshape(-1).view(np.int32))
+    assert np.all(run_gemm(wq, X, (packed, dev(steps), dev(zeros)), N, 4, sym=True) == 0)
+    W = synth.weight(synth.rng(23), N, K, 0.02)
+    (codes, st, z), qg = assert_quant_parity(wq, W, None, 4, True)
+    assert_close(run_gemm(wq, X, qg, N, 4, sym=True), O.gemm_ref(X, codes, st, z, 128))
+
+
+def test_tc_matches_gemv_path(wq):
+    """Both kernels on the same inputs agree with each other as well as the oracle."""
+    N, K, M = 512, 2048, 24
+    g = synth.rng(600)
+    W = synth.weight(g, N, K, 0.02)
+    X = synth.activations(g, M, K)
+    (codes, st, z), qg = assert_quant_parity(wq, W, None, 4, False)
+    ref = O.gemm_ref(X, codes, st, z, 128)
+    outs = {}
+    for path in (wq.WQ_PATH_GEMV, wq.WQ_PATH_TENSOR_CORE):
+        wq.wq_set_option(wq.WQ_OPT_GEMM_PATH, path)
+        try:
+            outs[path] = run_gemm(wq, X, qg, N, 4)
+        finally:
+            wq.wq_set_option(wq.WQ_OPT_GEMM_PATH, wq.WQ_PATH_AUTO)
+        assert_close(outs[path], ref)
+    assert_close(outs[wq.WQ_PATH_TENSOR_CORE], outs[wq.WQ_PATH_GEMV].astype(np.float64))

@@ -1,0 +1,241 @@
+"""Python binding of libwq.so: group-wise weight-only quantization for B200.
+
+A thin ctypes layer over the C ABI declared in ``include/wq.h``. Each
+``wq_*`` function here has the same name and meaning as the C entry point; it
+only checks tensor metadata, allocates outputs with torch (device memory is
+the one thing torch provides), passes raw pointers and the current CUDA
+stream, and raises :class:`WQError` on a non-OK status. Every step of the
+computation runs in the library's CUDA kernels; there is no CPU fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+__all__ = [
+    "WQError",
+    "lib",
+    "library_path",
+    "wq_abi_version",
+    "wq_status_string",
+    "wq_packed_words",
+    "wq_quantize_pack",
+    "wq_unpack_dequant",
+    "wq_gemm_workspace_bytes",
+    "wq_w4a16_gemm",
+    "wq_get_last_device_error",
+    "wq_set_option",
+    "wq_get_option",
+    "EXPORTED_SYMBOLS",
+]
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+library_path = os.path.join(_HERE, "libwq.so")
+
+# Every symbol include/wq.h declares.
+EXPORTED_SYMBOLS = (
+    "wq_abi_version",
+    "wq_status_string",
+    "wq_packed_words",
+    "wq_quantize_pack",
+    "wq_unpack_dequant",
+    "wq_gemm_workspace_bytes",
+    "wq_w4a16_gemm",
+    "wq_get_last_device_error",
+    "wq_set_option",
+    "wq_get_option",
+)
+
+WQ_OK = 0
+WQ_ERR_INVALID_ARG = 1
+WQ_ERR_UNSUPPORTED = 2
+WQ_ERR_ALIGNMENT = 3
+WQ_ERR_CUDA = 4
+WQ_ERR_TIMEOUT = 5
+WQ_ERR_WORKSPACE = 6
+WQ_ERR_RANGE = 7
+
+WQ_OPT_GEMM_PATH = 1
+WQ_OPT_CROSSOVER_M = 2
+WQ_OPT_TC_A_OPERAND = 3
+WQ_PATH_AUTO = 0
+WQ_PATH_GEMV = 1
+WQ_PATH_TENSOR_CORE = 2
+WQ_TC_A_TMEM = 0
+WQ_TC_A_SMEM = 1
+WQ_OPT_GEMV_VARIANT = 4
+WQ_GEMV_OFFSET_SUMS = 0
+WQ_GEMV_EXACT = 1
+
+
+class WQError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = int(status)
+        super().__init__(f"{where}: {lib().wq_status_string(self.status).decode()}")
+
+
+class _Cfg(ctypes.Structure):
+    _fields_ = [("bits", ctypes.c_int32), ("group_size", ctypes.c_int32), ("symmetric", ctypes.c_int32)]
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(library_path):
+        raise ImportError(
+            f"{library_path} is missing: build the CUDA library first "
+            "(python -m weight_only_quantization_group_b200.build)")
+    L = ctypes.CDLL(library_path)
+    vp, i32, i64, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
+    cfgp = ctypes.POINTER(_Cfg)
+    sig = {
+        "wq_abi_version": (i32, []),
+        "wq_status_string": (ctypes.c_char_p, [i32]),
+        "wq_packed_words": (sz, [i64, i64, cfgp]),
+        "wq_quantize_pack": (i32, [vp, vp, i64, i64, cfgp, vp, vp, vp, vp]),
+        "wq_unpack_dequant": (i32, [vp, vp, vp, i64, i64, cfgp, vp, vp]),
+        "wq_gemm_workspace_bytes": (sz, [i64, i64, i64, cfgp]),
+        "wq_w4a16_gemm": (i32, [vp, vp, vp, vp, i64, i64, i64, cfgp, vp, vp, sz, vp]),
+        "wq_get_last_device_error": (i32, [vp]),
+        "wq_set_option": (i32, [i32, i64]),
+        "wq_get_option": (i64, [i32]),
+    }
+    for name, (res, args) in sig.items():
+        f = getattr(L, name)
+        f.restype = res
+        f.argtypes = args
+    return L
+
+
+_lib_handle = None
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded libwq.so (loaded on first use; raises if it is missing)."""
+    global _lib_handle
+    if _lib_handle is None:
+        _lib_handle = _load()
+    return _lib_handle
+
+
+class _LazyLib:
+    def __getattr__(self, name):
+        return getattr(lib(), name)
+
+
+_lib = _LazyLib()
+
+
+def _cfg(bits: int, group_size: int, symmetric: bool) -> _Cfg:
+    return _Cfg(int(bits), int(group_size), 1 if symmetric else 0)
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _ptr(t: torch.Tensor | None) -> int | None:
+    return None if t is None else t.data_ptr()
+
+
+def _check(t: torch.Tensor, dtype, name: str):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def _raise(st: int, where: str):
+    if st != WQ_OK:
+        raise WQError(st, where)
+
+
+def wq_abi_version() -> int:
+    return int(_lib.wq_abi_version())
+
+
+def wq_status_string(status: int) -> str:
+    return _lib.wq_status_string(int(status)).decode()
+
+
+def wq_packed_words(N: int, K: int, bits: int = 4, group_size: int = 128, symmetric: bool = False) -> int:
+    c = _cfg(bits, group_size, symmetric)
+    return int(_lib.wq_packed_words(N, K, ctypes.byref(c)))
+
+
+def wq_quantize_pack(W: torch.Tensor, s: torch.Tensor | None = None, *, bits: int = 4, group_size: int = 128,
+                     symmetric: bool = False, out=None, stream=None):
+    """Quantize + pack an fp16 [N][K] weight; returns (packed u32 as int32, steps, zeros)."""
+    _check(W, torch.float16, "W")
+    if s is not None:
+        _check(s, torch.float16, "s")
+    N, K = W.shape
+    c = _cfg(bits, group_size, symmetric)
+    nw = int(_lib.wq_packed_words(N, K, ctypes.byref(c)))
+    if out is None:
+        G = K // group_size if group_size > 0 else 0
+        packed = torch.empty(max(nw, 1), dtype=torch.int32, device=W.device)
+        steps = torch.empty((N, G), dtype=torch.float16, device=W.device)
+        zeros = torch.empty((N, G), dtype=torch.float16, device=W.device)
+    else:
+        packed, steps, zeros = out
+    st = _lib.wq_quantize_pack(_ptr(W), _ptr(s), N, K, ctypes.byref(c), _ptr(packed), _ptr(steps),
+                               _ptr(zeros), _stream(stream))
+    _raise(st, "wq_quantize_pack")
+    return packed, steps, zeros
+
+
+def wq_unpack_dequant(packed: torch.Tensor, steps: torch.Tensor, zeros: torch.Tensor, N: int, K: int, *,
+                      bits: int = 4, group_size: int = 128, symmetric: bool = False, out=None, stream=None):
+    """fp16 [N][K] = fp16((q - zero) * step) from the packed form."""
+    c = _cfg(bits, group_size, symmetric)
+    if out is None:
+        out = torch.empty((N, K), dtype=torch.float16, device=packed.device)
+    st = _lib.wq_unpack_dequant(_ptr(packed), _ptr(steps), _ptr(zeros), N, K, ctypes.byref(c), _ptr(out),
+                                _stream(stream))
+    _raise(st, "wq_unpack_dequant")
+    return out
+
+
+def wq_gemm_workspace_bytes(M: int, N: int, K: int, *, bits: int = 4, group_size: int = 128,
+                            symmetric: bool = False) -> int:
+    c = _cfg(bits, group_size, symmetric)
+    return int(_lib.wq_gemm_workspace_bytes(M, N, K, ctypes.byref(c)))
+
+
+def wq_w4a16_gemm(X: torch.Tensor, packed: torch.Tensor, steps: torch.Tensor, zeros: torch.Tensor, N: int, *,
+                  bits: int = 4, group_size: int = 128, symmetric: bool = False, out=None, workspace=None,
+                  stream=None):
+    """Y[M][N] = X[M][K] * deq(W)^T with fp32 accumulation; returns Y (fp16)."""
+    _check(X, torch.float16, "X")
+    M, K = X.shape
+    c = _cfg(bits, group_size, symmetric)
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.float16, device=X.device)
+    ws_ptr, ws_bytes = None, 0
+    if workspace is not None:
+        ws_ptr, ws_bytes = workspace.data_ptr(), workspace.numel() * workspace.element_size()
+    st = _lib.wq_w4a16_gemm(_ptr(X), _ptr(packed), _ptr(steps), _ptr(zeros), M, N, K, ctypes.byref(c),
+                            _ptr(out), ws_ptr, ws_bytes, _stream(stream))
+    _raise(st, "wq_w4a16_gemm")
+    return out
+
+
+def wq_get_last_device_error(stream=None) -> int:
+    """Synchronize the stream and return (then clear) the device error flag."""
+    return int(_lib.wq_get_last_device_error(_stream(stream)))
+
+
+def wq_set_option(option: int, value: int) -> None:
+    """Set a process-wide tuning option (see include/wq.h)."""
+    _raise(_lib.wq_set_option(int(option), int(value)), "wq_set_option")
+
+
+def wq_get_option(option: int) -> int:
+    return int(_lib.wq_get_option(int(option)))

@@ -1,0 +1,198 @@
+// C ABI of libwq.so: argument validation, dispatch, and the device error flag.
+// Every entry point validates on the host, enqueues on the caller's stream and
+// returns; none allocates device memory.
+#include <mutex>
+
+#include "wq_common.cuh"
+
+namespace wq {
+cudaError_t launch_quantize_pack(const void* W, const void* s, int64_t N, int64_t K, int bits, bool sym,
+                                 uint32_t* packed, void* steps, void* zeros, int* err, cudaStream_t st);
+cudaError_t launch_unpack_dequant(const uint32_t* packed, const void* steps, const void* zeros, int64_t N,
+                                  int64_t K, int bits, void* out, cudaStream_t st);
+cudaError_t launch_gemv(const void* X, const uint32_t* packed, const void* steps, const void* zeros, int64_t M,
+                        int64_t N, int64_t K, int bits, void* Y, cudaStream_t st, bool exact);
+cudaError_t launch_gemm_tc(const void* X, const uint32_t* packed, const void* steps, const void* zeros, int64_t M,
+                           int64_t N, int64_t K, void* Y, int* err, cudaStream_t st, bool a_tmem);
+}  // namespace wq
+
+// One flag per device (each device holds its own copy of a __device__ variable).
+__device__ int g_wq_device_error;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+std::mutex g_flag_mu;
+int* g_flag_addr[kMaxDevices] = {};
+
+// Address of this device's error flag; looked up once per device with the
+// device current. Returns nullptr on failure.
+int* device_flag() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lk(g_flag_mu);
+  if (g_flag_addr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_wq_device_error) != cudaSuccess) return nullptr;
+    g_flag_addr[dev] = static_cast<int*>(p);
+  }
+  return g_flag_addr[dev];
+}
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+int32_t check_cfg(const wq_quant_cfg* cfg) {
+  if (cfg == nullptr) return WQ_ERR_INVALID_ARG;
+  if (cfg->bits != 3 && cfg->bits != 4) return cfg->bits >= 2 && cfg->bits <= 8 ? WQ_ERR_UNSUPPORTED : WQ_ERR_INVALID_ARG;
+  if (cfg->group_size != wq::kGroup)
+    return (cfg->group_size == 32 || cfg->group_size == 64) ? WQ_ERR_UNSUPPORTED : WQ_ERR_INVALID_ARG;
+  if (cfg->symmetric != 0 && cfg->symmetric != 1) return WQ_ERR_INVALID_ARG;
+  return WQ_OK;
+}
+
+int32_t check_shape(int64_t N, int64_t K) {
+  if (N < 1 || K < wq::kGroup || K % wq::kGroup != 0) return WQ_ERR_INVALID_ARG;
+  if (N > (int64_t)INT32_MAX / 2 || K > (int64_t)INT32_MAX / 2) return WQ_ERR_INVALID_ARG;
+  return WQ_OK;
+}
+
+int32_t cuda_status(cudaError_t e) { return e == cudaSuccess ? WQ_OK : WQ_ERR_CUDA; }
+
+// Process-wide tuning options (wq_set_option).
+int64_t g_opt_gemm_path = WQ_PATH_AUTO;
+int64_t g_opt_crossover_m = 16;
+int64_t g_opt_tc_a_operand = WQ_TC_A_TMEM;
+int64_t g_opt_gemv_variant = WQ_GEMV_OFFSET_SUMS;
+
+}  // namespace
+
+extern "C" {
+
+int32_t wq_abi_version(void) { return WQ_ABI_VERSION; }
+
+const char* wq_status_string(int32_t s) {
+  switch (s) {
+    case WQ_OK: return "WQ_OK";
+    case WQ_ERR_INVALID_ARG: return "WQ_ERR_INVALID_ARG: invalid argument";
+    case WQ_ERR_UNSUPPORTED: return "WQ_ERR_UNSUPPORTED: configuration not supported";
+    case WQ_ERR_ALIGNMENT: return "WQ_ERR_ALIGNMENT: pointer alignment";
+    case WQ_ERR_CUDA: return "WQ_ERR_CUDA: CUDA runtime error";
+    case WQ_ERR_TIMEOUT: return "WQ_ERR_TIMEOUT: bounded device wait gave up";
+    case WQ_ERR_WORKSPACE: return "WQ_ERR_WORKSPACE: workspace missing or too small";
+    case WQ_ERR_RANGE: return "WQ_ERR_RANGE: value not finite in fp16";
+  }
+  return "unknown wq status";
+}
+
+size_t wq_packed_words(int64_t N, int64_t K, const wq_quant_cfg* cfg) {
+  if (check_cfg(cfg) != WQ_OK || check_shape(N, K) != WQ_OK) return 0;
+  return cfg->bits == 4 ? (size_t)N * (size_t)K / 8 : (size_t)N * (size_t)K * 3 / 32;
+}
+
+int32_t wq_quantize_pack(const void* W, const void* s, int64_t N, int64_t K, const wq_quant_cfg* cfg,
+                         uint32_t* packed, void* steps, void* zeros, void* stream) {
+  int32_t st = check_cfg(cfg);
+  if (st != WQ_OK) return st;
+  if ((st = check_shape(N, K)) != WQ_OK) return st;
+  if (!W || !packed || !steps || !zeros) return WQ_ERR_INVALID_ARG;
+  if (!aligned(W, 16) || !aligned(packed, 16) || (s && !aligned(s, 16)) || !aligned(steps, 4) ||
+      !aligned(zeros, 4))
+    return WQ_ERR_ALIGNMENT;
+  int* flag = device_flag();
+  if (!flag) return WQ_ERR_CUDA;
+  return cuda_status(wq::launch_quantize_pack(W, s, N, K, cfg->bits, cfg->symmetric != 0, packed, steps, zeros,
+                                              flag, static_cast<cudaStream_t>(stream)));
+}
+
+int32_t wq_unpack_dequant(const uint32_t* packed, const void* steps, const void* zeros, int64_t N, int64_t K,
+                          const wq_quant_cfg* cfg, void* W_out, void* stream) {
+  int32_t st = check_cfg(cfg);
+  if (st != WQ_OK) return st;
+  if ((st = check_shape(N, K)) != WQ_OK) return st;
+  if (!packed || !steps || !zeros || !W_out) return WQ_ERR_INVALID_ARG;
+  if (!aligned(packed, 16) || !aligned(W_out, 16) || !aligned(steps, 4) || !aligned(zeros, 4))
+    return WQ_ERR_ALIGNMENT;
+  return cuda_status(wq::launch_unpack_dequant(packed, steps, zeros, N, K, cfg->bits, W_out,
+                                               static_cast<cudaStream_t>(stream)));
+}
+
+size_t wq_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, const wq_quant_cfg* cfg) {
+  (void)M; (void)N; (void)K; (void)cfg;
+  return 0;
+}
+
+int32_t wq_w4a16_gemm(const void* X, const uint32_t* packed, const void* steps, const void* zeros, int64_t M,
+                      int64_t N, int64_t K, const wq_quant_cfg* cfg, void* Y, void* workspace,
+                      size_t workspace_bytes, void* stream) {
+  (void)workspace; (void)workspace_bytes;
+  int32_t st = check_cfg(cfg);
+  if (st != WQ_OK) return st;
+  if ((st = check_shape(N, K)) != WQ_OK) return st;
+  if (M < 1 || M > (int64_t)INT32_MAX / 2) return WQ_ERR_INVALID_ARG;
+  if (!X || !packed || !steps || !zeros || !Y) return WQ_ERR_INVALID_ARG;
+  if (!aligned(X, 16) || !aligned(packed, 16) || !aligned(steps, 2) || !aligned(zeros, 2) || !aligned(Y, 2))
+    return WQ_ERR_ALIGNMENT;
+  // Shared copy of an X slice must fit one CTA (K up to ~100k at 8 rows).
+  if ((size_t)K * 8 * 18 / 8 / 8 > 200 * 1024) return WQ_ERR_UNSUPPORTED;
+  bool tensor_core = cfg->bits == 4 && M >= g_opt_crossover_m;
+  if (g_opt_gemm_path == WQ_PATH_GEMV) tensor_core = false;
+  if (g_opt_gemm_path == WQ_PATH_TENSOR_CORE) {
+    if (cfg->bits != 4) return WQ_ERR_UNSUPPORTED;
+    tensor_core = true;
+  }
+  if (tensor_core) {
+    int* flag = device_flag();
+    if (!flag) return WQ_ERR_CUDA;
+    return cuda_status(wq::launch_gemm_tc(X, packed, steps, zeros, M, N, K, Y, flag,
+                                          static_cast<cudaStream_t>(stream), g_opt_tc_a_operand == WQ_TC_A_TMEM));
+  }
+  return cuda_status(wq::launch_gemv(X, packed, steps, zeros, M, N, K, cfg->bits, Y,
+                                     static_cast<cudaStream_t>(stream), g_opt_gemv_variant == WQ_GEMV_EXACT));
+}
+
+int32_t wq_set_option(int32_t option, int64_t value) {
+  switch (option) {
+    case WQ_OPT_GEMM_PATH:
+      if (value < WQ_PATH_AUTO || value > WQ_PATH_TENSOR_CORE) return WQ_ERR_INVALID_ARG;
+      g_opt_gemm_path = value;
+      return WQ_OK;
+    case WQ_OPT_CROSSOVER_M:
+      if (value < 1) return WQ_ERR_INVALID_ARG;
+      g_opt_crossover_m = value;
+      return WQ_OK;
+    case WQ_OPT_TC_A_OPERAND:
+      if (value != WQ_TC_A_TMEM && value != WQ_TC_A_SMEM) return WQ_ERR_INVALID_ARG;
+      g_opt_tc_a_operand = value;
+      return WQ_OK;
+    case WQ_OPT_GEMV_VARIANT:
+      if (value != WQ_GEMV_OFFSET_SUMS && value != WQ_GEMV_EXACT) return WQ_ERR_INVALID_ARG;
+      g_opt_gemv_variant = value;
+      return WQ_OK;
+  }
+  return WQ_ERR_INVALID_ARG;
+}
+
+int64_t wq_get_option(int32_t option) {
+  switch (option) {
+    case WQ_OPT_GEMM_PATH: return g_opt_gemm_path;
+    case WQ_OPT_CROSSOVER_M: return g_opt_crossover_m;
+    case WQ_OPT_TC_A_OPERAND: return g_opt_tc_a_operand;
+    case WQ_OPT_GEMV_VARIANT: return g_opt_gemv_variant;
+  }
+  return -1;
+}
+
+int32_t wq_get_last_device_error(void* stream) {
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return WQ_ERR_CUDA;
+  int* flag = device_flag();
+  if (!flag) return WQ_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpy(&v, flag, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return WQ_ERR_CUDA;
+  if (v != 0) {
+    const int zero = 0;
+    if (cudaMemcpy(flag, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess) return WQ_ERR_CUDA;
+  }
+  return v;
+}
+
+}  // extern "C"

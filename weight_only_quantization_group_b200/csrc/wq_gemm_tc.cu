@@ -1,0 +1,337 @@
+// S6: W4A16 matmul on the 5th-generation tensor cores for M = 16..256 rows of X.
+//
+// When M grows the weight-only matmul stops being a pure weight stream and
+// becomes a dense contraction ("Quantising Large Language Models for
+// Efficient Inference", "Weight-only vs weight-and-activation quantisation":
+// weights are dequantized inside the matmul; tensor cores pay off for larger
+// batches). The weight is still read once, packed, and dequantized on chip.
+//
+// Tile: one CTA owns 128 output channels n and all M rows of X ("swap AB":
+// the dequantized weight tile is the 128-row A operand, X is the B operand
+// with N_mma = M rounded up to 16, D = W X^T lives in tensor memory as
+// [128 lanes = n][M columns]). K advances in stages of 64 input channels:
+//   warp 0    TMA producer: X tile (128-byte swizzle) + packed weight tile
+//   warp 1    TMEM owner and single-thread tcgen05.mma issuer
+//   warps 2-5 dequantize the packed tile (one output channel per thread) into
+//             the A operand -- either shared memory in the canonical 128-byte
+//             swizzled K-major layout, or tensor memory (A_TMEM) -- then run
+//             the epilogue (tcgen05.ld -> fp16 -> Y).
+// Every mbarrier wait is bounded; on a timeout the kernel latches
+// WQ_ERR_TIMEOUT, drains its own copies, frees its tensor memory and returns.
+#include "wq_sm100.cuh"
+
+namespace wq {
+
+using namespace sm100;
+
+constexpr int kTcThreads = 192;
+constexpr int kTcBK = 64;              // input channels per stage
+constexpr int kTcRows = 128;           // output channels per CTA
+constexpr int kTcPackedStage = kTcRows * kTcBK / 2;  // 4096 bytes
+constexpr int kTcAStage = kTcRows * kTcBK * 2;       // 16384 bytes
+constexpr long long kSpinLimitCycles = 4000000000LL; // ~2 s at 2 GHz
+
+struct TcArgs {
+  const __half* steps;
+  const __half* zeros;
+  __half* Y;
+  int M, N, K;
+  int BN;          // MMA N (M rounded up to 16)
+  int stages;
+  uint32_t tmem_cols;
+  int* err;
+};
+
+__device__ __forceinline__ __half2 u2h(uint32_t u) { return *reinterpret_cast<__half2*>(&u); }
+__device__ __forceinline__ uint32_t h2u(__half2 h) { return *reinterpret_cast<uint32_t*>(&h); }
+
+// Eight 4-bit codes (one packed word: k0..k7) -> four fp16 pairs
+// fp16_rn((q - zero) * step), in k order. (1024+q) - (1024+zero) and
+// (1024+16q)/16 - (64+zero) are exact, so the only rounding is the product.
+__device__ __forceinline__ uint4 dequant_word4(uint32_t w, __half2 zz, __half2 zz16n, __half2 s2) {
+  const __half2 one16 = __float2half2_rn(0.0625f);
+  const uint32_t w8 = w >> 8;
+  const uint32_t p0 = and_or(w, 0x000F000Fu, kHalf2Magic);
+  const uint32_t p1 = and_or(w, 0x00F000F0u, kHalf2Magic);
+  const uint32_t p2 = and_or(w8, 0x000F000Fu, kHalf2Magic);
+  const uint32_t p3 = and_or(w8, 0x00F000F0u, kHalf2Magic);
+  uint4 r;
+  r.x = h2u(__hmul2(__hsub2(u2h(p0), zz), s2));
+  r.y = h2u(__hmul2(__hfma2(u2h(p1), one16, zz16n), s2));
+  r.z = h2u(__hmul2(__hsub2(u2h(p2), zz), s2));
+  r.w = h2u(__hmul2(__hfma2(u2h(p3), one16, zz16n), s2));
+  return r;
+}
+
+template <bool A_TMEM>
+__global__ void __launch_bounds__(kTcThreads, 1)
+w4a16_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmP,
+                     TcArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int S = a.stages;
+  const int b_bytes = a.BN * 128;
+  const int stage_bytes = b_bytes + (A_TMEM ? 0 : kTcAStage) + kTcPackedStage;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + (size_t)S * stage_bytes);
+  uint64_t* deq = full + S;
+  uint64_t* empty = deq + S;
+  uint64_t* accum = empty + S;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accum + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  auto stageB = [&](int s) { return smem + (size_t)s * stage_bytes; };
+  auto stageA = [&](int s) { return smem + (size_t)s * stage_bytes + b_bytes; };
+  auto stageP = [&](int s) { return smem + (size_t)s * stage_bytes + b_bytes + (A_TMEM ? 0 : kTcAStage); };
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int n0 = blockIdx.x * kTcRows;
+  const int KT = a.K / kTcBK;
+  const int G = a.K / kGroup;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&deq[s], 128);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(accum, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, a.tmem_cols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t tmem_a = tmem + (uint32_t)a.BN;  // A stages follow the accumulator columns
+
+  if (warp == 0) {
+    // ---------------------------------------------------------- TMA producer
+    if (lane == 0) {
+      prefetch_tensormap(&tmX);
+      prefetch_tensormap(&tmP);
+      int issued = 0;
+      for (int kt = 0; kt < KT; ++kt) {
+        if (*abort_flag) break;
+        const int s = kt % S, u = kt / S;
+        if (u > 0 && !mbar_wait(&empty[s], (u - 1) & 1, a.err, kSpinLimitCycles)) { *abort_flag = 1; break; }
+        mbar_arrive_expect_tx(&full[s], (uint32_t)(b_bytes + kTcPackedStage));
+        tma_load_2d(stageB(s), &tmX, kt * kTcBK, 0, &full[s]);
+        tma_load_2d(stageP(s), &tmP, kt * (kTcBK / 8), n0, &full[s]);
+        issued = kt + 1;
+      }
+      // Drain: every copy this thread issued has landed before the CTA exits.
+      for (int kt = issued > S ? issued - S : 0; kt < issued; ++kt)
+        mbar_wait(&full[kt % S], (kt / S) & 1, a.err, kSpinLimitCycles);
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc = idesc_f16_f32(kTcRows, a.BN);
+      int committed = -1;
+      for (int kt = 0; kt < KT; ++kt) {
+        if (*abort_flag) break;
+        const int s = kt % S, u = kt / S;
+        if (!mbar_wait(&deq[s], u & 1, a.err, kSpinLimitCycles)) { *abort_flag = 1; break; }
+        tc_fence_after();
+        const uint32_t b_addr = smem_u32(stageB(s));
+#pragma unroll
+        for (int j = 0; j < kTcBK / 16; ++j) {
+          const uint64_t bd = desc_kmajor_sw128(b_addr + 32 * j);
+          const uint32_t acc = (kt > 0 || j > 0) ? 1u : 0u;
+          if (A_TMEM) {
+            mma_f16_ts(tmem, tmem_a + (uint32_t)(s * (kTcBK / 2) + 8 * j), bd, idesc, acc);
+          } else {
+            mma_f16_ss(tmem, desc_kmajor_sw128(smem_u32(stageA(s)) + 32 * j), bd, idesc, acc);
+          }
+        }
+        mma_commit(&empty[s]);
+        committed = kt;
+      }
+      mma_commit(accum);
+      if (*abort_flag && committed >= 0)  // let issued MMAs finish before teardown
+        mbar_wait(&empty[committed % S], (committed / S) & 1, a.err, kSpinLimitCycles);
+    }
+  } else {
+    // ---------------------------------------------------------- dequant + epilogue
+    const int q = warp & 3;             // TMEM lane quarter this warp may access
+    const int r = 32 * q + lane;        // output channel within the tile
+    const int n = n0 + r;
+    const bool row_ok = n < a.N;
+    __half2 s2 = __float2half2_rn(0.f), zz = s2, zz16n = s2;
+    for (int kt = 0; kt < KT; ++kt) {
+      if (__any_sync(0xffffffffu, *abort_flag != 0)) break;
+      const int s = kt % S, u = kt / S;
+      if ((kt * kTcBK) % kGroup == 0) {
+        const int g = kt * kTcBK / kGroup;
+        __half st = __float2half(0.f), zr = __float2half(0.f);
+        if (row_ok) {
+          st = a.steps[(size_t)n * G + g];
+          zr = a.zeros[(size_t)n * G + g];
+        }
+        s2 = __halves2half2(st, st);
+        const __half z1024 = __hadd(zr, __float2half(1024.f));
+        const __half z64n = __hneg(__hadd(zr, __float2half(64.f)));
+        zz = __halves2half2(z1024, z1024);
+        zz16n = __halves2half2(z64n, z64n);
+      }
+      const bool landed = mbar_wait(&full[s], u & 1, a.err, kSpinLimitCycles);
+      if (!__all_sync(0xffffffffu, landed)) { *abort_flag = 1; break; }
+      const uint4* prow = reinterpret_cast<const uint4*>(stageP(s) + r * 32);
+      const uint4 w0 = prow[0], w1 = prow[1];
+      const uint32_t words[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+      if (A_TMEM) {
+        uint32_t v[2][16];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const uint4 d = dequant_word4(words[j], zz, zz16n, s2);
+          v[j >> 2][(j & 3) * 4 + 0] = d.x;
+          v[j >> 2][(j & 3) * 4 + 1] = d.y;
+          v[j >> 2][(j & 3) * 4 + 2] = d.z;
+          v[j >> 2][(j & 3) * 4 + 3] = d.w;
+        }
+        const uint32_t ta = tmem_a + ((uint32_t)(32 * q) << 16) + (uint32_t)(s * (kTcBK / 2));
+        tmem_st16(ta, v[0]);
+        tmem_st16(ta + 16, v[1]);
+        tmem_st_wait();
+        tc_fence_before();
+      } else {
+        uint8_t* arow = stageA(s) + (r >> 3) * 1024 + (r & 7) * 128;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const uint4 d = dequant_word4(words[j], zz, zz16n, s2);
+          *reinterpret_cast<uint4*>(arow + ((j ^ (r & 7)) << 4)) = d;
+        }
+        fence_proxy_async_smem();
+      }
+      mbar_arrive(&deq[s]);
+    }
+    // Epilogue: D[n][m] from TMEM -> Y[m][n].
+    bool done = !__any_sync(0xffffffffu, *abort_flag != 0);
+    if (done) done = __all_sync(0xffffffffu, mbar_wait(accum, 0, a.err, kSpinLimitCycles));
+    if (done) {
+      tc_fence_after();
+      for (int c0 = 0; c0 < a.BN; c0 += 16) {
+        uint32_t v[16];
+        tmem_ld16(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)c0, v);
+        tmem_ld_wait();
+        if (row_ok) {
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const int m = c0 + i;
+            if (m < a.M) a.Y[(size_t)m * a.N + n] = __float2half_rn(__uint_as_float(v[i]));
+          }
+        }
+      }
+    } else {
+      *abort_flag = 1;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, a.tmem_cols);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Host side
+// ---------------------------------------------------------------------------
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (fn == nullptr) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+static int tc_stages(int BN, bool a_tmem) {
+  const int stage = BN * 128 + (a_tmem ? 0 : kTcAStage) + kTcPackedStage;
+  int s = (200 * 1024) / stage;
+  if (s > 8) s = 8;
+  if (a_tmem) {
+    // TMEM: BN accumulator columns + 32 per stage, within 256 (two CTAs per SM)
+    while (s > 2 && BN + 32 * s > 256) --s;
+  }
+  return s < 2 ? 2 : s;
+}
+
+static uint32_t pow2_cols(uint32_t c) {
+  uint32_t p = 32;
+  while (p < c) p <<= 1;
+  return p;
+}
+
+cudaError_t launch_gemm_tc(const void* X, const uint32_t* packed, const void* steps, const void* zeros, int64_t M,
+                           int64_t N, int64_t K, void* Y, int* err, cudaStream_t st, bool a_tmem) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return cudaErrorNotSupported;
+  for (int64_t m0 = 0; m0 < M; m0 += 256) {
+    const int mc = (int)((M - m0) < 256 ? (M - m0) : 256);
+    const int BN = ((mc + 15) / 16) * 16;
+    const bool use_tmem_a = a_tmem && BN <= 192;
+    CUtensorMap tmX, tmP;
+    {
+      cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)mc};
+      cuuint64_t strides[1] = {(cuuint64_t)K * 2};
+      cuuint32_t box[2] = {64, (cuuint32_t)BN};
+      cuuint32_t es[2] = {1, 1};
+      void* base = const_cast<__half*>(static_cast<const __half*>(X) + m0 * K);
+      if (enc(&tmX, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, base, dims, strides, box, es,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return cudaErrorInvalidValue;
+    }
+    {
+      cuuint64_t dims[2] = {(cuuint64_t)(K / 8), (cuuint64_t)N};
+      cuuint64_t strides[1] = {(cuuint64_t)(K / 2)};
+      cuuint32_t box[2] = {8, 128};
+      cuuint32_t es[2] = {1, 1};
+      if (enc(&tmP, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<uint32_t*>(packed), dims, strides, box, es,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return cudaErrorInvalidValue;
+    }
+    TcArgs a;
+    a.steps = static_cast<const __half*>(steps);
+    a.zeros = static_cast<const __half*>(zeros);
+    a.Y = static_cast<__half*>(Y) + m0 * N;
+    a.M = mc;
+    a.N = (int)N;
+    a.K = (int)K;
+    a.BN = BN;
+    a.stages = tc_stages(BN, use_tmem_a);
+    a.tmem_cols = pow2_cols((uint32_t)(BN + (use_tmem_a ? 32 * a.stages : 0)));
+    a.err = err;
+    const int stage = BN * 128 + (use_tmem_a ? 0 : kTcAStage) + kTcPackedStage;
+    size_t smem = 1024 + (size_t)a.stages * stage + (3 * a.stages + 1) * 8 + 16;
+    // Never more CTAs on an SM than its 512 TMEM columns can hold at once.
+    const size_t smem_floor = a.tmem_cols > 256 ? 120 * 1024 : a.tmem_cols > 128 ? 80 * 1024 : 0;
+    if (smem < smem_floor) smem = smem_floor;
+    auto kern = use_tmem_a ? w4a16_gemm_tc_kernel<true> : w4a16_gemm_tc_kernel<false>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    const dim3 grid((unsigned)((N + kTcRows - 1) / kTcRows));
+    kern<<<grid, kTcThreads, smem, st>>>(tmX, tmP, a);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
+
+}  // namespace wq

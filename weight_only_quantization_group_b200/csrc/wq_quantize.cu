@@ -1,0 +1,228 @@
+// S3: group-wise quantize + pack, and the inverse (unpack + dequantize).
+//
+// Quantizer: "LLM Quantization: 160GB Model on a Laptop", sections "Symmetric
+// Quantization" and "Asymmetric Quantization"; integer zero point as in "CMU
+// 11-868 L19-L20 Model Quantization", section "absmax and zero-point"; one
+// step and zero per 128 input channels of a row ("Quantising Large Language
+// Models for Efficient Inference", "Post-training methods for 4-bit weights").
+// Optional AWQ input-channel scaling W * diag(s) first ("MIT 6.5940 Lab 4 +
+// Lab 5", "Question 2").
+//
+// Mapping: 16 lanes per group, each lane owns 8 consecutive input channels
+// (one 16-byte load of W). The group's min/max is reduced with four
+// xor-shuffles inside the half warp. Every decision is an explicitly rounded
+// fp32 operation (no contraction) so the codes match the CPU reading bit for
+// bit. The kernel is HBM-bound: 2 B/weight in, 0.5 (0.375) B/weight out.
+#include "wq_common.cuh"
+
+namespace wq {
+
+template <int BITS, bool SYM, bool HAS_S>
+__global__ void __launch_bounds__(256)
+quantize_pack_kernel(const __half* __restrict__ W, const __half* __restrict__ s, int64_t N, int64_t K,
+                     uint32_t* __restrict__ packed, __half* __restrict__ steps,
+                     __half* __restrict__ zeros, int* err) {
+  __shared__ __align__(16) uint8_t code_buf[8][256];  // 3-bit: per-warp code staging
+  const int lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5;
+  const int sub = lane & 15;  // lane within the group
+  const int64_t G = K / kGroup;
+  const int64_t gidx = ((int64_t)blockIdx.x * 8 + warp) * 2 + (lane >> 4);
+  const bool valid = gidx < N * G;
+  const int64_t n = valid ? gidx / G : 0;
+  const int64_t gi = valid ? gidx % G : 0;
+  const int64_t k0 = gi * kGroup + sub * 8;
+
+  float w[8];
+  {
+    uint4 raw = make_uint4(0, 0, 0, 0);
+    if (valid) raw = *reinterpret_cast<const uint4*>(W + n * K + k0);
+    const __half2* h = reinterpret_cast<const __half2*>(&raw);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      float2 f = __half22float2(h[i]);
+      w[2 * i] = f.x;
+      w[2 * i + 1] = f.y;
+    }
+    if (HAS_S) {
+      uint4 sraw = make_uint4(0, 0, 0, 0);
+      if (valid) sraw = *reinterpret_cast<const uint4*>(s + k0);
+      const __half2* sh = reinterpret_cast<const __half2*>(&sraw);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        float2 f = __half22float2(sh[i]);
+        w[2 * i] = __fmul_rn(w[2 * i], f.x);  // exact: 11 x 11 significand bits
+        w[2 * i + 1] = __fmul_rn(w[2 * i + 1], f.y);
+      }
+    }
+  }
+
+  // Group statistics over the 16 lanes of this half warp.
+  float lo = w[0], hi = SYM ? fabsf(w[0]) : w[0];
+#pragma unroll
+  for (int i = 1; i < 8; ++i) {
+    if (SYM) {
+      hi = fmaxf(hi, fabsf(w[i]));
+    } else {
+      lo = fminf(lo, w[i]);
+      hi = fmaxf(hi, w[i]);
+    }
+  }
+#pragma unroll
+  for (int o = 8; o >= 1; o >>= 1) {
+    hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, o));
+    if (!SYM) lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, o));
+  }
+
+  float sf;       // the step as fp32 (exactly the stored fp16 value)
+  int zero;       // integer zero point
+  __half step_h;
+  int qlo, qhi;   // clamp range of (rint(w/step) + offset)
+  if (SYM) {
+    constexpr int qmax = (1 << (BITS - 1)) - 1;
+    step_h = (hi == 0.0f) ? __float2half_rn(1.0f) : __float2half_ru(__fdiv_rn(hi, (float)qmax));
+    sf = __half2float(step_h);
+    zero = 1 << (BITS - 1);
+    qlo = -qmax - 1 + zero;
+    qhi = qmax + zero;
+  } else {
+    constexpr int Q = (1 << BITS) - 1;
+    const float mn = fminf(lo, 0.0f);
+    const float mx = fmaxf(hi, 0.0f);
+    const float r = __fsub_rn(mx, mn);
+    step_h = (r == 0.0f) ? __float2half_rn(1.0f) : __float2half_ru(__fdiv_rn(r, (float)Q));
+    sf = __half2float(step_h);
+    const float zf = rintf(__fdiv_rn(-mn, sf));
+    zero = (int)fminf(fmaxf(zf, 0.0f), (float)Q);
+    qlo = 0;
+    qhi = Q;
+  }
+  if (valid && sub == 0) {
+    if (!isfinite(sf)) latch_error(err, WQ_ERR_RANGE);
+    steps[n * G + gi] = step_h;
+    zeros[n * G + gi] = __int2half_rn(zero);
+  }
+
+  int q[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int v = (int)rintf(__fdiv_rn(w[i], sf)) + (SYM ? (1 << (BITS - 1)) : zero);
+    q[i] = min(max(v, qlo), qhi);
+  }
+
+  if (BITS == 4) {
+    if (valid) {
+      const uint32_t word = (uint32_t)q[0] | ((uint32_t)q[2] << 4) | ((uint32_t)q[4] << 8) |
+                            ((uint32_t)q[6] << 12) | ((uint32_t)q[1] << 16) | ((uint32_t)q[3] << 20) |
+                            ((uint32_t)q[5] << 24) | ((uint32_t)q[7] << 28);
+      packed[(n * K + k0) / 8] = word;
+    }
+  } else {
+    // Stage the 8 codes, then 3 lanes of each 4-lane quad assemble the three
+    // words of the quad's 32 input channels.
+    uint8_t* buf = code_buf[warp];
+    uint2 c8;
+    c8.x = (uint32_t)q[0] | ((uint32_t)q[1] << 8) | ((uint32_t)q[2] << 16) | ((uint32_t)q[3] << 24);
+    c8.y = (uint32_t)q[4] | ((uint32_t)q[5] << 8) | ((uint32_t)q[6] << 16) | ((uint32_t)q[7] << 24);
+    *reinterpret_cast<uint2*>(buf + lane * 8) = c8;
+    __syncwarp();
+    const int t = lane & 3;
+    if (valid && t < 3) {
+      const uint8_t* c = buf + (lane >> 2) * 32;
+      uint32_t word = 0;
+#pragma unroll
+      for (int j = 0; j < 5; ++j) {
+        word |= (uint32_t)c[10 * t + 2 * j] << (3 * j);
+        word |= (uint32_t)c[10 * t + 2 * j + 1] << (16 + 3 * j);
+      }
+      word |= (uint32_t)((c[30] >> t) & 1) << 15;
+      word |= (uint32_t)((c[31] >> t) & 1) << 31;
+      const int64_t chunk = (n * K + gi * kGroup + (sub >> 2) * 32) / 32;
+      packed[chunk * 3 + t] = word;
+    }
+  }
+}
+
+// Inverse: one thread per 8 (4-bit) or 32 (3-bit) weights.
+template <int BITS>
+__global__ void __launch_bounds__(256)
+unpack_dequant_kernel(const uint32_t* __restrict__ packed, const __half* __restrict__ steps,
+                      const __half* __restrict__ zeros, int64_t N, int64_t K, __half* __restrict__ out) {
+  constexpr int PER = BITS == 4 ? 8 : 32;
+  const int64_t units = N * K / PER;
+  const int64_t u = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (u >= units) return;
+  const int64_t e0 = u * PER;  // first element (row-major)
+  const int64_t n = e0 / K;
+  const int64_t k = e0 % K;
+  const int64_t gidx = n * (K / kGroup) + k / kGroup;
+  const float sf = __half2float(steps[gidx]);
+  const float z = __half2float(zeros[gidx]);
+  int q[PER];
+  if (BITS == 4) {
+    const uint32_t w = packed[u];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      q[2 * j] = (w >> (4 * j)) & 0xF;
+      q[2 * j + 1] = (w >> (4 * (j + 4))) & 0xF;
+    }
+  } else {
+    const uint32_t w3[3] = {packed[3 * u], packed[3 * u + 1], packed[3 * u + 2]};
+#pragma unroll
+    for (int t = 0; t < 3; ++t) {
+#pragma unroll
+      for (int j = 0; j < 5; ++j) {
+        q[10 * t + 2 * j] = (w3[t] >> (3 * j)) & 7;
+        q[10 * t + 2 * j + 1] = (w3[t] >> (16 + 3 * j)) & 7;
+      }
+    }
+    q[30] = ((w3[0] >> 15) & 1) | (((w3[1] >> 15) & 1) << 1) | (((w3[2] >> 15) & 1) << 2);
+    q[31] = ((w3[0] >> 31) & 1) | (((w3[1] >> 31) & 1) << 1) | (((w3[2] >> 31) & 1) << 2);
+  }
+#pragma unroll
+  for (int i = 0; i < PER; i += 2) {
+    // (q - z) * step is exact in fp32; one rounding to fp16.
+    const float a = __fmul_rn((float)q[i] - z, sf);
+    const float b = __fmul_rn((float)q[i + 1] - z, sf);
+    *reinterpret_cast<__half2*>(out + e0 + i) = __floats2half2_rn(a, b);
+  }
+}
+
+cudaError_t launch_quantize_pack(const void* W, const void* s, int64_t N, int64_t K, int bits, bool sym,
+                                 uint32_t* packed, void* steps, void* zeros, int* err, cudaStream_t st) {
+  const int64_t groups = N * (K / kGroup);
+  const dim3 grid((unsigned)((groups + 15) / 16));
+  const dim3 block(256);
+  auto Wp = static_cast<const __half*>(W);
+  auto sp = static_cast<const __half*>(s);
+  auto stp = static_cast<__half*>(steps);
+  auto zp = static_cast<__half*>(zeros);
+#define WQ_QP(B, S, H) quantize_pack_kernel<B, S, H><<<grid, block, 0, st>>>(Wp, sp, N, K, packed, stp, zp, err)
+  if (bits == 4) {
+    if (sym) { if (s) WQ_QP(4, true, true); else WQ_QP(4, true, false); }
+    else     { if (s) WQ_QP(4, false, true); else WQ_QP(4, false, false); }
+  } else {
+    if (sym) { if (s) WQ_QP(3, true, true); else WQ_QP(3, true, false); }
+    else     { if (s) WQ_QP(3, false, true); else WQ_QP(3, false, false); }
+  }
+#undef WQ_QP
+  return cudaGetLastError();
+}
+
+cudaError_t launch_unpack_dequant(const uint32_t* packed, const void* steps, const void* zeros, int64_t N,
+                                  int64_t K, int bits, void* out, cudaStream_t st) {
+  const int per = bits == 4 ? 8 : 32;
+  const int64_t units = N * K / per;
+  const dim3 grid((unsigned)((units + 255) / 256));
+  if (bits == 4)
+    unpack_dequant_kernel<4><<<grid, 256, 0, st>>>(packed, static_cast<const __half*>(steps),
+                                                   static_cast<const __half*>(zeros), N, K,
+                                                   static_cast<__half*>(out));
+  else
+    unpack_dequant_kernel<3><<<grid, 256, 0, st>>>(packed, static_cast<const __half*>(steps),
+                                                   static_cast<const __half*>(zeros), N, K,
+                                                   static_cast<__half*>(out));
+  return cudaGetLastError();
+}
+
+}  // namespace wq
