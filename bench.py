@@ -192,7 +192,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     Ys = [[torch.empty((1, b["N"]), dtype=torch.float16, device=dev) for b in block] for _ in copies]
     s_cap = torch.cuda.Stream(device=dev)
     graphs = []
-    for ci, blk in enumerate(copies):
+    for ci, blk in enumerate([] if args.eager else copies):
         # warm the launch path (function attributes) before capture
         for b, y in zip(blk, Ys[ci]):
             wq.wq_w4a16_gemm(b["X"], *b["q"], b["N"], bits=4, out=y)
@@ -205,8 +205,17 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     torch.cuda.synchronize()
 
     stream = torch.cuda.current_stream()
+
+    def run_step(i):
+        if args.eager:  # same launches without graphs (for profilers)
+            ci = i % n_copies
+            for b, y in zip(copies[ci], Ys[ci]):
+                wq.wq_w4a16_gemm(b["X"], *b["q"], b["N"], bits=4, out=y)
+        else:
+            graphs[i % n_copies].replay()
+
     for i in range(args.warmup):
-        graphs[i % n_copies].replay()
+        run_step(i)
     torch.cuda.synchronize()
     barrier()
     torch.cuda.synchronize()
@@ -214,7 +223,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     with ClockSampler(local_rank) as clk:
         ev0.record(stream)
         for i in range(args.steps):
-            graphs[i % n_copies].replay()
+            run_step(i)
         ev1.record(stream)
         torch.cuda.synchronize()
     barrier()
@@ -289,7 +298,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
             "bytes_per_step": step_bytes,
             "block_copies": n_copies,
             "l2": f"inputs larger than L2: {n_copies} block copies, {n_copies * block_w_bytes / 1e6:.0f} MB of packed weight rotate",
-            "graph": "one CUDA graph of 7 launches per block copy",
+            "graph": "eager launches" if args.eager else "one CUDA graph of 7 launches per block copy",
             "parallelism": f"replicas x{world}",
         },
         "roofline": {
@@ -564,6 +573,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-rows", action="store_true", help="skip the per-row measurements")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--eager", action="store_true", help="launch eagerly instead of replaying CUDA graphs")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--ref-seconds", type=float, default=60.0)
     ap.add_argument("--case", choices=["gemm", "quantize"], default=None,

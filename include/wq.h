@@ -140,6 +140,35 @@ int32_t wq_w4a16_gemm(const void* X_dev, const uint32_t* packed_dev, const void*
                       const wq_quant_cfg* cfg, void* Y_dev, void* workspace_dev,
                       size_t workspace_bytes, void* stream);
 
+/* S1/S2/S4 -- AWQ activation-aware scale search for the linears that share
+ * one input ("MIT 6.5940 Lab 4 + Lab 5", sections "Starting point and setup"
+ * and "Question 2"; the loss is the layer-output reconstruction error of
+ * "CMU 11-868 L19-L20 Model Quantization", section "Quantizing during
+ * training vs. after it").
+ *   X_dev      fp16 [T][K] calibration inputs of the linears
+ *   W_dev[i]   host array of n_lin (1..8) device pointers, fp16 [N_i[i]][K]
+ *   alpha      host array of n_alpha (1..64) exponents (e.g. j/20, j < 20)
+ * Computes mu_k = sum_t |x_tk| / T (fp64, exact sum), candidates
+ * s_j,k = fp16_rn(max(mu_k, 2^-14)^alpha_j), and for every j the loss
+ * L_j = sum_i || X (W_i - Q(W_i diag s_j) diag(s_j)^-1)^T ||_F^2, where Q is
+ * this library's quantize-dequantize with `cfg` (the loss GEMM runs on the
+ * tensor cores with the error matrix in fp16 and fp32 accumulation; the
+ * squares are summed in fp64 in a fixed order, so results are deterministic).
+ * Writes s_out_dev (fp16 [K]) = s_best with best = the first index of the
+ * smallest L_j; optionally mu_out_dev (fp64 [K]), loss_out_dev (fp64
+ * [n_alpha]) and best_out_dev (int32, device). Quantize the weights with
+ * wq_quantize_pack(W, s_out) and feed the matmul X * diag(s)^-1 afterwards.
+ * workspace_dev: >= wq_awq_workspace_bytes(...) bytes, 256-byte aligned, no
+ * initial contents required. A non-finite candidate or loss latches
+ * WQ_ERR_RANGE in the device flag. */
+size_t wq_awq_workspace_bytes(int64_t T, int64_t K, const int64_t* N_i, int32_t n_lin, int32_t n_alpha,
+                              const wq_quant_cfg* cfg);
+int32_t wq_awq_scale_search(const void* X_dev, int64_t T, int64_t K, const void* const* W_dev,
+                            const int64_t* N_i, int32_t n_lin, const wq_quant_cfg* cfg,
+                            const double* alpha, int32_t n_alpha, void* s_out_dev, double* mu_out_dev,
+                            double* loss_out_dev, int32_t* best_out_dev, void* workspace_dev,
+                            size_t workspace_bytes, void* stream);
+
 /* Process-wide tuning options (not thread-safe against concurrent calls).
  *  WQ_OPT_GEMM_PATH     WQ_PATH_AUTO (default): GEMV kernel below the
  *                       crossover M, tensor-core kernel at or above it (4-bit);

@@ -28,6 +28,8 @@ __all__ = [
     "wq_get_last_device_error",
     "wq_set_option",
     "wq_get_option",
+    "wq_awq_workspace_bytes",
+    "wq_awq_scale_search",
     "EXPORTED_SYMBOLS",
 ]
 
@@ -46,6 +48,8 @@ EXPORTED_SYMBOLS = (
     "wq_get_last_device_error",
     "wq_set_option",
     "wq_get_option",
+    "wq_awq_workspace_bytes",
+    "wq_awq_scale_search",
 )
 
 WQ_OK = 0
@@ -99,6 +103,9 @@ def _load() -> ctypes.CDLL:
         "wq_get_last_device_error": (i32, [vp]),
         "wq_set_option": (i32, [i32, i64]),
         "wq_get_option": (i64, [i32]),
+        "wq_awq_workspace_bytes": (sz, [i64, i64, ctypes.POINTER(i64), i32, i32, cfgp]),
+        "wq_awq_scale_search": (i32, [vp, i64, i64, ctypes.POINTER(vp), ctypes.POINTER(i64), i32, cfgp,
+                                      ctypes.POINTER(ctypes.c_double), i32, vp, vp, vp, vp, vp, sz, vp]),
     }
     for name, (res, args) in sig.items():
         f = getattr(L, name)
@@ -239,3 +246,41 @@ def wq_set_option(option: int, value: int) -> None:
 
 def wq_get_option(option: int) -> int:
     return int(_lib.wq_get_option(int(option)))
+
+
+def wq_awq_workspace_bytes(T: int, K: int, Ns, n_alpha: int = 20, *, bits: int = 4, group_size: int = 128,
+                           symmetric: bool = False) -> int:
+    c = _cfg(bits, group_size, symmetric)
+    arr = (ctypes.c_int64 * len(Ns))(*[int(n) for n in Ns])
+    return int(_lib.wq_awq_workspace_bytes(T, K, arr, len(Ns), n_alpha, ctypes.byref(c)))
+
+
+def wq_awq_scale_search(X: torch.Tensor, Ws, alphas=None, *, bits: int = 4, group_size: int = 128,
+                        symmetric: bool = False, workspace: torch.Tensor | None = None, stream=None):
+    """AWQ scale search over the linears `Ws` (fp16 [N_i][K]) that share the
+    calibration input X (fp16 [T][K]). Returns a dict with s (fp16 [K]), mu
+    (fp64 [K]), losses (fp64 [n_alpha]) and best (int32 [1]), all on the device."""
+    _check(X, torch.float16, "X")
+    for i, W in enumerate(Ws):
+        _check(W, torch.float16, f"W[{i}]")
+    T, K = X.shape
+    if alphas is None:
+        alphas = [j / 20.0 for j in range(20)]
+    alphas = [float(a) for a in alphas]
+    c = _cfg(bits, group_size, symmetric)
+    Ns = [int(W.shape[0]) for W in Ws]
+    n_arr = (ctypes.c_int64 * len(Ns))(*Ns)
+    a_arr = (ctypes.c_double * len(alphas))(*alphas)
+    w_arr = (ctypes.c_void_p * len(Ws))(*[W.data_ptr() for W in Ws])
+    need = int(_lib.wq_awq_workspace_bytes(T, K, n_arr, len(Ns), len(alphas), ctypes.byref(c)))
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=X.device)
+    s = torch.empty(K, dtype=torch.float16, device=X.device)
+    mu = torch.empty(K, dtype=torch.float64, device=X.device)
+    losses = torch.empty(len(alphas), dtype=torch.float64, device=X.device)
+    best = torch.empty(1, dtype=torch.int32, device=X.device)
+    st = _lib.wq_awq_scale_search(_ptr(X), T, K, w_arr, n_arr, len(Ns), ctypes.byref(c), a_arr, len(alphas),
+                                  _ptr(s), _ptr(mu), _ptr(losses), _ptr(best), workspace.data_ptr(),
+                                  workspace.numel() * workspace.element_size(), _stream(stream))
+    _raise(st, "wq_awq_scale_search")
+    return {"s": s, "mu": mu, "losses": losses, "best": best}

@@ -14,6 +14,17 @@ cudaError_t launch_gemv(const void* X, const uint32_t* packed, const void* steps
                         int64_t N, int64_t K, int bits, void* Y, cudaStream_t st, bool exact);
 cudaError_t launch_gemm_tc(const void* X, const uint32_t* packed, const void* steps, const void* zeros, int64_t M,
                            int64_t N, int64_t K, void* Y, int* err, cudaStream_t st, bool a_tmem);
+struct AwqPlan {
+  int64_t N_total;
+  int t_tiles, n_tiles, tiles;
+  int batch;
+  size_t off_mu, off_S, off_partial, off_E, total;
+};
+AwqPlan plan_awq(int64_t T, int64_t K, const int64_t* N_i, int n_lin, int n_alpha);
+cudaError_t launch_awq_search(const void* X, int64_t T, int64_t K, const void* const* W, const int64_t* N_i,
+                              int n_lin, int bits, bool sym, const double* alpha, int n_alpha, void* s_out,
+                              double* mu_out, double* loss_out, int32_t* best_out, void* workspace, int* err,
+                              cudaStream_t st);
 }  // namespace wq
 
 // One flag per device (each device holds its own copy of a __device__ variable).
@@ -148,6 +159,53 @@ int32_t wq_w4a16_gemm(const void* X, const uint32_t* packed, const void* steps, 
   }
   return cuda_status(wq::launch_gemv(X, packed, steps, zeros, M, N, K, cfg->bits, Y,
                                      static_cast<cudaStream_t>(stream), g_opt_gemv_variant == WQ_GEMV_EXACT));
+}
+
+static int32_t check_awq(int64_t T, int64_t K, const int64_t* N_i, int32_t n_lin, int32_t n_alpha,
+                         const wq_quant_cfg* cfg) {
+  int32_t st = check_cfg(cfg);
+  if (st != WQ_OK) return st;
+  if (T < 1 || T > (int64_t)INT32_MAX / 2 || !N_i || n_lin < 1 || n_lin > 8 || n_alpha < 1 || n_alpha > 64)
+    return WQ_ERR_INVALID_ARG;
+  int64_t tot = 0;
+  for (int i = 0; i < n_lin; ++i) {
+    if ((st = check_shape(N_i[i], K)) != WQ_OK) return st;
+    tot += N_i[i];
+  }
+  if (tot > (int64_t)INT32_MAX / 2) return WQ_ERR_INVALID_ARG;
+  return WQ_OK;
+}
+
+size_t wq_awq_workspace_bytes(int64_t T, int64_t K, const int64_t* N_i, int32_t n_lin, int32_t n_alpha,
+                              const wq_quant_cfg* cfg) {
+  if (check_awq(T, K, N_i, n_lin, n_alpha, cfg) != WQ_OK) return 0;
+  return wq::plan_awq(T, K, N_i, n_lin, n_alpha).total;
+}
+
+int32_t wq_awq_scale_search(const void* X, int64_t T, int64_t K, const void* const* W, const int64_t* N_i,
+                            int32_t n_lin, const wq_quant_cfg* cfg, const double* alpha, int32_t n_alpha,
+                            void* s_out, double* mu_out, double* loss_out, int32_t* best_out, void* workspace,
+                            size_t workspace_bytes, void* stream) {
+  int32_t st = check_awq(T, K, N_i, n_lin, n_alpha, cfg);
+  if (st != WQ_OK) return st;
+  if (!X || !W || !alpha || !s_out) return WQ_ERR_INVALID_ARG;
+  for (int i = 0; i < n_lin; ++i) {
+    if (!W[i]) return WQ_ERR_INVALID_ARG;
+    if (!aligned(W[i], 16)) return WQ_ERR_ALIGNMENT;
+  }
+  for (int j = 0; j < n_alpha; ++j)
+    if (!(alpha[j] == alpha[j])) return WQ_ERR_INVALID_ARG;  // NaN
+  if (!aligned(X, 16) || !aligned(s_out, 2) || (mu_out && !aligned(mu_out, 8)) || (loss_out && !aligned(loss_out, 8)) ||
+      (best_out && !aligned(best_out, 4)))
+    return WQ_ERR_ALIGNMENT;
+  const size_t need = wq::plan_awq(T, K, N_i, n_lin, n_alpha).total;
+  if (!workspace || workspace_bytes < need) return WQ_ERR_WORKSPACE;
+  if (!aligned(workspace, 256)) return WQ_ERR_ALIGNMENT;
+  int* flag = device_flag();
+  if (!flag) return WQ_ERR_CUDA;
+  return cuda_status(wq::launch_awq_search(X, T, K, W, N_i, n_lin, cfg->bits, cfg->symmetric != 0, alpha, n_alpha,
+                                           s_out, mu_out, loss_out, best_out, workspace, flag,
+                                           static_cast<cudaStream_t>(stream)));
 }
 
 int32_t wq_set_option(int32_t option, int64_t value) {

@@ -1,0 +1,429 @@
+// S1, S2, S4: AWQ activation-aware scale search.
+//
+// "MIT 6.5940 Lab 4 + Lab 5", "Starting point and setup": forward hooks record
+// the mean absolute value of each linear layer's input over calibration
+// tokens; "Question 2": scale salient input channels by s (and the activation
+// by 1/s), searching the scale with "compute scale, scale up, quantize, scale
+// down" at each place of the block; the error measured is the layer output
+// reconstruction error of "CMU 11-868 L19-L20", "Quantizing during training
+// vs. after it" (||WX - W^X||^2).
+//
+// Pipeline, all on the caller's stream:
+//   absmean      mu_k = sum_t |x_tk| / T        (fp64; the sum is exact)
+//   candidates   s_j,k = fp16_rn(max(mu_k, 2^-14) ^ alpha_j)
+//   per batch of alphas:
+//     awq_error  E_j = W - Q(W diag s_j) diag(s_j)^-1, fp16, every linear of
+//                the group stacked row-wise (same decision code as the packer)
+//     awq_loss   tcgen05 GEMM D = E_j X^T per 128x128 tile, epilogue sums D^2
+//                in fp64 -> one partial per (alpha, tile)
+//   finalize     L_j = sum of partials in tile order (deterministic), first
+//                argmin, s_out = s_best
+#include "wq_quant_core.cuh"
+#include "wq_sm100.cuh"
+
+namespace wq {
+
+using namespace sm100;
+
+constexpr int kAwqMaxLinears = 8;
+constexpr int kAwqMaxAlpha = 64;
+constexpr size_t kAwqEBudget = size_t(1) << 30;  // bytes of E kept per alpha batch
+constexpr long long kAwqSpinLimit = 4000000000LL;
+
+// ------------------------------------------------------------------ S1
+__global__ void __launch_bounds__(256) absmean_kernel(const __half* __restrict__ X, int T, int K,
+                                                      double* __restrict__ mu) {
+  const int k = blockIdx.x * blockDim.x + threadIdx.x;
+  if (k >= K) return;
+  double acc = 0.0;  // fp16 magnitudes are multiples of 2^-24 below 2^16: exact
+  for (int t = 0; t < T; ++t) acc += fabs((double)__half2float(X[(size_t)t * K + k]));
+  mu[k] = acc / (double)T;
+}
+
+// ------------------------------------------------------------------ S2
+struct AlphaList {
+  double v[kAwqMaxAlpha];
+};
+
+__global__ void __launch_bounds__(256) candidates_kernel(const double* __restrict__ mu, int K, AlphaList al,
+                                                         int n_alpha, __half* __restrict__ S, int* err) {
+  const int k = blockIdx.x * blockDim.x + threadIdx.x;
+  const int j = blockIdx.y;
+  if (k >= K || j >= n_alpha) return;
+  const double m = fmax(mu[k], 6.103515625e-05);  // 2^-14
+  const double p = pow(m, al.v[j]);
+  const __half h = __double2half(p);
+  if (!isfinite(__half2float(h))) latch_error(err, WQ_ERR_RANGE);
+  S[(size_t)j * K + k] = h;
+}
+
+// ------------------------------------------------------------------ S4a: E
+struct LinearSet {
+  const __half* W[kAwqMaxLinears];
+  int row_off[kAwqMaxLinears + 1];  // prefix sums of N_i
+  int n_lin;
+  int n_total;                      // row_off[n_lin]
+};
+
+template <int BITS, bool SYM>
+__global__ void __launch_bounds__(256)
+awq_error_kernel(LinearSet ls, int K, const __half* __restrict__ S, int alpha0, __half* __restrict__ E) {
+  const int lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5;
+  const int sub = lane & 15;
+  const int N = ls.n_total;
+  const int G = K / kGroup;
+  const int64_t gidx = ((int64_t)blockIdx.x * 8 + warp) * 2 + (lane >> 4);
+  const bool valid = gidx < (int64_t)N * G;
+  const int n = valid ? (int)(gidx / G) : 0;
+  const int gi = valid ? (int)(gidx % G) : 0;
+  const int k0 = gi * kGroup + sub * 8;
+  const int b = blockIdx.y;
+  // Which stacked linear owns row n (unrolled so the parameter arrays stay in
+  // the constant bank).
+  const __half* Wrow = ls.W[0];
+  int roff = 0;
+#pragma unroll
+  for (int i = 1; i < kAwqMaxLinears; ++i)
+    if (i < ls.n_lin && n >= ls.row_off[i]) {
+      Wrow = ls.W[i];
+      roff = ls.row_off[i];
+    }
+  const __half* s = S + (size_t)(alpha0 + b) * K;
+
+  float w[8], x[8], sv[8];
+  {
+    uint4 raw = make_uint4(0, 0, 0, 0), sraw = make_uint4(0x3C003C00u, 0x3C003C00u, 0x3C003C00u, 0x3C003C00u);
+    if (valid) {
+      raw = *reinterpret_cast<const uint4*>(Wrow + (size_t)(n - roff) * K + k0);
+      sraw = *reinterpret_cast<const uint4*>(s + k0);
+    }
+    const __half2* h = reinterpret_cast<const __half2*>(&raw);
+    const __half2* sh = reinterpret_cast<const __half2*>(&sraw);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float2 f = __half22float2(h[i]);
+      const float2 g = __half22float2(sh[i]);
+      x[2 * i] = f.x;
+      x[2 * i + 1] = f.y;
+      sv[2 * i] = g.x;
+      sv[2 * i + 1] = g.y;
+      w[2 * i] = __fmul_rn(f.x, g.x);  // exact
+      w[2 * i + 1] = __fmul_rn(f.y, g.y);
+    }
+  }
+  const GroupQuant gq = group_quant_decide<BITS, SYM>(w);
+  uint32_t out[4];
+#pragma unroll
+  for (int i = 0; i < 8; i += 2) {
+    float e2[2];
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int q = group_quant_code<BITS, SYM>(w[i + u], gq);
+      const float deq = __fmul_rn((float)(q - gq.zero), gq.sf);  // exact
+      e2[u] = x[i + u] - deq * __frcp_rn(sv[i + u]);
+    }
+    const __half2 hv = __floats2half2_rn(e2[0], e2[1]);
+    out[i / 2] = *reinterpret_cast<const uint32_t*>(&hv);
+  }
+  if (valid)
+    *reinterpret_cast<uint4*>(E + ((size_t)b * N + n) * K + k0) = make_uint4(out[0], out[1], out[2], out[3]);
+}
+
+// ------------------------------------------------------------------ S4b: loss GEMM
+constexpr int kLossThreads = 192;
+constexpr int kLossStageBytes = 2 * 128 * 64 * 2;  // A (E) + B (X) tiles, 32 KB
+
+struct LossArgs {
+  double* partial;   // [n_alpha][tiles]
+  int alpha0;
+  int K;
+  int t_tiles, n_tiles;
+  int stages;
+  int* err;
+};
+
+__device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, int c0, int c1, int c2,
+                                            uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];"
+      ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(smem_u32(bar))
+      : "memory");
+}
+
+__global__ void __launch_bounds__(kLossThreads, 1)
+awq_loss_kernel(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CUtensorMap tmX, LossArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int S = a.stages;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + (size_t)S * kLossStageBytes);
+  uint64_t* empty = full + S;
+  uint64_t* accum = empty + S;
+  double* red = reinterpret_cast<double*>(accum + 1);  // [4]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(red + 4);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int tt = blockIdx.x, nt = blockIdx.y, b = blockIdx.z;
+  const int KT = a.K / 64;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(accum, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 128);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      prefetch_tensormap(&tmE);
+      prefetch_tensormap(&tmX);
+      int issued = 0;
+      for (int kt = 0; kt < KT; ++kt) {
+        if (*abort_flag) break;
+        const int s = kt % S, u = kt / S;
+        if (u > 0 && !mbar_wait(&empty[s], (u - 1) & 1, a.err, kAwqSpinLimit)) { *abort_flag = 1; break; }
+        uint8_t* st = smem + (size_t)s * kLossStageBytes;
+        mbar_arrive_expect_tx(&full[s], kLossStageBytes);
+        tma_load_3d(st, &tmE, kt * 64, nt * 128, b, &full[s]);
+        tma_load_2d(st + kLossStageBytes / 2, &tmX, kt * 64, tt * 128, &full[s]);
+        issued = kt + 1;
+      }
+      for (int kt = issued > S ? issued - S : 0; kt < issued; ++kt)
+        mbar_wait(&full[kt % S], (kt / S) & 1, a.err, kAwqSpinLimit);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t idesc = idesc_f16_f32(128, 128);
+      int committed = -1;
+      for (int kt = 0; kt < KT; ++kt) {
+        if (*abort_flag) break;
+        const int s = kt % S, u = kt / S;
+        if (!mbar_wait(&full[s], u & 1, a.err, kAwqSpinLimit)) { *abort_flag = 1; break; }
+        tc_fence_after();
+        const uint32_t base = smem_u32(smem + (size_t)s * kLossStageBytes);
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          mma_f16_ss(tmem, desc_kmajor_sw128(base + 32 * j), desc_kmajor_sw128(base + kLossStageBytes / 2 + 32 * j),
+                     idesc, (kt > 0 || j > 0) ? 1u : 0u);
+        mma_commit(&empty[s]);
+        committed = kt;
+      }
+      mma_commit(accum);
+      if (*abort_flag && committed >= 0)
+        mbar_wait(&empty[committed % S], (committed / S) & 1, a.err, kAwqSpinLimit);
+    }
+  } else {
+    const int q = warp & 3;
+    bool done = !__any_sync(0xffffffffu, *abort_flag != 0);
+    if (done) done = __all_sync(0xffffffffu, mbar_wait(accum, 0, a.err, kAwqSpinLimit));
+    double acc = 0.0;
+    if (done) {
+      tc_fence_after();
+#pragma unroll 1
+      for (int c0 = 0; c0 < 128; c0 += 16) {
+        uint32_t v[16];
+        tmem_ld16(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)c0, v);
+        tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const double d = (double)__uint_as_float(v[i]);
+          acc = fma(d, d, acc);
+        }
+      }
+    } else {
+      *abort_flag = 1;
+    }
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    if (lane == 0) red[q] = acc;
+    asm volatile("bar.sync 1, 128;" ::: "memory");
+    if (warp == 2 && lane == 0 && !*abort_flag) {
+      const double tot = ((red[0] + red[1]) + red[2]) + red[3];
+      a.partial[((size_t)(a.alpha0 + b) * a.n_tiles + nt) * a.t_tiles + tt] = tot;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 128);
+  }
+}
+
+// ------------------------------------------------------------------ finalize
+__global__ void __launch_bounds__(256)
+awq_finalize_kernel(const double* __restrict__ partial, int tiles, int n_alpha, const __half* __restrict__ S, int K,
+                    double* loss_out, int32_t* best_out, __half* __restrict__ s_out, int* err) {
+  __shared__ double loss[kAwqMaxAlpha];
+  __shared__ int best;
+  const int t = threadIdx.x;
+  if (t < n_alpha) {
+    double v = 0.0;
+    for (int i = 0; i < tiles; ++i) v += partial[(size_t)t * tiles + i];
+    loss[t] = v;
+    if (loss_out) loss_out[t] = v;
+  }
+  __syncthreads();
+  if (t == 0) {
+    int bi = 0;
+    bool bad = !isfinite(loss[0]);
+    for (int j = 1; j < n_alpha; ++j) {
+      if (!isfinite(loss[j])) bad = true;
+      if (loss[j] < loss[bi]) bi = j;
+    }
+    if (bad) latch_error(err, WQ_ERR_RANGE);
+    best = bi;
+    if (best_out) *best_out = bi;
+  }
+  __syncthreads();
+  for (int k = t; k < K; k += blockDim.x) s_out[k] = S[(size_t)best * K + k];
+}
+
+// ------------------------------------------------------------------ host
+typedef CUresult (*EncodeTiledFnA)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFnA awq_encode_fn() {
+  static EncodeTiledFnA fn = nullptr;
+  if (fn == nullptr) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFnA>(p);
+  }
+  return fn;
+}
+
+struct AwqPlan {
+  int64_t N_total;
+  int t_tiles, n_tiles, tiles;
+  int batch;  // alphas per E batch
+  size_t off_mu, off_S, off_partial, off_E, total;
+};
+
+static size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+AwqPlan plan_awq(int64_t T, int64_t K, const int64_t* N_i, int n_lin, int n_alpha) {
+  AwqPlan p;
+  p.N_total = 0;
+  for (int i = 0; i < n_lin; ++i) p.N_total += N_i[i];
+  p.t_tiles = (int)((T + 127) / 128);
+  p.n_tiles = (int)((p.N_total + 127) / 128);
+  p.tiles = p.t_tiles * p.n_tiles;
+  const size_t e_one = (size_t)p.N_total * (size_t)K * 2;
+  int b = (int)(kAwqEBudget / (e_one ? e_one : 1));
+  if (b < 1) b = 1;
+  if (b > n_alpha) b = n_alpha;
+  p.batch = b;
+  size_t off = 0;
+  p.off_mu = off;
+  off = align256(off + (size_t)K * 8);
+  p.off_S = off;
+  off = align256(off + (size_t)n_alpha * K * 2);
+  p.off_partial = off;
+  off = align256(off + (size_t)n_alpha * p.tiles * 8);
+  p.off_E = off;
+  off = align256(off + (size_t)p.batch * e_one);
+  p.total = off;
+  return p;
+}
+
+cudaError_t launch_awq_search(const void* X, int64_t T, int64_t K, const void* const* W, const int64_t* N_i,
+                              int n_lin, int bits, bool sym, const double* alpha, int n_alpha, void* s_out,
+                              double* mu_out, double* loss_out, int32_t* best_out, void* workspace, int* err,
+                              cudaStream_t st) {
+  EncodeTiledFnA enc = awq_encode_fn();
+  if (!enc) return cudaErrorNotSupported;
+  const AwqPlan p = plan_awq(T, K, N_i, n_lin, n_alpha);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  double* mu = mu_out ? mu_out : reinterpret_cast<double*>(ws + p.off_mu);
+  __half* S = reinterpret_cast<__half*>(ws + p.off_S);
+  double* partial = reinterpret_cast<double*>(ws + p.off_partial);
+  __half* E = reinterpret_cast<__half*>(ws + p.off_E);
+  const __half* Xh = static_cast<const __half*>(X);
+
+  absmean_kernel<<<(unsigned)((K + 255) / 256), 256, 0, st>>>(Xh, (int)T, (int)K, mu);
+  AlphaList al;
+  for (int j = 0; j < kAwqMaxAlpha; ++j) al.v[j] = j < n_alpha ? alpha[j] : 0.0;
+  candidates_kernel<<<dim3((unsigned)((K + 255) / 256), (unsigned)n_alpha), 256, 0, st>>>(mu, (int)K, al, n_alpha,
+                                                                                         S, err);
+  LinearSet ls;
+  ls.n_lin = n_lin;
+  ls.row_off[0] = 0;
+  for (int i = 0; i < kAwqMaxLinears; ++i) {
+    ls.W[i] = i < n_lin ? static_cast<const __half*>(W[i]) : nullptr;
+    if (i < n_lin) ls.row_off[i + 1] = ls.row_off[i] + (int)N_i[i];
+  }
+  for (int i = n_lin; i < kAwqMaxLinears; ++i) ls.row_off[i + 1] = ls.row_off[n_lin];
+  ls.n_total = ls.row_off[n_lin];
+
+  CUtensorMap tmX;
+  {
+    cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)T};
+    cuuint64_t strides[1] = {(cuuint64_t)K * 2};
+    cuuint32_t box[2] = {64, 128};
+    cuuint32_t es[2] = {1, 1};
+    if (enc(&tmX, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<__half*>(Xh), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  }
+  const int stages = 3;
+  const size_t smem = 1024 + (size_t)stages * kLossStageBytes + (2 * stages + 1) * 8 + 4 * 8 + 16;
+  cudaError_t e = cudaFuncSetAttribute(awq_loss_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  const int64_t groups = p.N_total * (K / kGroup);
+
+  for (int a0 = 0; a0 < n_alpha; a0 += p.batch) {
+    const int B = (n_alpha - a0) < p.batch ? (n_alpha - a0) : p.batch;
+    const dim3 eg((unsigned)((groups + 15) / 16), (unsigned)B);
+#define WQ_AE(BI, SY) awq_error_kernel<BI, SY><<<eg, 256, 0, st>>>(ls, (int)K, S, a0, E)
+    if (bits == 4) { if (sym) WQ_AE(4, true); else WQ_AE(4, false); }
+    else { if (sym) WQ_AE(3, true); else WQ_AE(3, false); }
+#undef WQ_AE
+    CUtensorMap tmE;
+    {
+      cuuint64_t dims[3] = {(cuuint64_t)K, (cuuint64_t)p.N_total, (cuuint64_t)B};
+      cuuint64_t strides[2] = {(cuuint64_t)K * 2, (cuuint64_t)p.N_total * (cuuint64_t)K * 2};
+      cuuint32_t box[3] = {64, 128, 1};
+      cuuint32_t es[3] = {1, 1, 1};
+      if (enc(&tmE, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, E, dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return cudaErrorInvalidValue;
+    }
+    LossArgs la;
+    la.partial = partial;
+    la.alpha0 = a0;
+    la.K = (int)K;
+    la.t_tiles = p.t_tiles;
+    la.n_tiles = p.n_tiles;
+    la.stages = stages;
+    la.err = err;
+    awq_loss_kernel<<<dim3((unsigned)p.t_tiles, (unsigned)p.n_tiles, (unsigned)B), kLossThreads, smem, st>>>(
+        tmE, tmX, la);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  awq_finalize_kernel<<<1, 256, 0, st>>>(partial, p.tiles, n_alpha, S, (int)K, loss_out, best_out,
+                                          static_cast<__half*>(s_out), err);
+  return cudaGetLastError();
+}
+
+}  // namespace wq

@@ -9,11 +9,10 @@
 // Lab 5", "Question 2").
 //
 // Mapping: 16 lanes per group, each lane owns 8 consecutive input channels
-// (one 16-byte load of W). The group's min/max is reduced with four
-// xor-shuffles inside the half warp. Every decision is an explicitly rounded
-// fp32 operation (no contraction) so the codes match the CPU reading bit for
-// bit. The kernel is HBM-bound: 2 B/weight in, 0.5 (0.375) B/weight out.
-#include "wq_common.cuh"
+// (one 16-byte load of W); group_quant_decide() reduces the group's range with
+// four xor-shuffles inside the half warp. The kernel is HBM-bound: 2 B/weight
+// in, 0.5 (0.375) B/weight out.
+#include "wq_quant_core.cuh"
 
 namespace wq {
 
@@ -57,58 +56,15 @@ quantize_pack_kernel(const __half* __restrict__ W, const __half* __restrict__ s,
     }
   }
 
-  // Group statistics over the 16 lanes of this half warp.
-  float lo = w[0], hi = SYM ? fabsf(w[0]) : w[0];
-#pragma unroll
-  for (int i = 1; i < 8; ++i) {
-    if (SYM) {
-      hi = fmaxf(hi, fabsf(w[i]));
-    } else {
-      lo = fminf(lo, w[i]);
-      hi = fmaxf(hi, w[i]);
-    }
-  }
-#pragma unroll
-  for (int o = 8; o >= 1; o >>= 1) {
-    hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, o));
-    if (!SYM) lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, o));
-  }
-
-  float sf;       // the step as fp32 (exactly the stored fp16 value)
-  int zero;       // integer zero point
-  __half step_h;
-  int qlo, qhi;   // clamp range of (rint(w/step) + offset)
-  if (SYM) {
-    constexpr int qmax = (1 << (BITS - 1)) - 1;
-    step_h = (hi == 0.0f) ? __float2half_rn(1.0f) : __float2half_ru(__fdiv_rn(hi, (float)qmax));
-    sf = __half2float(step_h);
-    zero = 1 << (BITS - 1);
-    qlo = -qmax - 1 + zero;
-    qhi = qmax + zero;
-  } else {
-    constexpr int Q = (1 << BITS) - 1;
-    const float mn = fminf(lo, 0.0f);
-    const float mx = fmaxf(hi, 0.0f);
-    const float r = __fsub_rn(mx, mn);
-    step_h = (r == 0.0f) ? __float2half_rn(1.0f) : __float2half_ru(__fdiv_rn(r, (float)Q));
-    sf = __half2float(step_h);
-    const float zf = rintf(__fdiv_rn(-mn, sf));
-    zero = (int)fminf(fmaxf(zf, 0.0f), (float)Q);
-    qlo = 0;
-    qhi = Q;
-  }
+  const GroupQuant gq = group_quant_decide<BITS, SYM>(w);
   if (valid && sub == 0) {
-    if (!isfinite(sf)) latch_error(err, WQ_ERR_RANGE);
-    steps[n * G + gi] = step_h;
-    zeros[n * G + gi] = __int2half_rn(zero);
+    if (!isfinite(gq.sf)) latch_error(err, WQ_ERR_RANGE);
+    steps[n * G + gi] = gq.step_h;
+    zeros[n * G + gi] = __int2half_rn(gq.zero);
   }
-
   int q[8];
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const int v = (int)rintf(__fdiv_rn(w[i], sf)) + (SYM ? (1 << (BITS - 1)) : zero);
-    q[i] = min(max(v, qlo), qhi);
-  }
+  for (int i = 0; i < 8; ++i) q[i] = group_quant_code<BITS, SYM>(w[i], gq);
 
   if (BITS == 4) {
     if (valid) {
