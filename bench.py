@@ -277,7 +277,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         return None
 
     clocks = clk.summary()
-    traffic = profiled_traffic("gemv_kernel<4,1,2>")
+    traffic = profiled_traffic("gemv_rows_kernel<1,4>")
     achieved = step_bytes / (ms_per_step * 1e-3) / 1e9
     line = {
         "metric": METRIC,
@@ -303,7 +303,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         },
         "roofline": {
             "bound": "hbm",
-            "kernel": "gemv_kernel<4,1,2>",
+            "kernel": "gemv_rows_kernel<1,4>",
             "achieved": round(achieved, 2),
             "peak": peaks["hbm_gbs"],
             "peak_source": f"{peaks['source']} HBM copy bandwidth",
@@ -384,11 +384,16 @@ def measure_rows(wq, torch, synth, dev, block, peaks):
     for bits in (4, 3):
         c = synth.config_llama65b_decode(bits)
         gemv_row(f"gemv_llama65b_8192x8192_w{bits}", 8192, 8192, bits, c.W, c.X)
-        wq.wq_set_option(wq.WQ_OPT_GEMV_VARIANT, wq.WQ_GEMV_EXACT)
-        try:
-            gemv_row(f"gemv_llama65b_8192x8192_w{bits}_exact", 8192, 8192, bits, c.W, c.X)
-        finally:
-            wq.wq_set_option(wq.WQ_OPT_GEMV_VARIANT, wq.WQ_GEMV_OFFSET_SUMS)
+        for tag, var in (("tiled", wq.WQ_GEMV_OFFSET_SUMS), ("tiled_exact", wq.WQ_GEMV_EXACT)):
+            if bits == 3 and tag == "tiled":
+                continue  # 3-bit always runs the tiled kernel
+            wq.wq_set_option(wq.WQ_OPT_GEMV_KERNEL, wq.WQ_GEMV_KERNEL_TILED)
+            wq.wq_set_option(wq.WQ_OPT_GEMV_VARIANT, var)
+            try:
+                gemv_row(f"gemv_llama65b_8192x8192_w{bits}_{tag}", 8192, 8192, bits, c.W, c.X)
+            finally:
+                wq.wq_set_option(wq.WQ_OPT_GEMV_KERNEL, wq.WQ_GEMV_KERNEL_AUTO)
+                wq.wq_set_option(wq.WQ_OPT_GEMV_VARIANT, wq.WQ_GEMV_OFFSET_SUMS)
     big = synth.config_smallm_sweep(1)
     for M in synth.SMALLM_SWEEP:
         gemv_row(f"smallm_M{M}_8192x28672_w4", 28672, 8192, 4, big.W, synth.smallm_activations(M), M=M)
@@ -541,6 +546,8 @@ def run_case(args):
     wq.wq_set_option(wq.WQ_OPT_GEMM_PATH, opts[args.path])
     wq.wq_set_option(wq.WQ_OPT_GEMV_VARIANT, wq.WQ_GEMV_EXACT if args.gemv_variant == "exact"
                      else wq.WQ_GEMV_OFFSET_SUMS)
+    wq.wq_set_option(wq.WQ_OPT_GEMV_KERNEL, wq.WQ_GEMV_KERNEL_TILED if args.gemv_variant == "tiled"
+                     else wq.WQ_GEMV_KERNEL_AUTO)
     wq.wq_set_option(wq.WQ_OPT_TC_A_OPERAND, wq.WQ_TC_A_SMEM if args.tc_a == "smem" else wq.WQ_TC_A_TMEM)
     q = wq.wq_quantize_pack(W, bits=args.bits)
     Y = torch.empty((args.M, args.N), dtype=torch.float16, device=dev)
@@ -584,7 +591,7 @@ def main():
     ap.add_argument("--bits", type=int, default=4)
     ap.add_argument("--reps", type=int, default=3)
     ap.add_argument("--path", choices=["auto", "gemv", "tc"], default="auto")
-    ap.add_argument("--gemv-variant", choices=["offset", "exact"], default="offset")
+    ap.add_argument("--gemv-variant", choices=["offset", "exact", "tiled"], default="offset")
     ap.add_argument("--tc-a", choices=["tmem", "smem"], default="tmem")
     args = ap.parse_args()
     if args.case:

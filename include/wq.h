@@ -183,7 +183,13 @@ int32_t wq_awq_scale_search(const void* X_dev, int64_t T, int64_t K, const void*
  *                       unpacked (1024 + q) and removes the offset with
  *                       per-chunk activation sums (fewer instructions);
  *                       WQ_GEMV_EXACT subtracts the zero point in fp16 first,
- *                       so every product is exact.
+ *                       so every product is exact (tiled kernel only).
+ *  WQ_OPT_GEMV_KERNEL   WQ_GEMV_KERNEL_AUTO (default): for 4-bit, M <= 2,
+ *                       K <= 16384 and offset sums, the row-streaming kernel
+ *                       (activations held in registers, warps split K);
+ *                       otherwise the tiled kernel (activations in shared
+ *                       memory, warps split rows, cluster split-K).
+ *                       WQ_GEMV_KERNEL_TILED forces the tiled kernel.
  * wq_set_option returns WQ_ERR_INVALID_ARG for an unknown option or value;
  * wq_get_option returns the current value, or -1 for an unknown option. */
 #define WQ_OPT_GEMM_PATH 1
@@ -197,6 +203,9 @@ int32_t wq_awq_scale_search(const void* X_dev, int64_t T, int64_t K, const void*
 #define WQ_OPT_GEMV_VARIANT 4
 #define WQ_GEMV_OFFSET_SUMS 0
 #define WQ_GEMV_EXACT 1
+#define WQ_OPT_GEMV_KERNEL 5
+#define WQ_GEMV_KERNEL_AUTO 0
+#define WQ_GEMV_KERNEL_TILED 2
 int32_t wq_set_option(int32_t option, int64_t value);
 int64_t wq_get_option(int32_t option);
 

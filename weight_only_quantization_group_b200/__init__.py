@@ -72,6 +72,9 @@ WQ_TC_A_SMEM = 1
 WQ_OPT_GEMV_VARIANT = 4
 WQ_GEMV_OFFSET_SUMS = 0
 WQ_GEMV_EXACT = 1
+WQ_OPT_GEMV_KERNEL = 5
+WQ_GEMV_KERNEL_AUTO = 0
+WQ_GEMV_KERNEL_TILED = 2
 
 
 class WQError(RuntimeError):

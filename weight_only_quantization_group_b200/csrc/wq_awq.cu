@@ -191,15 +191,15 @@ awq_loss_kernel(const __grid_constant__ CUtensorMap tmE, const __grid_constant__
       prefetch_tensormap(&tmE);
       prefetch_tensormap(&tmX);
       int issued = 0;
-      for (int kt = 0; kt < KT; ++kt) {
+      for (int kt = 0, s = 0, u = 0; kt < KT; ++kt) {  // s = kt % S, u = kt / S
         if (*abort_flag) break;
-        const int s = kt % S, u = kt / S;
         if (u > 0 && !mbar_wait(&empty[s], (u - 1) & 1, a.err, kAwqSpinLimit)) { *abort_flag = 1; break; }
         uint8_t* st = smem + (size_t)s * kLossStageBytes;
         mbar_arrive_expect_tx(&full[s], kLossStageBytes);
         tma_load_3d(st, &tmE, kt * 64, nt * 128, b, &full[s]);
         tma_load_2d(st + kLossStageBytes / 2, &tmX, kt * 64, tt * 128, &full[s]);
         issued = kt + 1;
+        if (++s == S) { s = 0; ++u; }
       }
       for (int kt = issued > S ? issued - S : 0; kt < issued; ++kt)
         mbar_wait(&full[kt % S], (kt / S) & 1, a.err, kAwqSpinLimit);
@@ -208,9 +208,8 @@ awq_loss_kernel(const __grid_constant__ CUtensorMap tmE, const __grid_constant__
     if (lane == 0) {
       const uint32_t idesc = idesc_f16_f32(128, 128);
       int committed = -1;
-      for (int kt = 0; kt < KT; ++kt) {
+      for (int kt = 0, s = 0, u = 0; kt < KT; ++kt) {  // s = kt % S, u = kt / S
         if (*abort_flag) break;
-        const int s = kt % S, u = kt / S;
         if (!mbar_wait(&full[s], u & 1, a.err, kAwqSpinLimit)) { *abort_flag = 1; break; }
         tc_fence_after();
         const uint32_t base = smem_u32(smem + (size_t)s * kLossStageBytes);
@@ -220,6 +219,7 @@ awq_loss_kernel(const __grid_constant__ CUtensorMap tmE, const __grid_constant__
                      idesc, (kt > 0 || j > 0) ? 1u : 0u);
         mma_commit(&empty[s]);
         committed = kt;
+        if (++s == S) { s = 0; ++u; }
       }
       mma_commit(accum);
       if (*abort_flag && committed >= 0)

@@ -12,10 +12,11 @@
 // [128 lanes = n][M columns]). K advances in stages of 64 input channels:
 //   warp 0    TMA producer: X tile (128-byte swizzle) + packed weight tile
 //   warp 1    TMEM owner and single-thread tcgen05.mma issuer
-//   warps 2-5 dequantize the packed tile (one output channel per thread) into
-//             the A operand -- either shared memory in the canonical 128-byte
-//             swizzled K-major layout, or tensor memory (A_TMEM) -- then run
-//             the epilogue (tcgen05.ld -> fp16 -> Y).
+//   warps 2-9 dequantize the packed tile into the A operand -- either shared
+//             memory in the canonical 128-byte swizzled K-major layout, or
+//             tensor memory (A_TMEM) -- then run the epilogue (tcgen05.ld ->
+//             fp16 -> Y). Warp w owns output channels 32*(w%4)..+31 (the TMEM
+//             lane quarter it may access) and half of each stage's channels.
 // Every mbarrier wait is bounded; on a timeout the kernel latches
 // WQ_ERR_TIMEOUT, drains its own copies, frees its tensor memory and returns.
 #include "wq_sm100.cuh"
@@ -24,8 +25,9 @@ namespace wq {
 
 using namespace sm100;
 
-constexpr int kTcThreads = 192;
-constexpr int kTcBK = 64;              // input channels per stage
+constexpr int kTcThreads = 320;      // 2 control warps + 8 dequant warps
+constexpr int kTcDequantThreads = 256;
+constexpr int kTcBK = 64;              // input channels per stage (half a group)
 constexpr int kTcRows = 128;           // output channels per CTA
 constexpr int kTcPackedStage = kTcRows * kTcBK / 2;  // 4096 bytes
 constexpr int kTcAStage = kTcRows * kTcBK * 2;       // 16384 bytes
@@ -92,7 +94,7 @@ w4a16_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&deq[s], 128);
+      mbar_init(&deq[s], kTcDequantThreads);
       mbar_init(&empty[s], 1);
     }
     mbar_init(accum, 1);
@@ -115,14 +117,14 @@ w4a16_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
       prefetch_tensormap(&tmX);
       prefetch_tensormap(&tmP);
       int issued = 0;
-      for (int kt = 0; kt < KT; ++kt) {
+      for (int kt = 0, s = 0, u = 0; kt < KT; ++kt) {  // s = kt % S, u = kt / S
         if (*abort_flag) break;
-        const int s = kt % S, u = kt / S;
         if (u > 0 && !mbar_wait(&empty[s], (u - 1) & 1, a.err, kSpinLimitCycles)) { *abort_flag = 1; break; }
         mbar_arrive_expect_tx(&full[s], (uint32_t)(b_bytes + kTcPackedStage));
         tma_load_2d(stageB(s), &tmX, kt * kTcBK, 0, &full[s]);
         tma_load_2d(stageP(s), &tmP, kt * (kTcBK / 8), n0, &full[s]);
         issued = kt + 1;
+        if (++s == S) { s = 0; ++u; }
       }
       // Drain: every copy this thread issued has landed before the CTA exits.
       for (int kt = issued > S ? issued - S : 0; kt < issued; ++kt)
@@ -133,9 +135,8 @@ w4a16_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
     if (lane == 0) {
       const uint32_t idesc = idesc_f16_f32(kTcRows, a.BN);
       int committed = -1;
-      for (int kt = 0; kt < KT; ++kt) {
+      for (int kt = 0, s = 0, u = 0; kt < KT; ++kt) {  // s = kt % S, u = kt / S
         if (*abort_flag) break;
-        const int s = kt % S, u = kt / S;
         if (!mbar_wait(&deq[s], u & 1, a.err, kSpinLimitCycles)) { *abort_flag = 1; break; }
         tc_fence_after();
         const uint32_t b_addr = smem_u32(stageB(s));
@@ -151,6 +152,7 @@ w4a16_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
         }
         mma_commit(&empty[s]);
         committed = kt;
+        if (++s == S) { s = 0; ++u; }
       }
       mma_commit(accum);
       if (*abort_flag && committed >= 0)  // let issued MMAs finish before teardown
@@ -159,15 +161,15 @@ w4a16_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
   } else {
     // ---------------------------------------------------------- dequant + epilogue
     const int q = warp & 3;             // TMEM lane quarter this warp may access
+    const int h = (warp - 2) >> 2;      // which half of a stage's 8 packed words
     const int r = 32 * q + lane;        // output channel within the tile
     const int n = n0 + r;
     const bool row_ok = n < a.N;
     __half2 s2 = __float2half2_rn(0.f), zz = s2, zz16n = s2;
-    for (int kt = 0; kt < KT; ++kt) {
+    for (int kt = 0, s = 0, u = 0; kt < KT; ++kt) {  // s = kt % S, u = kt / S
       if (__any_sync(0xffffffffu, *abort_flag != 0)) break;
-      const int s = kt % S, u = kt / S;
-      if ((kt * kTcBK) % kGroup == 0) {
-        const int g = kt * kTcBK / kGroup;
+      if ((kt & 1) == 0) {  // a new 128-channel group every two 64-channel stages
+        const int g = kt >> 1;
         __half st = __float2half(0.f), zr = __float2half(0.f);
         if (row_ok) {
           st = a.steps[(size_t)n * G + g];
@@ -181,41 +183,40 @@ w4a16_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
       }
       const bool landed = mbar_wait(&full[s], u & 1, a.err, kSpinLimitCycles);
       if (!__all_sync(0xffffffffu, landed)) { *abort_flag = 1; break; }
-      const uint4* prow = reinterpret_cast<const uint4*>(stageP(s) + r * 32);
-      const uint4 w0 = prow[0], w1 = prow[1];
-      const uint32_t words[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+      const uint4 w4 = reinterpret_cast<const uint4*>(stageP(s) + r * 32)[h];
+      const uint32_t words[4] = {w4.x, w4.y, w4.z, w4.w};
       if (A_TMEM) {
-        uint32_t v[2][16];
+        uint32_t v[16];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
+        for (int j = 0; j < 4; ++j) {
           const uint4 d = dequant_word4(words[j], zz, zz16n, s2);
-          v[j >> 2][(j & 3) * 4 + 0] = d.x;
-          v[j >> 2][(j & 3) * 4 + 1] = d.y;
-          v[j >> 2][(j & 3) * 4 + 2] = d.z;
-          v[j >> 2][(j & 3) * 4 + 3] = d.w;
+          v[4 * j + 0] = d.x;
+          v[4 * j + 1] = d.y;
+          v[4 * j + 2] = d.z;
+          v[4 * j + 3] = d.w;
         }
-        const uint32_t ta = tmem_a + ((uint32_t)(32 * q) << 16) + (uint32_t)(s * (kTcBK / 2));
-        tmem_st16(ta, v[0]);
-        tmem_st16(ta + 16, v[1]);
+        tmem_st16(tmem_a + ((uint32_t)(32 * q) << 16) + (uint32_t)(s * (kTcBK / 2) + 16 * h), v);
         tmem_st_wait();
         tc_fence_before();
       } else {
         uint8_t* arow = stageA(s) + (r >> 3) * 1024 + (r & 7) * 128;
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
+        for (int j = 0; j < 4; ++j) {
           const uint4 d = dequant_word4(words[j], zz, zz16n, s2);
-          *reinterpret_cast<uint4*>(arow + ((j ^ (r & 7)) << 4)) = d;
+          *reinterpret_cast<uint4*>(arow + (((4 * h + j) ^ (r & 7)) << 4)) = d;
         }
         fence_proxy_async_smem();
       }
       mbar_arrive(&deq[s]);
+      if (++s == S) { s = 0; ++u; }
     }
-    // Epilogue: D[n][m] from TMEM -> Y[m][n].
+    // Epilogue: D[n][m] from TMEM -> Y[m][n]; the two halves take alternate
+    // 16-column chunks.
     bool done = !__any_sync(0xffffffffu, *abort_flag != 0);
     if (done) done = __all_sync(0xffffffffu, mbar_wait(accum, 0, a.err, kSpinLimitCycles));
     if (done) {
       tc_fence_after();
-      for (int c0 = 0; c0 < a.BN; c0 += 16) {
+      for (int c0 = 16 * h; c0 < a.BN; c0 += 32) {
         uint32_t v[16];
         tmem_ld16(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)c0, v);
         tmem_ld_wait();
