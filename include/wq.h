@@ -169,6 +169,31 @@ int32_t wq_awq_scale_search(const void* X_dev, int64_t T, int64_t K, const void*
                             double* loss_out_dev, int32_t* best_out_dev, void* workspace_dev,
                             size_t workspace_bytes, void* stream);
 
+/* The AWQ search of wq_awq_scale_search without a caller workspace.
+ * No counterpart on the pages: an interface addition for callers that
+ * cannot allocate device memory -- code hosted by a framework that owns every
+ * device allocation (plugin hosts, fixed memory pools), or paths where the
+ * device-wide synchronization cudaMalloc may imply is not acceptable. The
+ * caller still passes every input and output buffer, with the meanings of
+ * wq_awq_scale_search; the results are the same (same kernels; alphas are
+ * processed one at a time and the error matrix is built in row chunks).
+ * Scratch: one 24 MiB array in the library's own device memory (a file-scope
+ * static device variable). Every GPU that loads the library holds it until
+ * the process exits. The first call on a device looks up the array's device
+ * address with that device current; make that first call before any stream
+ * capture. All calls share the array, which keeps the last call's contents
+ * (nothing in it has to start at zero), so calls that overlap on the GPU --
+ * from other streams or threads -- race and must be serialized by the caller.
+ * Limits: K <= 16384, n_alpha <= 64 and
+ * n_alpha * ceil(T/128) * ceil(sum_i N_i / 128) <= 786432; a larger problem
+ * returns WQ_ERR_WORKSPACE and enqueues nothing. Calls no cudaMalloc, no
+ * cudaFree and no allocating library routine. */
+int32_t wq_awq_scale_search_noalloc(const void* X_dev, int64_t T, int64_t K, const void* const* W_dev,
+                                    const int64_t* N_i, int32_t n_lin, const wq_quant_cfg* cfg,
+                                    const double* alpha, int32_t n_alpha, void* s_out_dev,
+                                    double* mu_out_dev, double* loss_out_dev, int32_t* best_out_dev,
+                                    void* stream);
+
 /* Process-wide tuning options (not thread-safe against concurrent calls).
  *  WQ_OPT_GEMM_PATH     WQ_PATH_AUTO (default): GEMV kernel below the
  *                       crossover M, tensor-core kernel at or above it (4-bit);

@@ -30,6 +30,7 @@ __all__ = [
     "wq_get_option",
     "wq_awq_workspace_bytes",
     "wq_awq_scale_search",
+    "wq_awq_scale_search_noalloc",
     "EXPORTED_SYMBOLS",
 ]
 
@@ -50,6 +51,7 @@ EXPORTED_SYMBOLS = (
     "wq_get_option",
     "wq_awq_workspace_bytes",
     "wq_awq_scale_search",
+    "wq_awq_scale_search_noalloc",
 )
 
 WQ_OK = 0
@@ -109,6 +111,8 @@ def _load() -> ctypes.CDLL:
         "wq_awq_workspace_bytes": (sz, [i64, i64, ctypes.POINTER(i64), i32, i32, cfgp]),
         "wq_awq_scale_search": (i32, [vp, i64, i64, ctypes.POINTER(vp), ctypes.POINTER(i64), i32, cfgp,
                                       ctypes.POINTER(ctypes.c_double), i32, vp, vp, vp, vp, vp, sz, vp]),
+        "wq_awq_scale_search_noalloc": (i32, [vp, i64, i64, ctypes.POINTER(vp), ctypes.POINTER(i64), i32, cfgp,
+                                              ctypes.POINTER(ctypes.c_double), i32, vp, vp, vp, vp, vp]),
     }
     for name, (res, args) in sig.items():
         f = getattr(L, name)
@@ -287,3 +291,32 @@ def wq_awq_scale_search(X: torch.Tensor, Ws, alphas=None, *, bits: int = 4, grou
                                   workspace.numel() * workspace.element_size(), _stream(stream))
     _raise(st, "wq_awq_scale_search")
     return {"s": s, "mu": mu, "losses": losses, "best": best}
+
+def wq_awq_scale_search_noalloc(X: torch.Tensor, Ws, alphas=None, *, bits: int = 4, group_size: int = 128,
+                                symmetric: bool = False, out=None, stream=None):
+    """wq_awq_scale_search without a workspace: the library's own fixed device
+    scratch is used instead (for callers that cannot allocate device memory;
+    see include/wq.h for its size, limits and sharing rules). `out`, if given,
+    is a dict with preallocated "s", "mu", "losses" and "best" tensors."""
+    _check(X, torch.float16, "X")
+    for i, W in enumerate(Ws):
+        _check(W, torch.float16, f"W[{i}]")
+    T, K = X.shape
+    if alphas is None:
+        alphas = [j / 20.0 for j in range(20)]
+    alphas = [float(a) for a in alphas]
+    c = _cfg(bits, group_size, symmetric)
+    Ns = [int(W.shape[0]) for W in Ws]
+    n_arr = (ctypes.c_int64 * len(Ns))(*Ns)
+    a_arr = (ctypes.c_double * len(alphas))(*alphas)
+    w_arr = (ctypes.c_void_p * len(Ws))(*[W.data_ptr() for W in Ws])
+    if out is None:
+        out = {"s": torch.empty(K, dtype=torch.float16, device=X.device),
+               "mu": torch.empty(K, dtype=torch.float64, device=X.device),
+               "losses": torch.empty(len(alphas), dtype=torch.float64, device=X.device),
+               "best": torch.empty(1, dtype=torch.int32, device=X.device)}
+    st = _lib.wq_awq_scale_search_noalloc(_ptr(X), T, K, w_arr, n_arr, len(Ns), ctypes.byref(c), a_arr,
+                                          len(alphas), _ptr(out["s"]), _ptr(out["mu"]), _ptr(out["losses"]),
+                                          _ptr(out["best"]), _stream(stream))
+    _raise(st, "wq_awq_scale_search_noalloc")
+    return out

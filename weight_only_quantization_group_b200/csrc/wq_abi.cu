@@ -29,6 +29,11 @@ cudaError_t launch_awq_search(const void* X, int64_t T, int64_t K, const void* c
                               int n_lin, int bits, bool sym, const double* alpha, int n_alpha, void* s_out,
                               double* mu_out, double* loss_out, int32_t* best_out, void* workspace, int* err,
                               cudaStream_t st);
+bool awq_noalloc_fits(int64_t T, int64_t K, int64_t N_total, int n_alpha);
+cudaError_t launch_awq_search_noalloc(const void* X, int64_t T, int64_t K, const void* const* W,
+                                      const int64_t* N_i, int n_lin, int bits, bool sym, const double* alpha,
+                                      int n_alpha, void* s_out, double* mu_out, double* loss_out, int32_t* best_out,
+                                      int* err, cudaStream_t st);
 }  // namespace wq
 
 // One flag per device (each device holds its own copy of a __device__ variable).
@@ -215,6 +220,31 @@ int32_t wq_awq_scale_search(const void* X, int64_t T, int64_t K, const void* con
   return cuda_status(wq::launch_awq_search(X, T, K, W, N_i, n_lin, cfg->bits, cfg->symmetric != 0, alpha, n_alpha,
                                            s_out, mu_out, loss_out, best_out, workspace, flag,
                                            static_cast<cudaStream_t>(stream)));
+}
+
+int32_t wq_awq_scale_search_noalloc(const void* X, int64_t T, int64_t K, const void* const* W, const int64_t* N_i,
+                                    int32_t n_lin, const wq_quant_cfg* cfg, const double* alpha, int32_t n_alpha,
+                                    void* s_out, double* mu_out, double* loss_out, int32_t* best_out, void* stream) {
+  int32_t st = check_awq(T, K, N_i, n_lin, n_alpha, cfg);
+  if (st != WQ_OK) return st;
+  if (!X || !W || !alpha || !s_out) return WQ_ERR_INVALID_ARG;
+  int64_t n_total = 0;
+  for (int i = 0; i < n_lin; ++i) {
+    if (!W[i]) return WQ_ERR_INVALID_ARG;
+    if (!aligned(W[i], 16)) return WQ_ERR_ALIGNMENT;
+    n_total += N_i[i];
+  }
+  for (int j = 0; j < n_alpha; ++j)
+    if (!(alpha[j] == alpha[j])) return WQ_ERR_INVALID_ARG;  // NaN
+  if (!aligned(X, 16) || !aligned(s_out, 2) || (mu_out && !aligned(mu_out, 8)) || (loss_out && !aligned(loss_out, 8)) ||
+      (best_out && !aligned(best_out, 4)))
+    return WQ_ERR_ALIGNMENT;
+  if (!wq::awq_noalloc_fits(T, K, n_total, n_alpha)) return WQ_ERR_WORKSPACE;
+  int* flag = device_flag();
+  if (!flag) return WQ_ERR_CUDA;
+  return cuda_status(wq::launch_awq_search_noalloc(X, T, K, W, N_i, n_lin, cfg->bits, cfg->symmetric != 0, alpha,
+                                                   n_alpha, s_out, mu_out, loss_out, best_out, flag,
+                                                   static_cast<cudaStream_t>(stream)));
 }
 
 int32_t wq_set_option(int32_t option, int64_t value) {

@@ -18,6 +18,8 @@
 //                in fp64 -> one partial per (alpha, tile)
 //   finalize     L_j = sum of partials in tile order (deterministic), first
 //                argmin, s_out = s_best
+#include <mutex>
+
 #include "wq_quant_core.cuh"
 #include "wq_sm100.cuh"
 
@@ -420,6 +422,142 @@ cudaError_t launch_awq_search(const void* X, int64_t T, int64_t K, const void* c
         tmE, tmX, la);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
+  }
+  awq_finalize_kernel<<<1, 256, 0, st>>>(partial, p.tiles, n_alpha, S, (int)K, loss_out, best_out,
+                                          static_cast<__half*>(s_out), err);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// The same search without caller scratch (wq_awq_scale_search_noalloc).
+//
+// For callers that cannot allocate device memory, the scratch lives in a
+// file-scope device array owned by the library. Its regions hold mu, the
+// candidate scales, the per-tile partial losses and the error-matrix rows of
+// one chunk; the search runs one alpha at a time and builds E in row chunks
+// of at most kAwqStaticE bytes, so the array stays small for any N.
+// ---------------------------------------------------------------------------
+
+constexpr int kAwqStaticMaxK = 16384;
+constexpr size_t kAwqStaticMu = size_t(kAwqStaticMaxK) * 8;                   // 128 KiB
+constexpr size_t kAwqStaticS = size_t(kAwqMaxAlpha) * kAwqStaticMaxK * 2;     // 2 MiB
+constexpr size_t kAwqStaticPartial = size_t(6) << 20;                          // 6 MiB
+constexpr size_t kAwqStaticE = size_t(16) << 20;                               // 16 MiB
+constexpr size_t kAwqStaticBytes = kAwqStaticMu + kAwqStaticS + kAwqStaticPartial + kAwqStaticE;
+
+static __device__ __align__(256) uint8_t g_awq_static_scratch[kAwqStaticBytes];
+
+// Device address of the array for the current device, looked up once per
+// device (with that device current). nullptr on failure.
+static uint8_t* awq_static_scratch() {
+  static std::mutex mu;
+  static uint8_t* addr[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lk(mu);
+  if (addr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_awq_static_scratch) != cudaSuccess) return nullptr;
+    addr[dev] = static_cast<uint8_t*>(p);
+  }
+  return addr[dev];
+}
+
+bool awq_noalloc_fits(int64_t T, int64_t K, int64_t N_total, int n_alpha) {
+  if (K > kAwqStaticMaxK || n_alpha > kAwqMaxAlpha) return false;
+  const int64_t tiles = ((T + 127) / 128) * ((N_total + 127) / 128);
+  return (size_t)n_alpha * (size_t)tiles * 8 <= kAwqStaticPartial;
+}
+
+cudaError_t launch_awq_search_noalloc(const void* X, int64_t T, int64_t K, const void* const* W,
+                                      const int64_t* N_i, int n_lin, int bits, bool sym, const double* alpha,
+                                      int n_alpha, void* s_out, double* mu_out, double* loss_out, int32_t* best_out,
+                                      int* err, cudaStream_t st) {
+  EncodeTiledFnA enc = awq_encode_fn();
+  if (!enc) return cudaErrorNotSupported;
+  uint8_t* ws = awq_static_scratch();
+  if (!ws) return cudaErrorInvalidSymbol;
+  const AwqPlan p = plan_awq(T, K, N_i, n_lin, n_alpha);  // tile counts only; no memory of its own
+  double* mu = mu_out ? mu_out : reinterpret_cast<double*>(ws);
+  __half* S = reinterpret_cast<__half*>(ws + kAwqStaticMu);
+  double* partial = reinterpret_cast<double*>(ws + kAwqStaticMu + kAwqStaticS);
+  __half* E = reinterpret_cast<__half*>(ws + kAwqStaticMu + kAwqStaticS + kAwqStaticPartial);
+  const __half* Xh = static_cast<const __half*>(X);
+
+  absmean_kernel<<<(unsigned)((K + 255) / 256), 256, 0, st>>>(Xh, (int)T, (int)K, mu);
+  AlphaList al;
+  for (int j = 0; j < kAwqMaxAlpha; ++j) al.v[j] = j < n_alpha ? alpha[j] : 0.0;
+  candidates_kernel<<<dim3((unsigned)((K + 255) / 256), (unsigned)n_alpha), 256, 0, st>>>(mu, (int)K, al, n_alpha,
+                                                                                         S, err);
+  CUtensorMap tmX;
+  {
+    cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)T};
+    cuuint64_t strides[1] = {(cuuint64_t)K * 2};
+    cuuint32_t box[2] = {64, 128};
+    cuuint32_t es[2] = {1, 1};
+    if (enc(&tmX, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<__half*>(Xh), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  }
+  const int stages = 3;
+  const size_t smem = 1024 + (size_t)stages * kLossStageBytes + (2 * stages + 1) * 8 + 4 * 8 + 16;
+  cudaError_t e = cudaFuncSetAttribute(awq_loss_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  const int64_t rows_chunk = (int64_t)(kAwqStaticE / ((size_t)K * 2)) / 128 * 128;
+  int64_t off[kAwqMaxLinears + 1];
+  off[0] = 0;
+  for (int i = 0; i < n_lin; ++i) off[i + 1] = off[i] + N_i[i];
+
+  for (int j = 0; j < n_alpha; ++j) {
+    for (int64_t r0 = 0; r0 < p.N_total; r0 += rows_chunk) {
+      const int64_t r1 = (r0 + rows_chunk) < p.N_total ? (r0 + rows_chunk) : p.N_total;
+      // the stacked linears' rows [r0, r1)
+      LinearSet lc = {};
+      lc.row_off[0] = 0;
+      int nl = 0;
+      for (int i = 0; i < n_lin; ++i) {
+        const int64_t lo = off[i] > r0 ? off[i] : r0;
+        const int64_t hi = off[i + 1] < r1 ? off[i + 1] : r1;
+        if (lo >= hi) continue;
+        lc.W[nl] = static_cast<const __half*>(W[i]) + (lo - off[i]) * K;
+        lc.row_off[nl + 1] = lc.row_off[nl] + (int)(hi - lo);
+        ++nl;
+      }
+      for (int i = nl; i < kAwqMaxLinears; ++i) lc.row_off[i + 1] = lc.row_off[nl];
+      lc.n_lin = nl;
+      lc.n_total = (int)(r1 - r0);
+      const int64_t groups = (r1 - r0) * (K / kGroup);
+      const dim3 eg((unsigned)((groups + 15) / 16), 1u);
+#define WQ_AE(BI, SY) awq_error_kernel<BI, SY><<<eg, 256, 0, st>>>(lc, (int)K, S, j, E)
+      if (bits == 4) { if (sym) WQ_AE(4, true); else WQ_AE(4, false); }
+      else { if (sym) WQ_AE(3, true); else WQ_AE(3, false); }
+#undef WQ_AE
+      CUtensorMap tmE;
+      {
+        cuuint64_t dims[3] = {(cuuint64_t)K, (cuuint64_t)(r1 - r0), 1};
+        cuuint64_t strides[2] = {(cuuint64_t)K * 2, (cuuint64_t)(r1 - r0) * (cuuint64_t)K * 2};
+        cuuint32_t box[3] = {64, 128, 1};
+        cuuint32_t es[3] = {1, 1, 1};
+        if (enc(&tmE, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, E, dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+          return cudaErrorInvalidValue;
+      }
+      // Tiles of this chunk land at their place in the full [alpha][n_tile][t_tile] array.
+      LossArgs la;
+      la.partial = partial + (size_t)(r0 / 128) * p.t_tiles;
+      la.alpha0 = j;
+      la.K = (int)K;
+      la.t_tiles = p.t_tiles;
+      la.n_tiles = p.n_tiles;
+      la.stages = stages;
+      la.err = err;
+      awq_loss_kernel<<<dim3((unsigned)p.t_tiles, (unsigned)((r1 - r0 + 127) / 128), 1u), kLossThreads, smem, st>>>(
+          tmE, tmX, la);
+      e = cudaGetLastError();
+      if (e != cudaSuccess) return e;
+    }
   }
   awq_finalize_kernel<<<1, 256, 0, st>>>(partial, p.tiles, n_alpha, S, (int)K, loss_out, best_out,
                                           static_cast<__half*>(s_out), err);
