@@ -270,7 +270,30 @@ def run_ours(args, rank: int, world: int, local_rank: int):
 
     rows = {}
     if rank == 0 and not args.no_rows:
-        rows = measure_rows(wq, torch, synth, dev, block, peaks)
+        # the same graphs' step time with programmatic dependent launch off
+        wq.wq_set_option(wq.WQ_OPT_PDL, 0)
+        try:
+            g_off = []
+            for ci, blk in enumerate(copies[:2]):
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g, stream=s_cap):
+                    for b, y in zip(blk, Ys[ci]):
+                        wq.wq_w4a16_gemm(b["X"], *b["q"], b["N"], bits=4, out=y)
+                g_off.append(g)
+            torch.cuda.synchronize()
+            for i in range(20):
+                g_off[i % 2].replay()
+            e0.record()
+            for i in range(400):
+                g_off[i % 2].replay()
+            e1.record()
+            torch.cuda.synchronize()
+            rows["block_step_pdl_off"] = {"us": e0.elapsed_time(e1) / 400 * 1e3,
+                                          "note": "2 block copies only (L2 may hold part)"}
+            del g_off
+        finally:
+            wq.wq_set_option(wq.WQ_OPT_PDL, 1)
+        rows = {**rows, **measure_rows(wq, torch, synth, dev, block, peaks)}
 
     del graphs
     if rank != 0:
@@ -395,6 +418,17 @@ def measure_rows(wq, torch, synth, dev, block, peaks):
                 wq.wq_set_option(wq.WQ_OPT_GEMV_KERNEL, wq.WQ_GEMV_KERNEL_AUTO)
                 wq.wq_set_option(wq.WQ_OPT_GEMV_VARIANT, wq.WQ_GEMV_OFFSET_SUMS)
     big = synth.config_smallm_sweep(1)
+    # row-streaming kernel shapes (rows per batch, channels per lane)
+    c65 = synth.config_llama65b_decode(4)
+    for shape, tag in ((1, "r4x32"), (2, "r4x64"), (3, "r8x32"), (4, "r2x64")):
+        wq.wq_set_option(wq.WQ_OPT_GEMV_ROWS_SHAPE, shape)
+        try:
+            gemv_row(f"gemv_rows_{tag}_8192x8192_w4", 8192, 8192, 4, c65.W, c65.X)
+            gemv_row(f"gemv_rows_{tag}_8192x28672_w4", 28672, 8192, 4, big.W, synth.smallm_activations(1))
+            b = block[6]
+            gemv_row(f"gemv_rows_{tag}_{b['name']}", b["N"], b["K"], 4, b["W"].cpu().numpy(), b["Xh"])
+        finally:
+            wq.wq_set_option(wq.WQ_OPT_GEMV_ROWS_SHAPE, 0)
     for M in synth.SMALLM_SWEEP:
         gemv_row(f"smallm_M{M}_8192x28672_w4", 28672, 8192, 4, big.W, synth.smallm_activations(M), M=M)
     # the other kernel on each side of the crossover, for the record

@@ -199,7 +199,7 @@ int32_t wq_awq_scale_search_noalloc(const void* X_dev, int64_t T, int64_t K, con
  *                       crossover M, tensor-core kernel at or above it (4-bit);
  *                       WQ_PATH_GEMV / WQ_PATH_TENSOR_CORE force one kernel
  *                       (the tensor-core kernel is 4-bit only).
- *  WQ_OPT_CROSSOVER_M   smallest M sent to the tensor-core kernel (default 16).
+ *  WQ_OPT_CROSSOVER_M   smallest M sent to the tensor-core kernel (default 3).
  *  WQ_OPT_TC_A_OPERAND  where the tensor-core kernel stages the dequantized
  *                       weight tile: WQ_TC_A_TMEM (tensor memory, default) or
  *                       WQ_TC_A_SMEM (128-byte swizzled shared memory).
@@ -215,6 +215,12 @@ int32_t wq_awq_scale_search_noalloc(const void* X_dev, int64_t T, int64_t K, con
  *                       otherwise the tiled kernel (activations in shared
  *                       memory, warps split rows, cluster split-K).
  *                       WQ_GEMV_KERNEL_TILED forces the tiled kernel.
+ *  WQ_OPT_PDL           1 (default): GEMV launches allow programmatic dependent
+ *                       launch (the kernel fetches its first weights before
+ *                       waiting for the previous kernel in the stream); 0: off.
+ *  WQ_OPT_GEMV_ROWS_SHAPE  rows per batch and input channels per lane of the
+ *                       row-streaming kernel: 0 default (4 rows, 64
+ *                       channels), 1 (4, 32), 2 (4, 64), 3 (8, 32), 4 (2, 64).
  * wq_set_option returns WQ_ERR_INVALID_ARG for an unknown option or value;
  * wq_get_option returns the current value, or -1 for an unknown option. */
 #define WQ_OPT_GEMM_PATH 1
@@ -231,6 +237,8 @@ int32_t wq_awq_scale_search_noalloc(const void* X_dev, int64_t T, int64_t K, con
 #define WQ_OPT_GEMV_KERNEL 5
 #define WQ_GEMV_KERNEL_AUTO 0
 #define WQ_GEMV_KERNEL_TILED 2
+#define WQ_OPT_GEMV_ROWS_SHAPE 6
+#define WQ_OPT_PDL 7
 int32_t wq_set_option(int32_t option, int64_t value);
 int64_t wq_get_option(int32_t option);
 

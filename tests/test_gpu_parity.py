@@ -289,3 +289,21 @@ def test_tc_matches_gemv_path(wq):
             wq.wq_set_option(wq.WQ_OPT_GEMM_PATH, wq.WQ_PATH_AUTO)
         assert_close(outs[path], ref)
     assert_close(outs[wq.WQ_PATH_TENSOR_CORE], outs[wq.WQ_PATH_GEMV].astype(np.float64))
+
+
+@pytest.mark.parametrize("shape", [1, 2, 3, 4])
+@pytest.mark.parametrize("M", [1, 2])
+@pytest.mark.parametrize("NK", [(333, 1152), (1000, 4096), (17, 11008), (130, 16384)])
+def test_gemv_rows_shapes(wq, shape, M, NK):
+    """Every (rows per batch, channels per lane) shape of the row-streaming kernel."""
+    N, K = NK
+    g = synth.rng(800 + shape + M)
+    W = synth.weight(g, N, K, 0.02, channel_frac=0.01, channel_mult=10.0)
+    X = synth.activations(g, M, K, channel_frac=0.01, channel_mult=20.0)
+    (codes, st, z), qg = assert_quant_parity(wq, W, None, 4, False)
+    wq.wq_set_option(wq.WQ_OPT_GEMV_ROWS_SHAPE, shape)
+    try:
+        Y = run_gemm(wq, X, qg, N, 4)
+    finally:
+        wq.wq_set_option(wq.WQ_OPT_GEMV_ROWS_SHAPE, 0)
+    assert_close(Y, O.gemm_ref(X, codes, st, z, 128))

@@ -77,6 +77,8 @@ WQ_GEMV_EXACT = 1
 WQ_OPT_GEMV_KERNEL = 5
 WQ_GEMV_KERNEL_AUTO = 0
 WQ_GEMV_KERNEL_TILED = 2
+WQ_OPT_GEMV_ROWS_SHAPE = 6
+WQ_OPT_PDL = 7
 
 
 class WQError(RuntimeError):
@@ -291,6 +293,7 @@ def wq_awq_scale_search(X: torch.Tensor, Ws, alphas=None, *, bits: int = 4, grou
                                   workspace.numel() * workspace.element_size(), _stream(stream))
     _raise(st, "wq_awq_scale_search")
     return {"s": s, "mu": mu, "losses": losses, "best": best}
+
 
 def wq_awq_scale_search_noalloc(X: torch.Tensor, Ws, alphas=None, *, bits: int = 4, group_size: int = 128,
                                 symmetric: bool = False, out=None, stream=None):

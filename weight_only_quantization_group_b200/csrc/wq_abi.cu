@@ -11,11 +11,11 @@ cudaError_t launch_quantize_pack(const void* W, const void* s, int64_t N, int64_
 cudaError_t launch_unpack_dequant(const uint32_t* packed, const void* steps, const void* zeros, int64_t N,
                                   int64_t K, int bits, void* out, cudaStream_t st);
 cudaError_t launch_gemv(const void* X, const uint32_t* packed, const void* steps, const void* zeros, int64_t M,
-                        int64_t N, int64_t K, int bits, void* Y, cudaStream_t st, int variant);
+                        int64_t N, int64_t K, int bits, void* Y, cudaStream_t st, int variant, bool pdl);
 size_t gemv_smem_bytes(int bits, int variant, int M, int N, int K);
 bool gemv_rows_supported(int bits, int64_t M, int64_t K);
 cudaError_t launch_gemv_rows(const void* X, const uint32_t* packed, const void* steps, const void* zeros, int64_t M,
-                             int64_t N, int64_t K, void* Y, cudaStream_t st);
+                             int64_t N, int64_t K, void* Y, cudaStream_t st, int shape, bool pdl);
 cudaError_t launch_gemm_tc(const void* X, const uint32_t* packed, const void* steps, const void* zeros, int64_t M,
                            int64_t N, int64_t K, void* Y, int* err, cudaStream_t st, bool a_tmem);
 struct AwqPlan {
@@ -80,10 +80,12 @@ int32_t cuda_status(cudaError_t e) { return e == cudaSuccess ? WQ_OK : WQ_ERR_CU
 
 // Process-wide tuning options (wq_set_option).
 int64_t g_opt_gemm_path = WQ_PATH_AUTO;
-int64_t g_opt_crossover_m = 16;
+int64_t g_opt_crossover_m = 3;
+int64_t g_opt_pdl = 1;
 int64_t g_opt_tc_a_operand = WQ_TC_A_TMEM;
 int64_t g_opt_gemv_variant = WQ_GEMV_OFFSET_SUMS;
 int64_t g_opt_gemv_kernel = WQ_GEMV_KERNEL_AUTO;
+int64_t g_opt_gemv_rows_shape = 0;
 
 }  // namespace
 
@@ -167,12 +169,13 @@ int32_t wq_w4a16_gemm(const void* X, const uint32_t* packed, const void* steps, 
   }
   if (g_opt_gemv_kernel != WQ_GEMV_KERNEL_TILED && g_opt_gemv_variant == WQ_GEMV_OFFSET_SUMS &&
       wq::gemv_rows_supported(cfg->bits, M, K))
-    return cuda_status(wq::launch_gemv_rows(X, packed, steps, zeros, M, N, K, Y, static_cast<cudaStream_t>(stream)));
+    return cuda_status(wq::launch_gemv_rows(X, packed, steps, zeros, M, N, K, Y, static_cast<cudaStream_t>(stream),
+                                            (int)g_opt_gemv_rows_shape, g_opt_pdl != 0));
   // The shared copy of an X slice must fit one CTA.
   if (wq::gemv_smem_bytes(cfg->bits, (int)g_opt_gemv_variant, (int)(M < 8 ? M : 8), (int)N, (int)K) > 200 * 1024)
     return WQ_ERR_UNSUPPORTED;
   return cuda_status(wq::launch_gemv(X, packed, steps, zeros, M, N, K, cfg->bits, Y,
-                                     static_cast<cudaStream_t>(stream), (int)g_opt_gemv_variant));
+                                     static_cast<cudaStream_t>(stream), (int)g_opt_gemv_variant, g_opt_pdl != 0));
 }
 
 static int32_t check_awq(int64_t T, int64_t K, const int64_t* N_i, int32_t n_lin, int32_t n_alpha,
@@ -265,6 +268,14 @@ int32_t wq_set_option(int32_t option, int64_t value) {
       if (value != WQ_GEMV_KERNEL_AUTO && value != WQ_GEMV_KERNEL_TILED) return WQ_ERR_INVALID_ARG;
       g_opt_gemv_kernel = value;
       return WQ_OK;
+    case WQ_OPT_PDL:
+      if (value != 0 && value != 1) return WQ_ERR_INVALID_ARG;
+      g_opt_pdl = value;
+      return WQ_OK;
+    case WQ_OPT_GEMV_ROWS_SHAPE:
+      if (value < 0 || value > 4) return WQ_ERR_INVALID_ARG;
+      g_opt_gemv_rows_shape = value;
+      return WQ_OK;
     case WQ_OPT_GEMV_VARIANT:
       if (value != WQ_GEMV_OFFSET_SUMS && value != WQ_GEMV_EXACT) return WQ_ERR_INVALID_ARG;
       g_opt_gemv_variant = value;
@@ -280,6 +291,8 @@ int64_t wq_get_option(int32_t option) {
     case WQ_OPT_TC_A_OPERAND: return g_opt_tc_a_operand;
     case WQ_OPT_GEMV_VARIANT: return g_opt_gemv_variant;
     case WQ_OPT_GEMV_KERNEL: return g_opt_gemv_kernel;
+    case WQ_OPT_GEMV_ROWS_SHAPE: return g_opt_gemv_rows_shape;
+    case WQ_OPT_PDL: return g_opt_pdl;
   }
   return -1;
 }

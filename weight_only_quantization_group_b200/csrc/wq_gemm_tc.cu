@@ -166,14 +166,20 @@ w4a16_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
     const int n = n0 + r;
     const bool row_ok = n < a.N;
     __half2 s2 = __float2half2_rn(0.f), zz = s2, zz16n = s2;
+    // step and zero of the next group, fetched a group ahead of their use
+    __half st_next = __float2half(0.f), zr_next = __float2half(0.f);
+    if (row_ok) {
+      st_next = a.steps[(size_t)n * G];
+      zr_next = a.zeros[(size_t)n * G];
+    }
     for (int kt = 0, s = 0, u = 0; kt < KT; ++kt) {  // s = kt % S, u = kt / S
       if (__any_sync(0xffffffffu, *abort_flag != 0)) break;
       if ((kt & 1) == 0) {  // a new 128-channel group every two 64-channel stages
         const int g = kt >> 1;
-        __half st = __float2half(0.f), zr = __float2half(0.f);
-        if (row_ok) {
-          st = a.steps[(size_t)n * G + g];
-          zr = a.zeros[(size_t)n * G + g];
+        const __half st = st_next, zr = zr_next;
+        if (row_ok && g + 1 < G) {
+          st_next = a.steps[(size_t)n * G + g + 1];
+          zr_next = a.zeros[(size_t)n * G + g + 1];
         }
         s2 = __halves2half2(st, st);
         const __half z1024 = __hadd(zr, __float2half(1024.f));

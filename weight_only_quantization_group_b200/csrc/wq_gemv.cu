@@ -503,7 +503,7 @@ static int gemv_regs() {
 }
 
 template <int BITS, int VAR, int M, int R>
-static cudaError_t launch_gemv_k(GemvArgs a, int N, int K, cudaStream_t st) {
+static cudaError_t launch_gemv_k(GemvArgs a, int N, int K, cudaStream_t st, bool pdl) {
   auto kern = gemv_kernel<BITS, VAR, M, R>;
   const GemvPlan p = plan_gemv(BITS, VAR, M, N, K, gemv_regs<BITS, VAR, M, R>());
   a.gps = p.gps;
@@ -527,27 +527,27 @@ static cudaError_t launch_gemv_k(GemvArgs a, int N, int K, cudaStream_t st) {
     attr[n].val.clusterDim.z = 1;
     ++n;
   }
-  cfg.attrs = attr;
-  cfg.numAttrs = n;
+  cfg.attrs = attr + (pdl ? 0 : 1);
+  cfg.numAttrs = pdl ? n : n - 1;
   return cudaLaunchKernelEx(&cfg, kern, a);
 }
 
 template <int BITS, int VAR, int M>
-static cudaError_t launch_gemv_m(const GemvArgs& a, cudaStream_t st) {
-  return launch_gemv_k<BITS, VAR, M, gemv_rows_per_warp(BITS, M)>(a, a.N, a.K, st);
+static cudaError_t launch_gemv_m(const GemvArgs& a, cudaStream_t st, bool pdl) {
+  return launch_gemv_k<BITS, VAR, M, gemv_rows_per_warp(BITS, M)>(a, a.N, a.K, st, pdl);
 }
 
 template <int BITS, int VAR>
-static cudaError_t launch_gemv_bits(const GemvArgs& a, int M, cudaStream_t st) {
+static cudaError_t launch_gemv_bits(const GemvArgs& a, int M, cudaStream_t st, bool pdl) {
   switch (M) {
-    case 1: return launch_gemv_m<BITS, VAR, 1>(a, st);
-    case 2: return launch_gemv_m<BITS, VAR, 2>(a, st);
-    case 3: return launch_gemv_m<BITS, VAR, 3>(a, st);
-    case 4: return launch_gemv_m<BITS, VAR, 4>(a, st);
-    case 5: return launch_gemv_m<BITS, VAR, 5>(a, st);
-    case 6: return launch_gemv_m<BITS, VAR, 6>(a, st);
-    case 7: return launch_gemv_m<BITS, VAR, 7>(a, st);
-    case 8: return launch_gemv_m<BITS, VAR, 8>(a, st);
+    case 1: return launch_gemv_m<BITS, VAR, 1>(a, st, pdl);
+    case 2: return launch_gemv_m<BITS, VAR, 2>(a, st, pdl);
+    case 3: return launch_gemv_m<BITS, VAR, 3>(a, st, pdl);
+    case 4: return launch_gemv_m<BITS, VAR, 4>(a, st, pdl);
+    case 5: return launch_gemv_m<BITS, VAR, 5>(a, st, pdl);
+    case 6: return launch_gemv_m<BITS, VAR, 6>(a, st, pdl);
+    case 7: return launch_gemv_m<BITS, VAR, 7>(a, st, pdl);
+    case 8: return launch_gemv_m<BITS, VAR, 8>(a, st, pdl);
   }
   return cudaErrorInvalidValue;
 }
@@ -555,7 +555,7 @@ static cudaError_t launch_gemv_bits(const GemvArgs& a, int M, cudaStream_t st) {
 // Y[M][N] for any M >= 1: slabs of up to 8 rows of X per launch.
 // variant: 0 offset sums, 1 exact.
 cudaError_t launch_gemv(const void* X, const uint32_t* packed, const void* steps, const void* zeros, int64_t M,
-                        int64_t N, int64_t K, int bits, void* Y, cudaStream_t st, int variant) {
+                        int64_t N, int64_t K, int bits, void* Y, cudaStream_t st, int variant, bool pdl) {
   for (int64_t m0 = 0; m0 < M; m0 += 8) {
     const int mc = (int)((M - m0) < 8 ? (M - m0) : 8);
     GemvArgs a;
@@ -568,9 +568,9 @@ cudaError_t launch_gemv(const void* X, const uint32_t* packed, const void* steps
     a.K = (int)K;
     cudaError_t e;
     if (bits == 4) {
-      e = variant == kExact ? launch_gemv_bits<4, kExact>(a, mc, st) : launch_gemv_bits<4, kOffset>(a, mc, st);
+      e = variant == kExact ? launch_gemv_bits<4, kExact>(a, mc, st, pdl) : launch_gemv_bits<4, kOffset>(a, mc, st, pdl);
     } else {
-      e = variant == kExact ? launch_gemv_bits<3, kExact>(a, mc, st) : launch_gemv_bits<3, kOffset>(a, mc, st);
+      e = variant == kExact ? launch_gemv_bits<3, kExact>(a, mc, st, pdl) : launch_gemv_bits<3, kOffset>(a, mc, st, pdl);
     }
     if (e != cudaSuccess) return e;
   }
