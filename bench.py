@@ -402,6 +402,8 @@ def measure_rows(wq, torch, synth, dev, block, peaks):
                       "frac_hbm": by / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"], "TFLOP/s": fl / (ms * 1e-3) / 1e12}
         del qs
 
+    c1 = synth.config_small_linear(0)
+    gemv_row("gemv_small_linear_K256_N128", 128, 256, 4, c1.W, c1.X)
     for b in block[:1] + block[4:5] + block[6:7]:
         gemv_row(f"gemv_{b['name']}", b["N"], b["K"], 4, b["W"].cpu().numpy(), b["Xh"])
     for bits in (4, 3):
@@ -432,20 +434,45 @@ def measure_rows(wq, torch, synth, dev, block, peaks):
     for M in synth.SMALLM_SWEEP:
         gemv_row(f"smallm_M{M}_8192x28672_w4", 28672, 8192, 4, big.W, synth.smallm_activations(M), M=M)
     # the other kernel on each side of the crossover, for the record
-    for M in (4, 8, 16, 32):
-        path = wq.WQ_PATH_TENSOR_CORE if M < 16 else wq.WQ_PATH_GEMV
+    for M in (2, 3, 4, 8, 16):
+        path = wq.WQ_PATH_TENSOR_CORE if M < 3 else wq.WQ_PATH_GEMV
         wq.wq_set_option(wq.WQ_OPT_GEMM_PATH, path)
         try:
             tag = "tc" if path == wq.WQ_PATH_TENSOR_CORE else "gemv"
             gemv_row(f"smallm_M{M}_8192x28672_w4_{tag}", 28672, 8192, 4, big.W, synth.smallm_activations(M), M=M)
         finally:
             wq.wq_set_option(wq.WQ_OPT_GEMM_PATH, wq.WQ_PATH_AUTO)
-    wq.wq_set_option(wq.WQ_OPT_TC_A_OPERAND, wq.WQ_TC_A_SMEM)
-    try:
-        for M in (16, 64, 128):
-            gemv_row(f"smallm_M{M}_8192x28672_w4_tc_smemA", 28672, 8192, 4, big.W, synth.smallm_activations(M), M=M)
-    finally:
-        wq.wq_set_option(wq.WQ_OPT_TC_A_OPERAND, wq.WQ_TC_A_TMEM)
+    # S1/S2/S4 AWQ scale search over one LLaMA-2-7B block (4 search places,
+    # T=512 calibration rows, 20 alphas), then packing with the chosen scales
+    groups = synth.config_awq_block(5)
+    prepared = []
+    for gname, X, named in groups:
+        Xd = dt(X)
+        Wd = [dt(W) for _, W in named]
+        need = wq.wq_awq_workspace_bytes(X.shape[0], X.shape[1], [W.shape[0] for W in Wd], 20)
+        ws = torch.empty(need, dtype=torch.uint8, device=dev)
+        prepared.append((gname, Xd, Wd, ws))
+    outs = [wq.wq_awq_scale_search(Xd, Wd, workspace=ws) for _, Xd, Wd, ws in prepared]  # warm-up
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    outs = [wq.wq_awq_scale_search(Xd, Wd, workspace=ws) for _, Xd, Wd, ws in prepared]
+    b.record()
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b)
+    flops = sum(2.0 * Xd.shape[0] * sum(W.shape[0] for W in Wd) * Xd.shape[1] * 20 for _, Xd, Wd, _ in prepared)
+    a.record()
+    for (_, Xd, Wd, _), o in zip(prepared, outs):
+        for W in Wd:
+            wq.wq_quantize_pack(W, o["s"], bits=4)
+    b.record()
+    torch.cuda.synchronize()
+    assert wq.wq_get_last_device_error() == 0
+    rows["awq_search_llama7b_block"] = {
+        "ms": ms, "loss_gemm_TFLOP/s": flops / (ms * 1e-3) / 1e12,
+        "frac_bf16_peak": flops / (ms * 1e-3) / 1e12 / peaks["bf16_tflops"],
+        "best_alpha": {g: int(o["best"].item()) / 20 for (g, _, _, _), o in zip(prepared, outs)},
+        "pack_with_s_ms": a.elapsed_time(b)}
     return rows
 
 
@@ -582,7 +609,6 @@ def run_case(args):
                      else wq.WQ_GEMV_OFFSET_SUMS)
     wq.wq_set_option(wq.WQ_OPT_GEMV_KERNEL, wq.WQ_GEMV_KERNEL_TILED if args.gemv_variant == "tiled"
                      else wq.WQ_GEMV_KERNEL_AUTO)
-    wq.wq_set_option(wq.WQ_OPT_TC_A_OPERAND, wq.WQ_TC_A_SMEM if args.tc_a == "smem" else wq.WQ_TC_A_TMEM)
     q = wq.wq_quantize_pack(W, bits=args.bits)
     Y = torch.empty((args.M, args.N), dtype=torch.float16, device=dev)
     torch.cuda.synchronize()
@@ -626,7 +652,6 @@ def main():
     ap.add_argument("--reps", type=int, default=3)
     ap.add_argument("--path", choices=["auto", "gemv", "tc"], default="auto")
     ap.add_argument("--gemv-variant", choices=["offset", "exact", "tiled"], default="offset")
-    ap.add_argument("--tc-a", choices=["tmem", "smem"], default="tmem")
     args = ap.parse_args()
     if args.case:
         run_case(args)

@@ -200,9 +200,6 @@ int32_t wq_awq_scale_search_noalloc(const void* X_dev, int64_t T, int64_t K, con
  *                       WQ_PATH_GEMV / WQ_PATH_TENSOR_CORE force one kernel
  *                       (the tensor-core kernel is 4-bit only).
  *  WQ_OPT_CROSSOVER_M   smallest M sent to the tensor-core kernel (default 3).
- *  WQ_OPT_TC_A_OPERAND  where the tensor-core kernel stages the dequantized
- *                       weight tile: WQ_TC_A_TMEM (tensor memory, default) or
- *                       WQ_TC_A_SMEM (128-byte swizzled shared memory).
  *  WQ_OPT_GEMV_VARIANT  how the GEMV kernel forms sum_k x_k (q_k - zero):
  *                       WQ_GEMV_OFFSET_SUMS (default) multiplies x by the
  *                       unpacked (1024 + q) and removes the offset with
@@ -225,12 +222,9 @@ int32_t wq_awq_scale_search_noalloc(const void* X_dev, int64_t T, int64_t K, con
  * wq_get_option returns the current value, or -1 for an unknown option. */
 #define WQ_OPT_GEMM_PATH 1
 #define WQ_OPT_CROSSOVER_M 2
-#define WQ_OPT_TC_A_OPERAND 3
 #define WQ_PATH_AUTO 0
 #define WQ_PATH_GEMV 1
 #define WQ_PATH_TENSOR_CORE 2
-#define WQ_TC_A_TMEM 0
-#define WQ_TC_A_SMEM 1
 #define WQ_OPT_GEMV_VARIANT 4
 #define WQ_GEMV_OFFSET_SUMS 0
 #define WQ_GEMV_EXACT 1

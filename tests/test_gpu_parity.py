@@ -236,17 +236,13 @@ def test_smallm_sweep_full_weight(wq):
 # ---------------------------------------------------------------------------
 
 @pytest.fixture
-def tc_path(wq, request):
-    placement = request.param
+def tc_path(wq):
     wq.wq_set_option(wq.WQ_OPT_GEMM_PATH, wq.WQ_PATH_TENSOR_CORE)
-    wq.wq_set_option(wq.WQ_OPT_TC_A_OPERAND, wq.WQ_TC_A_TMEM if placement == "tmem" else wq.WQ_TC_A_SMEM)
-    yield placement
+    yield
     wq.wq_set_option(wq.WQ_OPT_GEMM_PATH, wq.WQ_PATH_AUTO)
-    wq.wq_set_option(wq.WQ_OPT_TC_A_OPERAND, wq.WQ_TC_A_TMEM)
 
 
-@pytest.mark.parametrize("tc_path", ["tmem", "smem"], indirect=True)
-@pytest.mark.parametrize("M", [1, 16, 17, 48, 64, 100, 128, 200, 256, 300])
+@pytest.mark.parametrize("M", [1, 3, 16, 17, 48, 64, 100, 128, 200, 256, 300])
 @pytest.mark.parametrize("NK", [(333, 1152), (1000, 4096)])
 def test_tc_gemm_parity(wq, tc_path, M, NK):
     N, K = NK
@@ -257,7 +253,6 @@ def test_tc_gemm_parity(wq, tc_path, M, NK):
     assert_close(run_gemm(wq, X, qg, N, 4), O.gemm_ref(X, codes, st, z, 128))
 
 
-@pytest.mark.parametrize("tc_path", ["tmem", "smem"], indirect=True)
 def test_tc_gemm_symmetric_and_closed_form(wq, tc_path):
     N, K, M = 256, 1024, 32
     g = np.random.default_rng(21)

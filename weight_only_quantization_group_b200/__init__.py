@@ -65,12 +65,9 @@ WQ_ERR_RANGE = 7
 
 WQ_OPT_GEMM_PATH = 1
 WQ_OPT_CROSSOVER_M = 2
-WQ_OPT_TC_A_OPERAND = 3
 WQ_PATH_AUTO = 0
 WQ_PATH_GEMV = 1
 WQ_PATH_TENSOR_CORE = 2
-WQ_TC_A_TMEM = 0
-WQ_TC_A_SMEM = 1
 WQ_OPT_GEMV_VARIANT = 4
 WQ_GEMV_OFFSET_SUMS = 0
 WQ_GEMV_EXACT = 1

@@ -17,7 +17,7 @@ bool gemv_rows_supported(int bits, int64_t M, int64_t K);
 cudaError_t launch_gemv_rows(const void* X, const uint32_t* packed, const void* steps, const void* zeros, int64_t M,
                              int64_t N, int64_t K, void* Y, cudaStream_t st, int shape, bool pdl);
 cudaError_t launch_gemm_tc(const void* X, const uint32_t* packed, const void* steps, const void* zeros, int64_t M,
-                           int64_t N, int64_t K, void* Y, int* err, cudaStream_t st, bool a_tmem);
+                           int64_t N, int64_t K, void* Y, int* err, cudaStream_t st);
 struct AwqPlan {
   int64_t N_total;
   int t_tiles, n_tiles, tiles;
@@ -82,7 +82,6 @@ int32_t cuda_status(cudaError_t e) { return e == cudaSuccess ? WQ_OK : WQ_ERR_CU
 int64_t g_opt_gemm_path = WQ_PATH_AUTO;
 int64_t g_opt_crossover_m = 3;
 int64_t g_opt_pdl = 1;
-int64_t g_opt_tc_a_operand = WQ_TC_A_TMEM;
 int64_t g_opt_gemv_variant = WQ_GEMV_OFFSET_SUMS;
 int64_t g_opt_gemv_kernel = WQ_GEMV_KERNEL_AUTO;
 int64_t g_opt_gemv_rows_shape = 0;
@@ -165,7 +164,7 @@ int32_t wq_w4a16_gemm(const void* X, const uint32_t* packed, const void* steps, 
     int* flag = device_flag();
     if (!flag) return WQ_ERR_CUDA;
     return cuda_status(wq::launch_gemm_tc(X, packed, steps, zeros, M, N, K, Y, flag,
-                                          static_cast<cudaStream_t>(stream), g_opt_tc_a_operand == WQ_TC_A_TMEM));
+                                          static_cast<cudaStream_t>(stream)));
   }
   if (g_opt_gemv_kernel != WQ_GEMV_KERNEL_TILED && g_opt_gemv_variant == WQ_GEMV_OFFSET_SUMS &&
       wq::gemv_rows_supported(cfg->bits, M, K))
@@ -260,10 +259,6 @@ int32_t wq_set_option(int32_t option, int64_t value) {
       if (value < 1) return WQ_ERR_INVALID_ARG;
       g_opt_crossover_m = value;
       return WQ_OK;
-    case WQ_OPT_TC_A_OPERAND:
-      if (value != WQ_TC_A_TMEM && value != WQ_TC_A_SMEM) return WQ_ERR_INVALID_ARG;
-      g_opt_tc_a_operand = value;
-      return WQ_OK;
     case WQ_OPT_GEMV_KERNEL:
       if (value != WQ_GEMV_KERNEL_AUTO && value != WQ_GEMV_KERNEL_TILED) return WQ_ERR_INVALID_ARG;
       g_opt_gemv_kernel = value;
@@ -288,7 +283,6 @@ int64_t wq_get_option(int32_t option) {
   switch (option) {
     case WQ_OPT_GEMM_PATH: return g_opt_gemm_path;
     case WQ_OPT_CROSSOVER_M: return g_opt_crossover_m;
-    case WQ_OPT_TC_A_OPERAND: return g_opt_tc_a_operand;
     case WQ_OPT_GEMV_VARIANT: return g_opt_gemv_variant;
     case WQ_OPT_GEMV_KERNEL: return g_opt_gemv_kernel;
     case WQ_OPT_GEMV_ROWS_SHAPE: return g_opt_gemv_rows_shape;

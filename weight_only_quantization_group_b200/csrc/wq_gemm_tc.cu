@@ -1,4 +1,4 @@
-// S6: W4A16 matmul on the 5th-generation tensor cores for M = 16..256 rows of X.
+// S6: W4A16 matmul on the 5th-generation tensor cores for M = 3..256 rows of X.
 //
 // When M grows the weight-only matmul stops being a pure weight stream and
 // becomes a dense contraction ("Quantising Large Language Models for
@@ -7,16 +7,20 @@
 // batches). The weight is still read once, packed, and dequantized on chip.
 //
 // Tile: one CTA owns 128 output channels n and all M rows of X ("swap AB":
-// the dequantized weight tile is the 128-row A operand, X is the B operand
-// with N_mma = M rounded up to 16, D = W X^T lives in tensor memory as
-// [128 lanes = n][M columns]). K advances in stages of 64 input channels:
-//   warp 0    TMA producer: X tile (128-byte swizzle) + packed weight tile
-//   warp 1    TMEM owner and single-thread tcgen05.mma issuer
-//   warps 2-9 dequantize the packed tile into the A operand -- either shared
-//             memory in the canonical 128-byte swizzled K-major layout, or
-//             tensor memory (A_TMEM) -- then run the epilogue (tcgen05.ld ->
-//             fp16 -> Y). Warp w owns output channels 32*(w%4)..+31 (the TMEM
-//             lane quarter it may access) and half of each stage's channels.
+// the dequantized weight tile is the 128-row A operand, held in tensor
+// memory; X is the B operand with N_mma = M rounded up to 16; D = W X^T lives
+// in tensor memory as [128 lanes = n][M columns]). K advances in stages of one
+// quantization group (128 input channels):
+//   warp 0    TMA producer into a ring of NS shared-memory stages: the packed
+//             tile (128 rows x 64 bytes, 64-byte swizzle) and the X tile (two
+//             128-byte-swizzled 64-channel boxes)
+//   warp 1    TMEM owner and single-thread tcgen05.mma issuer (8 MMAs/stage)
+//   warps 2-9 dequantize the packed tile into one of two tensor-memory A
+//             buffers (warp w: output channels 32*(w%4)..+31 -- the TMEM lane
+//             quarter it may access -- and half of the group's channels), then
+//             run the epilogue (tcgen05.ld -> fp16 -> Y).
+// The shared-memory ring and the TMEM A ring are separate, so the TMA runs as
+// far ahead as shared memory allows while only two A buffers occupy TMEM.
 // Every mbarrier wait is bounded; on a timeout the kernel latches
 // WQ_ERR_TIMEOUT, drains its own copies, frees its tensor memory and returns.
 #include "wq_sm100.cuh"
@@ -25,13 +29,14 @@ namespace wq {
 
 using namespace sm100;
 
-constexpr int kTcThreads = 320;      // 2 control warps + 8 dequant warps
+constexpr int kTcThreads = 320;          // 2 control warps + 8 dequant warps
 constexpr int kTcDequantThreads = 256;
-constexpr int kTcBK = 64;              // input channels per stage (half a group)
-constexpr int kTcRows = 128;           // output channels per CTA
-constexpr int kTcPackedStage = kTcRows * kTcBK / 2;  // 4096 bytes
-constexpr int kTcAStage = kTcRows * kTcBK * 2;       // 16384 bytes
-constexpr long long kSpinLimitCycles = 4000000000LL; // ~2 s at 2 GHz
+constexpr int kTcBK = 128;               // input channels per stage (= one group)
+constexpr int kTcRows = 128;             // output channels per CTA
+constexpr int kTcPackedStage = kTcRows * kTcBK / 2;  // 8192 bytes
+constexpr int kTcABufs = 2;              // TMEM A buffers
+constexpr int kTcACols = kTcBK / 2;      // 64 TMEM columns per A buffer
+constexpr long long kSpinLimitCycles = 4000000000LL;  // ~2 s at 2 GHz
 
 struct TcArgs {
   const __half* steps;
@@ -39,7 +44,7 @@ struct TcArgs {
   __half* Y;
   int M, N, K;
   int BN;          // MMA N (M rounded up to 16)
-  int stages;
+  int stages;      // shared-memory ring depth
   uint32_t tmem_cols;
   int* err;
 };
@@ -65,37 +70,39 @@ __device__ __forceinline__ uint4 dequant_word4(uint32_t w, __half2 zz, __half2 z
   return r;
 }
 
-template <bool A_TMEM>
 __global__ void __launch_bounds__(kTcThreads, 1)
 w4a16_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmP,
                      TcArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int S = a.stages;
-  const int b_bytes = a.BN * 128;
-  const int stage_bytes = b_bytes + (A_TMEM ? 0 : kTcAStage) + kTcPackedStage;
+  const int xbox = a.BN * 128;                       // one 64-channel X box
+  const int stage_bytes = 2 * xbox + kTcPackedStage;  // X (two boxes) + packed
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + (size_t)S * stage_bytes);
-  uint64_t* deq = full + S;
-  uint64_t* empty = deq + S;
-  uint64_t* accum = empty + S;
+  uint64_t* sempty = full + S;
+  uint64_t* afull = sempty + S;
+  uint64_t* aempty = afull + kTcABufs;
+  uint64_t* accum = aempty + kTcABufs;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accum + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
-  auto stageB = [&](int s) { return smem + (size_t)s * stage_bytes; };
-  auto stageA = [&](int s) { return smem + (size_t)s * stage_bytes + b_bytes; };
-  auto stageP = [&](int s) { return smem + (size_t)s * stage_bytes + b_bytes + (A_TMEM ? 0 : kTcAStage); };
+  auto stageX = [&](int s) { return smem + (size_t)s * stage_bytes; };
+  auto stageP = [&](int s) { return smem + (size_t)s * stage_bytes + 2 * xbox; };
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int n0 = blockIdx.x * kTcRows;
-  const int KT = a.K / kTcBK;
+  const int KT = a.K / kTcBK;  // stages == groups
   const int G = a.K / kGroup;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&deq[s], kTcDequantThreads);
-      mbar_init(&empty[s], 1);
+      mbar_init(&sempty[s], 1);
+    }
+    for (int b = 0; b < kTcABufs; ++b) {
+      mbar_init(&afull[b], kTcDequantThreads);
+      mbar_init(&aempty[b], 1);
     }
     mbar_init(accum, 1);
     *abort_flag = 0;
@@ -109,7 +116,7 @@ w4a16_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t tmem_a = tmem + (uint32_t)a.BN;  // A stages follow the accumulator columns
+  const uint32_t tmem_a = tmem + (uint32_t)a.BN;  // A buffers follow the accumulator columns
 
   if (warp == 0) {
     // ---------------------------------------------------------- TMA producer
@@ -119,9 +126,10 @@ w4a16_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
       int issued = 0;
       for (int kt = 0, s = 0, u = 0; kt < KT; ++kt) {  // s = kt % S, u = kt / S
         if (*abort_flag) break;
-        if (u > 0 && !mbar_wait(&empty[s], (u - 1) & 1, a.err, kSpinLimitCycles)) { *abort_flag = 1; break; }
-        mbar_arrive_expect_tx(&full[s], (uint32_t)(b_bytes + kTcPackedStage));
-        tma_load_2d(stageB(s), &tmX, kt * kTcBK, 0, &full[s]);
+        if (u > 0 && !mbar_wait(&sempty[s], (u - 1) & 1, a.err, kSpinLimitCycles)) { *abort_flag = 1; break; }
+        mbar_arrive_expect_tx(&full[s], (uint32_t)stage_bytes);
+        tma_load_2d(stageX(s), &tmX, kt * kTcBK, 0, &full[s]);
+        tma_load_2d(stageX(s) + xbox, &tmX, kt * kTcBK + 64, 0, &full[s]);
         tma_load_2d(stageP(s), &tmP, kt * (kTcBK / 8), n0, &full[s]);
         issued = kt + 1;
         if (++s == S) { s = 0; ++u; }
@@ -135,86 +143,94 @@ w4a16_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
     if (lane == 0) {
       const uint32_t idesc = idesc_f16_f32(kTcRows, a.BN);
       int committed = -1;
-      for (int kt = 0, s = 0, u = 0; kt < KT; ++kt) {  // s = kt % S, u = kt / S
+      for (int kt = 0, s = 0, b = 0, ub = 0; kt < KT; ++kt) {
         if (*abort_flag) break;
-        if (!mbar_wait(&deq[s], u & 1, a.err, kSpinLimitCycles)) { *abort_flag = 1; break; }
+        if (!mbar_wait(&afull[b], ub & 1, a.err, kSpinLimitCycles)) { *abort_flag = 1; break; }
         tc_fence_after();
-        const uint32_t b_addr = smem_u32(stageB(s));
+        const uint32_t xaddr = smem_u32(stageX(s));
 #pragma unroll
         for (int j = 0; j < kTcBK / 16; ++j) {
-          const uint64_t bd = desc_kmajor_sw128(b_addr + 32 * j);
-          const uint32_t acc = (kt > 0 || j > 0) ? 1u : 0u;
-          if (A_TMEM) {
-            mma_f16_ts(tmem, tmem_a + (uint32_t)(s * (kTcBK / 2) + 8 * j), bd, idesc, acc);
-          } else {
-            mma_f16_ss(tmem, desc_kmajor_sw128(smem_u32(stageA(s)) + 32 * j), bd, idesc, acc);
-          }
+          const uint64_t bd = desc_kmajor_sw128(xaddr + (uint32_t)((j >> 2) * xbox + (j & 3) * 32));
+          mma_f16_ts(tmem, tmem_a + (uint32_t)(b * kTcACols + 8 * j), bd, idesc, (kt > 0 || j > 0) ? 1u : 0u);
         }
-        mma_commit(&empty[s]);
+        mma_commit(&aempty[b]);
+        mma_commit(&sempty[s]);
         committed = kt;
-        if (++s == S) { s = 0; ++u; }
+        if (++s == S) s = 0;
+        if (++b == kTcABufs) { b = 0; ++ub; }
       }
       mma_commit(accum);
       if (*abort_flag && committed >= 0)  // let issued MMAs finish before teardown
-        mbar_wait(&empty[committed % S], (committed / S) & 1, a.err, kSpinLimitCycles);
+        mbar_wait(&aempty[committed % kTcABufs], (committed / kTcABufs) & 1, a.err, kSpinLimitCycles);
     }
   } else {
     // ---------------------------------------------------------- dequant + epilogue
     const int q = warp & 3;             // TMEM lane quarter this warp may access
-    const int h = (warp - 2) >> 2;      // which half of a stage's 8 packed words
+    const int h = (warp - 2) >> 2;      // which half of the group's 16 packed words
     const int r = 32 * q + lane;        // output channel within the tile
     const int n = n0 + r;
     const bool row_ok = n < a.N;
-    __half2 s2 = __float2half2_rn(0.f), zz = s2, zz16n = s2;
-    // step and zero of the next group, fetched a group ahead of their use
+    // step and zero of the next group, fetched a stage ahead of their use
     __half st_next = __float2half(0.f), zr_next = __float2half(0.f);
     if (row_ok) {
       st_next = a.steps[(size_t)n * G];
       zr_next = a.zeros[(size_t)n * G];
     }
-    for (int kt = 0, s = 0, u = 0; kt < KT; ++kt) {  // s = kt % S, u = kt / S
+    // Software pipeline: stage kt is dequantized into registers while the
+    // tensor-memory stores of stage kt-1 complete; then kt-1 is published to
+    // the MMA issuer and kt's stores are issued.
+    uint32_t v0[16], v1[16];
+    int pend_b = -1;  // A buffer whose stores are in flight (-1: none)
+    for (int kt = 0, s = 0, u = 0, b = 0, ub = 0; kt < KT; ++kt) {
       if (__any_sync(0xffffffffu, *abort_flag != 0)) break;
-      if ((kt & 1) == 0) {  // a new 128-channel group every two 64-channel stages
-        const int g = kt >> 1;
-        const __half st = st_next, zr = zr_next;
-        if (row_ok && g + 1 < G) {
-          st_next = a.steps[(size_t)n * G + g + 1];
-          zr_next = a.zeros[(size_t)n * G + g + 1];
-        }
-        s2 = __halves2half2(st, st);
-        const __half z1024 = __hadd(zr, __float2half(1024.f));
-        const __half z64n = __hneg(__hadd(zr, __float2half(64.f)));
-        zz = __halves2half2(z1024, z1024);
-        zz16n = __halves2half2(z64n, z64n);
+      const __half st = st_next, zr = zr_next;
+      if (row_ok && kt + 1 < G) {
+        st_next = a.steps[(size_t)n * G + kt + 1];
+        zr_next = a.zeros[(size_t)n * G + kt + 1];
       }
+      const __half2 s2 = __halves2half2(st, st);
+      const __half z1024 = __hadd(zr, __float2half(1024.f));
+      const __half z64n = __hneg(__hadd(zr, __float2half(64.f)));
+      const __half2 zz = __halves2half2(z1024, z1024);
+      const __half2 zz16n = __halves2half2(z64n, z64n);
       const bool landed = mbar_wait(&full[s], u & 1, a.err, kSpinLimitCycles);
       if (!__all_sync(0xffffffffu, landed)) { *abort_flag = 1; break; }
-      const uint4 w4 = reinterpret_cast<const uint4*>(stageP(s) + r * 32)[h];
-      const uint32_t words[4] = {w4.x, w4.y, w4.z, w4.w};
-      if (A_TMEM) {
-        uint32_t v[16];
+      // the packed tile is 64-byte swizzled: 16-byte chunk c of row r sits at
+      // chunk c ^ ((r >> 1) & 3), which keeps a warp's loads conflict-free
+      const uint8_t* prow = stageP(s) + r * 64;
+      const int sw = (r >> 1) & 3;
+      const uint4 wa = *reinterpret_cast<const uint4*>(prow + (((2 * h) ^ sw) << 4));
+      const uint4 wb = *reinterpret_cast<const uint4*>(prow + (((2 * h + 1) ^ sw) << 4));
+      const uint32_t words[8] = {wa.x, wa.y, wa.z, wa.w, wb.x, wb.y, wb.z, wb.w};
+      uint32_t n0v[16], n1v[16];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const uint4 d = dequant_word4(words[j], zz, zz16n, s2);
-          v[4 * j + 0] = d.x;
-          v[4 * j + 1] = d.y;
-          v[4 * j + 2] = d.z;
-          v[4 * j + 3] = d.w;
-        }
-        tmem_st16(tmem_a + ((uint32_t)(32 * q) << 16) + (uint32_t)(s * (kTcBK / 2) + 16 * h), v);
+      for (int j = 0; j < 4; ++j) {
+        const uint4 d = dequant_word4(words[j], zz, zz16n, s2);
+        n0v[4 * j] = d.x; n0v[4 * j + 1] = d.y; n0v[4 * j + 2] = d.z; n0v[4 * j + 3] = d.w;
+        const uint4 e = dequant_word4(words[4 + j], zz, zz16n, s2);
+        n1v[4 * j] = e.x; n1v[4 * j + 1] = e.y; n1v[4 * j + 2] = e.z; n1v[4 * j + 3] = e.w;
+      }
+      if (pend_b >= 0) {  // publish the previous stage
         tmem_st_wait();
         tc_fence_before();
-      } else {
-        uint8_t* arow = stageA(s) + (r >> 3) * 1024 + (r & 7) * 128;
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const uint4 d = dequant_word4(words[j], zz, zz16n, s2);
-          *reinterpret_cast<uint4*>(arow + (((4 * h + j) ^ (r & 7)) << 4)) = d;
-        }
-        fence_proxy_async_smem();
+        mbar_arrive(&afull[pend_b]);
       }
-      mbar_arrive(&deq[s]);
+      bool ok = true;
+      if (kt >= kTcABufs) ok = mbar_wait(&aempty[b], (ub - 1) & 1, a.err, kSpinLimitCycles);
+      if (!__all_sync(0xffffffffu, ok)) { *abort_flag = 1; break; }
+#pragma unroll
+      for (int i = 0; i < 16; ++i) { v0[i] = n0v[i]; v1[i] = n1v[i]; }
+      const uint32_t ta = tmem_a + ((uint32_t)(32 * q) << 16) + (uint32_t)(b * kTcACols + 32 * h);
+      tmem_st16(ta, v0);
+      tmem_st16(ta + 16, v1);
+      pend_b = b;
       if (++s == S) { s = 0; ++u; }
+      if (++b == kTcABufs) { b = 0; ++ub; }
+    }
+    if (pend_b >= 0) {
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(&afull[pend_b]);
     }
     // Epilogue: D[n][m] from TMEM -> Y[m][n]; the two halves take alternate
     // 16-column chunks.
@@ -267,17 +283,6 @@ static EncodeTiledFn encode_fn() {
   return fn;
 }
 
-static int tc_stages(int BN, bool a_tmem) {
-  const int stage = BN * 128 + (a_tmem ? 0 : kTcAStage) + kTcPackedStage;
-  int s = (200 * 1024) / stage;
-  if (s > 8) s = 8;
-  if (a_tmem) {
-    // TMEM: BN accumulator columns + 32 per stage, within 256 (two CTAs per SM)
-    while (s > 2 && BN + 32 * s > 256) --s;
-  }
-  return s < 2 ? 2 : s;
-}
-
 static uint32_t pow2_cols(uint32_t c) {
   uint32_t p = 32;
   while (p < c) p <<= 1;
@@ -285,13 +290,12 @@ static uint32_t pow2_cols(uint32_t c) {
 }
 
 cudaError_t launch_gemm_tc(const void* X, const uint32_t* packed, const void* steps, const void* zeros, int64_t M,
-                           int64_t N, int64_t K, void* Y, int* err, cudaStream_t st, bool a_tmem) {
+                           int64_t N, int64_t K, void* Y, int* err, cudaStream_t st) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return cudaErrorNotSupported;
   for (int64_t m0 = 0; m0 < M; m0 += 256) {
     const int mc = (int)((M - m0) < 256 ? (M - m0) : 256);
     const int BN = ((mc + 15) / 16) * 16;
-    const bool use_tmem_a = a_tmem && BN <= 192;
     CUtensorMap tmX, tmP;
     {
       cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)mc};
@@ -307,10 +311,10 @@ cudaError_t launch_gemm_tc(const void* X, const uint32_t* packed, const void* st
     {
       cuuint64_t dims[2] = {(cuuint64_t)(K / 8), (cuuint64_t)N};
       cuuint64_t strides[1] = {(cuuint64_t)(K / 2)};
-      cuuint32_t box[2] = {8, 128};
+      cuuint32_t box[2] = {16, 128};
       cuuint32_t es[2] = {1, 1};
       if (enc(&tmP, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<uint32_t*>(packed), dims, strides, box, es,
-              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
         return cudaErrorInvalidValue;
     }
@@ -322,15 +326,22 @@ cudaError_t launch_gemm_tc(const void* X, const uint32_t* packed, const void* st
     a.N = (int)N;
     a.K = (int)K;
     a.BN = BN;
-    a.stages = tc_stages(BN, use_tmem_a);
-    a.tmem_cols = pow2_cols((uint32_t)(BN + (use_tmem_a ? 32 * a.stages : 0)));
+    a.tmem_cols = pow2_cols((uint32_t)(BN + kTcABufs * kTcACols));
+    // Two CTAs per SM when the tile's TMEM fits half of it; the ring gets the
+    // shared memory that leaves.
+    const bool two_per_sm = a.tmem_cols <= 256;
+    const int stage = 2 * BN * 128 + kTcPackedStage;
+    const size_t budget = two_per_sm ? 110 * 1024 : 220 * 1024;
+    int S = (int)((budget - 2048) / stage);
+    if (S > 16) S = 16;
+    if (S < 2) S = 2;
+    a.stages = S;
     a.err = err;
-    const int stage = BN * 128 + (use_tmem_a ? 0 : kTcAStage) + kTcPackedStage;
-    size_t smem = 1024 + (size_t)a.stages * stage + (3 * a.stages + 1) * 8 + 16;
+    size_t smem = 1024 + (size_t)S * stage + (2 * S + 2 * kTcABufs + 1) * 8 + 16;
     // Never more CTAs on an SM than its 512 TMEM columns can hold at once.
-    const size_t smem_floor = a.tmem_cols > 256 ? 120 * 1024 : a.tmem_cols > 128 ? 80 * 1024 : 0;
+    const size_t smem_floor = a.tmem_cols > 256 ? 120 * 1024 : 80 * 1024;
     if (smem < smem_floor) smem = smem_floor;
-    auto kern = use_tmem_a ? w4a16_gemm_tc_kernel<true> : w4a16_gemm_tc_kernel<false>;
+    auto kern = w4a16_gemm_tc_kernel;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     const dim3 grid((unsigned)((N + kTcRows - 1) / kTcRows));

@@ -458,7 +458,6 @@ static GemvPlan plan_gemv(int bits, int var, int M, int N, int K, int regs_per_t
   const int xbytes = 2;
   (void)var;
   const long row_blocks = (N + RB - 1) / RB;
-  const size_t per_chan = (size_t)M * xbytes + (size_t)M * 8 / 32;
   auto smem_for = [&](int S) {
     const int gps = (G + S - 1) / S;
     const int xs = ((gps * kGroup + step - 1) / step) * step;

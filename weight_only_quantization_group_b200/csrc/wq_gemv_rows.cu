@@ -22,8 +22,9 @@
 //     offsets and the zero point are removed per row with the lane's
 //     activation class sums, and the group step multiplies the lane's partial.
 //   * Per batch the R x M partials are reduced across lanes with a butterfly
-//     that halves the value count at each exchange, then across warps through
-//     shared memory in warp order (deterministic).
+//     that halves the value count at each exchange. Across warps they are
+//     summed through shared memory in warp order (deterministic), once per
+//     32/(R*M) batches, so the CTA meets at a barrier only that often.
 #include "wq_common.cuh"
 
 namespace wq {
@@ -131,7 +132,7 @@ __global__ void __launch_bounds__(CPL == 1 ? 512 : 256)
 gemv_rows_kernel(RowsArgs a) {
   constexpr int NV = R * M;
   constexpr int LK = 32 * CPL;  // input channels per lane
-  extern __shared__ __align__(16) float red[];  // [2][nseg][NV]
+  extern __shared__ __align__(16) float red[];  // [2][32 / NV][nseg][NV]
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
   const int nseg = blockDim.x >> 5;
@@ -171,34 +172,46 @@ gemv_rows_kernel(RowsArgs a) {
   }
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
+  // Cross-warp reduction once per NB batches: each batch's per-warp totals go
+  // to a slot of a double-buffered ring; after NB batches one barrier, then
+  // NB*NV threads sum the warps in order and write Y.
+  constexpr int NB = 32 / NV;
   float acc[NV];
-  int buf = 0;
-  auto finish = [&](int row0) {
-    int idx;
-    const float v = butterfly_reduce<NV>(acc, lane, idx);
-    if ((lane & (32 / NV - 1)) == 0) red[(buf * nseg + warp) * NV + idx] = v;
+  int slot = 0, half = 0, first = 0;  // first: local batch index of slot 0
+  auto flush = [&](int nslots) {
     __syncthreads();
-    if (threadIdx.x < NV) {
+    if (threadIdx.x < nslots * NV) {
+      const int sl = threadIdx.x / NV, idx = threadIdx.x % NV;
       float t = 0.f;
-      for (int w = 0; w < nseg; ++w) t += red[(buf * nseg + w) * NV + threadIdx.x];
-      const int r = threadIdx.x / M, m = threadIdx.x % M;
+      for (int w = 0; w < nseg; ++w) t += red[((half * NB + sl) * nseg + w) * NV + idx];
+      const int row0 = (blockIdx.x + (first + sl) * gridDim.x) * R;
+      const int r = idx / M, m = idx % M;
       if (row0 + r < a.N) a.Y[(size_t)m * a.N + row0 + r] = __float2half_rn(t);
     }
-    buf ^= 1;
+    half ^= 1;
+    first += nslots;
+    slot = 0;
+  };
+  auto finish = [&]() {
+    int idx;
+    const float v = butterfly_reduce<NV>(acc, lane, idx);
+    if ((lane & (32 / NV - 1)) == 0) red[((half * NB + slot) * nseg + warp) * NV + idx] = v;
+    if (++slot == NB) flush(NB);
   };
 
   for (int i = 0; i < my; i += 2) {
     const int b = blockIdx.x + i * gridDim.x;
     if (i + 1 < my) rows_issue<R, CPL>(s1, a, (b + gridDim.x) * R, active, row_words, G, lane_word, lane_group);
     rows_compute<M, R, CPL>(s0, acc, xh, c1, xsum);
-    finish(b * R);
+    finish();
     if (i + 1 < my) {
       if (i + 2 < my)
         rows_issue<R, CPL>(s0, a, (b + 2 * gridDim.x) * R, active, row_words, G, lane_word, lane_group);
       rows_compute<M, R, CPL>(s1, acc, xh, c1, xsum);
-      finish((b + gridDim.x) * R);
+      finish();
     }
   }
+  if (slot > 0) flush(slot);
 }
 
 static int rows_num_sms() {
@@ -219,7 +232,7 @@ static cudaError_t launch_rows(const RowsArgs& a, cudaStream_t st, bool pdl) {
   auto kern = gemv_rows_kernel<M, R, CPL>;
   const int nseg = (a.K + 1024 * CPL - 1) / (1024 * CPL);
   const int threads = 32 * nseg;
-  const size_t smem = 2 * (size_t)nseg * R * M * sizeof(float);
+  const size_t smem = 2 * (size_t)32 * nseg * sizeof(float);  // [2][32/NV][nseg][NV]
   int occ = 0;
   cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, threads, smem);
   if (e != cudaSuccess) return e;
