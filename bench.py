@@ -293,6 +293,42 @@ def run_ours(args, rank: int, world: int, local_rank: int):
             del g_off
         finally:
             wq.wq_set_option(wq.WQ_OPT_PDL, 1)
+        # the same seven linears with the ones that share an input concatenated
+        # along N (q|k|v, gate|up): four launches per step, identical codes and
+        # outputs (groups never cross rows)
+        fused_copies = []
+        for blk in copies[:n_copies]:
+            by = {b["name"].split("_")[2]: b for b in blk}
+            f = []
+            for names in (("q", "k", "v"), ("o",), ("gate", "up"), ("down",)):
+                parts = [by[n] for n in names]
+                q = tuple(torch.cat([p["q"][i] for p in parts], 0) for i in range(3))
+                N = sum(p["N"] for p in parts)
+                f.append((parts[0]["X"], q, N, torch.empty((1, N), dtype=torch.float16, device=dev)))
+            fused_copies.append(f)
+        g_fused = []
+        for f in fused_copies:
+            for X, q, N, y in f:
+                wq.wq_w4a16_gemm(X, *q, N, bits=4, out=y)
+            torch.cuda.synchronize()
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=s_cap):
+                for X, q, N, y in f:
+                    wq.wq_w4a16_gemm(X, *q, N, bits=4, out=y)
+            g_fused.append(g)
+        torch.cuda.synchronize()
+        for i in range(20):
+            g_fused[i % n_copies].replay()
+        e0.record()
+        for i in range(400):
+            g_fused[i % n_copies].replay()
+        e1.record()
+        torch.cuda.synchronize()
+        us = e0.elapsed_time(e1) / 400 * 1e3
+        rows["block_step_fused_4_launches"] = {"us": us, "GB/s": step_bytes / (us * 1e-6) / 1e9,
+                                               "frac_hbm": step_bytes / (us * 1e-6) / 1e9 / peaks["hbm_gbs"],
+                                               "note": "q|k|v and gate|up concatenated along N"}
+        del g_fused, fused_copies
         rows = {**rows, **measure_rows(wq, torch, synth, dev, block, peaks)}
 
     del graphs
@@ -300,7 +336,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         return None
 
     clocks = clk.summary()
-    traffic = profiled_traffic("gemv_rows_kernel<1,4>")
+    traffic = profiled_traffic("gemv_rows_kernel")
     achieved = step_bytes / (ms_per_step * 1e-3) / 1e9
     line = {
         "metric": METRIC,
@@ -326,7 +362,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         },
         "roofline": {
             "bound": "hbm",
-            "kernel": "gemv_rows_kernel<1,4>",
+            "kernel": "gemv_rows_kernel (ActHalf offset sums; R4 C32 S3 for K=4096, R4 C64 S2 for K=11008)",
             "achieved": round(achieved, 2),
             "peak": peaks["hbm_gbs"],
             "peak_source": f"{peaks['source']} HBM copy bandwidth",
@@ -422,17 +458,43 @@ def measure_rows(wq, torch, synth, dev, block, peaks):
     big = synth.config_smallm_sweep(1)
     # row-streaming kernel shapes (rows per batch, channels per lane)
     c65 = synth.config_llama65b_decode(4)
-    for shape, tag in ((1, "r4x32"), (2, "r4x64"), (3, "r8x32"), (4, "r2x64")):
+    # and the two ways of forming lane sums (int: integer digits, half: fp32
+    # offset sums), and the grid rule (g0 / g1)
+    shapes = {1: "r4x32s2", 2: "r4x64s2", 3: "r8x32s2", 4: "r2x64s2", 5: "r2x64s3", 6: "r4x32s3", 7: "r2x64s4",
+              8: "r4x64s3", 9: "r4x32s4"}
+    sweep = [("half", wq.WQ_GEMV_OFFSET_SUMS, sh, 1) for sh in shapes]
+    sweep += [("int", wq.WQ_GEMV_INT_DIGITS, sh, 1) for sh in (2, 6)]
+    sweep += [("half", wq.WQ_GEMV_OFFSET_SUMS, sh, 0) for sh in (2, 6)]
+    for vtag, var, shape, gm in sweep:
         wq.wq_set_option(wq.WQ_OPT_GEMV_ROWS_SHAPE, shape)
+        wq.wq_set_option(wq.WQ_OPT_GEMV_VARIANT, var)
+        wq.wq_set_option(wq.WQ_OPT_GEMV_GRID, gm)
         try:
-            gemv_row(f"gemv_rows_{tag}_8192x8192_w4", 8192, 8192, 4, c65.W, c65.X)
-            gemv_row(f"gemv_rows_{tag}_8192x28672_w4", 28672, 8192, 4, big.W, synth.smallm_activations(1))
-            b = block[6]
-            gemv_row(f"gemv_rows_{tag}_{b['name']}", b["N"], b["K"], 4, b["W"].cpu().numpy(), b["Xh"])
+            tag2 = f"{shapes[shape]}_{vtag}_g{gm}"
+            gemv_row(f"gemv_rows_{tag2}_8192x8192_w4", 8192, 8192, 4, c65.W, c65.X)
+            gemv_row(f"gemv_rows_{tag2}_8192x28672_w4", 28672, 8192, 4, big.W, synth.smallm_activations(1))
+            for b in (block[0], block[4], block[6]):
+                gemv_row(f"gemv_rows_{tag2}_{b['name']}", b["N"], b["K"], 4, b["W"].cpu().numpy(), b["Xh"])
+            if shape in (1, 2, 4):
+                gemv_row(f"gemv_rows_{tag2}_M2_8192x28672_w4", 28672, 8192, 4, big.W, synth.smallm_activations(2),
+                         M=2)
         finally:
             wq.wq_set_option(wq.WQ_OPT_GEMV_ROWS_SHAPE, 0)
+            wq.wq_set_option(wq.WQ_OPT_GEMV_VARIANT, wq.WQ_GEMV_OFFSET_SUMS)
+            wq.wq_set_option(wq.WQ_OPT_GEMV_GRID, 1)
     for M in synth.SMALLM_SWEEP:
         gemv_row(f"smallm_M{M}_8192x28672_w4", 28672, 8192, 4, big.W, synth.smallm_activations(M), M=M)
+    # tensor-core kernel ring depth (0 = library choice)
+    for M in (16, 64, 128):
+        for S in (0, 2, 3, 4, 5, 6):
+            wq.wq_set_option(wq.WQ_OPT_TC_STAGES, S)
+            try:
+                gemv_row(f"smallm_M{M}_8192x28672_w4_tc_s{S}", 28672, 8192, 4, big.W, synth.smallm_activations(M),
+                         M=M)
+            except wq.WQError as e:
+                rows[f"smallm_M{M}_8192x28672_w4_tc_s{S}"] = {"error": str(e)}
+            finally:
+                wq.wq_set_option(wq.WQ_OPT_TC_STAGES, 0)
     # the other kernel on each side of the crossover, for the record
     for M in (2, 3, 4, 8, 16):
         path = wq.WQ_PATH_TENSOR_CORE if M < 3 else wq.WQ_PATH_GEMV
@@ -605,10 +667,11 @@ def run_case(args):
     X = torch.from_numpy(synth.activations(g, args.M, args.K)).to(dev)
     opts = {"auto": wq.WQ_PATH_AUTO, "gemv": wq.WQ_PATH_GEMV, "tc": wq.WQ_PATH_TENSOR_CORE}
     wq.wq_set_option(wq.WQ_OPT_GEMM_PATH, opts[args.path])
-    wq.wq_set_option(wq.WQ_OPT_GEMV_VARIANT, wq.WQ_GEMV_EXACT if args.gemv_variant == "exact"
-                     else wq.WQ_GEMV_OFFSET_SUMS)
+    wq.wq_set_option(wq.WQ_OPT_GEMV_VARIANT, {"int": wq.WQ_GEMV_INT_DIGITS, "exact": wq.WQ_GEMV_EXACT}.get(
+        args.gemv_variant, wq.WQ_GEMV_OFFSET_SUMS))
     wq.wq_set_option(wq.WQ_OPT_GEMV_KERNEL, wq.WQ_GEMV_KERNEL_TILED if args.gemv_variant == "tiled"
                      else wq.WQ_GEMV_KERNEL_AUTO)
+    wq.wq_set_option(wq.WQ_OPT_GEMV_ROWS_SHAPE, args.rows_shape)
     q = wq.wq_quantize_pack(W, bits=args.bits)
     Y = torch.empty((args.M, args.N), dtype=torch.float16, device=dev)
     torch.cuda.synchronize()
@@ -651,7 +714,8 @@ def main():
     ap.add_argument("--bits", type=int, default=4)
     ap.add_argument("--reps", type=int, default=3)
     ap.add_argument("--path", choices=["auto", "gemv", "tc"], default="auto")
-    ap.add_argument("--gemv-variant", choices=["offset", "exact", "tiled"], default="offset")
+    ap.add_argument("--gemv-variant", choices=["int", "offset", "exact", "tiled"], default="offset")
+    ap.add_argument("--rows-shape", type=int, default=0, choices=list(range(10)))
     args = ap.parse_args()
     if args.case:
         run_case(args)

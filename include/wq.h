@@ -202,12 +202,20 @@ int32_t wq_awq_scale_search_noalloc(const void* X_dev, int64_t T, int64_t K, con
  *  WQ_OPT_CROSSOVER_M   smallest M sent to the tensor-core kernel (default 3).
  *  WQ_OPT_GEMV_VARIANT  how the GEMV kernel forms sum_k x_k (q_k - zero):
  *                       WQ_GEMV_OFFSET_SUMS (default) multiplies x by the
- *                       unpacked (1024 + q) and removes the offset with
- *                       per-chunk activation sums (fewer instructions);
+ *                       unpacked (1024 + q) in fp32 (exact products) and
+ *                       removes the offset with per-chunk activation sums;
+ *                       WQ_GEMV_INT_DIGITS turns each lane's activations into
+ *                       a 24-bit fixed-point image (exact for every value
+ *                       within 2^-13 of the lane's largest) and accumulates q
+ *                       times its base-256 digits in exact integers (dp4a),
+ *                       removing the zero point in integers; row-streaming
+ *                       kernel only (the tiled kernel treats it as offset
+ *                       sums), and zero points must be integers, as
+ *                       wq_quantize_pack writes them;
  *                       WQ_GEMV_EXACT subtracts the zero point in fp16 first,
  *                       so every product is exact (tiled kernel only).
  *  WQ_OPT_GEMV_KERNEL   WQ_GEMV_KERNEL_AUTO (default): for 4-bit, M <= 2,
- *                       K <= 16384 and offset sums, the row-streaming kernel
+ *                       K <= 16384 and not WQ_GEMV_EXACT, the row-streaming kernel
  *                       (activations held in registers, warps split K);
  *                       otherwise the tiled kernel (activations in shared
  *                       memory, warps split rows, cluster split-K).
@@ -215,9 +223,20 @@ int32_t wq_awq_scale_search_noalloc(const void* X_dev, int64_t T, int64_t K, con
  *  WQ_OPT_PDL           1 (default): GEMV launches allow programmatic dependent
  *                       launch (the kernel fetches its first weights before
  *                       waiting for the previous kernel in the stream); 0: off.
- *  WQ_OPT_GEMV_ROWS_SHAPE  rows per batch and input channels per lane of the
- *                       row-streaming kernel: 0 default (4 rows, 64
- *                       channels), 1 (4, 32), 2 (4, 64), 3 (8, 32), 4 (2, 64).
+ *  WQ_OPT_GEMV_ROWS_SHAPE  rows per batch R, input channels per lane C and
+ *                       register stages S of the row-streaming kernel:
+ *                       0 default (shape 6 for K <= 4096, else 2), 1 (4, 32, 2), 2 (4, 64, 2),
+ *                       3 (8, 32, 2), 4 (2, 64, 2), 5 (2, 64, 3), 6 (4, 32, 3),
+ *                       7 (2, 64, 4), 8 (4, 64, 3), 9 (4, 32, 4). Shapes with
+ *                       C = 32 apply for K <= 8192; above it shape 2 runs.
+ *  WQ_OPT_GEMV_GRID     grid of the row-streaming kernel (all CTAs resident, CTA c
+ *                       takes row batches c, c + grid, ...): 1 default, a CTA
+ *                       for every resident slot; 0 one CTA per batch for small
+ *                       problems, else the same number of batches per CTA.
+ *  WQ_OPT_TC_STAGES     shared-memory ring depth of the tensor-core kernel:
+ *                       0 default (library choice), 2..16 that depth (two CTAs
+ *                       per SM when it fits; the call fails with WQ_ERR_CUDA
+ *                       when one CTA's shared memory cannot hold it).
  * wq_set_option returns WQ_ERR_INVALID_ARG for an unknown option or value;
  * wq_get_option returns the current value, or -1 for an unknown option. */
 #define WQ_OPT_GEMM_PATH 1
@@ -228,11 +247,14 @@ int32_t wq_awq_scale_search_noalloc(const void* X_dev, int64_t T, int64_t K, con
 #define WQ_OPT_GEMV_VARIANT 4
 #define WQ_GEMV_OFFSET_SUMS 0
 #define WQ_GEMV_EXACT 1
+#define WQ_GEMV_INT_DIGITS 2
 #define WQ_OPT_GEMV_KERNEL 5
 #define WQ_GEMV_KERNEL_AUTO 0
 #define WQ_GEMV_KERNEL_TILED 2
 #define WQ_OPT_GEMV_ROWS_SHAPE 6
 #define WQ_OPT_PDL 7
+#define WQ_OPT_TC_STAGES 9
+#define WQ_OPT_GEMV_GRID 10
 int32_t wq_set_option(int32_t option, int64_t value);
 int64_t wq_get_option(int32_t option);
 

@@ -81,3 +81,33 @@ def test_argument_validation_without_gpu(wq):
     assert L.wq_w4a16_gemm(good, good, good, good, 1, 8, 256, by(c), None, None, 0, None) == wq.WQ_ERR_INVALID_ARG
     assert L.wq_unpack_dequant(good, good, good, 8, 256, by(_cfg(wq, bits=6)), good, None) == wq.WQ_ERR_UNSUPPORTED
     assert wq.wq_gemm_workspace_bytes(1, 4096, 4096) == 0
+
+
+def test_option_values_are_validated(wq):
+    """wq_set_option accepts exactly the documented values and wq_get_option
+    reads them back; unknown options and values are refused."""
+    cases = {
+        wq.WQ_OPT_GEMM_PATH: ([0, 1, 2], [-1, 3]),
+        wq.WQ_OPT_CROSSOVER_M: ([1, 3, 64], [0, -5]),
+        wq.WQ_OPT_GEMV_VARIANT: ([0, 1, 2], [3, -1]),
+        wq.WQ_OPT_GEMV_KERNEL: ([0, 2], [1, 3]),
+        wq.WQ_OPT_GEMV_ROWS_SHAPE: ([0, 1, 2, 3, 4, 5, 9, 0], [10, -1]),
+        wq.WQ_OPT_PDL: ([0, 1], [2]),
+        wq.WQ_OPT_TC_STAGES: ([0, 2, 5, 16], [1, 17, -1]),
+        wq.WQ_OPT_GEMV_GRID: ([1, 0], [2, -1]),
+    }
+    for opt, (good, bad) in cases.items():
+        old = wq.wq_get_option(opt)
+        try:
+            for v in good:
+                wq.wq_set_option(opt, v)
+                assert wq.wq_get_option(opt) == v
+            for v in bad:
+                with pytest.raises(wq.WQError):
+                    wq.wq_set_option(opt, v)
+                assert wq.wq_get_option(opt) == good[-1]
+        finally:
+            wq.wq_set_option(opt, old)
+    assert wq.wq_get_option(999) == -1
+    with pytest.raises(wq.WQError):
+        wq.wq_set_option(999, 0)

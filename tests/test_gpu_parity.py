@@ -164,12 +164,14 @@ def _gemv_error_bound(X, steps):
     return (2.0 ** -8) * (ax @ steps.astype(np.float64).T) + 2.0 ** -24
 
 
-@pytest.fixture(params=["rows", "tiled", "tiled_exact"])
+@pytest.fixture(params=["rows_int", "rows_half", "tiled", "tiled_exact"])
 def gemv_variant(wq, request):
-    """GEMV kernel choice: the row-streaming kernel where it applies (default),
-    the tiled kernel with offset sums, the tiled kernel with exact products."""
-    kern = wq.WQ_GEMV_KERNEL_AUTO if request.param == "rows" else wq.WQ_GEMV_KERNEL_TILED
-    var = wq.WQ_GEMV_EXACT if request.param == "tiled_exact" else wq.WQ_GEMV_OFFSET_SUMS
+    """GEMV kernel choice: the row-streaming kernel where it applies, with
+    integer digit products (default) or fp32 offset sums; the tiled kernel
+    with offset sums; the tiled kernel with exact fp16 (q - zero) products."""
+    kern = wq.WQ_GEMV_KERNEL_TILED if request.param.startswith("tiled") else wq.WQ_GEMV_KERNEL_AUTO
+    var = {"rows_int": wq.WQ_GEMV_INT_DIGITS, "rows_half": wq.WQ_GEMV_OFFSET_SUMS,
+           "tiled": wq.WQ_GEMV_OFFSET_SUMS, "tiled_exact": wq.WQ_GEMV_EXACT}[request.param]
     wq.wq_set_option(wq.WQ_OPT_GEMV_KERNEL, kern)
     wq.wq_set_option(wq.WQ_OPT_GEMV_VARIANT, var)
     yield request.param
@@ -253,6 +255,28 @@ def test_tc_gemm_parity(wq, tc_path, M, NK):
     assert_close(run_gemm(wq, X, qg, N, 4), O.gemm_ref(X, codes, st, z, 128))
 
 
+@pytest.mark.parametrize("S", [2, 3, 5, 16])
+@pytest.mark.parametrize("M", [16, 128, 200])
+def test_tc_gemm_ring_depths(wq, tc_path, S, M):
+    """Forced shared-memory ring depths (two CTAs per SM or one), including a
+    ring deeper than the K loop (K = 1152 has 9 stages)."""
+    N, K = 333, 1152
+    g = synth.rng(600 + M + S)
+    W = synth.weight(g, N, K, 0.02, channel_frac=0.01, channel_mult=10.0)
+    X = synth.activations(g, M, K, channel_frac=0.01, channel_mult=20.0)
+    (codes, st, z), qg = assert_quant_parity(wq, W, None, 4, False)
+    wq.wq_set_option(wq.WQ_OPT_TC_STAGES, S)
+    try:
+        if S * (2 * ((M + 15) // 16 * 16) * 128 + 8192) + 2048 > 220 * 1024:
+            with pytest.raises(wq.WQError):
+                run_gemm(wq, X, qg, N, 4)
+            return
+        Y = run_gemm(wq, X, qg, N, 4)
+    finally:
+        wq.wq_set_option(wq.WQ_OPT_TC_STAGES, 0)
+    assert_close(Y, O.gemm_ref(X, codes, st, z, 128))
+
+
 def test_tc_gemm_symmetric_and_closed_form(wq, tc_path):
     N, K, M = 256, 1024, 32
     g = np.random.default_rng(21)
@@ -286,19 +310,96 @@ def test_tc_matches_gemv_path(wq):
     assert_close(outs[wq.WQ_PATH_TENSOR_CORE], outs[wq.WQ_PATH_GEMV].astype(np.float64))
 
 
-@pytest.mark.parametrize("shape", [1, 2, 3, 4])
+@pytest.fixture
+def rows_shape(wq):
+    def set_shape(shape, variant):
+        wq.wq_set_option(wq.WQ_OPT_GEMV_ROWS_SHAPE, shape)
+        wq.wq_set_option(wq.WQ_OPT_GEMV_VARIANT, variant)
+    yield set_shape
+    wq.wq_set_option(wq.WQ_OPT_GEMV_ROWS_SHAPE, 0)
+    wq.wq_set_option(wq.WQ_OPT_GEMV_VARIANT, wq.WQ_GEMV_OFFSET_SUMS)
+
+
+@pytest.mark.parametrize("variant", ["int", "half"])
+@pytest.mark.parametrize("shape", [1, 2, 3, 4, 5, 6, 7, 8, 9])
 @pytest.mark.parametrize("M", [1, 2])
-@pytest.mark.parametrize("NK", [(333, 1152), (1000, 4096), (17, 11008), (130, 16384)])
-def test_gemv_rows_shapes(wq, shape, M, NK):
-    """Every (rows per batch, channels per lane) shape of the row-streaming kernel."""
+@pytest.mark.parametrize("NK", [(333, 1152), (1000, 4096), (17, 11008), (130, 16384), (4099, 256)])
+def test_gemv_rows_shapes(wq, rows_shape, variant, shape, M, NK):
+    """Every (rows per batch, channels per lane, register stages) shape of the
+    row-streaming kernel with both ways of forming the lane sums; ragged N,
+    inactive lanes (K = 256 leaves most lanes of the single warp idle), K up
+    to 16384, and CTAs with fewer row batches than stages (N = 17)."""
     N, K = NK
     g = synth.rng(800 + shape + M)
     W = synth.weight(g, N, K, 0.02, channel_frac=0.01, channel_mult=10.0)
     X = synth.activations(g, M, K, channel_frac=0.01, channel_mult=20.0)
     (codes, st, z), qg = assert_quant_parity(wq, W, None, 4, False)
-    wq.wq_set_option(wq.WQ_OPT_GEMV_ROWS_SHAPE, shape)
+    rows_shape(shape, wq.WQ_GEMV_INT_DIGITS if variant == "int" else wq.WQ_GEMV_OFFSET_SUMS)
+    assert_close(run_gemm(wq, X, qg, N, 4), O.gemm_ref(X, codes, st, z, 128))
+
+
+@pytest.mark.parametrize("shape", [2, 6])
+@pytest.mark.parametrize("NK", [(333, 1152), (4096, 4096), (17, 11008), (4099, 256)])
+def test_gemv_rows_grid_rule0(wq, rows_shape, shape, NK):
+    """Grid rule 0 (one CTA per batch, or equal batches per CTA) against the oracle."""
+    N, K = NK
+    g = synth.rng(870 + shape)
+    W = synth.weight(g, N, K, 0.02, channel_frac=0.01, channel_mult=10.0)
+    X = synth.activations(g, 1, K, channel_frac=0.01, channel_mult=20.0)
+    (codes, st, z), qg = assert_quant_parity(wq, W, None, 4, False)
+    rows_shape(shape, wq.WQ_GEMV_OFFSET_SUMS)
+    wq.wq_set_option(wq.WQ_OPT_GEMV_GRID, 0)
     try:
         Y = run_gemm(wq, X, qg, N, 4)
     finally:
-        wq.wq_set_option(wq.WQ_OPT_GEMV_ROWS_SHAPE, 0)
+        wq.wq_set_option(wq.WQ_OPT_GEMV_GRID, 1)
     assert_close(Y, O.gemm_ref(X, codes, st, z, 128))
+
+
+@pytest.mark.parametrize("M", [1, 2])
+def test_gemv_int_digits_error_bound(wq, rows_shape, M):
+    """The integer-digit variant rounds only its fixed-point image of X (exact
+    here for all but values below 2^-13 of a lane's largest), the fp32
+    combination of each lane's digit sums, the fp32 sums across lanes and
+    warps, and the fp16 output. So every output lies within half an fp16 ulp
+    of the exact value plus 2^-20 of sum_k |x_k (q_k - zero) step|, far inside
+    the offset-sum variant's 2^-8 step sum|x| per chunk."""
+    N, K = 777, 4096
+    g = synth.rng(900 + M)
+    W = synth.weight(g, N, K, 0.02, channel_frac=0.01, channel_mult=10.0)
+    X = synth.activations(g, M, K)
+    (codes, st, z), qg = assert_quant_parity(wq, W, None, 4, False)
+    rows_shape(0, wq.WQ_GEMV_INT_DIGITS)
+    Y = run_gemm(wq, X, qg, N, 4).astype(np.float64)
+    D = O.dequantize(codes, st, z, 128)
+    ref = X.astype(np.float64) @ D.T
+    mag = np.abs(X.astype(np.float64)) @ np.abs(D).T
+    assert np.all(np.abs(Y - ref) <= 2.0 ** -11 * np.abs(ref) + 2.0 ** -20 * mag + 2.0 ** -24)
+
+
+def test_gemv_int_digits_extreme_activations(wq, rows_shape):
+    """fp16 extremes inside one lane's channels (65504, subnormals, zeros,
+    mixed signs) and an all-zero lane: the per-lane exponent keeps every
+    image in range, and all-zero X gives exactly zero."""
+    N, K = 64, 1024
+    g = synth.rng(950)
+    W = synth.weight(g, N, K, 0.02)
+    (codes, st, z), qg = assert_quant_parity(wq, W, None, 4, False)
+    X = synth.activations(g, 2, K)
+    X[0, :64] = 0
+    X[0, 64] = 65504.0
+    X[0, 65] = -65504.0
+    X[0, 66:70] = np.float16(6e-8)
+    X[0, 70] = np.float16(-2.0 ** -14)
+    X[1, 128:192] = np.float16(-3e-5)
+    X[1, 192] = 1000.0
+    for variant in (wq.WQ_GEMV_INT_DIGITS, wq.WQ_GEMV_OFFSET_SUMS):
+        rows_shape(0, variant)
+        for M in (1, 2):
+            Xm = X[:M] if M == 1 else X
+            Y = run_gemm(wq, Xm, qg, N, 4)
+            ref = O.gemm_ref(Xm, codes, st, z, 128)
+            assert np.all(np.isfinite(Y))
+            assert_close(Y, ref)
+    rows_shape(0, wq.WQ_GEMV_INT_DIGITS)
+    assert np.all(run_gemm(wq, np.zeros((1, K), np.float16), qg, N, 4) == 0)

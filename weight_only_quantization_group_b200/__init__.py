@@ -71,11 +71,14 @@ WQ_PATH_TENSOR_CORE = 2
 WQ_OPT_GEMV_VARIANT = 4
 WQ_GEMV_OFFSET_SUMS = 0
 WQ_GEMV_EXACT = 1
+WQ_GEMV_INT_DIGITS = 2
 WQ_OPT_GEMV_KERNEL = 5
 WQ_GEMV_KERNEL_AUTO = 0
 WQ_GEMV_KERNEL_TILED = 2
 WQ_OPT_GEMV_ROWS_SHAPE = 6
 WQ_OPT_PDL = 7
+WQ_OPT_TC_STAGES = 9
+WQ_OPT_GEMV_GRID = 10
 
 
 class WQError(RuntimeError):

@@ -15,9 +15,10 @@ cudaError_t launch_gemv(const void* X, const uint32_t* packed, const void* steps
 size_t gemv_smem_bytes(int bits, int variant, int M, int N, int K);
 bool gemv_rows_supported(int bits, int64_t M, int64_t K);
 cudaError_t launch_gemv_rows(const void* X, const uint32_t* packed, const void* steps, const void* zeros, int64_t M,
-                             int64_t N, int64_t K, void* Y, cudaStream_t st, int shape, bool pdl);
+                             int64_t N, int64_t K, void* Y, cudaStream_t st, int shape, bool act_int, int grid_mode,
+                             bool pdl);
 cudaError_t launch_gemm_tc(const void* X, const uint32_t* packed, const void* steps, const void* zeros, int64_t M,
-                           int64_t N, int64_t K, void* Y, int* err, cudaStream_t st);
+                           int64_t N, int64_t K, void* Y, int* err, cudaStream_t st, int stages_opt);
 struct AwqPlan {
   int64_t N_total;
   int t_tiles, n_tiles, tiles;
@@ -85,6 +86,8 @@ int64_t g_opt_pdl = 1;
 int64_t g_opt_gemv_variant = WQ_GEMV_OFFSET_SUMS;
 int64_t g_opt_gemv_kernel = WQ_GEMV_KERNEL_AUTO;
 int64_t g_opt_gemv_rows_shape = 0;
+int64_t g_opt_tc_stages = 0;
+int64_t g_opt_gemv_grid = 1;
 
 }  // namespace
 
@@ -164,17 +167,21 @@ int32_t wq_w4a16_gemm(const void* X, const uint32_t* packed, const void* steps, 
     int* flag = device_flag();
     if (!flag) return WQ_ERR_CUDA;
     return cuda_status(wq::launch_gemm_tc(X, packed, steps, zeros, M, N, K, Y, flag,
-                                          static_cast<cudaStream_t>(stream)));
+                                          static_cast<cudaStream_t>(stream), (int)g_opt_tc_stages));
   }
-  if (g_opt_gemv_kernel != WQ_GEMV_KERNEL_TILED && g_opt_gemv_variant == WQ_GEMV_OFFSET_SUMS &&
+  if (g_opt_gemv_kernel != WQ_GEMV_KERNEL_TILED && g_opt_gemv_variant != WQ_GEMV_EXACT &&
       wq::gemv_rows_supported(cfg->bits, M, K))
     return cuda_status(wq::launch_gemv_rows(X, packed, steps, zeros, M, N, K, Y, static_cast<cudaStream_t>(stream),
-                                            (int)g_opt_gemv_rows_shape, g_opt_pdl != 0));
+                                            (int)g_opt_gemv_rows_shape, g_opt_gemv_variant == WQ_GEMV_INT_DIGITS,
+                                            (int)g_opt_gemv_grid, g_opt_pdl != 0));
   // The shared copy of an X slice must fit one CTA.
-  if (wq::gemv_smem_bytes(cfg->bits, (int)g_opt_gemv_variant, (int)(M < 8 ? M : 8), (int)N, (int)K) > 200 * 1024)
+  if (wq::gemv_smem_bytes(cfg->bits, g_opt_gemv_variant == WQ_GEMV_EXACT ? WQ_GEMV_EXACT : WQ_GEMV_OFFSET_SUMS,
+                          (int)(M < 8 ? M : 8), (int)N, (int)K) > 200 * 1024)
     return WQ_ERR_UNSUPPORTED;
+  // the tiled kernel forms the integer-digit variant's sums as offset sums
+  const int tiled_variant = g_opt_gemv_variant == WQ_GEMV_EXACT ? WQ_GEMV_EXACT : WQ_GEMV_OFFSET_SUMS;
   return cuda_status(wq::launch_gemv(X, packed, steps, zeros, M, N, K, cfg->bits, Y,
-                                     static_cast<cudaStream_t>(stream), (int)g_opt_gemv_variant, g_opt_pdl != 0));
+                                     static_cast<cudaStream_t>(stream), tiled_variant, g_opt_pdl != 0));
 }
 
 static int32_t check_awq(int64_t T, int64_t K, const int64_t* N_i, int32_t n_lin, int32_t n_alpha,
@@ -268,11 +275,20 @@ int32_t wq_set_option(int32_t option, int64_t value) {
       g_opt_pdl = value;
       return WQ_OK;
     case WQ_OPT_GEMV_ROWS_SHAPE:
-      if (value < 0 || value > 4) return WQ_ERR_INVALID_ARG;
+      if (value < 0 || value > 9) return WQ_ERR_INVALID_ARG;
       g_opt_gemv_rows_shape = value;
       return WQ_OK;
+    case WQ_OPT_GEMV_GRID:
+      if (value != 0 && value != 1) return WQ_ERR_INVALID_ARG;
+      g_opt_gemv_grid = value;
+      return WQ_OK;
+    case WQ_OPT_TC_STAGES:
+      if (value != 0 && (value < 2 || value > 16)) return WQ_ERR_INVALID_ARG;
+      g_opt_tc_stages = value;
+      return WQ_OK;
     case WQ_OPT_GEMV_VARIANT:
-      if (value != WQ_GEMV_OFFSET_SUMS && value != WQ_GEMV_EXACT) return WQ_ERR_INVALID_ARG;
+      if (value != WQ_GEMV_OFFSET_SUMS && value != WQ_GEMV_EXACT && value != WQ_GEMV_INT_DIGITS)
+        return WQ_ERR_INVALID_ARG;
       g_opt_gemv_variant = value;
       return WQ_OK;
   }
@@ -286,6 +302,8 @@ int64_t wq_get_option(int32_t option) {
     case WQ_OPT_GEMV_VARIANT: return g_opt_gemv_variant;
     case WQ_OPT_GEMV_KERNEL: return g_opt_gemv_kernel;
     case WQ_OPT_GEMV_ROWS_SHAPE: return g_opt_gemv_rows_shape;
+    case WQ_OPT_TC_STAGES: return g_opt_tc_stages;
+    case WQ_OPT_GEMV_GRID: return g_opt_gemv_grid;
     case WQ_OPT_PDL: return g_opt_pdl;
   }
   return -1;

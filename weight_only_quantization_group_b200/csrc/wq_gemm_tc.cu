@@ -289,8 +289,10 @@ static uint32_t pow2_cols(uint32_t c) {
   return p;
 }
 
+// stages_opt: 0 = library choice; otherwise the shared-memory ring depth (two
+// CTAs per SM when that ring and the tile's TMEM fit half an SM).
 cudaError_t launch_gemm_tc(const void* X, const uint32_t* packed, const void* steps, const void* zeros, int64_t M,
-                           int64_t N, int64_t K, void* Y, int* err, cudaStream_t st) {
+                           int64_t N, int64_t K, void* Y, int* err, cudaStream_t st, int stages_opt) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return cudaErrorNotSupported;
   for (int64_t m0 = 0; m0 < M; m0 += 256) {
@@ -327,14 +329,21 @@ cudaError_t launch_gemm_tc(const void* X, const uint32_t* packed, const void* st
     a.K = (int)K;
     a.BN = BN;
     a.tmem_cols = pow2_cols((uint32_t)(BN + kTcABufs * kTcACols));
-    // Two CTAs per SM when the tile's TMEM fits half of it; the ring gets the
-    // shared memory that leaves.
-    const bool two_per_sm = a.tmem_cols <= 256;
+    // Two CTAs per SM when the tile's TMEM fits half of it and half the shared
+    // memory still holds a ring of three stages; otherwise one CTA per SM with
+    // the deepest ring that fits.
     const int stage = 2 * BN * 128 + kTcPackedStage;
-    const size_t budget = two_per_sm ? 110 * 1024 : 220 * 1024;
-    int S = (int)((budget - 2048) / stage);
-    if (S > 16) S = 16;
-    if (S < 2) S = 2;
+    const size_t half_budget = 110 * 1024, full_budget = 220 * 1024;
+    int S;
+    if (stages_opt > 0) {
+      S = stages_opt;
+      if ((size_t)S * stage + 2048 > full_budget) return cudaErrorInvalidValue;
+    } else {
+      const bool two_per_sm = a.tmem_cols <= 256 && 3 * (size_t)stage + 2048 <= half_budget;
+      S = (int)(((two_per_sm ? half_budget : full_budget) - 2048) / stage);
+      if (S > 16) S = 16;
+      if (S < 2) S = 2;
+    }
     a.stages = S;
     a.err = err;
     size_t smem = 1024 + (size_t)S * stage + (2 * S + 2 * kTcABufs + 1) * 8 + 16;

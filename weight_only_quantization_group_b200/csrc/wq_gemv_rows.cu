@@ -7,24 +7,35 @@
 // minimal:
 //   * K is split across the warps of a CTA: warp w, lane l owns the LK = 32
 //     or 64 consecutive input channels (w*32 + l)*LK .. +LK-1 for the whole
-//     kernel. Its activations (and their class sums for the offset
-//     correction) live in registers, loaded once -- no shared-memory copy of
-//     X, no split-K, no clusters.
+//     kernel. Its activations live in registers, loaded once -- no
+//     shared-memory copy of X, no split-K, no clusters.
 //   * A CTA streams batches of R consecutive rows (persistent over row
 //     batches). Per row a lane issues LK/32 16-byte loads, and a warp reads
-//     16*LK contiguous bytes. The next batch is loaded while the
-//     current one is computed (two register stages); the first batch is
-//     requested before the programmatic-dependent-launch wait, since only X
-//     depends on the previous kernel.
-//   * Dequantization: one LOP3 with 0x6400 in both fp16 lanes gives
-//     (1024 + q, 1024 + q') or (1024 + 16q, 1024 + 16q'); a mixed fp16 x fp16
-//     -> fp32 FMA multiplies it by the activation pair (exact products). The
-//     offsets and the zero point are removed per row with the lane's
-//     activation class sums, and the group step multiplies the lane's partial.
+//     16*LK contiguous bytes. The next batch is loaded while the current one
+//     is computed (two register stages); the first batch is requested before
+//     the programmatic-dependent-launch wait, since only X depends on the
+//     previous kernel.
 //   * Per batch the R x M partials are reduced across lanes with a butterfly
 //     that halves the value count at each exchange. Across warps they are
 //     summed through shared memory in warp order (deterministic), once per
 //     32/(R*M) batches, so the CTA meets at a barrier only that often.
+//
+// Two ways to form a lane's sum_k x_k (q_k - zero) over its channels:
+//   ActInt (default): the lane's activations become one 24-bit fixed-point
+//     image x_k ~ X_k 2^-F (F per lane and row of X, |X_k| < 2^22, so every
+//     fp16 value within 2^-13 of the lane's largest is exact and the others
+//     are rounded by at most 2^-23 of it), split into three base-256 digits.
+//     A packed code word masked with 0xF0F0F0F0 -- before and after a 4-bit
+//     shift -- holds 16 q of four channels in its bytes, and dp4a multiplies
+//     them by four digits at once. Every product and sum is an exact
+//     integer; the zero point is removed per digit in integers, and the only
+//     roundings are the fixed-point image and the final fp32 combination of
+//     three digit sums per row and lane.
+//   ActHalf: one LOP3 with 0x6400 in both fp16 lanes gives (1024 + q,
+//     1024 + q') or (1024 + 16q, 1024 + 16q'); a mixed fp16 x fp16 -> fp32
+//     FMA multiplies it by the activation pair (exact products, fp32 sums).
+//     The offsets and the zero point are removed per row with the lane's
+//     activation class sums.
 #include "wq_common.cuh"
 
 namespace wq {
@@ -65,6 +76,196 @@ __device__ __forceinline__ void rows_issue(RowsStage<R, CPL>& s, const RowsArgs&
   }
 }
 
+template <int CPL>
+__device__ __forceinline__ uint32_t stage_word(const uint4 (&w)[CPL], int j) {
+  const uint4 wv = w[j >> 2];
+  return (j & 3) == 0 ? wv.x : (j & 3) == 1 ? wv.y : (j & 3) == 2 ? wv.z : wv.w;
+}
+
+// The lane's LK = 32*CPL activations of each of the M rows of X.
+template <int M, int CPL>
+__device__ __forceinline__ void load_lane_x(uint32_t (&xh)[M][16 * CPL], const RowsArgs& a, int k0, bool active) {
+#pragma unroll
+  for (int m = 0; m < M; ++m) {
+#pragma unroll
+    for (int j = 0; j < 4 * CPL; ++j) {
+      uint4 v = make_uint4(0, 0, 0, 0);
+      if (active) v = *reinterpret_cast<const uint4*>(a.X + (size_t)m * a.K + k0 + 8 * j);
+      xh[m][4 * j] = v.x; xh[m][4 * j + 1] = v.y; xh[m][4 * j + 2] = v.z; xh[m][4 * j + 3] = v.w;
+    }
+  }
+}
+
+// ---------------------------------------------------------------- ActHalf
+template <int M, int CPL>
+struct ActHalf {
+  uint32_t xh[M][16 * CPL];
+  float c1[M], xsum[M];
+
+  __device__ __forceinline__ void load(const RowsArgs& a, int k0, bool active) {
+    load_lane_x<M, CPL>(xh, a, k0, active);
+#pragma unroll
+    for (int m = 0; m < M; ++m) {
+      float x1 = 0.f, x2 = 0.f;  // channel classes {0,1,4,5} and {2,3,6,7} mod 8
+#pragma unroll
+      for (int i = 0; i < 16 * CPL; ++i) {
+        const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&xh[m][i]));
+        if ((i & 1) == 0) x1 += f.x + f.y;
+        else x2 += f.x + f.y;
+      }
+      c1[m] = 1024.f * x1 + 64.f * x2;
+      xsum[m] = x1 + x2;
+    }
+  }
+
+  template <int R>
+  __device__ __forceinline__ void compute(const RowsStage<R, CPL>& s, float (&acc)[R * M]) const {
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      float a[M][4];
+#pragma unroll
+      for (int m = 0; m < M; ++m) a[m][0] = a[m][1] = a[m][2] = a[m][3] = 0.f;
+#pragma unroll
+      for (int j = 0; j < 4 * CPL; ++j) {
+        const uint32_t w = stage_word<CPL>(s.w[r], j);
+        const uint32_t w8 = w >> 8;
+        const uint32_t p0 = and_or(w, 0x000F000Fu, kHalf2Magic);   // k+0,k+1   x1
+        const uint32_t p1 = and_or(w, 0x00F000F0u, kHalf2Magic);   // k+2,k+3   x16
+        const uint32_t p2 = and_or(w8, 0x000F000Fu, kHalf2Magic);  // k+4,k+5   x1
+        const uint32_t p3 = and_or(w8, 0x00F000F0u, kHalf2Magic);  // k+6,k+7   x16
+#pragma unroll
+        for (int m = 0; m < M; ++m) {
+          fma2_f16_f32(a[m][0], a[m][1], xh[m][4 * j + 0], p0);
+          fma2_f16_f32(a[m][2], a[m][3], xh[m][4 * j + 1], p1);
+          fma2_f16_f32(a[m][0], a[m][1], xh[m][4 * j + 2], p2);
+          fma2_f16_f32(a[m][2], a[m][3], xh[m][4 * j + 3], p3);
+        }
+      }
+      const float sc = __half2float(s.sc[r]);
+      const float z = __half2float(s.zh[r]);
+#pragma unroll
+      for (int m = 0; m < M; ++m) {
+        // sum_k x (q - z) = A1 + A2/16 - (1024 X1 + 64 X2) - z (X1 + X2)
+        float t = fmaf(a[m][2] + a[m][3], 0.0625f, a[m][0] + a[m][1]) - c1[m];
+        t = fmaf(-z, xsum[m], t);
+        acc[r * M + m] = sc * t;
+      }
+    }
+  }
+};
+
+// ---------------------------------------------------------------- ActInt
+__device__ __forceinline__ int dp4a_uu(uint32_t a, uint32_t b, int c) {
+  int d;
+  asm("dp4a.u32.u32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+__device__ __forceinline__ int dp4a_us(uint32_t a, uint32_t b, int c) {
+  int d;
+  asm("dp4a.u32.s32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+__device__ __forceinline__ uint32_t pack_bytes(int b0, int b1, int b2, int b3) {
+  return (uint32_t)(b0 & 0xFF) | ((uint32_t)(b1 & 0xFF) << 8) | ((uint32_t)(b2 & 0xFF) << 16) |
+         ((uint32_t)(b3 & 0xFF) << 24);
+}
+
+template <int M, int CPL>
+struct ActInt {
+  // Digit t of the fixed-point image, four channels per word in the byte
+  // order of the masked code words: lo[c] holds channels 8c + (0, 4, 1, 5)
+  // (the low nibbles of the word's bytes), hi[c] channels 8c + (2, 6, 3, 7).
+  uint32_t lo[M][3][4 * CPL], hi[M][3][4 * CPL];
+  int d16[M][3];  // 16 * sum over the lane's channels of digit t
+  float inv[M];   // 2^-(F + 4): undoes the image scale and the 16 of the masked codes
+
+  __device__ __forceinline__ void load(const RowsArgs& a, int k0, bool active) {
+    uint32_t xh[M][16 * CPL];
+    load_lane_x<M, CPL>(xh, a, k0, active);
+#pragma unroll
+    for (int m = 0; m < M; ++m) {
+      float mx = 0.f;
+#pragma unroll
+      for (int i = 0; i < 16 * CPL; ++i) {
+        const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&xh[m][i]));
+        mx = fmaxf(mx, fmaxf(fabsf(f.x), fabsf(f.y)));
+      }
+      // 2^(e-1) <= mx < 2^e; F = 22 - e keeps |x| 2^F <= 2^22. mx is 0 or at
+      // least 2^-24 (an fp16 value), so e lies in [-23, 17] and F in [5, 45].
+      const int e = mx > 0.f ? (int)((__float_as_uint(mx) >> 23) & 0xFF) - 126 : 22;
+      const int F = 22 - e;
+      const float scale = __uint_as_float((uint32_t)(F + 127) << 23);
+      inv[m] = __uint_as_float((uint32_t)(127 - F - 4) << 23);
+      int sum[3] = {0, 0, 0};
+#pragma unroll
+      for (int c = 0; c < 4 * CPL; ++c) {
+        int xi[8];
+#pragma unroll
+        for (int h = 0; h < 4; ++h) {
+          const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&xh[m][4 * c + h]));
+          xi[2 * h] = __float2int_rn(f.x * scale);
+          xi[2 * h + 1] = __float2int_rn(f.y * scale);
+        }
+#pragma unroll
+        for (int t = 0; t < 3; ++t) {
+          int d[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            d[i] = t == 2 ? (xi[i] >> 16) : ((xi[i] >> (8 * t)) & 0xFF);  // top digit signed
+            sum[t] += d[i];
+          }
+          lo[m][t][c] = pack_bytes(d[0], d[4], d[1], d[5]);
+          hi[m][t][c] = pack_bytes(d[2], d[6], d[3], d[7]);
+        }
+      }
+#pragma unroll
+      for (int t = 0; t < 3; ++t) d16[m][t] = 16 * sum[t];
+    }
+  }
+
+  template <int R>
+  __device__ __forceinline__ void compute(const RowsStage<R, CPL>& s, float (&acc)[R * M]) const {
+    // Words outer, rows inner: R*M*3 independent dp4a chains.
+    int a[R][M][3];
+#pragma unroll
+    for (int r = 0; r < R; ++r)
+#pragma unroll
+      for (int m = 0; m < M; ++m) a[r][m][0] = a[r][m][1] = a[r][m][2] = 0;
+#pragma unroll
+    for (int j = 0; j < 4 * CPL; ++j) {
+#pragma unroll
+      for (int r = 0; r < R; ++r) {
+        const uint32_t w = stage_word<CPL>(s.w[r], j);
+        const uint32_t l16 = (w << 4) & 0xF0F0F0F0u;  // 16 q of channels 0, 4, 1, 5
+        const uint32_t h16 = w & 0xF0F0F0F0u;         // 16 q of channels 2, 6, 3, 7
+#pragma unroll
+        for (int m = 0; m < M; ++m) {
+          a[r][m][0] = dp4a_uu(l16, lo[m][0][j], a[r][m][0]);
+          a[r][m][1] = dp4a_uu(l16, lo[m][1][j], a[r][m][1]);
+          a[r][m][2] = dp4a_us(l16, lo[m][2][j], a[r][m][2]);
+          a[r][m][0] = dp4a_uu(h16, hi[m][0][j], a[r][m][0]);
+          a[r][m][1] = dp4a_uu(h16, hi[m][1][j], a[r][m][1]);
+          a[r][m][2] = dp4a_us(h16, hi[m][2][j], a[r][m][2]);
+        }
+      }
+    }
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      // Zero points are integers in [0, 15]; 16 sum_k (q - z) d_t is exact in
+      // int32 and below 2^24 in magnitude, so exact in fp32 too.
+      const int z = __half2int_rn(s.zh[r]);
+      const float sc = __half2float(s.sc[r]);
+#pragma unroll
+      for (int m = 0; m < M; ++m) {
+        const float e0 = (float)(a[r][m][0] - z * d16[m][0]);
+        const float e1 = (float)(a[r][m][1] - z * d16[m][1]);
+        const float e2 = (float)(a[r][m][2] - z * d16[m][2]);
+        acc[r * M + m] = sc * (inv[m] * fmaf(65536.f, e2, fmaf(256.f, e1, e0)));
+      }
+    }
+  }
+};
+
 // Sum over the 32 lanes of v[idx] for every idx: afterwards lanes whose low
 // (5 - log2 NV) bits are zero hold one total each, for value `index`.
 template <int NV>
@@ -88,47 +289,9 @@ __device__ __forceinline__ float butterfly_reduce(float (&v)[NV], int lane, int&
   return t;
 }
 
-template <int M, int R, int CPL>
-__device__ __forceinline__ void rows_compute(const RowsStage<R, CPL>& s, float (&acc)[R * M],
-                                             const uint32_t (&xh)[M][16 * CPL], const float (&c1)[M],
-                                             const float (&xsum)[M]) {
-#pragma unroll
-  for (int r = 0; r < R; ++r) {
-    float a[M][4];
-#pragma unroll
-    for (int m = 0; m < M; ++m) a[m][0] = a[m][1] = a[m][2] = a[m][3] = 0.f;
-#pragma unroll
-    for (int j = 0; j < 4 * CPL; ++j) {
-      const uint4 wv = s.w[r][j >> 2];
-      const uint32_t w = (j & 3) == 0 ? wv.x : (j & 3) == 1 ? wv.y : (j & 3) == 2 ? wv.z : wv.w;
-      const uint32_t w8 = w >> 8;
-      const uint32_t p0 = and_or(w, 0x000F000Fu, kHalf2Magic);   // k+0,k+1   x1
-      const uint32_t p1 = and_or(w, 0x00F000F0u, kHalf2Magic);   // k+2,k+3   x16
-      const uint32_t p2 = and_or(w8, 0x000F000Fu, kHalf2Magic);  // k+4,k+5   x1
-      const uint32_t p3 = and_or(w8, 0x00F000F0u, kHalf2Magic);  // k+6,k+7   x16
-#pragma unroll
-      for (int m = 0; m < M; ++m) {
-        fma2_f16_f32(a[m][0], a[m][1], xh[m][4 * j + 0], p0);
-        fma2_f16_f32(a[m][2], a[m][3], xh[m][4 * j + 1], p1);
-        fma2_f16_f32(a[m][0], a[m][1], xh[m][4 * j + 2], p2);
-        fma2_f16_f32(a[m][2], a[m][3], xh[m][4 * j + 3], p3);
-      }
-    }
-    const float sc = __half2float(s.sc[r]);
-    const float z = __half2float(s.zh[r]);
-#pragma unroll
-    for (int m = 0; m < M; ++m) {
-      // sum_k x (q - z) = A1 + A2/16 - (1024 X1 + 64 X2) - z (X1 + X2)
-      float t = fmaf(a[m][2] + a[m][3], 0.0625f, a[m][0] + a[m][1]) - c1[m];
-      t = fmaf(-z, xsum[m], t);
-      acc[r * M + m] = sc * t;
-    }
-  }
-}
-
-// K <= 16384: at most 16 warps of 32 channels per lane, or 8 of 64.
-template <int M, int R, int CPL>
-__global__ void __launch_bounds__(CPL == 1 ? 512 : 256)
+// At most 8 warps: K <= 8192 with 32 channels per lane, K <= 16384 with 64.
+template <int M, int R, int CPL, int S, template <int, int> class Act>
+__global__ void __launch_bounds__(256)
 gemv_rows_kernel(RowsArgs a) {
   constexpr int NV = R * M;
   constexpr int LK = 32 * CPL;  // input channels per lane
@@ -145,31 +308,17 @@ gemv_rows_kernel(RowsArgs a) {
   const int nbatch = (a.N + R - 1) / R;
   const int my = blockIdx.x < nbatch ? (nbatch - 1 - blockIdx.x) / gridDim.x + 1 : 0;
 
-  RowsStage<R, CPL> s0, s1;
-  if (my > 0) rows_issue<R, CPL>(s0, a, blockIdx.x * R, active, row_words, G, lane_word, lane_group);
+  // S register stages: batches i+1 .. i+S-1 are in flight while batch i is
+  // computed. The first S-1 are requested before the dependent-launch wait.
+  RowsStage<R, CPL> st[S];
+#pragma unroll
+  for (int j = 0; j < S - 1; ++j)
+    if (j < my)
+      rows_issue<R, CPL>(st[j], a, (blockIdx.x + j * gridDim.x) * R, active, row_words, G, lane_word, lane_group);
   asm volatile("griddepcontrol.wait;" ::: "memory");
 
-  // Activations of this lane's LK channels, and their class sums.
-  uint32_t xh[M][16 * CPL];
-  float c1[M], xsum[M];
-#pragma unroll
-  for (int m = 0; m < M; ++m) {
-#pragma unroll
-    for (int j = 0; j < 4 * CPL; ++j) {
-      uint4 v = make_uint4(0, 0, 0, 0);
-      if (active) v = *reinterpret_cast<const uint4*>(a.X + (size_t)m * a.K + k0 + 8 * j);
-      xh[m][4 * j] = v.x; xh[m][4 * j + 1] = v.y; xh[m][4 * j + 2] = v.z; xh[m][4 * j + 3] = v.w;
-    }
-    float x1 = 0.f, x2 = 0.f;  // channel classes {0,1,4,5} and {2,3,6,7} mod 8
-#pragma unroll
-    for (int i = 0; i < 16 * CPL; ++i) {
-      const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&xh[m][i]));
-      if ((i & 1) == 0) x1 += f.x + f.y;
-      else x2 += f.x + f.y;
-    }
-    c1[m] = 1024.f * x1 + 64.f * x2;
-    xsum[m] = x1 + x2;
-  }
+  Act<M, CPL> act;
+  act.load(a, k0, active);
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
   // Cross-warp reduction once per NB batches: each batch's per-warp totals go
@@ -199,16 +348,17 @@ gemv_rows_kernel(RowsArgs a) {
     if (++slot == NB) flush(NB);
   };
 
-  for (int i = 0; i < my; i += 2) {
-    const int b = blockIdx.x + i * gridDim.x;
-    if (i + 1 < my) rows_issue<R, CPL>(s1, a, (b + gridDim.x) * R, active, row_words, G, lane_word, lane_group);
-    rows_compute<M, R, CPL>(s0, acc, xh, c1, xsum);
-    finish();
-    if (i + 1 < my) {
-      if (i + 2 < my)
-        rows_issue<R, CPL>(s0, a, (b + 2 * gridDim.x) * R, active, row_words, G, lane_word, lane_group);
-      rows_compute<M, R, CPL>(s1, acc, xh, c1, xsum);
-      finish();
+  for (int i = 0; i < my; i += S) {
+#pragma unroll
+    for (int j = 0; j < S; ++j) {
+      if (i + j < my) {
+        const int nx = i + j + S - 1;
+        if (nx < my)
+          rows_issue<R, CPL>(st[(j + S - 1) % S], a, (blockIdx.x + nx * gridDim.x) * R, active, row_words, G,
+                             lane_word, lane_group);
+        act.template compute<R>(st[j], acc);
+        finish();
+      }
     }
   }
   if (slot > 0) flush(slot);
@@ -227,30 +377,31 @@ static int rows_num_sms() {
 
 bool gemv_rows_supported(int bits, int64_t M, int64_t K) { return bits == 4 && M <= 2 && K <= 16384; }
 
-template <int M, int R, int CPL>
-static cudaError_t launch_rows(const RowsArgs& a, cudaStream_t st, bool pdl) {
-  auto kern = gemv_rows_kernel<M, R, CPL>;
+// Persistent grid, all CTAs resident; CTA c takes row batches c, c + grid, ...
+//   mode 0: small problems take one CTA per row batch (most loads in flight
+//           at once); larger ones give every CTA the same number of batches.
+//   mode 1 (default): every resident slot gets a CTA (grid = min(batches,
+//           slots)), so each SM receives batches in turn with its CTAs.
+static long rows_grid(long nbatch, int occ, int mode) {
+  const long slots = (long)(occ < 1 ? 1 : occ) * rows_num_sms();
+  if (mode == 1 || nbatch <= 2 * slots) return nbatch < slots ? nbatch : slots;
+  const long per_cta = (nbatch + slots - 1) / slots;
+  return (nbatch + per_cta - 1) / per_cta;
+}
+
+template <int M, int R, int CPL, int S, template <int, int> class Act>
+static cudaError_t launch_rows(const RowsArgs& a, cudaStream_t st, bool pdl, int grid_mode) {
+  auto kern = gemv_rows_kernel<M, R, CPL, S, Act>;
   const int nseg = (a.K + 1024 * CPL - 1) / (1024 * CPL);
   const int threads = 32 * nseg;
   const size_t smem = 2 * (size_t)32 * nseg * sizeof(float);  // [2][32/NV][nseg][NV]
   int occ = 0;
   cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, threads, smem);
   if (e != cudaSuccess) return e;
-  if (occ < 1) occ = 1;
-  // Persistent grid, all CTAs resident. Small problems take one CTA per row
-  // batch (most loads in flight at once); larger ones give every CTA the same
-  // number of batches.
+  if (occ < 1) return cudaErrorInvalidConfiguration;
   const long nbatch = (a.N + R - 1) / R;
-  const long slots = (long)occ * rows_num_sms();
-  long grid;
-  if (nbatch <= 2 * slots) {
-    grid = nbatch < slots ? nbatch : slots;
-  } else {
-    const long per_cta = (nbatch + slots - 1) / slots;
-    grid = (nbatch + per_cta - 1) / per_cta;
-  }
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)grid, 1, 1);
+  cfg.gridDim = dim3((unsigned)rows_grid(nbatch, occ, grid_mode), 1, 1);
   cfg.blockDim = dim3(threads, 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
@@ -262,9 +413,36 @@ static cudaError_t launch_rows(const RowsArgs& a, cudaStream_t st, bool pdl) {
   return cudaLaunchKernelEx(&cfg, kern, a);
 }
 
-// shape: 0 = default; 1 = (R 4, 32 channels/lane); 2 = (R 4, 64); 3 = (R 8, 32); 4 = (R 2, 64).
+template <int M, int R, int CPL, int S>
+static cudaError_t launch_rows_act(const RowsArgs& a, cudaStream_t st, bool pdl, bool act_int, int grid_mode) {
+  return act_int ? launch_rows<M, R, CPL, S, ActInt>(a, st, pdl, grid_mode)
+                 : launch_rows<M, R, CPL, S, ActHalf>(a, st, pdl, grid_mode);
+}
+
+// shape: rows per batch R, input channels per lane 32*CPL, register stages S
+//   0 = default (6 for K <= 4096, else 2), 1 = (4, 32, 2), 2 = (4, 64, 2), 3 = (8, 32, 2), 4 = (2, 64, 2),
+//   5 = (2, 64, 3), 6 = (4, 32, 3), 7 = (2, 64, 4), 8 = (4, 64, 3), 9 = (4, 32, 4).
+// Shapes with 32 channels per lane take K <= 8192; above that shape 2 runs.
+// act_int: integer digits (true) or fp16 FMA (false) for the lane's dot products.
+template <int M>
+static cudaError_t launch_rows_shape(const RowsArgs& a, cudaStream_t st, bool pdl, bool act_int, int shape,
+                                     int gm) {
+  switch (shape) {
+    case 1: return launch_rows_act<M, 4, 1, 2>(a, st, pdl, act_int, gm);
+    case 3: return launch_rows_act<M, 8, 1, 2>(a, st, pdl, act_int, gm);
+    case 4: return launch_rows_act<M, 2, 2, 2>(a, st, pdl, act_int, gm);
+    case 5: return launch_rows_act<M, 2, 2, 3>(a, st, pdl, act_int, gm);
+    case 6: return launch_rows_act<M, 4, 1, 3>(a, st, pdl, act_int, gm);
+    case 7: return launch_rows_act<M, 2, 2, 4>(a, st, pdl, act_int, gm);
+    case 8: return launch_rows_act<M, 4, 2, 3>(a, st, pdl, act_int, gm);
+    case 9: return launch_rows_act<M, 4, 1, 4>(a, st, pdl, act_int, gm);
+    default: return launch_rows_act<M, 4, 2, 2>(a, st, pdl, act_int, gm);
+  }
+}
+
 cudaError_t launch_gemv_rows(const void* X, const uint32_t* packed, const void* steps, const void* zeros, int64_t M,
-                             int64_t N, int64_t K, void* Y, cudaStream_t st, int shape, bool pdl) {
+                             int64_t N, int64_t K, void* Y, cudaStream_t st, int shape, bool act_int, int grid_mode,
+                             bool pdl) {
   RowsArgs a;
   a.X = static_cast<const __half*>(X);
   a.P = packed;
@@ -273,21 +451,10 @@ cudaError_t launch_gemv_rows(const void* X, const uint32_t* packed, const void* 
   a.Y = static_cast<__half*>(Y);
   a.N = (int)N;
   a.K = (int)K;
-  if (shape == 0) shape = 2;
-  if (M == 1) {
-    switch (shape) {
-      case 1: return launch_rows<1, 4, 1>(a, st, pdl);
-      case 3: return launch_rows<1, 8, 1>(a, st, pdl);
-      case 4: return launch_rows<1, 2, 2>(a, st, pdl);
-      default: return launch_rows<1, 4, 2>(a, st, pdl);
-    }
-  }
-  switch (shape) {
-    case 1: return launch_rows<2, 4, 1>(a, st, pdl);
-    case 3: return launch_rows<2, 8, 1>(a, st, pdl);
-    case 4: return launch_rows<2, 2, 2>(a, st, pdl);
-    default: return launch_rows<2, 4, 2>(a, st, pdl);
-  }
+  if (shape == 0) shape = K <= 4096 ? 6 : 2;  // measured fastest on 4096- and 8192/11008-channel rows
+  if (K > 8192 && (shape == 1 || shape == 3 || shape == 6 || shape == 9)) shape = 2;  // at most 8 warps
+  return M == 1 ? launch_rows_shape<1>(a, st, pdl, act_int, shape, grid_mode)
+                : launch_rows_shape<2>(a, st, pdl, act_int, shape, grid_mode);
 }
 
 }  // namespace wq
