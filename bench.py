@@ -674,6 +674,9 @@ def run_case(args):
     wq.wq_set_option(wq.WQ_OPT_GEMV_ROWS_SHAPE, args.rows_shape)
     q = wq.wq_quantize_pack(W, bits=args.bits)
     Y = torch.empty((args.M, args.N), dtype=torch.float16, device=dev)
+    if args.case == "awq":  # M calibration rows, one linear of N outputs, 20 alphas
+        ws = torch.empty(wq.wq_awq_workspace_bytes(args.M, args.K, [args.N], 20, bits=args.bits),
+                         dtype=torch.uint8, device=dev)
     torch.cuda.synchronize()
     times = []
     for _ in range(args.reps):
@@ -681,6 +684,8 @@ def run_case(args):
         a.record()
         if args.case == "gemm":
             wq.wq_w4a16_gemm(X, *q, args.N, bits=args.bits, out=Y)
+        elif args.case == "awq":
+            wq.wq_awq_scale_search(X, [W], bits=args.bits, workspace=ws)
         else:
             wq.wq_quantize_pack(W, bits=args.bits, out=q)
         b.record()
@@ -706,7 +711,7 @@ def main():
     ap.add_argument("--eager", action="store_true", help="launch eagerly instead of replaying CUDA graphs")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--ref-seconds", type=float, default=60.0)
-    ap.add_argument("--case", choices=["gemm", "quantize"], default=None,
+    ap.add_argument("--case", choices=["gemm", "quantize", "awq"], default=None,
                     help="run one small kernel configuration --reps times (for profiling)")
     ap.add_argument("--M", type=int, default=1)
     ap.add_argument("--N", type=int, default=8192)
