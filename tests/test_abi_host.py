@@ -91,7 +91,7 @@ def test_option_values_are_validated(wq):
         wq.WQ_OPT_CROSSOVER_M: ([1, 3, 64], [0, -5]),
         wq.WQ_OPT_GEMV_VARIANT: ([0, 1, 2], [3, -1]),
         wq.WQ_OPT_GEMV_KERNEL: ([0, 2], [1, 3]),
-        wq.WQ_OPT_GEMV_ROWS_SHAPE: ([0, 1, 2, 3, 4, 5, 9, 0], [10, -1]),
+        wq.WQ_OPT_GEMV_ROWS_SHAPE: ([0, 1, 2, 3, 4, 0], [5, -1]),
         wq.WQ_OPT_PDL: ([0, 1], [2]),
         wq.WQ_OPT_TC_STAGES: ([0, 2, 5, 16], [1, 17, -1]),
         wq.WQ_OPT_GEMV_GRID: ([1, 0], [2, -1]),

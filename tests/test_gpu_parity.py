@@ -321,7 +321,7 @@ def rows_shape(wq):
 
 
 @pytest.mark.parametrize("variant", ["int", "half"])
-@pytest.mark.parametrize("shape", [1, 2, 3, 4, 5, 6, 7, 8, 9])
+@pytest.mark.parametrize("shape", [1, 2, 3, 4])
 @pytest.mark.parametrize("M", [1, 2])
 @pytest.mark.parametrize("NK", [(333, 1152), (1000, 4096), (17, 11008), (130, 16384), (4099, 256)])
 def test_gemv_rows_shapes(wq, rows_shape, variant, shape, M, NK):
@@ -338,7 +338,7 @@ def test_gemv_rows_shapes(wq, rows_shape, variant, shape, M, NK):
     assert_close(run_gemm(wq, X, qg, N, 4), O.gemm_ref(X, codes, st, z, 128))
 
 
-@pytest.mark.parametrize("shape", [2, 6])
+@pytest.mark.parametrize("shape", [2, 4])
 @pytest.mark.parametrize("NK", [(333, 1152), (4096, 4096), (17, 11008), (4099, 256)])
 def test_gemv_rows_grid_rule0(wq, rows_shape, shape, NK):
     """Grid rule 0 (one CTA per batch, or equal batches per CTA) against the oracle."""

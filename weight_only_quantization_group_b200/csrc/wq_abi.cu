@@ -275,7 +275,7 @@ int32_t wq_set_option(int32_t option, int64_t value) {
       g_opt_pdl = value;
       return WQ_OK;
     case WQ_OPT_GEMV_ROWS_SHAPE:
-      if (value < 0 || value > 9) return WQ_ERR_INVALID_ARG;
+      if (value < 0 || value > 4) return WQ_ERR_INVALID_ARG;
       g_opt_gemv_rows_shape = value;
       return WQ_OK;
     case WQ_OPT_GEMV_GRID:

@@ -420,8 +420,7 @@ static cudaError_t launch_rows_act(const RowsArgs& a, cudaStream_t st, bool pdl,
 }
 
 // shape: rows per batch R, input channels per lane 32*CPL, register stages S
-//   0 = default (6 for K <= 4096, else 2), 1 = (4, 32, 2), 2 = (4, 64, 2), 3 = (8, 32, 2), 4 = (2, 64, 2),
-//   5 = (2, 64, 3), 6 = (4, 32, 3), 7 = (2, 64, 4), 8 = (4, 64, 3), 9 = (4, 32, 4).
+//   0 = default (4 for K <= 4096, else 2), 1 = (4, 32, 2), 2 = (4, 64, 2), 3 = (2, 64, 2), 4 = (4, 32, 3).
 // Shapes with 32 channels per lane take K <= 8192; above that shape 2 runs.
 // act_int: integer digits (true) or fp16 FMA (false) for the lane's dot products.
 template <int M>
@@ -429,13 +428,8 @@ static cudaError_t launch_rows_shape(const RowsArgs& a, cudaStream_t st, bool pd
                                      int gm) {
   switch (shape) {
     case 1: return launch_rows_act<M, 4, 1, 2>(a, st, pdl, act_int, gm);
-    case 3: return launch_rows_act<M, 8, 1, 2>(a, st, pdl, act_int, gm);
-    case 4: return launch_rows_act<M, 2, 2, 2>(a, st, pdl, act_int, gm);
-    case 5: return launch_rows_act<M, 2, 2, 3>(a, st, pdl, act_int, gm);
-    case 6: return launch_rows_act<M, 4, 1, 3>(a, st, pdl, act_int, gm);
-    case 7: return launch_rows_act<M, 2, 2, 4>(a, st, pdl, act_int, gm);
-    case 8: return launch_rows_act<M, 4, 2, 3>(a, st, pdl, act_int, gm);
-    case 9: return launch_rows_act<M, 4, 1, 4>(a, st, pdl, act_int, gm);
+    case 3: return launch_rows_act<M, 2, 2, 2>(a, st, pdl, act_int, gm);
+    case 4: return launch_rows_act<M, 4, 1, 3>(a, st, pdl, act_int, gm);
     default: return launch_rows_act<M, 4, 2, 2>(a, st, pdl, act_int, gm);
   }
 }
@@ -451,8 +445,8 @@ cudaError_t launch_gemv_rows(const void* X, const uint32_t* packed, const void* 
   a.Y = static_cast<__half*>(Y);
   a.N = (int)N;
   a.K = (int)K;
-  if (shape == 0) shape = K <= 4096 ? 6 : 2;  // measured fastest on 4096- and 8192/11008-channel rows
-  if (K > 8192 && (shape == 1 || shape == 3 || shape == 6 || shape == 9)) shape = 2;  // at most 8 warps
+  if (shape == 0) shape = K <= 4096 ? 4 : 2;  // measured fastest on 4096- and 8192/11008-channel rows
+  if (K > 8192 && (shape == 1 || shape == 4)) shape = 2;  // at most 8 warps
   return M == 1 ? launch_rows_shape<1>(a, st, pdl, act_int, shape, grid_mode)
                 : launch_rows_shape<2>(a, st, pdl, act_int, shape, grid_mode);
 }
