@@ -55,23 +55,34 @@ struct RowsStage {
   __half sc[R], zh[R];
 };
 
+// Loads of one row batch for this lane: pw / ps / pz point at the lane's words,
+// step and zero in the batch's first row; nrows = rows of the batch inside N
+// (0 for a lane past K). Full batches take the unpredicated path.
 template <int R, int CPL>
-__device__ __forceinline__ void rows_issue(RowsStage<R, CPL>& s, const RowsArgs& a, int row0, bool active,
-                                           size_t row_words, int G, int lane_word, int lane_group) {
-  const uint32_t* pw = a.P + (size_t)row0 * row_words + lane_word;
-  const size_t sg = (size_t)row0 * G + lane_group;
+__device__ __forceinline__ void rows_issue(RowsStage<R, CPL>& s, const uint32_t* pw, const __half* ps,
+                                           const __half* pz, size_t row_words, int G, int nrows) {
+  if (nrows >= R) {
 #pragma unroll
-  for (int r = 0; r < R; ++r) {
-    if (active && row0 + r < a.N) {
+    for (int r = 0; r < R; ++r) {
 #pragma unroll
       for (int c = 0; c < CPL; ++c) s.w[r][c] = ld_stream_v4(pw + r * row_words + 4 * c);
-      s.sc[r] = a.steps[sg + (size_t)r * G];
-      s.zh[r] = a.zeros[sg + (size_t)r * G];
-    } else {
+      s.sc[r] = ps[(size_t)r * G];
+      s.zh[r] = pz[(size_t)r * G];
+    }
+  } else {
 #pragma unroll
-      for (int c = 0; c < CPL; ++c) s.w[r][c] = make_uint4(0, 0, 0, 0);
-      s.sc[r] = __float2half(0.f);
-      s.zh[r] = __float2half(0.f);
+    for (int r = 0; r < R; ++r) {
+      if (r < nrows) {
+#pragma unroll
+        for (int c = 0; c < CPL; ++c) s.w[r][c] = ld_stream_v4(pw + r * row_words + 4 * c);
+        s.sc[r] = ps[(size_t)r * G];
+        s.zh[r] = pz[(size_t)r * G];
+      } else {
+#pragma unroll
+        for (int c = 0; c < CPL; ++c) s.w[r][c] = make_uint4(0, 0, 0, 0);
+        s.sc[r] = __float2half(0.f);
+        s.zh[r] = __float2half(0.f);
+      }
     }
   }
 }
@@ -311,10 +322,16 @@ gemv_rows_kernel(RowsArgs a) {
   // S register stages: batches i+1 .. i+S-1 are in flight while batch i is
   // computed. The first S-1 are requested before the dependent-launch wait.
   RowsStage<R, CPL> st[S];
+  auto issue = [&](RowsStage<R, CPL>& stage, int j) {  // local batch j of this CTA
+    const int row0 = (blockIdx.x + j * gridDim.x) * R;
+    const int left = a.N - row0;
+    const size_t sg = (size_t)row0 * G + lane_group;
+    rows_issue<R, CPL>(stage, a.P + (size_t)row0 * row_words + lane_word, a.steps + sg, a.zeros + sg, row_words, G,
+                       active ? (left < R ? left : R) : 0);
+  };
 #pragma unroll
   for (int j = 0; j < S - 1; ++j)
-    if (j < my)
-      rows_issue<R, CPL>(st[j], a, (blockIdx.x + j * gridDim.x) * R, active, row_words, G, lane_word, lane_group);
+    if (j < my) issue(st[j], j);
   asm volatile("griddepcontrol.wait;" ::: "memory");
 
   Act<M, CPL> act;
@@ -353,9 +370,7 @@ gemv_rows_kernel(RowsArgs a) {
     for (int j = 0; j < S; ++j) {
       if (i + j < my) {
         const int nx = i + j + S - 1;
-        if (nx < my)
-          rows_issue<R, CPL>(st[(j + S - 1) % S], a, (blockIdx.x + nx * gridDim.x) * R, active, row_words, G,
-                             lane_word, lane_group);
+        if (nx < my) issue(st[(j + S - 1) % S], nx);
         act.template compute<R>(st[j], acc);
         finish();
       }
