@@ -483,17 +483,21 @@ def measure_rows(wq, torch, synth, dev, block, peaks):
             wq.wq_set_option(wq.WQ_OPT_GEMV_GRID, 1)
     for M in synth.SMALLM_SWEEP:
         gemv_row(f"smallm_M{M}_8192x28672_w4", 28672, 8192, 4, big.W, synth.smallm_activations(M), M=M)
-    # tensor-core kernel ring depth (0 = library choice)
-    for M in (16, 64, 128):
-        for S in (0, 2, 3, 4, 5, 6):
+    # tensor-core kernel: dequantizing warps, channels per stage, ring depth (0 = library choice)
+    for M in (4, 16, 64, 128):
+        for dw, bk, S in ((8, 128, 0), (4, 128, 0), (4, 128, 5), (4, 64, 0), (8, 64, 5), (8, 128, 5)):
             wq.wq_set_option(wq.WQ_OPT_TC_STAGES, S)
+            wq.wq_set_option(wq.WQ_OPT_TC_BK, bk)
+            wq.wq_set_option(wq.WQ_OPT_TC_DEQUANT_WARPS, dw)
+            name = f"smallm_M{M}_8192x28672_w4_tc_dw{dw}_bk{bk}_s{S}"
             try:
-                gemv_row(f"smallm_M{M}_8192x28672_w4_tc_s{S}", 28672, 8192, 4, big.W, synth.smallm_activations(M),
-                         M=M)
+                gemv_row(name, 28672, 8192, 4, big.W, synth.smallm_activations(M), M=M)
             except wq.WQError as e:
-                rows[f"smallm_M{M}_8192x28672_w4_tc_s{S}"] = {"error": str(e)}
+                rows[name] = {"error": str(e)}
             finally:
                 wq.wq_set_option(wq.WQ_OPT_TC_STAGES, 0)
+                wq.wq_set_option(wq.WQ_OPT_TC_BK, 0)
+                wq.wq_set_option(wq.WQ_OPT_TC_DEQUANT_WARPS, 0)
     # the other kernel on each side of the crossover, for the record
     for M in (2, 3, 4, 8, 16):
         path = wq.WQ_PATH_TENSOR_CORE if M < 3 else wq.WQ_PATH_GEMV

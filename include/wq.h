@@ -236,6 +236,11 @@ int32_t wq_awq_scale_search_noalloc(const void* X_dev, int64_t T, int64_t K, con
  *                       0 default (library choice), 2..16 that depth (two CTAs
  *                       per SM when it fits; the call fails with WQ_ERR_CUDA
  *                       when one CTA's shared memory cannot hold it).
+ *  WQ_OPT_TC_BK         input channels per stage of the tensor-core kernel: 0
+ *                       default (64 when M rounded up to 16 is at least 96,
+ *                       else 128), 64 or 128.
+ *  WQ_OPT_TC_DEQUANT_WARPS  warps that dequantize in the tensor-core kernel:
+ *                       0 default (4), 4 or 8.
  * wq_set_option returns WQ_ERR_INVALID_ARG for an unknown option or value;
  * wq_get_option returns the current value, or -1 for an unknown option. */
 #define WQ_OPT_GEMM_PATH 1
@@ -254,6 +259,8 @@ int32_t wq_awq_scale_search_noalloc(const void* X_dev, int64_t T, int64_t K, con
 #define WQ_OPT_PDL 7
 #define WQ_OPT_TC_STAGES 9
 #define WQ_OPT_GEMV_GRID 10
+#define WQ_OPT_TC_BK 11
+#define WQ_OPT_TC_DEQUANT_WARPS 12
 int32_t wq_set_option(int32_t option, int64_t value);
 int64_t wq_get_option(int32_t option);
 

@@ -95,6 +95,8 @@ def test_option_values_are_validated(wq):
         wq.WQ_OPT_PDL: ([0, 1], [2]),
         wq.WQ_OPT_TC_STAGES: ([0, 2, 5, 16], [1, 17, -1]),
         wq.WQ_OPT_GEMV_GRID: ([1, 0], [2, -1]),
+        wq.WQ_OPT_TC_BK: ([64, 128, 0], [32, 1, -1]),
+        wq.WQ_OPT_TC_DEQUANT_WARPS: ([4, 8, 0], [2, 6, -1]),
     }
     for opt, (good, bad) in cases.items():
         old = wq.wq_get_option(opt)

@@ -267,13 +267,38 @@ def test_tc_gemm_ring_depths(wq, tc_path, S, M):
     (codes, st, z), qg = assert_quant_parity(wq, W, None, 4, False)
     wq.wq_set_option(wq.WQ_OPT_TC_STAGES, S)
     try:
-        if S * (2 * ((M + 15) // 16 * 16) * 128 + 8192) + 2048 > 220 * 1024:
+        BN = (M + 15) // 16 * 16
+        BK = 64 if BN >= 96 else 128
+        if S * ((BK // 64) * BN * 128 + 128 * BK // 2) + 2048 > 220 * 1024:
             with pytest.raises(wq.WQError):
                 run_gemm(wq, X, qg, N, 4)
             return
         Y = run_gemm(wq, X, qg, N, 4)
     finally:
         wq.wq_set_option(wq.WQ_OPT_TC_STAGES, 0)
+    assert_close(Y, O.gemm_ref(X, codes, st, z, 128))
+
+
+@pytest.mark.parametrize("dw", [4, 8])
+@pytest.mark.parametrize("bk", [64, 128])
+@pytest.mark.parametrize("M", [3, 16, 100, 128, 200, 300])
+@pytest.mark.parametrize("NK", [(333, 1152), (1000, 4096)])
+def test_tc_gemm_stage_width(wq, tc_path, dw, bk, M, NK):
+    """Both stage widths (half a group and a whole group per stage) and both
+    dequantizing-warp counts at every tile width, including two M chunks
+    (M = 300)."""
+    N, K = NK
+    g = synth.rng(700 + M + bk)
+    W = synth.weight(g, N, K, 0.02, channel_frac=0.01, channel_mult=10.0)
+    X = synth.activations(g, M, K, channel_frac=0.01, channel_mult=20.0)
+    (codes, st, z), qg = assert_quant_parity(wq, W, None, 4, False)
+    wq.wq_set_option(wq.WQ_OPT_TC_BK, bk)
+    wq.wq_set_option(wq.WQ_OPT_TC_DEQUANT_WARPS, dw)
+    try:
+        Y = run_gemm(wq, X, qg, N, 4)
+    finally:
+        wq.wq_set_option(wq.WQ_OPT_TC_BK, 0)
+        wq.wq_set_option(wq.WQ_OPT_TC_DEQUANT_WARPS, 0)
     assert_close(Y, O.gemm_ref(X, codes, st, z, 128))
 
 

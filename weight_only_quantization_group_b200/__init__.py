@@ -79,6 +79,8 @@ WQ_OPT_GEMV_ROWS_SHAPE = 6
 WQ_OPT_PDL = 7
 WQ_OPT_TC_STAGES = 9
 WQ_OPT_GEMV_GRID = 10
+WQ_OPT_TC_BK = 11
+WQ_OPT_TC_DEQUANT_WARPS = 12
 
 
 class WQError(RuntimeError):

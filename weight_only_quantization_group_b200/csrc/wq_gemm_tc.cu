@@ -9,16 +9,18 @@
 // Tile: one CTA owns 128 output channels n and all M rows of X ("swap AB":
 // the dequantized weight tile is the 128-row A operand, held in tensor
 // memory; X is the B operand with N_mma = M rounded up to 16; D = W X^T lives
-// in tensor memory as [128 lanes = n][M columns]). K advances in stages of one
-// quantization group (128 input channels):
-//   warp 0    TMA producer into a ring of NS shared-memory stages: the packed
-//             tile (128 rows x 64 bytes, 64-byte swizzle) and the X tile (two
-//             128-byte-swizzled 64-channel boxes)
-//   warp 1    TMEM owner and single-thread tcgen05.mma issuer (8 MMAs/stage)
-//   warps 2-9 dequantize the packed tile into one of two tensor-memory A
-//             buffers (warp w: output channels 32*(w%4)..+31 -- the TMEM lane
-//             quarter it may access -- and half of the group's channels), then
-//             run the epilogue (tcgen05.ld -> fp16 -> Y).
+// in tensor memory as [128 lanes = n][M columns]). K advances in stages of
+// BK = 128 (one quantization group) or 64 input channels:
+//   warp 0    TMA producer into a ring of S shared-memory stages: the packed
+//             tile (128 rows x BK/2 bytes, 64- or 32-byte swizzle) and the X
+//             tile (BK/64 128-byte-swizzled 64-channel boxes)
+//   warp 1    TMEM owner and single-thread tcgen05.mma issuer (BK/16 MMAs
+//             per stage)
+//   warps 2.. 4 (default) or 8 warps dequantize the packed tile into one of
+//             two tensor-memory A buffers (warp w: output channels
+//             32*(w%4)..+31 -- the TMEM lane quarter it may access -- and all
+//             or half of the stage's channels), then run the epilogue
+//             (tcgen05.ld -> fp16 -> Y).
 // The shared-memory ring and the TMEM A ring are separate, so the TMA runs as
 // far ahead as shared memory allows while only two A buffers occupy TMEM.
 // Every mbarrier wait is bounded; on a timeout the kernel latches
@@ -29,13 +31,8 @@ namespace wq {
 
 using namespace sm100;
 
-constexpr int kTcThreads = 320;          // 2 control warps + 8 dequant warps
-constexpr int kTcDequantThreads = 256;
-constexpr int kTcBK = 128;               // input channels per stage (= one group)
 constexpr int kTcRows = 128;             // output channels per CTA
-constexpr int kTcPackedStage = kTcRows * kTcBK / 2;  // 8192 bytes
 constexpr int kTcABufs = 2;              // TMEM A buffers
-constexpr int kTcACols = kTcBK / 2;      // 64 TMEM columns per A buffer
 constexpr long long kSpinLimitCycles = 4000000000LL;  // ~2 s at 2 GHz
 
 struct TcArgs {
@@ -70,14 +67,25 @@ __device__ __forceinline__ uint4 dequant_word4(uint32_t w, __half2 zz, __half2 z
   return r;
 }
 
-__global__ void __launch_bounds__(kTcThreads, 1)
+// BK: input channels per stage, 128 (one group) or 64 (half a group; shallower
+// shared-memory stages, so a deeper ring fits when M is large).
+// NH: dequantizing warp quartets; each of the NH owns 1/NH of a stage's words
+// of every row (more warps hide more latency, fewer amortize the per-stage
+// waits over more weights).
+template <int BK, int NH>
+__global__ void __launch_bounds__(64 + 128 * NH, 1)
 w4a16_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmP,
                      TcArgs a) {
+  constexpr int kPackedStage = kTcRows * BK / 2;  // bytes of the packed tile
+  constexpr int kACols = BK / 2;                  // TMEM columns per A buffer
+  constexpr int kXBoxes = BK / 64;                // 64-channel X boxes per stage
+  constexpr int kWords = BK / 8 / NH;             // packed words per dequant thread and stage
+  constexpr int kChunks = kWords / 4;             // 16-byte chunks per dequant thread and stage
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int S = a.stages;
   const int xbox = a.BN * 128;                       // one 64-channel X box
-  const int stage_bytes = 2 * xbox + kTcPackedStage;  // X (two boxes) + packed
+  const int stage_bytes = kXBoxes * xbox + kPackedStage;  // X boxes + packed
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + (size_t)S * stage_bytes);
   uint64_t* sempty = full + S;
   uint64_t* afull = sempty + S;
@@ -87,12 +95,12 @@ w4a16_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   auto stageX = [&](int s) { return smem + (size_t)s * stage_bytes; };
-  auto stageP = [&](int s) { return smem + (size_t)s * stage_bytes + 2 * xbox; };
+  auto stageP = [&](int s) { return smem + (size_t)s * stage_bytes + kXBoxes * xbox; };
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int n0 = blockIdx.x * kTcRows;
-  const int KT = a.K / kTcBK;  // stages == groups
+  const int KT = a.K / BK;
   const int G = a.K / kGroup;
 
   if (threadIdx.x == 0) {
@@ -101,7 +109,7 @@ w4a16_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
       mbar_init(&sempty[s], 1);
     }
     for (int b = 0; b < kTcABufs; ++b) {
-      mbar_init(&afull[b], kTcDequantThreads);
+      mbar_init(&afull[b], 128 * NH);
       mbar_init(&aempty[b], 1);
     }
     mbar_init(accum, 1);
@@ -128,9 +136,9 @@ w4a16_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
         if (*abort_flag) break;
         if (u > 0 && !mbar_wait(&sempty[s], (u - 1) & 1, a.err, kSpinLimitCycles)) { *abort_flag = 1; break; }
         mbar_arrive_expect_tx(&full[s], (uint32_t)stage_bytes);
-        tma_load_2d(stageX(s), &tmX, kt * kTcBK, 0, &full[s]);
-        tma_load_2d(stageX(s) + xbox, &tmX, kt * kTcBK + 64, 0, &full[s]);
-        tma_load_2d(stageP(s), &tmP, kt * (kTcBK / 8), n0, &full[s]);
+#pragma unroll
+        for (int i = 0; i < kXBoxes; ++i) tma_load_2d(stageX(s) + i * xbox, &tmX, kt * BK + 64 * i, 0, &full[s]);
+        tma_load_2d(stageP(s), &tmP, kt * (BK / 8), n0, &full[s]);
         issued = kt + 1;
         if (++s == S) { s = 0; ++u; }
       }
@@ -149,9 +157,9 @@ w4a16_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
         tc_fence_after();
         const uint32_t xaddr = smem_u32(stageX(s));
 #pragma unroll
-        for (int j = 0; j < kTcBK / 16; ++j) {
+        for (int j = 0; j < BK / 16; ++j) {
           const uint64_t bd = desc_kmajor_sw128(xaddr + (uint32_t)((j >> 2) * xbox + (j & 3) * 32));
-          mma_f16_ts(tmem, tmem_a + (uint32_t)(b * kTcACols + 8 * j), bd, idesc, (kt > 0 || j > 0) ? 1u : 0u);
+          mma_f16_ts(tmem, tmem_a + (uint32_t)(b * kACols + 8 * j), bd, idesc, (kt > 0 || j > 0) ? 1u : 0u);
         }
         mma_commit(&aempty[b]);
         mma_commit(&sempty[s]);
@@ -166,11 +174,13 @@ w4a16_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
   } else {
     // ---------------------------------------------------------- dequant + epilogue
     const int q = warp & 3;             // TMEM lane quarter this warp may access
-    const int h = (warp - 2) >> 2;      // which half of the group's 16 packed words
+    const int h = (warp - 2) >> 2;      // which 1/NH of the stage's packed words of a row
     const int r = 32 * q + lane;        // output channel within the tile
     const int n = n0 + r;
     const bool row_ok = n < a.N;
-    // step and zero of the next group, fetched a stage ahead of their use
+    // step and zero of the current group, and of the next one, fetched a
+    // group ahead of their use
+    __half st_cur = __float2half(0.f), zr_cur = __float2half(0.f);
     __half st_next = __float2half(0.f), zr_next = __float2half(0.f);
     if (row_ok) {
       st_next = a.steps[(size_t)n * G];
@@ -178,37 +188,45 @@ w4a16_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
     }
     // Software pipeline: stage kt is dequantized into registers while the
     // tensor-memory stores of stage kt-1 complete; then kt-1 is published to
-    // the MMA issuer and kt's stores are issued.
-    uint32_t v0[16], v1[16];
+    // the MMA issuer and kt's stores are issued (tcgen05.st reads its source
+    // registers when it issues, so they need no copy).
     int pend_b = -1;  // A buffer whose stores are in flight (-1: none)
     for (int kt = 0, s = 0, u = 0, b = 0, ub = 0; kt < KT; ++kt) {
       if (__any_sync(0xffffffffu, *abort_flag != 0)) break;
-      const __half st = st_next, zr = zr_next;
-      if (row_ok && kt + 1 < G) {
-        st_next = a.steps[(size_t)n * G + kt + 1];
-        zr_next = a.zeros[(size_t)n * G + kt + 1];
+      const int g = (kt * BK) / kGroup;
+      if ((kt * BK) % kGroup == 0) {  // a new group starts: take its prefetched scales, fetch the next
+        st_cur = st_next;
+        zr_cur = zr_next;
+        if (row_ok && g + 1 < G) {
+          st_next = a.steps[(size_t)n * G + g + 1];
+          zr_next = a.zeros[(size_t)n * G + g + 1];
+        }
       }
-      const __half2 s2 = __halves2half2(st, st);
-      const __half z1024 = __hadd(zr, __float2half(1024.f));
-      const __half z64n = __hneg(__hadd(zr, __float2half(64.f)));
+      const __half2 s2 = __halves2half2(st_cur, st_cur);
+      const __half z1024 = __hadd(zr_cur, __float2half(1024.f));
+      const __half z64n = __hneg(__hadd(zr_cur, __float2half(64.f)));
       const __half2 zz = __halves2half2(z1024, z1024);
       const __half2 zz16n = __halves2half2(z64n, z64n);
       const bool landed = mbar_wait(&full[s], u & 1, a.err, kSpinLimitCycles);
       if (!__all_sync(0xffffffffu, landed)) { *abort_flag = 1; break; }
-      // the packed tile is 64-byte swizzled: 16-byte chunk c of row r sits at
-      // chunk c ^ ((r >> 1) & 3), which keeps a warp's loads conflict-free
-      const uint8_t* prow = stageP(s) + r * 64;
-      const int sw = (r >> 1) & 3;
-      const uint4 wa = *reinterpret_cast<const uint4*>(prow + (((2 * h) ^ sw) << 4));
-      const uint4 wb = *reinterpret_cast<const uint4*>(prow + (((2 * h + 1) ^ sw) << 4));
-      const uint32_t words[8] = {wa.x, wa.y, wa.z, wa.w, wb.x, wb.y, wb.z, wb.w};
-      uint32_t n0v[16], n1v[16];
+      // The packed tile is swizzled by the TMA: with 64-byte rows (BK = 128)
+      // 16-byte chunk c of row r sits at chunk c ^ ((r >> 1) & 3), with
+      // 32-byte rows (BK = 64) at c ^ ((r >> 2) & 1); both keep a warp's loads
+      // conflict-free.
+      uint32_t words[kWords];
+      const uint8_t* prow = stageP(s) + r * (BK / 2);
+      const int sw = BK == 128 ? (r >> 1) & 3 : (r >> 2) & 1;
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
+      for (int i = 0; i < kChunks; ++i) {
+        const uint4 v = *reinterpret_cast<const uint4*>(prow + (((h * kChunks + i) ^ sw) << 4));
+        words[4 * i] = v.x; words[4 * i + 1] = v.y; words[4 * i + 2] = v.z; words[4 * i + 3] = v.w;
+      }
+      uint32_t nv[kWords / 4][16];
+#pragma unroll
+      for (int j = 0; j < kWords; ++j) {
         const uint4 d = dequant_word4(words[j], zz, zz16n, s2);
-        n0v[4 * j] = d.x; n0v[4 * j + 1] = d.y; n0v[4 * j + 2] = d.z; n0v[4 * j + 3] = d.w;
-        const uint4 e = dequant_word4(words[4 + j], zz, zz16n, s2);
-        n1v[4 * j] = e.x; n1v[4 * j + 1] = e.y; n1v[4 * j + 2] = e.z; n1v[4 * j + 3] = e.w;
+        nv[j >> 2][4 * (j & 3)] = d.x; nv[j >> 2][4 * (j & 3) + 1] = d.y;
+        nv[j >> 2][4 * (j & 3) + 2] = d.z; nv[j >> 2][4 * (j & 3) + 3] = d.w;
       }
       if (pend_b >= 0) {  // publish the previous stage
         tmem_st_wait();
@@ -218,11 +236,9 @@ w4a16_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
       bool ok = true;
       if (kt >= kTcABufs) ok = mbar_wait(&aempty[b], (ub - 1) & 1, a.err, kSpinLimitCycles);
       if (!__all_sync(0xffffffffu, ok)) { *abort_flag = 1; break; }
+      const uint32_t ta = tmem_a + ((uint32_t)(32 * q) << 16) + (uint32_t)(b * kACols + (kACols / NH) * h);
 #pragma unroll
-      for (int i = 0; i < 16; ++i) { v0[i] = n0v[i]; v1[i] = n1v[i]; }
-      const uint32_t ta = tmem_a + ((uint32_t)(32 * q) << 16) + (uint32_t)(b * kTcACols + 32 * h);
-      tmem_st16(ta, v0);
-      tmem_st16(ta + 16, v1);
+      for (int i = 0; i < kWords / 4; ++i) tmem_st16(ta + 16 * i, nv[i]);
       pend_b = b;
       if (++s == S) { s = 0; ++u; }
       if (++b == kTcABufs) { b = 0; ++ub; }
@@ -232,13 +248,13 @@ w4a16_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
       tc_fence_before();
       mbar_arrive(&afull[pend_b]);
     }
-    // Epilogue: D[n][m] from TMEM -> Y[m][n]; the two halves take alternate
-    // 16-column chunks.
+    // Epilogue: D[n][m] from TMEM -> Y[m][n]; the NH warp quartets take
+    // alternate 16-column chunks.
     bool done = !__any_sync(0xffffffffu, *abort_flag != 0);
     if (done) done = __all_sync(0xffffffffu, mbar_wait(accum, 0, a.err, kSpinLimitCycles));
     if (done) {
       tc_fence_after();
-      for (int c0 = 16 * h; c0 < a.BN; c0 += 32) {
+      for (int c0 = 16 * h; c0 < a.BN; c0 += 16 * NH) {
         uint32_t v[16];
         tmem_ld16(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)c0, v);
         tmem_ld_wait();
@@ -291,13 +307,19 @@ static uint32_t pow2_cols(uint32_t c) {
 
 // stages_opt: 0 = library choice; otherwise the shared-memory ring depth (two
 // CTAs per SM when that ring and the tile's TMEM fit half an SM).
+// bk_opt: 0 = library choice, else 64 or 128 input channels per stage.
+// dw_opt: 0 = library choice (4), else 4 or 8 dequantizing warps.
 cudaError_t launch_gemm_tc(const void* X, const uint32_t* packed, const void* steps, const void* zeros, int64_t M,
-                           int64_t N, int64_t K, void* Y, int* err, cudaStream_t st, int stages_opt) {
+                           int64_t N, int64_t K, void* Y, int* err, cudaStream_t st, int stages_opt, int bk_opt,
+                           int dw_opt) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return cudaErrorNotSupported;
   for (int64_t m0 = 0; m0 < M; m0 += 256) {
     const int mc = (int)((M - m0) < 256 ? (M - m0) : 256);
     const int BN = ((mc + 15) / 16) * 16;
+    // Half-group stages for wide X tiles (BN >= 96: a 5-deep ring still fits
+    // two CTAs per SM), whole-group stages otherwise (fewer waits per weight).
+    const int BK = bk_opt != 0 ? bk_opt : (BN >= 96 ? 64 : 128);
     CUtensorMap tmX, tmP;
     {
       cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)mc};
@@ -313,11 +335,11 @@ cudaError_t launch_gemm_tc(const void* X, const uint32_t* packed, const void* st
     {
       cuuint64_t dims[2] = {(cuuint64_t)(K / 8), (cuuint64_t)N};
       cuuint64_t strides[1] = {(cuuint64_t)(K / 2)};
-      cuuint32_t box[2] = {16, 128};
+      cuuint32_t box[2] = {(cuuint32_t)(BK / 8), 128};
       cuuint32_t es[2] = {1, 1};
       if (enc(&tmP, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<uint32_t*>(packed), dims, strides, box, es,
-              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+              CU_TENSOR_MAP_INTERLEAVE_NONE, BK == 128 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
         return cudaErrorInvalidValue;
     }
     TcArgs a;
@@ -328,11 +350,11 @@ cudaError_t launch_gemm_tc(const void* X, const uint32_t* packed, const void* st
     a.N = (int)N;
     a.K = (int)K;
     a.BN = BN;
-    a.tmem_cols = pow2_cols((uint32_t)(BN + kTcABufs * kTcACols));
+    a.tmem_cols = pow2_cols((uint32_t)(BN + kTcABufs * BK / 2));
     // Two CTAs per SM when the tile's TMEM fits half of it and half the shared
     // memory still holds a ring of three stages; otherwise one CTA per SM with
     // the deepest ring that fits.
-    const int stage = 2 * BN * 128 + kTcPackedStage;
+    const int stage = (BK / 64) * BN * 128 + kTcRows * BK / 2;
     const size_t half_budget = 110 * 1024, full_budget = 220 * 1024;
     int S;
     if (stages_opt > 0) {
@@ -350,11 +372,13 @@ cudaError_t launch_gemm_tc(const void* X, const uint32_t* packed, const void* st
     // Never more CTAs on an SM than its 512 TMEM columns can hold at once.
     const size_t smem_floor = a.tmem_cols > 256 ? 120 * 1024 : 80 * 1024;
     if (smem < smem_floor) smem = smem_floor;
-    auto kern = w4a16_gemm_tc_kernel;
+    const int NH = dw_opt == 8 ? 2 : 1;  // 4 dequantizing warps unless asked for 8
+    auto kern = BK == 128 ? (NH == 1 ? w4a16_gemm_tc_kernel<128, 1> : w4a16_gemm_tc_kernel<128, 2>)
+                          : (NH == 1 ? w4a16_gemm_tc_kernel<64, 1> : w4a16_gemm_tc_kernel<64, 2>);
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     const dim3 grid((unsigned)((N + kTcRows - 1) / kTcRows));
-    kern<<<grid, kTcThreads, smem, st>>>(tmX, tmP, a);
+    kern<<<grid, 64 + 128 * NH, smem, st>>>(tmX, tmP, a);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
