@@ -67,6 +67,14 @@ struct LinearSet {
   int n_total;                      // row_off[n_lin]
 };
 
+// 1/x to within one ulp (x a normal fp32: the AWQ scales are at least
+// (2^-14)^0.95); the products it feeds are rounded to fp16.
+__device__ __forceinline__ float rcp_approx(float x) {
+  float r;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+  return r;
+}
+
 template <int BITS, bool SYM>
 __global__ void __launch_bounds__(256)
 awq_error_kernel(LinearSet ls, int K, const __half* __restrict__ S, int alpha0, __half* __restrict__ E) {
@@ -123,7 +131,7 @@ awq_error_kernel(LinearSet ls, int K, const __half* __restrict__ S, int alpha0, 
     for (int u = 0; u < 2; ++u) {
       const int q = group_quant_code<BITS, SYM>(w[i + u], gq);
       const float deq = __fmul_rn((float)(q - gq.zero), gq.sf);  // exact
-      e2[u] = x[i + u] - deq * __frcp_rn(sv[i + u]);
+      e2[u] = x[i + u] - deq * rcp_approx(sv[i + u]);  // E is rounded to fp16 next
     }
     const __half2 hv = __floats2half2_rn(e2[0], e2[1]);
     out[i / 2] = *reinterpret_cast<const uint32_t*>(&hv);

@@ -8,10 +8,10 @@
 // Optional AWQ input-channel scaling W * diag(s) first ("MIT 6.5940 Lab 4 +
 // Lab 5", "Question 2").
 //
-// Mapping: 16 lanes per group, each lane owns 8 consecutive input channels
-// (one 16-byte load of W); group_quant_decide() reduces the group's range with
-// four xor-shuffles inside the half warp. The kernel is HBM-bound: 2 B/weight
-// in, 0.5 (0.375) B/weight out.
+// Mapping: 4 lanes per group, each lane owns 32 consecutive input channels
+// (four 16-byte loads of W; one 16-byte store of 4-bit codes, or the three
+// words of a 3-bit chunk); group_quant_decide() reduces the group's range
+// with two xor-shuffles. 2 B/weight in, 0.5 (0.375) B/weight out.
 #include "wq_quant_core.cuh"
 
 namespace wq {
@@ -21,81 +21,80 @@ __global__ void __launch_bounds__(256)
 quantize_pack_kernel(const __half* __restrict__ W, const __half* __restrict__ s, int64_t N, int64_t K,
                      uint32_t* __restrict__ packed, __half* __restrict__ steps,
                      __half* __restrict__ zeros, int* err) {
-  __shared__ __align__(16) uint8_t code_buf[8][256];  // 3-bit: per-warp code staging
   const int lane = threadIdx.x & 31;
-  const int warp = threadIdx.x >> 5;
-  const int sub = lane & 15;  // lane within the group
+  const int sub = lane & 3;  // lane within the group
   const int64_t G = K / kGroup;
-  const int64_t gidx = ((int64_t)blockIdx.x * 8 + warp) * 2 + (lane >> 4);
+  const int64_t gidx = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 2;
   const bool valid = gidx < N * G;
   const int64_t n = valid ? gidx / G : 0;
   const int64_t gi = valid ? gidx % G : 0;
-  const int64_t k0 = gi * kGroup + sub * 8;
+  const int64_t k0 = gi * kGroup + sub * 32;
 
-  float w[8];
-  {
+  float w[32];
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
     uint4 raw = make_uint4(0, 0, 0, 0);
-    if (valid) raw = *reinterpret_cast<const uint4*>(W + n * K + k0);
+    if (valid) raw = *reinterpret_cast<const uint4*>(W + n * K + k0 + 8 * c);
     const __half2* h = reinterpret_cast<const __half2*>(&raw);
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      float2 f = __half22float2(h[i]);
-      w[2 * i] = f.x;
-      w[2 * i + 1] = f.y;
+      const float2 f = __half22float2(h[i]);
+      w[8 * c + 2 * i] = f.x;
+      w[8 * c + 2 * i + 1] = f.y;
     }
     if (HAS_S) {
       uint4 sraw = make_uint4(0, 0, 0, 0);
-      if (valid) sraw = *reinterpret_cast<const uint4*>(s + k0);
+      if (valid) sraw = *reinterpret_cast<const uint4*>(s + k0 + 8 * c);
       const __half2* sh = reinterpret_cast<const __half2*>(&sraw);
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
-        float2 f = __half22float2(sh[i]);
-        w[2 * i] = __fmul_rn(w[2 * i], f.x);  // exact: 11 x 11 significand bits
-        w[2 * i + 1] = __fmul_rn(w[2 * i + 1], f.y);
+        const float2 f = __half22float2(sh[i]);
+        w[8 * c + 2 * i] = __fmul_rn(w[8 * c + 2 * i], f.x);  // exact: 11 x 11 significand bits
+        w[8 * c + 2 * i + 1] = __fmul_rn(w[8 * c + 2 * i + 1], f.y);
       }
     }
   }
 
-  const GroupQuant gq = group_quant_decide<BITS, SYM>(w);
+  const GroupQuant gq = group_quant_decide<BITS, SYM, 32, 4>(w);
   if (valid && sub == 0) {
     if (!isfinite(gq.sf)) latch_error(err, WQ_ERR_RANGE);
     steps[n * G + gi] = gq.step_h;
     zeros[n * G + gi] = __int2half_rn(gq.zero);
   }
-  int q[8];
+  uint32_t q[32];
 #pragma unroll
-  for (int i = 0; i < 8; ++i) q[i] = group_quant_code<BITS, SYM>(w[i], gq);
+  for (int i = 0; i < 32; ++i) q[i] = (uint32_t)group_quant_code<BITS, SYM>(w[i], gq);
+  if (!valid) return;
 
   if (BITS == 4) {
-    if (valid) {
-      const uint32_t word = (uint32_t)q[0] | ((uint32_t)q[2] << 4) | ((uint32_t)q[4] << 8) |
-                            ((uint32_t)q[6] << 12) | ((uint32_t)q[1] << 16) | ((uint32_t)q[3] << 20) |
-                            ((uint32_t)q[5] << 24) | ((uint32_t)q[7] << 28);
-      packed[(n * K + k0) / 8] = word;
+    // word c holds channels 8c..8c+7 in slot order [0, 2, 4, 6, 1, 3, 5, 7]
+    uint4 out;
+    uint32_t* o = reinterpret_cast<uint32_t*>(&out);
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      const uint32_t* v = q + 8 * c;
+      o[c] = v[0] | (v[2] << 4) | (v[4] << 8) | (v[6] << 12) | (v[1] << 16) | (v[3] << 20) | (v[5] << 24) |
+             (v[7] << 28);
     }
+    *reinterpret_cast<uint4*>(packed + (n * K + k0) / 8) = out;
   } else {
-    // Stage the 8 codes, then 3 lanes of each 4-lane quad assemble the three
-    // words of the quad's 32 input channels.
-    uint8_t* buf = code_buf[warp];
-    uint2 c8;
-    c8.x = (uint32_t)q[0] | ((uint32_t)q[1] << 8) | ((uint32_t)q[2] << 16) | ((uint32_t)q[3] << 24);
-    c8.y = (uint32_t)q[4] | ((uint32_t)q[5] << 8) | ((uint32_t)q[6] << 16) | ((uint32_t)q[7] << 24);
-    *reinterpret_cast<uint2*>(buf + lane * 8) = c8;
-    __syncwarp();
-    const int t = lane & 3;
-    if (valid && t < 3) {
-      const uint8_t* c = buf + (lane >> 2) * 32;
+    // the lane's 32 channels are one 3-word chunk: word t holds channel pairs
+    // (10t + 2j, 10t + 2j + 1) at bits 3j and 16 + 3j, and bit t of channels
+    // 30 / 31 at bit 15 / 31
+    uint32_t o[3];
+#pragma unroll
+    for (int t = 0; t < 3; ++t) {
       uint32_t word = 0;
 #pragma unroll
-      for (int j = 0; j < 5; ++j) {
-        word |= (uint32_t)c[10 * t + 2 * j] << (3 * j);
-        word |= (uint32_t)c[10 * t + 2 * j + 1] << (16 + 3 * j);
-      }
-      word |= (uint32_t)((c[30] >> t) & 1) << 15;
-      word |= (uint32_t)((c[31] >> t) & 1) << 31;
-      const int64_t chunk = (n * K + gi * kGroup + (sub >> 2) * 32) / 32;
-      packed[chunk * 3 + t] = word;
+      for (int j = 0; j < 5; ++j) word |= (q[10 * t + 2 * j] << (3 * j)) | (q[10 * t + 2 * j + 1] << (16 + 3 * j));
+      word |= ((q[30] >> t) & 1u) << 15;
+      word |= ((q[31] >> t) & 1u) << 31;
+      o[t] = word;
     }
+    uint32_t* dst = packed + (n * K + k0) / 32 * 3;
+    dst[0] = o[0];
+    dst[1] = o[1];
+    dst[2] = o[2];
   }
 }
 
@@ -147,7 +146,7 @@ unpack_dequant_kernel(const uint32_t* __restrict__ packed, const __half* __restr
 cudaError_t launch_quantize_pack(const void* W, const void* s, int64_t N, int64_t K, int bits, bool sym,
                                  uint32_t* packed, void* steps, void* zeros, int* err, cudaStream_t st) {
   const int64_t groups = N * (K / kGroup);
-  const dim3 grid((unsigned)((groups + 15) / 16));
+  const dim3 grid((unsigned)((groups + 63) / 64));  // 4 lanes per group
   const dim3 block(256);
   auto Wp = static_cast<const __half*>(W);
   auto sp = static_cast<const __half*>(s);
