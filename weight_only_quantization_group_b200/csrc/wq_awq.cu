@@ -78,16 +78,15 @@ __device__ __forceinline__ float rcp_approx(float x) {
 template <int BITS, bool SYM>
 __global__ void __launch_bounds__(256)
 awq_error_kernel(LinearSet ls, int K, const __half* __restrict__ S, int alpha0, __half* __restrict__ E) {
-  const int lane = threadIdx.x & 31;
-  const int warp = threadIdx.x >> 5;
-  const int sub = lane & 15;
+  // 4 lanes per group, 32 consecutive input channels per lane.
+  const int sub = threadIdx.x & 3;
   const int N = ls.n_total;
   const int G = K / kGroup;
-  const int64_t gidx = ((int64_t)blockIdx.x * 8 + warp) * 2 + (lane >> 4);
+  const int64_t gidx = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 2;
   const bool valid = gidx < (int64_t)N * G;
   const int n = valid ? (int)(gidx / G) : 0;
   const int gi = valid ? (int)(gidx % G) : 0;
-  const int k0 = gi * kGroup + sub * 8;
+  const int k0 = gi * kGroup + sub * 32;
   const int b = blockIdx.y;
   // Which stacked linear owns row n (unrolled so the parameter arrays stay in
   // the constant bank).
@@ -101,43 +100,47 @@ awq_error_kernel(LinearSet ls, int K, const __half* __restrict__ S, int alpha0, 
     }
   const __half* s = S + (size_t)(alpha0 + b) * K;
 
-  float w[8], x[8], sv[8];
-  {
-    uint4 raw = make_uint4(0, 0, 0, 0), sraw = make_uint4(0x3C003C00u, 0x3C003C00u, 0x3C003C00u, 0x3C003C00u);
+  uint4 xraw[4], sraw[4];
+  float w[32];
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    xraw[c] = make_uint4(0, 0, 0, 0);
+    sraw[c] = make_uint4(0x3C003C00u, 0x3C003C00u, 0x3C003C00u, 0x3C003C00u);  // s = 1 off the end
     if (valid) {
-      raw = *reinterpret_cast<const uint4*>(Wrow + (size_t)(n - roff) * K + k0);
-      sraw = *reinterpret_cast<const uint4*>(s + k0);
+      xraw[c] = *reinterpret_cast<const uint4*>(Wrow + (size_t)(n - roff) * K + k0 + 8 * c);
+      sraw[c] = *reinterpret_cast<const uint4*>(s + k0 + 8 * c);
     }
-    const __half2* h = reinterpret_cast<const __half2*>(&raw);
-    const __half2* sh = reinterpret_cast<const __half2*>(&sraw);
+    const __half2* h = reinterpret_cast<const __half2*>(&xraw[c]);
+    const __half2* sh = reinterpret_cast<const __half2*>(&sraw[c]);
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       const float2 f = __half22float2(h[i]);
       const float2 g = __half22float2(sh[i]);
-      x[2 * i] = f.x;
-      x[2 * i + 1] = f.y;
-      sv[2 * i] = g.x;
-      sv[2 * i + 1] = g.y;
-      w[2 * i] = __fmul_rn(f.x, g.x);  // exact
-      w[2 * i + 1] = __fmul_rn(f.y, g.y);
+      w[8 * c + 2 * i] = __fmul_rn(f.x, g.x);  // exact
+      w[8 * c + 2 * i + 1] = __fmul_rn(f.y, g.y);
     }
   }
-  const GroupQuant gq = group_quant_decide<BITS, SYM>(w);
-  uint32_t out[4];
+  const GroupQuant gq = group_quant_decide<BITS, SYM, 32, 4>(w);
 #pragma unroll
-  for (int i = 0; i < 8; i += 2) {
-    float e2[2];
+  for (int c = 0; c < 4; ++c) {
+    const __half2* h = reinterpret_cast<const __half2*>(&xraw[c]);
+    const __half2* sh = reinterpret_cast<const __half2*>(&sraw[c]);
+    uint32_t out[4];
 #pragma unroll
-    for (int u = 0; u < 2; ++u) {
-      const int q = group_quant_code<BITS, SYM>(w[i + u], gq);
-      const float deq = __fmul_rn((float)(q - gq.zero), gq.sf);  // exact
-      e2[u] = x[i + u] - deq * rcp_approx(sv[i + u]);  // E is rounded to fp16 next
+    for (int i = 0; i < 4; ++i) {
+      const float2 f = __half22float2(h[i]);
+      const float2 g = __half22float2(sh[i]);
+      const int q0 = group_quant_code<BITS, SYM>(w[8 * c + 2 * i], gq);
+      const int q1 = group_quant_code<BITS, SYM>(w[8 * c + 2 * i + 1], gq);
+      const float d0 = __fmul_rn((float)(q0 - gq.zero), gq.sf);  // exact
+      const float d1 = __fmul_rn((float)(q1 - gq.zero), gq.sf);
+      // E is rounded to fp16 next, so an approximate 1/s is enough
+      const __half2 hv = __floats2half2_rn(f.x - d0 * rcp_approx(g.x), f.y - d1 * rcp_approx(g.y));
+      out[i] = *reinterpret_cast<const uint32_t*>(&hv);
     }
-    const __half2 hv = __floats2half2_rn(e2[0], e2[1]);
-    out[i / 2] = *reinterpret_cast<const uint32_t*>(&hv);
+    if (valid)
+      *reinterpret_cast<uint4*>(E + ((size_t)b * N + n) * K + k0 + 8 * c) = make_uint4(out[0], out[1], out[2], out[3]);
   }
-  if (valid)
-    *reinterpret_cast<uint4*>(E + ((size_t)b * N + n) * K + k0) = make_uint4(out[0], out[1], out[2], out[3]);
 }
 
 // ------------------------------------------------------------------ S4b: loss GEMM
@@ -402,7 +405,7 @@ cudaError_t launch_awq_search(const void* X, int64_t T, int64_t K, const void* c
 
   for (int a0 = 0; a0 < n_alpha; a0 += p.batch) {
     const int B = (n_alpha - a0) < p.batch ? (n_alpha - a0) : p.batch;
-    const dim3 eg((unsigned)((groups + 15) / 16), (unsigned)B);
+    const dim3 eg((unsigned)((groups + 63) / 64), (unsigned)B);  // 4 lanes per group
 #define WQ_AE(BI, SY) awq_error_kernel<BI, SY><<<eg, 256, 0, st>>>(ls, (int)K, S, a0, E)
     if (bits == 4) { if (sym) WQ_AE(4, true); else WQ_AE(4, false); }
     else { if (sym) WQ_AE(3, true); else WQ_AE(3, false); }
@@ -536,7 +539,7 @@ cudaError_t launch_awq_search_noalloc(const void* X, int64_t T, int64_t K, const
       lc.n_lin = nl;
       lc.n_total = (int)(r1 - r0);
       const int64_t groups = (r1 - r0) * (K / kGroup);
-      const dim3 eg((unsigned)((groups + 15) / 16), 1u);
+      const dim3 eg((unsigned)((groups + 63) / 64), 1u);
 #define WQ_AE(BI, SY) awq_error_kernel<BI, SY><<<eg, 256, 0, st>>>(lc, (int)K, S, j, E)
       if (bits == 4) { if (sym) WQ_AE(4, true); else WQ_AE(4, false); }
       else { if (sym) WQ_AE(3, true); else WQ_AE(3, false); }
