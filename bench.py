@@ -445,9 +445,13 @@ def measure_rows(wq, torch, synth, dev, block, peaks):
     for bits in (4, 3):
         c = synth.config_llama65b_decode(bits)
         gemv_row(f"gemv_llama65b_8192x8192_w{bits}", 8192, 8192, bits, c.W, c.X)
+        if bits == 3:  # 3-bit rows with two rows per batch
+            wq.wq_set_option(wq.WQ_OPT_GEMV_ROWS_SHAPE, 3)
+            try:
+                gemv_row("gemv_llama65b_8192x8192_w3_rows_r2", 8192, 8192, bits, c.W, c.X)
+            finally:
+                wq.wq_set_option(wq.WQ_OPT_GEMV_ROWS_SHAPE, 0)
         for tag, var in (("tiled", wq.WQ_GEMV_OFFSET_SUMS), ("tiled_exact", wq.WQ_GEMV_EXACT)):
-            if bits == 3 and tag == "tiled":
-                continue  # 3-bit always runs the tiled kernel
             wq.wq_set_option(wq.WQ_OPT_GEMV_KERNEL, wq.WQ_GEMV_KERNEL_TILED)
             wq.wq_set_option(wq.WQ_OPT_GEMV_VARIANT, var)
             try:

@@ -214,8 +214,9 @@ int32_t wq_awq_scale_search_noalloc(const void* X_dev, int64_t T, int64_t K, con
  *                       wq_quantize_pack writes them;
  *                       WQ_GEMV_EXACT subtracts the zero point in fp16 first,
  *                       so every product is exact (tiled kernel only).
- *  WQ_OPT_GEMV_KERNEL   WQ_GEMV_KERNEL_AUTO (default): for 4-bit, M <= 2,
- *                       K <= 16384 and not WQ_GEMV_EXACT, the row-streaming kernel
+ *  WQ_OPT_GEMV_KERNEL   WQ_GEMV_KERNEL_AUTO (default): for M <= 2, K <= 16384
+ *                       and not WQ_GEMV_EXACT, the row-streaming kernel (3-bit
+ *                       rows always with offset sums)
  *                       (activations held in registers, warps split K);
  *                       otherwise the tiled kernel (activations in shared
  *                       memory, warps split rows, cluster split-K).

@@ -202,6 +202,29 @@ def test_gemv_closed_forms(wq, gemv_variant):
     assert abs(Y[0, n] - ref[0, n]) <= bound[0, n] + 2 ** -11 * abs(ref[0, n])
 
 
+@pytest.mark.parametrize("bits", [3, 4])
+def test_gemv_every_channel_position(wq, gemv_variant, bits):
+    """Row n holds one code away from its zero point, at channel
+    (n mod 32) + 224 (n div 32): every position of a 32-channel packing unit
+    (and several units and groups) must map back to its own activation, so
+    Y[n] = x_k (q - zero) step up to the kernel's rounding bound."""
+    N, K = 64, 1024
+    g = np.random.default_rng(31 + bits)
+    Q = (1 << bits) - 1
+    X = synth.activations(synth.rng(32), 1, K)
+    zeros = g.integers(0, Q + 1, (N, K // 128)).astype(np.float16)
+    steps = g.uniform(0.001, 0.1, (N, K // 128)).astype(np.float16)
+    codes = np.repeat(zeros.astype(np.uint8), 128, axis=1)
+    for n in range(N):
+        k = (n % 32) + 224 * (n // 32)
+        codes[n, k] = (int(zeros[n, k // 128]) + 1 + n % Q) % (Q + 1)
+    packed = dev(O.pack_codes(codes, bits).reshape(-1).view(np.int32))
+    Y = run_gemm(wq, X, (packed, dev(steps), dev(zeros)), N, bits).astype(np.float64)
+    ref = O.gemm_ref(X, codes, steps, zeros, 128)
+    bound = _gemv_error_bound(X, steps)
+    assert np.all(np.abs(Y - ref) <= bound + 2 ** -11 * np.abs(ref)), np.max(np.abs(Y - ref) - bound)
+
+
 def test_gemv_small_linear(wq):
     c = synth.config_small_linear(0)
     (codes, st, z), qg = assert_quant_parity(wq, c.W, None, 4, False)
@@ -345,22 +368,24 @@ def rows_shape(wq):
     wq.wq_set_option(wq.WQ_OPT_GEMV_VARIANT, wq.WQ_GEMV_OFFSET_SUMS)
 
 
+@pytest.mark.parametrize("bits", [3, 4])
 @pytest.mark.parametrize("variant", ["int", "half"])
 @pytest.mark.parametrize("shape", [1, 2, 3, 4])
 @pytest.mark.parametrize("M", [1, 2])
 @pytest.mark.parametrize("NK", [(333, 1152), (1000, 4096), (17, 11008), (130, 16384), (4099, 256)])
-def test_gemv_rows_shapes(wq, rows_shape, variant, shape, M, NK):
+def test_gemv_rows_shapes(wq, rows_shape, bits, variant, shape, M, NK):
     """Every (rows per batch, channels per lane, register stages) shape of the
-    row-streaming kernel with both ways of forming the lane sums; ragged N,
+    row-streaming kernel with both ways of forming the lane sums, at 4 and 3
+    bits (3-bit rows run shapes 2 and 3 with offset sums); ragged N,
     inactive lanes (K = 256 leaves most lanes of the single warp idle), K up
     to 16384, and CTAs with fewer row batches than stages (N = 17)."""
     N, K = NK
     g = synth.rng(800 + shape + M)
     W = synth.weight(g, N, K, 0.02, channel_frac=0.01, channel_mult=10.0)
     X = synth.activations(g, M, K, channel_frac=0.01, channel_mult=20.0)
-    (codes, st, z), qg = assert_quant_parity(wq, W, None, 4, False)
+    (codes, st, z), qg = assert_quant_parity(wq, W, None, bits, False)
     rows_shape(shape, wq.WQ_GEMV_INT_DIGITS if variant == "int" else wq.WQ_GEMV_OFFSET_SUMS)
-    assert_close(run_gemm(wq, X, qg, N, 4), O.gemm_ref(X, codes, st, z, 128))
+    assert_close(run_gemm(wq, X, qg, N, bits), O.gemm_ref(X, codes, st, z, 128))
 
 
 @pytest.mark.parametrize("shape", [2, 4])

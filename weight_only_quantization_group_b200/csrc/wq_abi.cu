@@ -15,8 +15,8 @@ cudaError_t launch_gemv(const void* X, const uint32_t* packed, const void* steps
 size_t gemv_smem_bytes(int bits, int variant, int M, int N, int K);
 bool gemv_rows_supported(int bits, int64_t M, int64_t K);
 cudaError_t launch_gemv_rows(const void* X, const uint32_t* packed, const void* steps, const void* zeros, int64_t M,
-                             int64_t N, int64_t K, void* Y, cudaStream_t st, int shape, bool act_int, int grid_mode,
-                             bool pdl);
+                             int64_t N, int64_t K, int bits, void* Y, cudaStream_t st, int shape, bool act_int,
+                             int grid_mode, bool pdl);
 cudaError_t launch_gemm_tc(const void* X, const uint32_t* packed, const void* steps, const void* zeros, int64_t M,
                            int64_t N, int64_t K, void* Y, int* err, cudaStream_t st, int stages_opt, int bk_opt,
                            int dw_opt);
@@ -175,7 +175,8 @@ int32_t wq_w4a16_gemm(const void* X, const uint32_t* packed, const void* steps, 
   }
   if (g_opt_gemv_kernel != WQ_GEMV_KERNEL_TILED && g_opt_gemv_variant != WQ_GEMV_EXACT &&
       wq::gemv_rows_supported(cfg->bits, M, K))
-    return cuda_status(wq::launch_gemv_rows(X, packed, steps, zeros, M, N, K, Y, static_cast<cudaStream_t>(stream),
+    return cuda_status(wq::launch_gemv_rows(X, packed, steps, zeros, M, N, K, cfg->bits, Y,
+                                            static_cast<cudaStream_t>(stream),
                                             (int)g_opt_gemv_rows_shape, g_opt_gemv_variant == WQ_GEMV_INT_DIGITS,
                                             (int)g_opt_gemv_grid, g_opt_pdl != 0));
   // The shared copy of an X slice must fit one CTA.

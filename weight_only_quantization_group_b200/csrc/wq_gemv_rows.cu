@@ -1,4 +1,4 @@
-// S5 for M <= 2 (4-bit): row-streaming decode GEMV with activations in registers.
+// S5 for M <= 2 (4- and 3-bit): row-streaming decode GEMV with activations in registers.
 //
 // The decode GEMV streams the packed weight once ("MIT 6.5940 Lab 4 + Lab 5",
 // "Starting point and setup"; "CMU 11-868 L19-L20", "where does the speed
@@ -49,23 +49,48 @@ struct RowsArgs {
   int N, K;
 };
 
-template <int R, int CPL>
+// One row batch of this lane: WPR packed words per row (4-bit: 4 per 32
+// channels, 3-bit: 3 per 32 channels) and the rows' step and zero.
+template <int R, int WPR>
 struct RowsStage {
-  uint4 w[R][CPL];
+  uint32_t w[R][WPR];
   __half sc[R], zh[R];
 };
+
+__device__ __forceinline__ uint2 ld_stream_v2(const void* p) {
+  uint2 r;
+  asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0,%1}, [%2];" : "=r"(r.x), "=r"(r.y) : "l"(p));
+  return r;
+}
+
+template <int WPR>
+__device__ __forceinline__ void load_row_words(uint32_t (&w)[WPR], const uint32_t* p) {
+  if constexpr (WPR % 4 == 0) {
+#pragma unroll
+    for (int c = 0; c < WPR / 4; ++c) {
+      const uint4 v = ld_stream_v4(p + 4 * c);
+      w[4 * c] = v.x; w[4 * c + 1] = v.y; w[4 * c + 2] = v.z; w[4 * c + 3] = v.w;
+    }
+  } else {
+    static_assert(WPR % 2 == 0, "row words come in 8-byte pairs");
+#pragma unroll
+    for (int c = 0; c < WPR / 2; ++c) {
+      const uint2 v = ld_stream_v2(p + 2 * c);
+      w[2 * c] = v.x; w[2 * c + 1] = v.y;
+    }
+  }
+}
 
 // Loads of one row batch for this lane: pw / ps / pz point at the lane's words,
 // step and zero in the batch's first row; nrows = rows of the batch inside N
 // (0 for a lane past K). Full batches take the unpredicated path.
-template <int R, int CPL>
-__device__ __forceinline__ void rows_issue(RowsStage<R, CPL>& s, const uint32_t* pw, const __half* ps,
+template <int R, int WPR>
+__device__ __forceinline__ void rows_issue(RowsStage<R, WPR>& s, const uint32_t* pw, const __half* ps,
                                            const __half* pz, size_t row_words, int G, int nrows) {
   if (nrows >= R) {
 #pragma unroll
     for (int r = 0; r < R; ++r) {
-#pragma unroll
-      for (int c = 0; c < CPL; ++c) s.w[r][c] = ld_stream_v4(pw + r * row_words + 4 * c);
+      load_row_words<WPR>(s.w[r], pw + r * row_words);
       s.sc[r] = ps[(size_t)r * G];
       s.zh[r] = pz[(size_t)r * G];
     }
@@ -73,13 +98,12 @@ __device__ __forceinline__ void rows_issue(RowsStage<R, CPL>& s, const uint32_t*
 #pragma unroll
     for (int r = 0; r < R; ++r) {
       if (r < nrows) {
-#pragma unroll
-        for (int c = 0; c < CPL; ++c) s.w[r][c] = ld_stream_v4(pw + r * row_words + 4 * c);
+        load_row_words<WPR>(s.w[r], pw + r * row_words);
         s.sc[r] = ps[(size_t)r * G];
         s.zh[r] = pz[(size_t)r * G];
       } else {
 #pragma unroll
-        for (int c = 0; c < CPL; ++c) s.w[r][c] = make_uint4(0, 0, 0, 0);
+        for (int c = 0; c < WPR; ++c) s.w[r][c] = 0;
         s.sc[r] = __float2half(0.f);
         s.zh[r] = __float2half(0.f);
       }
@@ -87,11 +111,6 @@ __device__ __forceinline__ void rows_issue(RowsStage<R, CPL>& s, const uint32_t*
   }
 }
 
-template <int CPL>
-__device__ __forceinline__ uint32_t stage_word(const uint4 (&w)[CPL], int j) {
-  const uint4 wv = w[j >> 2];
-  return (j & 3) == 0 ? wv.x : (j & 3) == 1 ? wv.y : (j & 3) == 2 ? wv.z : wv.w;
-}
 
 // The lane's LK = 32*CPL activations of each of the M rows of X.
 template <int M, int CPL>
@@ -130,7 +149,7 @@ struct ActHalf {
   }
 
   template <int R>
-  __device__ __forceinline__ void compute(const RowsStage<R, CPL>& s, float (&acc)[R * M]) const {
+  __device__ __forceinline__ void compute(const RowsStage<R, 4 * CPL>& s, float (&acc)[R * M]) const {
 #pragma unroll
     for (int r = 0; r < R; ++r) {
       float a[M][4];
@@ -138,7 +157,7 @@ struct ActHalf {
       for (int m = 0; m < M; ++m) a[m][0] = a[m][1] = a[m][2] = a[m][3] = 0.f;
 #pragma unroll
       for (int j = 0; j < 4 * CPL; ++j) {
-        const uint32_t w = stage_word<CPL>(s.w[r], j);
+        const uint32_t w = s.w[r][j];
         const uint32_t w8 = w >> 8;
         const uint32_t p0 = and_or(w, 0x000F000Fu, kHalf2Magic);   // k+0,k+1   x1
         const uint32_t p1 = and_or(w, 0x00F000F0u, kHalf2Magic);   // k+2,k+3   x16
@@ -158,6 +177,89 @@ struct ActHalf {
       for (int m = 0; m < M; ++m) {
         // sum_k x (q - z) = A1 + A2/16 - (1024 X1 + 64 X2) - z (X1 + X2)
         float t = fmaf(a[m][2] + a[m][3], 0.0625f, a[m][0] + a[m][1]) - c1[m];
+        t = fmaf(-z, xsum[m], t);
+        acc[r * M + m] = sc * t;
+      }
+    }
+  }
+};
+
+// ---------------------------------------------------------------- ActHalf3
+// 3-bit rows: per 32 channels three words; word t holds the channel pairs
+// (10t + 2j, 10t + 2j + 1) at bits 3j and 16 + 3j (j < 5), and bit t of
+// channels 30 / 31 at bit 15 / 31. A LOP3 with 0x6400 leaves pair j of a word
+// as (1024 + q, 1024 + q') times 1 (j = 0), 8 (j = 1) or 64 (j = 2); after a
+// 9-bit shift pairs 3 and 4 follow as x1 and x8. Three shifted LOP3s gather
+// the bits of channels 30 and 31. The offsets and the zero point are removed
+// per row with the lane's activation class sums, as in ActHalf.
+template <int M, int CPL>
+struct ActHalf3 {
+  uint32_t xh[M][16 * CPL];
+  float c1[M], xsum[M];
+
+  __device__ __forceinline__ void load(const RowsArgs& a, int k0, bool active) {
+    load_lane_x<M, CPL>(xh, a, k0, active);
+#pragma unroll
+    for (int m = 0; m < M; ++m) {
+      float x1 = 0.f, x8 = 0.f, x64 = 0.f;
+#pragma unroll
+      for (int i = 0; i < 16 * CPL; ++i) {
+        const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&xh[m][i]));
+        const int wi = i & 15;  // x word within the 32-channel chunk
+        const int j = wi % 5;
+        if (wi == 15 || j == 0 || j == 3) x1 += f.x + f.y;
+        else if (j == 2) x64 += f.x + f.y;
+        else x8 += f.x + f.y;
+      }
+      c1[m] = 1024.f * x1 + 128.f * x8 + 16.f * x64;
+      xsum[m] = x1 + x8 + x64;
+    }
+  }
+
+  template <int R>
+  __device__ __forceinline__ void compute(const RowsStage<R, 3 * CPL>& s, float (&acc)[R * M]) const {
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      float a[M][6];  // (x1, x8, x64) classes, low and high lanes
+#pragma unroll
+      for (int m = 0; m < M; ++m)
+#pragma unroll
+        for (int i = 0; i < 6; ++i) a[m][i] = 0.f;
+#pragma unroll
+      for (int c = 0; c < CPL; ++c) {
+        const uint32_t w0 = s.w[r][3 * c], w1 = s.w[r][3 * c + 1], w2 = s.w[r][3 * c + 2];
+        const uint32_t wt[3] = {w0, w1, w2};
+#pragma unroll
+        for (int t = 0; t < 3; ++t) {
+          const uint32_t w = wt[t];
+          const uint32_t w9 = w >> 9;
+          const uint32_t p0 = and_or(w, 0x00070007u, kHalf2Magic);   // x1
+          const uint32_t p1 = and_or(w, 0x00380038u, kHalf2Magic);   // x8
+          const uint32_t p2 = and_or(w, 0x01C001C0u, kHalf2Magic);   // x64
+          const uint32_t p3 = and_or(w9, 0x00070007u, kHalf2Magic);  // x1
+          const uint32_t p4 = and_or(w9, 0x00380038u, kHalf2Magic);  // x8
+          const int xw = 16 * c + 5 * t;
+#pragma unroll
+          for (int m = 0; m < M; ++m) {
+            fma2_f16_f32(a[m][0], a[m][1], xh[m][xw + 0], p0);
+            fma2_f16_f32(a[m][2], a[m][3], xh[m][xw + 1], p1);
+            fma2_f16_f32(a[m][4], a[m][5], xh[m][xw + 2], p2);
+            fma2_f16_f32(a[m][0], a[m][1], xh[m][xw + 3], p3);
+            fma2_f16_f32(a[m][2], a[m][3], xh[m][xw + 4], p4);
+          }
+        }
+        uint32_t p30 = and_or(w0 >> 15, 0x00010001u, kHalf2Magic);
+        p30 = and_or(w1 >> 14, 0x00020002u, p30);
+        p30 = and_or(w2 >> 13, 0x00040004u, p30);
+#pragma unroll
+        for (int m = 0; m < M; ++m) fma2_f16_f32(a[m][0], a[m][1], xh[m][16 * c + 15], p30);
+      }
+      const float sc = __half2float(s.sc[r]);
+      const float z = __half2float(s.zh[r]);
+#pragma unroll
+      for (int m = 0; m < M; ++m) {
+        // sum_k x (q - z) = A1 + A8/8 + A64/64 - (1024 X1 + 128 X8 + 16 X64) - z (X1 + X8 + X64)
+        float t = fmaf(a[m][4] + a[m][5], 0.015625f, fmaf(a[m][2] + a[m][3], 0.125f, a[m][0] + a[m][1])) - c1[m];
         t = fmaf(-z, xsum[m], t);
         acc[r * M + m] = sc * t;
       }
@@ -235,7 +337,7 @@ struct ActInt {
   }
 
   template <int R>
-  __device__ __forceinline__ void compute(const RowsStage<R, CPL>& s, float (&acc)[R * M]) const {
+  __device__ __forceinline__ void compute(const RowsStage<R, 4 * CPL>& s, float (&acc)[R * M]) const {
     // Words outer, rows inner: R*M*3 independent dp4a chains.
     int a[R][M][3];
 #pragma unroll
@@ -246,7 +348,7 @@ struct ActInt {
     for (int j = 0; j < 4 * CPL; ++j) {
 #pragma unroll
       for (int r = 0; r < R; ++r) {
-        const uint32_t w = stage_word<CPL>(s.w[r], j);
+        const uint32_t w = s.w[r][j];
         const uint32_t l16 = (w << 4) & 0xF0F0F0F0u;  // 16 q of channels 0, 4, 1, 5
         const uint32_t h16 = w & 0xF0F0F0F0u;         // 16 q of channels 2, 6, 3, 7
 #pragma unroll
@@ -301,9 +403,10 @@ __device__ __forceinline__ float butterfly_reduce(float (&v)[NV], int lane, int&
 }
 
 // At most 8 warps: K <= 8192 with 32 channels per lane, K <= 16384 with 64.
-template <int M, int R, int CPL, int S, template <int, int> class Act>
+template <int M, int R, int CPL, int S, int BITS, template <int, int> class Act>
 __global__ void __launch_bounds__(256)
 gemv_rows_kernel(RowsArgs a) {
+  constexpr int WPR = BITS * CPL;  // packed words per row and lane
   constexpr int NV = R * M;
   constexpr int LK = 32 * CPL;  // input channels per lane
   extern __shared__ __align__(16) float red[];  // [2][32 / NV][nseg][NV]
@@ -313,20 +416,20 @@ gemv_rows_kernel(RowsArgs a) {
   const int k0 = warp * 32 * LK + lane * LK;  // this lane's first input channel
   const bool active = k0 < a.K;
   const int G = a.K / kGroup;
-  const size_t row_words = (size_t)a.K / 8;
-  const int lane_word = k0 / 8;
+  const size_t row_words = (size_t)a.K * BITS / 32;
+  const int lane_word = k0 * BITS / 32;
   const int lane_group = k0 / kGroup;
   const int nbatch = (a.N + R - 1) / R;
   const int my = blockIdx.x < nbatch ? (nbatch - 1 - blockIdx.x) / gridDim.x + 1 : 0;
 
   // S register stages: batches i+1 .. i+S-1 are in flight while batch i is
   // computed. The first S-1 are requested before the dependent-launch wait.
-  RowsStage<R, CPL> st[S];
-  auto issue = [&](RowsStage<R, CPL>& stage, int j) {  // local batch j of this CTA
+  RowsStage<R, WPR> st[S];
+  auto issue = [&](RowsStage<R, WPR>& stage, int j) {  // local batch j of this CTA
     const int row0 = (blockIdx.x + j * gridDim.x) * R;
     const int left = a.N - row0;
     const size_t sg = (size_t)row0 * G + lane_group;
-    rows_issue<R, CPL>(stage, a.P + (size_t)row0 * row_words + lane_word, a.steps + sg, a.zeros + sg, row_words, G,
+    rows_issue<R, WPR>(stage, a.P + (size_t)row0 * row_words + lane_word, a.steps + sg, a.zeros + sg, row_words, G,
                        active ? (left < R ? left : R) : 0);
   };
 #pragma unroll
@@ -390,7 +493,7 @@ static int rows_num_sms() {
   return sms;
 }
 
-bool gemv_rows_supported(int bits, int64_t M, int64_t K) { return bits == 4 && M <= 2 && K <= 16384; }
+bool gemv_rows_supported(int bits, int64_t M, int64_t K) { return (bits == 4 || bits == 3) && M <= 2 && K <= 16384; }
 
 // Persistent grid, all CTAs resident; CTA c takes row batches c, c + grid, ...
 //   mode 0: small problems take one CTA per row batch (most loads in flight
@@ -404,9 +507,9 @@ static long rows_grid(long nbatch, int occ, int mode) {
   return (nbatch + per_cta - 1) / per_cta;
 }
 
-template <int M, int R, int CPL, int S, template <int, int> class Act>
+template <int M, int R, int CPL, int S, int BITS, template <int, int> class Act>
 static cudaError_t launch_rows(const RowsArgs& a, cudaStream_t st, bool pdl, int grid_mode) {
-  auto kern = gemv_rows_kernel<M, R, CPL, S, Act>;
+  auto kern = gemv_rows_kernel<M, R, CPL, S, BITS, Act>;
   const int nseg = (a.K + 1024 * CPL - 1) / (1024 * CPL);
   const int threads = 32 * nseg;
   const size_t smem = 2 * (size_t)32 * nseg * sizeof(float);  // [2][32/NV][nseg][NV]
@@ -430,8 +533,8 @@ static cudaError_t launch_rows(const RowsArgs& a, cudaStream_t st, bool pdl, int
 
 template <int M, int R, int CPL, int S>
 static cudaError_t launch_rows_act(const RowsArgs& a, cudaStream_t st, bool pdl, bool act_int, int grid_mode) {
-  return act_int ? launch_rows<M, R, CPL, S, ActInt>(a, st, pdl, grid_mode)
-                 : launch_rows<M, R, CPL, S, ActHalf>(a, st, pdl, grid_mode);
+  return act_int ? launch_rows<M, R, CPL, S, 4, ActInt>(a, st, pdl, grid_mode)
+                 : launch_rows<M, R, CPL, S, 4, ActHalf>(a, st, pdl, grid_mode);
 }
 
 // shape: rows per batch R, input channels per lane 32*CPL, register stages S
@@ -449,9 +552,17 @@ static cudaError_t launch_rows_shape(const RowsArgs& a, cudaStream_t st, bool pd
   }
 }
 
+// 3-bit rows: 64 channels per lane (six words, three 8-byte loads), shape 2
+// or 3, offset sums only.
+template <int M>
+static cudaError_t launch_rows3(const RowsArgs& a, cudaStream_t st, bool pdl, int shape, int gm) {
+  return shape == 3 ? launch_rows<M, 2, 2, 2, 3, ActHalf3>(a, st, pdl, gm)
+                    : launch_rows<M, 4, 2, 2, 3, ActHalf3>(a, st, pdl, gm);
+}
+
 cudaError_t launch_gemv_rows(const void* X, const uint32_t* packed, const void* steps, const void* zeros, int64_t M,
-                             int64_t N, int64_t K, void* Y, cudaStream_t st, int shape, bool act_int, int grid_mode,
-                             bool pdl) {
+                             int64_t N, int64_t K, int bits, void* Y, cudaStream_t st, int shape, bool act_int,
+                             int grid_mode, bool pdl) {
   RowsArgs a;
   a.X = static_cast<const __half*>(X);
   a.P = packed;
@@ -460,6 +571,8 @@ cudaError_t launch_gemv_rows(const void* X, const uint32_t* packed, const void* 
   a.Y = static_cast<__half*>(Y);
   a.N = (int)N;
   a.K = (int)K;
+  if (bits == 3)
+    return M == 1 ? launch_rows3<1>(a, st, pdl, shape, grid_mode) : launch_rows3<2>(a, st, pdl, shape, grid_mode);
   if (shape == 0) shape = K <= 4096 ? 4 : 2;  // measured fastest on 4096- and 8192/11008-channel rows
   if (K > 8192 && (shape == 1 || shape == 4)) shape = 2;  // at most 8 warps
   return M == 1 ? launch_rows_shape<1>(a, st, pdl, act_int, shape, grid_mode)
