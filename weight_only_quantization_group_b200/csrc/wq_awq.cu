@@ -77,8 +77,9 @@ __device__ __forceinline__ float rcp_approx(float x) {
 
 template <int BITS, bool SYM>
 __global__ void __launch_bounds__(256)
-awq_error_kernel(LinearSet ls, int K, const __half* __restrict__ S, int alpha0, __half* __restrict__ E) {
-  // 4 lanes per group, 32 consecutive input channels per lane.
+awq_error_kernel(LinearSet ls, int K, const __half* __restrict__ S, int alpha0, int nb, __half* __restrict__ E) {
+  // 4 lanes per group, 32 consecutive input channels per lane; the lane's W
+  // is read once and its error rows are written for all nb alphas.
   const int sub = threadIdx.x & 3;
   const int N = ls.n_total;
   const int G = K / kGroup;
@@ -87,7 +88,6 @@ awq_error_kernel(LinearSet ls, int K, const __half* __restrict__ S, int alpha0, 
   const int n = valid ? (int)(gidx / G) : 0;
   const int gi = valid ? (int)(gidx % G) : 0;
   const int k0 = gi * kGroup + sub * 32;
-  const int b = blockIdx.y;
   // Which stacked linear owns row n (unrolled so the parameter arrays stay in
   // the constant bank).
   const __half* Wrow = ls.W[0];
@@ -98,48 +98,53 @@ awq_error_kernel(LinearSet ls, int K, const __half* __restrict__ S, int alpha0, 
       Wrow = ls.W[i];
       roff = ls.row_off[i];
     }
-  const __half* s = S + (size_t)(alpha0 + b) * K;
-
-  uint4 xraw[4], sraw[4];
-  float w[32];
+  uint4 xraw[4];
 #pragma unroll
   for (int c = 0; c < 4; ++c) {
     xraw[c] = make_uint4(0, 0, 0, 0);
-    sraw[c] = make_uint4(0x3C003C00u, 0x3C003C00u, 0x3C003C00u, 0x3C003C00u);  // s = 1 off the end
-    if (valid) {
-      xraw[c] = *reinterpret_cast<const uint4*>(Wrow + (size_t)(n - roff) * K + k0 + 8 * c);
-      sraw[c] = *reinterpret_cast<const uint4*>(s + k0 + 8 * c);
-    }
-    const __half2* h = reinterpret_cast<const __half2*>(&xraw[c]);
-    const __half2* sh = reinterpret_cast<const __half2*>(&sraw[c]);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const float2 f = __half22float2(h[i]);
-      const float2 g = __half22float2(sh[i]);
-      w[8 * c + 2 * i] = __fmul_rn(f.x, g.x);  // exact
-      w[8 * c + 2 * i + 1] = __fmul_rn(f.y, g.y);
-    }
+    if (valid) xraw[c] = *reinterpret_cast<const uint4*>(Wrow + (size_t)(n - roff) * K + k0 + 8 * c);
   }
-  const GroupQuant gq = group_quant_decide<BITS, SYM, 32, 4>(w);
+
+  for (int b = 0; b < nb; ++b) {
+    const __half* s = S + (size_t)(alpha0 + b) * K;
+    uint4 sraw[4];
+    float w[32];
 #pragma unroll
-  for (int c = 0; c < 4; ++c) {
-    const __half2* h = reinterpret_cast<const __half2*>(&xraw[c]);
-    const __half2* sh = reinterpret_cast<const __half2*>(&sraw[c]);
-    uint32_t out[4];
+    for (int c = 0; c < 4; ++c) {
+      sraw[c] = make_uint4(0x3C003C00u, 0x3C003C00u, 0x3C003C00u, 0x3C003C00u);  // s = 1 off the end
+      if (valid) sraw[c] = *reinterpret_cast<const uint4*>(s + k0 + 8 * c);
+      const __half2* h = reinterpret_cast<const __half2*>(&xraw[c]);
+      const __half2* sh = reinterpret_cast<const __half2*>(&sraw[c]);
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const float2 f = __half22float2(h[i]);
-      const float2 g = __half22float2(sh[i]);
-      const int q0 = group_quant_code<BITS, SYM>(w[8 * c + 2 * i], gq);
-      const int q1 = group_quant_code<BITS, SYM>(w[8 * c + 2 * i + 1], gq);
-      const float d0 = __fmul_rn((float)(q0 - gq.zero), gq.sf);  // exact
-      const float d1 = __fmul_rn((float)(q1 - gq.zero), gq.sf);
-      // E is rounded to fp16 next, so an approximate 1/s is enough
-      const __half2 hv = __floats2half2_rn(f.x - d0 * rcp_approx(g.x), f.y - d1 * rcp_approx(g.y));
-      out[i] = *reinterpret_cast<const uint32_t*>(&hv);
+      for (int i = 0; i < 4; ++i) {
+        const float2 f = __half22float2(h[i]);
+        const float2 g = __half22float2(sh[i]);
+        w[8 * c + 2 * i] = __fmul_rn(f.x, g.x);  // exact
+        w[8 * c + 2 * i + 1] = __fmul_rn(f.y, g.y);
+      }
     }
-    if (valid)
-      *reinterpret_cast<uint4*>(E + ((size_t)b * N + n) * K + k0 + 8 * c) = make_uint4(out[0], out[1], out[2], out[3]);
+    const GroupQuant gq = group_quant_decide<BITS, SYM, 32, 4>(w);
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      const __half2* h = reinterpret_cast<const __half2*>(&xraw[c]);
+      const __half2* sh = reinterpret_cast<const __half2*>(&sraw[c]);
+      uint32_t out[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float2 f = __half22float2(h[i]);
+        const float2 g = __half22float2(sh[i]);
+        const int q0 = group_quant_code<BITS, SYM>(w[8 * c + 2 * i], gq);
+        const int q1 = group_quant_code<BITS, SYM>(w[8 * c + 2 * i + 1], gq);
+        const float d0 = __fmul_rn((float)(q0 - gq.zero), gq.sf);  // exact
+        const float d1 = __fmul_rn((float)(q1 - gq.zero), gq.sf);
+        // E is rounded to fp16 next, so an approximate 1/s is enough
+        const __half2 hv = __floats2half2_rn(f.x - d0 * rcp_approx(g.x), f.y - d1 * rcp_approx(g.y));
+        out[i] = *reinterpret_cast<const uint32_t*>(&hv);
+      }
+      if (valid)
+        *reinterpret_cast<uint4*>(E + ((size_t)b * N + n) * K + k0 + 8 * c) =
+            make_uint4(out[0], out[1], out[2], out[3]);
+    }
   }
 }
 
@@ -405,8 +410,8 @@ cudaError_t launch_awq_search(const void* X, int64_t T, int64_t K, const void* c
 
   for (int a0 = 0; a0 < n_alpha; a0 += p.batch) {
     const int B = (n_alpha - a0) < p.batch ? (n_alpha - a0) : p.batch;
-    const dim3 eg((unsigned)((groups + 63) / 64), (unsigned)B);  // 4 lanes per group
-#define WQ_AE(BI, SY) awq_error_kernel<BI, SY><<<eg, 256, 0, st>>>(ls, (int)K, S, a0, E)
+    const dim3 eg((unsigned)((groups + 63) / 64));  // 4 lanes per group, all B alphas per thread
+#define WQ_AE(BI, SY) awq_error_kernel<BI, SY><<<eg, 256, 0, st>>>(ls, (int)K, S, a0, B, E)
     if (bits == 4) { if (sym) WQ_AE(4, true); else WQ_AE(4, false); }
     else { if (sym) WQ_AE(3, true); else WQ_AE(3, false); }
 #undef WQ_AE
@@ -540,7 +545,7 @@ cudaError_t launch_awq_search_noalloc(const void* X, int64_t T, int64_t K, const
       lc.n_total = (int)(r1 - r0);
       const int64_t groups = (r1 - r0) * (K / kGroup);
       const dim3 eg((unsigned)((groups + 63) / 64), 1u);
-#define WQ_AE(BI, SY) awq_error_kernel<BI, SY><<<eg, 256, 0, st>>>(lc, (int)K, S, j, E)
+#define WQ_AE(BI, SY) awq_error_kernel<BI, SY><<<eg, 256, 0, st>>>(lc, (int)K, S, j, 1, E)
       if (bits == 4) { if (sym) WQ_AE(4, true); else WQ_AE(4, false); }
       else { if (sym) WQ_AE(3, true); else WQ_AE(3, false); }
 #undef WQ_AE
