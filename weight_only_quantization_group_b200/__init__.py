@@ -144,13 +144,28 @@ class _LazyLib:
 _lib = _LazyLib()
 
 
+_CFG_CACHE: dict = {}
+
+
 def _cfg(bits: int, group_size: int, symmetric: bool) -> _Cfg:
-    return _Cfg(int(bits), int(group_size), 1 if symmetric else 0)
+    """A config struct per (bits, group, symmetric); the library only reads it."""
+    key = (int(bits), int(group_size), bool(symmetric))
+    c = _CFG_CACHE.get(key)
+    if c is None:
+        c = _CFG_CACHE[key] = _Cfg(key[0], key[1], 1 if key[2] else 0)
+    return c
 
 
-def _stream(stream) -> int:
+_raw_stream = getattr(torch._C, "_cuda_getCurrentRawStream", None)
+
+
+def _stream(stream, device=None) -> int:
+    """The caller's stream, or the current stream of `device` (default: the
+    current device) when none is given."""
     if stream is None:
-        return torch.cuda.current_stream().cuda_stream
+        if _raw_stream is not None:
+            return _raw_stream(torch.cuda.current_device() if device is None else device)
+        return torch.cuda.current_stream(device).cuda_stream
     return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
 
 
@@ -239,8 +254,8 @@ def wq_w4a16_gemm(X: torch.Tensor, packed: torch.Tensor, steps: torch.Tensor, ze
     ws_ptr, ws_bytes = None, 0
     if workspace is not None:
         ws_ptr, ws_bytes = workspace.data_ptr(), workspace.numel() * workspace.element_size()
-    st = _lib.wq_w4a16_gemm(_ptr(X), _ptr(packed), _ptr(steps), _ptr(zeros), M, N, K, ctypes.byref(c),
-                            _ptr(out), ws_ptr, ws_bytes, _stream(stream))
+    st = lib().wq_w4a16_gemm(X.data_ptr(), packed.data_ptr(), steps.data_ptr(), zeros.data_ptr(), M, N, K,
+                             ctypes.byref(c), out.data_ptr(), ws_ptr, ws_bytes, _stream(stream, X.device.index))
     _raise(st, "wq_w4a16_gemm")
     return out
 
