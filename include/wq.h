@@ -242,6 +242,14 @@ int32_t wq_awq_scale_search_noalloc(const void* X_dev, int64_t T, int64_t K, con
  *                       else 128), 64 or 128.
  *  WQ_OPT_TC_DEQUANT_WARPS  warps that dequantize in the tensor-core kernel:
  *                       0 default (4), 4 or 8.
+ *  WQ_OPT_WAIT_LIMIT_MS how long a bounded mbarrier wait in the tensor-core
+ *                       kernel may last before it latches WQ_ERR_TIMEOUT
+ *                       (1..60000, default 2000).
+ *  WQ_OPT_TEST_STALL    test hook, 0 (default) or 1: the tensor-core kernel's
+ *                       producer issues no loads, so its consumers' waits run
+ *                       out; the kernel then frees its tensor memory, returns,
+ *                       and wq_get_last_device_error reports WQ_ERR_TIMEOUT.
+ *                       Y is not written. For failure-handling tests only.
  * wq_set_option returns WQ_ERR_INVALID_ARG for an unknown option or value;
  * wq_get_option returns the current value, or -1 for an unknown option. */
 #define WQ_OPT_GEMM_PATH 1
@@ -262,6 +270,8 @@ int32_t wq_awq_scale_search_noalloc(const void* X_dev, int64_t T, int64_t K, con
 #define WQ_OPT_GEMV_GRID 10
 #define WQ_OPT_TC_BK 11
 #define WQ_OPT_TC_DEQUANT_WARPS 12
+#define WQ_OPT_WAIT_LIMIT_MS 13
+#define WQ_OPT_TEST_STALL 14
 int32_t wq_set_option(int32_t option, int64_t value);
 int64_t wq_get_option(int32_t option);
 

@@ -81,6 +81,8 @@ WQ_OPT_TC_STAGES = 9
 WQ_OPT_GEMV_GRID = 10
 WQ_OPT_TC_BK = 11
 WQ_OPT_TC_DEQUANT_WARPS = 12
+WQ_OPT_WAIT_LIMIT_MS = 13
+WQ_OPT_TEST_STALL = 14
 
 
 class WQError(RuntimeError):

@@ -19,7 +19,7 @@ cudaError_t launch_gemv_rows(const void* X, const uint32_t* packed, const void* 
                              int grid_mode, bool pdl);
 cudaError_t launch_gemm_tc(const void* X, const uint32_t* packed, const void* steps, const void* zeros, int64_t M,
                            int64_t N, int64_t K, void* Y, int* err, cudaStream_t st, int stages_opt, int bk_opt,
-                           int dw_opt);
+                           int dw_opt, int wait_ms, bool stall);
 struct AwqPlan {
   int64_t N_total;
   int t_tiles, n_tiles, tiles;
@@ -91,6 +91,8 @@ int64_t g_opt_tc_stages = 0;
 int64_t g_opt_gemv_grid = 1;
 int64_t g_opt_tc_bk = 0;
 int64_t g_opt_tc_dequant_warps = 0;
+int64_t g_opt_wait_limit_ms = 2000;
+int64_t g_opt_test_stall = 0;
 
 }  // namespace
 
@@ -171,7 +173,8 @@ int32_t wq_w4a16_gemm(const void* X, const uint32_t* packed, const void* steps, 
     if (!flag) return WQ_ERR_CUDA;
     return cuda_status(wq::launch_gemm_tc(X, packed, steps, zeros, M, N, K, Y, flag,
                                           static_cast<cudaStream_t>(stream), (int)g_opt_tc_stages,
-                                          (int)g_opt_tc_bk, (int)g_opt_tc_dequant_warps));
+                                          (int)g_opt_tc_bk, (int)g_opt_tc_dequant_warps,
+                                          (int)g_opt_wait_limit_ms, g_opt_test_stall != 0));
   }
   if (g_opt_gemv_kernel != WQ_GEMV_KERNEL_TILED && g_opt_gemv_variant != WQ_GEMV_EXACT &&
       wq::gemv_rows_supported(cfg->bits, M, K))
@@ -283,6 +286,14 @@ int32_t wq_set_option(int32_t option, int64_t value) {
       if (value < 0 || value > 4) return WQ_ERR_INVALID_ARG;
       g_opt_gemv_rows_shape = value;
       return WQ_OK;
+    case WQ_OPT_WAIT_LIMIT_MS:
+      if (value < 1 || value > 60000) return WQ_ERR_INVALID_ARG;
+      g_opt_wait_limit_ms = value;
+      return WQ_OK;
+    case WQ_OPT_TEST_STALL:
+      if (value != 0 && value != 1) return WQ_ERR_INVALID_ARG;
+      g_opt_test_stall = value;
+      return WQ_OK;
     case WQ_OPT_TC_DEQUANT_WARPS:
       if (value != 0 && value != 4 && value != 8) return WQ_ERR_INVALID_ARG;
       g_opt_tc_dequant_warps = value;
@@ -319,6 +330,8 @@ int64_t wq_get_option(int32_t option) {
     case WQ_OPT_GEMV_GRID: return g_opt_gemv_grid;
     case WQ_OPT_TC_BK: return g_opt_tc_bk;
     case WQ_OPT_TC_DEQUANT_WARPS: return g_opt_tc_dequant_warps;
+    case WQ_OPT_WAIT_LIMIT_MS: return g_opt_wait_limit_ms;
+    case WQ_OPT_TEST_STALL: return g_opt_test_stall;
     case WQ_OPT_PDL: return g_opt_pdl;
   }
   return -1;

@@ -33,7 +33,6 @@ using namespace sm100;
 
 constexpr int kTcRows = 128;             // output channels per CTA
 constexpr int kTcABufs = 2;              // TMEM A buffers
-constexpr long long kSpinLimitCycles = 4000000000LL;  // ~2 s at 2 GHz
 
 struct TcArgs {
   const __half* steps;
@@ -44,6 +43,8 @@ struct TcArgs {
   int stages;      // shared-memory ring depth
   uint32_t tmem_cols;
   int* err;
+  long long spin_limit;  // SM clock cycles a bounded wait may last
+  int stall;             // test hook: issue no loads, so every consumer wait runs out
 };
 
 __device__ __forceinline__ __half2 u2h(uint32_t u) { return *reinterpret_cast<__half2*>(&u); }
@@ -132,9 +133,9 @@ w4a16_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
       prefetch_tensormap(&tmX);
       prefetch_tensormap(&tmP);
       int issued = 0;
-      for (int kt = 0, s = 0, u = 0; kt < KT; ++kt) {  // s = kt % S, u = kt / S
+      for (int kt = 0, s = 0, u = 0; kt < (a.stall ? 0 : KT); ++kt) {  // s = kt % S, u = kt / S
         if (*abort_flag) break;
-        if (u > 0 && !mbar_wait(&sempty[s], (u - 1) & 1, a.err, kSpinLimitCycles)) { *abort_flag = 1; break; }
+        if (u > 0 && !mbar_wait(&sempty[s], (u - 1) & 1, a.err, a.spin_limit)) { *abort_flag = 1; break; }
         mbar_arrive_expect_tx(&full[s], (uint32_t)stage_bytes);
 #pragma unroll
         for (int i = 0; i < kXBoxes; ++i) tma_load_2d(stageX(s) + i * xbox, &tmX, kt * BK + 64 * i, 0, &full[s]);
@@ -144,7 +145,7 @@ w4a16_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
       }
       // Drain: every copy this thread issued has landed before the CTA exits.
       for (int kt = issued > S ? issued - S : 0; kt < issued; ++kt)
-        mbar_wait(&full[kt % S], (kt / S) & 1, a.err, kSpinLimitCycles);
+        mbar_wait(&full[kt % S], (kt / S) & 1, a.err, a.spin_limit);
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------- MMA issuer
@@ -153,7 +154,7 @@ w4a16_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
       int committed = -1;
       for (int kt = 0, s = 0, b = 0, ub = 0; kt < KT; ++kt) {
         if (*abort_flag) break;
-        if (!mbar_wait(&afull[b], ub & 1, a.err, kSpinLimitCycles)) { *abort_flag = 1; break; }
+        if (!mbar_wait(&afull[b], ub & 1, a.err, a.spin_limit)) { *abort_flag = 1; break; }
         tc_fence_after();
         const uint32_t xaddr = smem_u32(stageX(s));
 #pragma unroll
@@ -169,7 +170,7 @@ w4a16_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
       }
       mma_commit(accum);
       if (*abort_flag && committed >= 0)  // let issued MMAs finish before teardown
-        mbar_wait(&aempty[committed % kTcABufs], (committed / kTcABufs) & 1, a.err, kSpinLimitCycles);
+        mbar_wait(&aempty[committed % kTcABufs], (committed / kTcABufs) & 1, a.err, a.spin_limit);
     }
   } else {
     // ---------------------------------------------------------- dequant + epilogue
@@ -207,7 +208,7 @@ w4a16_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
       const __half z64n = __hneg(__hadd(zr_cur, __float2half(64.f)));
       const __half2 zz = __halves2half2(z1024, z1024);
       const __half2 zz16n = __halves2half2(z64n, z64n);
-      const bool landed = mbar_wait(&full[s], u & 1, a.err, kSpinLimitCycles);
+      const bool landed = mbar_wait(&full[s], u & 1, a.err, a.spin_limit);
       if (!__all_sync(0xffffffffu, landed)) { *abort_flag = 1; break; }
       // The packed tile is swizzled by the TMA: with 64-byte rows (BK = 128)
       // 16-byte chunk c of row r sits at chunk c ^ ((r >> 1) & 3), with
@@ -234,7 +235,7 @@ w4a16_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
         mbar_arrive(&afull[pend_b]);
       }
       bool ok = true;
-      if (kt >= kTcABufs) ok = mbar_wait(&aempty[b], (ub - 1) & 1, a.err, kSpinLimitCycles);
+      if (kt >= kTcABufs) ok = mbar_wait(&aempty[b], (ub - 1) & 1, a.err, a.spin_limit);
       if (!__all_sync(0xffffffffu, ok)) { *abort_flag = 1; break; }
       const uint32_t ta = tmem_a + ((uint32_t)(32 * q) << 16) + (uint32_t)(b * kACols + (kACols / NH) * h);
 #pragma unroll
@@ -251,7 +252,7 @@ w4a16_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
     // Epilogue: D[n][m] from TMEM -> Y[m][n]; the NH warp quartets take
     // alternate 16-column chunks.
     bool done = !__any_sync(0xffffffffu, *abort_flag != 0);
-    if (done) done = __all_sync(0xffffffffu, mbar_wait(accum, 0, a.err, kSpinLimitCycles));
+    if (done) done = __all_sync(0xffffffffu, mbar_wait(accum, 0, a.err, a.spin_limit));
     if (done) {
       tc_fence_after();
       for (int c0 = 16 * h; c0 < a.BN; c0 += 16 * NH) {
@@ -309,9 +310,12 @@ static uint32_t pow2_cols(uint32_t c) {
 // CTAs per SM when that ring and the tile's TMEM fit half an SM).
 // bk_opt: 0 = library choice, else 64 or 128 input channels per stage.
 // dw_opt: 0 = library choice (4), else 4 or 8 dequantizing warps.
+// wait_ms: how long a bounded mbarrier wait may last; stall: test hook (the
+// producer issues no loads, so the kernel's waits run out and it returns with
+// WQ_ERR_TIMEOUT latched).
 cudaError_t launch_gemm_tc(const void* X, const uint32_t* packed, const void* steps, const void* zeros, int64_t M,
                            int64_t N, int64_t K, void* Y, int* err, cudaStream_t st, int stages_opt, int bk_opt,
-                           int dw_opt) {
+                           int dw_opt, int wait_ms, bool stall) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return cudaErrorNotSupported;
   for (int64_t m0 = 0; m0 < M; m0 += 256) {
@@ -368,6 +372,8 @@ cudaError_t launch_gemm_tc(const void* X, const uint32_t* packed, const void* st
     }
     a.stages = S;
     a.err = err;
+    a.spin_limit = (long long)wait_ms * 2000000LL;  // cycles at <= 2 GHz: at least wait_ms
+    a.stall = stall ? 1 : 0;
     size_t smem = 1024 + (size_t)S * stage + (2 * S + 2 * kTcABufs + 1) * 8 + 16;
     // Never more CTAs on an SM than its 512 TMEM columns can hold at once.
     const size_t smem_floor = a.tmem_cols > 256 ? 120 * 1024 : 80 * 1024;
