@@ -93,6 +93,10 @@ typedef struct wq_quant_cfg {
 } wq_quant_cfg;
 
 /* ABI version of the loaded library (WQ_ABI_VERSION). */
+/* Version of the packed layout documented above (codes, steps, zeros). A
+ * stored quantized weight records it; a reader refuses another value. */
+#define WQ_LAYOUT_VERSION 1
+int32_t wq_layout_version(void);
 int32_t wq_abi_version(void);
 
 /* Static string for a status code. Never NULL. */

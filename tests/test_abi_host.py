@@ -115,3 +115,29 @@ def test_option_values_are_validated(wq):
     assert wq.wq_get_option(999) == -1
     with pytest.raises(wq.WQError):
         wq.wq_set_option(999, 0)
+
+
+def test_packed_weight_round_trip_and_header_checks(wq, tmp_path):
+    """save_packed / load_packed keep the three tensors bit for bit and refuse
+    a file whose layout version or sizes do not match."""
+    import torch
+    N, K = 5, 256
+    g = torch.Generator().manual_seed(3)
+    packed = torch.randint(-2**31, 2**31 - 1, (N * K // 8,), dtype=torch.int32, generator=g)
+    steps = torch.rand((N, K // 128), generator=g).to(torch.float16)
+    zeros = torch.randint(0, 16, (N, K // 128), generator=g).to(torch.float16)
+    p = tmp_path / "w.pt"
+    wq.save_packed(p, packed, steps, zeros, N, K, bits=4)
+    pk, st, zr, h = wq.load_packed(p)
+    assert torch.equal(pk, packed) and torch.equal(st, steps) and torch.equal(zr, zeros)
+    assert h["layout_version"] == wq.wq_layout_version() == 1 and (h["N"], h["K"], h["bits"]) == (N, K, 4)
+    d = torch.load(p, weights_only=True)
+    d["header"]["layout_version"] = 2
+    torch.save(d, tmp_path / "v2.pt")
+    with pytest.raises(ValueError):
+        wq.load_packed(tmp_path / "v2.pt")
+    d["header"]["layout_version"] = 1
+    d["header"]["K"] = 384
+    torch.save(d, tmp_path / "bad.pt")
+    with pytest.raises(ValueError):
+        wq.load_packed(tmp_path / "bad.pt")

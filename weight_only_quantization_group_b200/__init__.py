@@ -16,6 +16,9 @@ import torch
 
 __all__ = [
     "WQError",
+    "save_packed",
+    "load_packed",
+    "wq_layout_version",
     "lib",
     "library_path",
     "wq_abi_version",
@@ -40,6 +43,7 @@ library_path = os.path.join(_HERE, "libwq.so")
 # Every symbol include/wq.h declares.
 EXPORTED_SYMBOLS = (
     "wq_abi_version",
+    "wq_layout_version",
     "wq_status_string",
     "wq_packed_words",
     "wq_quantize_pack",
@@ -105,6 +109,7 @@ def _load() -> ctypes.CDLL:
     cfgp = ctypes.POINTER(_Cfg)
     sig = {
         "wq_abi_version": (i32, []),
+        "wq_layout_version": (i32, []),
         "wq_status_string": (ctypes.c_char_p, [i32]),
         "wq_packed_words": (sz, [i64, i64, cfgp]),
         "wq_quantize_pack": (i32, [vp, vp, i64, i64, cfgp, vp, vp, vp, vp]),
@@ -189,6 +194,37 @@ def _check(t: torch.Tensor, dtype, name: str):
 def _raise(st: int, where: str):
     if st != WQ_OK:
         raise WQError(st, where)
+
+
+def wq_layout_version() -> int:
+    return int(lib().wq_layout_version())
+
+
+def save_packed(path, packed: torch.Tensor, steps: torch.Tensor, zeros: torch.Tensor, N: int, K: int, *,
+                bits: int = 4, group_size: int = 128, symmetric: bool = False) -> None:
+    """Store a quantized weight (the three tensors of wq_quantize_pack) with a
+    header naming the layout version and the quantization config."""
+    header = {"format": "wq-packed", "layout_version": wq_layout_version(), "bits": int(bits),
+              "group_size": int(group_size), "symmetric": bool(symmetric), "N": int(N), "K": int(K)}
+    torch.save({"header": header, "packed": packed.detach().cpu(), "steps": steps.detach().cpu(),
+                "zeros": zeros.detach().cpu()}, path)
+
+
+def load_packed(path, device=None):
+    """Read what save_packed wrote; checks the header against this library's
+    layout and the tensor sizes. Returns (packed, steps, zeros, header)."""
+    d = torch.load(path, map_location="cpu", weights_only=True)
+    h = d.get("header", {})
+    if h.get("format") != "wq-packed" or h.get("layout_version") != wq_layout_version():
+        raise ValueError(f"{path}: not a wq-packed file of layout version {wq_layout_version()}")
+    N, K, bits = h["N"], h["K"], h["bits"]
+    words = wq_packed_words(N, K, bits=bits, group_size=h["group_size"], symmetric=h["symmetric"])
+    G = K // h["group_size"]
+    if (words == 0 or d["packed"].numel() != words or tuple(d["steps"].shape) != (N, G)
+            or tuple(d["zeros"].shape) != (N, G)):
+        raise ValueError(f"{path}: tensor sizes do not match the header")
+    out = [d[k] if device is None else d[k].to(device) for k in ("packed", "steps", "zeros")]
+    return out[0], out[1], out[2], h
 
 
 def wq_abi_version() -> int:

@@ -2,6 +2,7 @@
 // Every entry point validates on the host, enqueues on the caller's stream and
 // returns; none allocates device memory.
 #include <mutex>
+#include <nvtx3/nvToolsExt.h>
 
 #include "wq_common.cuh"
 
@@ -61,6 +62,14 @@ int* device_flag() {
   return g_flag_addr[dev];
 }
 
+// NVTX range around each entry point (a no-op unless a profiler is attached).
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
+
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
 int32_t check_cfg(const wq_quant_cfg* cfg) {
@@ -99,6 +108,7 @@ int64_t g_opt_test_stall = 0;
 extern "C" {
 
 int32_t wq_abi_version(void) { return WQ_ABI_VERSION; }
+int32_t wq_layout_version(void) { return WQ_LAYOUT_VERSION; }
 
 const char* wq_status_string(int32_t s) {
   switch (s) {
@@ -121,6 +131,7 @@ size_t wq_packed_words(int64_t N, int64_t K, const wq_quant_cfg* cfg) {
 
 int32_t wq_quantize_pack(const void* W, const void* s, int64_t N, int64_t K, const wq_quant_cfg* cfg,
                          uint32_t* packed, void* steps, void* zeros, void* stream) {
+  NvtxRange nvtx_range("wq_quantize_pack");
   int32_t st = check_cfg(cfg);
   if (st != WQ_OK) return st;
   if ((st = check_shape(N, K)) != WQ_OK) return st;
@@ -136,6 +147,7 @@ int32_t wq_quantize_pack(const void* W, const void* s, int64_t N, int64_t K, con
 
 int32_t wq_unpack_dequant(const uint32_t* packed, const void* steps, const void* zeros, int64_t N, int64_t K,
                           const wq_quant_cfg* cfg, void* W_out, void* stream) {
+  NvtxRange nvtx_range("wq_unpack_dequant");
   int32_t st = check_cfg(cfg);
   if (st != WQ_OK) return st;
   if ((st = check_shape(N, K)) != WQ_OK) return st;
@@ -154,6 +166,7 @@ size_t wq_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, const wq_quant_c
 int32_t wq_w4a16_gemm(const void* X, const uint32_t* packed, const void* steps, const void* zeros, int64_t M,
                       int64_t N, int64_t K, const wq_quant_cfg* cfg, void* Y, void* workspace,
                       size_t workspace_bytes, void* stream) {
+  NvtxRange nvtx_range("wq_w4a16_gemm");
   (void)workspace; (void)workspace_bytes;
   int32_t st = check_cfg(cfg);
   if (st != WQ_OK) return st;
@@ -217,6 +230,7 @@ int32_t wq_awq_scale_search(const void* X, int64_t T, int64_t K, const void* con
                             int32_t n_lin, const wq_quant_cfg* cfg, const double* alpha, int32_t n_alpha,
                             void* s_out, double* mu_out, double* loss_out, int32_t* best_out, void* workspace,
                             size_t workspace_bytes, void* stream) {
+  NvtxRange nvtx_range("wq_awq_scale_search");
   int32_t st = check_awq(T, K, N_i, n_lin, n_alpha, cfg);
   if (st != WQ_OK) return st;
   if (!X || !W || !alpha || !s_out) return WQ_ERR_INVALID_ARG;
@@ -242,6 +256,7 @@ int32_t wq_awq_scale_search(const void* X, int64_t T, int64_t K, const void* con
 int32_t wq_awq_scale_search_noalloc(const void* X, int64_t T, int64_t K, const void* const* W, const int64_t* N_i,
                                     int32_t n_lin, const wq_quant_cfg* cfg, const double* alpha, int32_t n_alpha,
                                     void* s_out, double* mu_out, double* loss_out, int32_t* best_out, void* stream) {
+  NvtxRange nvtx_range("wq_awq_scale_search_noalloc");
   int32_t st = check_awq(T, K, N_i, n_lin, n_alpha, cfg);
   if (st != WQ_OK) return st;
   if (!X || !W || !alpha || !s_out) return WQ_ERR_INVALID_ARG;
