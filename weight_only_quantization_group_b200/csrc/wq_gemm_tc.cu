@@ -25,6 +25,8 @@
 // far ahead as shared memory allows while only two A buffers occupy TMEM.
 // Every mbarrier wait is bounded; on a timeout the kernel latches
 // WQ_ERR_TIMEOUT, drains its own copies, frees its tensor memory and returns.
+#include <type_traits>
+
 #include "wq_sm100.cuh"
 
 namespace wq {
@@ -32,7 +34,7 @@ namespace wq {
 using namespace sm100;
 
 constexpr int kTcRows = 128;             // output channels per CTA
-constexpr int kTcABufs = 2;              // TMEM A buffers
+constexpr int kTcMaxABufs = 3;           // TMEM A buffers at most (barrier space)
 
 struct TcArgs {
   const __half* steps;
@@ -73,7 +75,8 @@ __device__ __forceinline__ uint4 dequant_word4(uint32_t w, __half2 zz, __half2 z
 // NH: dequantizing warp quartets; each of the NH owns 1/NH of a stage's words
 // of every row (more warps hide more latency, fewer amortize the per-stage
 // waits over more weights).
-template <int BK, int NH>
+// NA: depth of the TMEM A ring (2, or 3 when the tile leaves room).
+template <int BK, int NH, int NA>
 __global__ void __launch_bounds__(64 + 128 * NH, 1)
 w4a16_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmP,
                      TcArgs a) {
@@ -90,8 +93,8 @@ w4a16_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + (size_t)S * stage_bytes);
   uint64_t* sempty = full + S;
   uint64_t* afull = sempty + S;
-  uint64_t* aempty = afull + kTcABufs;
-  uint64_t* accum = aempty + kTcABufs;
+  uint64_t* aempty = afull + kTcMaxABufs;
+  uint64_t* accum = aempty + kTcMaxABufs;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accum + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -109,7 +112,7 @@ w4a16_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
       mbar_init(&full[s], 1);
       mbar_init(&sempty[s], 1);
     }
-    for (int b = 0; b < kTcABufs; ++b) {
+    for (int b = 0; b < NA; ++b) {
       mbar_init(&afull[b], 128 * NH);
       mbar_init(&aempty[b], 1);
     }
@@ -166,11 +169,11 @@ w4a16_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
         mma_commit(&sempty[s]);
         committed = kt;
         if (++s == S) s = 0;
-        if (++b == kTcABufs) { b = 0; ++ub; }
+        if (++b == NA) { b = 0; ++ub; }
       }
       mma_commit(accum);
       if (*abort_flag && committed >= 0)  // let issued MMAs finish before teardown
-        mbar_wait(&aempty[committed % kTcABufs], (committed / kTcABufs) & 1, a.err, a.spin_limit);
+        mbar_wait(&aempty[committed % NA], (committed / NA) & 1, a.err, a.spin_limit);
     }
   } else {
     // ---------------------------------------------------------- dequant + epilogue
@@ -235,14 +238,14 @@ w4a16_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
         mbar_arrive(&afull[pend_b]);
       }
       bool ok = true;
-      if (kt >= kTcABufs) ok = mbar_wait(&aempty[b], (ub - 1) & 1, a.err, a.spin_limit);
+      if (kt >= NA) ok = mbar_wait(&aempty[b], (ub - 1) & 1, a.err, a.spin_limit);
       if (!__all_sync(0xffffffffu, ok)) { *abort_flag = 1; break; }
       const uint32_t ta = tmem_a + ((uint32_t)(32 * q) << 16) + (uint32_t)(b * kACols + (kACols / NH) * h);
 #pragma unroll
       for (int i = 0; i < kWords / 4; ++i) tmem_st16(ta + 16 * i, nv[i]);
       pend_b = b;
       if (++s == S) { s = 0; ++u; }
-      if (++b == kTcABufs) { b = 0; ++ub; }
+      if (++b == NA) { b = 0; ++ub; }
     }
     if (pend_b >= 0) {
       tmem_st_wait();
@@ -354,19 +357,23 @@ cudaError_t launch_gemm_tc(const void* X, const uint32_t* packed, const void* st
     a.N = (int)N;
     a.K = (int)K;
     a.BN = BN;
-    a.tmem_cols = pow2_cols((uint32_t)(BN + kTcABufs * BK / 2));
-    // Two CTAs per SM when the tile's TMEM fits half of it and half the shared
-    // memory still holds a ring of three stages; otherwise one CTA per SM with
-    // the deepest ring that fits.
+    // A third A buffer when it still fits the same TMEM allocation
+    const int NA = pow2_cols((uint32_t)(BN + 3 * BK / 2)) == pow2_cols((uint32_t)(BN + 2 * BK / 2)) ? 3 : 2;
+    a.tmem_cols = pow2_cols((uint32_t)(BN + NA * BK / 2));
+    // CTAs per SM: as many as the 512 TMEM columns hold (1, 2 or 4), fewer
+    // while their share of shared memory cannot hold a ring of three stages.
+    // The ring then takes that share (at most 16 stages).
     const int stage = (BK / 64) * BN * 128 + kTcRows * BK / 2;
-    const size_t half_budget = 110 * 1024, full_budget = 220 * 1024;
+    auto share = [](int c) { return (size_t)(225 * 1024) / (size_t)c - 3 * 1024; };
+    int cps = 512 / (int)a.tmem_cols;
     int S;
     if (stages_opt > 0) {
       S = stages_opt;
-      if ((size_t)S * stage + 2048 > full_budget) return cudaErrorInvalidValue;
+      while (cps > 1 && (size_t)S * stage + 2048 > share(cps)) cps /= 2;
+      if ((size_t)S * stage + 2048 > share(1)) return cudaErrorInvalidValue;
     } else {
-      const bool two_per_sm = a.tmem_cols <= 256 && 3 * (size_t)stage + 2048 <= half_budget;
-      S = (int)(((two_per_sm ? half_budget : full_budget) - 2048) / stage);
+      while (cps > 1 && 3 * (size_t)stage + 2048 > share(cps)) cps /= 2;
+      S = (int)((share(cps) - 2048) / stage);
       if (S > 16) S = 16;
       if (S < 2) S = 2;
     }
@@ -374,13 +381,22 @@ cudaError_t launch_gemm_tc(const void* X, const uint32_t* packed, const void* st
     a.err = err;
     a.spin_limit = (long long)wait_ms * 2000000LL;  // cycles at <= 2 GHz: at least wait_ms
     a.stall = stall ? 1 : 0;
-    size_t smem = 1024 + (size_t)S * stage + (2 * S + 2 * kTcABufs + 1) * 8 + 16;
-    // Never more CTAs on an SM than its 512 TMEM columns can hold at once.
-    const size_t smem_floor = a.tmem_cols > 256 ? 120 * 1024 : 80 * 1024;
+    size_t smem = 1024 + (size_t)S * stage + (2 * S + 2 * kTcMaxABufs + 1) * 8 + 16;
+    // At most cps CTAs per SM (their TMEM must fit at once): ask for more than
+    // 1/(cps+1) of the SM's shared memory.
+    const size_t smem_floor = (size_t)(228 * 1024) / (size_t)(cps + 1) + 1024;
     if (smem < smem_floor) smem = smem_floor;
     const int NH = dw_opt == 8 ? 2 : 1;  // 4 dequantizing warps unless asked for 8
-    auto kern = BK == 128 ? (NH == 1 ? w4a16_gemm_tc_kernel<128, 1> : w4a16_gemm_tc_kernel<128, 2>)
-                          : (NH == 1 ? w4a16_gemm_tc_kernel<64, 1> : w4a16_gemm_tc_kernel<64, 2>);
+    auto pick = [&](auto bk, auto nh) {
+      constexpr int B = decltype(bk)::value, H = decltype(nh)::value;
+      return NA == 3 ? w4a16_gemm_tc_kernel<B, H, 3> : w4a16_gemm_tc_kernel<B, H, 2>;
+    };
+    using I64 = std::integral_constant<int, 64>;
+    using I128 = std::integral_constant<int, 128>;
+    using I1 = std::integral_constant<int, 1>;
+    using I2 = std::integral_constant<int, 2>;
+    auto kern = BK == 128 ? (NH == 1 ? pick(I128{}, I1{}) : pick(I128{}, I2{}))
+                          : (NH == 1 ? pick(I64{}, I1{}) : pick(I64{}, I2{}));
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     const dim3 grid((unsigned)((N + kTcRows - 1) / kTcRows));
