@@ -94,6 +94,18 @@ def profiled_traffic(kernel: str):
     return e.get("dram_bytes_per_launch")
 
 
+def max_over_ranks(ms: float, world: int, device) -> float:
+    """The slowest rank's time: every rank reports its own device time and all
+    take the maximum (the same collective on every rank, in the same order)."""
+    if world <= 1:
+        return ms
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([ms], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 class ClockSampler:
     """nvidia-smi clocks and throttle reasons sampled every 200 ms."""
 
@@ -228,11 +240,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         torch.cuda.synchronize()
     barrier()
     torch.cuda.synchronize()
-    ms = ev0.elapsed_time(ev1)
-    if world > 1:
-        t = torch.tensor([ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(ev0.elapsed_time(ev1), world, dev)
     assert wq.wq_get_last_device_error() == 0
     ms_per_step = ms / args.steps
     value = world * step_bytes * args.steps / (ms * 1e-3) / 1e9  # GB/s, all ranks
@@ -270,11 +278,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         e2e_step(copies[i % n_copies])
     e1.record()
     torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1)
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
     e2e_value = world * step_bytes * e2e_steps / (e2e_ms * 1e-3) / 1e9
 
     rows = {}
