@@ -133,10 +133,9 @@ awq_error_kernel(LinearSet ls, int K, const __half* __restrict__ S, int alpha0, 
       for (int i = 0; i < 4; ++i) {
         const float2 f = __half22float2(h[i]);
         const float2 g = __half22float2(sh[i]);
-        const int q0 = group_quant_code<BITS, SYM>(w[8 * c + 2 * i], gq);
-        const int q1 = group_quant_code<BITS, SYM>(w[8 * c + 2 * i + 1], gq);
-        const float d0 = __fmul_rn((float)(q0 - gq.zero), gq.sf);  // exact
-        const float d1 = __fmul_rn((float)(q1 - gq.zero), gq.sf);
+        // (q - zero) * step is exact in fp32
+        const float d0 = __fmul_rn(__fsub_rn(group_quant_level<BITS, SYM>(w[8 * c + 2 * i], gq), gq.zf), gq.sf);
+        const float d1 = __fmul_rn(__fsub_rn(group_quant_level<BITS, SYM>(w[8 * c + 2 * i + 1], gq), gq.zf), gq.sf);
         // E is rounded to fp16 next, so an approximate 1/s is enough
         const __half2 hv = __floats2half2_rn(f.x - d0 * rcp_approx(g.x), f.y - d1 * rcp_approx(g.y));
         out[i] = *reinterpret_cast<const uint32_t*>(&hv);

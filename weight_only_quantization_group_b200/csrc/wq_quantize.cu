@@ -63,7 +63,7 @@ quantize_pack_kernel(const __half* __restrict__ W, const __half* __restrict__ s,
   }
   uint32_t q[32];
 #pragma unroll
-  for (int i = 0; i < 32; ++i) q[i] = (uint32_t)group_quant_code<BITS, SYM>(w[i], gq);
+  for (int i = 0; i < 32; ++i) q[i] = group_quant_code<BITS, SYM>(w[i], gq);
   if (!valid) return;
 
   if (BITS == 4) {
