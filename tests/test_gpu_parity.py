@@ -93,6 +93,91 @@ def test_quantize_pack_edge_groups(wq):
             assert_quant_parity(wq, W16, None, bits, sym)
 
 
+def _near_half_case(bits, sym, rows=12, groups=6, seed=5):
+    """Weights and AWQ scales whose scaled values w * s sit on, or within
+    2^-16 of, half-integer multiples of the group step: ties (rounded to even
+    by the contract), values that the sign of w * s - h * step settles, and
+    values only the exact fp32 quotient settles (closer than 2^-18).
+
+    Each group's first two channels (s = 1) fix its step at 2^-7; the other
+    channels take fp16 (w, s) pairs found by enumerating every fp16 s in
+    [1, 2)."""
+    step = 2.0 ** -7
+    qmax = (1 << (bits - 1)) - 1
+    lo_m, hi_m = (-qmax, qmax) if sym else (-(((1 << bits) - 1) // 2), 1 << (bits - 1))
+    s_all = np.arange(0x3C00, 0x4000, dtype=np.uint16).view(np.float16)
+    pairs = []
+    for m in range(lo_m, hi_m):
+        h = m + 0.5
+        if abs(h) >= (qmax if sym else 99):
+            continue
+        w0 = (h * step / s_all.astype(np.float64)).astype(np.float16)
+        for w in (np.nextafter(w0, np.float16(-1)), w0, np.nextafter(w0, np.float16(1))):
+            a = (w.astype(np.float32) * s_all.astype(np.float32)).astype(np.float64) / step
+            dist = np.abs(a - h)
+            for i in np.nonzero(dist <= 2.0 ** -16)[0]:
+                pairs.append((w[i], s_all[i], dist[i]))
+    g = np.random.default_rng(seed)
+    g.shuffle(pairs)
+    K = 128 * groups
+    s = np.ones(K, np.float16)
+    W = np.zeros((rows, K), np.float16)
+    free = [k for k in range(K) if k % 128 >= 2]
+    used = []
+    for k, (w, sv, dist) in zip(free, pairs):
+        s[k] = sv
+        W[:, k] = w
+        used.append(dist)
+    for k in free[len(used):]:
+        s[k] = np.float16(1.0 + g.random())
+    # every row: a random third of the channels take other values in range
+    bound = 0.95 * (qmax if sym else min(-lo_m, hi_m)) * step
+    for r in range(rows):
+        sel = np.array(free)[g.random(len(free)) < 1 / 3]
+        W[r, sel] = (g.uniform(-bound, bound, len(sel)) / s[sel].astype(np.float64)).astype(np.float16)
+    W[:, 0::128] = np.float16(lo_m * step)
+    W[:, 1::128] = np.float16(hi_m * step)
+    used = np.array(used)
+    classes = ((used == 0).sum(), ((used > 0) & (used < 2.0 ** -18)).sum(), (used >= 2.0 ** -18).sum())
+    return W, s, classes
+
+
+@pytest.mark.parametrize("bits", [3, 4])
+@pytest.mark.parametrize("sym", [False, True])
+def test_quantize_pack_near_half_quotients(wq, bits, sym):
+    W, s, (ties, by_division, by_sign) = _near_half_case(bits, sym)
+    assert ties > 0 and by_division > 0 and by_sign > 0, (ties, by_division, by_sign)
+    codes, st, _ = O.quantize_groups(W, bits, 128, sym, s16=s)
+    assert np.all(st.astype(np.float64) == 2.0 ** -7)
+    assert_quant_parity(wq, W, s, bits, sym)
+    # the same values without scaling: fp16 ties only
+    assert_quant_parity(wq, (W.astype(np.float32) * s.astype(np.float32)).astype(np.float16), None, bits, sym)
+
+
+@pytest.mark.parametrize("bits", [3, 4])
+@pytest.mark.parametrize("sym", [False, True])
+@pytest.mark.parametrize("lo,hi", [(-0.0546875, 0.0625), (-0.0713, 0.01831), (-3.1e-3, 2.9e-2)])
+def test_quantize_pack_every_fp16_value_in_range(wq, bits, sym, lo, hi):
+    """Every finite fp16 value between lo and hi, 126 to a group, each group
+    also holding lo and hi so that all groups share one step (whatever the
+    rounded-up range over 2^b - 1 gives: here steps with long significands)."""
+    lo16, hi16 = np.float16(lo), np.float16(hi)
+    allv = np.arange(0, 0x10000, dtype=np.uint32).astype(np.uint16).view(np.float16)
+    allv = allv[np.isfinite(allv)]
+    vals = np.unique(allv[(allv >= lo16) & (allv <= hi16)])
+    per = 126
+    groups = -(-vals.size // per)
+    vals = np.concatenate([vals, np.zeros(groups * per - vals.size, np.float16)]).reshape(groups, per)
+    grp = np.concatenate([np.full((groups, 1), lo16), np.full((groups, 1), hi16), vals], axis=1)
+    gpr = 8  # groups per row
+    rows = -(-groups // gpr)
+    pad = np.zeros((rows * gpr - groups, 128), np.float16)
+    W = np.concatenate([grp, pad]).reshape(rows, gpr * 128)
+    _, st, _ = O.quantize_groups(W, bits, 128, sym)
+    assert np.unique(st[: groups // gpr]).size == 1
+    assert_quant_parity(wq, W, None, bits, sym)
+
+
 def test_quantize_pack_small_linear(wq):
     c = synth.config_small_linear(0)
     assert_quant_parity(wq, c.W, None, 4, False)

@@ -75,6 +75,28 @@ __device__ __forceinline__ float rcp_approx(float x) {
   return r;
 }
 
+// E for one 8-channel chunk: w - deq(w * s) / s, with deq = (level - zero) *
+// step exact in fp32 (the offset level minus 1.5 * 2^23 is level - zero,
+// exactly); E is rounded to fp16 next, so an approximate 1/s is enough.
+template <int BITS, bool SYM>
+__device__ __forceinline__ uint4 chunk_errors(uint4 x, uint4 sv, const GroupQuant& gq) {
+  const __half2* h = reinterpret_cast<const __half2*>(&x);
+  const __half2* sh = reinterpret_cast<const __half2*>(&sv);
+  uint4 out;
+  uint32_t* o = reinterpret_cast<uint32_t*>(&out);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 f = __half22float2(h[i]);
+    const float2 g = __half22float2(sh[i]);
+    const float l0 = __fsub_rn(group_offset_level<BITS, SYM>(__fmul_rn(f.x, g.x), gq), kRoundMagic);
+    const float l1 = __fsub_rn(group_offset_level<BITS, SYM>(__fmul_rn(f.y, g.y), gq), kRoundMagic);
+    const float d0 = __fmul_rn(l0, gq.sf), d1 = __fmul_rn(l1, gq.sf);
+    const __half2 hv = __floats2half2_rn(f.x - d0 * rcp_approx(g.x), f.y - d1 * rcp_approx(g.y));
+    o[i] = *reinterpret_cast<const uint32_t*>(&hv);
+  }
+  return out;
+}
+
 template <int BITS, bool SYM>
 __global__ void __launch_bounds__(256)
 awq_error_kernel(LinearSet ls, int K, const __half* __restrict__ S, int alpha0, int nb, __half* __restrict__ E) {
@@ -126,23 +148,8 @@ awq_error_kernel(LinearSet ls, int K, const __half* __restrict__ S, int alpha0, 
     const GroupQuant gq = group_quant_decide<BITS, SYM, 32, 4>(w);
 #pragma unroll
     for (int c = 0; c < 4; ++c) {
-      const __half2* h = reinterpret_cast<const __half2*>(&xraw[c]);
-      const __half2* sh = reinterpret_cast<const __half2*>(&sraw[c]);
-      uint32_t out[4];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const float2 f = __half22float2(h[i]);
-        const float2 g = __half22float2(sh[i]);
-        // (q - zero) * step is exact in fp32
-        const float d0 = __fmul_rn(__fsub_rn(group_quant_level<BITS, SYM>(w[8 * c + 2 * i], gq), gq.zf), gq.sf);
-        const float d1 = __fmul_rn(__fsub_rn(group_quant_level<BITS, SYM>(w[8 * c + 2 * i + 1], gq), gq.zf), gq.sf);
-        // E is rounded to fp16 next, so an approximate 1/s is enough
-        const __half2 hv = __floats2half2_rn(f.x - d0 * rcp_approx(g.x), f.y - d1 * rcp_approx(g.y));
-        out[i] = *reinterpret_cast<const uint32_t*>(&hv);
-      }
-      if (valid)
-        *reinterpret_cast<uint4*>(E + ((size_t)b * N + n) * K + k0 + 8 * c) =
-            make_uint4(out[0], out[1], out[2], out[3]);
+      const uint4 out = chunk_errors<BITS, SYM>(xraw[c], sraw[c], gq);
+      if (valid) *reinterpret_cast<uint4*>(E + ((size_t)b * N + n) * K + k0 + 8 * c) = out;
     }
   }
 }

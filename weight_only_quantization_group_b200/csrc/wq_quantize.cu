@@ -10,91 +10,105 @@
 //
 // Mapping: 4 lanes per group, each lane owns 32 consecutive input channels
 // (four 16-byte loads of W; one 16-byte store of 4-bit codes, or the three
-// words of a 3-bit chunk); group_quant_decide() reduces the group's range
-// with two xor-shuffles. 2 B/weight in, 0.5 (0.375) B/weight out.
+// words of a 3-bit chunk); the group's range is reduced with two
+// xor-shuffles. 2 B/weight in, 0.5 (0.375) B/weight out.
 #include "wq_quant_core.cuh"
 
 namespace wq {
+
+// A lane's 32 codes packed: four 4-bit words, or one 3-bit chunk of three.
+// level(i) returns the offset level of channel i (group_offset_level).
+template <int BITS, class F>
+__device__ __forceinline__ void pack_lane(F level, int zero, uint32_t (&o)[4]) {
+  if constexpr (BITS == 4) {
+#pragma unroll
+    for (int c = 0; c < 4; ++c) o[c] = pack_word4([&](int i) { return level(8 * c + i); }, zero);
+  } else {
+    uint32_t t[3];
+    pack_chunk3(level, zero, t);
+    o[0] = t[0], o[1] = t[1], o[2] = t[2], o[3] = 0;
+  }
+}
+
+// One lane unit u: channels [32u, 32u + 32) of the row-major weight, a
+// quarter of group u / 4. The group's decision (shared by its 4 lanes), then
+// the lane's 32 codes, packed and stored. sk: the unit's 32 AWQ scales.
+template <int BITS, bool SYM, bool HAS_S>
+__device__ __forceinline__ void quantize_unit(const uint4 (&raw)[4], const __half* __restrict__ sk, int64_t u,
+                                              bool valid, uint32_t* __restrict__ packed,
+                                              __half* __restrict__ steps, __half* __restrict__ zeros, int* err) {
+  // with AWQ scaling the products w * s in fp32 (exact: 11 x 11 significand bits)
+  float ws[HAS_S ? 32 : 1];
+  GroupQuant gq;
+  if constexpr (HAS_S) {
+    uint4 sr[4];
+#pragma unroll
+    for (int c = 0; c < 4; ++c) sr[c] = valid ? *reinterpret_cast<const uint4*>(sk + 8 * c) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+    for (int i = 0; i < 32; ++i) ws[i] = __fmul_rn(lane_half(raw, i), lane_half(sr, i));
+    gq = group_quant_decide<BITS, SYM, 32, 4>(ws);
+  } else {
+    gq = group_quant_decide_h<BITS, SYM, 4>(raw);
+  }
+  if (valid && (u & 3) == 0) {
+    if (!isfinite(gq.sf)) latch_error(err, WQ_ERR_RANGE);
+    steps[u >> 2] = gq.step_h;
+    zeros[u >> 2] = __int2half_rn(gq.zero);
+  }
+  auto value = [&](int i) -> float {
+    if constexpr (HAS_S) return ws[i]; else return lane_half(raw, i);
+  };
+
+  uint32_t o[4];
+  pack_lane<BITS>([&](int i) { return group_offset_level<BITS, SYM>(value(i), gq); }, gq.zero, o);
+  if (!valid) return;
+
+  if constexpr (BITS == 4) {
+    reinterpret_cast<uint4*>(packed)[u] = make_uint4(o[0], o[1], o[2], o[3]);
+  } else {
+    uint32_t* dst = packed + 3 * u;
+    dst[0] = o[0];
+    dst[1] = o[1];
+    dst[2] = o[2];
+  }
+}
 
 template <int BITS, bool SYM, bool HAS_S>
 __global__ void __launch_bounds__(256)
 quantize_pack_kernel(const __half* __restrict__ W, const __half* __restrict__ s, int64_t N, int64_t K,
                      uint32_t* __restrict__ packed, __half* __restrict__ steps,
                      __half* __restrict__ zeros, int* err) {
+  // Grid-stride over lane units (a lane's 32 channels of one group; unit u
+  // starts at element 32u of the row-major weight); the next unit's 64 bytes
+  // of W are in flight while this one is quantized.
   const int lane = threadIdx.x & 31;
-  const int sub = lane & 3;  // lane within the group
-  const int64_t G = K / kGroup;
-  const int64_t gidx = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 2;
-  const bool valid = gidx < N * G;
-  const int64_t n = valid ? gidx / G : 0;
-  const int64_t gi = valid ? gidx % G : 0;
-  const int64_t k0 = gi * kGroup + sub * 32;
+  const int64_t units = N * K / 32;
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  int64_t u = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const uint4* w4 = reinterpret_cast<const uint4*>(W);
+  // the column of unit u, tracked for the AWQ scales only
+  const int64_t kunits = K / 32, step_cols = stride % kunits;
+  int64_t col = HAS_S ? u % kunits : 0;
 
-  float w[32];
+  auto load = [&](uint4 (&r)[4]) {
 #pragma unroll
-  for (int c = 0; c < 4; ++c) {
-    uint4 raw = make_uint4(0, 0, 0, 0);
-    if (valid) raw = *reinterpret_cast<const uint4*>(W + n * K + k0 + 8 * c);
-    const __half2* h = reinterpret_cast<const __half2*>(&raw);
+    for (int c = 0; c < 4; ++c) r[c] = u < units ? w4[4 * u + c] : make_uint4(0, 0, 0, 0);
+  };
+  uint4 next[4];
+  load(next);
+  while (u - lane < units) {  // warp-uniform: the group shuffles need every lane
+    const int64_t cur = u;
+    const __half* sk = HAS_S ? s + 32 * col : nullptr;
+    uint4 raw[4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const float2 f = __half22float2(h[i]);
-      w[8 * c + 2 * i] = f.x;
-      w[8 * c + 2 * i + 1] = f.y;
-    }
+    for (int c = 0; c < 4; ++c) raw[c] = next[c];
+    u += stride;
     if (HAS_S) {
-      uint4 sraw = make_uint4(0, 0, 0, 0);
-      if (valid) sraw = *reinterpret_cast<const uint4*>(s + k0 + 8 * c);
-      const __half2* sh = reinterpret_cast<const __half2*>(&sraw);
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const float2 f = __half22float2(sh[i]);
-        w[8 * c + 2 * i] = __fmul_rn(w[8 * c + 2 * i], f.x);  // exact: 11 x 11 significand bits
-        w[8 * c + 2 * i + 1] = __fmul_rn(w[8 * c + 2 * i + 1], f.y);
-      }
+      col += step_cols;
+      if (col >= kunits) col -= kunits;
     }
-  }
-
-  const GroupQuant gq = group_quant_decide<BITS, SYM, 32, 4>(w);
-  if (valid && sub == 0) {
-    if (!isfinite(gq.sf)) latch_error(err, WQ_ERR_RANGE);
-    steps[n * G + gi] = gq.step_h;
-    zeros[n * G + gi] = __int2half_rn(gq.zero);
-  }
-  uint32_t q[32];
-#pragma unroll
-  for (int i = 0; i < 32; ++i) q[i] = group_quant_code<BITS, SYM>(w[i], gq);
-  if (!valid) return;
-
-  if (BITS == 4) {
-    // word c holds channels 8c..8c+7 in slot order [0, 2, 4, 6, 1, 3, 5, 7]
-    uint4 out;
-    uint32_t* o = reinterpret_cast<uint32_t*>(&out);
-#pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      const uint32_t* v = q + 8 * c;
-      o[c] = v[0] | (v[2] << 4) | (v[4] << 8) | (v[6] << 12) | (v[1] << 16) | (v[3] << 20) | (v[5] << 24) |
-             (v[7] << 28);
-    }
-    *reinterpret_cast<uint4*>(packed + (n * K + k0) / 8) = out;
-  } else {
-    // the lane's 32 channels are one 3-word chunk: word t holds channel pairs
-    // (10t + 2j, 10t + 2j + 1) at bits 3j and 16 + 3j, and bit t of channels
-    // 30 / 31 at bit 15 / 31
-    uint32_t o[3];
-#pragma unroll
-    for (int t = 0; t < 3; ++t) {
-      uint32_t word = 0;
-#pragma unroll
-      for (int j = 0; j < 5; ++j) word |= (q[10 * t + 2 * j] << (3 * j)) | (q[10 * t + 2 * j + 1] << (16 + 3 * j));
-      word |= ((q[30] >> t) & 1u) << 15;
-      word |= ((q[31] >> t) & 1u) << 31;
-      o[t] = word;
-    }
-    uint32_t* dst = packed + (n * K + k0) / 32 * 3;
-    dst[0] = o[0];
-    dst[1] = o[1];
-    dst[2] = o[2];
+    load(next);
+    quantize_unit<BITS, SYM, HAS_S>(raw, sk, cur, cur < units, packed, steps, zeros, err);
   }
 }
 
@@ -145,14 +159,26 @@ unpack_dequant_kernel(const uint32_t* __restrict__ packed, const __half* __restr
 
 cudaError_t launch_quantize_pack(const void* W, const void* s, int64_t N, int64_t K, int bits, bool sym,
                                  uint32_t* packed, void* steps, void* zeros, int* err, cudaStream_t st) {
-  const int64_t groups = N * (K / kGroup);
-  const dim3 grid((unsigned)((groups + 63) / 64));  // 4 lanes per group
+  const int64_t units = N * (K / kGroup) * 4;  // 4 lanes per group
   const dim3 block(256);
   auto Wp = static_cast<const __half*>(W);
   auto sp = static_cast<const __half*>(s);
   auto stp = static_cast<__half*>(steps);
   auto zp = static_cast<__half*>(zeros);
-#define WQ_QP(B, S, H) quantize_pack_kernel<B, S, H><<<grid, block, 0, st>>>(Wp, sp, N, K, packed, stp, zp, err)
+  // one wave of resident blocks (fewer when the matrix is small)
+  auto launch = [&](auto kern) {
+    static const int resident = [&] {
+      int dev = 0, sms = 0, occ = 0;
+      cudaGetDevice(&dev);
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, 256, 0);
+      return (sms > 0 ? sms : 1) * (occ > 0 ? occ : 1);
+    }();
+    const int64_t need = (units + 255) / 256;
+    const dim3 grid((unsigned)(need < resident ? need : resident));
+    kern<<<grid, block, 0, st>>>(Wp, sp, N, K, packed, stp, zp, err);
+  };
+#define WQ_QP(B, S, H) launch(quantize_pack_kernel<B, S, H>)
   if (bits == 4) {
     if (sym) { if (s) WQ_QP(4, true, true); else WQ_QP(4, true, false); }
     else     { if (s) WQ_QP(4, false, true); else WQ_QP(4, false, false); }
