@@ -112,7 +112,9 @@ size_t wq_packed_words(int64_t N, int64_t K, const wq_quant_cfg* cfg);
  * "MIT 6.5940 Lab 4 + Lab 5", section "Question 2"), and writes packed_dev
  * (uint32, wq_packed_words(N,K,cfg) words), steps_dev and zeros_dev (fp16
  * [N][K/128] each). One kernel launch. A step that is not finite in fp16
- * latches WQ_ERR_RANGE in the device flag. */
+ * (a group holding an infinite or NaN weight, or a range too large for fp16)
+ * latches WQ_ERR_RANGE in the device flag; that group's codes are then
+ * unspecified. */
 int32_t wq_quantize_pack(const void* W_dev, const void* s_dev, int64_t N, int64_t K,
                          const wq_quant_cfg* cfg, uint32_t* packed_dev, void* steps_dev,
                          void* zeros_dev, void* stream);

@@ -178,6 +178,35 @@ def test_quantize_pack_every_fp16_value_in_range(wq, bits, sym, lo, hi):
     assert_quant_parity(wq, W, None, bits, sym)
 
 
+@pytest.mark.parametrize("bad", [np.nan, np.inf, -np.inf])
+@pytest.mark.parametrize("sym", [False, True])
+@pytest.mark.parametrize("awq", [False, True])
+def test_quantize_pack_non_finite_weight(wq, bad, sym, awq):
+    """A non-finite weight makes its group's step non-finite and latches
+    WQ_ERR_RANGE; every other group is still quantized per the contract."""
+    g = synth.rng(300)
+    W = synth.weight(g, 8, 512, 0.02)
+    s = _awq_scale(512, 9) if awq else None
+    W[3, 200] = bad
+    packed, steps, zeros = wq.wq_quantize_pack(dev(W), None if s is None else dev(s), bits=4, symmetric=sym)
+    assert wq.wq_get_last_device_error() == wq.WQ_ERR_RANGE
+    assert wq.wq_get_last_device_error() == 0
+    Wc = W.copy()
+    Wc[3, 200] = 0
+    codes, st, z = O.quantize_groups(Wc, 4, 128, sym, s16=s)
+    gs = steps.cpu().numpy()
+    keep = np.ones(gs.shape, bool)
+    keep[3, 1] = False
+    assert not np.isfinite(gs[3, 1])
+    assert np.array_equal(gs.view(np.uint16)[keep], st.view(np.uint16)[keep])
+    assert np.array_equal(zeros.cpu().numpy().view(np.uint16)[keep], z.view(np.uint16)[keep])
+    words = O.pack_codes(codes, 4).reshape(8, 64)
+    gp = packed.cpu().numpy().view(np.uint32).reshape(8, 64)
+    wkeep = np.ones(gp.shape, bool)
+    wkeep[3, 16:32] = False
+    assert np.array_equal(gp[wkeep], words[wkeep])
+
+
 def test_quantize_pack_small_linear(wq):
     c = synth.config_small_linear(0)
     assert_quant_parity(wq, c.W, None, 4, False)
