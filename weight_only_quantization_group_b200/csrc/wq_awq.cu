@@ -33,13 +33,29 @@ constexpr size_t kAwqEBudget = size_t(1) << 30;  // bytes of E kept per alpha ba
 constexpr long long kAwqSpinLimit = 4000000000LL;
 
 // ------------------------------------------------------------------ S1
+// A block owns 32 columns (one per lane); its 8 warps take every 8th row and
+// the warps' sums meet in shared memory in warp order. fp16 magnitudes are
+// multiples of 2^-24 below 2^16, so while T <= 2^13 every partial sum stays
+// below 2^53 units of 2^-24: exact in fp64, whatever the order of the
+// additions. Beyond that the fixed order keeps the result deterministic.
 __global__ void __launch_bounds__(256) absmean_kernel(const __half* __restrict__ X, int T, int K,
                                                       double* __restrict__ mu) {
-  const int k = blockIdx.x * blockDim.x + threadIdx.x;
-  if (k >= K) return;
-  double acc = 0.0;  // fp16 magnitudes are multiples of 2^-24 below 2^16: exact
-  for (int t = 0; t < T; ++t) acc += fabs((double)__half2float(X[(size_t)t * K + k]));
-  mu[k] = acc / (double)T;
+  __shared__ double part[8][32];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int k = blockIdx.x * 32 + lane;
+  double acc = 0.0;
+  if (k < K) {
+#pragma unroll 8
+    for (int t = warp; t < T; t += 8) acc += fabs((double)__half2float(X[(size_t)t * K + k]));
+  }
+  part[warp][lane] = acc;
+  __syncthreads();
+  if (warp == 0 && k < K) {
+    double v = 0.0;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) v += part[w][lane];
+    mu[k] = v / (double)T;
+  }
 }
 
 // ------------------------------------------------------------------ S2
@@ -289,17 +305,24 @@ awq_loss_kernel(const __grid_constant__ CUtensorMap tmE, const __grid_constant__
 }
 
 // ------------------------------------------------------------------ finalize
+// One warp per alpha: lane l sums tiles l, l + 32, ... in that order, then a
+// fixed butterfly; the sums are deterministic.
 __global__ void __launch_bounds__(256)
 awq_finalize_kernel(const double* __restrict__ partial, int tiles, int n_alpha, const __half* __restrict__ S, int K,
                     double* loss_out, int32_t* best_out, __half* __restrict__ s_out, int* err) {
   __shared__ double loss[kAwqMaxAlpha];
   __shared__ int best;
   const int t = threadIdx.x;
-  if (t < n_alpha) {
+  const int lane = t & 31, warp = t >> 5;
+  for (int j = warp; j < n_alpha; j += blockDim.x >> 5) {
     double v = 0.0;
-    for (int i = 0; i < tiles; ++i) v += partial[(size_t)t * tiles + i];
-    loss[t] = v;
-    if (loss_out) loss_out[t] = v;
+    for (int i = lane; i < tiles; i += 32) v += partial[(size_t)j * tiles + i];
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    if (lane == 0) {
+      loss[j] = v;
+      if (loss_out) loss_out[j] = v;
+    }
   }
   __syncthreads();
   if (t == 0) {
@@ -382,7 +405,7 @@ cudaError_t launch_awq_search(const void* X, int64_t T, int64_t K, const void* c
   __half* E = reinterpret_cast<__half*>(ws + p.off_E);
   const __half* Xh = static_cast<const __half*>(X);
 
-  absmean_kernel<<<(unsigned)((K + 255) / 256), 256, 0, st>>>(Xh, (int)T, (int)K, mu);
+  absmean_kernel<<<(unsigned)((K + 31) / 32), 256, 0, st>>>(Xh, (int)T, (int)K, mu);
   AlphaList al;
   for (int j = 0; j < kAwqMaxAlpha; ++j) al.v[j] = j < n_alpha ? alpha[j] : 0.0;
   candidates_kernel<<<dim3((unsigned)((K + 255) / 256), (unsigned)n_alpha), 256, 0, st>>>(mu, (int)K, al, n_alpha,
@@ -506,7 +529,7 @@ cudaError_t launch_awq_search_noalloc(const void* X, int64_t T, int64_t K, const
   __half* E = reinterpret_cast<__half*>(ws + kAwqStaticMu + kAwqStaticS + kAwqStaticPartial);
   const __half* Xh = static_cast<const __half*>(X);
 
-  absmean_kernel<<<(unsigned)((K + 255) / 256), 256, 0, st>>>(Xh, (int)T, (int)K, mu);
+  absmean_kernel<<<(unsigned)((K + 31) / 32), 256, 0, st>>>(Xh, (int)T, (int)K, mu);
   AlphaList al;
   for (int j = 0; j < kAwqMaxAlpha; ++j) al.v[j] = j < n_alpha ? alpha[j] : 0.0;
   candidates_kernel<<<dim3((unsigned)((K + 255) / 256), (unsigned)n_alpha), 256, 0, st>>>(mu, (int)K, al, n_alpha,
