@@ -69,27 +69,32 @@ def load_peaks():
             "bf16_tflops_sustained": 1400.0, "source": "fallback"}
 
 
-def kernel_source_hash() -> str:
+# Source files of each kernel whose DRAM traffic the bench reports.
+KERNEL_SOURCES = {"gemv_rows_kernel": ("wq_gemv_rows.cu", "wq_common.cuh")}
+
+
+def kernel_source_hash(kernel: str = "gemv_rows_kernel") -> str:
+    """Hash of the files that define `kernel`: a stored traffic figure is
+    used only while they are unchanged."""
     h = hashlib.sha256()
     d = os.path.join(ROOT, "weight_only_quantization_group_b200", "csrc")
-    for name in sorted(os.listdir(d)):
-        if name.endswith((".cu", ".cuh")):
-            with open(os.path.join(d, name), "rb") as f:
-                h.update(name.encode())
-                h.update(f.read())
+    for name in KERNEL_SOURCES[kernel]:
+        with open(os.path.join(d, name), "rb") as f:
+            h.update(name.encode())
+            h.update(f.read())
     return h.hexdigest()[:16]
 
 
 def profiled_traffic(kernel: str):
     """Per-launch DRAM bytes of `kernel` from the committed ncu summary, if the
-    kernel sources have not changed since it was captured."""
+    kernel's sources have not changed since it was captured."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
     with open(p) as f:
         d = json.load(f)
     e = d.get(kernel)
-    if not e or e.get("source_hash") != kernel_source_hash():
+    if not e or kernel not in KERNEL_SOURCES or e.get("source_hash") != kernel_source_hash(kernel):
         return None
     return e.get("dram_bytes_per_launch")
 
