@@ -266,25 +266,50 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     h2d = xh_all.numel() * 2
     d2h = yh_all.numel() * 2
 
-    def e2e_step(blk):
+    def e2e_calls(blk):
         x_all.copy_(xh_all, non_blocking=True)
         for b, x, y in zip(blk, x_views, y_views):
             wq.wq_w4a16_gemm(x, *b["q"], b["N"], bits=4, out=y)
         yh_all.copy_(y_all, non_blocking=True)
+
+    # As a decode loop runs it: the step's calls (copy in, seven GEMVs, copy
+    # out) captured once per weight copy and replayed, then a host sync on the
+    # result; eagerly issued calls are timed too (row e2e_eager).
+    e2e_graphs = []
+    if not args.eager:
+        for blk in copies:
+            e2e_calls(blk)
+            torch.cuda.synchronize()
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=s_cap):
+                e2e_calls(blk)
+            e2e_graphs.append(g)
+        torch.cuda.synchronize()
+
+    def e2e_step(i, graphs):
+        if graphs:
+            graphs[i % n_copies].replay()
+        else:
+            e2e_calls(copies[i % n_copies])
         torch.cuda.current_stream().synchronize()
 
-    for i in range(3):
-        e2e_step(copies[i % n_copies])
-    barrier()
-    torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for i in range(e2e_steps):
-        e2e_step(copies[i % n_copies])
-    e1.record()
-    torch.cuda.synchronize()
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
+    def time_e2e(graphs):
+        for i in range(3):
+            e2e_step(i, graphs)
+        barrier()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for i in range(e2e_steps):
+            e2e_step(i, graphs)
+        e1.record()
+        torch.cuda.synchronize()
+        return max_over_ranks(e0.elapsed_time(e1), world, dev)
+
+    e2e_ms = time_e2e(e2e_graphs)
     e2e_value = world * step_bytes * e2e_steps / (e2e_ms * 1e-3) / 1e9
+    e2e_eager_ms = time_e2e([]) if e2e_graphs else e2e_ms
+    del e2e_graphs
 
     rows = {}
     if rank == 0 and not args.no_rows:
@@ -391,8 +416,13 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         },
         "e2e": {"value": round(e2e_value, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "steps": e2e_steps, "ms_per_step": e2e_ms / e2e_steps,
-                "path": "one pinned copy of the 7 inputs in, wq_w4a16_gemm per linear, one copy of the 7 outputs "
-                        "out, stream sync per step"},
+                "path": ("CUDA graph of the step's public calls: one pinned copy of the 7 inputs in, "
+                         "wq_w4a16_gemm per linear, one copy of the 7 outputs out; host sync on the result per step"
+                         if not args.eager else
+                         "one pinned copy of the 7 inputs in, wq_w4a16_gemm per linear, one copy of the 7 outputs "
+                         "out, stream sync per step"),
+                "eager_value": round(world * step_bytes * e2e_steps / (e2e_eager_ms * 1e-3) / 1e9, 2),
+                "eager_ms_per_step": e2e_eager_ms / e2e_steps},
         "gpu_launches": 7 * args.steps,
         "clocks": clocks,
         "rows": rows,
