@@ -312,6 +312,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     del e2e_graphs
 
     rows = {}
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if rank == 0 and not args.no_rows:
         # the same graphs' step time with programmatic dependent launch off
         wq.wq_set_option(wq.WQ_OPT_PDL, 0)
