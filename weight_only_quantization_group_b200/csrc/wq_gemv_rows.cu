@@ -404,7 +404,7 @@ __device__ __forceinline__ float butterfly_reduce(float (&v)[NV], int lane, int&
 
 // At most 8 warps: K <= 8192 with 32 channels per lane, K <= 16384 with 64.
 template <int M, int R, int CPL, int S, int BITS, template <int, int> class Act>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(256, M == 1 ? 2 : 1)
 gemv_rows_kernel(RowsArgs a) {
   constexpr int WPR = BITS * CPL;  // packed words per row and lane
   constexpr int NV = R * M;
