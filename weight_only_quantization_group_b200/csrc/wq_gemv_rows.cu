@@ -403,8 +403,10 @@ __device__ __forceinline__ float butterfly_reduce(float (&v)[NV], int lane, int&
 }
 
 // At most 8 warps: K <= 8192 with 32 channels per lane, K <= 16384 with 64.
-template <int M, int R, int CPL, int S, int BITS, template <int, int> class Act>
-__global__ void __launch_bounds__(256, M == 1 ? 2 : 1)
+// MINB: 2 caps the registers at 128 (the M = 1 instances: measured faster on
+// every layer shape, one more CTA per SM), else 1 (M = 2 would spill).
+template <int M, int R, int CPL, int S, int BITS, template <int, int> class Act, int MINB = 1>
+__global__ void __launch_bounds__(256, MINB)
 gemv_rows_kernel(RowsArgs a) {
   constexpr int WPR = BITS * CPL;  // packed words per row and lane
   constexpr int NV = R * M;
@@ -509,8 +511,8 @@ static long rows_grid(long nbatch, int occ, int mode) {
 
 template <int M, int R, int CPL, int S, int BITS, template <int, int> class Act>
 static cudaError_t launch_rows(const RowsArgs& a, cudaStream_t st, bool pdl, int grid_mode) {
-  auto kern = gemv_rows_kernel<M, R, CPL, S, BITS, Act>;
   const int nseg = (a.K + 1024 * CPL - 1) / (1024 * CPL);
+  auto kern = gemv_rows_kernel<M, R, CPL, S, BITS, Act, M == 1 ? 2 : 1>;
   const int threads = 32 * nseg;
   const size_t smem = 2 * (size_t)32 * nseg * sizeof(float);  // [2][32/NV][nseg][NV]
   int occ = 0;
