@@ -406,7 +406,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         },
         "roofline": {
             "bound": "hbm",
-            "kernel": "gemv_rows_kernel (ActHalf offset sums; R4 C32 S3 for K=4096, R4 C64 S2 for K=11008)",
+            "kernel": "gemv_rows_kernel (ActHalf offset sums; R4 C32 S2 for K=4096, R4 C64 S2 for K=11008)",
             "achieved": round(achieved, 2),
             "peak": peaks["hbm_gbs"],
             "peak_source": f"{peaks['source']} HBM copy bandwidth",

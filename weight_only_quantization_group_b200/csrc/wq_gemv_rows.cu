@@ -512,7 +512,7 @@ static long rows_grid(long nbatch, int occ, int mode) {
 template <int M, int R, int CPL, int S, int BITS, template <int, int> class Act>
 static cudaError_t launch_rows(const RowsArgs& a, cudaStream_t st, bool pdl, int grid_mode) {
   const int nseg = (a.K + 1024 * CPL - 1) / (1024 * CPL);
-  auto kern = gemv_rows_kernel<M, R, CPL, S, BITS, Act, M == 1 ? 2 : 1>;
+  auto kern = gemv_rows_kernel<M, R, CPL, S, BITS, Act, M == 1 ? (CPL == 1 && S == 2 ? 3 : 2) : 1>;
   const int threads = 32 * nseg;
   const size_t smem = 2 * (size_t)32 * nseg * sizeof(float);  // [2][32/NV][nseg][NV]
   int occ = 0;
@@ -575,7 +575,10 @@ cudaError_t launch_gemv_rows(const void* X, const uint32_t* packed, const void* 
   a.K = (int)K;
   if (bits == 3)
     return M == 1 ? launch_rows3<1>(a, st, pdl, shape, grid_mode) : launch_rows3<2>(a, st, pdl, shape, grid_mode);
-  if (shape == 0) shape = K <= 4096 ? 4 : 2;  // measured fastest on 4096- and 8192/11008-channel rows
+  // measured fastest on the LLaMA-2-7B block: 4096-channel rows take
+  // (4, 32, 2) at six CTAs per SM (an 85-register cap) for M = 1, (4, 32, 3)
+  // for M = 2; longer rows take (4, 64, 2)
+  if (shape == 0) shape = K <= 4096 ? (M == 1 ? 1 : 4) : 2;
   if (K > 8192 && (shape == 1 || shape == 4)) shape = 2;  // at most 8 warps
   return M == 1 ? launch_rows_shape<1>(a, st, pdl, act_int, shape, grid_mode)
                 : launch_rows_shape<2>(a, st, pdl, act_int, shape, grid_mode);
