@@ -575,10 +575,14 @@ cudaError_t launch_gemv_rows(const void* X, const uint32_t* packed, const void* 
   a.K = (int)K;
   if (bits == 3)
     return M == 1 ? launch_rows3<1>(a, st, pdl, shape, grid_mode) : launch_rows3<2>(a, st, pdl, shape, grid_mode);
-  // measured fastest on the LLaMA-2-7B block: 4096-channel rows take
-  // (4, 32, 2) at six CTAs per SM (an 85-register cap) for M = 1, (4, 32, 3)
-  // for M = 2; longer rows take (4, 64, 2)
-  if (shape == 0) shape = K <= 4096 ? (M == 1 ? 1 : 4) : 2;
+  // measured fastest: at M = 1, (4, 32, 2) under an 85-register cap for
+  // 4096-channel rows and for 8192-channel rows of at most 2^27 weights (more
+  // CTAs per SM), else (4, 64, 2) (fewer cross-warp sums per weight); at
+  // M = 2, (4, 32, 3) for 4096-channel rows, else (4, 64, 2)
+  if (shape == 0) {
+    if (M == 1) shape = (K <= 4096 || (K <= 8192 && N * K <= (int64_t(1) << 27))) ? 1 : 2;
+    else shape = K <= 4096 ? 4 : 2;
+  }
   if (K > 8192 && (shape == 1 || shape == 4)) shape = 2;  // at most 8 warps
   return M == 1 ? launch_rows_shape<1>(a, st, pdl, act_int, shape, grid_mode)
                 : launch_rows_shape<2>(a, st, pdl, act_int, shape, grid_mode);
