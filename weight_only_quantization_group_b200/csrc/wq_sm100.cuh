@@ -1,5 +1,5 @@
 // Thin inline-PTX wrappers for the sm_100a features the tensor-core kernels
-// use: mbarriers, TMA tile loads (no multicast), tensor-memory allocation,
+// use: mbarriers, TMA tile loads into the issuing CTA, tensor-memory allocation,
 // tcgen05 MMA / commit / load / store, and UMMA descriptors.
 #pragma once
 
