@@ -1,0 +1,109 @@
+"""Exact-arithmetic checks (CPU, rational numbers) of the two rounding
+arguments the quantizer relies on, independent of any CUDA code:
+
+* the quotient w / step is formed without a division as
+  q0 = RN(w y), r = w - step q0, q = RN(q0 + r y) (Markstein's correction),
+  with y any fp32 number within one ulp of 1/step (the kernel's reciprocal is
+  closer than that); for an fp16 step (11 significant bits) and the small
+  integer divisors 3, 7, 15, q must equal RN(w / step) exactly, r must be
+  representable in fp32, and the cases include exact ties and near-ties;
+* rint by adding 1.5 * 2^23 rounds to nearest with ties to even for |x| < 2^22.
+"""
+import random
+from fractions import Fraction as F
+
+import numpy as np
+import pytest
+
+
+def rn32(x: F) -> F:
+    """Round a rational to the nearest fp32 value, ties to even (normal range)."""
+    if x == 0:
+        return F(0)
+    sign = 1 if x > 0 else -1
+    a = abs(x)
+    e = a.numerator.bit_length() - a.denominator.bit_length()
+    while F(2) ** e > a:
+        e -= 1
+    while F(2) ** (e + 1) <= a:
+        e += 1
+    ulp = F(2) ** (max(e, -126) - 23)
+    q = a / ulp
+    fl = q.numerator // q.denominator
+    rem = q - fl
+    if rem > F(1, 2) or (rem == F(1, 2) and fl % 2 == 1):
+        fl += 1
+    return sign * fl * ulp
+
+
+def neighbours_of(x: F):
+    """The fp32 numbers that bracket x (both equal when x is representable)."""
+    y = rn32(x)
+    f = np.float32(float(y))
+    up = F(float(np.nextafter(f, np.float32(np.inf))))
+    dn = F(float(np.nextafter(f, np.float32(-np.inf))))
+    if y == x:
+        return [y]
+    return [y, up if y < x else dn]
+
+
+def corrected_quotient_ok(w: float, b: float) -> bool:
+    w, b = F(w), F(b)
+    for y in neighbours_of(1 / b):
+        q0 = rn32(w * y)
+        r = w - b * q0
+        if rn32(r) != r:
+            return False
+        if rn32(q0 + r * y) != rn32(w / b):
+            return False
+    return True
+
+
+def _fp16_positive():
+    v = np.arange(1, 0x7C00, dtype=np.uint16).view(np.float16).astype(np.float64)
+    return v[v > 0]
+
+
+@pytest.mark.filterwarnings("ignore:overflow encountered")
+def test_corrected_quotient_fp16_steps():
+    rng = random.Random(11)
+    steps = _fp16_positive()
+    n = 0
+    for i in range(3000):
+        b = float(rng.choice(steps))
+        kind = i % 3
+        if kind == 0:    # an fp16 weight, |w / step| < 16
+            w = float(np.float16(rng.uniform(-15.9, 15.9) * b))
+        elif kind == 1:  # an AWQ-scaled weight: fp16 x fp16, exact in fp32
+            w = float(np.float32(np.float16(rng.uniform(-4, 4) * b)) * np.float32(np.float16(rng.uniform(0.25, 4))))
+        else:            # a tie or a near-tie of a half-integer multiple of the step
+            k = rng.randint(-15, 14)
+            w = float(np.float32((k + 0.5) * b * (1 + rng.choice([0.0, 2.0 ** -23, -2.0 ** -23]))))
+        if not np.isfinite(w) or w == 0 or abs(w / b) >= 16:
+            continue
+        n += 1
+        assert corrected_quotient_ok(w, b), (w, b)
+    assert n > 2500
+
+
+@pytest.mark.parametrize("d", [3, 7, 15])
+def test_corrected_quotient_small_divisors(d):
+    rng = random.Random(d)
+    for _ in range(800):
+        a = float(np.float32(rng.uniform(0, 1) * 2.0 ** rng.randint(-40, 15)))
+        if a == 0:
+            continue
+        assert corrected_quotient_ok(a, d), a
+
+
+def test_round_by_magic_addition():
+    magic = F(12582912)  # 1.5 * 2^23
+    rng = random.Random(3)
+    xs = [F(k, 2) for k in range(-64, 65)]  # every half-integer tie in range
+    xs += [F(float(np.float32(rng.uniform(-1e4, 1e4)))) for _ in range(2000)]
+    for x in xs:
+        got = rn32(x + magic) - magic
+        fl = x.numerator // x.denominator
+        rem = x - fl
+        want = fl + (1 if rem > F(1, 2) or (rem == F(1, 2) and fl % 2 == 1) else 0)
+        assert got == want, x
