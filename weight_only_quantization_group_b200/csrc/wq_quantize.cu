@@ -37,15 +37,22 @@ template <int BITS, bool SYM, bool HAS_S>
 __device__ __forceinline__ void quantize_unit(const uint4 (&raw)[4], const __half* __restrict__ sk, int64_t u,
                                               bool valid, uint32_t* __restrict__ packed,
                                               __half* __restrict__ steps, __half* __restrict__ zeros, int* err) {
-  // with AWQ scaling the products w * s in fp32 (exact: 11 x 11 significand bits)
+  // with AWQ scaling the products w * s in fp32 (exact: 11 x 11 significand
+  // bits; a zero product is +0 whatever the signs, which no decision sees)
   float ws[HAS_S ? 32 : 1];
   GroupQuant gq;
   if constexpr (HAS_S) {
     uint4 sr[4];
 #pragma unroll
     for (int c = 0; c < 4; ++c) sr[c] = valid ? *reinterpret_cast<const uint4*>(sk + 8 * c) : make_uint4(0, 0, 0, 0);
+    // w * s straight from the fp16 pairs with the mixed fp16 x fp16 -> fp32
+    // fma (exact product, plus zero)
 #pragma unroll
-    for (int i = 0; i < 32; ++i) ws[i] = __fmul_rn(lane_half(raw, i), lane_half(sr, i));
+    for (int i = 0; i < 16; ++i) {
+      ws[2 * i] = 0.f;
+      ws[2 * i + 1] = 0.f;
+      fma2_f16_f32(ws[2 * i], ws[2 * i + 1], (&raw[i >> 2].x)[i & 3], (&sr[i >> 2].x)[i & 3]);
+    }
     gq = group_quant_decide<BITS, SYM, 32, 4>(ws);
   } else {
     gq = group_quant_decide_h<BITS, SYM, 4>(raw);
