@@ -8,10 +8,14 @@
 // Optional AWQ input-channel scaling W * diag(s) first ("MIT 6.5940 Lab 4 +
 // Lab 5", "Question 2").
 //
-// Mapping: 4 lanes per group, each lane owns 32 consecutive input channels
-// (four 16-byte loads of W; one 16-byte store of 4-bit codes, or the three
-// words of a 3-bit chunk); the group's range is reduced with two
-// xor-shuffles. 2 B/weight in, 0.5 (0.375) B/weight out.
+// Mapping: a lane unit is 32 consecutive input channels of one group, four
+// lanes per group (four 16-byte loads of W; one 16-byte store of 4-bit codes,
+// or the three words of a 3-bit chunk); the group's range is reduced with two
+// xor-shuffles. One wave of resident CTAs walks the units grid-stride, the
+// next unit's loads in flight while the current one is quantized. Per weight:
+// the correctly rounded quotient without a division (group_quotient), rint by
+// the 1.5 * 2^23 addition, and one integer multiply-add into the packed word.
+// 2 B/weight in, 0.5 (0.375) B/weight out.
 #include "wq_quant_core.cuh"
 
 namespace wq {
