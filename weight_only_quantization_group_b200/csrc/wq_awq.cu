@@ -16,8 +16,8 @@
 //                the group stacked row-wise (same decision code as the packer)
 //     awq_loss   tcgen05 GEMM D = E_j X^T per 128x128 tile, epilogue sums D^2
 //                in fp64 -> one partial per (alpha, tile)
-//   finalize     L_j = sum of partials in tile order (deterministic), first
-//                argmin, s_out = s_best
+//   finalize     L_j = sum of the partials, one warp per alpha in a fixed
+//                order (deterministic), first argmin, s_out = s_best
 #include <mutex>
 
 #include "wq_quant_core.cuh"
