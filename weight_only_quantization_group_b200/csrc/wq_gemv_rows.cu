@@ -403,8 +403,10 @@ __device__ __forceinline__ float butterfly_reduce(float (&v)[NV], int lane, int&
 }
 
 // At most 8 warps: K <= 8192 with 32 channels per lane, K <= 16384 with 64.
-// MINB: 2 caps the registers at 128 (the M = 1 instances: measured faster on
-// every layer shape, one more CTA per SM), else 1 (M = 2 would spill).
+// MINB: minimum CTAs per SM for the register allocation: 3 (85 registers)
+// for the M = 1, 32-channel, two-stage instance, 2 (128 registers) for the
+// other M = 1 instances (each measured faster, more CTAs per SM), 1 for M = 2
+// (a cap would spill).
 template <int M, int R, int CPL, int S, int BITS, template <int, int> class Act, int MINB = 1>
 __global__ void __launch_bounds__(256, MINB)
 gemv_rows_kernel(RowsArgs a) {
@@ -540,7 +542,7 @@ static cudaError_t launch_rows_act(const RowsArgs& a, cudaStream_t st, bool pdl,
 }
 
 // shape: rows per batch R, input channels per lane 32*CPL, register stages S
-//   0 = default (4 for K <= 4096, else 2), 1 = (4, 32, 2), 2 = (4, 64, 2), 3 = (2, 64, 2), 4 = (4, 32, 3).
+//   0 = default (see launch_gemv_rows), 1 = (4, 32, 2), 2 = (4, 64, 2), 3 = (2, 64, 2), 4 = (4, 32, 3).
 // Shapes with 32 channels per lane take K <= 8192; above that shape 2 runs.
 // act_int: integer digits (true) or fp16 FMA (false) for the lane's dot products.
 template <int M>
