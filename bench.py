@@ -26,6 +26,7 @@ import hashlib
 import json
 import math
 import os
+import re
 import statistics
 import subprocess
 import sys
@@ -73,15 +74,23 @@ def load_peaks():
 KERNEL_SOURCES = {"gemv_rows_kernel": ("wq_gemv_rows.cu", "wq_common.cuh")}
 
 
+def _code_only(text: str) -> str:
+    """C++ source without comments and whitespace."""
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", "", text)
+    return re.sub(r"\s+", "", text)
+
+
 def kernel_source_hash(kernel: str = "gemv_rows_kernel") -> str:
-    """Hash of the files that define `kernel`: a stored traffic figure is
-    used only while they are unchanged."""
+    """Hash of the code (comments and whitespace dropped) of the files that
+    define `kernel`: a stored traffic figure is used only while it is
+    unchanged."""
     h = hashlib.sha256()
     d = os.path.join(ROOT, "weight_only_quantization_group_b200", "csrc")
     for name in KERNEL_SOURCES[kernel]:
-        with open(os.path.join(d, name), "rb") as f:
+        with open(os.path.join(d, name), encoding="utf-8") as f:
             h.update(name.encode())
-            h.update(f.read())
+            h.update(_code_only(f.read()).encode())
     return h.hexdigest()[:16]
 
 
