@@ -107,3 +107,36 @@ def test_round_by_magic_addition():
         rem = x - fl
         want = fl + (1 if rem > F(1, 2) or (rem == F(1, 2) and fl % 2 == 1) else 0)
         assert got == want, x
+
+
+def _bits(v: float) -> int:
+    return int(np.array([v], dtype=np.float32).view(np.uint32)[0])
+
+
+@pytest.mark.parametrize("bits", [3, 4])
+def test_offset_level_packing_identity(bits):
+    """The packer adds the bit patterns of the offset levels 1.5*2^23 + (l - z),
+    each shifted to its field, and subtracts one constant per word:
+    sum_j (magic_bits << s_j) - z * sum_j (1 << s_j) (mod 2^32). Since the
+    levels l in [0, 2^b - 1] fill disjoint fields, the result must be the
+    packed word for every zero point z and every level pattern."""
+    magic, mbits = 12582912.0, 0x4B400000
+    rng = np.random.default_rng(bits)
+    if bits == 4:
+        shifts = [4 * (4 + (i >> 1) if i & 1 else i >> 1) for i in range(8)]  # slots [0,2,4,6,1,3,5,7]
+    else:
+        shifts = [3 * (i // 2) + (16 if i & 1 else 0) for i in range(10)]     # pairs at 3j and 16 + 3j
+    G = sum((mbits << s) & 0xFFFFFFFF for s in shifts) & 0xFFFFFFFF
+    U = sum(1 << s for s in shifts) & 0xFFFFFFFF
+    Q = (1 << bits) - 1
+    for z in range(Q + 1):
+        for _ in range(200):
+            lv = rng.integers(0, Q + 1, len(shifts))
+            acc = 0
+            for l, s in zip(lv, shifts):
+                acc = (acc + (_bits(magic + float(l) - float(z)) << s)) & 0xFFFFFFFF
+            word = (acc - ((G - z * U) & 0xFFFFFFFF)) & 0xFFFFFFFF
+            want = 0
+            for l, s in zip(lv, shifts):
+                want |= int(l) << s
+            assert word == want, (z, lv)
