@@ -141,3 +141,69 @@ def test_packed_weight_round_trip_and_header_checks(wq, tmp_path):
     torch.save(d, tmp_path / "bad.pt")
     with pytest.raises(ValueError):
         wq.load_packed(tmp_path / "bad.pt")
+
+
+def test_binding_checks_tensor_sizes_before_the_abi(wq):
+    """The C ABI takes bare pointers, so the binding checks every tensor's
+    dtype, contiguity and byte size first: a buffer too short for the call
+    (the kernels would read or write past its end) raises instead. CPU tensors
+    stand in for device ones; the device checks come after these."""
+    import torch
+    c = wq._cfg(4, 128, False)
+    N, K, M = 64, 512, 3
+    X = torch.zeros((M, K), dtype=torch.float16)
+    packed = torch.zeros(N * K // 8, dtype=torch.int32)
+    steps = torch.zeros((N, K // 128), dtype=torch.float16)
+    zeros = torch.zeros((N, K // 128), dtype=torch.float16)
+    out = torch.zeros((M, N), dtype=torch.float16)
+    wq._gemm_operands(X, packed, steps, zeros, N, c, out)  # exact sizes pass
+    wq._gemm_operands(X, packed.view(torch.uint8), steps, zeros, N, c, None)  # any integer view of the words
+    with pytest.raises(ValueError, match="packed holds"):
+        wq._gemm_operands(X, packed[:-1], steps, zeros, N, c, out)
+    with pytest.raises(ValueError, match="packed holds"):
+        wq._gemm_operands(X, packed, steps, zeros, N + 1, c, None)   # N larger than the weight
+    with pytest.raises(ValueError, match="steps holds"):
+        wq._gemm_operands(X, packed, steps[:-1], zeros, N, c, out)
+    with pytest.raises(TypeError, match="zeros must be"):
+        wq._gemm_operands(X, packed, steps, zeros.float(), N, c, out)
+    with pytest.raises(ValueError, match="out holds"):
+        wq._gemm_operands(X, packed, steps, zeros, N, c, out[:-1])
+    with pytest.raises(ValueError, match="contiguous"):
+        wq._gemm_operands(X, packed, steps.t(), zeros, N, c, out)
+    with pytest.raises(ValueError, match=r"X must be \[M\]\[K\]"):
+        wq._gemm_operands(X[0], packed, steps, zeros, N, c, out)
+    with pytest.raises(TypeError, match="must be a torch.Tensor"):
+        wq._gemm_operands(X, list(range(8)), steps, zeros, N, c, out)
+    # 3-bit: three words per 32 channels
+    c3 = wq._cfg(3, 128, False)
+    p3 = torch.zeros(N * K * 3 // 32 // 4, dtype=torch.int32)   # a quarter of what is needed
+    with pytest.raises(ValueError, match="packed holds"):
+        wq._quant_operands(N, K, c3, p3, steps, zeros)
+    wq._quant_operands(N, K, c3, torch.zeros(N * K * 3 // 32, dtype=torch.int32), steps, zeros)
+    # an invalid shape needs nothing here: the library reports it itself
+    wq._quant_operands(N, 200, c, packed[:0], steps[:0], zeros[:0])
+
+
+def test_binding_checks_awq_shapes(wq):
+    import torch
+    X = torch.zeros((16, 256), dtype=torch.float16)
+    wq._awq_operands(X, [torch.zeros((8, 256), dtype=torch.float16)] * 2)
+    with pytest.raises(ValueError, match=r"W\[1\] must be \[N\]\[256\]"):
+        wq._awq_operands(X, [torch.zeros((8, 256), dtype=torch.float16), torch.zeros((8, 128), dtype=torch.float16)])
+    with pytest.raises(ValueError, match="at least one weight"):
+        wq._awq_operands(X, [])
+    with pytest.raises(ValueError, match=r"X must be \[T\]\[K\]"):
+        wq._awq_operands(X.view(-1), [torch.zeros((8, 256), dtype=torch.float16)])
+
+
+def test_binding_checks_devices(wq):
+    """Every tensor of a call must live on the first operand's device."""
+    import torch
+    a = torch.zeros(4)
+    wq._on_device_of(a, b=torch.zeros(2), c=None)
+    with pytest.raises(ValueError, match="must be a CUDA tensor on cpu, got meta"):
+        wq._on_device_of(a, b=torch.zeros(2, device="meta"))
+    N, K = 8, 256  # a host buffer never reaches the ABI as a device pointer
+    with pytest.raises(ValueError, match="packed must be a CUDA tensor"):
+        wq.wq_unpack_dequant(torch.zeros(N * K // 8, dtype=torch.int32), torch.zeros((N, 2), dtype=torch.float16),
+                             torch.zeros((N, 2), dtype=torch.float16), N, K)

@@ -191,6 +191,75 @@ def _check(t: torch.Tensor, dtype, name: str):
         raise ValueError(f"{name} must be contiguous")
 
 
+def _need(t, name: str, dtype, nbytes: int):
+    """t: a contiguous tensor (of `dtype`, when given) holding at least
+    `nbytes` bytes. The C ABI receives bare pointers, so a short buffer would
+    be read or written past its end; these checks run before it is called
+    (one combined test on the common path, the precise error otherwise)."""
+    try:
+        if (dtype is None or t.dtype == dtype) and t.is_contiguous() and t.nbytes >= nbytes:
+            return
+    except AttributeError:
+        raise TypeError(f"{name} must be a torch.Tensor") from None
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    raise ValueError(f"{name} holds {t.nbytes} bytes; this call needs {nbytes}")
+
+
+def _on_device_of(ref: torch.Tensor, **named):
+    """Every named tensor lives on ref's device (ref is a CUDA tensor)."""
+    dev = ref.device
+    for name, t in named.items():
+        if t is not None and t.device != dev:
+            raise ValueError(f"{name} must be a CUDA tensor on {dev}, got {t.device}")
+
+
+_NW_CACHE: dict = {}
+
+
+def _packed_words_of(N: int, K: int, c: "_Cfg") -> int:
+    key = (N, K, c.bits, c.group_size, c.symmetric)
+    nw = _NW_CACHE.get(key)
+    if nw is None:
+        nw = _NW_CACHE[key] = int(_lib.wq_packed_words(N, K, ctypes.byref(c)))
+    return nw
+
+
+def _quant_operands(N: int, K: int, c: "_Cfg", packed, steps, zeros):
+    """Sizes of the packed form of an [N][K] weight (0 when the config or the
+    shape is invalid: the library reports those itself)."""
+    nw = _packed_words_of(N, K, c)
+    G = K // c.group_size if nw > 0 else 0
+    _need(packed, "packed", None, 4 * nw)
+    _need(steps, "steps", torch.float16, 2 * N * G)
+    _need(zeros, "zeros", torch.float16, 2 * N * G)
+
+
+def _gemm_operands(X, packed, steps, zeros, N: int, c: "_Cfg", out):
+    """The tensors of wq_w4a16_gemm: X [M][K] fp16, the packed weight of an
+    [N][K] matrix, and out (fp16, M*N values) when given."""
+    if X.dim() != 2:
+        raise ValueError(f"X must be [M][K], got shape {tuple(X.shape)}")
+    M, K = X.shape
+    _quant_operands(N, K, c, packed, steps, zeros)
+    if out is not None:
+        _need(out, "out", torch.float16, 2 * M * N)
+
+
+def _awq_operands(X, Ws):
+    """X [T][K] and every W [N_i][K] (the same K)."""
+    if X.dim() != 2:
+        raise ValueError(f"X must be [T][K], got shape {tuple(X.shape)}")
+    K = X.shape[1]
+    if len(Ws) == 0:
+        raise ValueError("at least one weight is needed")
+    for i, W in enumerate(Ws):
+        if W.dim() != 2 or W.shape[1] != K:
+            raise ValueError(f"W[{i}] must be [N][{K}], got shape {tuple(W.shape)}")
+
+
 def _raise(st: int, where: str):
     if st != WQ_OK:
         raise WQError(st, where)
@@ -244,9 +313,12 @@ def wq_quantize_pack(W: torch.Tensor, s: torch.Tensor | None = None, *, bits: in
                      symmetric: bool = False, out=None, stream=None):
     """Quantize + pack an fp16 [N][K] weight; returns (packed u32 as int32, steps, zeros)."""
     _check(W, torch.float16, "W")
+    if W.dim() != 2:
+        raise ValueError(f"W must be [N][K], got shape {tuple(W.shape)}")
+    N, K = W.shape
     if s is not None:
         _check(s, torch.float16, "s")
-    N, K = W.shape
+        _need(s, "s", torch.float16, 2 * K)
     c = _cfg(bits, group_size, symmetric)
     nw = int(_lib.wq_packed_words(N, K, ctypes.byref(c)))
     if out is None:
@@ -256,6 +328,8 @@ def wq_quantize_pack(W: torch.Tensor, s: torch.Tensor | None = None, *, bits: in
         zeros = torch.empty((N, G), dtype=torch.float16, device=W.device)
     else:
         packed, steps, zeros = out
+        _quant_operands(N, K, c, packed, steps, zeros)
+    _on_device_of(W, s=s, packed=packed, steps=steps, zeros=zeros)
     st = _lib.wq_quantize_pack(_ptr(W), _ptr(s), N, K, ctypes.byref(c), _ptr(packed), _ptr(steps),
                                _ptr(zeros), _stream(stream))
     _raise(st, "wq_quantize_pack")
@@ -266,8 +340,13 @@ def wq_unpack_dequant(packed: torch.Tensor, steps: torch.Tensor, zeros: torch.Te
                       bits: int = 4, group_size: int = 128, symmetric: bool = False, out=None, stream=None):
     """fp16 [N][K] = fp16((q - zero) * step) from the packed form."""
     c = _cfg(bits, group_size, symmetric)
+    _quant_operands(N, K, c, packed, steps, zeros)
+    if not packed.is_cuda:
+        raise ValueError("packed must be a CUDA tensor")
     if out is None:
         out = torch.empty((N, K), dtype=torch.float16, device=packed.device)
+    _need(out, "out", torch.float16, 2 * N * K)
+    _on_device_of(packed, steps=steps, zeros=zeros, out=out)
     st = _lib.wq_unpack_dequant(_ptr(packed), _ptr(steps), _ptr(zeros), N, K, ctypes.byref(c), _ptr(out),
                                 _stream(stream))
     _raise(st, "wq_unpack_dequant")
@@ -285,10 +364,12 @@ def wq_w4a16_gemm(X: torch.Tensor, packed: torch.Tensor, steps: torch.Tensor, ze
                   stream=None):
     """Y[M][N] = X[M][K] * deq(W)^T with fp32 accumulation; returns Y (fp16)."""
     _check(X, torch.float16, "X")
-    M, K = X.shape
     c = _cfg(bits, group_size, symmetric)
+    _gemm_operands(X, packed, steps, zeros, N, c, out)
+    M, K = X.shape
     if out is None:
         out = torch.empty((M, N), dtype=torch.float16, device=X.device)
+    _on_device_of(X, packed=packed, steps=steps, zeros=zeros, out=out, workspace=workspace)
     ws_ptr, ws_bytes = None, 0
     if workspace is not None:
         ws_ptr, ws_bytes = workspace.data_ptr(), workspace.numel() * workspace.element_size()
@@ -327,6 +408,8 @@ def wq_awq_scale_search(X: torch.Tensor, Ws, alphas=None, *, bits: int = 4, grou
     _check(X, torch.float16, "X")
     for i, W in enumerate(Ws):
         _check(W, torch.float16, f"W[{i}]")
+    _awq_operands(X, Ws)
+    _on_device_of(X, **{f"W[{i}]": W for i, W in enumerate(Ws)}, workspace=workspace)
     T, K = X.shape
     if alphas is None:
         alphas = [j / 20.0 for j in range(20)]
@@ -339,6 +422,8 @@ def wq_awq_scale_search(X: torch.Tensor, Ws, alphas=None, *, bits: int = 4, grou
     need = int(_lib.wq_awq_workspace_bytes(T, K, n_arr, len(Ns), len(alphas), ctypes.byref(c)))
     if workspace is None:
         workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=X.device)
+    elif not workspace.is_contiguous():
+        raise ValueError("workspace must be contiguous")
     s = torch.empty(K, dtype=torch.float16, device=X.device)
     mu = torch.empty(K, dtype=torch.float64, device=X.device)
     losses = torch.empty(len(alphas), dtype=torch.float64, device=X.device)
@@ -359,6 +444,8 @@ def wq_awq_scale_search_noalloc(X: torch.Tensor, Ws, alphas=None, *, bits: int =
     _check(X, torch.float16, "X")
     for i, W in enumerate(Ws):
         _check(W, torch.float16, f"W[{i}]")
+    _awq_operands(X, Ws)
+    _on_device_of(X, **{f"W[{i}]": W for i, W in enumerate(Ws)})
     T, K = X.shape
     if alphas is None:
         alphas = [j / 20.0 for j in range(20)]
@@ -373,6 +460,12 @@ def wq_awq_scale_search_noalloc(X: torch.Tensor, Ws, alphas=None, *, bits: int =
                "mu": torch.empty(K, dtype=torch.float64, device=X.device),
                "losses": torch.empty(len(alphas), dtype=torch.float64, device=X.device),
                "best": torch.empty(1, dtype=torch.int32, device=X.device)}
+    else:
+        _need(out["s"], "out['s']", torch.float16, 2 * K)
+        _need(out["mu"], "out['mu']", torch.float64, 8 * K)
+        _need(out["losses"], "out['losses']", torch.float64, 8 * len(alphas))
+        _need(out["best"], "out['best']", torch.int32, 4)
+        _on_device_of(X, **{f"out['{k}']": out[k] for k in ("s", "mu", "losses", "best")})
     st = _lib.wq_awq_scale_search_noalloc(_ptr(X), T, K, w_arr, n_arr, len(Ns), ctypes.byref(c), a_arr,
                                           len(alphas), _ptr(out["s"]), _ptr(out["mu"]), _ptr(out["losses"]),
                                           _ptr(out["best"]), _stream(stream))
