@@ -207,3 +207,20 @@ def test_binding_checks_devices(wq):
     with pytest.raises(ValueError, match="packed must be a CUDA tensor"):
         wq.wq_unpack_dequant(torch.zeros(N * K // 8, dtype=torch.int32), torch.zeros((N, 2), dtype=torch.float16),
                              torch.zeros((N, 2), dtype=torch.float16), N, K)
+
+
+def test_awq_workspace_size_is_its_layout(wq):
+    """wq_awq_workspace_bytes is the sum of the search's regions, each rounded
+    up to 256 bytes: mu (fp64 [K]), the candidates (fp16 [n_alpha][K]), one
+    fp64 partial loss per (alpha, 128x128 tile), and the fp16 error matrices
+    of one batch of alphas (as many as fit 1 GiB, at least one)."""
+    def a256(x):
+        return (x + 255) // 256 * 256
+
+    for T, K, Ns, n_alpha in [(512, 4096, [4096] * 3, 20), (8, 256, [16], 20), (131, 640, [1, 129, 7], 6),
+                              (512, 11008, [4096], 20)]:
+        N = sum(Ns)
+        tiles = -(-T // 128) * -(-N // 128)
+        batch = max(1, min(n_alpha, (1 << 30) // (N * K * 2)))
+        want = a256(K * 8) + a256(n_alpha * K * 2) + a256(n_alpha * tiles * 8) + a256(batch * N * K * 2)
+        assert wq.wq_awq_workspace_bytes(T, K, Ns, n_alpha) == want, (T, K, Ns)

@@ -5,39 +5,7 @@
 #include <nvtx3/nvToolsExt.h>
 
 #include "wq_common.cuh"
-
-namespace wq {
-cudaError_t launch_quantize_pack(const void* W, const void* s, int64_t N, int64_t K, int bits, bool sym,
-                                 uint32_t* packed, void* steps, void* zeros, int* err, cudaStream_t st);
-cudaError_t launch_unpack_dequant(const uint32_t* packed, const void* steps, const void* zeros, int64_t N,
-                                  int64_t K, int bits, void* out, cudaStream_t st);
-cudaError_t launch_gemv(const void* X, const uint32_t* packed, const void* steps, const void* zeros, int64_t M,
-                        int64_t N, int64_t K, int bits, void* Y, cudaStream_t st, int variant, bool pdl);
-size_t gemv_smem_bytes(int bits, int variant, int M, int N, int K);
-bool gemv_rows_supported(int bits, int64_t M, int64_t K);
-cudaError_t launch_gemv_rows(const void* X, const uint32_t* packed, const void* steps, const void* zeros, int64_t M,
-                             int64_t N, int64_t K, int bits, void* Y, cudaStream_t st, int shape, bool act_int,
-                             int grid_mode, bool pdl);
-cudaError_t launch_gemm_tc(const void* X, const uint32_t* packed, const void* steps, const void* zeros, int64_t M,
-                           int64_t N, int64_t K, void* Y, int* err, cudaStream_t st, int stages_opt, int bk_opt,
-                           int dw_opt, int wait_ms, bool stall);
-struct AwqPlan {
-  int64_t N_total;
-  int t_tiles, n_tiles, tiles;
-  int batch;
-  size_t off_mu, off_S, off_partial, off_E, total;
-};
-AwqPlan plan_awq(int64_t T, int64_t K, const int64_t* N_i, int n_lin, int n_alpha);
-cudaError_t launch_awq_search(const void* X, int64_t T, int64_t K, const void* const* W, const int64_t* N_i,
-                              int n_lin, int bits, bool sym, const double* alpha, int n_alpha, void* s_out,
-                              double* mu_out, double* loss_out, int32_t* best_out, void* workspace, int* err,
-                              cudaStream_t st);
-bool awq_noalloc_fits(int64_t T, int64_t K, int64_t N_total, int n_alpha);
-cudaError_t launch_awq_search_noalloc(const void* X, int64_t T, int64_t K, const void* const* W,
-                                      const int64_t* N_i, int n_lin, int bits, bool sym, const double* alpha,
-                                      int n_alpha, void* s_out, double* mu_out, double* loss_out, int32_t* best_out,
-                                      int* err, cudaStream_t st);
-}  // namespace wq
+#include "wq_launch.h"
 
 // One flag per device (each device holds its own copy of a __device__ variable).
 __device__ int g_wq_device_error;

@@ -22,6 +22,7 @@
 
 #include "wq_quant_core.cuh"
 #include "wq_sm100.cuh"
+#include "wq_launch.h"
 
 namespace wq {
 
@@ -356,13 +357,6 @@ static EncodeTiledFnA awq_encode_fn() {
   }
   return fn;
 }
-
-struct AwqPlan {
-  int64_t N_total;
-  int t_tiles, n_tiles, tiles;
-  int batch;  // alphas per E batch
-  size_t off_mu, off_S, off_partial, off_E, total;
-};
 
 static size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 

@@ -28,6 +28,7 @@
 #include <type_traits>
 
 #include "wq_sm100.cuh"
+#include "wq_launch.h"
 
 namespace wq {
 

@@ -31,6 +31,7 @@
 #include <cooperative_groups.h>
 
 #include "wq_common.cuh"
+#include "wq_launch.h"
 
 namespace cg = cooperative_groups;
 

@@ -37,6 +37,7 @@
 //     The offsets and the zero point are removed per row with the lane's
 //     activation class sums.
 #include "wq_common.cuh"
+#include "wq_launch.h"
 
 namespace wq {
 

@@ -17,6 +17,7 @@
 // the 1.5 * 2^23 addition, and one integer multiply-add into the packed word.
 // 2 B/weight in, 0.5 (0.375) B/weight out.
 #include "wq_quant_core.cuh"
+#include "wq_launch.h"
 
 namespace wq {
 
