@@ -200,7 +200,9 @@ int32_t wq_awq_scale_search_noalloc(const void* X_dev, int64_t T, int64_t K, con
                                     double* mu_out_dev, double* loss_out_dev, int32_t* best_out_dev,
                                     void* stream);
 
-/* Process-wide tuning options (not thread-safe against concurrent calls).
+/* Process-wide tuning options. Each is an atomic value, so a thread may set
+ * one while another calls the library; a call reads each option it uses
+ * once, so it runs wholly under the old or wholly under the new value.
  *  WQ_OPT_GEMM_PATH     WQ_PATH_AUTO (default): GEMV kernel below the
  *                       crossover M, tensor-core kernel at or above it (4-bit);
  *                       WQ_PATH_GEMV / WQ_PATH_TENSOR_CORE force one kernel

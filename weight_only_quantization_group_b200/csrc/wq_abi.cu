@@ -1,6 +1,7 @@
 // C ABI of libwq.so: argument validation, dispatch, and the device error flag.
 // Every entry point validates on the host, enqueues on the caller's stream and
 // returns; none allocates device memory.
+#include <atomic>
 #include <mutex>
 #include <nvtx3/nvToolsExt.h>
 
@@ -57,19 +58,20 @@ int32_t check_shape(int64_t N, int64_t K) {
 
 int32_t cuda_status(cudaError_t e) { return e == cudaSuccess ? WQ_OK : WQ_ERR_CUDA; }
 
-// Process-wide tuning options (wq_set_option).
-int64_t g_opt_gemm_path = WQ_PATH_AUTO;
-int64_t g_opt_crossover_m = 3;
-int64_t g_opt_pdl = 1;
-int64_t g_opt_gemv_variant = WQ_GEMV_OFFSET_SUMS;
-int64_t g_opt_gemv_kernel = WQ_GEMV_KERNEL_AUTO;
-int64_t g_opt_gemv_rows_shape = 0;
-int64_t g_opt_tc_stages = 0;
-int64_t g_opt_gemv_grid = 1;
-int64_t g_opt_tc_bk = 0;
-int64_t g_opt_tc_dequant_warps = 0;
-int64_t g_opt_wait_limit_ms = 2000;
-int64_t g_opt_test_stall = 0;
+// Process-wide tuning options (wq_set_option). Atomic, so setting one from
+// another thread is not a data race; a call reads each option once.
+std::atomic<int64_t> g_opt_gemm_path{WQ_PATH_AUTO};
+std::atomic<int64_t> g_opt_crossover_m{3};
+std::atomic<int64_t> g_opt_pdl{1};
+std::atomic<int64_t> g_opt_gemv_variant{WQ_GEMV_OFFSET_SUMS};
+std::atomic<int64_t> g_opt_gemv_kernel{WQ_GEMV_KERNEL_AUTO};
+std::atomic<int64_t> g_opt_gemv_rows_shape{0};
+std::atomic<int64_t> g_opt_tc_stages{0};
+std::atomic<int64_t> g_opt_gemv_grid{1};
+std::atomic<int64_t> g_opt_tc_bk{0};
+std::atomic<int64_t> g_opt_tc_dequant_warps{0};
+std::atomic<int64_t> g_opt_wait_limit_ms{2000};
+std::atomic<int64_t> g_opt_test_stall{0};
 
 }  // namespace
 
@@ -143,9 +145,11 @@ int32_t wq_w4a16_gemm(const void* X, const uint32_t* packed, const void* steps, 
   if (!X || !packed || !steps || !zeros || !Y) return WQ_ERR_INVALID_ARG;
   if (!aligned(X, 16) || !aligned(packed, 16) || !aligned(steps, 2) || !aligned(zeros, 2) || !aligned(Y, 2))
     return WQ_ERR_ALIGNMENT;
+  // one reading of every option this call uses
+  const int64_t path = g_opt_gemm_path, variant = g_opt_gemv_variant, pdl = g_opt_pdl;
   bool tensor_core = cfg->bits == 4 && M >= g_opt_crossover_m;
-  if (g_opt_gemm_path == WQ_PATH_GEMV) tensor_core = false;
-  if (g_opt_gemm_path == WQ_PATH_TENSOR_CORE) {
+  if (path == WQ_PATH_GEMV) tensor_core = false;
+  if (path == WQ_PATH_TENSOR_CORE) {
     if (cfg->bits != 4) return WQ_ERR_UNSUPPORTED;
     tensor_core = true;
   }
@@ -157,20 +161,19 @@ int32_t wq_w4a16_gemm(const void* X, const uint32_t* packed, const void* steps, 
                                           (int)g_opt_tc_bk, (int)g_opt_tc_dequant_warps,
                                           (int)g_opt_wait_limit_ms, g_opt_test_stall != 0));
   }
-  if (g_opt_gemv_kernel != WQ_GEMV_KERNEL_TILED && g_opt_gemv_variant != WQ_GEMV_EXACT &&
+  if (g_opt_gemv_kernel != WQ_GEMV_KERNEL_TILED && variant != WQ_GEMV_EXACT &&
       wq::gemv_rows_supported(cfg->bits, M, K))
     return cuda_status(wq::launch_gemv_rows(X, packed, steps, zeros, M, N, K, cfg->bits, Y,
                                             static_cast<cudaStream_t>(stream),
-                                            (int)g_opt_gemv_rows_shape, g_opt_gemv_variant == WQ_GEMV_INT_DIGITS,
-                                            (int)g_opt_gemv_grid, g_opt_pdl != 0));
-  // The shared copy of an X slice must fit one CTA.
-  if (wq::gemv_smem_bytes(cfg->bits, g_opt_gemv_variant == WQ_GEMV_EXACT ? WQ_GEMV_EXACT : WQ_GEMV_OFFSET_SUMS,
-                          (int)(M < 8 ? M : 8), (int)N, (int)K) > 200 * 1024)
-    return WQ_ERR_UNSUPPORTED;
+                                            (int)g_opt_gemv_rows_shape, variant == WQ_GEMV_INT_DIGITS,
+                                            (int)g_opt_gemv_grid, pdl != 0));
   // the tiled kernel forms the integer-digit variant's sums as offset sums
-  const int tiled_variant = g_opt_gemv_variant == WQ_GEMV_EXACT ? WQ_GEMV_EXACT : WQ_GEMV_OFFSET_SUMS;
+  const int tiled_variant = variant == WQ_GEMV_EXACT ? WQ_GEMV_EXACT : WQ_GEMV_OFFSET_SUMS;
+  // The shared copy of an X slice must fit one CTA.
+  if (wq::gemv_smem_bytes(cfg->bits, tiled_variant, (int)(M < 8 ? M : 8), (int)N, (int)K) > 200 * 1024)
+    return WQ_ERR_UNSUPPORTED;
   return cuda_status(wq::launch_gemv(X, packed, steps, zeros, M, N, K, cfg->bits, Y,
-                                     static_cast<cudaStream_t>(stream), tiled_variant, g_opt_pdl != 0));
+                                     static_cast<cudaStream_t>(stream), tiled_variant, pdl != 0));
 }
 
 static int32_t check_awq(int64_t T, int64_t K, const int64_t* N_i, int32_t n_lin, int32_t n_alpha,
