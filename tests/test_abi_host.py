@@ -203,6 +203,8 @@ def test_binding_checks_devices(wq):
     wq._on_device_of(a, b=torch.zeros(2), c=None)
     with pytest.raises(ValueError, match="must be a CUDA tensor on cpu, got meta"):
         wq._on_device_of(a, b=torch.zeros(2, device="meta"))
+    import contextlib
+    assert isinstance(wq._device_of(a), contextlib.nullcontext)  # nothing to switch for a host tensor
     N, K = 8, 256  # a host buffer never reaches the ABI as a device pointer
     with pytest.raises(ValueError, match="packed must be a CUDA tensor"):
         wq.wq_unpack_dequant(torch.zeros(N * K // 8, dtype=torch.int32), torch.zeros((N, 2), dtype=torch.float16),

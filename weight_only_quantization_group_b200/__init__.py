@@ -9,6 +9,7 @@ computation runs in the library's CUDA kernels; there is no CPU fallback.
 """
 from __future__ import annotations
 
+import contextlib
 import ctypes
 import os
 
@@ -176,6 +177,15 @@ def _stream(stream, device=None) -> int:
     return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
 
 
+def _device_of(t: torch.Tensor):
+    """A context making t's device the current one for the call: the library
+    launches on the current device, and the tensors may live on another."""
+    idx = t.device.index
+    if idx is None or idx == torch.cuda.current_device():
+        return contextlib.nullcontext()
+    return torch.cuda.device(idx)
+
+
 def _ptr(t: torch.Tensor | None) -> int | None:
     return None if t is None else t.data_ptr()
 
@@ -330,8 +340,9 @@ def wq_quantize_pack(W: torch.Tensor, s: torch.Tensor | None = None, *, bits: in
         packed, steps, zeros = out
         _quant_operands(N, K, c, packed, steps, zeros)
     _on_device_of(W, s=s, packed=packed, steps=steps, zeros=zeros)
-    st = _lib.wq_quantize_pack(_ptr(W), _ptr(s), N, K, ctypes.byref(c), _ptr(packed), _ptr(steps),
-                               _ptr(zeros), _stream(stream))
+    with _device_of(W):
+        st = _lib.wq_quantize_pack(_ptr(W), _ptr(s), N, K, ctypes.byref(c), _ptr(packed), _ptr(steps),
+                                   _ptr(zeros), _stream(stream, W.device.index))
     _raise(st, "wq_quantize_pack")
     return packed, steps, zeros
 
@@ -347,8 +358,9 @@ def wq_unpack_dequant(packed: torch.Tensor, steps: torch.Tensor, zeros: torch.Te
         out = torch.empty((N, K), dtype=torch.float16, device=packed.device)
     _need(out, "out", torch.float16, 2 * N * K)
     _on_device_of(packed, steps=steps, zeros=zeros, out=out)
-    st = _lib.wq_unpack_dequant(_ptr(packed), _ptr(steps), _ptr(zeros), N, K, ctypes.byref(c), _ptr(out),
-                                _stream(stream))
+    with _device_of(packed):
+        st = _lib.wq_unpack_dequant(_ptr(packed), _ptr(steps), _ptr(zeros), N, K, ctypes.byref(c), _ptr(out),
+                                    _stream(stream, packed.device.index))
     _raise(st, "wq_unpack_dequant")
     return out
 
@@ -373,8 +385,9 @@ def wq_w4a16_gemm(X: torch.Tensor, packed: torch.Tensor, steps: torch.Tensor, ze
     ws_ptr, ws_bytes = None, 0
     if workspace is not None:
         ws_ptr, ws_bytes = workspace.data_ptr(), workspace.numel() * workspace.element_size()
-    st = lib().wq_w4a16_gemm(X.data_ptr(), packed.data_ptr(), steps.data_ptr(), zeros.data_ptr(), M, N, K,
-                             ctypes.byref(c), out.data_ptr(), ws_ptr, ws_bytes, _stream(stream, X.device.index))
+    with _device_of(X):
+        st = lib().wq_w4a16_gemm(X.data_ptr(), packed.data_ptr(), steps.data_ptr(), zeros.data_ptr(), M, N, K,
+                                 ctypes.byref(c), out.data_ptr(), ws_ptr, ws_bytes, _stream(stream, X.device.index))
     _raise(st, "wq_w4a16_gemm")
     return out
 
@@ -428,9 +441,10 @@ def wq_awq_scale_search(X: torch.Tensor, Ws, alphas=None, *, bits: int = 4, grou
     mu = torch.empty(K, dtype=torch.float64, device=X.device)
     losses = torch.empty(len(alphas), dtype=torch.float64, device=X.device)
     best = torch.empty(1, dtype=torch.int32, device=X.device)
-    st = _lib.wq_awq_scale_search(_ptr(X), T, K, w_arr, n_arr, len(Ns), ctypes.byref(c), a_arr, len(alphas),
-                                  _ptr(s), _ptr(mu), _ptr(losses), _ptr(best), workspace.data_ptr(),
-                                  workspace.numel() * workspace.element_size(), _stream(stream))
+    with _device_of(X):
+        st = _lib.wq_awq_scale_search(_ptr(X), T, K, w_arr, n_arr, len(Ns), ctypes.byref(c), a_arr, len(alphas),
+                                      _ptr(s), _ptr(mu), _ptr(losses), _ptr(best), workspace.data_ptr(),
+                                      workspace.numel() * workspace.element_size(), _stream(stream, X.device.index))
     _raise(st, "wq_awq_scale_search")
     return {"s": s, "mu": mu, "losses": losses, "best": best}
 
@@ -466,8 +480,9 @@ def wq_awq_scale_search_noalloc(X: torch.Tensor, Ws, alphas=None, *, bits: int =
         _need(out["losses"], "out['losses']", torch.float64, 8 * len(alphas))
         _need(out["best"], "out['best']", torch.int32, 4)
         _on_device_of(X, **{f"out['{k}']": out[k] for k in ("s", "mu", "losses", "best")})
-    st = _lib.wq_awq_scale_search_noalloc(_ptr(X), T, K, w_arr, n_arr, len(Ns), ctypes.byref(c), a_arr,
-                                          len(alphas), _ptr(out["s"]), _ptr(out["mu"]), _ptr(out["losses"]),
-                                          _ptr(out["best"]), _stream(stream))
+    with _device_of(X):
+        st = _lib.wq_awq_scale_search_noalloc(_ptr(X), T, K, w_arr, n_arr, len(Ns), ctypes.byref(c), a_arr,
+                                              len(alphas), _ptr(out["s"]), _ptr(out["mu"]), _ptr(out["losses"]),
+                                              _ptr(out["best"]), _stream(stream, X.device.index))
     _raise(st, "wq_awq_scale_search_noalloc")
     return out
