@@ -226,3 +226,18 @@ def test_awq_workspace_size_is_its_layout(wq):
         batch = max(1, min(n_alpha, (1 << 30) // (N * K * 2)))
         want = a256(K * 8) + a256(n_alpha * K * 2) + a256(n_alpha * tiles * 8) + a256(batch * N * K * 2)
         assert wq.wq_awq_workspace_bytes(T, K, Ns, n_alpha) == want, (T, K, Ns)
+
+
+def test_binding_constants_match_the_header(wq):
+    """Every numeric #define of include/wq.h (status codes, options and their
+    values) has the same value in the Python binding; the two version numbers
+    are read from the library instead."""
+    src = open(HEADER).read()
+    defines = dict((n, int(v)) for n, v in re.findall(r"#define (WQ_[A-Z0-9_]+) (-?\d+)\b", src))
+    assert defines["WQ_ABI_VERSION"] == wq.wq_abi_version()
+    assert defines["WQ_LAYOUT_VERSION"] == wq.wq_layout_version()
+    for name, value in defines.items():
+        if name in ("WQ_ABI_VERSION", "WQ_LAYOUT_VERSION"):
+            continue
+        assert getattr(wq, name) == value, name
+    assert sum(n.startswith("WQ_OPT_") for n in defines) >= 12
