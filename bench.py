@@ -601,6 +601,25 @@ def measure_rows(wq, torch, synth, dev, block, peaks):
         "frac_bf16_peak": flops / (ms * 1e-3) / 1e12 / peaks["bf16_tflops"],
         "best_alpha": {g: int(o["best"].item()) / 20 for (g, _, _, _), o in zip(prepared, outs)},
         "pack_with_s_ms": a.elapsed_time(b)}
+    # the same search with the error matrix built inside the loss GEMM
+    old = wq.wq_get_option(wq.WQ_OPT_AWQ_LOSS)
+    wq.wq_set_option(wq.WQ_OPT_AWQ_LOSS, wq.WQ_AWQ_LOSS_FUSED)
+    try:
+        fused = [wq.wq_awq_scale_search(Xd, Wd, workspace=ws) for _, Xd, Wd, ws in prepared]  # warm-up
+        torch.cuda.synchronize()
+        a.record()
+        fused = [wq.wq_awq_scale_search(Xd, Wd, workspace=ws) for _, Xd, Wd, ws in prepared]
+        b.record()
+        torch.cuda.synchronize()
+    finally:
+        wq.wq_set_option(wq.WQ_OPT_AWQ_LOSS, old)
+    assert wq.wq_get_last_device_error() == 0
+    fms = a.elapsed_time(b)
+    rows["awq_search_llama7b_block_fused_loss"] = {
+        "ms": fms, "loss_gemm_TFLOP/s": flops / (fms * 1e-3) / 1e12,
+        "frac_bf16_peak": flops / (fms * 1e-3) / 1e12 / peaks["bf16_tflops"],
+        "same_alpha_as_two_kernels": all(int(f["best"].item()) == int(o["best"].item())
+                                         for f, o in zip(fused, outs))}
     return rows
 
 

@@ -260,6 +260,15 @@ int32_t wq_awq_scale_search_noalloc(const void* X_dev, int64_t T, int64_t K, con
  *                       out; the kernel then frees its tensor memory, returns,
  *                       and wq_get_last_device_error reports WQ_ERR_TIMEOUT.
  *                       Y is not written. For failure-handling tests only.
+ *  WQ_OPT_AWQ_LOSS     how wq_awq_scale_search forms the losses:
+ *                       WQ_AWQ_LOSS_TWO_KERNELS (default) writes the error
+ *                       matrix E = W - Q(W diag s) diag(s)^-1 of a batch of
+ *                       alphas to the workspace and reads it back in a
+ *                       tensor-core GEMM; WQ_AWQ_LOSS_FUSED builds each E tile
+ *                       in shared memory inside the GEMM, in place of the
+ *                       weights it came from (no E in global memory). Both
+ *                       round E to fp16 the same way. The noalloc search always
+ *                       uses the two kernels.
  * wq_set_option returns WQ_ERR_INVALID_ARG for an unknown option or value;
  * wq_get_option returns the current value, or -1 for an unknown option. */
 #define WQ_OPT_GEMM_PATH 1
@@ -282,6 +291,11 @@ int32_t wq_awq_scale_search_noalloc(const void* X_dev, int64_t T, int64_t K, con
 #define WQ_OPT_TC_DEQUANT_WARPS 12
 #define WQ_OPT_WAIT_LIMIT_MS 13
 #define WQ_OPT_TEST_STALL 14
+#define WQ_OPT_AWQ_LOSS 15
+
+#define WQ_AWQ_LOSS_TWO_KERNELS 0
+#define WQ_AWQ_LOSS_FUSED 1
+
 int32_t wq_set_option(int32_t option, int64_t value);
 int64_t wq_get_option(int32_t option);
 

@@ -72,6 +72,7 @@ std::atomic<int64_t> g_opt_tc_bk{0};
 std::atomic<int64_t> g_opt_tc_dequant_warps{0};
 std::atomic<int64_t> g_opt_wait_limit_ms{2000};
 std::atomic<int64_t> g_opt_test_stall{0};
+std::atomic<int64_t> g_opt_awq_loss{WQ_AWQ_LOSS_TWO_KERNELS};
 
 }  // namespace
 
@@ -221,7 +222,7 @@ int32_t wq_awq_scale_search(const void* X, int64_t T, int64_t K, const void* con
   if (!flag) return WQ_ERR_CUDA;
   return cuda_status(wq::launch_awq_search(X, T, K, W, N_i, n_lin, cfg->bits, cfg->symmetric != 0, alpha, n_alpha,
                                            s_out, mu_out, loss_out, best_out, workspace, flag,
-                                           static_cast<cudaStream_t>(stream)));
+                                           g_opt_awq_loss == WQ_AWQ_LOSS_FUSED, static_cast<cudaStream_t>(stream)));
 }
 
 int32_t wq_awq_scale_search_noalloc(const void* X, int64_t T, int64_t K, const void* const* W, const int64_t* N_i,
@@ -280,6 +281,10 @@ int32_t wq_set_option(int32_t option, int64_t value) {
       if (value != 0 && value != 1) return WQ_ERR_INVALID_ARG;
       g_opt_test_stall = value;
       return WQ_OK;
+    case WQ_OPT_AWQ_LOSS:
+      if (value != WQ_AWQ_LOSS_TWO_KERNELS && value != WQ_AWQ_LOSS_FUSED) return WQ_ERR_INVALID_ARG;
+      g_opt_awq_loss = value;
+      return WQ_OK;
     case WQ_OPT_TC_DEQUANT_WARPS:
       if (value != 0 && value != 4 && value != 8) return WQ_ERR_INVALID_ARG;
       g_opt_tc_dequant_warps = value;
@@ -319,6 +324,7 @@ int64_t wq_get_option(int32_t option) {
     case WQ_OPT_WAIT_LIMIT_MS: return g_opt_wait_limit_ms;
     case WQ_OPT_TEST_STALL: return g_opt_test_stall;
     case WQ_OPT_PDL: return g_opt_pdl;
+    case WQ_OPT_AWQ_LOSS: return g_opt_awq_loss;
   }
   return -1;
 }

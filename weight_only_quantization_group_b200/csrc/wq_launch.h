@@ -27,6 +27,7 @@ cudaError_t launch_gemm_tc(const void* X, const uint32_t* packed, const void* st
 struct AwqPlan {
   int64_t N_total;
   int t_tiles, n_tiles, tiles;
+  int fused_tiles, t_chunks;  // the fused loss kernel's row tiles and 512-token chunks
   int batch;  // alphas per E batch
   size_t off_mu, off_S, off_partial, off_E, total;
 };
@@ -34,7 +35,7 @@ AwqPlan plan_awq(int64_t T, int64_t K, const int64_t* N_i, int n_lin, int n_alph
 cudaError_t launch_awq_search(const void* X, int64_t T, int64_t K, const void* const* W, const int64_t* N_i,
                               int n_lin, int bits, bool sym, const double* alpha, int n_alpha, void* s_out,
                               double* mu_out, double* loss_out, int32_t* best_out, void* workspace, int* err,
-                              cudaStream_t st);
+                              bool fused, cudaStream_t st);
 bool awq_noalloc_fits(int64_t T, int64_t K, int64_t N_total, int n_alpha);
 cudaError_t launch_awq_search_noalloc(const void* X, int64_t T, int64_t K, const void* const* W,
                                       const int64_t* N_i, int n_lin, int bits, bool sym, const double* alpha,
