@@ -316,7 +316,7 @@ awq_loss_kernel(const __grid_constant__ CUtensorMap tmE, const __grid_constant__
 //
 //   W producer (warp 0)  one quantization group of W per stage (TMA, two
 //                        64-channel boxes, 128-byte swizzle), and the group's
-//                        s (fp16) and 1/s (fp32) in a small ring;
+//                        s (fp16) and -1/s (fp32) in a small ring;
 //   error rows (2-5)     each thread owns one row: it copies the row's 128
 //                        weights to registers (which frees the W stage),
 //                        decides the group's step and zero point from w * s
@@ -338,7 +338,7 @@ constexpr int kFusedSSlots = 2;
 constexpr int kFusedXStage = kFusedTokens * 64 * 2;     // 64 KB
 constexpr int kFusedESlot = 128 * 64 * 2;               // 16 KB
 constexpr int kFusedWStage = 128 * kGroup * 2;          // 32 KB (two 16 KB boxes)
-constexpr int kFusedSSlot = kGroup * 2 + kGroup * 4;    // s as fp16, then 1/s as fp32
+constexpr int kFusedSSlot = kGroup * 2 + kGroup * 4;    // s as fp16, then -1/s as fp32
 constexpr int kFusedEOff = kFusedXStages * kFusedXStage;
 constexpr int kFusedWOff = kFusedEOff + kFusedESlots * kFusedESlot;
 constexpr int kFusedSOff = kFusedWOff + kFusedWStage;
@@ -364,6 +364,34 @@ struct FusedArgs {
   int n_lin;
   int* err;
 };
+
+// Packed fp32 pairs (sm_100 f32x2 arithmetic): each lane of the pair is an
+// IEEE round-to-nearest operation, bit-identical to the scalar instruction.
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ float2 f2_unpack(uint64_t v) {
+  float2 r;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(r.x), "=f"(r.y) : "l"(v));
+  return r;
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
 
 // Byte offset of 16-byte chunk c of row r in a 128-row tile of 128-byte rows
 // stored with the 128-byte swizzle (what TMA writes for such a box, and what
@@ -458,7 +486,7 @@ awq_loss_fused_kernel(const __grid_constant__ FusedWMaps wm, const __grid_consta
         const int c = lane + 32 * i;
         const __half v = s[g * kGroup + c];
         sh[c] = v;
-        rs[c] = rcp_approx(__half2float(v));
+        rs[c] = -rcp_approx(__half2float(v));
       }
       mbar_arrive(w_full);  // this lane's s values are in place
     }
@@ -534,7 +562,7 @@ awq_loss_fused_kernel(const __grid_constant__ FusedWMaps wm, const __grid_consta
       mbar_arrive(w_empty);  // the W stage may be refilled
       const uint8_t* slot = smem + kFusedSOff + (g % kFusedSSlots) * kFusedSSlot;
       const uint4* sh = reinterpret_cast<const uint4*>(slot);                 // 8 scales per uint4
-      const float4* rs = reinterpret_cast<const float4*>(slot + kGroup * 2);  // 4 reciprocals per float4
+      const float4* rs = reinterpret_cast<const float4*>(slot + kGroup * 2);  // 4 of -1/s per float4
 
       // The group's range of w * s (exact fp16 x fp16 products in fp32).
       float lo = 0.0f, hi = 0.0f;
@@ -565,6 +593,17 @@ awq_loss_fused_kernel(const __grid_constant__ FusedWMaps wm, const __grid_consta
         }
       }
       const GroupQuant gq = group_quant_from_range<BITS, SYM>(lo, hi);
+      // The error pass on pairs of channels. Per channel it is the sequence of
+      // the packer's group_offset_level (Markstein-corrected quotient, plus
+      // 1.5 * 2^23, clamp) and then deq = (level - 1.5 * 2^23) * step, formed
+      // as one fma with -1.5 * 2^23 * step (exact: the product has 13
+      // significant bits and the result at most 15), and e = w + deq * (-1/s).
+      const uint64_t rcp2 = f2_pack(gq.rcp, gq.rcp);
+      const uint64_t nsf2 = f2_pack(-gq.sf, -gq.sf);
+      const uint64_t sf2 = f2_pack(gq.sf, gq.sf);
+      const uint64_t magic2 = f2_pack(kRoundMagic, kRoundMagic);
+      const float nms = __fmul_rn(-kRoundMagic, gq.sf);
+      const uint64_t nms2 = f2_pack(nms, nms);
 
       // E, one 64-channel slot at a time.
 #pragma unroll
@@ -590,12 +629,19 @@ awq_loss_fused_kernel(const __grid_constant__ FusedWMaps wm, const __grid_consta
           for (int i = 0; i < 4; ++i) {
             float p0 = 0.0f, p1 = 0.0f;
             fma2_f16_f32(p0, p1, wv[i], svv[i]);  // w * s, exact
-            const float l0 = __fsub_rn(group_offset_level<BITS, SYM>(p0, gq), kRoundMagic);
-            const float l1 = __fsub_rn(group_offset_level<BITS, SYM>(p1, gq), kRoundMagic);
-            const float d0 = __fmul_rn(l0, gq.sf), d1 = __fmul_rn(l1, gq.sf);
+            const uint64_t ws2 = f2_pack(p0, p1);
+            const uint64_t q0 = f2_mul(ws2, rcp2);
+            const uint64_t rr = f2_fma(q0, nsf2, ws2);          // ws - q0 * step, exact
+            uint64_t lv = f2_add(f2_fma(rr, rcp2, q0), magic2);  // rounded quotient + 1.5 * 2^23
+            if (!SYM) {
+              const float2 l = f2_unpack(lv);
+              lv = f2_pack(fminf(l.x, gq.hi_b), fminf(l.y, gq.hi_b));
+            }
+            const uint64_t deq = f2_fma(lv, sf2, nms2);          // (level - zero) * step, exact
             const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&wv[i]));
-            const __half2 e = __floats2half2_rn(__fmaf_rn(-d0, rv[2 * i], f.x), __fmaf_rn(-d1, rv[2 * i + 1], f.y));
-            o[i] = *reinterpret_cast<const uint32_t*>(&e);
+            const float2 e = f2_unpack(f2_fma(deq, f2_pack(rv[2 * i], rv[2 * i + 1]), f2_pack(f.x, f.y)));
+            const __half2 eh = __floats2half2_rn(e.x, e.y);
+            o[i] = *reinterpret_cast<const uint32_t*>(&eh);
           }
           *reinterpret_cast<uint4*>(eslot + sw128_offset(r, (uint32_t)c8)) = out;
         }
