@@ -165,7 +165,10 @@ int32_t wq_w4a16_gemm(const void* X_dev, const uint32_t* packed_dev, const void*
  * [n_alpha]) and best_out_dev (int32, device). Quantize the weights with
  * wq_quantize_pack(W, s_out) and feed the matmul X * diag(s)^-1 afterwards.
  * workspace_dev: >= wq_awq_workspace_bytes(...) bytes, 256-byte aligned, no
- * initial contents required. A non-finite candidate or loss latches
+ * initial contents required. The size depends on WQ_OPT_AWQ_LOSS when it is
+ * asked for: the two-kernel path keeps the error matrices of a batch of
+ * alphas (up to 1 GiB), the fused path none; a workspace too small for the
+ * path selected at the call returns WQ_ERR_WORKSPACE. A non-finite candidate or loss latches
  * WQ_ERR_RANGE in the device flag. */
 size_t wq_awq_workspace_bytes(int64_t T, int64_t K, const int64_t* N_i, int32_t n_lin, int32_t n_alpha,
                               const wq_quant_cfg* cfg);

@@ -195,7 +195,7 @@ static int32_t check_awq(int64_t T, int64_t K, const int64_t* N_i, int32_t n_lin
 size_t wq_awq_workspace_bytes(int64_t T, int64_t K, const int64_t* N_i, int32_t n_lin, int32_t n_alpha,
                               const wq_quant_cfg* cfg) {
   if (check_awq(T, K, N_i, n_lin, n_alpha, cfg) != WQ_OK) return 0;
-  return wq::plan_awq(T, K, N_i, n_lin, n_alpha).total;
+  return wq::plan_awq(T, K, N_i, n_lin, n_alpha, g_opt_awq_loss == WQ_AWQ_LOSS_FUSED).total;
 }
 
 int32_t wq_awq_scale_search(const void* X, int64_t T, int64_t K, const void* const* W, const int64_t* N_i,
@@ -215,7 +215,7 @@ int32_t wq_awq_scale_search(const void* X, int64_t T, int64_t K, const void* con
   if (!aligned(X, 16) || !aligned(s_out, 2) || (mu_out && !aligned(mu_out, 8)) || (loss_out && !aligned(loss_out, 8)) ||
       (best_out && !aligned(best_out, 4)))
     return WQ_ERR_ALIGNMENT;
-  const size_t need = wq::plan_awq(T, K, N_i, n_lin, n_alpha).total;
+  const size_t need = wq::plan_awq(T, K, N_i, n_lin, n_alpha, g_opt_awq_loss == WQ_AWQ_LOSS_FUSED).total;
   if (!workspace || workspace_bytes < need) return WQ_ERR_WORKSPACE;
   if (!aligned(workspace, 256)) return WQ_ERR_ALIGNMENT;
   int* flag = device_flag();

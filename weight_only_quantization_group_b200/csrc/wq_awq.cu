@@ -717,7 +717,9 @@ static EncodeTiledFnA awq_encode_fn() {
 
 static size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
-AwqPlan plan_awq(int64_t T, int64_t K, const int64_t* N_i, int n_lin, int n_alpha) {
+// Workspace layout: mu, the candidate scales, the partial losses, and (two-
+// kernel path only) the error matrices of one batch of alphas.
+AwqPlan plan_awq(int64_t T, int64_t K, const int64_t* N_i, int n_lin, int n_alpha, bool fused) {
   AwqPlan p;
   p.N_total = 0;
   for (int i = 0; i < n_lin; ++i) p.N_total += N_i[i];
@@ -742,7 +744,7 @@ AwqPlan plan_awq(int64_t T, int64_t K, const int64_t* N_i, int n_lin, int n_alph
   p.off_partial = off;
   off = align256(off + partials * 8);
   p.off_E = off;
-  off = align256(off + (size_t)p.batch * e_one);
+  if (!fused) off = align256(off + (size_t)p.batch * e_one);
   p.total = off;
   return p;
 }
@@ -795,7 +797,7 @@ cudaError_t launch_awq_search(const void* X, int64_t T, int64_t K, const void* c
                               bool fused, cudaStream_t st) {
   EncodeTiledFnA enc = awq_encode_fn();
   if (!enc) return cudaErrorNotSupported;
-  const AwqPlan p = plan_awq(T, K, N_i, n_lin, n_alpha);
+  const AwqPlan p = plan_awq(T, K, N_i, n_lin, n_alpha, fused);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   double* mu = mu_out ? mu_out : reinterpret_cast<double*>(ws + p.off_mu);
   __half* S = reinterpret_cast<__half*>(ws + p.off_S);
@@ -931,7 +933,7 @@ cudaError_t launch_awq_search_noalloc(const void* X, int64_t T, int64_t K, const
   if (!enc) return cudaErrorNotSupported;
   uint8_t* ws = awq_static_scratch();
   if (!ws) return cudaErrorInvalidSymbol;
-  const AwqPlan p = plan_awq(T, K, N_i, n_lin, n_alpha);  // tile counts only; no memory of its own
+  const AwqPlan p = plan_awq(T, K, N_i, n_lin, n_alpha, false);  // tile counts only; no memory of its own
   double* mu = mu_out ? mu_out : reinterpret_cast<double*>(ws);
   __half* S = reinterpret_cast<__half*>(ws + kAwqStaticMu);
   double* partial = reinterpret_cast<double*>(ws + kAwqStaticMu + kAwqStaticS);
