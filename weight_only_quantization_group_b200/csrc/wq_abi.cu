@@ -215,14 +215,15 @@ int32_t wq_awq_scale_search(const void* X, int64_t T, int64_t K, const void* con
   if (!aligned(X, 16) || !aligned(s_out, 2) || (mu_out && !aligned(mu_out, 8)) || (loss_out && !aligned(loss_out, 8)) ||
       (best_out && !aligned(best_out, 4)))
     return WQ_ERR_ALIGNMENT;
-  const size_t need = wq::plan_awq(T, K, N_i, n_lin, n_alpha, g_opt_awq_loss == WQ_AWQ_LOSS_FUSED).total;
+  const bool fused = g_opt_awq_loss == WQ_AWQ_LOSS_FUSED;  // one reading: the size check and the launch agree
+  const size_t need = wq::plan_awq(T, K, N_i, n_lin, n_alpha, fused).total;
   if (!workspace || workspace_bytes < need) return WQ_ERR_WORKSPACE;
   if (!aligned(workspace, 256)) return WQ_ERR_ALIGNMENT;
   int* flag = device_flag();
   if (!flag) return WQ_ERR_CUDA;
   return cuda_status(wq::launch_awq_search(X, T, K, W, N_i, n_lin, cfg->bits, cfg->symmetric != 0, alpha, n_alpha,
                                            s_out, mu_out, loss_out, best_out, workspace, flag,
-                                           g_opt_awq_loss == WQ_AWQ_LOSS_FUSED, static_cast<cudaStream_t>(stream)));
+                                           fused, static_cast<cudaStream_t>(stream)));
 }
 
 int32_t wq_awq_scale_search_noalloc(const void* X, int64_t T, int64_t K, const void* const* W, const int64_t* N_i,
