@@ -270,8 +270,8 @@ int32_t wq_awq_scale_search_noalloc(const void* X_dev, int64_t T, int64_t K, con
  *                       tensor-core GEMM; WQ_AWQ_LOSS_FUSED builds each E tile
  *                       in shared memory inside the GEMM, in place of the
  *                       weights it came from (no E in global memory). Both
- *                       round E to fp16 the same way. The noalloc search always
- *                       uses the two kernels.
+ *                       round E to fp16 the same way; the noalloc search
+ *                       follows the same option (fused: no error-matrix chunks).
  * wq_set_option returns WQ_ERR_INVALID_ARG for an unknown option or value;
  * wq_get_option returns the current value, or -1 for an unknown option. */
 #define WQ_OPT_GEMM_PATH 1

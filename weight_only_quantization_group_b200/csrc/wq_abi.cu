@@ -233,22 +233,21 @@ int32_t wq_awq_scale_search_noalloc(const void* X, int64_t T, int64_t K, const v
   int32_t st = check_awq(T, K, N_i, n_lin, n_alpha, cfg);
   if (st != WQ_OK) return st;
   if (!X || !W || !alpha || !s_out) return WQ_ERR_INVALID_ARG;
-  int64_t n_total = 0;
   for (int i = 0; i < n_lin; ++i) {
     if (!W[i]) return WQ_ERR_INVALID_ARG;
     if (!aligned(W[i], 16)) return WQ_ERR_ALIGNMENT;
-    n_total += N_i[i];
   }
   for (int j = 0; j < n_alpha; ++j)
     if (!(alpha[j] == alpha[j])) return WQ_ERR_INVALID_ARG;  // NaN
   if (!aligned(X, 16) || !aligned(s_out, 2) || (mu_out && !aligned(mu_out, 8)) || (loss_out && !aligned(loss_out, 8)) ||
       (best_out && !aligned(best_out, 4)))
     return WQ_ERR_ALIGNMENT;
-  if (!wq::awq_noalloc_fits(T, K, n_total, n_alpha)) return WQ_ERR_WORKSPACE;
+  const bool fused = g_opt_awq_loss == WQ_AWQ_LOSS_FUSED;  // one reading: the fit check and the launch agree
+  if (!wq::awq_noalloc_fits(T, K, N_i, n_lin, n_alpha, fused)) return WQ_ERR_WORKSPACE;
   int* flag = device_flag();
   if (!flag) return WQ_ERR_CUDA;
   return cuda_status(wq::launch_awq_search_noalloc(X, T, K, W, N_i, n_lin, cfg->bits, cfg->symmetric != 0, alpha,
-                                                   n_alpha, s_out, mu_out, loss_out, best_out, flag,
+                                                   n_alpha, s_out, mu_out, loss_out, best_out, flag, fused,
                                                    static_cast<cudaStream_t>(stream)));
 }
 

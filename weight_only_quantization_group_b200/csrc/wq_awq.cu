@@ -919,21 +919,22 @@ static uint8_t* awq_static_scratch() {
   return addr[dev];
 }
 
-bool awq_noalloc_fits(int64_t T, int64_t K, int64_t N_total, int n_alpha) {
+bool awq_noalloc_fits(int64_t T, int64_t K, const int64_t* N_i, int n_lin, int n_alpha, bool fused) {
   if (K > kAwqStaticMaxK || n_alpha > kAwqMaxAlpha) return false;
-  const int64_t tiles = ((T + 127) / 128) * ((N_total + 127) / 128);
+  const AwqPlan p = plan_awq(T, K, N_i, n_lin, n_alpha, fused);  // tile counts only
+  const int64_t tiles = fused ? (int64_t)p.fused_tiles * p.t_chunks : (int64_t)p.tiles;
   return (size_t)n_alpha * (size_t)tiles * 8 <= kAwqStaticPartial;
 }
 
 cudaError_t launch_awq_search_noalloc(const void* X, int64_t T, int64_t K, const void* const* W,
                                       const int64_t* N_i, int n_lin, int bits, bool sym, const double* alpha,
                                       int n_alpha, void* s_out, double* mu_out, double* loss_out, int32_t* best_out,
-                                      int* err, cudaStream_t st) {
+                                      int* err, bool fused, cudaStream_t st) {
   EncodeTiledFnA enc = awq_encode_fn();
   if (!enc) return cudaErrorNotSupported;
   uint8_t* ws = awq_static_scratch();
   if (!ws) return cudaErrorInvalidSymbol;
-  const AwqPlan p = plan_awq(T, K, N_i, n_lin, n_alpha, false);  // tile counts only; no memory of its own
+  const AwqPlan p = plan_awq(T, K, N_i, n_lin, n_alpha, fused);  // tile counts only; no memory of its own
   double* mu = mu_out ? mu_out : reinterpret_cast<double*>(ws);
   __half* S = reinterpret_cast<__half*>(ws + kAwqStaticMu);
   double* partial = reinterpret_cast<double*>(ws + kAwqStaticMu + kAwqStaticS);
@@ -955,6 +956,17 @@ cudaError_t launch_awq_search_noalloc(const void* X, int64_t T, int64_t K, const
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return cudaErrorInvalidValue;
+  }
+  if (fused) {  // no error matrix: the partial losses are the only scratch
+    cudaError_t e;
+#define WQ_FL(BI, SY) e = launch_fused_loss<BI, SY>(enc, tmX, p, K, W, N_i, n_lin, S, n_alpha, partial, err, st)
+    if (bits == 4) { if (sym) WQ_FL(4, true); else WQ_FL(4, false); }
+    else { if (sym) WQ_FL(3, true); else WQ_FL(3, false); }
+#undef WQ_FL
+    if (e != cudaSuccess) return e;
+    awq_finalize_kernel<<<1, 256, 0, st>>>(partial, p.fused_tiles * p.t_chunks, n_alpha, S, (int)K, loss_out,
+                                            best_out, static_cast<__half*>(s_out), err);
+    return cudaGetLastError();
   }
   const int stages = 3;
   const size_t smem = 1024 + (size_t)stages * kLossStageBytes + (2 * stages + 1) * 8 + 4 * 8 + 16;

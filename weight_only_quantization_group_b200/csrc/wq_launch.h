@@ -37,9 +37,9 @@ cudaError_t launch_awq_search(const void* X, int64_t T, int64_t K, const void* c
                               int n_lin, int bits, bool sym, const double* alpha, int n_alpha, void* s_out,
                               double* mu_out, double* loss_out, int32_t* best_out, void* workspace, int* err,
                               bool fused, cudaStream_t st);
-bool awq_noalloc_fits(int64_t T, int64_t K, int64_t N_total, int n_alpha);
+bool awq_noalloc_fits(int64_t T, int64_t K, const int64_t* N_i, int n_lin, int n_alpha, bool fused);
 cudaError_t launch_awq_search_noalloc(const void* X, int64_t T, int64_t K, const void* const* W,
                                       const int64_t* N_i, int n_lin, int bits, bool sym, const double* alpha,
                                       int n_alpha, void* s_out, double* mu_out, double* loss_out, int32_t* best_out,
-                                      int* err, cudaStream_t st);
+                                      int* err, bool fused, cudaStream_t st);
 }  // namespace wq
