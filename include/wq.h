@@ -263,6 +263,11 @@ int32_t wq_awq_scale_search_noalloc(const void* X_dev, int64_t T, int64_t K, con
  *                       out; the kernel then frees its tensor memory, returns,
  *                       and wq_get_last_device_error reports WQ_ERR_TIMEOUT.
  *                       Y is not written. For failure-handling tests only.
+ *  WQ_OPT_TC_A_SOURCE  where the tensor-core kernel's dequantized weight tile
+ *                       lives: WQ_TC_A_TMEM (default) in tensor memory (written
+ *                       with tcgen05.st), WQ_TC_A_SMEM in shared memory (the
+ *                       MMA reads both operands from shared memory; tensor
+ *                       memory holds only the accumulator). Same results.
  *  WQ_OPT_AWQ_LOSS     how wq_awq_scale_search forms the losses:
  *                       WQ_AWQ_LOSS_TWO_KERNELS (default) writes the error
  *                       matrix E = W - Q(W diag s) diag(s)^-1 of a batch of
@@ -298,6 +303,10 @@ int32_t wq_awq_scale_search_noalloc(const void* X_dev, int64_t T, int64_t K, con
 
 #define WQ_AWQ_LOSS_TWO_KERNELS 0
 #define WQ_AWQ_LOSS_FUSED 1
+#define WQ_OPT_TC_A_SOURCE 16
+
+#define WQ_TC_A_TMEM 0
+#define WQ_TC_A_SMEM 1
 
 int32_t wq_set_option(int32_t option, int64_t value);
 int64_t wq_get_option(int32_t option);

@@ -100,6 +100,7 @@ def test_option_values_are_validated(wq):
         wq.WQ_OPT_WAIT_LIMIT_MS: ([1, 60000, 2000], [0, 60001]),
         wq.WQ_OPT_TEST_STALL: ([1, 0], [2, -1]),
         wq.WQ_OPT_AWQ_LOSS: ([1, 0], [2, -1]),
+        wq.WQ_OPT_TC_A_SOURCE: ([1, 0], [2, -1]),
     }
     for opt, (good, bad) in cases.items():
         old = wq.wq_get_option(opt)

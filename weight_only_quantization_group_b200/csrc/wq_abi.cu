@@ -73,6 +73,7 @@ std::atomic<int64_t> g_opt_tc_dequant_warps{0};
 std::atomic<int64_t> g_opt_wait_limit_ms{2000};
 std::atomic<int64_t> g_opt_test_stall{0};
 std::atomic<int64_t> g_opt_awq_loss{WQ_AWQ_LOSS_TWO_KERNELS};
+std::atomic<int64_t> g_opt_tc_a_source{WQ_TC_A_TMEM};
 
 }  // namespace
 
@@ -160,7 +161,8 @@ int32_t wq_w4a16_gemm(const void* X, const uint32_t* packed, const void* steps, 
     return cuda_status(wq::launch_gemm_tc(X, packed, steps, zeros, M, N, K, Y, flag,
                                           static_cast<cudaStream_t>(stream), (int)g_opt_tc_stages,
                                           (int)g_opt_tc_bk, (int)g_opt_tc_dequant_warps,
-                                          (int)g_opt_wait_limit_ms, g_opt_test_stall != 0));
+                                          (int)g_opt_wait_limit_ms, g_opt_test_stall != 0,
+                                          g_opt_tc_a_source == WQ_TC_A_SMEM));
   }
   if (g_opt_gemv_kernel != WQ_GEMV_KERNEL_TILED && variant != WQ_GEMV_EXACT &&
       wq::gemv_rows_supported(cfg->bits, M, K))
@@ -285,6 +287,10 @@ int32_t wq_set_option(int32_t option, int64_t value) {
       if (value != WQ_AWQ_LOSS_TWO_KERNELS && value != WQ_AWQ_LOSS_FUSED) return WQ_ERR_INVALID_ARG;
       g_opt_awq_loss = value;
       return WQ_OK;
+    case WQ_OPT_TC_A_SOURCE:
+      if (value != WQ_TC_A_TMEM && value != WQ_TC_A_SMEM) return WQ_ERR_INVALID_ARG;
+      g_opt_tc_a_source = value;
+      return WQ_OK;
     case WQ_OPT_TC_DEQUANT_WARPS:
       if (value != 0 && value != 4 && value != 8) return WQ_ERR_INVALID_ARG;
       g_opt_tc_dequant_warps = value;
@@ -325,6 +331,7 @@ int64_t wq_get_option(int32_t option) {
     case WQ_OPT_TEST_STALL: return g_opt_test_stall;
     case WQ_OPT_PDL: return g_opt_pdl;
     case WQ_OPT_AWQ_LOSS: return g_opt_awq_loss;
+    case WQ_OPT_TC_A_SOURCE: return g_opt_tc_a_source;
   }
   return -1;
 }

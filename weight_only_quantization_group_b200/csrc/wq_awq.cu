@@ -365,11 +365,6 @@ struct FusedArgs {
   int* err;
 };
 
-// Byte offset of 16-byte chunk c of row r in a 128-row tile of 128-byte rows
-// stored with the 128-byte swizzle (what TMA writes for such a box, and what
-// desc_kmajor_sw128 describes): chunk c lands at c ^ (r mod 8).
-__device__ __forceinline__ uint32_t sw128_offset(uint32_t r, uint32_t c) { return r * 128u + ((c ^ (r & 7u)) << 4); }
-
 template <int BITS, bool SYM>
 __global__ void __launch_bounds__(kFusedThreads, 1)
 awq_loss_fused_kernel(const __grid_constant__ FusedWMaps wm, const __grid_constant__ CUtensorMap tmX, FusedArgs a) {

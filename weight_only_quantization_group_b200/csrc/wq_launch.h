@@ -21,7 +21,7 @@ cudaError_t launch_gemv_rows(const void* X, const uint32_t* packed, const void* 
                              int grid_mode, bool pdl);
 cudaError_t launch_gemm_tc(const void* X, const uint32_t* packed, const void* steps, const void* zeros, int64_t M,
                            int64_t N, int64_t K, void* Y, int* err, cudaStream_t st, int stages_opt, int bk_opt,
-                           int dw_opt, int wait_ms, bool stall);
+                           int dw_opt, int wait_ms, bool stall, bool a_smem);
 // Workspace layout of the AWQ search (wq_awq.cu): mu, the candidate scales,
 // the per-tile partial losses, and (two-kernel loss path only) the error
 // matrices of one batch of alphas.
