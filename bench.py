@@ -562,17 +562,21 @@ def measure_rows(wq, torch, synth, dev, block, peaks):
                 wq.wq_set_option(wq.WQ_OPT_TC_BK, 0)
                 wq.wq_set_option(wq.WQ_OPT_TC_DEQUANT_WARPS, 0)
     # tensor-core kernel with the dequantized weight tile in shared memory
+    # (64-channel stages keep two CTAs per SM at M = 64, where a 128-channel A
+    # ring leaves room for one)
     for M in (4, 16, 64, 128):
-        for S in (0, 5):
+        for S, bk in ((0, 0), (5, 0), (0, 64)):
             wq.wq_set_option(wq.WQ_OPT_TC_A_SOURCE, wq.WQ_TC_A_SMEM)
             wq.wq_set_option(wq.WQ_OPT_TC_STAGES, S)
-            name = f"smallm_M{M}_8192x28672_w4_tc_smem_a_s{S}"
+            wq.wq_set_option(wq.WQ_OPT_TC_BK, bk)
+            name = f"smallm_M{M}_8192x28672_w4_tc_smem_a_bk{bk}_s{S}"
             try:
                 gemv_row(name, 28672, 8192, 4, big.W, synth.smallm_activations(M), M=M)
             except wq.WQError as e:
                 rows[name] = {"error": str(e)}
             finally:
                 wq.wq_set_option(wq.WQ_OPT_TC_STAGES, 0)
+                wq.wq_set_option(wq.WQ_OPT_TC_BK, 0)
                 wq.wq_set_option(wq.WQ_OPT_TC_A_SOURCE, wq.WQ_TC_A_TMEM)
     # the other kernel on each side of the crossover, for the record
     for M in (2, 3, 4, 8, 16):

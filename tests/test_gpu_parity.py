@@ -592,17 +592,20 @@ def test_tc_gemm_smem_a_parity(wq, tc_smem_a, M, NK):
     assert_close(run_gemm(wq, X, qg, N, 4), O.gemm_ref(X, codes, st, z, 128))
 
 
-@pytest.mark.parametrize("S", [2, 5])
-@pytest.mark.parametrize("M", [16, 128])
-def test_tc_gemm_smem_a_ring_depths(wq, tc_smem_a, S, M):
+@pytest.mark.parametrize("S,BK", [(2, 0), (5, 0), (0, 64), (3, 64)])
+@pytest.mark.parametrize("M", [16, 64, 128])
+def test_tc_gemm_smem_a_ring_depths(wq, tc_smem_a, S, BK, M):
+    """Forced ring depths and 64-channel stages with shared-memory A tiles."""
     N, K = 333, 1152
-    g = synth.rng(800 + M + S)
+    g = synth.rng(800 + M + S + BK)
     W = synth.weight(g, N, K, 0.02, channel_frac=0.01, channel_mult=10.0)
     X = synth.activations(g, M, K, channel_frac=0.01, channel_mult=20.0)
     (codes, st, z), qg = assert_quant_parity(wq, W, None, 4, False)
     wq.wq_set_option(wq.WQ_OPT_TC_STAGES, S)
+    wq.wq_set_option(wq.WQ_OPT_TC_BK, BK)
     try:
         Y = run_gemm(wq, X, qg, N, 4)
     finally:
         wq.wq_set_option(wq.WQ_OPT_TC_STAGES, 0)
+        wq.wq_set_option(wq.WQ_OPT_TC_BK, 0)
     assert_close(Y, O.gemm_ref(X, codes, st, z, 128))
