@@ -609,3 +609,18 @@ def test_tc_gemm_smem_a_ring_depths(wq, tc_smem_a, S, BK, M):
         wq.wq_set_option(wq.WQ_OPT_TC_STAGES, 0)
         wq.wq_set_option(wq.WQ_OPT_TC_BK, 0)
     assert_close(Y, O.gemm_ref(X, codes, st, z, 128))
+
+
+@pytest.mark.parametrize("bits", [3, 4])
+@pytest.mark.parametrize("M", [1, 2, 5])
+@pytest.mark.parametrize("NK", [(64, 32768), (333, 16512)])
+def test_gemv_beyond_row_kernel_k(wq, bits, M, NK):
+    """K above the row-streaming kernel's 16384 channels: the default dispatch
+    sends M <= 2 to the tiled kernel (activations in shared memory, cluster
+    split-K for few rows); M = 5 with 3 bits also takes the tiled kernel."""
+    N, K = NK
+    g = synth.rng(950 + M + bits)
+    W = synth.weight(g, N, K, 0.02, channel_frac=0.01, channel_mult=10.0)
+    X = synth.activations(g, M, K, channel_frac=0.01, channel_mult=20.0)
+    (codes, st, z), qg = assert_quant_parity(wq, W, None, bits, False)
+    assert_close(run_gemm(wq, X, qg, N, bits), O.gemm_ref(X, codes, st, z, 128))
