@@ -561,6 +561,23 @@ def measure_rows(wq, torch, synth, dev, block, peaks):
                 wq.wq_set_option(wq.WQ_OPT_TC_STAGES, 0)
                 wq.wq_set_option(wq.WQ_OPT_TC_BK, 0)
                 wq.wq_set_option(wq.WQ_OPT_TC_DEQUANT_WARPS, 0)
+    # tensor-core kernel with the dequantized weight tile in shared memory
+    # (64-channel stages keep two CTAs per SM at M = 64, where a 128-channel A
+    # ring leaves room for one)
+    for M in (4, 16, 64, 128):
+        for S, bk in ((0, 0), (5, 0), (0, 64)):
+            wq.wq_set_option(wq.WQ_OPT_TC_A_SOURCE, wq.WQ_TC_A_SMEM)
+            wq.wq_set_option(wq.WQ_OPT_TC_STAGES, S)
+            wq.wq_set_option(wq.WQ_OPT_TC_BK, bk)
+            name = f"smallm_M{M}_8192x28672_w4_tc_smem_a_bk{bk}_s{S}"
+            try:
+                gemv_row(name, 28672, 8192, 4, big.W, synth.smallm_activations(M), M=M)
+            except wq.WQError as e:
+                rows[name] = {"error": str(e)}
+            finally:
+                wq.wq_set_option(wq.WQ_OPT_TC_STAGES, 0)
+                wq.wq_set_option(wq.WQ_OPT_TC_BK, 0)
+                wq.wq_set_option(wq.WQ_OPT_TC_A_SOURCE, wq.WQ_TC_A_TMEM)
     # the other kernel on each side of the crossover, for the record
     for M in (2, 3, 4, 8, 16):
         path = wq.WQ_PATH_TENSOR_CORE if M < 3 else wq.WQ_PATH_GEMV
@@ -601,6 +618,25 @@ def measure_rows(wq, torch, synth, dev, block, peaks):
         "frac_bf16_peak": flops / (ms * 1e-3) / 1e12 / peaks["bf16_tflops"],
         "best_alpha": {g: int(o["best"].item()) / 20 for (g, _, _, _), o in zip(prepared, outs)},
         "pack_with_s_ms": a.elapsed_time(b)}
+    # the same search with the error matrix built inside the loss GEMM
+    old = wq.wq_get_option(wq.WQ_OPT_AWQ_LOSS)
+    wq.wq_set_option(wq.WQ_OPT_AWQ_LOSS, wq.WQ_AWQ_LOSS_FUSED)
+    try:
+        fused = [wq.wq_awq_scale_search(Xd, Wd, workspace=ws) for _, Xd, Wd, ws in prepared]  # warm-up
+        torch.cuda.synchronize()
+        a.record()
+        fused = [wq.wq_awq_scale_search(Xd, Wd, workspace=ws) for _, Xd, Wd, ws in prepared]
+        b.record()
+        torch.cuda.synchronize()
+    finally:
+        wq.wq_set_option(wq.WQ_OPT_AWQ_LOSS, old)
+    assert wq.wq_get_last_device_error() == 0
+    fms = a.elapsed_time(b)
+    rows["awq_search_llama7b_block_fused_loss"] = {
+        "ms": fms, "loss_gemm_TFLOP/s": flops / (fms * 1e-3) / 1e12,
+        "frac_bf16_peak": flops / (fms * 1e-3) / 1e12 / peaks["bf16_tflops"],
+        "same_alpha_as_two_kernels": all(int(f["best"].item()) == int(o["best"].item())
+                                         for f, o in zip(fused, outs))}
     return rows
 
 

@@ -165,7 +165,10 @@ int32_t wq_w4a16_gemm(const void* X_dev, const uint32_t* packed_dev, const void*
  * [n_alpha]) and best_out_dev (int32, device). Quantize the weights with
  * wq_quantize_pack(W, s_out) and feed the matmul X * diag(s)^-1 afterwards.
  * workspace_dev: >= wq_awq_workspace_bytes(...) bytes, 256-byte aligned, no
- * initial contents required. A non-finite candidate or loss latches
+ * initial contents required. The size depends on WQ_OPT_AWQ_LOSS when it is
+ * asked for: the two-kernel path keeps the error matrices of a batch of
+ * alphas (up to 1 GiB), the fused path none; a workspace too small for the
+ * path selected at the call returns WQ_ERR_WORKSPACE. A non-finite candidate or loss latches
  * WQ_ERR_RANGE in the device flag. */
 size_t wq_awq_workspace_bytes(int64_t T, int64_t K, const int64_t* N_i, int32_t n_lin, int32_t n_alpha,
                               const wq_quant_cfg* cfg);
@@ -260,6 +263,20 @@ int32_t wq_awq_scale_search_noalloc(const void* X_dev, int64_t T, int64_t K, con
  *                       out; the kernel then frees its tensor memory, returns,
  *                       and wq_get_last_device_error reports WQ_ERR_TIMEOUT.
  *                       Y is not written. For failure-handling tests only.
+ *  WQ_OPT_TC_A_SOURCE  where the tensor-core kernel's dequantized weight tile
+ *                       lives: WQ_TC_A_TMEM (default) in tensor memory (written
+ *                       with tcgen05.st), WQ_TC_A_SMEM in shared memory (the
+ *                       MMA reads both operands from shared memory; tensor
+ *                       memory holds only the accumulator). Same results.
+ *  WQ_OPT_AWQ_LOSS     how wq_awq_scale_search forms the losses:
+ *                       WQ_AWQ_LOSS_TWO_KERNELS (default) writes the error
+ *                       matrix E = W - Q(W diag s) diag(s)^-1 of a batch of
+ *                       alphas to the workspace and reads it back in a
+ *                       tensor-core GEMM; WQ_AWQ_LOSS_FUSED builds each E tile
+ *                       in shared memory inside the GEMM, in place of the
+ *                       weights it came from (no E in global memory). Both
+ *                       round E to fp16 the same way; the noalloc search
+ *                       follows the same option (fused: no error-matrix chunks).
  * wq_set_option returns WQ_ERR_INVALID_ARG for an unknown option or value;
  * wq_get_option returns the current value, or -1 for an unknown option. */
 #define WQ_OPT_GEMM_PATH 1
@@ -282,6 +299,15 @@ int32_t wq_awq_scale_search_noalloc(const void* X_dev, int64_t T, int64_t K, con
 #define WQ_OPT_TC_DEQUANT_WARPS 12
 #define WQ_OPT_WAIT_LIMIT_MS 13
 #define WQ_OPT_TEST_STALL 14
+#define WQ_OPT_AWQ_LOSS 15
+
+#define WQ_AWQ_LOSS_TWO_KERNELS 0
+#define WQ_AWQ_LOSS_FUSED 1
+#define WQ_OPT_TC_A_SOURCE 16
+
+#define WQ_TC_A_TMEM 0
+#define WQ_TC_A_SMEM 1
+
 int32_t wq_set_option(int32_t option, int64_t value);
 int64_t wq_get_option(int32_t option);
 

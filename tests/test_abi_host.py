@@ -99,6 +99,8 @@ def test_option_values_are_validated(wq):
         wq.WQ_OPT_TC_DEQUANT_WARPS: ([4, 8, 0], [2, 6, -1]),
         wq.WQ_OPT_WAIT_LIMIT_MS: ([1, 60000, 2000], [0, 60001]),
         wq.WQ_OPT_TEST_STALL: ([1, 0], [2, -1]),
+        wq.WQ_OPT_AWQ_LOSS: ([1, 0], [2, -1]),
+        wq.WQ_OPT_TC_A_SOURCE: ([1, 0], [2, -1]),
     }
     for opt, (good, bad) in cases.items():
         old = wq.wq_get_option(opt)
@@ -214,15 +216,18 @@ def test_binding_checks_devices(wq):
 def test_awq_workspace_size_is_its_layout(wq):
     """wq_awq_workspace_bytes is the sum of the search's regions, each rounded
     up to 256 bytes: mu (fp64 [K]), the candidates (fp16 [n_alpha][K]), one
-    fp64 partial loss per (alpha, 128x128 tile), and the fp16 error matrices
-    of one batch of alphas (as many as fit 1 GiB, at least one)."""
+    fp64 partial loss per (alpha, tile) -- 128x128 tiles of the two-kernel
+    loss or (alpha, 128-row tile of one linear, 512-token chunk) of the fused
+    one, whichever count is larger -- and the fp16 error matrices of one batch
+    of alphas (as many as fit 1 GiB, at least one; the default two-kernel
+    path)."""
     def a256(x):
         return (x + 255) // 256 * 256
 
     for T, K, Ns, n_alpha in [(512, 4096, [4096] * 3, 20), (8, 256, [16], 20), (131, 640, [1, 129, 7], 6),
                               (512, 11008, [4096], 20)]:
         N = sum(Ns)
-        tiles = -(-T // 128) * -(-N // 128)
+        tiles = max(-(-T // 128) * -(-N // 128), sum(-(-n // 128) for n in Ns) * -(-T // 512))
         batch = max(1, min(n_alpha, (1 << 30) // (N * K * 2)))
         want = a256(K * 8) + a256(n_alpha * K * 2) + a256(n_alpha * tiles * 8) + a256(batch * N * K * 2)
         assert wq.wq_awq_workspace_bytes(T, K, Ns, n_alpha) == want, (T, K, Ns)
@@ -241,3 +246,20 @@ def test_binding_constants_match_the_header(wq):
             continue
         assert getattr(wq, name) == value, name
     assert sum(n.startswith("WQ_OPT_") for n in defines) >= 12
+
+
+def test_awq_workspace_follows_the_loss_path(wq):
+    """The fused loss path keeps no error matrix, so its workspace is smaller
+    by the E batch (here every alpha fits one 1 GiB batch: 20 x N x K x 2)."""
+    T, K, Ns = 512, 4096, [4096, 4096, 4096]
+    old = wq.wq_get_option(wq.WQ_OPT_AWQ_LOSS)
+    try:
+        wq.wq_set_option(wq.WQ_OPT_AWQ_LOSS, wq.WQ_AWQ_LOSS_TWO_KERNELS)
+        two = wq.wq_awq_workspace_bytes(T, K, Ns, 20)
+        wq.wq_set_option(wq.WQ_OPT_AWQ_LOSS, wq.WQ_AWQ_LOSS_FUSED)
+        fused = wq.wq_awq_workspace_bytes(T, K, Ns, 20)
+    finally:
+        wq.wq_set_option(wq.WQ_OPT_AWQ_LOSS, old)
+    batch = min(20, (1 << 30) // (sum(Ns) * K * 2))
+    assert two - fused == batch * sum(Ns) * K * 2
+    assert 0 < fused < 8 << 20

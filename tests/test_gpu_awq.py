@@ -40,21 +40,40 @@ def _near_f16_midpoint(v):
     return np.any(np.abs(mids - v[None]) <= 1e-12 * np.abs(v[None]), axis=0)
 
 
+LOSS_PATHS = ("two_kernels", "fused")
+
+
 def check_search(wq, X, Ws, bits=4, sym=False, alphas=None):
+    """Both ways of forming the losses (the error matrix in global memory, or
+    built inside the loss GEMM) against one oracle search."""
     alphas = O.awq_alpha_grid(20) if alphas is None else np.asarray(alphas, np.float64)
     ref = O.awq_search(X, Ws, bits, 128, sym, alphas)
-    out = wq.wq_awq_scale_search(dev(X), [dev(W) for W in Ws], list(alphas), bits=bits, symmetric=sym)
-    assert wq.wq_get_last_device_error() == 0
+    res = None
+    for path in LOSS_PATHS:
+        r = _check_one(wq, X, Ws, bits, sym, alphas, ref, path)
+        res = res or r
+    return res
+
+
+def _check_one(wq, X, Ws, bits, sym, alphas, ref, path):
+    old = wq.wq_get_option(wq.WQ_OPT_AWQ_LOSS)
+    wq.wq_set_option(wq.WQ_OPT_AWQ_LOSS,
+                     wq.WQ_AWQ_LOSS_FUSED if path == "fused" else wq.WQ_AWQ_LOSS_TWO_KERNELS)
+    try:
+        out = wq.wq_awq_scale_search(dev(X), [dev(W) for W in Ws], list(alphas), bits=bits, symmetric=sym)
+        assert wq.wq_get_last_device_error() == 0, path
+    finally:
+        wq.wq_set_option(wq.WQ_OPT_AWQ_LOSS, old)
     mu = out["mu"].cpu().numpy()
     assert np.array_equal(mu, ref["mu"]), "activation statistic differs"
     losses = out["losses"].cpu().numpy()
     rel = np.abs(losses - ref["losses"]) / ref["losses"]
-    assert np.all(rel <= LOSS_RTOL), rel
+    assert np.all(rel <= LOSS_RTOL), (path, rel)
     best = int(out["best"].cpu().numpy()[0])
     order = np.argsort(ref["losses"], kind="stable")
     if best != ref["best"]:
         gap = (ref["losses"][order[1]] - ref["losses"][order[0]]) / ref["losses"][order[0]]
-        assert gap < LOSS_RTOL and best == order[1], ("alpha differs", best, ref["best"], gap)
+        assert gap < LOSS_RTOL and best == order[1], ("alpha differs", path, best, ref["best"], gap)
     s = out["s"].cpu().numpy()
     cand = O.awq_candidates(ref["mu"], alphas)[best]
     diff = s.view(np.uint16) != cand.view(np.uint16)
@@ -88,15 +107,33 @@ def test_awq_search_ragged_and_zero_channel(wq):
     check_search(wq, X, Ws, 4, False, alphas=[0.0, 0.1, 0.25, 0.5, 0.8, 1.0])
 
 
-def test_awq_alpha_zero_only_equals_rtn(wq):
+@pytest.mark.parametrize("path", LOSS_PATHS)
+def test_awq_alpha_zero_only_equals_rtn(wq, path):
     g = synth.rng(702)
     X = synth.activations(g, 40, 256)
     W = synth.weight(g, 64, 256, 0.02)
-    out = wq.wq_awq_scale_search(dev(X), [dev(W)], [0.0])
+    old = wq.wq_get_option(wq.WQ_OPT_AWQ_LOSS)
+    wq.wq_set_option(wq.WQ_OPT_AWQ_LOSS, wq.WQ_AWQ_LOSS_FUSED if path == "fused" else wq.WQ_AWQ_LOSS_TWO_KERNELS)
+    try:
+        out = wq.wq_awq_scale_search(dev(X), [dev(W)], [0.0])
+    finally:
+        wq.wq_set_option(wq.WQ_OPT_AWQ_LOSS, old)
+    assert wq.wq_get_last_device_error() == 0
     assert np.all(out["s"].cpu().numpy() == 1.0)
     L = float(out["losses"].cpu().numpy()[0])
     ref = O.awq_loss(X, [W], np.ones(256, np.float16), 4, 128, False)
     assert abs(L - ref) <= LOSS_RTOL * ref
+
+
+@pytest.mark.parametrize("T", [1, 511, 512, 513, 1100])
+def test_awq_fused_token_chunks(wq, T):
+    """The fused kernel covers 512 tokens per CTA: one token, a ragged chunk,
+    exactly one chunk, and several chunks give the same losses as the oracle
+    and as the two-kernel path (rows and tokens past the end read as zeros)."""
+    g = synth.rng(703 + T)
+    X = synth.activations(g, T, 384, channel_frac=0.02, channel_mult=20.0)
+    Ws = [synth.weight(g, 130, 384, 0.02), synth.weight(g, 3, 384, 0.02)]
+    check_search(wq, X, Ws, 4, False, alphas=[0.0, 0.3, 0.6])
 
 
 def test_awq_block_o_and_down_full(wq):

@@ -567,3 +567,60 @@ def test_gemv_int_digits_extreme_activations(wq, rows_shape):
             assert_close(Y, ref)
     rows_shape(0, wq.WQ_GEMV_INT_DIGITS)
     assert np.all(run_gemm(wq, np.zeros((1, K), np.float16), qg, N, 4) == 0)
+
+
+@pytest.fixture
+def tc_smem_a(wq):
+    """The tensor-core kernel with its dequantized weight tile in shared memory."""
+    wq.wq_set_option(wq.WQ_OPT_GEMM_PATH, wq.WQ_PATH_TENSOR_CORE)
+    wq.wq_set_option(wq.WQ_OPT_TC_A_SOURCE, wq.WQ_TC_A_SMEM)
+    yield
+    wq.wq_set_option(wq.WQ_OPT_TC_A_SOURCE, wq.WQ_TC_A_TMEM)
+    wq.wq_set_option(wq.WQ_OPT_GEMM_PATH, wq.WQ_PATH_AUTO)
+
+
+@pytest.mark.parametrize("M", [1, 3, 16, 17, 64, 100, 128, 200, 300])
+@pytest.mark.parametrize("NK", [(333, 1152), (1000, 4096)])
+def test_tc_gemm_smem_a_parity(wq, tc_smem_a, M, NK):
+    """Shared-memory A tiles: the same tolerance against the fp64 reference
+    (128- and 64-channel stages, one to several 256-row X chunks, ragged N)."""
+    N, K = NK
+    g = synth.rng(700 + M)
+    W = synth.weight(g, N, K, 0.02, channel_frac=0.01, channel_mult=10.0)
+    X = synth.activations(g, M, K, channel_frac=0.01, channel_mult=20.0)
+    (codes, st, z), qg = assert_quant_parity(wq, W, None, 4, False)
+    assert_close(run_gemm(wq, X, qg, N, 4), O.gemm_ref(X, codes, st, z, 128))
+
+
+@pytest.mark.parametrize("S,BK", [(2, 0), (5, 0), (0, 64), (3, 64)])
+@pytest.mark.parametrize("M", [16, 64, 128])
+def test_tc_gemm_smem_a_ring_depths(wq, tc_smem_a, S, BK, M):
+    """Forced ring depths and 64-channel stages with shared-memory A tiles."""
+    N, K = 333, 1152
+    g = synth.rng(800 + M + S + BK)
+    W = synth.weight(g, N, K, 0.02, channel_frac=0.01, channel_mult=10.0)
+    X = synth.activations(g, M, K, channel_frac=0.01, channel_mult=20.0)
+    (codes, st, z), qg = assert_quant_parity(wq, W, None, 4, False)
+    wq.wq_set_option(wq.WQ_OPT_TC_STAGES, S)
+    wq.wq_set_option(wq.WQ_OPT_TC_BK, BK)
+    try:
+        Y = run_gemm(wq, X, qg, N, 4)
+    finally:
+        wq.wq_set_option(wq.WQ_OPT_TC_STAGES, 0)
+        wq.wq_set_option(wq.WQ_OPT_TC_BK, 0)
+    assert_close(Y, O.gemm_ref(X, codes, st, z, 128))
+
+
+@pytest.mark.parametrize("bits", [3, 4])
+@pytest.mark.parametrize("M", [1, 2, 5])
+@pytest.mark.parametrize("NK", [(64, 32768), (333, 16512)])
+def test_gemv_beyond_row_kernel_k(wq, bits, M, NK):
+    """K above the row-streaming kernel's 16384 channels: the default dispatch
+    sends M <= 2 to the tiled kernel (activations in shared memory, cluster
+    split-K for few rows); M = 5 with 3 bits also takes the tiled kernel."""
+    N, K = NK
+    g = synth.rng(950 + M + bits)
+    W = synth.weight(g, N, K, 0.02, channel_frac=0.01, channel_mult=10.0)
+    X = synth.activations(g, M, K, channel_frac=0.01, channel_mult=20.0)
+    (codes, st, z), qg = assert_quant_parity(wq, W, None, bits, False)
+    assert_close(run_gemm(wq, X, qg, N, bits), O.gemm_ref(X, codes, st, z, 128))

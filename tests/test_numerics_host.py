@@ -7,7 +7,9 @@ arguments the quantizer relies on, independent of any CUDA code:
   closer than that); for an fp16 step (11 significant bits) and the small
   integer divisors 3, 7, 15, q must equal RN(w / step) exactly, r must be
   representable in fp32, and the cases include exact ties and near-ties;
-* rint by adding 1.5 * 2^23 rounds to nearest with ties to even for |x| < 2^22.
+* rint by adding 1.5 * 2^23 rounds to nearest with ties to even for |x| < 2^22;
+* the dequantized value (level - zero) * step is one exact fma of the offset
+  level with the step and the constant -(1.5 * 2^23) * step.
 """
 import random
 from fractions import Fraction as F
@@ -140,3 +142,25 @@ def test_offset_level_packing_identity(bits):
             for l, s in zip(lv, shifts):
                 want |= int(l) << s
             assert word == want, (z, lv)
+
+
+def test_dequant_as_one_fma_is_exact():
+    """The AWQ error pass forms deq = (level - zero) * step as one fma,
+    fma(1.5 * 2^23 + level - zero, step, -(1.5 * 2^23) * step): for every
+    finite fp16 step and every offset level - zero in [-15, 15] the constant
+    -(1.5 * 2^23) * step is an fp32 number, and the fma's single rounding of
+    the exact value returns exactly (level - zero) * step."""
+    magic = 12582912.0
+    steps = _fp16_positive()
+    offs = np.arange(-15, 16, dtype=np.float64)
+    c = -magic * steps                                   # the fp32 constant
+    assert np.all(c.astype(np.float32).astype(np.float64) == c)
+    lv = magic + offs[:, None]                           # the offset level, an fp32 number
+    assert np.all(lv.astype(np.float32).astype(np.float64) == lv)
+    # lv * step has at most 24 + 11 significant bits, so the fp64 sum below is
+    # the fma's exact value; one rounding to fp32 is the fma's result.
+    exact = lv * steps[None, :] + c[None, :]
+    fused = exact.astype(np.float32).astype(np.float64)
+    want = offs[:, None] * steps[None, :]
+    assert np.array_equal(fused, want)
+    assert np.array_equal(want.astype(np.float32).astype(np.float64), want)

@@ -32,7 +32,18 @@ def dev(a):
     return torch.from_numpy(np.ascontiguousarray(a)).cuda()
 
 
-def test_noalloc_matches_workspace_entry_point_twice(wq):
+@pytest.mark.parametrize("path", ["two_kernels", "fused"])
+def test_noalloc_matches_workspace_entry_point_twice(wq, path):
+    """Both loss paths: the fused one needs no error-matrix chunks at all."""
+    old = wq.wq_get_option(wq.WQ_OPT_AWQ_LOSS)
+    wq.wq_set_option(wq.WQ_OPT_AWQ_LOSS, wq.WQ_AWQ_LOSS_FUSED if path == "fused" else wq.WQ_AWQ_LOSS_TWO_KERNELS)
+    try:
+        _noalloc_matches(wq)
+    finally:
+        wq.wq_set_option(wq.WQ_OPT_AWQ_LOSS, old)
+
+
+def _noalloc_matches(wq):
     g = synth.rng(900)
     K = 4096  # 2048-row error chunks: the stacked 3200 rows span two chunks
     X = dev(synth.activations(g, 256, K, channel_frac=0.01, channel_mult=20.0))

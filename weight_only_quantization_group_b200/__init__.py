@@ -88,6 +88,12 @@ WQ_OPT_TC_BK = 11
 WQ_OPT_TC_DEQUANT_WARPS = 12
 WQ_OPT_WAIT_LIMIT_MS = 13
 WQ_OPT_TEST_STALL = 14
+WQ_OPT_AWQ_LOSS = 15
+WQ_AWQ_LOSS_TWO_KERNELS = 0
+WQ_AWQ_LOSS_FUSED = 1
+WQ_OPT_TC_A_SOURCE = 16
+WQ_TC_A_TMEM = 0
+WQ_TC_A_SMEM = 1
 
 
 class WQError(RuntimeError):

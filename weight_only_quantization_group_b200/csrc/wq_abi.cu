@@ -72,6 +72,8 @@ std::atomic<int64_t> g_opt_tc_bk{0};
 std::atomic<int64_t> g_opt_tc_dequant_warps{0};
 std::atomic<int64_t> g_opt_wait_limit_ms{2000};
 std::atomic<int64_t> g_opt_test_stall{0};
+std::atomic<int64_t> g_opt_awq_loss{WQ_AWQ_LOSS_TWO_KERNELS};
+std::atomic<int64_t> g_opt_tc_a_source{WQ_TC_A_TMEM};
 
 }  // namespace
 
@@ -159,7 +161,8 @@ int32_t wq_w4a16_gemm(const void* X, const uint32_t* packed, const void* steps, 
     return cuda_status(wq::launch_gemm_tc(X, packed, steps, zeros, M, N, K, Y, flag,
                                           static_cast<cudaStream_t>(stream), (int)g_opt_tc_stages,
                                           (int)g_opt_tc_bk, (int)g_opt_tc_dequant_warps,
-                                          (int)g_opt_wait_limit_ms, g_opt_test_stall != 0));
+                                          (int)g_opt_wait_limit_ms, g_opt_test_stall != 0,
+                                          g_opt_tc_a_source == WQ_TC_A_SMEM));
   }
   if (g_opt_gemv_kernel != WQ_GEMV_KERNEL_TILED && variant != WQ_GEMV_EXACT &&
       wq::gemv_rows_supported(cfg->bits, M, K))
@@ -194,7 +197,7 @@ static int32_t check_awq(int64_t T, int64_t K, const int64_t* N_i, int32_t n_lin
 size_t wq_awq_workspace_bytes(int64_t T, int64_t K, const int64_t* N_i, int32_t n_lin, int32_t n_alpha,
                               const wq_quant_cfg* cfg) {
   if (check_awq(T, K, N_i, n_lin, n_alpha, cfg) != WQ_OK) return 0;
-  return wq::plan_awq(T, K, N_i, n_lin, n_alpha).total;
+  return wq::plan_awq(T, K, N_i, n_lin, n_alpha, g_opt_awq_loss == WQ_AWQ_LOSS_FUSED).total;
 }
 
 int32_t wq_awq_scale_search(const void* X, int64_t T, int64_t K, const void* const* W, const int64_t* N_i,
@@ -214,14 +217,15 @@ int32_t wq_awq_scale_search(const void* X, int64_t T, int64_t K, const void* con
   if (!aligned(X, 16) || !aligned(s_out, 2) || (mu_out && !aligned(mu_out, 8)) || (loss_out && !aligned(loss_out, 8)) ||
       (best_out && !aligned(best_out, 4)))
     return WQ_ERR_ALIGNMENT;
-  const size_t need = wq::plan_awq(T, K, N_i, n_lin, n_alpha).total;
+  const bool fused = g_opt_awq_loss == WQ_AWQ_LOSS_FUSED;  // one reading: the size check and the launch agree
+  const size_t need = wq::plan_awq(T, K, N_i, n_lin, n_alpha, fused).total;
   if (!workspace || workspace_bytes < need) return WQ_ERR_WORKSPACE;
   if (!aligned(workspace, 256)) return WQ_ERR_ALIGNMENT;
   int* flag = device_flag();
   if (!flag) return WQ_ERR_CUDA;
   return cuda_status(wq::launch_awq_search(X, T, K, W, N_i, n_lin, cfg->bits, cfg->symmetric != 0, alpha, n_alpha,
                                            s_out, mu_out, loss_out, best_out, workspace, flag,
-                                           static_cast<cudaStream_t>(stream)));
+                                           fused, static_cast<cudaStream_t>(stream)));
 }
 
 int32_t wq_awq_scale_search_noalloc(const void* X, int64_t T, int64_t K, const void* const* W, const int64_t* N_i,
@@ -231,22 +235,21 @@ int32_t wq_awq_scale_search_noalloc(const void* X, int64_t T, int64_t K, const v
   int32_t st = check_awq(T, K, N_i, n_lin, n_alpha, cfg);
   if (st != WQ_OK) return st;
   if (!X || !W || !alpha || !s_out) return WQ_ERR_INVALID_ARG;
-  int64_t n_total = 0;
   for (int i = 0; i < n_lin; ++i) {
     if (!W[i]) return WQ_ERR_INVALID_ARG;
     if (!aligned(W[i], 16)) return WQ_ERR_ALIGNMENT;
-    n_total += N_i[i];
   }
   for (int j = 0; j < n_alpha; ++j)
     if (!(alpha[j] == alpha[j])) return WQ_ERR_INVALID_ARG;  // NaN
   if (!aligned(X, 16) || !aligned(s_out, 2) || (mu_out && !aligned(mu_out, 8)) || (loss_out && !aligned(loss_out, 8)) ||
       (best_out && !aligned(best_out, 4)))
     return WQ_ERR_ALIGNMENT;
-  if (!wq::awq_noalloc_fits(T, K, n_total, n_alpha)) return WQ_ERR_WORKSPACE;
+  const bool fused = g_opt_awq_loss == WQ_AWQ_LOSS_FUSED;  // one reading: the fit check and the launch agree
+  if (!wq::awq_noalloc_fits(T, K, N_i, n_lin, n_alpha, fused)) return WQ_ERR_WORKSPACE;
   int* flag = device_flag();
   if (!flag) return WQ_ERR_CUDA;
   return cuda_status(wq::launch_awq_search_noalloc(X, T, K, W, N_i, n_lin, cfg->bits, cfg->symmetric != 0, alpha,
-                                                   n_alpha, s_out, mu_out, loss_out, best_out, flag,
+                                                   n_alpha, s_out, mu_out, loss_out, best_out, flag, fused,
                                                    static_cast<cudaStream_t>(stream)));
 }
 
@@ -279,6 +282,14 @@ int32_t wq_set_option(int32_t option, int64_t value) {
     case WQ_OPT_TEST_STALL:
       if (value != 0 && value != 1) return WQ_ERR_INVALID_ARG;
       g_opt_test_stall = value;
+      return WQ_OK;
+    case WQ_OPT_AWQ_LOSS:
+      if (value != WQ_AWQ_LOSS_TWO_KERNELS && value != WQ_AWQ_LOSS_FUSED) return WQ_ERR_INVALID_ARG;
+      g_opt_awq_loss = value;
+      return WQ_OK;
+    case WQ_OPT_TC_A_SOURCE:
+      if (value != WQ_TC_A_TMEM && value != WQ_TC_A_SMEM) return WQ_ERR_INVALID_ARG;
+      g_opt_tc_a_source = value;
       return WQ_OK;
     case WQ_OPT_TC_DEQUANT_WARPS:
       if (value != 0 && value != 4 && value != 8) return WQ_ERR_INVALID_ARG;
@@ -319,6 +330,8 @@ int64_t wq_get_option(int32_t option) {
     case WQ_OPT_WAIT_LIMIT_MS: return g_opt_wait_limit_ms;
     case WQ_OPT_TEST_STALL: return g_opt_test_stall;
     case WQ_OPT_PDL: return g_opt_pdl;
+    case WQ_OPT_AWQ_LOSS: return g_opt_awq_loss;
+    case WQ_OPT_TC_A_SOURCE: return g_opt_tc_a_source;
   }
   return -1;
 }

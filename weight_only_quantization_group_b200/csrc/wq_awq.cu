@@ -16,8 +16,12 @@
 //                the group stacked row-wise (same decision code as the packer)
 //     awq_loss   tcgen05 GEMM D = E_j X^T per 128x128 tile, epilogue sums D^2
 //                in fp64 -> one partial per (alpha, tile)
+//   (or, with the fused loss option, one launch of awq_loss_fused, which
+//    builds each E tile in shared memory inside the GEMM: no E in global
+//    memory, one partial per (alpha, row tile, 512-token chunk))
 //   finalize     L_j = sum of the partials, one warp per alpha in a fixed
 //                order (deterministic), first argmin, s_out = s_best
+#include <cstring>
 #include <mutex>
 
 #include "wq_quant_core.cuh"
@@ -305,6 +309,354 @@ awq_loss_kernel(const __grid_constant__ CUtensorMap tmE, const __grid_constant__
   }
 }
 
+// ------------------------------------------------------------------ S4, fused: E built inside the loss GEMM
+// One CTA: one alpha, 128 rows of one linear (the MMA's A operand, M = 128)
+// and 512 calibration tokens (B, two N = 256 halves; D fills the 512 fp32
+// columns of tensor memory). The error matrix never reaches global memory:
+//
+//   W producer (warp 0)  one quantization group of W per stage (TMA, two
+//                        64-channel boxes, 128-byte swizzle), and the group's
+//                        s (fp16) and -1/s (fp32) in a small ring;
+//   error rows (2-5)     each thread owns one row: it copies the row's 128
+//                        weights to registers (which frees the W stage),
+//                        decides the group's step and zero point from w * s
+//                        with the packer's decision code, and writes
+//                        E = w - deq(Q(w s)) / s in fp16 into a ring of
+//                        64-channel slots, in the swizzled K-major layout the
+//                        MMA reads; then the epilogue (sum of D^2 in fp64);
+//   MMA (warp 1)         owns tensor memory; per 64-channel slot, 4 K steps x
+//                        2 token halves of tcgen05.mma;
+//   X producer (warp 6)  64 channels x 512 tokens of X per stage (TMA).
+//
+// The three producers run independently, so W is fetched a group ahead of
+// the error rows, and the error rows run up to two groups ahead of the MMA.
+constexpr int kFusedThreads = 224;
+constexpr int kFusedTokens = 512;                       // tokens per CTA = TMEM columns
+constexpr int kFusedXStages = 2;
+constexpr int kFusedESlots = 4;                         // 64-channel E slots (two groups)
+constexpr int kFusedSSlots = 2;
+constexpr int kFusedXStage = kFusedTokens * 64 * 2;     // 64 KB
+constexpr int kFusedESlot = 128 * 64 * 2;               // 16 KB
+constexpr int kFusedWStage = 128 * kGroup * 2;          // 32 KB (two 16 KB boxes)
+constexpr int kFusedSSlot = kGroup * 2 + kGroup * 4;    // s as fp16, then -1/s as fp32
+constexpr int kFusedEOff = kFusedXStages * kFusedXStage;
+constexpr int kFusedWOff = kFusedEOff + kFusedESlots * kFusedESlot;
+constexpr int kFusedSOff = kFusedWOff + kFusedWStage;
+constexpr int kFusedBarOff = kFusedSOff + kFusedSSlots * kFusedSSlot;
+// x_full[2], x_empty[2], w_full, w_empty, e_full[4], e_empty[4], accum
+constexpr int kFusedBars = 2 * kFusedXStages + 2 + 2 * kFusedESlots + 1;
+constexpr int kFusedSmem = kFusedBarOff + kFusedBars * 8 + 4 * 8 + 16;
+constexpr size_t kFusedSmemLaunch = 1024 + (size_t)kFusedSmem;  // + alignment slack
+static_assert(kFusedSmemLaunch <= 232448, "one CTA's shared memory");
+
+struct FusedWMaps {
+  CUtensorMap m[kAwqMaxLinears];  // W_i as [N_i][K] fp16, box 64 x 128, 128-byte swizzle
+};
+
+struct FusedArgs {
+  const __half* S;                    // [n_alpha][K] candidate scales
+  double* partial;                    // [n_alpha][tiles][t_chunks]
+  int K;
+  int n_alpha;
+  int tiles;                          // tile_off[n_lin]
+  int t_chunks;                       // ceil(T / 512)
+  int tile_off[kAwqMaxLinears + 1];   // prefix sums of ceil(N_i / 128)
+  int n_lin;
+  int* err;
+};
+
+template <int BITS, bool SYM>
+__global__ void __launch_bounds__(kFusedThreads, 1)
+awq_loss_fused_kernel(const __grid_constant__ FusedWMaps wm, const __grid_constant__ CUtensorMap tmX, FusedArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* x_full = reinterpret_cast<uint64_t*>(smem + kFusedBarOff);
+  uint64_t* x_empty = x_full + kFusedXStages;
+  uint64_t* w_full = x_empty + kFusedXStages;
+  uint64_t* w_empty = w_full + 1;
+  uint64_t* e_full = w_empty + 1;
+  uint64_t* e_empty = e_full + kFusedESlots;
+  uint64_t* accum = e_empty + kFusedESlots;
+  double* red = reinterpret_cast<double*>(accum + 1);  // [4]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(red + 4);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int alpha = (int)(blockIdx.x % (unsigned)a.n_alpha);
+  const int tile = (int)(blockIdx.x / (unsigned)a.n_alpha);
+  const int tc = blockIdx.y;
+  const int G = a.K / kGroup;
+  const int KT = 2 * G;  // 64-channel slots
+  // The linear that owns the tile, and the tile's first row within it (the
+  // loop is unrolled so the parameter arrays are never indexed at run time).
+  int lin = 0, toff = 0;
+#pragma unroll
+  for (int i = 1; i < kAwqMaxLinears; ++i)
+    if (i < a.n_lin && tile >= a.tile_off[i]) {
+      lin = i;
+      toff = a.tile_off[i];
+    }
+  const int row0 = (tile - toff) * 128;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kFusedXStages; ++s) {
+      mbar_init(&x_full[s], 1);
+      mbar_init(&x_empty[s], 1);
+    }
+    mbar_init(w_full, 1 + 32);  // the TMA's expect_tx arrival + one per producer lane (s ring)
+    mbar_init(w_empty, 128);    // every error row has copied its weights
+    for (int s = 0; s < kFusedESlots; ++s) {
+      mbar_init(&e_full[s], 128);
+      mbar_init(&e_empty[s], 1);
+    }
+    mbar_init(accum, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, kFusedTokens);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ---------------------------------------------------------------- W producer
+    const CUtensorMap* wmap = &wm.m[lin];
+    const __half* s = a.S + (size_t)alpha * a.K;
+    if (lane == 0) prefetch_tensormap(wmap);
+    int issued = 0;
+    for (int g = 0; g < G; ++g) {
+      // The stage is free once every error row has copied group g - 1; by then
+      // they are also done with the s slot of group g - 2.
+      bool w = true;
+      if (lane == 0 && g > 0) w = !*abort_flag && mbar_wait(w_empty, (g - 1) & 1, a.err, kAwqSpinLimit);
+      if (__shfl_sync(0xffffffffu, w ? 1 : 0, 0) == 0) {
+        if (lane == 0) *abort_flag = 1;
+        break;
+      }
+      if (lane == 0) {
+        uint8_t* wdst = smem + kFusedWOff;
+        mbar_arrive_expect_tx(w_full, kFusedWStage);
+        tma_load_2d(wdst, wmap, g * kGroup, row0, w_full);
+        tma_load_2d(wdst + kFusedWStage / 2, wmap, g * kGroup + 64, row0, w_full);
+      }
+      issued = g + 1;
+      uint8_t* slot = smem + kFusedSOff + (g % kFusedSSlots) * kFusedSSlot;
+      __half* sh = reinterpret_cast<__half*>(slot);
+      float* rs = reinterpret_cast<float*>(slot + kGroup * 2);
+#pragma unroll
+      for (int i = 0; i < kGroup / 32; ++i) {
+        const int c = lane + 32 * i;
+        const __half v = s[g * kGroup + c];
+        sh[c] = v;
+        rs[c] = -rcp_approx(__half2float(v));
+      }
+      mbar_arrive(w_full);  // this lane's s values are in place
+    }
+    // The last load must land before the CTA may exit.
+    if (lane == 0 && issued > 0) mbar_wait(w_full, (issued - 1) & 1, a.err, kAwqSpinLimit);
+  } else if (warp == 6) {
+    // ---------------------------------------------------------------- X producer
+    if (lane == 0) {
+      prefetch_tensormap(&tmX);
+      const int t0 = tc * kFusedTokens;
+      int issued = 0;
+      for (int kt = 0; kt < KT; ++kt) {
+        const int xs = kt % kFusedXStages;
+        if (kt >= kFusedXStages &&
+            (*abort_flag || !mbar_wait(&x_empty[xs], ((kt / kFusedXStages) - 1) & 1, a.err, kAwqSpinLimit))) {
+          *abort_flag = 1;
+          break;
+        }
+        uint8_t* xdst = smem + xs * kFusedXStage;
+        mbar_arrive_expect_tx(&x_full[xs], kFusedXStage);
+#pragma unroll
+        for (int b = 0; b < kFusedTokens / 128; ++b)  // rows past T read as zeros
+          tma_load_2d(xdst + b * (128 * 64 * 2), &tmX, kt * 64, t0 + 128 * b, &x_full[xs]);
+        issued = kt + 1;
+      }
+      for (int kt = issued > kFusedXStages ? issued - kFusedXStages : 0; kt < issued; ++kt)
+        mbar_wait(&x_full[kt % kFusedXStages], (kt / kFusedXStages) & 1, a.err, kAwqSpinLimit);
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- MMA
+    if (lane == 0) {
+      const uint32_t idesc = idesc_f16_f32(128, 256);
+      bool ok = true;
+      for (int kt = 0; kt < KT; ++kt) {
+        const int es = kt % kFusedESlots, xs = kt % kFusedXStages;
+        if (*abort_flag || !mbar_wait(&e_full[es], (kt / kFusedESlots) & 1, a.err, kAwqSpinLimit) ||
+            !mbar_wait(&x_full[xs], (kt / kFusedXStages) & 1, a.err, kAwqSpinLimit)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t abase = smem_u32(smem + kFusedEOff + es * kFusedESlot);
+        const uint32_t bbase = smem_u32(smem + xs * kFusedXStage);
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+#pragma unroll
+          for (int n = 0; n < 2; ++n)
+            mma_f16_ss(tmem + 256u * n, desc_kmajor_sw128(abase + 32 * j),
+                       desc_kmajor_sw128(bbase + n * (kFusedXStage / 2) + 32 * j), idesc,
+                       (kt > 0 || j > 0) ? 1u : 0u);
+        mma_commit(&x_empty[xs]);
+        mma_commit(&e_empty[es]);
+      }
+      mma_commit(accum);
+      if (!ok) {
+        *abort_flag = 1;
+        mbar_wait(accum, 0, a.err, kAwqSpinLimit);  // no MMA of ours still reads shared memory
+      }
+    }
+  } else {
+    // ---------------------------------------------------------------- error rows
+    const uint32_t r = threadIdx.x - 64;  // the E row (A row, TMEM lane) this thread builds
+    for (int g = 0; g < G; ++g) {
+      if (*abort_flag || !mbar_wait(w_full, g & 1, a.err, kAwqSpinLimit)) {
+        *abort_flag = 1;
+        break;
+      }
+      uint4 wr[16];  // the row's 128 weights, channel order
+#pragma unroll
+      for (int c = 0; c < 16; ++c)
+        wr[c] = *reinterpret_cast<const uint4*>(smem + kFusedWOff + (c >> 3) * (kFusedWStage / 2) +
+                                                sw128_offset(r, (uint32_t)(c & 7)));
+      mbar_arrive(w_empty);  // the W stage may be refilled
+      const uint8_t* slot = smem + kFusedSOff + (g % kFusedSSlots) * kFusedSSlot;
+      const uint4* sh = reinterpret_cast<const uint4*>(slot);                 // 8 scales per uint4
+      const float4* rs = reinterpret_cast<const float4*>(slot + kGroup * 2);  // 4 of -1/s per float4
+
+      // The group's range of w * s (exact fp16 x fp16 products in fp32).
+      float lo = 0.0f, hi = 0.0f;
+#pragma unroll
+      for (int c = 0; c < 16; ++c) {
+        const uint4 sv = sh[c];
+        const uint32_t* wv = &wr[c].x;
+        const uint32_t* svv = &sv.x;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          float p0 = 0.0f, p1 = 0.0f;
+          fma2_f16_f32(p0, p1, wv[i], svv[i]);
+          if (c == 0 && i == 0) {
+            lo = p0;
+            hi = SYM ? fabsf(p0) : p0;
+          } else if (SYM) {
+            hi = max_nan(hi, fabsf(p0));
+          } else {
+            lo = min_nan(lo, p0);
+            hi = max_nan(hi, p0);
+          }
+          if (SYM) {
+            hi = max_nan(hi, fabsf(p1));
+          } else {
+            lo = min_nan(lo, p1);
+            hi = max_nan(hi, p1);
+          }
+        }
+      }
+      const GroupQuant gq = group_quant_from_range<BITS, SYM>(lo, hi);
+      // The error pass on pairs of channels. Per channel it is the sequence of
+      // the packer's group_offset_level (Markstein-corrected quotient, plus
+      // 1.5 * 2^23, clamp) and then deq = (level - 1.5 * 2^23) * step, formed
+      // as one fma with -1.5 * 2^23 * step (exact: the product has 13
+      // significant bits and the result at most 15), and e = w + deq * (-1/s).
+      const uint64_t rcp2 = f2_pack(gq.rcp, gq.rcp);
+      const uint64_t nsf2 = f2_pack(-gq.sf, -gq.sf);
+      const uint64_t sf2 = f2_pack(gq.sf, gq.sf);
+      const uint64_t magic2 = f2_pack(kRoundMagic, kRoundMagic);
+      const float nms = __fmul_rn(-kRoundMagic, gq.sf);
+      const uint64_t nms2 = f2_pack(nms, nms);
+
+      // E, one 64-channel slot at a time.
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int kt = 2 * g + h, es = kt % kFusedESlots;
+        if (kt >= kFusedESlots &&
+            (*abort_flag || !mbar_wait(&e_empty[es], ((kt / kFusedESlots) - 1) & 1, a.err, kAwqSpinLimit))) {
+          *abort_flag = 1;
+          break;
+        }
+        uint8_t* eslot = smem + kFusedEOff + es * kFusedESlot;
+#pragma unroll
+        for (int c8 = 0; c8 < 8; ++c8) {
+          const int c = 8 * h + c8;
+          const uint4 sv = sh[c];
+          const float4 r0 = rs[2 * c], r1 = rs[2 * c + 1];
+          const float rv[8] = {r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, r1.z, r1.w};
+          const uint32_t* wv = &wr[c].x;
+          const uint32_t* svv = &sv.x;
+          uint4 out;
+          uint32_t* o = &out.x;
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            float p0 = 0.0f, p1 = 0.0f;
+            fma2_f16_f32(p0, p1, wv[i], svv[i]);  // w * s, exact
+            const uint64_t ws2 = f2_pack(p0, p1);
+            const uint64_t q0 = f2_mul(ws2, rcp2);
+            const uint64_t rr = f2_fma(q0, nsf2, ws2);          // ws - q0 * step, exact
+            uint64_t lv = f2_add(f2_fma(rr, rcp2, q0), magic2);  // rounded quotient + 1.5 * 2^23
+            if (!SYM) {
+              const float2 l = f2_unpack(lv);
+              lv = f2_pack(fminf(l.x, gq.hi_b), fminf(l.y, gq.hi_b));
+            }
+            const uint64_t deq = f2_fma(lv, sf2, nms2);          // (level - zero) * step, exact
+            const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&wv[i]));
+            const float2 e = f2_unpack(f2_fma(deq, f2_pack(rv[2 * i], rv[2 * i + 1]), f2_pack(f.x, f.y)));
+            const __half2 eh = __floats2half2_rn(e.x, e.y);
+            o[i] = *reinterpret_cast<const uint32_t*>(&eh);
+          }
+          *reinterpret_cast<uint4*>(eslot + sw128_offset(r, (uint32_t)c8)) = out;
+        }
+        fence_proxy_async_smem();  // these generic writes -> the MMA's async-proxy reads
+        mbar_arrive(&e_full[es]);
+      }
+      if (*abort_flag) break;
+    }
+
+    // ---------------------------------------------------------------- epilogue
+    const int q = warp & 3;  // this warp's TMEM lane quarter
+    bool done = !__any_sync(0xffffffffu, *abort_flag != 0);
+    if (done) done = __all_sync(0xffffffffu, mbar_wait(accum, 0, a.err, kAwqSpinLimit));
+    double acc = 0.0;
+    if (done) {
+      tc_fence_after();
+#pragma unroll 1
+      for (int c0 = 0; c0 < kFusedTokens; c0 += 16) {
+        uint32_t v[16];
+        tmem_ld16(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)c0, v);
+        tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const double d = (double)__uint_as_float(v[i]);
+          acc = fma(d, d, acc);
+        }
+      }
+    } else {
+      *abort_flag = 1;
+    }
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    if (lane == 0) red[q] = acc;
+    asm volatile("bar.sync 1, 128;" ::: "memory");
+    if (warp == 2 && lane == 0 && !*abort_flag) {
+      const double tot = ((red[0] + red[1]) + red[2]) + red[3];
+      a.partial[((size_t)alpha * a.tiles + tile) * a.t_chunks + tc] = tot;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kFusedTokens);
+  }
+}
+
 // ------------------------------------------------------------------ finalize
 // One warp per alpha: lane l sums tiles l, l + 32, ... in that order, then a
 // fixed butterfly; the sums are deterministic.
@@ -360,13 +712,20 @@ static EncodeTiledFnA awq_encode_fn() {
 
 static size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
-AwqPlan plan_awq(int64_t T, int64_t K, const int64_t* N_i, int n_lin, int n_alpha) {
+// Workspace layout: mu, the candidate scales, the partial losses, and (two-
+// kernel path only) the error matrices of one batch of alphas.
+AwqPlan plan_awq(int64_t T, int64_t K, const int64_t* N_i, int n_lin, int n_alpha, bool fused) {
   AwqPlan p;
   p.N_total = 0;
   for (int i = 0; i < n_lin; ++i) p.N_total += N_i[i];
   p.t_tiles = (int)((T + 127) / 128);
   p.n_tiles = (int)((p.N_total + 127) / 128);
   p.tiles = p.t_tiles * p.n_tiles;
+  p.fused_tiles = 0;
+  for (int i = 0; i < n_lin; ++i) p.fused_tiles += (int)((N_i[i] + 127) / 128);
+  p.t_chunks = (int)((T + kFusedTokens - 1) / kFusedTokens);
+  const size_t partials = (size_t)n_alpha * (size_t)(p.tiles > p.fused_tiles * p.t_chunks ? p.tiles
+                                                                                        : p.fused_tiles * p.t_chunks);
   const size_t e_one = (size_t)p.N_total * (size_t)K * 2;
   int b = (int)(kAwqEBudget / (e_one ? e_one : 1));
   if (b < 1) b = 1;
@@ -378,20 +737,62 @@ AwqPlan plan_awq(int64_t T, int64_t K, const int64_t* N_i, int n_lin, int n_alph
   p.off_S = off;
   off = align256(off + (size_t)n_alpha * K * 2);
   p.off_partial = off;
-  off = align256(off + (size_t)n_alpha * p.tiles * 8);
+  off = align256(off + partials * 8);
   p.off_E = off;
-  off = align256(off + (size_t)p.batch * e_one);
+  if (!fused) off = align256(off + (size_t)p.batch * e_one);
   p.total = off;
   return p;
+}
+
+// The loss of every alpha by the fused kernel: one launch over
+// (alpha, row tile of one linear) x 512-token chunks, then the finalize.
+template <int BITS, bool SYM>
+static cudaError_t launch_fused_loss(EncodeTiledFnA enc, const CUtensorMap& tmX, const AwqPlan& p, int64_t K,
+                                     const void* const* W, const int64_t* N_i, int n_lin, const __half* S,
+                                     int n_alpha, double* partial, int* err, cudaStream_t st) {
+  FusedWMaps wm;
+  memset(&wm, 0, sizeof(wm));
+  FusedArgs fa;
+  fa.S = S;
+  fa.partial = partial;
+  fa.K = (int)K;
+  fa.n_alpha = n_alpha;
+  fa.t_chunks = p.t_chunks;
+  fa.n_lin = n_lin;
+  fa.err = err;
+  fa.tile_off[0] = 0;
+  for (int i = 0; i < kAwqMaxLinears; ++i) {
+    if (i < n_lin) {
+      cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)N_i[i]};
+      cuuint64_t strides[1] = {(cuuint64_t)K * 2};
+      cuuint32_t box[2] = {64, 128};
+      cuuint32_t es[2] = {1, 1};
+      if (enc(&wm.m[i], CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(W[i]), dims, strides, box, es,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return cudaErrorInvalidValue;
+      fa.tile_off[i + 1] = fa.tile_off[i] + (int)((N_i[i] + 127) / 128);
+    } else {
+      fa.tile_off[i + 1] = fa.tile_off[i];
+    }
+  }
+  fa.tiles = fa.tile_off[n_lin];
+  if ((int64_t)fa.tiles * n_alpha > (int64_t)INT32_MAX || p.t_chunks > 65535) return cudaErrorInvalidConfiguration;
+  cudaError_t e = cudaFuncSetAttribute(awq_loss_fused_kernel<BITS, SYM>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)kFusedSmemLaunch);
+  if (e != cudaSuccess) return e;
+  awq_loss_fused_kernel<BITS, SYM><<<dim3((unsigned)(fa.tiles * n_alpha), (unsigned)p.t_chunks), kFusedThreads,
+                                     kFusedSmemLaunch, st>>>(wm, tmX, fa);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_awq_search(const void* X, int64_t T, int64_t K, const void* const* W, const int64_t* N_i,
                               int n_lin, int bits, bool sym, const double* alpha, int n_alpha, void* s_out,
                               double* mu_out, double* loss_out, int32_t* best_out, void* workspace, int* err,
-                              cudaStream_t st) {
+                              bool fused, cudaStream_t st) {
   EncodeTiledFnA enc = awq_encode_fn();
   if (!enc) return cudaErrorNotSupported;
-  const AwqPlan p = plan_awq(T, K, N_i, n_lin, n_alpha);
+  const AwqPlan p = plan_awq(T, K, N_i, n_lin, n_alpha, fused);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   double* mu = mu_out ? mu_out : reinterpret_cast<double*>(ws + p.off_mu);
   __half* S = reinterpret_cast<__half*>(ws + p.off_S);
@@ -424,6 +825,17 @@ cudaError_t launch_awq_search(const void* X, int64_t T, int64_t K, const void* c
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return cudaErrorInvalidValue;
+  }
+  if (fused) {
+    cudaError_t e;
+#define WQ_FL(BI, SY) e = launch_fused_loss<BI, SY>(enc, tmX, p, K, W, N_i, n_lin, S, n_alpha, partial, err, st)
+    if (bits == 4) { if (sym) WQ_FL(4, true); else WQ_FL(4, false); }
+    else { if (sym) WQ_FL(3, true); else WQ_FL(3, false); }
+#undef WQ_FL
+    if (e != cudaSuccess) return e;
+    awq_finalize_kernel<<<1, 256, 0, st>>>(partial, p.fused_tiles * p.t_chunks, n_alpha, S, (int)K, loss_out,
+                                            best_out, static_cast<__half*>(s_out), err);
+    return cudaGetLastError();
   }
   const int stages = 3;
   const size_t smem = 1024 + (size_t)stages * kLossStageBytes + (2 * stages + 1) * 8 + 4 * 8 + 16;
@@ -502,21 +914,22 @@ static uint8_t* awq_static_scratch() {
   return addr[dev];
 }
 
-bool awq_noalloc_fits(int64_t T, int64_t K, int64_t N_total, int n_alpha) {
+bool awq_noalloc_fits(int64_t T, int64_t K, const int64_t* N_i, int n_lin, int n_alpha, bool fused) {
   if (K > kAwqStaticMaxK || n_alpha > kAwqMaxAlpha) return false;
-  const int64_t tiles = ((T + 127) / 128) * ((N_total + 127) / 128);
+  const AwqPlan p = plan_awq(T, K, N_i, n_lin, n_alpha, fused);  // tile counts only
+  const int64_t tiles = fused ? (int64_t)p.fused_tiles * p.t_chunks : (int64_t)p.tiles;
   return (size_t)n_alpha * (size_t)tiles * 8 <= kAwqStaticPartial;
 }
 
 cudaError_t launch_awq_search_noalloc(const void* X, int64_t T, int64_t K, const void* const* W,
                                       const int64_t* N_i, int n_lin, int bits, bool sym, const double* alpha,
                                       int n_alpha, void* s_out, double* mu_out, double* loss_out, int32_t* best_out,
-                                      int* err, cudaStream_t st) {
+                                      int* err, bool fused, cudaStream_t st) {
   EncodeTiledFnA enc = awq_encode_fn();
   if (!enc) return cudaErrorNotSupported;
   uint8_t* ws = awq_static_scratch();
   if (!ws) return cudaErrorInvalidSymbol;
-  const AwqPlan p = plan_awq(T, K, N_i, n_lin, n_alpha);  // tile counts only; no memory of its own
+  const AwqPlan p = plan_awq(T, K, N_i, n_lin, n_alpha, fused);  // tile counts only; no memory of its own
   double* mu = mu_out ? mu_out : reinterpret_cast<double*>(ws);
   __half* S = reinterpret_cast<__half*>(ws + kAwqStaticMu);
   double* partial = reinterpret_cast<double*>(ws + kAwqStaticMu + kAwqStaticS);
@@ -538,6 +951,17 @@ cudaError_t launch_awq_search_noalloc(const void* X, int64_t T, int64_t K, const
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return cudaErrorInvalidValue;
+  }
+  if (fused) {  // no error matrix: the partial losses are the only scratch
+    cudaError_t e;
+#define WQ_FL(BI, SY) e = launch_fused_loss<BI, SY>(enc, tmX, p, K, W, N_i, n_lin, S, n_alpha, partial, err, st)
+    if (bits == 4) { if (sym) WQ_FL(4, true); else WQ_FL(4, false); }
+    else { if (sym) WQ_FL(3, true); else WQ_FL(3, false); }
+#undef WQ_FL
+    if (e != cudaSuccess) return e;
+    awq_finalize_kernel<<<1, 256, 0, st>>>(partial, p.fused_tiles * p.t_chunks, n_alpha, S, (int)K, loss_out,
+                                            best_out, static_cast<__half*>(s_out), err);
+    return cudaGetLastError();
   }
   const int stages = 3;
   const size_t smem = 1024 + (size_t)stages * kLossStageBytes + (2 * stages + 1) * 8 + 4 * 8 + 16;

@@ -284,6 +284,196 @@ w4a16_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
   }
 }
 
+// The same GEMM with the dequantized weight tile in shared memory: the
+// dequantizing warps store it (128-byte swizzled, K-major: the layout
+// desc_kmajor_sw128 describes) into a two-buffer ring and both MMA operands
+// come from shared memory; tensor memory holds only the accumulator. A
+// buffer is published with fence.proxy.async and an mbarrier arrival right
+// after its stores, where the tensor-memory A path must first wait for its
+// tcgen05.st to complete. One warp quartet dequantizes (each thread a row).
+template <int BK>
+__global__ void __launch_bounds__(192, 1)
+w4a16_gemm_tc_smem_a_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmP,
+                            TcArgs a) {
+  constexpr int NA = 2;                           // A buffers
+  constexpr int kPackedStage = kTcRows * BK / 2;  // bytes of the packed tile
+  constexpr int kABytes = kTcRows * BK * 2;       // one dequantized A tile
+  constexpr int kXBoxes = BK / 64;
+  constexpr int kWords = BK / 8;                  // packed words per thread (its row) and stage
+  constexpr int kChunks = kWords / 4;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int S = a.stages;
+  const int xbox = a.BN * 128;
+  const int stage_bytes = kXBoxes * xbox + kPackedStage;
+  uint8_t* abuf = smem + (size_t)S * stage_bytes;  // stage_bytes is a multiple of 1024
+  uint64_t* full = reinterpret_cast<uint64_t*>(abuf + NA * kABytes);
+  uint64_t* sempty = full + S;
+  uint64_t* afull = sempty + S;
+  uint64_t* aempty = afull + NA;
+  uint64_t* accum = aempty + NA;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accum + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  auto stageX = [&](int s) { return smem + (size_t)s * stage_bytes; };
+  auto stageP = [&](int s) { return smem + (size_t)s * stage_bytes + kXBoxes * xbox; };
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int n0 = blockIdx.x * kTcRows;
+  const int KT = a.K / BK;
+  const int G = a.K / kGroup;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&sempty[s], 1);
+    }
+    for (int b = 0; b < NA; ++b) {
+      mbar_init(&afull[b], 128);
+      mbar_init(&aempty[b], 1);
+    }
+    mbar_init(accum, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, a.tmem_cols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ---------------------------------------------------------- TMA producer
+    if (lane == 0) {
+      prefetch_tensormap(&tmX);
+      prefetch_tensormap(&tmP);
+      int issued = 0;
+      for (int kt = 0, s = 0, u = 0; kt < (a.stall ? 0 : KT); ++kt) {  // s = kt % S, u = kt / S
+        if (*abort_flag) break;
+        if (u > 0 && !mbar_wait(&sempty[s], (u - 1) & 1, a.err, a.spin_limit)) { *abort_flag = 1; break; }
+        mbar_arrive_expect_tx(&full[s], (uint32_t)stage_bytes);
+#pragma unroll
+        for (int i = 0; i < kXBoxes; ++i) tma_load_2d(stageX(s) + i * xbox, &tmX, kt * BK + 64 * i, 0, &full[s]);
+        tma_load_2d(stageP(s), &tmP, kt * (BK / 8), n0, &full[s]);
+        issued = kt + 1;
+        if (++s == S) { s = 0; ++u; }
+      }
+      for (int kt = issued > S ? issued - S : 0; kt < issued; ++kt)
+        mbar_wait(&full[kt % S], (kt / S) & 1, a.err, a.spin_limit);
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc = idesc_f16_f32(kTcRows, a.BN);
+      int committed = -1;
+      for (int kt = 0, s = 0, b = 0, ub = 0; kt < KT; ++kt) {
+        if (*abort_flag) break;
+        if (!mbar_wait(&afull[b], ub & 1, a.err, a.spin_limit)) { *abort_flag = 1; break; }
+        tc_fence_after();
+        const uint32_t xaddr = smem_u32(stageX(s));
+        const uint32_t aaddr = smem_u32(abuf + b * kABytes);
+#pragma unroll
+        for (int j = 0; j < BK / 16; ++j) {
+          const uint32_t koff = (uint32_t)((j >> 2) * (kTcRows * 128) + (j & 3) * 32);
+          const uint64_t ad = desc_kmajor_sw128(aaddr + koff);
+          const uint64_t bd = desc_kmajor_sw128(xaddr + (uint32_t)((j >> 2) * xbox + (j & 3) * 32));
+          mma_f16_ss(tmem, ad, bd, idesc, (kt > 0 || j > 0) ? 1u : 0u);
+        }
+        mma_commit(&aempty[b]);
+        mma_commit(&sempty[s]);
+        committed = kt;
+        if (++s == S) s = 0;
+        if (++b == NA) { b = 0; ++ub; }
+      }
+      mma_commit(accum);
+      if (*abort_flag && committed >= 0)  // let issued MMAs finish before teardown
+        mbar_wait(&aempty[committed % NA], (committed / NA) & 1, a.err, a.spin_limit);
+    }
+  } else {
+    // ---------------------------------------------------------- dequant + epilogue
+    const int q = warp & 3;             // TMEM lane quarter this warp may access
+    const int r = 32 * q + lane;        // output channel within the tile (the A row it writes)
+    const int n = n0 + r;
+    const bool row_ok = n < a.N;
+    __half st_cur = __float2half(0.f), zr_cur = __float2half(0.f);
+    __half st_next = __float2half(0.f), zr_next = __float2half(0.f);
+    if (row_ok) {
+      st_next = a.steps[(size_t)n * G];
+      zr_next = a.zeros[(size_t)n * G];
+    }
+    for (int kt = 0, s = 0, u = 0, b = 0, ub = 0; kt < KT; ++kt) {
+      if (__any_sync(0xffffffffu, *abort_flag != 0)) break;
+      const int g = (kt * BK) / kGroup;
+      if ((kt * BK) % kGroup == 0) {  // a new group starts: take its prefetched scales, fetch the next
+        st_cur = st_next;
+        zr_cur = zr_next;
+        if (row_ok && g + 1 < G) {
+          st_next = a.steps[(size_t)n * G + g + 1];
+          zr_next = a.zeros[(size_t)n * G + g + 1];
+        }
+      }
+      const __half2 s2 = __halves2half2(st_cur, st_cur);
+      const __half z1024 = __hadd(zr_cur, __float2half(1024.f));
+      const __half z64n = __hneg(__hadd(zr_cur, __float2half(64.f)));
+      const __half2 zz = __halves2half2(z1024, z1024);
+      const __half2 zz16n = __halves2half2(z64n, z64n);
+      const bool landed = mbar_wait(&full[s], u & 1, a.err, a.spin_limit);
+      if (!__all_sync(0xffffffffu, landed)) { *abort_flag = 1; break; }
+      uint32_t words[kWords];
+      const uint8_t* prow = stageP(s) + r * (BK / 2);
+      const int sw = BK == 128 ? (r >> 1) & 3 : (r >> 2) & 1;  // the packed tile's TMA swizzle
+#pragma unroll
+      for (int i = 0; i < kChunks; ++i) {
+        const uint4 v = *reinterpret_cast<const uint4*>(prow + ((i ^ sw) << 4));
+        words[4 * i] = v.x; words[4 * i + 1] = v.y; words[4 * i + 2] = v.z; words[4 * i + 3] = v.w;
+      }
+      bool ok = true;
+      if (kt >= NA) ok = mbar_wait(&aempty[b], (ub - 1) & 1, a.err, a.spin_limit);
+      if (!__all_sync(0xffffffffu, ok)) { *abort_flag = 1; break; }
+      uint8_t* arow = abuf + b * kABytes;
+#pragma unroll
+      for (int j = 0; j < kWords; ++j)  // word j: channels 8j .. 8j + 7, one 16-byte chunk of the row
+        *reinterpret_cast<uint4*>(arow + (j >> 3) * (kTcRows * 128) + sw128_offset((uint32_t)r, (uint32_t)(j & 7))) =
+            dequant_word4(words[j], zz, zz16n, s2);
+      fence_proxy_async_smem();  // these generic writes -> the MMA's async-proxy reads
+      mbar_arrive(&afull[b]);
+      if (++s == S) { s = 0; ++u; }
+      if (++b == NA) { b = 0; ++ub; }
+    }
+    // Epilogue: D[n][m] from TMEM -> Y[m][n].
+    bool done = !__any_sync(0xffffffffu, *abort_flag != 0);
+    if (done) done = __all_sync(0xffffffffu, mbar_wait(accum, 0, a.err, a.spin_limit));
+    if (done) {
+      tc_fence_after();
+      for (int c0 = 0; c0 < a.BN; c0 += 16) {
+        uint32_t v[16];
+        tmem_ld16(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)c0, v);
+        tmem_ld_wait();
+        if (row_ok) {
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const int m = c0 + i;
+            if (m < a.M) a.Y[(size_t)m * a.N + n] = __float2half_rn(__uint_as_float(v[i]));
+          }
+        }
+      }
+    } else {
+      *abort_flag = 1;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, a.tmem_cols);
+  }
+}
+
 // ---------------------------------------------------------------------------
 // Host side
 // ---------------------------------------------------------------------------
@@ -319,7 +509,7 @@ static uint32_t pow2_cols(uint32_t c) {
 // WQ_ERR_TIMEOUT latched).
 cudaError_t launch_gemm_tc(const void* X, const uint32_t* packed, const void* steps, const void* zeros, int64_t M,
                            int64_t N, int64_t K, void* Y, int* err, cudaStream_t st, int stages_opt, int bk_opt,
-                           int dw_opt, int wait_ms, bool stall) {
+                           int dw_opt, int wait_ms, bool stall, bool a_smem) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return cudaErrorNotSupported;
   for (int64_t m0 = 0; m0 < M; m0 += 256) {
@@ -358,6 +548,39 @@ cudaError_t launch_gemm_tc(const void* X, const uint32_t* packed, const void* st
     a.N = (int)N;
     a.K = (int)K;
     a.BN = BN;
+    a.err = err;
+    a.spin_limit = (long long)wait_ms * 2000000LL;  // cycles at <= 2 GHz: at least wait_ms
+    a.stall = stall ? 1 : 0;
+    if (a_smem) {  // A tiles in shared memory (two buffers); TMEM holds only the accumulator
+      a.tmem_cols = pow2_cols((uint32_t)BN);
+      const int stage = (BK / 64) * BN * 128 + kTcRows * BK / 2;
+      const size_t abytes = 2 * (size_t)kTcRows * BK * 2;
+      auto share = [](int c) { return (size_t)(225 * 1024) / (size_t)c - 3 * 1024; };
+      int cps = 512 / (int)a.tmem_cols;
+      if (cps > 4) cps = 4;
+      int S;
+      if (stages_opt > 0) {
+        S = stages_opt;
+        while (cps > 1 && (size_t)S * stage + abytes + 2048 > share(cps)) cps /= 2;
+        if ((size_t)S * stage + abytes + 2048 > share(1)) return cudaErrorInvalidValue;
+      } else {
+        while (cps > 1 && 3 * (size_t)stage + abytes + 2048 > share(cps)) cps /= 2;
+        S = (int)((share(cps) - abytes - 2048) / stage);
+        if (S > 16) S = 16;
+        if (S < 2) S = 2;
+      }
+      a.stages = S;
+      size_t smem = 1024 + (size_t)S * stage + abytes + (2 * S + 2 * 2 + 1) * 8 + 16;
+      const size_t smem_floor = (size_t)(228 * 1024) / (size_t)(cps + 1) + 1024;
+      if (smem < smem_floor) smem = smem_floor;
+      auto kern = BK == 128 ? w4a16_gemm_tc_smem_a_kernel<128> : w4a16_gemm_tc_smem_a_kernel<64>;
+      cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      if (e != cudaSuccess) return e;
+      kern<<<dim3((unsigned)((N + kTcRows - 1) / kTcRows)), 192, smem, st>>>(tmX, tmP, a);
+      e = cudaGetLastError();
+      if (e != cudaSuccess) return e;
+      continue;
+    }
     // A third A buffer when it still fits the same TMEM allocation
     const int NA = pow2_cols((uint32_t)(BN + 3 * BK / 2)) == pow2_cols((uint32_t)(BN + 2 * BK / 2)) ? 3 : 2;
     a.tmem_cols = pow2_cols((uint32_t)(BN + NA * BK / 2));
@@ -379,9 +602,6 @@ cudaError_t launch_gemm_tc(const void* X, const uint32_t* packed, const void* st
       if (S < 2) S = 2;
     }
     a.stages = S;
-    a.err = err;
-    a.spin_limit = (long long)wait_ms * 2000000LL;  // cycles at <= 2 GHz: at least wait_ms
-    a.stall = stall ? 1 : 0;
     size_t smem = 1024 + (size_t)S * stage + (2 * S + 2 * kTcMaxABufs + 1) * 8 + 16;
     // At most cps CTAs per SM (their TMEM must fit at once): ask for more than
     // 1/(cps+1) of the SM's shared memory.

@@ -51,11 +51,13 @@ struct RowsArgs {
 };
 
 // One row batch of this lane: WPR packed words per row (4-bit: 4 per 32
-// channels, 3-bit: 3 per 32 channels) and the rows' step and zero.
-template <int R, int WPR>
+// channels, 3-bit: 3 per 32 channels) and the step and zero of RL rows: all R
+// rows, or (group-first reduction) the RL rows whose group totals this lane
+// finishes.
+template <int R, int WPR, int RL = R>
 struct RowsStage {
   uint32_t w[R][WPR];
-  __half sc[R], zh[R];
+  __half sc[RL], zh[RL];
 };
 
 __device__ __forceinline__ uint2 ld_stream_v2(const void* p) {
@@ -84,30 +86,34 @@ __device__ __forceinline__ void load_row_words(uint32_t (&w)[WPR], const uint32_
 
 // Loads of one row batch for this lane: pw / ps / pz point at the lane's words,
 // step and zero in the batch's first row; nrows = rows of the batch inside N
-// (0 for a lane past K). Full batches take the unpredicated path.
-template <int R, int WPR>
-__device__ __forceinline__ void rows_issue(RowsStage<R, WPR>& s, const uint32_t* pw, const __half* ps,
-                                           const __half* pz, size_t row_words, int G, int nrows) {
+// (0 for a lane past K); the step and zero are those of rows lrow0 .. lrow0 +
+// RL - 1 of the batch. Full batches take the unpredicated path.
+template <int R, int WPR, int RL>
+__device__ __forceinline__ void rows_issue(RowsStage<R, WPR, RL>& s, const uint32_t* pw, const __half* ps,
+                                           const __half* pz, size_t row_words, int G, int nrows, int lrow0) {
   if (nrows >= R) {
 #pragma unroll
-    for (int r = 0; r < R; ++r) {
-      load_row_words<WPR>(s.w[r], pw + r * row_words);
-      s.sc[r] = ps[(size_t)r * G];
-      s.zh[r] = pz[(size_t)r * G];
+    for (int r = 0; r < R; ++r) load_row_words<WPR>(s.w[r], pw + r * row_words);
+#pragma unroll
+    for (int i = 0; i < RL; ++i) {
+      s.sc[i] = ps[(size_t)(lrow0 + i) * G];
+      s.zh[i] = pz[(size_t)(lrow0 + i) * G];
     }
   } else {
 #pragma unroll
     for (int r = 0; r < R; ++r) {
       if (r < nrows) {
         load_row_words<WPR>(s.w[r], pw + r * row_words);
-        s.sc[r] = ps[(size_t)r * G];
-        s.zh[r] = pz[(size_t)r * G];
       } else {
 #pragma unroll
         for (int c = 0; c < WPR; ++c) s.w[r][c] = 0;
-        s.sc[r] = __float2half(0.f);
-        s.zh[r] = __float2half(0.f);
       }
+    }
+#pragma unroll
+    for (int i = 0; i < RL; ++i) {
+      const bool in = lrow0 + i < nrows;
+      s.sc[i] = in ? ps[(size_t)(lrow0 + i) * G] : __float2half(0.f);
+      s.zh[i] = in ? pz[(size_t)(lrow0 + i) * G] : __float2half(0.f);
     }
   }
 }
@@ -128,13 +134,43 @@ __device__ __forceinline__ void load_lane_x(uint32_t (&xh)[M][16 * CPL], const R
 }
 
 // ---------------------------------------------------------------- ActHalf
+// Group totals of a lane's offset term c1 and activation sum: the LPG = 4/CPL
+// lanes of one quantization group share step and zero, so the zero point and
+// the offsets are removed once per group (group-first reduction).
+template <int M, int CPL>
+__device__ __forceinline__ void group_totals(const float (&c1)[M], const float (&xsum)[M], float (&c1g)[M],
+                                             float (&xg)[M]) {
+#pragma unroll
+  for (int m = 0; m < M; ++m) {
+    float c = c1[m], x = xsum[m];
+#pragma unroll
+    for (int o = 1; o < 4 / CPL; o <<= 1) {
+      c += __shfl_xor_sync(0xffffffffu, c, o);
+      x += __shfl_xor_sync(0xffffffffu, x, o);
+    }
+    c1g[m] = c;
+    xg[m] = x;
+  }
+}
+
+// step * (T - c1g - zero * xg) for a group total T of activation row m.
+template <int M>
+__device__ __forceinline__ float group_epilogue(const float (&c1g)[M], const float (&xg)[M], int m, float t,
+                                                __half sc, __half zh) {
+  const float c = (M == 1 || m == 0) ? c1g[0] : c1g[M - 1];
+  const float x = (M == 1 || m == 0) ? xg[0] : xg[M - 1];
+  return __half2float(sc) * fmaf(-__half2float(zh), x, t - c);
+}
+
 template <int M, int CPL>
 struct ActHalf {
+  static constexpr bool kGroupFirst = true;  // compute() leaves step and zero to the group epilogue
   uint32_t xh[M][16 * CPL];
-  float c1[M], xsum[M];
+  float c1g[M], xg[M];
 
   __device__ __forceinline__ void load(const RowsArgs& a, int k0, bool active) {
     load_lane_x<M, CPL>(xh, a, k0, active);
+    float c1[M], xsum[M];
 #pragma unroll
     for (int m = 0; m < M; ++m) {
       float x1 = 0.f, x2 = 0.f;  // channel classes {0,1,4,5} and {2,3,6,7} mod 8
@@ -147,10 +183,17 @@ struct ActHalf {
       c1[m] = 1024.f * x1 + 64.f * x2;
       xsum[m] = x1 + x2;
     }
+    group_totals<M, CPL>(c1, xsum, c1g, xg);
   }
 
-  template <int R>
-  __device__ __forceinline__ void compute(const RowsStage<R, 4 * CPL>& s, float (&acc)[R * M]) const {
+  __device__ __forceinline__ float epilogue(int m, float t, __half sc, __half zh) const {
+    return group_epilogue<M>(c1g, xg, m, t, sc, zh);
+  }
+
+  // acc[r*M + m] = this lane's A1 + A2/16 (sum_k x (1024 + q) with the x16
+  // class scaled back), before the offsets, the zero point and the step.
+  template <int R, int RL>
+  __device__ __forceinline__ void compute(const RowsStage<R, 4 * CPL, RL>& s, float (&acc)[R * M]) const {
 #pragma unroll
     for (int r = 0; r < R; ++r) {
       float a[M][4];
@@ -172,15 +215,9 @@ struct ActHalf {
           fma2_f16_f32(a[m][2], a[m][3], xh[m][4 * j + 3], p3);
         }
       }
-      const float sc = __half2float(s.sc[r]);
-      const float z = __half2float(s.zh[r]);
 #pragma unroll
-      for (int m = 0; m < M; ++m) {
-        // sum_k x (q - z) = A1 + A2/16 - (1024 X1 + 64 X2) - z (X1 + X2)
-        float t = fmaf(a[m][2] + a[m][3], 0.0625f, a[m][0] + a[m][1]) - c1[m];
-        t = fmaf(-z, xsum[m], t);
-        acc[r * M + m] = sc * t;
-      }
+      for (int m = 0; m < M; ++m)  // sum_k x (q - z) = A1 + A2/16 - (1024 X1 + 64 X2) - z (X1 + X2)
+        acc[r * M + m] = fmaf(a[m][2] + a[m][3], 0.0625f, a[m][0] + a[m][1]);
     }
   }
 };
@@ -195,11 +232,17 @@ struct ActHalf {
 // per row with the lane's activation class sums, as in ActHalf.
 template <int M, int CPL>
 struct ActHalf3 {
+  static constexpr bool kGroupFirst = true;  // compute() leaves step and zero to the group epilogue
   uint32_t xh[M][16 * CPL];
-  float c1[M], xsum[M];
+  float c1g[M], xg[M];
+
+  __device__ __forceinline__ float epilogue(int m, float t, __half sc, __half zh) const {
+    return group_epilogue<M>(c1g, xg, m, t, sc, zh);
+  }
 
   __device__ __forceinline__ void load(const RowsArgs& a, int k0, bool active) {
     load_lane_x<M, CPL>(xh, a, k0, active);
+    float c1[M], xsum[M];
 #pragma unroll
     for (int m = 0; m < M; ++m) {
       float x1 = 0.f, x8 = 0.f, x64 = 0.f;
@@ -215,10 +258,13 @@ struct ActHalf3 {
       c1[m] = 1024.f * x1 + 128.f * x8 + 16.f * x64;
       xsum[m] = x1 + x8 + x64;
     }
+    group_totals<M, CPL>(c1, xsum, c1g, xg);
   }
 
-  template <int R>
-  __device__ __forceinline__ void compute(const RowsStage<R, 3 * CPL>& s, float (&acc)[R * M]) const {
+  // acc[r*M + m] = this lane's A1 + A8/8 + A64/64, before the offsets, the
+  // zero point and the step.
+  template <int R, int RL>
+  __device__ __forceinline__ void compute(const RowsStage<R, 3 * CPL, RL>& s, float (&acc)[R * M]) const {
 #pragma unroll
     for (int r = 0; r < R; ++r) {
       float a[M][6];  // (x1, x8, x64) classes, low and high lanes
@@ -255,15 +301,10 @@ struct ActHalf3 {
 #pragma unroll
         for (int m = 0; m < M; ++m) fma2_f16_f32(a[m][0], a[m][1], xh[m][16 * c + 15], p30);
       }
-      const float sc = __half2float(s.sc[r]);
-      const float z = __half2float(s.zh[r]);
 #pragma unroll
-      for (int m = 0; m < M; ++m) {
+      for (int m = 0; m < M; ++m)
         // sum_k x (q - z) = A1 + A8/8 + A64/64 - (1024 X1 + 128 X8 + 16 X64) - z (X1 + X8 + X64)
-        float t = fmaf(a[m][4] + a[m][5], 0.015625f, fmaf(a[m][2] + a[m][3], 0.125f, a[m][0] + a[m][1])) - c1[m];
-        t = fmaf(-z, xsum[m], t);
-        acc[r * M + m] = sc * t;
-      }
+        acc[r * M + m] = fmaf(a[m][4] + a[m][5], 0.015625f, fmaf(a[m][2] + a[m][3], 0.125f, a[m][0] + a[m][1]));
     }
   }
 };
@@ -286,6 +327,7 @@ __device__ __forceinline__ uint32_t pack_bytes(int b0, int b1, int b2, int b3) {
 
 template <int M, int CPL>
 struct ActInt {
+  static constexpr bool kGroupFirst = false;  // per-lane fixed-point scale: step applied per lane
   // Digit t of the fixed-point image, four channels per word in the byte
   // order of the masked code words: lo[c] holds channels 8c + (0, 4, 1, 5)
   // (the low nibbles of the word's bytes), hi[c] channels 8c + (2, 6, 3, 7).
@@ -337,8 +379,11 @@ struct ActInt {
     }
   }
 
-  template <int R>
-  __device__ __forceinline__ void compute(const RowsStage<R, 4 * CPL>& s, float (&acc)[R * M]) const {
+  __device__ __forceinline__ float epilogue(int, float t, __half, __half) const { return t; }
+
+  template <int R, int RL>
+  __device__ __forceinline__ void compute(const RowsStage<R, 4 * CPL, RL>& s, float (&acc)[R * M]) const {
+    static_assert(RL == R, "the integer-digit path applies every row's step per lane");
     // Words outer, rows inner: R*M*3 independent dp4a chains.
     int a[R][M][3];
 #pragma unroll
@@ -403,6 +448,58 @@ __device__ __forceinline__ float butterfly_reduce(float (&v)[NV], int lane, int&
   return t;
 }
 
+// Group-first variant: the transposing halvings run over the low lane bits
+// first, so after the LPG lanes of a quantization group (which share step and
+// zero) have been combined, each lane holds group totals of consecutive values
+// index, index + 1, ...; epi(i, t) turns value index + i's total t into its
+// stepped, zero-corrected contribution; the remaining lane bits then finish
+// the sum. Afterwards lane l < NV holds the total of value `index` (= l's
+// bit-reversal-free position: the halvings assign it), and every lane whose
+// low log2(NV) bits equal l's holds the same total.
+template <int NV, int LPG>
+__device__ __forceinline__ int group_first_index(int lane) {
+  int index = 0, c = NV;
+#pragma unroll
+  for (int o = 1; o < LPG; o <<= 1) {
+    if (c > 1) {
+      c /= 2;
+      if (lane & o) index += c;
+    }
+  }
+  return index;
+}
+
+template <int NV, int LPG, class Epi>
+__device__ __forceinline__ float group_first_reduce(float (&v)[NV], int lane, int& index, Epi epi) {
+  index = 0;
+  int c = NV;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    if (o == LPG) {  // the group's lanes are combined: apply step and zero
+#pragma unroll
+      for (int i = 0; i < NV; ++i)
+        if (i < c) v[i] = epi(i, v[i]);
+    }
+    if (c > 1) {
+      const int half = c / 2;
+      const bool upper = (lane & o) != 0;
+#pragma unroll
+      for (int i = 0; i < NV / 2; ++i) {
+        if (i < half) {
+          const float send = upper ? v[i] : v[i + half];
+          const float keep = upper ? v[i + half] : v[i];
+          v[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+        }
+      }
+      if (upper) index += half;
+      c = half;
+    } else {
+      v[0] += __shfl_xor_sync(0xffffffffu, v[0], o);
+    }
+  }
+  return v[0];
+}
+
 // At most 8 warps: K <= 8192 with 32 channels per lane, K <= 16384 with 64.
 // MINB: minimum CTAs per SM for the register allocation: 3 (85 registers)
 // for the M = 1, 32-channel, two-stage instance, 2 (128 registers) for the
@@ -427,15 +524,25 @@ gemv_rows_kernel(RowsArgs a) {
   const int nbatch = (a.N + R - 1) / R;
   const int my = blockIdx.x < nbatch ? (nbatch - 1 - blockIdx.x) / gridDim.x + 1 : 0;
 
+  // Group-first reduction (step and zero applied to group totals): this lane
+  // finishes the values gidx .. gidx + CG - 1 of each batch, so it loads the
+  // step and zero of their RL rows only.
+  constexpr bool GF = Act<M, CPL>::kGroupFirst;
+  constexpr int LPG = 4 / CPL;  // lanes of one quantization group
+  constexpr int CG = GF ? (NV / LPG > 1 ? NV / LPG : 1) : NV;
+  constexpr int RL = GF ? (CG / M > 1 ? CG / M : 1) : R;
+  const int gidx = GF ? group_first_index<NV, LPG>(lane) : 0;
+  const int lrow0 = gidx / M;
+
   // S register stages: batches i+1 .. i+S-1 are in flight while batch i is
   // computed. The first S-1 are requested before the dependent-launch wait.
-  RowsStage<R, WPR> st[S];
-  auto issue = [&](RowsStage<R, WPR>& stage, int j) {  // local batch j of this CTA
+  RowsStage<R, WPR, RL> st[S];
+  auto issue = [&](RowsStage<R, WPR, RL>& stage, int j) {  // local batch j of this CTA
     const int row0 = (blockIdx.x + j * gridDim.x) * R;
     const int left = a.N - row0;
     const size_t sg = (size_t)row0 * G + lane_group;
-    rows_issue<R, WPR>(stage, a.P + (size_t)row0 * row_words + lane_word, a.steps + sg, a.zeros + sg, row_words, G,
-                       active ? (left < R ? left : R) : 0);
+    rows_issue<R, WPR, RL>(stage, a.P + (size_t)row0 * row_words + lane_word, a.steps + sg, a.zeros + sg,
+                           row_words, G, active ? (left < R ? left : R) : 0, lrow0);
   };
 #pragma unroll
   for (int j = 0; j < S - 1; ++j)
@@ -466,10 +573,20 @@ gemv_rows_kernel(RowsArgs a) {
     first += nslots;
     slot = 0;
   };
-  auto finish = [&]() {
+  auto finish = [&](const RowsStage<R, WPR, RL>& sg) {
     int idx;
-    const float v = butterfly_reduce<NV>(acc, lane, idx);
-    if ((lane & (32 / NV - 1)) == 0) red[((half * NB + slot) * nseg + warp) * NV + idx] = v;
+    float v;
+    if constexpr (GF) {
+      v = group_first_reduce<NV, LPG>(acc, lane, idx, [&](int i, float t) {
+        const int gi = gidx + i;        // value index: batch row gi / M, activation row gi % M
+        const int rr = gi / M - lrow0;  // which of this lane's RL step/zero rows
+        return act.epilogue(gi % M, t, rr == 0 ? sg.sc[0] : sg.sc[RL - 1], rr == 0 ? sg.zh[0] : sg.zh[RL - 1]);
+      });
+    } else {
+      v = butterfly_reduce<NV>(acc, lane, idx);
+    }
+    const bool writer = GF ? lane < NV : (lane & (32 / NV - 1)) == 0;
+    if (writer) red[((half * NB + slot) * nseg + warp) * NV + idx] = v;
     if (++slot == NB) flush(NB);
   };
 
@@ -479,8 +596,8 @@ gemv_rows_kernel(RowsArgs a) {
       if (i + j < my) {
         const int nx = i + j + S - 1;
         if (nx < my) issue(st[(j + S - 1) % S], nx);
-        act.template compute<R>(st[j], acc);
-        finish();
+        act.template compute<R, RL>(st[j], acc);
+        finish(st[j]);
       }
     }
   }

@@ -21,23 +21,25 @@ cudaError_t launch_gemv_rows(const void* X, const uint32_t* packed, const void* 
                              int grid_mode, bool pdl);
 cudaError_t launch_gemm_tc(const void* X, const uint32_t* packed, const void* steps, const void* zeros, int64_t M,
                            int64_t N, int64_t K, void* Y, int* err, cudaStream_t st, int stages_opt, int bk_opt,
-                           int dw_opt, int wait_ms, bool stall);
+                           int dw_opt, int wait_ms, bool stall, bool a_smem);
 // Workspace layout of the AWQ search (wq_awq.cu): mu, the candidate scales,
-// the per-tile partial losses, and the error matrices of one batch of alphas.
+// the per-tile partial losses, and (two-kernel loss path only) the error
+// matrices of one batch of alphas.
 struct AwqPlan {
   int64_t N_total;
   int t_tiles, n_tiles, tiles;
+  int fused_tiles, t_chunks;  // the fused loss kernel's row tiles and 512-token chunks
   int batch;  // alphas per E batch
   size_t off_mu, off_S, off_partial, off_E, total;
 };
-AwqPlan plan_awq(int64_t T, int64_t K, const int64_t* N_i, int n_lin, int n_alpha);
+AwqPlan plan_awq(int64_t T, int64_t K, const int64_t* N_i, int n_lin, int n_alpha, bool fused);
 cudaError_t launch_awq_search(const void* X, int64_t T, int64_t K, const void* const* W, const int64_t* N_i,
                               int n_lin, int bits, bool sym, const double* alpha, int n_alpha, void* s_out,
                               double* mu_out, double* loss_out, int32_t* best_out, void* workspace, int* err,
-                              cudaStream_t st);
-bool awq_noalloc_fits(int64_t T, int64_t K, int64_t N_total, int n_alpha);
+                              bool fused, cudaStream_t st);
+bool awq_noalloc_fits(int64_t T, int64_t K, const int64_t* N_i, int n_lin, int n_alpha, bool fused);
 cudaError_t launch_awq_search_noalloc(const void* X, int64_t T, int64_t K, const void* const* W,
                                       const int64_t* N_i, int n_lin, int bits, bool sym, const double* alpha,
                                       int n_alpha, void* s_out, double* mu_out, double* loss_out, int32_t* best_out,
-                                      int* err, cudaStream_t st);
+                                      int* err, bool fused, cudaStream_t st);
 }  // namespace wq

@@ -14,7 +14,8 @@
 // xor-shuffles. One wave of resident CTAs walks the units grid-stride, the
 // next unit's loads in flight while the current one is quantized. Per weight:
 // the correctly rounded quotient without a division (group_quotient), rint by
-// the 1.5 * 2^23 addition, and one integer multiply-add into the packed word.
+// the 1.5 * 2^23 addition (both on packed fp32 pairs, two channels per
+// instruction), and one integer multiply-add into the packed word.
 // 2 B/weight in, 0.5 (0.375) B/weight out.
 #include "wq_quant_core.cuh"
 #include "wq_launch.h"
@@ -71,8 +72,19 @@ __device__ __forceinline__ void quantize_unit(const uint4 (&raw)[4], const __hal
     if constexpr (HAS_S) return ws[i]; else return lane_half(raw, i);
   };
 
+  // the 32 offset levels, two channels per packed fp32 instruction
+  const uint64_t rcp2 = f2_pack(gq.rcp, gq.rcp);
+  const uint64_t nsf2 = f2_pack(-gq.sf, -gq.sf);
+  const uint64_t magic2 = f2_pack(kRoundMagic, kRoundMagic);
+  float lv[32];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const float2 l = group_offset_level2<BITS, SYM>(value(2 * i), value(2 * i + 1), gq, rcp2, nsf2, magic2);
+    lv[2 * i] = l.x;
+    lv[2 * i + 1] = l.y;
+  }
   uint32_t o[4];
-  pack_lane<BITS>([&](int i) { return group_offset_level<BITS, SYM>(value(i), gq); }, gq.zero, o);
+  pack_lane<BITS>([&](int i) { return lv[i]; }, gq.zero, o);
   if (!valid) return;
 
   if constexpr (BITS == 4) {

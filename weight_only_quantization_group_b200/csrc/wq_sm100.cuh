@@ -162,6 +162,11 @@ __device__ __forceinline__ uint64_t desc_kmajor_sw128(uint32_t addr) {
   return d;
 }
 
+// Byte offset of 16-byte chunk c of row r in a 128-row tile of 128-byte rows
+// stored with the 128-byte swizzle (what TMA writes for such a box, and what
+// desc_kmajor_sw128 describes): chunk c lands at c ^ (r mod 8).
+__device__ __forceinline__ uint32_t sw128_offset(uint32_t r, uint32_t c) { return r * 128u + ((c ^ (r & 7u)) << 4); }
+
 // Instruction descriptor: kind::f16, fp16 A and B (both K-major), fp32 D.
 __host__ __device__ constexpr uint32_t idesc_f16_f32(int m, int n) {
   return (1u << 4)                       // D format fp32
