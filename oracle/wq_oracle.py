@@ -54,6 +54,10 @@ __all__ = [
     "awq_error_matrix",
     "awq_loss",
     "awq_search",
+    "awq_fold_into_norm",
+    "awq_fold_into_linear_rows",
+    "decoder_block_ref",
+    "awq_fold_block",
     "MU_FLOOR",
 ]
 
@@ -374,3 +378,99 @@ def awq_search(X16: np.ndarray, Ws, bits: int, group: int, symmetric: bool,
     best = int(np.argmin(losses))
     return {"mu": mu, "candidates": S, "losses": losses, "best": best, "s": S[best].copy(),
             "alphas": np.asarray(alphas, dtype=np.float64)}
+
+
+# ---------------------------------------------------------------------------
+# AWQ scale folding ([MIT-Lab4/5] "Question 2": the searched scales are folded
+# into the previous LayerNorm or linear layer)
+# ---------------------------------------------------------------------------
+
+def awq_fold_into_norm(gamma: np.ndarray, s: np.ndarray) -> np.ndarray:
+    """gamma'_k = gamma_k / s_k: a normalisation layer whose output feeds the
+    scaled linears absorbs diag(s)^-1 into its per-channel weight
+    ([MIT-Lab4/5] "Question 2", scale_ln_fcs).
+
+    fp16 inputs: the library's stored form, fp16_RN(fp32(gamma) / fp32(s))
+    (one IEEE fp32 division, then one rounding to fp16). fp64 inputs: the
+    quotient in fp64 (used by the block-equivalence check).
+    """
+    gamma, s = np.asarray(gamma), np.asarray(s)
+    assert gamma.shape == s.shape and gamma.ndim == 1
+    if gamma.dtype == np.float16:
+        assert s.dtype == np.float16
+        return (gamma.astype(np.float32) / s.astype(np.float32)).astype(np.float16)
+    return gamma.astype(np.float64) / s.astype(np.float64)
+
+
+def awq_fold_into_linear_rows(W: np.ndarray, s: np.ndarray, b: np.ndarray | None = None):
+    """W'[n][k] = W[n][k] / s_n and b'_n = b_n / s_n: a linear whose output
+    feeds the scaled linears (v_proj before o_proj, up_proj before down_proj)
+    absorbs diag(s)^-1 into its output rows ([MIT-Lab4/5] "Question 2",
+    scale_fc_fc). s has one entry per output row of W. fp16 inputs follow
+    the stored-form contract of ``awq_fold_into_norm``; fp64 inputs fold in
+    fp64. Returns (W', b') (b' is None without a bias)."""
+    W, s = np.asarray(W), np.asarray(s)
+    assert W.ndim == 2 and s.shape == (W.shape[0],)
+    if W.dtype == np.float16:
+        assert s.dtype == np.float16
+        s32 = s.astype(np.float32)
+        Wf = (W.astype(np.float32) / s32[:, None]).astype(np.float16)
+        bf = None if b is None else (np.asarray(b).astype(np.float32) / s32).astype(np.float16)
+        return Wf, bf
+    s64 = s.astype(np.float64)
+    Wf = W.astype(np.float64) / s64[:, None]
+    bf = None if b is None else np.asarray(b, dtype=np.float64) / s64
+    return Wf, bf
+
+
+def _rmsnorm(x: np.ndarray, gamma: np.ndarray, eps: float) -> np.ndarray:
+    return x / np.sqrt(np.mean(x * x, axis=-1, keepdims=True) + eps) * gamma
+
+
+def decoder_block_ref(x: np.ndarray, p: dict, n_heads: int, eps: float = 1e-6) -> np.ndarray:
+    """One LLaMA-shaped decoder block in fp64, the computation the folded
+    scales must leave unchanged: pre-norm (RMS) causal multi-head attention
+    with q/k/v/o projections, then a pre-norm SwiGLU MLP (gate, up, down),
+    each with a residual connection. Linear weights are nn.Linear [out][in]
+    (y = x W^T). ``p`` holds gamma1, wq, wk, wv, wo, gamma2, wg, wu, wd."""
+    x = np.asarray(x, dtype=np.float64)
+    T, D = x.shape
+    hd = D // n_heads
+    h = _rmsnorm(x, p["gamma1"], eps)
+    q, k, v = h @ p["wq"].T, h @ p["wk"].T, h @ p["wv"].T
+    att = np.empty_like(q)
+    mask = np.triu(np.ones((T, T), dtype=bool), 1)
+    for i in range(n_heads):
+        sl = slice(i * hd, (i + 1) * hd)
+        a = q[:, sl] @ k[:, sl].T / np.sqrt(hd)
+        a[mask] = -np.inf
+        a = np.exp(a - a.max(axis=1, keepdims=True))
+        att[:, sl] = (a / a.sum(axis=1, keepdims=True)) @ v[:, sl]
+    y = x + att @ p["wo"].T
+    h2 = _rmsnorm(y, p["gamma2"], eps)
+    g, u = h2 @ p["wg"].T, h2 @ p["wu"].T
+    return y + ((g / (1.0 + np.exp(-g))) * u) @ p["wd"].T
+
+
+def awq_fold_block(p: dict, s_qkv, s_o, s_gu, s_down) -> dict:
+    """The four search places of a LLaMA block with their scales applied
+    ([MIT-Lab4/5] "Question 2": scales searched at the attention input, the
+    attention output, the MLP input and the down projection's input, then
+    folded into the previous norm or linear): each scaled linear's weight
+    becomes W diag(s) and the op that produces its input absorbs diag(s)^-1
+    (gamma1 for q/k/v, v_proj's rows for o_proj, gamma2 for gate/up,
+    up_proj's rows for down_proj). Every parameter is returned in fp64."""
+    f = {k: np.asarray(v, dtype=np.float64) for k, v in p.items()}
+    s_qkv, s_o, s_gu, s_down = (np.asarray(t, dtype=np.float64) for t in (s_qkv, s_o, s_gu, s_down))
+    out = dict(f)
+    out["gamma1"] = awq_fold_into_norm(f["gamma1"], s_qkv)
+    for name in ("wq", "wk", "wv"):
+        out[name] = f[name] * s_qkv[None, :]
+    out["wv"], _ = awq_fold_into_linear_rows(out["wv"], s_o)
+    out["wo"] = f["wo"] * s_o[None, :]
+    out["gamma2"] = awq_fold_into_norm(f["gamma2"], s_gu)
+    out["wg"] = f["wg"] * s_gu[None, :]
+    out["wu"] = f["wu"] * s_gu[None, :]
+    out["wu"], _ = awq_fold_into_linear_rows(out["wu"], s_down)
+    out["wd"] = f["wd"] * s_down[None, :]
+    return out

@@ -387,3 +387,96 @@ def test_awq_search_picks_minimum_and_beats_rtn():
     assert np.array_equal(r["s"], r["candidates"][r["best"]])
     # the loss at the chosen alpha is what awq_loss reports for that scale
     assert r["losses"][r["best"]] == O.awq_loss(X, Ws, r["s"], 4, 128, False)
+
+
+# ---------------------------------------------------------------------------
+# AWQ scale folding ("MIT 6.5940 Lab 4 + Lab 5", "Question 2")
+# ---------------------------------------------------------------------------
+
+def _block_params(g, D=64, H=96):
+    return {"gamma1": 1.0 + 0.1 * g.standard_normal(D), "wq": g.normal(0, 0.1, (D, D)),
+            "wk": g.normal(0, 0.1, (D, D)), "wv": g.normal(0, 0.1, (D, D)), "wo": g.normal(0, 0.1, (D, D)),
+            "gamma2": 1.0 + 0.1 * g.standard_normal(D), "wg": g.normal(0, 0.1, (H, D)),
+            "wu": g.normal(0, 0.1, (H, D)), "wd": g.normal(0, 0.1, (D, H))}
+
+
+def test_decoder_block_ref_closed_forms():
+    """Residual paths only when o and down are zero; one token attends to itself
+    (softmax over one key is 1), so its attention output is v."""
+    g = np.random.default_rng(31)
+    p = _block_params(g)
+    x = g.normal(0, 1, (5, 64))
+    z = dict(p, wo=np.zeros((64, 64)), wd=np.zeros((64, 96)))
+    assert np.array_equal(O.decoder_block_ref(x, z, 4), x)
+    x1 = x[:1]
+    h = x1 / np.sqrt(np.mean(x1 * x1) + 1e-6) * p["gamma1"]
+    y_attn_only = x1 + (h @ p["wv"].T) @ p["wo"].T
+    q = dict(p, wd=np.zeros((64, 96)))
+    assert np.allclose(O.decoder_block_ref(x1, q, 4), y_attn_only, rtol=1e-13, atol=1e-13)
+
+
+def test_fold_block_equivalence_fp64():
+    """Folding the four places' s^-1 into gamma1, v_proj's rows, gamma2 and
+    up_proj's rows while the scaled linears take W diag(s) leaves the block's
+    output unchanged (fp64: to rounding)."""
+    g = np.random.default_rng(32)
+    p = _block_params(g)
+    x = g.normal(0, 1, (7, 64))
+    s = [np.exp(g.normal(0, 1, n)) for n in (64, 64, 64, 96)]
+    y = O.decoder_block_ref(x, p, 4)
+    yf = O.decoder_block_ref(x, O.awq_fold_block(p, *s), 4)
+    assert np.max(np.abs(yf - y)) <= 1e-12 * np.max(np.abs(y))
+    # the check discriminates: the o_proj scale folded into v_proj's input
+    # columns instead of its output rows, or a place left unfolded, changes y
+    bad = O.awq_fold_block(p, *s)
+    bad["wv"] = p["wv"] * s[0][None, :] / s[1][None, :]
+    assert np.max(np.abs(O.decoder_block_ref(x, bad, 4) - y)) > 1e-3 * np.max(np.abs(y))
+    bad = O.awq_fold_block(p, *s)
+    bad["gamma2"] = p["gamma2"]
+    assert np.max(np.abs(O.decoder_block_ref(x, bad, 4) - y)) > 1e-3 * np.max(np.abs(y))
+
+
+def _fp16_half_ulp(v):
+    """Half the fp16 spacing at |v| (normal range)."""
+    e = np.floor(np.log2(np.abs(v)))
+    return 2.0 ** (np.maximum(e, -14) - 10) / 2
+
+
+def test_fold_fp16_within_half_ulp_of_exact_quotient():
+    """Stored fold results lie within fp16 rounding (plus one fp32 rounding) of
+    the exact quotient, per element and along the right axis."""
+    g = np.random.default_rng(33)
+    gam = (1.0 + 0.2 * g.standard_normal(300)).astype(np.float16)
+    s = np.exp(g.normal(0, 1.5, 300)).astype(np.float16)
+    out = O.awq_fold_into_norm(gam, s)
+    for a, b, o in zip(gam.astype(float), s.astype(float), out.astype(float)):
+        exact = Fraction(a) / Fraction(b)
+        assert abs(Fraction(o) - exact) <= Fraction(_fp16_half_ulp(float(exact))) * (1 + Fraction(1, 2 ** 12))
+    W = g.normal(0, 0.05, (5, 7)).astype(np.float16)
+    sr = np.exp(g.normal(0, 1, 5)).astype(np.float16)
+    b = g.normal(0, 0.05, 5).astype(np.float16)
+    Wf, bf = O.awq_fold_into_linear_rows(W, sr, b)
+    for n in range(5):
+        for k in range(7):
+            exact = Fraction(float(W[n, k])) / Fraction(float(sr[n]))
+            assert abs(Fraction(float(Wf[n, k])) - exact) <= \
+                Fraction(_fp16_half_ulp(float(exact))) * (1 + Fraction(1, 2 ** 12))
+        exact = Fraction(float(b[n])) / Fraction(float(sr[n]))
+        assert abs(Fraction(float(bf[n])) - exact) <= Fraction(_fp16_half_ulp(float(exact))) * (1 + Fraction(1, 2 ** 12))
+
+
+def test_fold_fp16_hand_values():
+    """Hand-derived stored values: quotients exact in fp16 stay exact, and
+    1/3 and 1/7 round to the nearest fp16 (spacing 2^-12 on [0.25, 0.5),
+    2^-13 on [0.125, 0.25)). A quotient of two fp16 values is never itself
+    an fp16 rounding midpoint (it would need 12 significant bits while the
+    dividend has 11), so only the fp32 step can create a tie."""
+    gam = np.array([1.0 + 2.0 ** -10, 1.0 + 3 * 2.0 ** -10, 3.0], dtype=np.float16)
+    s = np.array([2.0, 2.0, 2.0], dtype=np.float16)
+    out = O.awq_fold_into_norm(gam, s).astype(np.float64)
+    # (1 + 2^-10)/2 = 0.5 + 2^-11 is representable (fp16 spacing at 0.5 is 2^-11)
+    assert out[0] == 0.5 + 2.0 ** -11 and out[1] == 0.5 + 3 * 2.0 ** -11 and out[2] == 1.5
+    gam = np.array([1.0, 1.0], dtype=np.float16)
+    s = np.array([3.0, 7.0], dtype=np.float16)
+    out = O.awq_fold_into_norm(gam, s).astype(np.float64)
+    assert out[0] == 0.333251953125 and out[1] == 0.142822265625
