@@ -132,7 +132,17 @@ class ClockSampler:
         self.proc = None
         self.lines = []
 
+    def _once(self):
+        """One immediate sample (a short timed region may see no periodic one)."""
+        try:
+            r = subprocess.run(["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.QUERY}",
+                                "--format=csv,noheader,nounits"], capture_output=True, text=True, timeout=10)
+            self.lines += [ln for ln in r.stdout.splitlines() if ln.strip()]
+        except (OSError, subprocess.SubprocessError):
+            pass
+
     def __enter__(self):
+        self._once()
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
@@ -149,7 +159,8 @@ class ClockSampler:
             except subprocess.TimeoutExpired:
                 self.proc.kill()
                 out, _ = self.proc.communicate()
-            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+            self.lines += [ln for ln in out.splitlines() if ln.strip()]
+        self._once()
         return False
 
     def summary(self):
@@ -386,7 +397,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
 
     del graphs
     if rank != 0:
-        return None
+        return None, None
 
     clocks = clk.summary()
     traffic = profiled_traffic("gemv_rows_kernel")
@@ -435,11 +446,11 @@ def run_ours(args, rank: int, world: int, local_rank: int):
                 "eager_ms_per_step": e2e_eager_ms / e2e_steps},
         "gpu_launches": 7 * args.steps,
         "clocks": clocks,
-        "rows": rows,
+        "rows_line": "printed on the line before this one" if rows else "not measured (--no-rows)",
     }
     if not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(cases, args.cpu_seconds)
-    return line
+    return line, rows
 
 
 def _time_graph(torch, fn_list, reps: int = 5, inner: int = 1):
@@ -640,22 +651,72 @@ def measure_rows(wq, torch, synth, dev, block, peaks):
     return rows
 
 
+def _oracle_rows(task):
+    """Oracle GEMV of one block of output rows (unpack, fp64 dequantize, fp64
+    matmul); a process-pool task of the all-cores baseline."""
+    import oracle as O
+    try:
+        from threadpoolctl import threadpool_limits
+        lim = threadpool_limits(limits=1)
+    except ImportError:  # pragma: no cover
+        lim = None
+    X, words, st, z, K, reps = task
+    for _ in range(reps):
+        O.gemm_ref(X, O.unpack_codes(words, 4, K), st, z, 128)
+    if lim is not None:
+        lim.__exit__(None, None, None)
+    return reps
+
+
+def _oracle_sample(cases, frac: int):
+    """The first 1/frac of each linear's output rows, quantized and packed by
+    the oracle: (X, packed words, steps, zeros, rows, K) per linear."""
+    import oracle as O
+    out = []
+    for c in cases:
+        N, K = c.W.shape
+        rows = max(1, N // frac)
+        codes, st, z = O.quantize_groups(c.W[:rows], 4, 128, False)
+        out.append((c.X, O.pack_codes(codes, 4), st, z, rows, K))
+    return out
+
+
+class OraclePool:
+    """The oracle GEMV over output rows on every host core: a spawn-started
+    process pool (safe after CUDA initialisation), one row block per core and
+    linear. Every worker runs the oracle single-threaded."""
+
+    def __init__(self):
+        import multiprocessing as mp
+        self.cores = os.cpu_count() or 1
+        self.pool = mp.get_context("spawn").Pool(self.cores)
+
+    def run(self, prepared, reps: int) -> int:
+        tasks = []
+        for X, words, st, z, rows, K in prepared:
+            bounds = np.linspace(0, rows, self.cores + 1).astype(int)
+            for a, b in zip(bounds[:-1], bounds[1:]):
+                if b > a:
+                    tasks.append((X, words[a:b], st[a:b], z[a:b], K, reps))
+        self.pool.map(_oracle_rows, tasks, chunksize=1)
+        return sum(gemm_bytes(1, rows, K, 4) for _, _, _, _, rows, K in prepared) * reps
+
+    def close(self):
+        self.pool.close()
+        self.pool.join()
+
+
 def cpu_baseline(cases, seconds: float):
     """The oracle (numpy, fp64 dequantize + matmul), as it stands, on a sample of
-    each linear's output rows, repeated until about `seconds` of CPU time."""
+    each linear's output rows: single-threaded, and over output rows on every
+    host core, each for about `seconds`."""
     import oracle as O
     try:
         from threadpoolctl import threadpool_limits
     except ImportError:  # pragma: no cover
         threadpool_limits = None
-    prepared = []
     frac = 16
-    for c in cases:
-        N, K = c.W.shape
-        rows = N // frac
-        codes, st, z = O.quantize_groups(c.W[:rows], 4, 128, False)
-        words = O.pack_codes(codes, 4)
-        prepared.append((c.X, words, st, z, rows, K))
+    prepared = _oracle_sample(cases, frac)
     ctx = threadpool_limits(limits=1) if threadpool_limits else None
     t0 = time.perf_counter()
     done_bytes, reps = 0, 0
@@ -674,9 +735,21 @@ def cpu_baseline(cases, seconds: float):
         if ctx:
             ctx.__exit__(None, None, None)
     el = time.perf_counter() - t0
-    return {"value": round(done_bytes / el / 1e9, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
-            "sample": f"1/{frac} of the output rows of each of the 7 linears (unpack + fp64 dequantize + fp64 "
-                      f"matmul), {reps} passes in {el:.1f} s, one thread"}
+    one = done_bytes / el / 1e9
+    pool = OraclePool()
+    try:
+        pool.run(prepared, 1)  # workers started and warm
+        t0 = time.perf_counter()
+        by = pool.run(prepared, reps)
+        el_all = time.perf_counter() - t0
+    finally:
+        pool.close()
+    sample = f"1/{frac} of the output rows of each of the 7 linears (unpack + fp64 dequantize + fp64 matmul)"
+    return {"value": round(by / el_all / 1e9, 4), "unit": "GB/s", "cores": pool.cores, "kind": "oracle",
+            "sample": f"{sample}, {reps} passes in {el_all:.1f} s over output rows on {pool.cores} host cores "
+                      f"(spawned processes, one thread each)",
+            "single_thread": {"value": round(one, 4), "unit": "GB/s", "cores": 1,
+                              "sample": f"{sample}, {reps} passes in {el:.1f} s, one thread"}}
 
 
 # ---------------------------------------------------------------------------
@@ -684,53 +757,39 @@ def cpu_baseline(cases, seconds: float):
 # ---------------------------------------------------------------------------
 
 def run_reference(args, rank: int, world: int):
+    """The reference arm: the oracle as it stands, over output rows on every
+    host core (one single-threaded process per core), on a sample of each
+    linear's rows sized so the whole run takes about --ref-seconds."""
     if rank != 0:
         return None
     import oracle as O
     import synth
-    try:
-        from threadpoolctl import threadpool_limits
-        lim = threadpool_limits(limits=1)
-    except ImportError:  # pragma: no cover
-        lim = None
     cases = synth.config_llama7b_decode(1)
     budget = float(args.ref_seconds)
-    # calibrate rows per step so the whole run fits the budget
-    c0 = cases[0]
-    codes, st, z = O.quantize_groups(c0.W[:64], 4, 128, False)
-    words = O.pack_codes(codes, 4)
-    t0 = time.perf_counter()
-    O.gemm_ref(c0.X, O.unpack_codes(words, 4, c0.K if hasattr(c0, "K") else c0.W.shape[1]), st, z, 128)
-    per_row = (time.perf_counter() - t0) / 64
-    total_rows_per_step = sum(c.W.shape[0] for c in cases)
-    steps_total = args.steps + args.warmup
-    frac = min(1.0, budget / max(steps_total * per_row * total_rows_per_step, 1e-9))
-    prepared = []
-    for c in cases:
-        N, K = c.W.shape
-        rows = max(1, int(N * frac))
-        codes, st, z = O.quantize_groups(c.W[:rows], 4, 128, False)
-        prepared.append((c.X, O.pack_codes(codes, 4), st, z, rows, K))
-
-    def step():
-        b = 0
-        for X, words, st, z, rows, K in prepared:
-            O.gemm_ref(X, O.unpack_codes(words, 4, K), st, z, 128)
-            b += gemm_bytes(1, rows, K, 4)
-        return b
-
-    for _ in range(args.warmup):
-        step()
-    t0 = time.perf_counter()
-    by = 0
-    for _ in range(args.steps):
-        by += step()
-    el = time.perf_counter() - t0
-    if lim is not None:
-        lim.__exit__(None, None, None)
+    pool = OraclePool()
+    try:
+        # calibrate the sample so the whole run fits the budget
+        probe = _oracle_sample(cases, 64)
+        pool.run(probe, 1)
+        t0 = time.perf_counter()
+        pool.run(probe, 1)
+        per_step_1_64 = time.perf_counter() - t0
+        steps_total = args.steps + args.warmup
+        frac = max(1, int(math.ceil(64 * steps_total * per_step_1_64 / budget)))
+        frac = 1 << max(0, (frac - 1).bit_length())  # a power of two >= the estimate
+        prepared = _oracle_sample(cases, frac) if frac != 64 else probe
+        for _ in range(args.warmup):
+            pool.run(prepared, 1)
+        t0 = time.perf_counter()
+        by = 0
+        for _ in range(args.steps):
+            by += pool.run(prepared, 1)
+        el = time.perf_counter() - t0
+    finally:
+        pool.close()
     value = by / el / 1e9
-    sample = (f"{frac:.5f} of the output rows of each of the 7 linears per step "
-              f"(unpack + fp64 dequantize + fp64 matmul), one thread")
+    sample = (f"1/{frac} of the output rows of each of the 7 linears per step (unpack + fp64 dequantize + fp64 "
+              f"matmul), over output rows on {pool.cores} host cores (spawned processes, one thread each)")
     return {
         "impl": "reference",
         "metric": METRIC,
@@ -746,7 +805,8 @@ def run_reference(args, rank: int, world: int):
         "dtype": "f64",
         "data": "synthetic",
         "config": {"workload": WORKLOAD, "parallelism": "host cores (rank 0 only)"},
-        "cpu_baseline": {"value": round(value, 5), "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": sample},
+        "cpu_baseline": {"value": round(value, 5), "unit": "GB/s", "cores": pool.cores, "kind": "oracle",
+                         "sample": sample},
         "e2e": {"value": round(value, 5), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
 
@@ -809,6 +869,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=200)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-rows", action="store_true", help="skip the per-row measurements")
+    ap.add_argument("--rows-out", default=None, help="also write the per-row measurements to this JSON file")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--eager", action="store_true", help="launch eagerly instead of replaying CUDA graphs")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
@@ -849,12 +910,19 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local_rank))
     try:
-        line = run_ours(args, rank, world, local_rank)
+        line, rows = run_ours(args, rank, world, local_rank)
     finally:
         if world > 1:
             import torch.distributed as dist
             dist.destroy_process_group()
     if line is not None:
+        if rows:
+            # the other hot-path rows: their own line (and file), so that the
+            # last line stays a compact headline
+            if args.rows_out:
+                with open(args.rows_out, "w") as f:
+                    json.dump(rows, f, indent=1)
+            print(json.dumps({"rows": rows}), flush=True)
         print(json.dumps(line), flush=True)
 
 
