@@ -158,8 +158,9 @@ int32_t wq_w4a16_gemm(const void* X_dev, const uint32_t* packed_dev, const void*
  * s_j,k = fp16_rn(max(mu_k, 2^-14)^alpha_j), and for every j the loss
  * L_j = sum_i || X (W_i - Q(W_i diag s_j) diag(s_j)^-1)^T ||_F^2, where Q is
  * this library's quantize-dequantize with `cfg` (the loss GEMM runs on the
- * tensor cores with the error matrix in fp16 and fp32 accumulation; the
- * squares are summed in fp64 in a fixed order, so results are deterministic).
+ * tensor cores with fp32 accumulation; by default the error matrix enters it
+ * as two fp16 parts, E_hi + E_lo, about 22 significant bits; the squares are
+ * summed in fp64 in a fixed order, so results are deterministic).
  * Writes s_out_dev (fp16 [K]) = s_best with best = the first index of the
  * smallest L_j; optionally mu_out_dev (fp64 [K]), loss_out_dev (fp64
  * [n_alpha]) and best_out_dev (int32, device). Quantize the weights with
@@ -202,6 +203,30 @@ int32_t wq_awq_scale_search_noalloc(const void* X_dev, int64_t T, int64_t K, con
                                     const double* alpha, int32_t n_alpha, void* s_out_dev,
                                     double* mu_out_dev, double* loss_out_dev, int32_t* best_out_dev,
                                     void* stream);
+
+/* AWQ scale folding ("MIT 6.5940 Lab 4 + Lab 5", section "Question 2": the
+ * scales searched at each place are folded into the previous LayerNorm or
+ * linear layer). After wq_awq_scale_search picked s for a set of linears and
+ * they were packed with wq_quantize_pack(W, s), the op that produces their
+ * input absorbs diag(s)^-1, so the matmul takes the unscaled activations:
+ *   wq_awq_fold_norm         gamma_out[k] = gamma[k] / s[k]: the weight of a
+ *                            normalisation layer (RMSNorm / LayerNorm scale)
+ *                            feeding q/k/v or gate/up. fp16 [K] each.
+ *   wq_awq_fold_linear_rows  W_out[n][k] = W[n][k] / s[n] and b_out[n] =
+ *                            b[n] / s[n]: a linear whose output feeds the
+ *                            scaled linear (v_proj before o_proj, up_proj
+ *                            before down_proj); s has N entries (the scaled
+ *                            linear's input channels). W fp16 [N][K]; b and
+ *                            b_out fp16 [N], both NULL when there is no bias.
+ *                            Fold before that linear is itself quantized.
+ * Each result is fp16_rn(the fp32 quotient of IEEE division). Outputs may be
+ * the inputs (in place). Pointers: device, 2-byte aligned (16-byte alignment
+ * and K % 8 == 0 take the vectorized path). A result that is not finite in
+ * fp16 latches WQ_ERR_RANGE in the device flag. One launch each (two with a
+ * bias), asynchronous on `stream`. */
+int32_t wq_awq_fold_norm(const void* gamma_dev, const void* s_dev, int64_t K, void* gamma_out_dev, void* stream);
+int32_t wq_awq_fold_linear_rows(const void* W_dev, const void* b_dev, const void* s_dev, int64_t N, int64_t K,
+                                void* W_out_dev, void* b_out_dev, void* stream);
 
 /* Process-wide tuning options. Each is an atomic value, so a thread may set
  * one while another calls the library; a call reads each option it uses
@@ -269,14 +294,18 @@ int32_t wq_awq_scale_search_noalloc(const void* X_dev, int64_t T, int64_t K, con
  *                       MMA reads both operands from shared memory; tensor
  *                       memory holds only the accumulator). Same results.
  *  WQ_OPT_AWQ_LOSS     how wq_awq_scale_search forms the losses:
- *                       WQ_AWQ_LOSS_TWO_KERNELS (default) writes the error
- *                       matrix E = W - Q(W diag s) diag(s)^-1 of a batch of
- *                       alphas to the workspace and reads it back in a
- *                       tensor-core GEMM; WQ_AWQ_LOSS_FUSED builds each E tile
- *                       in shared memory inside the GEMM, in place of the
- *                       weights it came from (no E in global memory). Both
- *                       round E to fp16 the same way; the noalloc search
- *                       follows the same option (fused: no error-matrix chunks).
+ *                       WQ_AWQ_LOSS_FUSED (default) builds each tile of the
+ *                       error matrix E = W - Q(W diag s) diag(s)^-1 in shared
+ *                       memory inside the tensor-core GEMM, from the weights
+ *                       it came from (no E in global memory), as
+ *                       E_hi = fp16(E) and E_lo = fp16(E - E_hi), both
+ *                       multiplied into the same fp32 accumulator (losses to
+ *                       about 1e-7 relative);
+ *                       WQ_AWQ_LOSS_TWO_KERNELS writes E of a batch of alphas
+ *                       to the workspace in fp16 only and reads it back in a
+ *                       second kernel (losses to about 1e-4 relative; twice
+ *                       the HBM traffic). The noalloc search follows the same
+ *                       option (fused: no error-matrix chunks).
  * wq_set_option returns WQ_ERR_INVALID_ARG for an unknown option or value;
  * wq_get_option returns the current value, or -1 for an unknown option. */
 #define WQ_OPT_GEMM_PATH 1

@@ -41,6 +41,7 @@ import numpy as np
 __all__ = [
     "f16_round_up",
     "quantize_groups",
+    "quantize_groups_f32",
     "dequantize",
     "pack_codes",
     "unpack_codes",
@@ -58,6 +59,9 @@ __all__ = [
     "awq_fold_into_linear_rows",
     "decoder_block_ref",
     "awq_fold_block",
+    "gptq_hessian",
+    "gptq_quantize",
+    "GPTQ_DAMP",
     "MU_FLOOR",
 ]
 
@@ -123,6 +127,13 @@ def quantize_groups(W16: np.ndarray, bits: int, group: int, symmetric: bool,
         s16 = np.asarray(s16)
         assert s16.dtype == np.float16 and s16.shape == (K,)
         w = w * s16.astype(np.float32)[None, :]
+    return quantize_groups_f32(w, bits, group, symmetric)
+
+
+def quantize_groups_f32(w: np.ndarray, bits: int, group: int, symmetric: bool):
+    """The decisions of ``quantize_groups`` on an fp32 [N][K] array that need
+    not hold fp16 values (GPTQ quantizes weights it has already updated)."""
+    N, K = w.shape
     G = K // group
     wg = w.reshape(N, G, group)
 
@@ -474,3 +485,86 @@ def awq_fold_block(p: dict, s_qkv, s_o, s_gu, s_down) -> dict:
     out["wu"], _ = awq_fold_into_linear_rows(out["wu"], s_down)
     out["wd"] = f["wd"] * s_down[None, :]
     return out
+
+
+# ---------------------------------------------------------------------------
+# GPTQ ([CMU-L19/20] "The algorithm in four steps" and "Why it can actually
+# run: from OBS to GPTQ"), written into the same group-wise packed format
+# ---------------------------------------------------------------------------
+
+GPTQ_DAMP = 0.01
+
+
+def gptq_hessian(X16: np.ndarray, damp: float = GPTQ_DAMP):
+    """H = 2 X^T X + lambda I in fp64 for calibration inputs X [T][K] (the
+    pages' 2XX^T with X stored tokens-major), lambda = damp * mean(diag H).
+
+    Readings (the pages write "+ lambda I" without a value): lambda is 1 % of
+    the mean diagonal, and an input channel that is zero on every token has
+    H_kk := 1 (its weights are set to 0 by ``gptq_quantize``), so H stays
+    positive definite. Returns (H, dead) with dead the zero channels."""
+    X = np.asarray(X16, dtype=np.float64)
+    H = 2.0 * (X.T @ X)
+    dead = np.diag(H) == 0
+    H[dead, dead] = 1.0
+    H += damp * np.mean(np.diag(H)) * np.eye(H.shape[0])
+    return H, dead
+
+
+def gptq_quantize(W16: np.ndarray, X16: np.ndarray, bits: int, group: int, symmetric: bool,
+                  block: int = 128, damp: float = GPTQ_DAMP):
+    """GPTQ in the page's four steps, in fp64:
+
+    1. G = Cholesky((2 X X^T + lambda I)^-1)^T, the upper triangular factor
+       with H^-1 = G^T G (two library calls: inverse, Cholesky).
+    2. Within a block of ``block`` columns, quantize one column (all rows at
+       once). When a column starts a quantization group, the group's step and
+       zero point are chosen from the group's current (already updated)
+       weights with the library's round-to-nearest decisions
+       (``quantize_groups`` on the fp32 values).
+    3. The column's error, divided by G's diagonal entry.
+    4. Update the remaining columns of the block with it; when the block is
+       done, update every column to its right in one batch (lazy batch
+       update).
+
+    Returns (codes uint8 [N][K], steps fp16 [N][K/group], zeros fp16
+    [N][K/group]), the format of ``quantize_groups``."""
+    W = np.asarray(W16).astype(np.float64).copy()
+    N, K = W.shape
+    assert K % group == 0 and (block % group == 0 or group % block == 0)
+    H, dead = gptq_hessian(X16, damp)
+    W[:, dead] = 0.0
+    G = np.linalg.cholesky(np.linalg.inv(H)).T
+    codes = np.zeros((N, K), dtype=np.uint8)
+    steps = np.zeros((N, K // group), dtype=np.float16)
+    zeros = np.zeros((N, K // group), dtype=np.float16)
+    step_g = zero_g = None
+    for b0 in range(0, K, block):
+        b1 = min(b0 + block, K)
+        Err = np.zeros((N, b1 - b0))
+        for i in range(b0, b1):
+            if i % group == 0:
+                gc, gs, gz = quantize_groups_f32(W[:, i:i + group].astype(np.float32), bits, group, symmetric)
+                steps[:, i // group], zeros[:, i // group] = gs[:, 0], gz[:, 0]
+                step_g, zero_g = gs[:, 0].astype(np.float64), gz[:, 0].astype(np.float64)
+            q = _code_of(W[:, i].astype(np.float32), steps[:, i // group], zeros[:, i // group], bits, symmetric)
+            codes[:, i] = q
+            deq = (q.astype(np.float64) - zero_g) * step_g
+            err = (W[:, i] - deq) / G[i, i]
+            W[:, i + 1:b1] -= np.outer(err, G[i, i + 1:b1])
+            Err[:, i - b0] = err
+        W[:, b1:] -= Err @ G[b0:b1, b1:]
+    return codes, steps, zeros
+
+
+def _code_of(w32: np.ndarray, step_h: np.ndarray, zero_h: np.ndarray, bits: int, symmetric: bool) -> np.ndarray:
+    """Code of one fp32 value per row under its group's (step, zero): the
+    rounding and clamp of ``quantize_groups`` (fp32 division, ties to even)."""
+    sf = step_h.astype(np.float32)
+    if symmetric:
+        qmax = (1 << (bits - 1)) - 1
+        qs = np.clip(np.rint(w32 / sf), -qmax - 1, qmax).astype(np.int32)
+        return (qs + (1 << (bits - 1))).astype(np.uint8)
+    Q = (1 << bits) - 1
+    q = np.rint(w32 / sf).astype(np.int32) + zero_h.astype(np.int32)
+    return np.clip(q, 0, Q).astype(np.uint8)

@@ -81,6 +81,13 @@ def test_argument_validation_without_gpu(wq):
     assert L.wq_w4a16_gemm(good, good, good, good, 1, 8, 256, by(c), None, None, 0, None) == wq.WQ_ERR_INVALID_ARG
     assert L.wq_unpack_dequant(good, good, good, 8, 256, by(_cfg(wq, bits=6)), good, None) == wq.WQ_ERR_UNSUPPORTED
     assert wq.wq_gemm_workspace_bytes(1, 4096, 4096) == 0
+    # scale folding
+    assert L.wq_awq_fold_norm(None, good, 8, good, None) == wq.WQ_ERR_INVALID_ARG
+    assert L.wq_awq_fold_norm(good, good, 0, good, None) == wq.WQ_ERR_INVALID_ARG
+    assert L.wq_awq_fold_norm(good + 1, good, 8, good, None) == wq.WQ_ERR_ALIGNMENT
+    assert L.wq_awq_fold_linear_rows(good, good, good, 4, 8, good, None, None) == wq.WQ_ERR_INVALID_ARG
+    assert L.wq_awq_fold_linear_rows(good, None, good, 0, 8, good, None, None) == wq.WQ_ERR_INVALID_ARG
+    assert L.wq_awq_fold_linear_rows(good, None, good + 1, 4, 8, good, None, None) == wq.WQ_ERR_ALIGNMENT
 
 
 def test_option_values_are_validated(wq):

@@ -480,3 +480,109 @@ def test_fold_fp16_hand_values():
     s = np.array([3.0, 7.0], dtype=np.float16)
     out = O.awq_fold_into_norm(gam, s).astype(np.float64)
     assert out[0] == 0.333251953125 and out[1] == 0.142822265625
+
+
+# ---------------------------------------------------------------------------
+# GPTQ ("CMU 11-868 L19-L20 Model Quantization", "The algorithm in four
+# steps" and "Why it can actually run: from OBS to GPTQ")
+# ---------------------------------------------------------------------------
+
+def _obs_sequential(W16, X16, bits, group, sym, damp=0.01):
+    """Optimal Brain Surgeon in its original form: quantize the columns in
+    order; after each, move the remaining weights by the closed-form optimal
+    compensation -err / [H_F^-1]_qq * [H_F^-1]_q,: and remove the quantized
+    column from the inverse Hessian by the rank-one downdate. No Cholesky
+    factor, no blocks."""
+    W = W16.astype(np.float64).copy()
+    X = X16.astype(np.float64)
+    N, K = W.shape
+    H = 2.0 * X.T @ X
+    H += damp * np.mean(np.diag(H)) * np.eye(K)
+    Hinv = np.linalg.inv(H)
+    codes = np.zeros((N, K), np.uint8)
+    st = np.zeros((N, K // group), np.float16)
+    zr = np.zeros((N, K // group), np.float16)
+    for i in range(K):
+        if i % group == 0:
+            _, s, z = O.quantize_groups_f32(W[:, i:i + group].astype(np.float32), bits, group, sym)
+            st[:, i // group], zr[:, i // group] = s[:, 0], z[:, 0]
+        sf = st[:, i // group].astype(np.float32)
+        if sym:
+            qmax = (1 << (bits - 1)) - 1
+            q = np.clip(np.rint(W[:, i].astype(np.float32) / sf), -qmax - 1, qmax).astype(np.int32) + (1 << (bits - 1))
+        else:
+            q = np.clip(np.rint(W[:, i].astype(np.float32) / sf).astype(np.int32) + zr[:, i // group].astype(np.int32),
+                        0, (1 << bits) - 1)
+        codes[:, i] = q
+        deq = (q - zr[:, i // group].astype(np.float64)) * st[:, i // group].astype(np.float64)
+        d = Hinv[i, i]
+        W[:, i + 1:] -= np.outer((W[:, i] - deq) / d, Hinv[i, i + 1:])
+        Hinv = Hinv - np.outer(Hinv[:, i], Hinv[i, :]) / d
+    return codes, st, zr
+
+
+@pytest.mark.parametrize("block", [1, 4, 32, 64])
+@pytest.mark.parametrize("sym", [False, True])
+def test_gptq_equals_obs_sequential(block, sym):
+    """The Cholesky reformulation and the lazy batch updates change the order
+    of computation, not the result: codes, steps and zeros equal the
+    sequential OBS procedure on small problems (4-bit, groups of 32)."""
+    g = np.random.default_rng(61 + block)
+    N, K, T = 12, 64, 40
+    W = (0.02 * g.standard_normal((N, K))).astype(np.float16)
+    base = g.standard_normal((T, 8))
+    X = (base @ g.standard_normal((8, K)) + 0.3 * g.standard_normal((T, K))).astype(np.float16)  # correlated
+    ref = _obs_sequential(W, X, 4, 32, sym)
+    got = O.gptq_quantize(W, X, 4, 32, sym, block=block)
+    for a, b in zip(got, ref):
+        assert np.array_equal(a.view(np.uint8) if a.dtype == np.uint8 else a.view(np.uint16),
+                              b.view(np.uint8) if b.dtype == np.uint8 else b.view(np.uint16))
+
+
+def test_gptq_with_uncorrelated_inputs_is_rtn():
+    """With orthogonal input channels H is diagonal, so is G: no error is
+    passed on and GPTQ gives exactly the round-to-nearest codes."""
+    g = np.random.default_rng(62)
+    K, N = 128, 16
+    X = np.zeros((K, K), np.float16)
+    X[np.arange(K), np.arange(K)] = (1.0 + g.random(K)).astype(np.float16)  # exactly orthogonal
+    W = (0.02 * g.standard_normal((N, K))).astype(np.float16)
+    for bits, sym in ((4, False), (3, True)):
+        got = O.gptq_quantize(W, X, bits, 128, sym)
+        ref = O.quantize_groups(W, bits, 128, sym)
+        assert np.array_equal(got[0], ref[0])
+        assert np.array_equal(got[1].view(np.uint16), ref[1].view(np.uint16))
+
+
+def test_gptq_hessian_damping_and_dead_channels():
+    """H = 2 X^T X + lambda I, lambda = 1 % of the mean diagonal; a channel
+    that is zero on every token gets H_kk = 1 before the damping and its
+    weights quantize as zeros."""
+    X = np.array([[1.0, 0.0, 2.0], [3.0, 0.0, -1.0]], np.float16)
+    H, dead = O.gptq_hessian(X)
+    base = np.array([[20.0, 0.0, -2.0], [0.0, 1.0, 0.0], [-2.0, 0.0, 10.0]])
+    lam = 0.01 * (20.0 + 1.0 + 10.0) / 3
+    assert np.array_equal(dead, [False, True, False])
+    assert np.allclose(H, base + lam * np.eye(3), rtol=0, atol=1e-15)
+    g = np.random.default_rng(63)
+    Xc = (g.standard_normal((20, 128))).astype(np.float16)
+    Xc[:, 7] = 0
+    W = (0.02 * g.standard_normal((4, 128))).astype(np.float16)
+    codes, st, z = O.gptq_quantize(W, Xc, 4, 128, False)
+    assert np.all(O.dequantize(codes, st, z, 128)[:, 7] == 0.0)
+
+
+def test_gptq_beats_rtn_on_correlated_inputs():
+    """The layer-wise objective ||W X - W^ X||^2 ("CMU 11-868 L19-L20",
+    "Two core moves") is lower after GPTQ than after round to nearest."""
+    g = np.random.default_rng(64)
+    N, K, T = 64, 256, 128
+    W = (0.02 * g.standard_normal((N, K))).astype(np.float16)
+    X = (g.standard_normal((T, 16)) @ g.standard_normal((16, K)) + 0.2 * g.standard_normal((T, K))).astype(np.float16)
+
+    def loss(c, s, z):
+        E = W.astype(np.float64) - O.dequantize(c, s, z, 128)
+        return float(np.sum((X.astype(np.float64) @ E.T) ** 2))
+
+    for bits in (3, 4):
+        assert loss(*O.gptq_quantize(W, X, bits, 128, False)) < 0.8 * loss(*O.quantize_groups(W, bits, 128, False))

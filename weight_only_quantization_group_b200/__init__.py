@@ -35,6 +35,8 @@ __all__ = [
     "wq_awq_workspace_bytes",
     "wq_awq_scale_search",
     "wq_awq_scale_search_noalloc",
+    "wq_awq_fold_norm",
+    "wq_awq_fold_linear_rows",
     "EXPORTED_SYMBOLS",
 ]
 
@@ -57,6 +59,8 @@ EXPORTED_SYMBOLS = (
     "wq_awq_workspace_bytes",
     "wq_awq_scale_search",
     "wq_awq_scale_search_noalloc",
+    "wq_awq_fold_norm",
+    "wq_awq_fold_linear_rows",
 )
 
 WQ_OK = 0
@@ -131,6 +135,8 @@ def _load() -> ctypes.CDLL:
                                       ctypes.POINTER(ctypes.c_double), i32, vp, vp, vp, vp, vp, sz, vp]),
         "wq_awq_scale_search_noalloc": (i32, [vp, i64, i64, ctypes.POINTER(vp), ctypes.POINTER(i64), i32, cfgp,
                                               ctypes.POINTER(ctypes.c_double), i32, vp, vp, vp, vp, vp]),
+        "wq_awq_fold_norm": (i32, [vp, vp, i64, vp, vp]),
+        "wq_awq_fold_linear_rows": (i32, [vp, vp, vp, i64, i64, vp, vp, vp]),
     }
     for name, (res, args) in sig.items():
         f = getattr(L, name)
@@ -492,3 +498,47 @@ def wq_awq_scale_search_noalloc(X: torch.Tensor, Ws, alphas=None, *, bits: int =
                                               _ptr(out["best"]), _stream(stream, X.device.index))
     _raise(st, "wq_awq_scale_search_noalloc")
     return out
+
+
+def wq_awq_fold_norm(gamma: torch.Tensor, s: torch.Tensor, *, out: torch.Tensor | None = None, stream=None):
+    """gamma / s (fp16 [K] each): a normalisation weight absorbing the AWQ
+    scales of the linears it feeds. out may be gamma (in place)."""
+    _check(gamma, torch.float16, "gamma")
+    K = gamma.numel()
+    _need(s, "s", torch.float16, 2 * K)
+    if out is None:
+        out = torch.empty_like(gamma)
+    _need(out, "out", torch.float16, 2 * K)
+    _on_device_of(gamma, s=s, out=out)
+    with _device_of(gamma):
+        st = _lib.wq_awq_fold_norm(_ptr(gamma), _ptr(s), K, _ptr(out), _stream(stream, gamma.device.index))
+    _raise(st, "wq_awq_fold_norm")
+    return out
+
+
+def wq_awq_fold_linear_rows(W: torch.Tensor, s: torch.Tensor, b: torch.Tensor | None = None, *, out=None,
+                            stream=None):
+    """W[n][k] / s[n] (and b[n] / s[n]): the linear before a scaled linear
+    absorbs its AWQ scales in its output rows. Returns (W', b') (b' None
+    without a bias); `out` = (W_out, b_out) may be the inputs (in place)."""
+    _check(W, torch.float16, "W")
+    if W.dim() != 2:
+        raise ValueError(f"W must be [N][K], got shape {tuple(W.shape)}")
+    N, K = W.shape
+    _need(s, "s", torch.float16, 2 * N)
+    if b is not None:
+        _need(b, "b", torch.float16, 2 * N)
+    if out is None:
+        out = (torch.empty_like(W), None if b is None else torch.empty_like(b))
+    W_out, b_out = out
+    _need(W_out, "out[0]", torch.float16, 2 * N * K)
+    if (b is None) != (b_out is None):
+        raise ValueError("b and out[1] must both be given or both be None")
+    if b_out is not None:
+        _need(b_out, "out[1]", torch.float16, 2 * N)
+    _on_device_of(W, s=s, b=b, W_out=W_out, b_out=b_out)
+    with _device_of(W):
+        st = _lib.wq_awq_fold_linear_rows(_ptr(W), _ptr(b), _ptr(s), N, K, _ptr(W_out), _ptr(b_out),
+                                          _stream(stream, W.device.index))
+    _raise(st, "wq_awq_fold_linear_rows")
+    return W_out, b_out

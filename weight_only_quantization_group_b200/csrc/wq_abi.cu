@@ -72,7 +72,7 @@ std::atomic<int64_t> g_opt_tc_bk{0};
 std::atomic<int64_t> g_opt_tc_dequant_warps{0};
 std::atomic<int64_t> g_opt_wait_limit_ms{2000};
 std::atomic<int64_t> g_opt_test_stall{0};
-std::atomic<int64_t> g_opt_awq_loss{WQ_AWQ_LOSS_TWO_KERNELS};
+std::atomic<int64_t> g_opt_awq_loss{WQ_AWQ_LOSS_FUSED};
 std::atomic<int64_t> g_opt_tc_a_source{WQ_TC_A_TMEM};
 
 }  // namespace
@@ -251,6 +251,31 @@ int32_t wq_awq_scale_search_noalloc(const void* X, int64_t T, int64_t K, const v
   return cuda_status(wq::launch_awq_search_noalloc(X, T, K, W, N_i, n_lin, cfg->bits, cfg->symmetric != 0, alpha,
                                                    n_alpha, s_out, mu_out, loss_out, best_out, flag, fused,
                                                    static_cast<cudaStream_t>(stream)));
+}
+
+int32_t wq_awq_fold_norm(const void* gamma, const void* s, int64_t K, void* gamma_out, void* stream) {
+  NvtxRange nvtx_range("wq_awq_fold_norm");
+  if (!gamma || !s || !gamma_out) return WQ_ERR_INVALID_ARG;
+  if (K < 1 || K > (int64_t)INT32_MAX) return WQ_ERR_INVALID_ARG;
+  if (!aligned(gamma, 2) || !aligned(s, 2) || !aligned(gamma_out, 2)) return WQ_ERR_ALIGNMENT;
+  int* flag = device_flag();
+  if (!flag) return WQ_ERR_CUDA;
+  return cuda_status(wq::launch_fold(gamma, s, gamma_out, 1, K, false, flag, static_cast<cudaStream_t>(stream)));
+}
+
+int32_t wq_awq_fold_linear_rows(const void* W, const void* b, const void* s, int64_t N, int64_t K, void* W_out,
+                                void* b_out, void* stream) {
+  NvtxRange nvtx_range("wq_awq_fold_linear_rows");
+  if (!W || !s || !W_out || (b == nullptr) != (b_out == nullptr)) return WQ_ERR_INVALID_ARG;
+  if (N < 1 || K < 1 || N > (int64_t)INT32_MAX || K > (int64_t)INT32_MAX) return WQ_ERR_INVALID_ARG;
+  if (!aligned(W, 2) || !aligned(s, 2) || !aligned(W_out, 2) || (b && (!aligned(b, 2) || !aligned(b_out, 2))))
+    return WQ_ERR_ALIGNMENT;
+  int* flag = device_flag();
+  if (!flag) return WQ_ERR_CUDA;
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e = wq::launch_fold(W, s, W_out, N, K, true, flag, st);
+  if (e == cudaSuccess && b) e = wq::launch_fold(b, s, b_out, 1, N, false, flag, st);
+  return cuda_status(e);
 }
 
 int32_t wq_set_option(int32_t option, int64_t value) {

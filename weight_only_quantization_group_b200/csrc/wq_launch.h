@@ -42,4 +42,7 @@ cudaError_t launch_awq_search_noalloc(const void* X, int64_t T, int64_t K, const
                                       const int64_t* N_i, int n_lin, int bits, bool sym, const double* alpha,
                                       int n_alpha, void* s_out, double* mu_out, double* loss_out, int32_t* best_out,
                                       int* err, bool fused, cudaStream_t st);
+// AWQ scale folding (wq_fold.cu): out = in / s along rows (s[R]) or columns (s[C]).
+cudaError_t launch_fold(const void* in, const void* s, void* out, int64_t R, int64_t C, bool row_axis, int* err,
+                        cudaStream_t st);
 }  // namespace wq
