@@ -572,23 +572,6 @@ def measure_rows(wq, torch, synth, dev, block, peaks):
                 wq.wq_set_option(wq.WQ_OPT_TC_STAGES, 0)
                 wq.wq_set_option(wq.WQ_OPT_TC_BK, 0)
                 wq.wq_set_option(wq.WQ_OPT_TC_DEQUANT_WARPS, 0)
-    # tensor-core kernel with the dequantized weight tile in shared memory
-    # (64-channel stages keep two CTAs per SM at M = 64, where a 128-channel A
-    # ring leaves room for one)
-    for M in (4, 16, 64, 128):
-        for S, bk in ((0, 0), (5, 0), (0, 64)):
-            wq.wq_set_option(wq.WQ_OPT_TC_A_SOURCE, wq.WQ_TC_A_SMEM)
-            wq.wq_set_option(wq.WQ_OPT_TC_STAGES, S)
-            wq.wq_set_option(wq.WQ_OPT_TC_BK, bk)
-            name = f"smallm_M{M}_8192x28672_w4_tc_smem_a_bk{bk}_s{S}"
-            try:
-                gemv_row(name, 28672, 8192, 4, big.W, synth.smallm_activations(M), M=M)
-            except wq.WQError as e:
-                rows[name] = {"error": str(e)}
-            finally:
-                wq.wq_set_option(wq.WQ_OPT_TC_STAGES, 0)
-                wq.wq_set_option(wq.WQ_OPT_TC_BK, 0)
-                wq.wq_set_option(wq.WQ_OPT_TC_A_SOURCE, wq.WQ_TC_A_TMEM)
     # the other kernel on each side of the crossover, for the record
     for M in (2, 3, 4, 8, 16):
         path = wq.WQ_PATH_TENSOR_CORE if M < 3 else wq.WQ_PATH_GEMV
@@ -598,25 +581,69 @@ def measure_rows(wq, torch, synth, dev, block, peaks):
             gemv_row(f"smallm_M{M}_8192x28672_w4_{tag}", 28672, 8192, 4, big.W, synth.smallm_activations(M), M=M)
         finally:
             wq.wq_set_option(wq.WQ_OPT_GEMM_PATH, wq.WQ_PATH_AUTO)
+    # small-M sweeps on the LLaMA-65B-shaped 8192 x 8192 weight, 4- and 3-bit
+    # (64 row tiles: M >= 3 splits K over clusters of CTAs)
+    for bits in (4, 3):
+        cb = synth.config_llama65b_decode(bits)
+        for M in synth.SMALLM_SWEEP:
+            gemv_row(f"smallm{bits}_M{M}_8192x8192_w{bits}", 8192, 8192, bits, cb.W, synth.smallm_activations(M), M=M)
+    # the K split forced, M = 16, 8192 x 8192 4-bit
+    c4 = synth.config_llama65b_decode(4)
+    for ks in (1, 2, 4, 8):
+        wq.wq_set_option(wq.WQ_OPT_TC_KSPLIT, ks)
+        try:
+            gemv_row(f"smallm4_M16_8192x8192_w4_ksplit{ks}", 8192, 8192, 4, c4.W, synth.smallm_activations(16), M=16)
+        except wq.WQError as e:
+            rows[f"smallm4_M16_8192x8192_w4_ksplit{ks}"] = {"error": str(e)}
+        finally:
+            wq.wq_set_option(wq.WQ_OPT_TC_KSPLIT, 0)
+    # groups of 32 and 64 channels (8192 x 28672, 4-bit): decode GEMV and M = 16
+    for group in (32, 64):
+        for M in (1, 16):
+            name = f"group{group}_M{M}_8192x28672_w4"
+            W16 = big.W
+            packed, steps, zeros = wq.wq_quantize_pack(dt(W16), bits=4, group_size=group)
+            nc = max(2, math.ceil(4 * L2_BYTES / (28672 * 8192 // 2)))
+            qs = [(packed, steps, zeros)] + [tuple(t.clone() for t in (packed, steps, zeros)) for _ in range(nc - 1)]
+            X = dt(synth.smallm_activations(M))
+            Y = torch.empty((M, 28672), dtype=torch.float16, device=dev)
+            fns = [lambda q=q: wq.wq_w4a16_gemm(X, *q, 28672, bits=4, group_size=group, out=Y) for q in qs]
+            ms = _time_graph(torch, fns) / nc
+            by = 28672 * 8192 // 2 + 28672 * (8192 // group) * 4 + M * 8192 * 2 + M * 28672 * 2
+            rows[name] = {"M": M, "group": group, "us": ms * 1e3, "GB/s": by / (ms * 1e-3) / 1e9,
+                          "frac_hbm": by / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"]}
+            del qs
     # S1/S2/S4 AWQ scale search over one LLaMA-2-7B block (4 search places,
     # T=512 calibration rows, 20 alphas), then packing with the chosen scales
     groups = synth.config_awq_block(5)
-    prepared = []
-    for gname, X, named in groups:
-        Xd = dt(X)
-        Wd = [dt(W) for _, W in named]
-        need = wq.wq_awq_workspace_bytes(X.shape[0], X.shape[1], [W.shape[0] for W in Wd], 20)
-        ws = torch.empty(need, dtype=torch.uint8, device=dev)
-        prepared.append((gname, Xd, Wd, ws))
-    outs = [wq.wq_awq_scale_search(Xd, Wd, workspace=ws) for _, Xd, Wd, ws in prepared]  # warm-up
-    torch.cuda.synchronize()
+    flops = sum(2.0 * X.shape[0] * sum(W.shape[0] for _, W in named) * X.shape[1] * 20 for _, X, named in groups)
+
+    def awq_block(bits, loss_path):
+        old = wq.wq_get_option(wq.WQ_OPT_AWQ_LOSS)
+        wq.wq_set_option(wq.WQ_OPT_AWQ_LOSS, loss_path)
+        try:
+            prepared = []
+            for gname, X, named in groups:
+                Xd = dt(X)
+                Wd = [dt(W) for _, W in named]
+                need = wq.wq_awq_workspace_bytes(X.shape[0], X.shape[1], [W.shape[0] for W in Wd], 20, bits=bits)
+                prepared.append((gname, Xd, Wd, torch.empty(need, dtype=torch.uint8, device=dev)))
+            outs = [wq.wq_awq_scale_search(Xd, Wd, bits=bits, workspace=ws) for _, Xd, Wd, ws in prepared]
+            torch.cuda.synchronize()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            outs = [wq.wq_awq_scale_search(Xd, Wd, bits=bits, workspace=ws) for _, Xd, Wd, ws in prepared]
+            b.record()
+            torch.cuda.synchronize()
+            ms = a.elapsed_time(b)
+            assert wq.wq_get_last_device_error() == 0
+            return prepared, outs, ms
+        finally:
+            wq.wq_set_option(wq.WQ_OPT_AWQ_LOSS, old)
+
+    # default: the error tiles built inside the loss GEMM (no E in HBM)
+    prepared, outs, ms = awq_block(4, wq.WQ_AWQ_LOSS_FUSED)
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    a.record()
-    outs = [wq.wq_awq_scale_search(Xd, Wd, workspace=ws) for _, Xd, Wd, ws in prepared]
-    b.record()
-    torch.cuda.synchronize()
-    ms = a.elapsed_time(b)
-    flops = sum(2.0 * Xd.shape[0] * sum(W.shape[0] for W in Wd) * Xd.shape[1] * 20 for _, Xd, Wd, _ in prepared)
     a.record()
     for (_, Xd, Wd, _), o in zip(prepared, outs):
         for W in Wd:
@@ -629,25 +656,54 @@ def measure_rows(wq, torch, synth, dev, block, peaks):
         "frac_bf16_peak": flops / (ms * 1e-3) / 1e12 / peaks["bf16_tflops"],
         "best_alpha": {g: int(o["best"].item()) / 20 for (g, _, _, _), o in zip(prepared, outs)},
         "pack_with_s_ms": a.elapsed_time(b)}
-    # the same search with the error matrix built inside the loss GEMM
-    old = wq.wq_get_option(wq.WQ_OPT_AWQ_LOSS)
-    wq.wq_set_option(wq.WQ_OPT_AWQ_LOSS, wq.WQ_AWQ_LOSS_FUSED)
-    try:
-        fused = [wq.wq_awq_scale_search(Xd, Wd, workspace=ws) for _, Xd, Wd, ws in prepared]  # warm-up
-        torch.cuda.synchronize()
-        a.record()
-        fused = [wq.wq_awq_scale_search(Xd, Wd, workspace=ws) for _, Xd, Wd, ws in prepared]
-        b.record()
-        torch.cuda.synchronize()
-    finally:
-        wq.wq_set_option(wq.WQ_OPT_AWQ_LOSS, old)
+    # the option: E written to global memory in fp16 and read back by a second kernel
+    _, outs2, ms2 = awq_block(4, wq.WQ_AWQ_LOSS_TWO_KERNELS)
+    rows["awq_search_llama7b_block_two_kernels"] = {
+        "ms": ms2, "loss_gemm_TFLOP/s": flops / (ms2 * 1e-3) / 1e12,
+        "same_alpha_as_default": all(int(f["best"].item()) == int(o["best"].item()) for f, o in zip(outs2, outs))}
+    del prepared, outs, outs2
+
+    # the 3-bit group-128 pipeline at block scale: AWQ search, pack with s,
+    # then one decode step (7 GEMVs, X diag(s)^-1 prepared once)
+    prepared, outs, ms3 = awq_block(3, wq.WQ_AWQ_LOSS_FUSED)
+    packs = []
+    a.record()
+    for (_, Xd, Wd, _), o in zip(prepared, outs):
+        for W in Wd:
+            packs.append((W.shape[0], W.shape[1], o["s"], wq.wq_quantize_pack(W, o["s"], bits=3)))
+    b.record()
+    torch.cuda.synchronize()
+    pack3_ms = a.elapsed_time(b)
+    xs = [torch.randn((1, K), device=dev).half() / s for N, K, s, _ in packs]
+    ys = [torch.empty((1, N), dtype=torch.float16, device=dev) for N, _, _, _ in packs]
+    fns = [lambda i=i: wq.wq_w4a16_gemm(xs[i], *packs[i][3], packs[i][0], bits=3, out=ys[i]) for i in range(len(packs))]
+    step3 = _time_graph(torch, fns)
+    by3 = sum(gemm_bytes(1, N, K, 3) for N, K, _, _ in packs)
     assert wq.wq_get_last_device_error() == 0
-    fms = a.elapsed_time(b)
-    rows["awq_search_llama7b_block_fused_loss"] = {
-        "ms": fms, "loss_gemm_TFLOP/s": flops / (fms * 1e-3) / 1e12,
-        "frac_bf16_peak": flops / (fms * 1e-3) / 1e12 / peaks["bf16_tflops"],
-        "same_alpha_as_two_kernels": all(int(f["best"].item()) == int(o["best"].item())
-                                         for f, o in zip(fused, outs))}
+    rows["awq_pipeline_llama7b_block_w3"] = {
+        "search_ms": ms3, "pack_with_s_ms": pack3_ms, "decode_step_us": step3 * 1e3,
+        "decode_step_GB/s": by3 / (step3 * 1e-3) / 1e9,
+        "note": "decode step: the block's 7 linears once (weights L2-resident after packing, not rotated)",
+        "best_alpha": {g: int(o["best"].item()) / 20 for (g, _, _, _), o in zip(prepared, outs)}}
+    del prepared, outs, packs
+
+    # AWQ scale folding over the block: s_qkv into the first norm's weight,
+    # s_o into v_proj's rows, s_gate_up into the second norm's weight,
+    # s_down into up_proj's rows (fp16 in, fp16 out: 4 bytes per element)
+    g0 = synth.rng(77)
+    gam = dt((1.0 + 0.1 * g0.standard_normal(4096)).astype(np.float16))
+    sv = dt(np.exp(0.3 * g0.standard_normal(11008)).astype(np.float16))
+    Wv, Wu = block[2]["W"], block[5]["W"]
+    outv, outu, outg = torch.empty_like(Wv), torch.empty_like(Wu), torch.empty_like(gam)
+    fns = [lambda: wq.wq_awq_fold_norm(gam, sv[:4096], out=outg),
+           lambda: wq.wq_awq_fold_linear_rows(Wv, sv[:4096], out=(outv, None)),
+           lambda: wq.wq_awq_fold_norm(gam, sv[:4096], out=outg),
+           lambda: wq.wq_awq_fold_linear_rows(Wu, sv, out=(outu, None))]
+    fms = _time_graph(torch, fns)
+    fby = 4 * (2 * 4096 + Wv.numel() + Wu.numel())
+    assert wq.wq_get_last_device_error() == 0
+    rows["awq_fold_llama7b_block"] = {"us": fms * 1e3, "GB/s": fby / (fms * 1e-3) / 1e9,
+                                      "frac_hbm": fby / (fms * 1e-3) / 1e9 / peaks["hbm_gbs"]}
     return rows
 
 

@@ -138,7 +138,7 @@ size_t wq_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, const wq_quant_c
  * dequantized on the fly inside the matmul; "TinyChat (AWQ on-device
  * runtime)", "Notable features": fused dequant + GEMM). Small M runs a
  * bandwidth-bound GEMV kernel that streams the packed weights once; larger M
- * (4-bit) runs a tcgen05 tensor-core kernel. workspace_dev may be NULL when
+ * (3- and 4-bit) runs a tcgen05 tensor-core kernel. workspace_dev may be NULL when
  * wq_gemm_workspace_bytes() is 0. X must already be multiplied by
  * diag(s)^-1 when the weight was packed with AWQ scales s. */
 int32_t wq_w4a16_gemm(const void* X_dev, const uint32_t* packed_dev, const void* steps_dev,
@@ -158,9 +158,10 @@ int32_t wq_w4a16_gemm(const void* X_dev, const uint32_t* packed_dev, const void*
  * s_j,k = fp16_rn(max(mu_k, 2^-14)^alpha_j), and for every j the loss
  * L_j = sum_i || X (W_i - Q(W_i diag s_j) diag(s_j)^-1)^T ||_F^2, where Q is
  * this library's quantize-dequantize with `cfg` (the loss GEMM runs on the
- * tensor cores with fp32 accumulation; by default the error matrix enters it
- * as two fp16 parts, E_hi + E_lo, about 22 significant bits; the squares are
- * summed in fp64 in a fixed order, so results are deterministic).
+ * tensor cores with the error matrix in fp16 and fp32 accumulation; the
+ * squares are summed in fp64 in a fixed order, so results are deterministic.
+ * Against fp64 the losses come out low by about 2e-9 * K relative -- the
+ * accumulator rounds toward zero -- nearly the same for every alpha).
  * Writes s_out_dev (fp16 [K]) = s_best with best = the first index of the
  * smallest L_j; optionally mu_out_dev (fp64 [K]), loss_out_dev (fp64
  * [n_alpha]) and best_out_dev (int32, device). Quantize the weights with
@@ -204,6 +205,30 @@ int32_t wq_awq_scale_search_noalloc(const void* X_dev, int64_t T, int64_t K, con
                                     double* mu_out_dev, double* loss_out_dev, int32_t* best_out_dev,
                                     void* stream);
 
+/* GPTQ -- quantize + pack with error feedback ("CMU 11-868 L19-L20 Model
+ * Quantization", sections "The algorithm in four steps" and "Why it can
+ * actually run: from OBS to GPTQ"), writing the same packed layout, steps
+ * and zeros as wq_quantize_pack, so the matmul takes the result as it is.
+ *   X_dev  fp16 [T][K] calibration inputs of the linear
+ *   W_dev  fp16 [N][K] weight
+ * Computes, in fp64 on the device: H = 2 X^T X + lambda I with lambda =
+ * damp * mean(diag H) (damp >= 0, e.g. 0.01; an input channel that is zero
+ * on every token gets H_kk = 1 and zero weights), G = Cholesky(H^-1)^T (upper,
+ * H^-1 = G^T G), then the columns in order in blocks of 128: when a column
+ * starts a group its step and zero point come from the group's current
+ * weights by the quantizer's decisions above (on their fp32 values); the
+ * column's codes; its error divided by G_kk, subtracted from the rest of the
+ * block times G's row; after each block, every later column is updated by
+ * the block's errors times G (one batched product).
+ * workspace_dev: >= wq_gptq_workspace_bytes(N, K, cfg) bytes (two K x K fp64
+ * matrices, the N x K fp64 running weights), 256-byte aligned, no initial
+ * contents required. H not positive definite (only possible for damp == 0)
+ * latches WQ_ERR_RANGE. Many small launches on `stream` (about 5 K / 64). */
+size_t wq_gptq_workspace_bytes(int64_t N, int64_t K, const wq_quant_cfg* cfg);
+int32_t wq_gptq_quantize_pack(const void* X_dev, int64_t T, const void* W_dev, int64_t N, int64_t K,
+                              const wq_quant_cfg* cfg, double damp, uint32_t* packed_dev, void* steps_dev,
+                              void* zeros_dev, void* workspace_dev, size_t workspace_bytes, void* stream);
+
 /* AWQ scale folding ("MIT 6.5940 Lab 4 + Lab 5", section "Question 2": the
  * scales searched at each place are folded into the previous LayerNorm or
  * linear layer). After wq_awq_scale_search picked s for a set of linears and
@@ -232,9 +257,8 @@ int32_t wq_awq_fold_linear_rows(const void* W_dev, const void* b_dev, const void
  * one while another calls the library; a call reads each option it uses
  * once, so it runs wholly under the old or wholly under the new value.
  *  WQ_OPT_GEMM_PATH     WQ_PATH_AUTO (default): GEMV kernel below the
- *                       crossover M, tensor-core kernel at or above it (4-bit);
- *                       WQ_PATH_GEMV / WQ_PATH_TENSOR_CORE force one kernel
- *                       (the tensor-core kernel is 4-bit only).
+ *                       crossover M, tensor-core kernel at or above it;
+ *                       WQ_PATH_GEMV / WQ_PATH_TENSOR_CORE force one kernel.
  *  WQ_OPT_CROSSOVER_M   smallest M sent to the tensor-core kernel (default 3).
  *  WQ_OPT_GEMV_VARIANT  how the GEMV kernel forms sum_k x_k (q_k - zero):
  *                       WQ_GEMV_OFFSET_SUMS (default) multiplies x by the
@@ -280,6 +304,15 @@ int32_t wq_awq_fold_linear_rows(const void* W_dev, const void* b_dev, const void
  *                       else 128), 64 or 128.
  *  WQ_OPT_TC_DEQUANT_WARPS  warps that dequantize in the tensor-core kernel:
  *                       0 default (4), 4 or 8.
+ *  WQ_OPT_TC_KSPLIT     CTAs of a thread-block cluster that share one 128-row
+ *                       tile of the tensor-core kernel along K (their fp32
+ *                       partial tiles are added in rank order in the first
+ *                       CTA's shared memory): 0 default (library choice: the
+ *                       largest of 1, 2, 4, 8 with all CTAs resident at once
+ *                       and at least 4 stages each), 1, 2, 4 or 8 (the call
+ *                       fails with WQ_ERR_CUDA when the first CTA's ring
+ *                       cannot hold the other partial tiles or K has fewer
+ *                       stages than CTAs).
  *  WQ_OPT_WAIT_LIMIT_MS how long a bounded mbarrier wait in the tensor-core
  *                       kernel may last before it latches WQ_ERR_TIMEOUT
  *                       (1..60000, default 2000).
@@ -288,23 +321,15 @@ int32_t wq_awq_fold_linear_rows(const void* W_dev, const void* b_dev, const void
  *                       out; the kernel then frees its tensor memory, returns,
  *                       and wq_get_last_device_error reports WQ_ERR_TIMEOUT.
  *                       Y is not written. For failure-handling tests only.
- *  WQ_OPT_TC_A_SOURCE  where the tensor-core kernel's dequantized weight tile
- *                       lives: WQ_TC_A_TMEM (default) in tensor memory (written
- *                       with tcgen05.st), WQ_TC_A_SMEM in shared memory (the
- *                       MMA reads both operands from shared memory; tensor
- *                       memory holds only the accumulator). Same results.
  *  WQ_OPT_AWQ_LOSS     how wq_awq_scale_search forms the losses:
  *                       WQ_AWQ_LOSS_FUSED (default) builds each tile of the
  *                       error matrix E = W - Q(W diag s) diag(s)^-1 in shared
  *                       memory inside the tensor-core GEMM, from the weights
- *                       it came from (no E in global memory), as
- *                       E_hi = fp16(E) and E_lo = fp16(E - E_hi), both
- *                       multiplied into the same fp32 accumulator (losses to
- *                       about 1e-7 relative);
+ *                       it came from (no E in global memory);
  *                       WQ_AWQ_LOSS_TWO_KERNELS writes E of a batch of alphas
- *                       to the workspace in fp16 only and reads it back in a
- *                       second kernel (losses to about 1e-4 relative; twice
- *                       the HBM traffic). The noalloc search follows the same
+ *                       to the workspace and reads it back in a second
+ *                       kernel (twice the HBM traffic of W per alpha). Both
+ *                       round E to fp16; the noalloc search follows the same
  *                       option (fused: no error-matrix chunks).
  * wq_set_option returns WQ_ERR_INVALID_ARG for an unknown option or value;
  * wq_get_option returns the current value, or -1 for an unknown option. */
@@ -329,13 +354,10 @@ int32_t wq_awq_fold_linear_rows(const void* W_dev, const void* b_dev, const void
 #define WQ_OPT_WAIT_LIMIT_MS 13
 #define WQ_OPT_TEST_STALL 14
 #define WQ_OPT_AWQ_LOSS 15
+#define WQ_OPT_TC_KSPLIT 16
 
 #define WQ_AWQ_LOSS_TWO_KERNELS 0
 #define WQ_AWQ_LOSS_FUSED 1
-#define WQ_OPT_TC_A_SOURCE 16
-
-#define WQ_TC_A_TMEM 0
-#define WQ_TC_A_SMEM 1
 
 int32_t wq_set_option(int32_t option, int64_t value);
 int64_t wq_get_option(int32_t option);

@@ -65,7 +65,9 @@ def test_argument_validation_without_gpu(wq):
     # unsupported / invalid configs
     assert L.wq_quantize_pack(good, None, 8, 256, by(_cfg(wq, bits=5)), good, good, good, None) == wq.WQ_ERR_UNSUPPORTED
     assert L.wq_quantize_pack(good, None, 8, 256, by(_cfg(wq, bits=1)), good, good, good, None) == wq.WQ_ERR_INVALID_ARG
-    assert L.wq_quantize_pack(good, None, 8, 256, by(_cfg(wq, group=64)), good, good, good, None) == wq.WQ_ERR_UNSUPPORTED
+    assert L.wq_quantize_pack(good, None, 8, 256, by(_cfg(wq, group=48)), good, good, good, None) == wq.WQ_ERR_INVALID_ARG
+    n_i = (ctypes.c_int64 * 1)(16)
+    assert L.wq_awq_workspace_bytes(8, 256, n_i, 1, 20, by(_cfg(wq, group=64))) == 0  # AWQ: groups of 128 only
     assert L.wq_quantize_pack(good, None, 8, 256, by(_cfg(wq, sym=2)), good, good, good, None) == wq.WQ_ERR_INVALID_ARG
     assert L.wq_quantize_pack(good, None, 8, 256, None, good, good, good, None) == wq.WQ_ERR_INVALID_ARG
     # shapes
@@ -107,7 +109,7 @@ def test_option_values_are_validated(wq):
         wq.WQ_OPT_WAIT_LIMIT_MS: ([1, 60000, 2000], [0, 60001]),
         wq.WQ_OPT_TEST_STALL: ([1, 0], [2, -1]),
         wq.WQ_OPT_AWQ_LOSS: ([1, 0], [2, -1]),
-        wq.WQ_OPT_TC_A_SOURCE: ([1, 0], [2, -1]),
+        wq.WQ_OPT_TC_KSPLIT: ([0, 1, 2, 4, 8], [3, 16, -1]),
     }
     for opt, (good, bad) in cases.items():
         old = wq.wq_get_option(opt)
@@ -225,9 +227,9 @@ def test_awq_workspace_size_is_its_layout(wq):
     up to 256 bytes: mu (fp64 [K]), the candidates (fp16 [n_alpha][K]), one
     fp64 partial loss per (alpha, tile) -- 128x128 tiles of the two-kernel
     loss or (alpha, 128-row tile of one linear, 512-token chunk) of the fused
-    one, whichever count is larger -- and the fp16 error matrices of one batch
-    of alphas (as many as fit 1 GiB, at least one; the default two-kernel
-    path)."""
+    one, whichever count is larger -- and, on the two-kernel loss path only,
+    the fp16 error matrices of one batch of alphas (as many as fit 1 GiB, at
+    least one). The default fused path keeps no error matrix."""
     def a256(x):
         return (x + 255) // 256 * 256
 
@@ -236,8 +238,14 @@ def test_awq_workspace_size_is_its_layout(wq):
         N = sum(Ns)
         tiles = max(-(-T // 128) * -(-N // 128), sum(-(-n // 128) for n in Ns) * -(-T // 512))
         batch = max(1, min(n_alpha, (1 << 30) // (N * K * 2)))
-        want = a256(K * 8) + a256(n_alpha * K * 2) + a256(n_alpha * tiles * 8) + a256(batch * N * K * 2)
+        want = a256(K * 8) + a256(n_alpha * K * 2) + a256(n_alpha * tiles * 8)
         assert wq.wq_awq_workspace_bytes(T, K, Ns, n_alpha) == want, (T, K, Ns)
+        old = wq.wq_get_option(wq.WQ_OPT_AWQ_LOSS)
+        try:
+            wq.wq_set_option(wq.WQ_OPT_AWQ_LOSS, wq.WQ_AWQ_LOSS_TWO_KERNELS)
+            assert wq.wq_awq_workspace_bytes(T, K, Ns, n_alpha) == want + a256(batch * N * K * 2), (T, K, Ns)
+        finally:
+            wq.wq_set_option(wq.WQ_OPT_AWQ_LOSS, old)
 
 
 def test_binding_constants_match_the_header(wq):

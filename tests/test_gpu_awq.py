@@ -2,12 +2,27 @@
 
 mu (activation statistic) and the candidate scales must match bit for bit
 (a candidate may differ only where fp64 pow lands within 1e-12 of an fp16
-rounding midpoint -- flagged, never seen); losses must agree to 1e-4 relative
-(the GPU loss GEMM runs on the tensor cores with the error matrix in fp16 and
-fp32 accumulation); the chosen alpha must be the oracle's unless the oracle's
-two best losses are within that tolerance of each other; the output scale is
-the chosen candidate bit for bit, and packing with it matches the oracle.
+rounding midpoint -- flagged, never seen).
+
+Losses: the loss GEMM multiplies the fp16 error matrix by X on the tensor
+cores with fp32 accumulation, and that accumulator rounds toward zero: every
+16-channel step of K loses up to an ulp of the running sum, so the GPU
+losses come out low by a nearly alpha-independent factor that grows with K
+(measured on the LLaMA-2-7B block: -7e-6 to -9e-6 at K = 4096, -2.4e-5 at
+K = 11008); the fp16 rounding of E adds a zero-mean part. Bound used:
+LOSS_RTOL = 1e-4 (2 * (K / 16) * 2^-24 = 1.3e-4 at K = 11008 if every step
+lost a whole ulp of |D|).
+
+alpha: what decides it is the alpha-dependent part of the error, measured
+below 3e-6 relative at full size; the chosen alpha must be the oracle's
+unless the oracle's two best losses are within ALPHA_TIE = 1e-5 of each
+other (then the runner-up is accepted). The output scale is the chosen
+candidate bit for bit, and packing with it matches the oracle.
 """
+import hashlib
+import json
+import os
+
 import numpy as np
 import pytest
 import torch
@@ -17,7 +32,11 @@ import synth
 
 pytestmark = pytest.mark.gpu
 
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+
 LOSS_RTOL = 1e-4
+ALPHA_TIE = 1e-5
+LOSS_TOL = {"two_kernels": (LOSS_RTOL, ALPHA_TIE), "fused": (LOSS_RTOL, ALPHA_TIE)}
 
 
 @pytest.fixture(scope="module")
@@ -67,13 +86,14 @@ def _check_one(wq, X, Ws, bits, sym, alphas, ref, path):
     mu = out["mu"].cpu().numpy()
     assert np.array_equal(mu, ref["mu"]), "activation statistic differs"
     losses = out["losses"].cpu().numpy()
+    rtol, tie = LOSS_TOL[path]
     rel = np.abs(losses - ref["losses"]) / ref["losses"]
-    assert np.all(rel <= LOSS_RTOL), (path, rel)
+    assert np.all(rel <= rtol), (path, rel)
     best = int(out["best"].cpu().numpy()[0])
     order = np.argsort(ref["losses"], kind="stable")
     if best != ref["best"]:
         gap = (ref["losses"][order[1]] - ref["losses"][order[0]]) / ref["losses"][order[0]]
-        assert gap < LOSS_RTOL and best == order[1], ("alpha differs", path, best, ref["best"], gap)
+        assert gap < tie and best == order[1], ("alpha differs", path, best, ref["best"], gap)
     s = out["s"].cpu().numpy()
     cand = O.awq_candidates(ref["mu"], alphas)[best]
     diff = s.view(np.uint16) != cand.view(np.uint16)
@@ -122,7 +142,7 @@ def test_awq_alpha_zero_only_equals_rtn(wq, path):
     assert np.all(out["s"].cpu().numpy() == 1.0)
     L = float(out["losses"].cpu().numpy()[0])
     ref = O.awq_loss(X, [W], np.ones(256, np.float16), 4, 128, False)
-    assert abs(L - ref) <= LOSS_RTOL * ref
+    assert abs(L - ref) <= LOSS_TOL[path][0] * ref
 
 
 @pytest.mark.parametrize("T", [1, 511, 512, 513, 1100])
@@ -136,9 +156,10 @@ def test_awq_fused_token_chunks(wq, T):
     check_search(wq, X, Ws, 4, False, alphas=[0.0, 0.3, 0.6])
 
 
-def test_awq_block_o_and_down_full(wq):
+def test_awq_block_o_and_down_full_both_paths(wq):
     """Two of the four search places of a LLaMA-2-7B block at full size
-    (T=512; o: K=4096,N=4096; down: K=11008,N=4096)."""
+    (T=512; o: K=4096,N=4096; down: K=11008,N=4096), both loss paths against
+    the oracle computed here."""
     groups = synth.config_awq_block(5)
     for name, X, named in groups:
         if name not in ("o", "down"):
@@ -147,13 +168,54 @@ def test_awq_block_o_and_down_full(wq):
         print(name, "best", best, "max rel loss err", float(rel.max()))
 
 
-def test_awq_block_qkv_gateup_rows(wq):
-    """The other two places with the first 1024 rows of each linear (full K, T)."""
-    groups = synth.config_awq_block(5)
-    for name, X, named in groups:
-        if name not in ("qkv", "gate_up"):
-            continue
-        check_search(wq, X, [W[:1024] for _, W in named])
+def _digest(a):
+    return hashlib.sha256(np.ascontiguousarray(a).tobytes()).hexdigest()
+
+
+@pytest.mark.parametrize("bits", [4, 3])
+def test_awq_block_all_places_full_size(wq, bits):
+    """All four search places of a LLaMA-2-7B-shaped block at full size (q|k|v
+    N=12288, o, gate|up N=22016, down K=11008; T=512; 20 alphas) on the
+    default (fused) path, against the oracle's search stored by
+    tests/golden/make_awq_block_golden.py: mu and the chosen s bit for bit
+    (SHA-256 of their bytes), the losses within LOSS_RTOL, alpha equal
+    unless the oracle's two best are within ALPHA_TIE, and the alpha-dependent
+    part of the loss error (its spread over the 20 alphas) below ALPHA_TIE / 2.
+    Then the weights are packed with s and run through the decode GEMV
+    against the oracle."""
+    with open(os.path.join(GOLDEN, f"awq_llama7b_block_w{bits}_oracle.json")) as f:
+        gold = json.load(f)
+    worst = 0.0
+    for name, X, named in synth.config_awq_block(5):
+        g = gold["places"][name]
+        Ws = [W for _, W in named]
+        out = wq.wq_awq_scale_search(dev(X), [dev(W) for W in Ws], bits=bits)
+        assert wq.wq_get_last_device_error() == 0
+        assert _digest(out["mu"].cpu().numpy()) == g["mu_sha256"], name
+        ref = np.array([float.fromhex(h) for h in g["losses_hex"]])
+        losses = out["losses"].cpu().numpy()
+        rel = np.abs(losses - ref) / ref
+        worst = max(worst, float(rel.max()))
+        assert np.all(rel <= LOSS_RTOL), (name, rel.max())
+        signed = (losses - ref) / ref
+        assert signed.max() - signed.min() <= ALPHA_TIE / 2, (name, signed.min(), signed.max())
+        best = int(out["best"].item())
+        if best != g["best"]:
+            assert g["gap12"] < ALPHA_TIE, (name, best, g["best"], g["gap12"])
+        else:
+            assert _digest(out["s"].cpu().numpy().view(np.uint16)) == g["s_sha256"], name
+        # the chosen scale drives the packing and the decode matmul: X diag(s)^-1
+        # against the oracle's fp64 matmul of the dequantized weight
+        s = out["s"].cpu().numpy()
+        W = Ws[0]
+        codes, st, z = O.quantize_groups(W, bits, 128, False, s16=s)
+        packed, steps, zeros = wq.wq_quantize_pack(dev(W), dev(s), bits=bits)
+        assert np.array_equal(packed.cpu().numpy().view(np.uint32), O.pack_codes(codes, bits).reshape(-1))
+        xs = (X[:1].astype(np.float32) / s.astype(np.float32)).astype(np.float16)
+        y = wq.wq_w4a16_gemm(dev(xs), packed, steps, zeros, W.shape[0], bits=bits).cpu().numpy()
+        yref = O.gemm_ref(xs, codes, st, z, 128)
+        assert np.linalg.norm(y - yref) / np.linalg.norm(yref) <= 1e-3, name
+    print(f"{bits}-bit block: worst relative loss error {worst:.3g}")
 
 
 def test_workspace_errors(wq):

@@ -30,16 +30,17 @@ def dev(a):
     return torch.from_numpy(np.ascontiguousarray(a)).cuda()
 
 
-def gpu_quantize(wq, W, s, bits, sym):
-    packed, steps, zeros = wq.wq_quantize_pack(dev(W), None if s is None else dev(s), bits=bits, symmetric=sym)
+def gpu_quantize(wq, W, s, bits, sym, group=128):
+    packed, steps, zeros = wq.wq_quantize_pack(dev(W), None if s is None else dev(s), bits=bits, symmetric=sym,
+                                               group_size=group)
     assert wq.wq_get_last_device_error() == 0
     return packed, steps, zeros
 
 
-def assert_quant_parity(wq, W, s, bits, sym):
-    codes, st, z = O.quantize_groups(W, bits, 128, sym, s16=s)
+def assert_quant_parity(wq, W, s, bits, sym, group=128):
+    codes, st, z = O.quantize_groups(W, bits, group, sym, s16=s)
     words = O.pack_codes(codes, bits).reshape(-1)
-    packed, steps, zeros = gpu_quantize(wq, W, s, bits, sym)
+    packed, steps, zeros = gpu_quantize(wq, W, s, bits, sym, group)
     gs, gz = steps.cpu().numpy(), zeros.cpu().numpy()
     assert np.array_equal(gs.view(np.uint16), st.view(np.uint16)), "steps differ"
     assert np.array_equal(gz.view(np.uint16), z.view(np.uint16)), "zeros differ"
@@ -75,6 +76,33 @@ def test_quantize_pack_parity_ragged(wq, bits, sym, awq):
     W = synth.weight(g, 333, 1152, 0.02, channel_frac=0.01, channel_mult=10.0, heavy_frac=0.01)
     s = _awq_scale(1152, 7) if awq else None
     assert_quant_parity(wq, W, s, bits, sym)
+
+
+@pytest.mark.parametrize("group", [32, 64])
+@pytest.mark.parametrize("bits", [3, 4])
+@pytest.mark.parametrize("sym", [False, True])
+@pytest.mark.parametrize("awq", [False, True])
+def test_quantize_pack_small_groups(wq, group, bits, sym, awq):
+    """Groups of 32 and 64 channels ("Quantising Large Language Models",
+    group-size sweep; the W4A8 linear of "MIT 6.5940 Lab 4 + Lab 5" uses 32):
+    codes, words, steps and zeros bit-exact, ragged N, heavy-tailed weights,
+    with and without AWQ scales, and an all-zero group."""
+    g = synth.rng(110 + bits + group)
+    W = synth.weight(g, 333, 1152, 0.02, channel_frac=0.01, channel_mult=10.0, heavy_frac=0.01)
+    W[5, :group] = 0
+    s = _awq_scale(1152, 8) if awq else None
+    assert_quant_parity(wq, W, s, bits, sym, group)
+
+
+@pytest.mark.parametrize("group", [32, 64])
+@pytest.mark.parametrize("bits", [3, 4])
+def test_unpack_dequant_small_groups(wq, group, bits):
+    g = synth.rng(210 + group)
+    W = synth.weight(g, 77, 768, 0.02, channel_frac=0.02, channel_mult=8.0)
+    (codes, st, z), (packed, steps, zeros) = assert_quant_parity(wq, W, None, bits, False, group)
+    out = wq.wq_unpack_dequant(packed, steps, zeros, 77, 768, bits=bits, group_size=group).cpu().numpy()
+    ref = O.dequantize(codes, st, z, group).astype(np.float16)
+    assert np.array_equal(out.view(np.uint16), ref.view(np.uint16))
 
 
 def test_quantize_pack_edge_groups(wq):
@@ -237,9 +265,9 @@ def test_unpack_dequant_bit_exact(wq, bits):
 # S5 GEMV (small M)
 # ---------------------------------------------------------------------------
 
-def run_gemm(wq, X, quant_gpu, N, bits, sym=False):
+def run_gemm(wq, X, quant_gpu, N, bits, sym=False, group=128):
     packed, steps, zeros = quant_gpu
-    Y = wq.wq_w4a16_gemm(dev(X), packed, steps, zeros, N, bits=bits, symmetric=sym)
+    Y = wq.wq_w4a16_gemm(dev(X), packed, steps, zeros, N, bits=bits, symmetric=sym, group_size=group)
     assert wq.wq_get_last_device_error() == 0
     return Y.cpu().numpy()
 
@@ -371,7 +399,7 @@ def test_smallm_sweep_full_weight(wq):
 
 
 # ---------------------------------------------------------------------------
-# S6 tensor-core path (tcgen05), forced, both placements of the A operand
+# S6 tensor-core path (tcgen05), forced, 3- and 4-bit
 # ---------------------------------------------------------------------------
 
 @pytest.fixture
@@ -381,39 +409,81 @@ def tc_path(wq):
     wq.wq_set_option(wq.WQ_OPT_GEMM_PATH, wq.WQ_PATH_AUTO)
 
 
+@pytest.mark.parametrize("bits", [3, 4])
 @pytest.mark.parametrize("M", [1, 3, 16, 17, 48, 64, 100, 128, 200, 256, 300])
 @pytest.mark.parametrize("NK", [(333, 1152), (1000, 4096)])
-def test_tc_gemm_parity(wq, tc_path, M, NK):
+def test_tc_gemm_parity(wq, tc_path, bits, M, NK):
     N, K = NK
-    g = synth.rng(500 + M)
+    g = synth.rng(500 + M + 10 * bits)
     W = synth.weight(g, N, K, 0.02, channel_frac=0.01, channel_mult=10.0)
     X = synth.activations(g, M, K, channel_frac=0.01, channel_mult=20.0)
-    (codes, st, z), qg = assert_quant_parity(wq, W, None, 4, False)
-    assert_close(run_gemm(wq, X, qg, N, 4), O.gemm_ref(X, codes, st, z, 128))
+    (codes, st, z), qg = assert_quant_parity(wq, W, None, bits, False)
+    assert_close(run_gemm(wq, X, qg, N, bits), O.gemm_ref(X, codes, st, z, 128))
 
 
+@pytest.mark.parametrize("bits", [3, 4])
 @pytest.mark.parametrize("S", [2, 3, 5, 16])
 @pytest.mark.parametrize("M", [16, 128, 200])
-def test_tc_gemm_ring_depths(wq, tc_path, S, M):
+def test_tc_gemm_ring_depths(wq, tc_path, bits, S, M):
     """Forced shared-memory ring depths (two CTAs per SM or one), including a
-    ring deeper than the K loop (K = 1152 has 9 stages)."""
+    ring deeper than the K loop (K = 1152 has 9 stages of 128 channels); a
+    depth that one CTA's shared memory cannot hold is refused."""
     N, K = 333, 1152
-    g = synth.rng(600 + M + S)
+    g = synth.rng(600 + M + S + bits)
     W = synth.weight(g, N, K, 0.02, channel_frac=0.01, channel_mult=10.0)
     X = synth.activations(g, M, K, channel_frac=0.01, channel_mult=20.0)
-    (codes, st, z), qg = assert_quant_parity(wq, W, None, 4, False)
+    (codes, st, z), qg = assert_quant_parity(wq, W, None, bits, False)
     wq.wq_set_option(wq.WQ_OPT_TC_STAGES, S)
     try:
         BN = (M + 15) // 16 * 16
-        BK = 64 if BN >= 96 else 128
-        if S * ((BK // 64) * BN * 128 + 128 * BK // 2) + 2048 > 220 * 1024:
+        BK = 64 if BN >= 96 and bits == 4 else 128
+        if S * ((BK // 64) * BN * 128 + 128 * BK * bits // 8) + 2048 > 220 * 1024:
             with pytest.raises(wq.WQError):
-                run_gemm(wq, X, qg, N, 4)
+                run_gemm(wq, X, qg, N, bits)
             return
-        Y = run_gemm(wq, X, qg, N, 4)
+        Y = run_gemm(wq, X, qg, N, bits)
     finally:
         wq.wq_set_option(wq.WQ_OPT_TC_STAGES, 0)
     assert_close(Y, O.gemm_ref(X, codes, st, z, 128))
+
+
+@pytest.mark.parametrize("sym", [False, True])
+def test_tc_gemm_3bit_closed_forms_and_symmetric(wq, tc_path, sym):
+    """3-bit tiles: all codes at the zero point give exactly 0; one nonzero
+    code per row at every channel position of a 32-channel chunk (the three
+    classes of the unpack and the two gathered high-bit channels) gives
+    x_k (q - z) step; symmetric codes against the oracle."""
+    N, K, M = 128, 512, 16
+    X = synth.activations(synth.rng(24), M, K)
+    zeros = np.full((N, K // 128), 4, np.float16)
+    steps = np.random.default_rng(25).uniform(0.001, 0.1, (N, K // 128)).astype(np.float16)
+    codes = np.full((N, K), 4, np.uint8)
+    packed = dev(O.pack_codes(codes, 3).reshape(-1).view(np.int32))
+    assert np.all(run_gemm(wq, X, (packed, dev(steps), dev(zeros)), N, 3) == 0)
+    k_of = (np.arange(N) * 37) % K          # row n: one code at channel k_of[n]
+    q = (np.arange(N) % 7 + (np.arange(N) % 7 >= 4)).astype(np.uint8)  # values 0..7 except 4
+    codes[np.arange(N), k_of] = q
+    packed = dev(O.pack_codes(codes, 3).reshape(-1).view(np.int32))
+    Y = run_gemm(wq, X, (packed, dev(steps), dev(zeros)), N, 3).astype(np.float64)
+    st = steps[np.arange(N), k_of // 128].astype(np.float64)
+    ref = X[:, k_of].astype(np.float64) * ((q.astype(np.float64) - 4) * st)[None, :]
+    assert np.all(np.abs(Y - ref) <= 2.0 ** -10 * np.abs(ref) + 2.0 ** -24)
+    assert set((k_of % 32).tolist()) == set(range(32))
+    W = synth.weight(synth.rng(26), 300, K, 0.02)
+    Xs = synth.activations(synth.rng(27), 40, K)
+    (codes, st, z), qg = assert_quant_parity(wq, W, None, 3, sym)
+    assert_close(run_gemm(wq, Xs, qg, 300, 3, sym=sym), O.gemm_ref(Xs, codes, st, z, 128))
+
+
+def test_smallm_sweep_3bit_full_weight(wq):
+    """The LLaMA-65B-shaped 8192 x 8192 weight at 3 bits through the sweep's
+    batch sizes (M >= 3 on the tensor cores), against the fp64 oracle."""
+    c = synth.config_llama65b_decode(3)
+    (codes, st, z), qg = assert_quant_parity(wq, c.W, None, 3, False)
+    D = O.dequantize(codes, st, z, 128)
+    for M in synth.SMALLM_SWEEP:
+        X = synth.smallm_activations(M)
+        assert_close(run_gemm(wq, X, qg, 8192, 3), X.astype(np.float64) @ D.T)
 
 
 @pytest.mark.parametrize("dw", [4, 8])
@@ -569,48 +639,6 @@ def test_gemv_int_digits_extreme_activations(wq, rows_shape):
     assert np.all(run_gemm(wq, np.zeros((1, K), np.float16), qg, N, 4) == 0)
 
 
-@pytest.fixture
-def tc_smem_a(wq):
-    """The tensor-core kernel with its dequantized weight tile in shared memory."""
-    wq.wq_set_option(wq.WQ_OPT_GEMM_PATH, wq.WQ_PATH_TENSOR_CORE)
-    wq.wq_set_option(wq.WQ_OPT_TC_A_SOURCE, wq.WQ_TC_A_SMEM)
-    yield
-    wq.wq_set_option(wq.WQ_OPT_TC_A_SOURCE, wq.WQ_TC_A_TMEM)
-    wq.wq_set_option(wq.WQ_OPT_GEMM_PATH, wq.WQ_PATH_AUTO)
-
-
-@pytest.mark.parametrize("M", [1, 3, 16, 17, 64, 100, 128, 200, 300])
-@pytest.mark.parametrize("NK", [(333, 1152), (1000, 4096)])
-def test_tc_gemm_smem_a_parity(wq, tc_smem_a, M, NK):
-    """Shared-memory A tiles: the same tolerance against the fp64 reference
-    (128- and 64-channel stages, one to several 256-row X chunks, ragged N)."""
-    N, K = NK
-    g = synth.rng(700 + M)
-    W = synth.weight(g, N, K, 0.02, channel_frac=0.01, channel_mult=10.0)
-    X = synth.activations(g, M, K, channel_frac=0.01, channel_mult=20.0)
-    (codes, st, z), qg = assert_quant_parity(wq, W, None, 4, False)
-    assert_close(run_gemm(wq, X, qg, N, 4), O.gemm_ref(X, codes, st, z, 128))
-
-
-@pytest.mark.parametrize("S,BK", [(2, 0), (5, 0), (0, 64), (3, 64)])
-@pytest.mark.parametrize("M", [16, 64, 128])
-def test_tc_gemm_smem_a_ring_depths(wq, tc_smem_a, S, BK, M):
-    """Forced ring depths and 64-channel stages with shared-memory A tiles."""
-    N, K = 333, 1152
-    g = synth.rng(800 + M + S + BK)
-    W = synth.weight(g, N, K, 0.02, channel_frac=0.01, channel_mult=10.0)
-    X = synth.activations(g, M, K, channel_frac=0.01, channel_mult=20.0)
-    (codes, st, z), qg = assert_quant_parity(wq, W, None, 4, False)
-    wq.wq_set_option(wq.WQ_OPT_TC_STAGES, S)
-    wq.wq_set_option(wq.WQ_OPT_TC_BK, BK)
-    try:
-        Y = run_gemm(wq, X, qg, N, 4)
-    finally:
-        wq.wq_set_option(wq.WQ_OPT_TC_STAGES, 0)
-        wq.wq_set_option(wq.WQ_OPT_TC_BK, 0)
-    assert_close(Y, O.gemm_ref(X, codes, st, z, 128))
-
-
 @pytest.mark.parametrize("bits", [3, 4])
 @pytest.mark.parametrize("M", [1, 2, 5])
 @pytest.mark.parametrize("NK", [(64, 32768), (333, 16512)])
@@ -624,3 +652,96 @@ def test_gemv_beyond_row_kernel_k(wq, bits, M, NK):
     X = synth.activations(g, M, K, channel_frac=0.01, channel_mult=20.0)
     (codes, st, z), qg = assert_quant_parity(wq, W, None, bits, False)
     assert_close(run_gemm(wq, X, qg, N, bits), O.gemm_ref(X, codes, st, z, 128))
+
+
+# ---------------------------------------------------------------------------
+# groups of 32 and 64 channels through the matmul (row-streaming GEMV for
+# M <= 2 where its lanes hold whole groups, the tensor cores otherwise)
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("group", [32, 64])
+@pytest.mark.parametrize("bits", [3, 4])
+@pytest.mark.parametrize("M", [1, 2, 3, 16, 130])
+@pytest.mark.parametrize("NK", [(333, 1152), (1000, 4096), (64, 11008)])
+def test_gemm_small_groups(wq, group, bits, M, NK):
+    N, K = NK
+    g = synth.rng(1200 + M + bits + group)
+    W = synth.weight(g, N, K, 0.02, channel_frac=0.01, channel_mult=10.0)
+    X = synth.activations(g, M, K, channel_frac=0.01, channel_mult=20.0)
+    (codes, st, z), qg = assert_quant_parity(wq, W, None, bits, False, group)
+    assert_close(run_gemm(wq, X, qg, N, bits, group=group), O.gemm_ref(X, codes, st, z, group))
+
+
+@pytest.mark.parametrize("group", [32, 64])
+def test_gemm_small_groups_variants(wq, group):
+    """Every row-kernel shape and both lane-sum variants at M = 1 and 2, the
+    tensor-core kernel forced at M = 1 and with 64-channel stages, symmetric
+    codes: all against the oracle."""
+    N, K = 300, 2048
+    g = synth.rng(1300 + group)
+    W = synth.weight(g, N, K, 0.02, channel_frac=0.01, channel_mult=10.0)
+    (codes, st, z), qg = assert_quant_parity(wq, W, None, 4, True, group)
+    for M in (1, 2):
+        X = synth.activations(g, M, K, channel_frac=0.01, channel_mult=20.0)
+        ref = O.gemm_ref(X, codes, st, z, group)
+        for shape in (1, 2, 3, 4):
+            for variant in (wq.WQ_GEMV_OFFSET_SUMS, wq.WQ_GEMV_INT_DIGITS):
+                wq.wq_set_option(wq.WQ_OPT_GEMV_ROWS_SHAPE, shape)
+                wq.wq_set_option(wq.WQ_OPT_GEMV_VARIANT, variant)
+                try:
+                    assert_close(run_gemm(wq, X, qg, N, 4, sym=True, group=group), ref)
+                finally:
+                    wq.wq_set_option(wq.WQ_OPT_GEMV_ROWS_SHAPE, 0)
+                    wq.wq_set_option(wq.WQ_OPT_GEMV_VARIANT, wq.WQ_GEMV_OFFSET_SUMS)
+        wq.wq_set_option(wq.WQ_OPT_GEMM_PATH, wq.WQ_PATH_TENSOR_CORE)
+        try:
+            assert_close(run_gemm(wq, X, qg, N, 4, sym=True, group=group), ref)
+        finally:
+            wq.wq_set_option(wq.WQ_OPT_GEMM_PATH, wq.WQ_PATH_AUTO)
+    X = synth.activations(g, 100, K)
+    wq.wq_set_option(wq.WQ_OPT_TC_BK, 64)
+    try:
+        assert_close(run_gemm(wq, X, qg, N, 4, sym=True, group=group), O.gemm_ref(X, codes, st, z, group))
+    finally:
+        wq.wq_set_option(wq.WQ_OPT_TC_BK, 0)
+
+
+
+@pytest.mark.parametrize("bits", [3, 4])
+@pytest.mark.parametrize("M,ks", [(3, 2), (3, 4), (3, 8), (16, 2), (16, 4), (16, 8), (64, 2), (100, 2), (128, 2)])
+def test_tc_gemm_split_k(wq, tc_path, ks, bits, M):
+    """K split over a cluster of 2, 4 or 8 CTAs per row tile (partial tiles
+    added in rank order through distributed shared memory): ragged N, ranges
+    that do not divide K evenly (K = 4224 has 33 stages of 128 channels), and
+    groups of 128 or 32 channels. (Wider tiles with more CTAs do not fit their
+    partial tiles in the first CTA's ring and are refused; see below.)"""
+    N, K = 333, 4224
+    g = synth.rng(1400 + ks + M + bits)
+    W = synth.weight(g, N, K, 0.02, channel_frac=0.01, channel_mult=10.0)
+    X = synth.activations(g, M, K, channel_frac=0.01, channel_mult=20.0)
+    for group in (128, 32):
+        (codes, st, z), qg = assert_quant_parity(wq, W, None, bits, False, group)
+        wq.wq_set_option(wq.WQ_OPT_TC_KSPLIT, ks)
+        try:
+            Y = run_gemm(wq, X, qg, N, bits, group=group)
+        finally:
+            wq.wq_set_option(wq.WQ_OPT_TC_KSPLIT, 0)
+        assert_close(Y, O.gemm_ref(X, codes, st, z, group))
+
+
+def test_tc_gemm_split_k_refused_when_partials_do_not_fit(wq, tc_path):
+    """A split whose partial tiles exceed the first CTA's ring is refused
+    (WQ_ERR_CUDA), not run: M = 256 with a two-stage ring at 8 CTAs."""
+    N, K, M = 256, 4096, 256
+    g = synth.rng(1500)
+    W = synth.weight(g, N, K, 0.02)
+    (_, _, _), qg = assert_quant_parity(wq, W, None, 4, False)
+    wq.wq_set_option(wq.WQ_OPT_TC_KSPLIT, 8)
+    wq.wq_set_option(wq.WQ_OPT_TC_STAGES, 2)
+    try:
+        with pytest.raises(wq.WQError) as e:
+            run_gemm(wq, synth.activations(g, M, K), qg, N, 4)
+        assert e.value.status == wq.WQ_ERR_CUDA
+    finally:
+        wq.wq_set_option(wq.WQ_OPT_TC_KSPLIT, 0)
+        wq.wq_set_option(wq.WQ_OPT_TC_STAGES, 0)

@@ -17,7 +17,13 @@ import synth
 
 pytestmark = pytest.mark.gpu
 
-LOSS_RTOL = 1e-4  # the loss tolerance of the AWQ parity tests
+# the loss tolerance of the AWQ parity tests (both loss paths)
+LOSS_RTOL = {"fused": 1e-4, "two_kernels": 1e-4}
+
+# (T, N_i, bits, symmetric): two row chunks that both end on a 128-row
+# boundary; and a ragged case -- T not a multiple of 128, a last chunk whose
+# rows end inside a 128-row tile, 3-bit symmetric codes
+CASES = {"even": (256, (1700, 1500), 4, False), "ragged": (200, (2100, 1101), 3, True)}
 
 
 @pytest.fixture(scope="module")
@@ -32,30 +38,31 @@ def dev(a):
     return torch.from_numpy(np.ascontiguousarray(a)).cuda()
 
 
+@pytest.mark.parametrize("case", sorted(CASES))
 @pytest.mark.parametrize("path", ["two_kernels", "fused"])
-def test_noalloc_matches_workspace_entry_point_twice(wq, path):
+def test_noalloc_matches_workspace_entry_point_twice(wq, path, case):
     """Both loss paths: the fused one needs no error-matrix chunks at all."""
     old = wq.wq_get_option(wq.WQ_OPT_AWQ_LOSS)
     wq.wq_set_option(wq.WQ_OPT_AWQ_LOSS, wq.WQ_AWQ_LOSS_FUSED if path == "fused" else wq.WQ_AWQ_LOSS_TWO_KERNELS)
     try:
-        _noalloc_matches(wq)
+        _noalloc_matches(wq, LOSS_RTOL[path], *CASES[case])
     finally:
         wq.wq_set_option(wq.WQ_OPT_AWQ_LOSS, old)
 
 
-def _noalloc_matches(wq):
-    g = synth.rng(900)
-    K = 4096  # 2048-row error chunks: the stacked 3200 rows span two chunks
-    X = dev(synth.activations(g, 256, K, channel_frac=0.01, channel_mult=20.0))
-    Ws = [dev(synth.weight(g, 1700, K, 0.02)), dev(synth.weight(g, 1500, K, 0.02))]
-    ref = wq.wq_awq_scale_search(X, Ws)
+def _noalloc_matches(wq, rtol, T, Ns, bits, sym):
+    g = synth.rng(900 + T)
+    K = 4096  # 2048-row error chunks: the stacked rows span two chunks
+    X = dev(synth.activations(g, T, K, channel_frac=0.01, channel_mult=20.0))
+    Ws = [dev(synth.weight(g, n, K, 0.02)) for n in Ns]
+    ref = wq.wq_awq_scale_search(X, Ws, bits=bits, symmetric=sym)
     assert wq.wq_get_last_device_error() == 0
     for _ in range(2):
-        out = wq.wq_awq_scale_search_noalloc(X, Ws)
+        out = wq.wq_awq_scale_search_noalloc(X, Ws, bits=bits, symmetric=sym)
         assert wq.wq_get_last_device_error() == 0
         assert torch.equal(out["mu"], ref["mu"])
         rel = (out["losses"] - ref["losses"]).abs() / ref["losses"]
-        assert float(rel.max()) <= LOSS_RTOL
+        assert float(rel.max()) <= rtol
         assert int(out["best"].item()) == int(ref["best"].item())
         assert torch.equal(out["s"].view(torch.int16), ref["s"].view(torch.int16))
 

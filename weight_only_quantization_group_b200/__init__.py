@@ -37,6 +37,8 @@ __all__ = [
     "wq_awq_scale_search_noalloc",
     "wq_awq_fold_norm",
     "wq_awq_fold_linear_rows",
+    "wq_gptq_workspace_bytes",
+    "wq_gptq_quantize_pack",
     "EXPORTED_SYMBOLS",
 ]
 
@@ -61,6 +63,8 @@ EXPORTED_SYMBOLS = (
     "wq_awq_scale_search_noalloc",
     "wq_awq_fold_norm",
     "wq_awq_fold_linear_rows",
+    "wq_gptq_workspace_bytes",
+    "wq_gptq_quantize_pack",
 )
 
 WQ_OK = 0
@@ -93,11 +97,9 @@ WQ_OPT_TC_DEQUANT_WARPS = 12
 WQ_OPT_WAIT_LIMIT_MS = 13
 WQ_OPT_TEST_STALL = 14
 WQ_OPT_AWQ_LOSS = 15
+WQ_OPT_TC_KSPLIT = 16
 WQ_AWQ_LOSS_TWO_KERNELS = 0
 WQ_AWQ_LOSS_FUSED = 1
-WQ_OPT_TC_A_SOURCE = 16
-WQ_TC_A_TMEM = 0
-WQ_TC_A_SMEM = 1
 
 
 class WQError(RuntimeError):
@@ -136,6 +138,8 @@ def _load() -> ctypes.CDLL:
         "wq_awq_scale_search_noalloc": (i32, [vp, i64, i64, ctypes.POINTER(vp), ctypes.POINTER(i64), i32, cfgp,
                                               ctypes.POINTER(ctypes.c_double), i32, vp, vp, vp, vp, vp]),
         "wq_awq_fold_norm": (i32, [vp, vp, i64, vp, vp]),
+        "wq_gptq_workspace_bytes": (sz, [i64, i64, cfgp]),
+        "wq_gptq_quantize_pack": (i32, [vp, i64, vp, i64, i64, cfgp, ctypes.c_double, vp, vp, vp, vp, sz, vp]),
         "wq_awq_fold_linear_rows": (i32, [vp, vp, vp, i64, i64, vp, vp, vp]),
     }
     for name, (res, args) in sig.items():
@@ -542,3 +546,45 @@ def wq_awq_fold_linear_rows(W: torch.Tensor, s: torch.Tensor, b: torch.Tensor | 
                                           _stream(stream, W.device.index))
     _raise(st, "wq_awq_fold_linear_rows")
     return W_out, b_out
+
+
+def wq_gptq_workspace_bytes(N: int, K: int, *, bits: int = 4, group_size: int = 128, symmetric: bool = False) -> int:
+    c = _cfg(bits, group_size, symmetric)
+    return int(_lib.wq_gptq_workspace_bytes(N, K, ctypes.byref(c)))
+
+
+def wq_gptq_quantize_pack(W: torch.Tensor, X: torch.Tensor, *, bits: int = 4, group_size: int = 128,
+                          symmetric: bool = False, damp: float = 0.01, workspace: torch.Tensor | None = None,
+                          out=None, stream=None):
+    """GPTQ quantize + pack of an fp16 [N][K] weight with calibration inputs X
+    (fp16 [T][K]); returns (packed u32 as int32, steps, zeros) in the layout of
+    wq_quantize_pack. `workspace` (uint8, >= wq_gptq_workspace_bytes) is
+    allocated when not given."""
+    _check(W, torch.float16, "W")
+    _check(X, torch.float16, "X")
+    if W.dim() != 2 or X.dim() != 2 or X.shape[1] != W.shape[1]:
+        raise ValueError(f"W must be [N][K] and X [T][K], got {tuple(W.shape)} and {tuple(X.shape)}")
+    N, K = W.shape
+    T = X.shape[0]
+    c = _cfg(bits, group_size, symmetric)
+    nw = _packed_words_of(N, K, c)
+    if out is None:
+        G = K // group_size if group_size > 0 else 0
+        packed = torch.empty(max(nw, 1), dtype=torch.int32, device=W.device)
+        steps = torch.empty((N, G), dtype=torch.float16, device=W.device)
+        zeros = torch.empty((N, G), dtype=torch.float16, device=W.device)
+    else:
+        packed, steps, zeros = out
+        _quant_operands(N, K, c, packed, steps, zeros)
+    need = int(_lib.wq_gptq_workspace_bytes(N, K, ctypes.byref(c)))
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=W.device)
+    elif not workspace.is_contiguous():
+        raise ValueError("workspace must be contiguous")
+    _on_device_of(W, X=X, packed=packed, steps=steps, zeros=zeros, workspace=workspace)
+    with _device_of(W):
+        st = _lib.wq_gptq_quantize_pack(_ptr(X), T, _ptr(W), N, K, ctypes.byref(c), float(damp), _ptr(packed),
+                                        _ptr(steps), _ptr(zeros), workspace.data_ptr(),
+                                        workspace.numel() * workspace.element_size(), _stream(stream, W.device.index))
+    _raise(st, "wq_gptq_quantize_pack")
+    return packed, steps, zeros

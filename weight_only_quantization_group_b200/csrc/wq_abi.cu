@@ -44,8 +44,7 @@ bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) %
 int32_t check_cfg(const wq_quant_cfg* cfg) {
   if (cfg == nullptr) return WQ_ERR_INVALID_ARG;
   if (cfg->bits != 3 && cfg->bits != 4) return cfg->bits >= 2 && cfg->bits <= 8 ? WQ_ERR_UNSUPPORTED : WQ_ERR_INVALID_ARG;
-  if (cfg->group_size != wq::kGroup)
-    return (cfg->group_size == 32 || cfg->group_size == 64) ? WQ_ERR_UNSUPPORTED : WQ_ERR_INVALID_ARG;
+  if (cfg->group_size != 32 && cfg->group_size != 64 && cfg->group_size != wq::kGroup) return WQ_ERR_INVALID_ARG;
   if (cfg->symmetric != 0 && cfg->symmetric != 1) return WQ_ERR_INVALID_ARG;
   return WQ_OK;
 }
@@ -73,7 +72,7 @@ std::atomic<int64_t> g_opt_tc_dequant_warps{0};
 std::atomic<int64_t> g_opt_wait_limit_ms{2000};
 std::atomic<int64_t> g_opt_test_stall{0};
 std::atomic<int64_t> g_opt_awq_loss{WQ_AWQ_LOSS_FUSED};
-std::atomic<int64_t> g_opt_tc_a_source{WQ_TC_A_TMEM};
+std::atomic<int64_t> g_opt_tc_ksplit{0};
 
 }  // namespace
 
@@ -113,8 +112,8 @@ int32_t wq_quantize_pack(const void* W, const void* s, int64_t N, int64_t K, con
     return WQ_ERR_ALIGNMENT;
   int* flag = device_flag();
   if (!flag) return WQ_ERR_CUDA;
-  return cuda_status(wq::launch_quantize_pack(W, s, N, K, cfg->bits, cfg->symmetric != 0, packed, steps, zeros,
-                                              flag, static_cast<cudaStream_t>(stream)));
+  return cuda_status(wq::launch_quantize_pack(W, s, N, K, cfg->bits, cfg->group_size, cfg->symmetric != 0, packed,
+                                              steps, zeros, flag, static_cast<cudaStream_t>(stream)));
 }
 
 int32_t wq_unpack_dequant(const uint32_t* packed, const void* steps, const void* zeros, int64_t N, int64_t K,
@@ -126,7 +125,7 @@ int32_t wq_unpack_dequant(const uint32_t* packed, const void* steps, const void*
   if (!packed || !steps || !zeros || !W_out) return WQ_ERR_INVALID_ARG;
   if (!aligned(packed, 16) || !aligned(W_out, 16) || !aligned(steps, 4) || !aligned(zeros, 4))
     return WQ_ERR_ALIGNMENT;
-  return cuda_status(wq::launch_unpack_dequant(packed, steps, zeros, N, K, cfg->bits, W_out,
+  return cuda_status(wq::launch_unpack_dequant(packed, steps, zeros, N, K, cfg->bits, cfg->group_size, W_out,
                                                static_cast<cudaStream_t>(stream)));
 }
 
@@ -149,24 +148,26 @@ int32_t wq_w4a16_gemm(const void* X, const uint32_t* packed, const void* steps, 
     return WQ_ERR_ALIGNMENT;
   // one reading of every option this call uses
   const int64_t path = g_opt_gemm_path, variant = g_opt_gemv_variant, pdl = g_opt_pdl;
-  bool tensor_core = cfg->bits == 4 && M >= g_opt_crossover_m;
+  const int group = cfg->group_size;
+  const bool rows_ok = g_opt_gemv_kernel != WQ_GEMV_KERNEL_TILED && variant != WQ_GEMV_EXACT &&
+                       wq::gemv_rows_supported(cfg->bits, group, M, K);
+  bool tensor_core = M >= g_opt_crossover_m;
   if (path == WQ_PATH_GEMV) tensor_core = false;
-  if (path == WQ_PATH_TENSOR_CORE) {
-    if (cfg->bits != 4) return WQ_ERR_UNSUPPORTED;
-    tensor_core = true;
-  }
+  if (path == WQ_PATH_TENSOR_CORE) tensor_core = true;
+  // groups of 32 or 64 channels that the row-streaming kernel does not take
+  // (M > 2, 3-bit groups of 32, groups of 32 with K > 8192) run on the tensor
+  // cores: the tiled GEMV handles groups of 128 only
+  if (group != wq::kGroup && !rows_ok) tensor_core = true;
   if (tensor_core) {
     int* flag = device_flag();
     if (!flag) return WQ_ERR_CUDA;
-    return cuda_status(wq::launch_gemm_tc(X, packed, steps, zeros, M, N, K, Y, flag,
+    return cuda_status(wq::launch_gemm_tc(X, packed, steps, zeros, M, N, K, cfg->bits, group, Y, flag,
                                           static_cast<cudaStream_t>(stream), (int)g_opt_tc_stages,
-                                          (int)g_opt_tc_bk, (int)g_opt_tc_dequant_warps,
-                                          (int)g_opt_wait_limit_ms, g_opt_test_stall != 0,
-                                          g_opt_tc_a_source == WQ_TC_A_SMEM));
+                                          (int)g_opt_tc_bk, (int)g_opt_tc_dequant_warps, (int)g_opt_tc_ksplit,
+                                          (int)g_opt_wait_limit_ms, g_opt_test_stall != 0));
   }
-  if (g_opt_gemv_kernel != WQ_GEMV_KERNEL_TILED && variant != WQ_GEMV_EXACT &&
-      wq::gemv_rows_supported(cfg->bits, M, K))
-    return cuda_status(wq::launch_gemv_rows(X, packed, steps, zeros, M, N, K, cfg->bits, Y,
+  if (rows_ok)
+    return cuda_status(wq::launch_gemv_rows(X, packed, steps, zeros, M, N, K, cfg->bits, group, Y,
                                             static_cast<cudaStream_t>(stream),
                                             (int)g_opt_gemv_rows_shape, variant == WQ_GEMV_INT_DIGITS,
                                             (int)g_opt_gemv_grid, pdl != 0));
@@ -183,6 +184,7 @@ static int32_t check_awq(int64_t T, int64_t K, const int64_t* N_i, int32_t n_lin
                          const wq_quant_cfg* cfg) {
   int32_t st = check_cfg(cfg);
   if (st != WQ_OK) return st;
+  if (cfg->group_size != wq::kGroup) return WQ_ERR_UNSUPPORTED;
   if (T < 1 || T > (int64_t)INT32_MAX / 2 || !N_i || n_lin < 1 || n_lin > 8 || n_alpha < 1 || n_alpha > 64)
     return WQ_ERR_INVALID_ARG;
   int64_t tot = 0;
@@ -253,6 +255,30 @@ int32_t wq_awq_scale_search_noalloc(const void* X, int64_t T, int64_t K, const v
                                                    static_cast<cudaStream_t>(stream)));
 }
 
+size_t wq_gptq_workspace_bytes(int64_t N, int64_t K, const wq_quant_cfg* cfg) {
+  if (check_cfg(cfg) != WQ_OK || check_shape(N, K) != WQ_OK) return 0;
+  return wq::plan_gptq(N, K).total;
+}
+
+int32_t wq_gptq_quantize_pack(const void* X, int64_t T, const void* W, int64_t N, int64_t K, const wq_quant_cfg* cfg,
+                              double damp, uint32_t* packed, void* steps, void* zeros, void* workspace,
+                              size_t workspace_bytes, void* stream) {
+  NvtxRange nvtx_range("wq_gptq_quantize_pack");
+  int32_t st = check_cfg(cfg);
+  if (st != WQ_OK) return st;
+  if ((st = check_shape(N, K)) != WQ_OK) return st;
+  if (T < 1 || T > (int64_t)INT32_MAX / 2 || !(damp >= 0.0 && damp < 1e6)) return WQ_ERR_INVALID_ARG;
+  if (!X || !W || !packed || !steps || !zeros) return WQ_ERR_INVALID_ARG;
+  if (!aligned(X, 2) || !aligned(W, 2) || !aligned(packed, 16) || !aligned(steps, 2) || !aligned(zeros, 2))
+    return WQ_ERR_ALIGNMENT;
+  if (!workspace || workspace_bytes < wq::plan_gptq(N, K).total) return WQ_ERR_WORKSPACE;
+  if (!aligned(workspace, 256)) return WQ_ERR_ALIGNMENT;
+  int* flag = device_flag();
+  if (!flag) return WQ_ERR_CUDA;
+  return cuda_status(wq::launch_gptq(X, T, W, N, K, cfg->bits, cfg->group_size, cfg->symmetric != 0, damp, packed,
+                                     steps, zeros, workspace, flag, static_cast<cudaStream_t>(stream)));
+}
+
 int32_t wq_awq_fold_norm(const void* gamma, const void* s, int64_t K, void* gamma_out, void* stream) {
   NvtxRange nvtx_range("wq_awq_fold_norm");
   if (!gamma || !s || !gamma_out) return WQ_ERR_INVALID_ARG;
@@ -312,9 +338,9 @@ int32_t wq_set_option(int32_t option, int64_t value) {
       if (value != WQ_AWQ_LOSS_TWO_KERNELS && value != WQ_AWQ_LOSS_FUSED) return WQ_ERR_INVALID_ARG;
       g_opt_awq_loss = value;
       return WQ_OK;
-    case WQ_OPT_TC_A_SOURCE:
-      if (value != WQ_TC_A_TMEM && value != WQ_TC_A_SMEM) return WQ_ERR_INVALID_ARG;
-      g_opt_tc_a_source = value;
+    case WQ_OPT_TC_KSPLIT:
+      if (value != 0 && value != 1 && value != 2 && value != 4 && value != 8) return WQ_ERR_INVALID_ARG;
+      g_opt_tc_ksplit = value;
       return WQ_OK;
     case WQ_OPT_TC_DEQUANT_WARPS:
       if (value != 0 && value != 4 && value != 8) return WQ_ERR_INVALID_ARG;
@@ -356,7 +382,7 @@ int64_t wq_get_option(int32_t option) {
     case WQ_OPT_TEST_STALL: return g_opt_test_stall;
     case WQ_OPT_PDL: return g_opt_pdl;
     case WQ_OPT_AWQ_LOSS: return g_opt_awq_loss;
-    case WQ_OPT_TC_A_SOURCE: return g_opt_tc_a_source;
+    case WQ_OPT_TC_KSPLIT: return g_opt_tc_ksplit;
   }
   return -1;
 }

@@ -330,6 +330,10 @@ awq_loss_kernel(const __grid_constant__ CUtensorMap tmE, const __grid_constant__
 //
 // The three producers run independently, so W is fetched a group ahead of
 // the error rows, and the error rows run up to two groups ahead of the MMA.
+// (A variant that also multiplied E - fp16(E) into the same accumulator,
+// for about 22 significant bits of E, measured no closer to the fp64 losses:
+// at K >= 4096 the accumulator's own rounding toward zero, about -1e-5 of
+// the loss, dominates, and the second product doubled it.)
 constexpr int kFusedThreads = 224;
 constexpr int kFusedTokens = 512;                       // tokens per CTA = TMEM columns
 constexpr int kFusedXStages = 2;
@@ -453,7 +457,7 @@ awq_loss_fused_kernel(const __grid_constant__ FusedWMaps wm, const __grid_consta
         const int c = lane + 32 * i;
         const __half v = s[g * kGroup + c];
         sh[c] = v;
-        rs[c] = -rcp_approx(__half2float(v));
+        rs[c] = -rcp_refined(__half2float(v));  // within 2^-24 (1 + 2^-19): no bias in E
       }
       mbar_arrive(w_full);  // this lane's s values are in place
     }

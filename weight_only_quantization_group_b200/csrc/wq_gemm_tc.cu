@@ -1,4 +1,5 @@
-// S6: W4A16 matmul on the 5th-generation tensor cores for M = 3..256 rows of X.
+// S6: W4A16 / W3A16 matmul on the 5th-generation tensor cores for M = 3..256
+// rows of X per launch (larger M in chunks of 256).
 //
 // When M grows the weight-only matmul stops being a pure weight stream and
 // becomes a dense contraction ("Quantising Large Language Models for
@@ -12,7 +13,8 @@
 // in tensor memory as [128 lanes = n][M columns]). K advances in stages of
 // BK = 128 (one quantization group) or 64 input channels:
 //   warp 0    TMA producer into a ring of S shared-memory stages: the packed
-//             tile (128 rows x BK/2 bytes, 64- or 32-byte swizzle) and the X
+//             tile (128 rows x BK/2 bytes for 4-bit, 64- or 32-byte swizzle;
+//             128 rows x 48 bytes for 3-bit, unswizzled) and the X
 //             tile (BK/64 128-byte-swizzled 64-channel boxes)
 //   warp 1    TMEM owner and single-thread tcgen05.mma issuer (BK/16 MMAs
 //             per stage)
@@ -23,8 +25,14 @@
 //             (tcgen05.ld -> fp16 -> Y).
 // The shared-memory ring and the TMEM A ring are separate, so the TMA runs as
 // far ahead as shared memory allows while only two A buffers occupy TMEM.
+// Split K: when the row tiles cannot fill the GPU (N = 8192 gives 64 tiles
+// for 148 SMs), the KS CTAs of a thread-block cluster take consecutive K
+// ranges of the same tile; ranks 1.. send their fp32 partial tiles to rank 0's
+// shared memory (its idle ring) over distributed shared memory, and rank 0
+// adds them in rank order (deterministic) and writes Y.
 // Every mbarrier wait is bounded; on a timeout the kernel latches
 // WQ_ERR_TIMEOUT, drains its own copies, frees its tensor memory and returns.
+#include <cooperative_groups.h>
 #include <type_traits>
 
 #include "wq_sm100.cuh"
@@ -48,6 +56,7 @@ struct TcArgs {
   int* err;
   long long spin_limit;  // SM clock cycles a bounded wait may last
   int stall;             // test hook: issue no loads, so every consumer wait runs out
+  int ksplit;            // CTAs of a cluster sharing one row tile along K (grid.y)
 };
 
 __device__ __forceinline__ __half2 u2h(uint32_t u) { return *reinterpret_cast<__half2*>(&u); }
@@ -71,21 +80,56 @@ __device__ __forceinline__ uint4 dequant_word4(uint32_t w, __half2 zz, __half2 z
   return r;
 }
 
+// 32 3-bit codes (three packed words: k0..k31) -> sixteen fp16 pairs
+// fp16_rn((q - zero) * step), in k order. One LOP3 leaves a pair as
+// 1024 + c q with c = 1, 8 or 64 (the code's bit offset in its 16-bit lane);
+// (1024 + c q) / c - (1024 / c + zero) is exact, so again the only rounding
+// is the product. Pair j of word t holds k = 10t + 2j, 10t + 2j + 1; bit b of
+// k = 30 and 31 sits in bit 15 and 31 of word b.
+__device__ __forceinline__ void dequant_chunk3(const uint32_t* w3, __half2 zz, __half2 zz8n, __half2 zz64n, __half2 s2,
+                                               uint32_t (&o)[16]) {
+  const __half2 i8 = __float2half2_rn(0.125f), i64 = __float2half2_rn(0.015625f);
+#pragma unroll
+  for (int t = 0; t < 3; ++t) {
+    const uint32_t w = w3[t], w9 = w >> 9;
+    o[5 * t + 0] = h2u(__hmul2(__hsub2(u2h(and_or(w, 0x00070007u, kHalf2Magic)), zz), s2));
+    o[5 * t + 1] = h2u(__hmul2(__hfma2(u2h(and_or(w, 0x00380038u, kHalf2Magic)), i8, zz8n), s2));
+    o[5 * t + 2] = h2u(__hmul2(__hfma2(u2h(and_or(w, 0x01C001C0u, kHalf2Magic)), i64, zz64n), s2));
+    o[5 * t + 3] = h2u(__hmul2(__hsub2(u2h(and_or(w9, 0x00070007u, kHalf2Magic)), zz), s2));
+    o[5 * t + 4] = h2u(__hmul2(__hfma2(u2h(and_or(w9, 0x00380038u, kHalf2Magic)), i8, zz8n), s2));
+  }
+  uint32_t hb = and_or(w3[0] >> 15, 0x00010001u, kHalf2Magic);
+  hb = and_or(w3[1] >> 14, 0x00020002u, hb);
+  hb = and_or(w3[2] >> 13, 0x00040004u, hb);
+  o[15] = h2u(__hmul2(__hsub2(u2h(hb), zz), s2));
+}
+
+// BITS: 4 (packed words of 8 codes) or 3 (chunks of three words per 32 codes;
+// 128-channel stages, rows of 48 bytes, no swizzle needed: a quarter warp's
+// 16-byte reads at a 48-byte row pitch already fall on distinct banks).
 // BK: input channels per stage, 128 (one group) or 64 (half a group; shallower
-// shared-memory stages, so a deeper ring fits when M is large).
+// shared-memory stages, so a deeper ring fits when M is large; 4-bit only).
 // NH: dequantizing warp quartets; each of the NH owns 1/NH of a stage's words
 // of every row (more warps hide more latency, fewer amortize the per-stage
 // waits over more weights).
 // NA: depth of the TMEM A ring (2, or 3 when the tile leaves room).
-template <int BK, int NH, int NA>
+// GS: quantization group (128, or 32 / 64 channels: then every stage holds
+// BK / GS groups, and each dequantizing thread applies the step and zero of
+// the NGT groups of its part of the stage).
+template <int BITS, int BK, int NH, int NA, int GS>
 __global__ void __launch_bounds__(64 + 128 * NH, 1)
 w4a16_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmP,
                      TcArgs a) {
-  constexpr int kPackedStage = kTcRows * BK / 2;  // bytes of the packed tile
+  static_assert(BITS == 4 || (BITS == 3 && BK == 128 && NH == 1), "3-bit tiles: 128-channel stages, 4 warps");
+  static_assert(GS >= BK || GS <= BK / NH, "small groups: whole groups in every thread's part");
+  constexpr int NGT = GS < BK ? BK / NH / GS : 1;  // groups in one thread's part of a stage
+  constexpr int kRowBytes = BK * BITS / 8;        // packed bytes of one row and stage
+  constexpr int kPackedStage = kTcRows * kRowBytes;  // bytes of the packed tile
   constexpr int kACols = BK / 2;                  // TMEM columns per A buffer
   constexpr int kXBoxes = BK / 64;                // 64-channel X boxes per stage
-  constexpr int kWords = BK / 8 / NH;             // packed words per dequant thread and stage
+  constexpr int kWords = BK * BITS / 32 / NH;     // packed words per dequant thread and stage
   constexpr int kChunks = kWords / 4;             // 16-byte chunks per dequant thread and stage
+  constexpr int kRegs = BK / 2 / NH;              // fp16 pairs per dequant thread and stage
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int S = a.stages;
@@ -105,8 +149,12 @@ w4a16_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int n0 = blockIdx.x * kTcRows;
-  const int KT = a.K / BK;
-  const int G = a.K / kGroup;
+  // this CTA's stages: [kt0, kt0 + KT) of the row's K / BK (split K: rank y
+  // of the cluster takes the y-th of ksplit consecutive ranges)
+  const int KT_all = a.K / BK;
+  const int kt0 = (int)(((int64_t)KT_all * blockIdx.y) / a.ksplit);
+  const int KT = (int)(((int64_t)KT_all * (blockIdx.y + 1)) / a.ksplit) - kt0;
+  const int G = a.K / GS;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
@@ -141,9 +189,10 @@ w4a16_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
         if (*abort_flag) break;
         if (u > 0 && !mbar_wait(&sempty[s], (u - 1) & 1, a.err, a.spin_limit)) { *abort_flag = 1; break; }
         mbar_arrive_expect_tx(&full[s], (uint32_t)stage_bytes);
+        const int kg = kt0 + kt;  // stage index along the whole row
 #pragma unroll
-        for (int i = 0; i < kXBoxes; ++i) tma_load_2d(stageX(s) + i * xbox, &tmX, kt * BK + 64 * i, 0, &full[s]);
-        tma_load_2d(stageP(s), &tmP, kt * (BK / 8), n0, &full[s]);
+        for (int i = 0; i < kXBoxes; ++i) tma_load_2d(stageX(s) + i * xbox, &tmX, kg * BK + 64 * i, 0, &full[s]);
+        tma_load_2d(stageP(s), &tmP, kg * (kRowBytes / 4), n0, &full[s]);
         issued = kt + 1;
         if (++s == S) { s = 0; ++u; }
       }
@@ -183,13 +232,17 @@ w4a16_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
     const int r = 32 * q + lane;        // output channel within the tile
     const int n = n0 + r;
     const bool row_ok = n < a.N;
-    // step and zero of the current group, and of the next one, fetched a
-    // group ahead of their use
-    __half st_cur = __float2half(0.f), zr_cur = __float2half(0.f);
-    __half st_next = __float2half(0.f), zr_next = __float2half(0.f);
-    if (row_ok) {
-      st_next = a.steps[(size_t)n * G];
-      zr_next = a.zeros[(size_t)n * G];
+    // step and zero of the current group(s), and of the next, fetched a
+    // group (or, for groups smaller than a stage, a stage) ahead of their use
+    __half st_cur[NGT], zr_cur[NGT], st_next[NGT], zr_next[NGT];
+    // first group of this thread's part of stage kt (small groups)
+    auto part_group = [&](int kt) { return ((kt0 + kt) * BK + h * (BK / NH)) / GS; };
+#pragma unroll
+    for (int i = 0; i < NGT; ++i) {
+      const int g0 = GS < BK ? part_group(0) + i : (kt0 * BK) / GS;
+      st_cur[i] = zr_cur[i] = __float2half(0.f);
+      st_next[i] = row_ok ? a.steps[(size_t)n * G + g0] : __float2half(0.f);
+      zr_next[i] = row_ok ? a.zeros[(size_t)n * G + g0] : __float2half(0.f);
     }
     // Software pipeline: stage kt is dequantized into registers while the
     // tensor-memory stores of stage kt-1 complete; then kt-1 is published to
@@ -198,40 +251,69 @@ w4a16_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
     int pend_b = -1;  // A buffer whose stores are in flight (-1: none)
     for (int kt = 0, s = 0, u = 0, b = 0, ub = 0; kt < KT; ++kt) {
       if (__any_sync(0xffffffffu, *abort_flag != 0)) break;
-      const int g = (kt * BK) / kGroup;
-      if ((kt * BK) % kGroup == 0) {  // a new group starts: take its prefetched scales, fetch the next
-        st_cur = st_next;
-        zr_cur = zr_next;
-        if (row_ok && g + 1 < G) {
-          st_next = a.steps[(size_t)n * G + g + 1];
-          zr_next = a.zeros[(size_t)n * G + g + 1];
+      if constexpr (GS < BK) {  // every stage: this part's groups, and the next stage's fetched
+#pragma unroll
+        for (int i = 0; i < NGT; ++i) {
+          st_cur[i] = st_next[i];
+          zr_cur[i] = zr_next[i];
+          const int gn = part_group(kt + 1) + i;
+          if (row_ok && kt + 1 < KT) {
+            st_next[i] = a.steps[(size_t)n * G + gn];
+            zr_next[i] = a.zeros[(size_t)n * G + gn];
+          }
+        }
+      } else {
+        const int g = ((kt0 + kt) * BK) / GS;
+        if (kt == 0 || ((kt0 + kt) * BK) % GS == 0) {  // a new group: take its prefetched scales, fetch the next
+          st_cur[0] = st_next[0];
+          zr_cur[0] = zr_next[0];
+          if (row_ok && g + 1 < G) {
+            st_next[0] = a.steps[(size_t)n * G + g + 1];
+            zr_next[0] = a.zeros[(size_t)n * G + g + 1];
+          }
         }
       }
-      const __half2 s2 = __halves2half2(st_cur, st_cur);
-      const __half z1024 = __hadd(zr_cur, __float2half(1024.f));
-      const __half z64n = __hneg(__hadd(zr_cur, __float2half(64.f)));
-      const __half2 zz = __halves2half2(z1024, z1024);
-      const __half2 zz16n = __halves2half2(z64n, z64n);
+      __half2 s2[NGT], zz[NGT], zz16n[NGT];
+#pragma unroll
+      for (int i = 0; i < NGT; ++i) {
+        s2[i] = __halves2half2(st_cur[i], st_cur[i]);
+        const __half z1024 = __hadd(zr_cur[i], __float2half(1024.f));
+        const __half z64n = __hneg(__hadd(zr_cur[i], __float2half(64.f)));
+        zz[i] = __halves2half2(z1024, z1024);
+        zz16n[i] = __halves2half2(z64n, z64n);
+      }
       const bool landed = mbar_wait(&full[s], u & 1, a.err, a.spin_limit);
       if (!__all_sync(0xffffffffu, landed)) { *abort_flag = 1; break; }
-      // The packed tile is swizzled by the TMA: with 64-byte rows (BK = 128)
-      // 16-byte chunk c of row r sits at chunk c ^ ((r >> 1) & 3), with
+      // The 4-bit packed tile is swizzled by the TMA: with 64-byte rows (BK =
+      // 128) 16-byte chunk c of row r sits at chunk c ^ ((r >> 1) & 3), with
       // 32-byte rows (BK = 64) at c ^ ((r >> 2) & 1); both keep a warp's loads
-      // conflict-free.
+      // conflict-free. 3-bit rows (48 bytes) are not swizzled.
       uint32_t words[kWords];
-      const uint8_t* prow = stageP(s) + r * (BK / 2);
-      const int sw = BK == 128 ? (r >> 1) & 3 : (r >> 2) & 1;
+      const uint8_t* prow = stageP(s) + r * kRowBytes;
+      const int sw = BITS == 3 ? 0 : BK == 128 ? (r >> 1) & 3 : (r >> 2) & 1;
 #pragma unroll
       for (int i = 0; i < kChunks; ++i) {
         const uint4 v = *reinterpret_cast<const uint4*>(prow + (((h * kChunks + i) ^ sw) << 4));
         words[4 * i] = v.x; words[4 * i + 1] = v.y; words[4 * i + 2] = v.z; words[4 * i + 3] = v.w;
       }
-      uint32_t nv[kWords / 4][16];
+      uint32_t nv[kRegs / 16][16];
+      if constexpr (BITS == 4) {
 #pragma unroll
-      for (int j = 0; j < kWords; ++j) {
-        const uint4 d = dequant_word4(words[j], zz, zz16n, s2);
-        nv[j >> 2][4 * (j & 3)] = d.x; nv[j >> 2][4 * (j & 3) + 1] = d.y;
-        nv[j >> 2][4 * (j & 3) + 2] = d.z; nv[j >> 2][4 * (j & 3) + 3] = d.w;
+        for (int j = 0; j < kWords; ++j) {
+          const int gi = 8 * j / (GS < BK ? GS : 8 * kWords);  // word j's group within the part
+          const uint4 d = dequant_word4(words[j], zz[gi], zz16n[gi], s2[gi]);
+          nv[j >> 2][4 * (j & 3)] = d.x; nv[j >> 2][4 * (j & 3) + 1] = d.y;
+          nv[j >> 2][4 * (j & 3) + 2] = d.z; nv[j >> 2][4 * (j & 3) + 3] = d.w;
+        }
+      } else {
+#pragma unroll
+        for (int c = 0; c < kRegs / 16; ++c) {  // 32 channels from three words
+          const int gi = 32 * c / (GS < BK ? GS : 32 * (kRegs / 16));
+          const __half z128n = __hneg(__hadd(zr_cur[gi], __float2half(128.f)));
+          const __half z16n = __hneg(__hadd(zr_cur[gi], __float2half(16.f)));
+          dequant_chunk3(&words[3 * c], zz[gi], __halves2half2(z128n, z128n), __halves2half2(z16n, z16n), s2[gi],
+                         nv[c]);
+        }
       }
       if (pend_b >= 0) {  // publish the previous stage
         tmem_st_wait();
@@ -243,7 +325,7 @@ w4a16_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
       if (!__all_sync(0xffffffffu, ok)) { *abort_flag = 1; break; }
       const uint32_t ta = tmem_a + ((uint32_t)(32 * q) << 16) + (uint32_t)(b * kACols + (kACols / NH) * h);
 #pragma unroll
-      for (int i = 0; i < kWords / 4; ++i) tmem_st16(ta + 16 * i, nv[i]);
+      for (int i = 0; i < kRegs / 16; ++i) tmem_st16(ta + 16 * i, nv[i]);
       pend_b = b;
       if (++s == S) { s = 0; ++u; }
       if (++b == NA) { b = 0; ++ub; }
@@ -257,7 +339,7 @@ w4a16_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
     // alternate 16-column chunks.
     bool done = !__any_sync(0xffffffffu, *abort_flag != 0);
     if (done) done = __all_sync(0xffffffffu, mbar_wait(accum, 0, a.err, a.spin_limit));
-    if (done) {
+    if (done && a.ksplit == 1) {
       tc_fence_after();
       for (int c0 = 16 * h; c0 < a.BN; c0 += 16 * NH) {
         uint32_t v[16];
@@ -271,198 +353,57 @@ w4a16_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
           }
         }
       }
-    } else {
+    } else if (!done) {
       *abort_flag = 1;
     }
   }
 
-  tc_fence_before();
-  __syncthreads();
-  if (warp == 1) {
-    tc_fence_after();
-    tmem_dealloc(tmem, a.tmem_cols);
-  }
-}
-
-// The same GEMM with the dequantized weight tile in shared memory: the
-// dequantizing warps store it (128-byte swizzled, K-major: the layout
-// desc_kmajor_sw128 describes) into a two-buffer ring and both MMA operands
-// come from shared memory; tensor memory holds only the accumulator. A
-// buffer is published with fence.proxy.async and an mbarrier arrival right
-// after its stores, where the tensor-memory A path must first wait for its
-// tcgen05.st to complete. One warp quartet dequantizes (each thread a row).
-template <int BK>
-__global__ void __launch_bounds__(192, 1)
-w4a16_gemm_tc_smem_a_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmP,
-                            TcArgs a) {
-  constexpr int NA = 2;                           // A buffers
-  constexpr int kPackedStage = kTcRows * BK / 2;  // bytes of the packed tile
-  constexpr int kABytes = kTcRows * BK * 2;       // one dequantized A tile
-  constexpr int kXBoxes = BK / 64;
-  constexpr int kWords = BK / 8;                  // packed words per thread (its row) and stage
-  constexpr int kChunks = kWords / 4;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  const int S = a.stages;
-  const int xbox = a.BN * 128;
-  const int stage_bytes = kXBoxes * xbox + kPackedStage;
-  uint8_t* abuf = smem + (size_t)S * stage_bytes;  // stage_bytes is a multiple of 1024
-  uint64_t* full = reinterpret_cast<uint64_t*>(abuf + NA * kABytes);
-  uint64_t* sempty = full + S;
-  uint64_t* afull = sempty + S;
-  uint64_t* aempty = afull + NA;
-  uint64_t* accum = aempty + NA;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accum + 1);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-
-  auto stageX = [&](int s) { return smem + (size_t)s * stage_bytes; };
-  auto stageP = [&](int s) { return smem + (size_t)s * stage_bytes + kXBoxes * xbox; };
-
-  const int warp = threadIdx.x >> 5;
-  const int lane = threadIdx.x & 31;
-  const int n0 = blockIdx.x * kTcRows;
-  const int KT = a.K / BK;
-  const int G = a.K / kGroup;
-
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < S; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&sempty[s], 1);
-    }
-    for (int b = 0; b < NA; ++b) {
-      mbar_init(&afull[b], 128);
-      mbar_init(&aempty[b], 1);
-    }
-    mbar_init(accum, 1);
-    *abort_flag = 0;
-    fence_mbar_init();
-  }
-  if (warp == 1) {
-    tmem_alloc(tmem_slot, a.tmem_cols);
-    tmem_relinquish();
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = *tmem_slot;
-
-  if (warp == 0) {
-    // ---------------------------------------------------------- TMA producer
-    if (lane == 0) {
-      prefetch_tensormap(&tmX);
-      prefetch_tensormap(&tmP);
-      int issued = 0;
-      for (int kt = 0, s = 0, u = 0; kt < (a.stall ? 0 : KT); ++kt) {  // s = kt % S, u = kt / S
-        if (*abort_flag) break;
-        if (u > 0 && !mbar_wait(&sempty[s], (u - 1) & 1, a.err, a.spin_limit)) { *abort_flag = 1; break; }
-        mbar_arrive_expect_tx(&full[s], (uint32_t)stage_bytes);
-#pragma unroll
-        for (int i = 0; i < kXBoxes; ++i) tma_load_2d(stageX(s) + i * xbox, &tmX, kt * BK + 64 * i, 0, &full[s]);
-        tma_load_2d(stageP(s), &tmP, kt * (BK / 8), n0, &full[s]);
-        issued = kt + 1;
-        if (++s == S) { s = 0; ++u; }
-      }
-      for (int kt = issued > S ? issued - S : 0; kt < issued; ++kt)
-        mbar_wait(&full[kt % S], (kt / S) & 1, a.err, a.spin_limit);
-    }
-  } else if (warp == 1) {
-    // ---------------------------------------------------------- MMA issuer
-    if (lane == 0) {
-      const uint32_t idesc = idesc_f16_f32(kTcRows, a.BN);
-      int committed = -1;
-      for (int kt = 0, s = 0, b = 0, ub = 0; kt < KT; ++kt) {
-        if (*abort_flag) break;
-        if (!mbar_wait(&afull[b], ub & 1, a.err, a.spin_limit)) { *abort_flag = 1; break; }
-        tc_fence_after();
-        const uint32_t xaddr = smem_u32(stageX(s));
-        const uint32_t aaddr = smem_u32(abuf + b * kABytes);
-#pragma unroll
-        for (int j = 0; j < BK / 16; ++j) {
-          const uint32_t koff = (uint32_t)((j >> 2) * (kTcRows * 128) + (j & 3) * 32);
-          const uint64_t ad = desc_kmajor_sw128(aaddr + koff);
-          const uint64_t bd = desc_kmajor_sw128(xaddr + (uint32_t)((j >> 2) * xbox + (j & 3) * 32));
-          mma_f16_ss(tmem, ad, bd, idesc, (kt > 0 || j > 0) ? 1u : 0u);
-        }
-        mma_commit(&aempty[b]);
-        mma_commit(&sempty[s]);
-        committed = kt;
-        if (++s == S) s = 0;
-        if (++b == NA) { b = 0; ++ub; }
-      }
-      mma_commit(accum);
-      if (*abort_flag && committed >= 0)  // let issued MMAs finish before teardown
-        mbar_wait(&aempty[committed % NA], (committed / NA) & 1, a.err, a.spin_limit);
-    }
-  } else {
-    // ---------------------------------------------------------- dequant + epilogue
-    const int q = warp & 3;             // TMEM lane quarter this warp may access
-    const int r = 32 * q + lane;        // output channel within the tile (the A row it writes)
+  if (a.ksplit > 1) {
+    // Split K: every CTA of the cluster is past its K loop (rank 0's ring is
+    // idle) before rank r > 0 writes its partial tile [row][m] (fp32) into
+    // slot r - 1 of rank 0's ring; after the second cluster barrier rank 0 adds
+    // them to its own accumulator in rank order. All threads of every CTA
+    // reach both barriers, on every path.
+    namespace cg = cooperative_groups;
+    cg::cluster_group cl = cg::this_cluster();
+    const unsigned rank = cl.block_rank();
+    const bool epi = warp >= 2 && warp < 2 + 4 * NH;
+    const int q = warp & 3, h = (warp - 2) >> 2;
+    const int r = 32 * q + (int)(threadIdx.x & 31);
     const int n = n0 + r;
-    const bool row_ok = n < a.N;
-    __half st_cur = __float2half(0.f), zr_cur = __float2half(0.f);
-    __half st_next = __float2half(0.f), zr_next = __float2half(0.f);
-    if (row_ok) {
-      st_next = a.steps[(size_t)n * G];
-      zr_next = a.zeros[(size_t)n * G];
-    }
-    for (int kt = 0, s = 0, u = 0, b = 0, ub = 0; kt < KT; ++kt) {
-      if (__any_sync(0xffffffffu, *abort_flag != 0)) break;
-      const int g = (kt * BK) / kGroup;
-      if ((kt * BK) % kGroup == 0) {  // a new group starts: take its prefetched scales, fetch the next
-        st_cur = st_next;
-        zr_cur = zr_next;
-        if (row_ok && g + 1 < G) {
-          st_next = a.steps[(size_t)n * G + g + 1];
-          zr_next = a.zeros[(size_t)n * G + g + 1];
-        }
-      }
-      const __half2 s2 = __halves2half2(st_cur, st_cur);
-      const __half z1024 = __hadd(zr_cur, __float2half(1024.f));
-      const __half z64n = __hneg(__hadd(zr_cur, __float2half(64.f)));
-      const __half2 zz = __halves2half2(z1024, z1024);
-      const __half2 zz16n = __halves2half2(z64n, z64n);
-      const bool landed = mbar_wait(&full[s], u & 1, a.err, a.spin_limit);
-      if (!__all_sync(0xffffffffu, landed)) { *abort_flag = 1; break; }
-      uint32_t words[kWords];
-      const uint8_t* prow = stageP(s) + r * (BK / 2);
-      const int sw = BK == 128 ? (r >> 1) & 3 : (r >> 2) & 1;  // the packed tile's TMA swizzle
-#pragma unroll
-      for (int i = 0; i < kChunks; ++i) {
-        const uint4 v = *reinterpret_cast<const uint4*>(prow + ((i ^ sw) << 4));
-        words[4 * i] = v.x; words[4 * i + 1] = v.y; words[4 * i + 2] = v.z; words[4 * i + 3] = v.w;
-      }
-      bool ok = true;
-      if (kt >= NA) ok = mbar_wait(&aempty[b], (ub - 1) & 1, a.err, a.spin_limit);
-      if (!__all_sync(0xffffffffu, ok)) { *abort_flag = 1; break; }
-      uint8_t* arow = abuf + b * kABytes;
-#pragma unroll
-      for (int j = 0; j < kWords; ++j)  // word j: channels 8j .. 8j + 7, one 16-byte chunk of the row
-        *reinterpret_cast<uint4*>(arow + (j >> 3) * (kTcRows * 128) + sw128_offset((uint32_t)r, (uint32_t)(j & 7))) =
-            dequant_word4(words[j], zz, zz16n, s2);
-      fence_proxy_async_smem();  // these generic writes -> the MMA's async-proxy reads
-      mbar_arrive(&afull[b]);
-      if (++s == S) { s = 0; ++u; }
-      if (++b == NA) { b = 0; ++ub; }
-    }
-    // Epilogue: D[n][m] from TMEM -> Y[m][n].
-    bool done = !__any_sync(0xffffffffu, *abort_flag != 0);
-    if (done) done = __all_sync(0xffffffffu, mbar_wait(accum, 0, a.err, a.spin_limit));
-    if (done) {
-      tc_fence_after();
-      for (int c0 = 0; c0 < a.BN; c0 += 16) {
+    tc_fence_before();
+    cl.sync();
+    tc_fence_after();
+    const bool ok = !*abort_flag;  // read after the barrier: one value per CTA
+    float* part = reinterpret_cast<float*>(smem);  // rank 0's ring: [ksplit - 1][128][BN]
+    if (epi && rank > 0 && ok) {
+      float* dst = cl.map_shared_rank(part, 0) + ((size_t)(rank - 1) * kTcRows + r) * a.BN;
+      for (int c0 = 16 * h; c0 < a.BN; c0 += 16 * NH) {
         uint32_t v[16];
         tmem_ld16(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)c0, v);
         tmem_ld_wait();
-        if (row_ok) {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) dst[c0 + i] = __uint_as_float(v[i]);
+      }
+    }
+    tc_fence_before();
+    cl.sync();
+    tc_fence_after();
+    if (epi && rank == 0 && ok) {
+      for (int c0 = 16 * h; c0 < a.BN; c0 += 16 * NH) {
+        uint32_t v[16];
+        tmem_ld16(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)c0, v);
+        tmem_ld_wait();
+        if (n < a.N) {
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
             const int m = c0 + i;
-            if (m < a.M) a.Y[(size_t)m * a.N + n] = __float2half_rn(__uint_as_float(v[i]));
+            float t = __uint_as_float(v[i]);
+            for (int k = 1; k < a.ksplit; ++k) t += part[((size_t)(k - 1) * kTcRows + r) * a.BN + m];
+            if (m < a.M) a.Y[(size_t)m * a.N + n] = __float2half_rn(t);
           }
         }
       }
-    } else {
-      *abort_flag = 1;
     }
   }
 
@@ -494,6 +435,17 @@ static EncodeTiledFn encode_fn() {
   return fn;
 }
 
+static int tc_num_sms() {
+  static int sms = 0;
+  if (sms == 0) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (sms <= 0) sms = 148;
+  }
+  return sms;
+}
+
 static uint32_t pow2_cols(uint32_t c) {
   uint32_t p = 32;
   while (p < c) p <<= 1;
@@ -504,12 +456,13 @@ static uint32_t pow2_cols(uint32_t c) {
 // CTAs per SM when that ring and the tile's TMEM fit half an SM).
 // bk_opt: 0 = library choice, else 64 or 128 input channels per stage.
 // dw_opt: 0 = library choice (4), else 4 or 8 dequantizing warps.
+// ksplit_opt: 0 = library choice, else 1, 2, 4 or 8 CTAs of a cluster along K.
 // wait_ms: how long a bounded mbarrier wait may last; stall: test hook (the
 // producer issues no loads, so the kernel's waits run out and it returns with
 // WQ_ERR_TIMEOUT latched).
 cudaError_t launch_gemm_tc(const void* X, const uint32_t* packed, const void* steps, const void* zeros, int64_t M,
-                           int64_t N, int64_t K, void* Y, int* err, cudaStream_t st, int stages_opt, int bk_opt,
-                           int dw_opt, int wait_ms, bool stall, bool a_smem) {
+                           int64_t N, int64_t K, int bits, int group, void* Y, int* err, cudaStream_t st,
+                           int stages_opt, int bk_opt, int dw_opt, int ksplit_opt, int wait_ms, bool stall) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return cudaErrorNotSupported;
   for (int64_t m0 = 0; m0 < M; m0 += 256) {
@@ -517,7 +470,9 @@ cudaError_t launch_gemm_tc(const void* X, const uint32_t* packed, const void* st
     const int BN = ((mc + 15) / 16) * 16;
     // Half-group stages for wide X tiles (BN >= 96: a 5-deep ring still fits
     // two CTAs per SM), whole-group stages otherwise (fewer waits per weight).
-    const int BK = bk_opt != 0 ? bk_opt : (BN >= 96 ? 64 : 128);
+    // 3-bit tiles always take 128-channel stages (a 64-channel row would be
+    // 24 bytes, not a whole number of 16-byte TMA units).
+    const int BK = bits == 3 ? 128 : bk_opt != 0 ? bk_opt : (BN >= 96 ? 64 : 128);
     CUtensorMap tmX, tmP;
     {
       cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)mc};
@@ -531,13 +486,17 @@ cudaError_t launch_gemm_tc(const void* X, const uint32_t* packed, const void* st
         return cudaErrorInvalidValue;
     }
     {
-      cuuint64_t dims[2] = {(cuuint64_t)(K / 8), (cuuint64_t)N};
-      cuuint64_t strides[1] = {(cuuint64_t)(K / 2)};
-      cuuint32_t box[2] = {(cuuint32_t)(BK / 8), 128};
+      // [N][K * bits / 32] words; a box is 128 rows of one stage's words
+      // (64 or 32 bytes, swizzled, for 4-bit; 48 bytes, unswizzled, for 3-bit)
+      cuuint64_t dims[2] = {(cuuint64_t)(K * bits / 32), (cuuint64_t)N};
+      cuuint64_t strides[1] = {(cuuint64_t)(K * bits / 8)};
+      cuuint32_t box[2] = {(cuuint32_t)(BK * bits / 32), 128};
       cuuint32_t es[2] = {1, 1};
+      const CUtensorMapSwizzle swz = bits == 3 ? CU_TENSOR_MAP_SWIZZLE_NONE
+                                     : BK == 128 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B;
       if (enc(&tmP, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<uint32_t*>(packed), dims, strides, box, es,
-              CU_TENSOR_MAP_INTERLEAVE_NONE, BK == 128 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B,
-              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+              CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
         return cudaErrorInvalidValue;
     }
     TcArgs a;
@@ -551,43 +510,13 @@ cudaError_t launch_gemm_tc(const void* X, const uint32_t* packed, const void* st
     a.err = err;
     a.spin_limit = (long long)wait_ms * 2000000LL;  // cycles at <= 2 GHz: at least wait_ms
     a.stall = stall ? 1 : 0;
-    if (a_smem) {  // A tiles in shared memory (two buffers); TMEM holds only the accumulator
-      a.tmem_cols = pow2_cols((uint32_t)BN);
-      const int stage = (BK / 64) * BN * 128 + kTcRows * BK / 2;
-      const size_t abytes = 2 * (size_t)kTcRows * BK * 2;
-      auto share = [](int c) { return (size_t)(225 * 1024) / (size_t)c - 3 * 1024; };
-      int cps = 512 / (int)a.tmem_cols;
-      if (cps > 4) cps = 4;
-      int S;
-      if (stages_opt > 0) {
-        S = stages_opt;
-        while (cps > 1 && (size_t)S * stage + abytes + 2048 > share(cps)) cps /= 2;
-        if ((size_t)S * stage + abytes + 2048 > share(1)) return cudaErrorInvalidValue;
-      } else {
-        while (cps > 1 && 3 * (size_t)stage + abytes + 2048 > share(cps)) cps /= 2;
-        S = (int)((share(cps) - abytes - 2048) / stage);
-        if (S > 16) S = 16;
-        if (S < 2) S = 2;
-      }
-      a.stages = S;
-      size_t smem = 1024 + (size_t)S * stage + abytes + (2 * S + 2 * 2 + 1) * 8 + 16;
-      const size_t smem_floor = (size_t)(228 * 1024) / (size_t)(cps + 1) + 1024;
-      if (smem < smem_floor) smem = smem_floor;
-      auto kern = BK == 128 ? w4a16_gemm_tc_smem_a_kernel<128> : w4a16_gemm_tc_smem_a_kernel<64>;
-      cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-      if (e != cudaSuccess) return e;
-      kern<<<dim3((unsigned)((N + kTcRows - 1) / kTcRows)), 192, smem, st>>>(tmX, tmP, a);
-      e = cudaGetLastError();
-      if (e != cudaSuccess) return e;
-      continue;
-    }
     // A third A buffer when it still fits the same TMEM allocation
     const int NA = pow2_cols((uint32_t)(BN + 3 * BK / 2)) == pow2_cols((uint32_t)(BN + 2 * BK / 2)) ? 3 : 2;
     a.tmem_cols = pow2_cols((uint32_t)(BN + NA * BK / 2));
     // CTAs per SM: as many as the 512 TMEM columns hold (1, 2 or 4), fewer
     // while their share of shared memory cannot hold a ring of three stages.
     // The ring then takes that share (at most 16 stages).
-    const int stage = (BK / 64) * BN * 128 + kTcRows * BK / 2;
+    const int stage = (BK / 64) * BN * 128 + kTcRows * BK * bits / 8;
     auto share = [](int c) { return (size_t)(225 * 1024) / (size_t)c - 3 * 1024; };
     int cps = 512 / (int)a.tmem_cols;
     int S;
@@ -607,22 +536,63 @@ cudaError_t launch_gemm_tc(const void* X, const uint32_t* packed, const void* st
     // 1/(cps+1) of the SM's shared memory.
     const size_t smem_floor = (size_t)(228 * 1024) / (size_t)(cps + 1) + 1024;
     if (smem < smem_floor) smem = smem_floor;
-    const int NH = dw_opt == 8 ? 2 : 1;  // 4 dequantizing warps unless asked for 8
-    auto pick = [&](auto bk, auto nh) {
-      constexpr int B = decltype(bk)::value, H = decltype(nh)::value;
-      return NA == 3 ? w4a16_gemm_tc_kernel<B, H, 3> : w4a16_gemm_tc_kernel<B, H, 2>;
-    };
-    using I64 = std::integral_constant<int, 64>;
-    using I128 = std::integral_constant<int, 128>;
+    // 4 dequantizing warps unless asked for 8 (4-bit, 128-channel groups only)
+    const int NH = dw_opt == 8 && bits == 4 && group == kGroup ? 2 : 1;
     using I1 = std::integral_constant<int, 1>;
     using I2 = std::integral_constant<int, 2>;
-    auto kern = BK == 128 ? (NH == 1 ? pick(I128{}, I1{}) : pick(I128{}, I2{}))
-                          : (NH == 1 ? pick(I64{}, I1{}) : pick(I64{}, I2{}));
+    using I32 = std::integral_constant<int, 32>;
+    using I64 = std::integral_constant<int, 64>;
+    using I128 = std::integral_constant<int, 128>;
+    auto pick = [&](auto bits_c, auto bk, auto nh, auto gs) {
+      constexpr int B = decltype(bits_c)::value, K_ = decltype(bk)::value, H = decltype(nh)::value,
+                    S_ = decltype(gs)::value;
+      return NA == 3 ? w4a16_gemm_tc_kernel<B, K_, H, 3, S_> : w4a16_gemm_tc_kernel<B, K_, H, 2, S_>;
+    };
+    using B3 = std::integral_constant<int, 3>;
+    using B4 = std::integral_constant<int, 4>;
+    decltype(pick(B4{}, I128{}, I1{}, I128{})) kern;
+    if (bits == 3)
+      kern = group == 32 ? pick(B3{}, I128{}, I1{}, I32{}) : group == 64 ? pick(B3{}, I128{}, I1{}, I64{})
+                                                                         : pick(B3{}, I128{}, I1{}, I128{});
+    else if (group == 32)
+      kern = BK == 128 ? pick(B4{}, I128{}, I1{}, I32{}) : pick(B4{}, I64{}, I1{}, I32{});
+    else if (group == 64)
+      kern = BK == 128 ? pick(B4{}, I128{}, I1{}, I64{}) : pick(B4{}, I64{}, I1{}, I64{});
+    else
+      kern = BK == 128 ? (NH == 1 ? pick(B4{}, I128{}, I1{}, I128{}) : pick(B4{}, I128{}, I2{}, I128{}))
+                       : (NH == 1 ? pick(B4{}, I64{}, I1{}, I128{}) : pick(B4{}, I64{}, I2{}, I128{}));
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    const dim3 grid((unsigned)((N + kTcRows - 1) / kTcRows));
-    kern<<<grid, 64 + 128 * NH, smem, st>>>(tmX, tmP, a);
-    e = cudaGetLastError();
+    // Split K over a cluster while the row tiles leave resident CTA slots
+    // idle: double it while twice the CTAs still fit the resident slots,
+    // every CTA keeps at least 4 stages, and rank 0's ring holds the other
+    // ranks' fp32 partial tiles.
+    const int tiles = (int)((N + kTcRows - 1) / kTcRows);
+    const int KT_all = (int)(K / BK);
+    const size_t ring = (size_t)S * stage, part = (size_t)kTcRows * BN * 4;
+    int ks = 1;
+    if (ksplit_opt > 0) {
+      ks = ksplit_opt;
+      if ((size_t)(ks - 1) * part > ring || KT_all < ks) return cudaErrorInvalidValue;
+    } else {
+      const long slots = (long)cps * tc_num_sms();
+      while (ks < 8 && (long)tiles * ks * 2 <= slots && KT_all / (ks * 2) >= 4 && (size_t)(2 * ks - 1) * part <= ring)
+        ks *= 2;
+    }
+    a.ksplit = ks;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)tiles, (unsigned)ks, 1);
+    cfg.blockDim = dim3(64 + 128 * NH, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 1;
+    attr[0].val.clusterDim.y = (unsigned)ks;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = ks > 1 ? 1 : 0;
+    e = cudaLaunchKernelEx(&cfg, kern, tmX, tmP, a);
     if (e != cudaSuccess) return e;
   }
   return cudaSuccess;

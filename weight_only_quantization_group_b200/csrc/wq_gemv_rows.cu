@@ -134,17 +134,18 @@ __device__ __forceinline__ void load_lane_x(uint32_t (&xh)[M][16 * CPL], const R
 }
 
 // ---------------------------------------------------------------- ActHalf
-// Group totals of a lane's offset term c1 and activation sum: the LPG = 4/CPL
-// lanes of one quantization group share step and zero, so the zero point and
-// the offsets are removed once per group (group-first reduction).
-template <int M, int CPL>
+// Group totals of a lane's offset term c1 and activation sum: the LPG lanes
+// of one quantization group (group size / channels per lane) share step and
+// zero, so the zero point and the offsets are removed once per group
+// (group-first reduction).
+template <int M, int LPG>
 __device__ __forceinline__ void group_totals(const float (&c1)[M], const float (&xsum)[M], float (&c1g)[M],
                                              float (&xg)[M]) {
 #pragma unroll
   for (int m = 0; m < M; ++m) {
     float c = c1[m], x = xsum[m];
 #pragma unroll
-    for (int o = 1; o < 4 / CPL; o <<= 1) {
+    for (int o = 1; o < LPG; o <<= 1) {
       c += __shfl_xor_sync(0xffffffffu, c, o);
       x += __shfl_xor_sync(0xffffffffu, x, o);
     }
@@ -168,6 +169,7 @@ struct ActHalf {
   uint32_t xh[M][16 * CPL];
   float c1g[M], xg[M];
 
+  template <int LPG>
   __device__ __forceinline__ void load(const RowsArgs& a, int k0, bool active) {
     load_lane_x<M, CPL>(xh, a, k0, active);
     float c1[M], xsum[M];
@@ -183,7 +185,7 @@ struct ActHalf {
       c1[m] = 1024.f * x1 + 64.f * x2;
       xsum[m] = x1 + x2;
     }
-    group_totals<M, CPL>(c1, xsum, c1g, xg);
+    group_totals<M, LPG>(c1, xsum, c1g, xg);
   }
 
   __device__ __forceinline__ float epilogue(int m, float t, __half sc, __half zh) const {
@@ -240,6 +242,7 @@ struct ActHalf3 {
     return group_epilogue<M>(c1g, xg, m, t, sc, zh);
   }
 
+  template <int LPG>
   __device__ __forceinline__ void load(const RowsArgs& a, int k0, bool active) {
     load_lane_x<M, CPL>(xh, a, k0, active);
     float c1[M], xsum[M];
@@ -258,7 +261,7 @@ struct ActHalf3 {
       c1[m] = 1024.f * x1 + 128.f * x8 + 16.f * x64;
       xsum[m] = x1 + x8 + x64;
     }
-    group_totals<M, CPL>(c1, xsum, c1g, xg);
+    group_totals<M, LPG>(c1, xsum, c1g, xg);
   }
 
   // acc[r*M + m] = this lane's A1 + A8/8 + A64/64, before the offsets, the
@@ -335,6 +338,7 @@ struct ActInt {
   int d16[M][3];  // 16 * sum over the lane's channels of digit t
   float inv[M];   // 2^-(F + 4): undoes the image scale and the 16 of the masked codes
 
+  template <int LPG>
   __device__ __forceinline__ void load(const RowsArgs& a, int k0, bool active) {
     uint32_t xh[M][16 * CPL];
     load_lane_x<M, CPL>(xh, a, k0, active);
@@ -505,7 +509,7 @@ __device__ __forceinline__ float group_first_reduce(float (&v)[NV], int lane, in
 // for the M = 1, 32-channel, two-stage instance, 2 (128 registers) for the
 // other M = 1 instances (each measured faster, more CTAs per SM), 1 for M = 2
 // (a cap would spill).
-template <int M, int R, int CPL, int S, int BITS, template <int, int> class Act, int MINB = 1>
+template <int M, int R, int CPL, int S, int BITS, template <int, int> class Act, int MINB = 1, int GS = kGroup>
 __global__ void __launch_bounds__(256, MINB)
 gemv_rows_kernel(RowsArgs a) {
   constexpr int WPR = BITS * CPL;  // packed words per row and lane
@@ -517,10 +521,11 @@ gemv_rows_kernel(RowsArgs a) {
   const int nseg = blockDim.x >> 5;
   const int k0 = warp * 32 * LK + lane * LK;  // this lane's first input channel
   const bool active = k0 < a.K;
-  const int G = a.K / kGroup;
+  static_assert(GS >= 32 * CPL, "a lane's channels lie in one group");
+  const int G = a.K / GS;
   const size_t row_words = (size_t)a.K * BITS / 32;
   const int lane_word = k0 * BITS / 32;
-  const int lane_group = k0 / kGroup;
+  const int lane_group = k0 / GS;
   const int nbatch = (a.N + R - 1) / R;
   const int my = blockIdx.x < nbatch ? (nbatch - 1 - blockIdx.x) / gridDim.x + 1 : 0;
 
@@ -528,7 +533,7 @@ gemv_rows_kernel(RowsArgs a) {
   // finishes the values gidx .. gidx + CG - 1 of each batch, so it loads the
   // step and zero of their RL rows only.
   constexpr bool GF = Act<M, CPL>::kGroupFirst;
-  constexpr int LPG = 4 / CPL;  // lanes of one quantization group
+  constexpr int LPG = GS / LK;  // lanes of one quantization group
   constexpr int CG = GF ? (NV / LPG > 1 ? NV / LPG : 1) : NV;
   constexpr int RL = GF ? (CG / M > 1 ? CG / M : 1) : R;
   const int gidx = GF ? group_first_index<NV, LPG>(lane) : 0;
@@ -550,7 +555,7 @@ gemv_rows_kernel(RowsArgs a) {
   asm volatile("griddepcontrol.wait;" ::: "memory");
 
   Act<M, CPL> act;
-  act.load(a, k0, active);
+  act.template load<LPG>(a, k0, active);
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
   // Cross-warp reduction once per NB batches: each batch's per-warp totals go
@@ -577,10 +582,11 @@ gemv_rows_kernel(RowsArgs a) {
     int idx;
     float v;
     if constexpr (GF) {
+      // value gidx + i: batch row lrow0 + i / M, activation row i % M (gidx is
+      // a multiple of M), so the step and zero are this lane's row i / M
       v = group_first_reduce<NV, LPG>(acc, lane, idx, [&](int i, float t) {
-        const int gi = gidx + i;        // value index: batch row gi / M, activation row gi % M
-        const int rr = gi / M - lrow0;  // which of this lane's RL step/zero rows
-        return act.epilogue(gi % M, t, rr == 0 ? sg.sc[0] : sg.sc[RL - 1], rr == 0 ? sg.zh[0] : sg.zh[RL - 1]);
+        const int rr = i / M < RL ? i / M : RL - 1;  // i < NV / LPG = RL * M wherever it is called
+        return act.epilogue(i % M, t, sg.sc[rr], sg.zh[rr]);
       });
     } else {
       v = butterfly_reduce<NV>(acc, lane, idx);
@@ -615,7 +621,6 @@ static int rows_num_sms() {
   return sms;
 }
 
-bool gemv_rows_supported(int bits, int64_t M, int64_t K) { return (bits == 4 || bits == 3) && M <= 2 && K <= 16384; }
 
 // Persistent grid, all CTAs resident; CTA c takes row batches c, c + grid, ...
 //   mode 0: small problems take one CTA per row batch (most loads in flight
@@ -629,10 +634,10 @@ static long rows_grid(long nbatch, int occ, int mode) {
   return (nbatch + per_cta - 1) / per_cta;
 }
 
-template <int M, int R, int CPL, int S, int BITS, template <int, int> class Act>
+template <int M, int R, int CPL, int S, int BITS, template <int, int> class Act, int GS>
 static cudaError_t launch_rows(const RowsArgs& a, cudaStream_t st, bool pdl, int grid_mode) {
   const int nseg = (a.K + 1024 * CPL - 1) / (1024 * CPL);
-  auto kern = gemv_rows_kernel<M, R, CPL, S, BITS, Act, M == 1 ? (CPL == 1 && S == 2 ? 3 : 2) : 1>;
+  auto kern = gemv_rows_kernel<M, R, CPL, S, BITS, Act, M == 1 ? (CPL == 1 && S == 2 ? 3 : 2) : 1, GS>;
   const int threads = 32 * nseg;
   const size_t smem = 2 * (size_t)32 * nseg * sizeof(float);  // [2][32/NV][nseg][NV]
   int occ = 0;
@@ -653,38 +658,50 @@ static cudaError_t launch_rows(const RowsArgs& a, cudaStream_t st, bool pdl, int
   return cudaLaunchKernelEx(&cfg, kern, a);
 }
 
-template <int M, int R, int CPL, int S>
+template <int M, int R, int CPL, int S, int GS>
 static cudaError_t launch_rows_act(const RowsArgs& a, cudaStream_t st, bool pdl, bool act_int, int grid_mode) {
-  return act_int ? launch_rows<M, R, CPL, S, 4, ActInt>(a, st, pdl, grid_mode)
-                 : launch_rows<M, R, CPL, S, 4, ActHalf>(a, st, pdl, grid_mode);
+  return act_int ? launch_rows<M, R, CPL, S, 4, ActInt, GS>(a, st, pdl, grid_mode)
+                 : launch_rows<M, R, CPL, S, 4, ActHalf, GS>(a, st, pdl, grid_mode);
 }
 
 // shape: rows per batch R, input channels per lane 32*CPL, register stages S
 //   0 = default (see launch_gemv_rows), 1 = (4, 32, 2), 2 = (4, 64, 2), 3 = (2, 64, 2), 4 = (4, 32, 3).
 // Shapes with 32 channels per lane take K <= 8192; above that shape 2 runs.
 // act_int: integer digits (true) or fp16 FMA (false) for the lane's dot products.
-template <int M>
+// Groups of 32 channels take the 32-channel shapes only (a lane's channels
+// must lie in one group).
+template <int M, int GS>
 static cudaError_t launch_rows_shape(const RowsArgs& a, cudaStream_t st, bool pdl, bool act_int, int shape,
                                      int gm) {
-  switch (shape) {
-    case 1: return launch_rows_act<M, 4, 1, 2>(a, st, pdl, act_int, gm);
-    case 3: return launch_rows_act<M, 2, 2, 2>(a, st, pdl, act_int, gm);
-    case 4: return launch_rows_act<M, 4, 1, 3>(a, st, pdl, act_int, gm);
-    default: return launch_rows_act<M, 4, 2, 2>(a, st, pdl, act_int, gm);
+  if constexpr (GS == 32) {
+    return shape == 4 ? launch_rows_act<M, 4, 1, 3, GS>(a, st, pdl, act_int, gm)
+                      : launch_rows_act<M, 4, 1, 2, GS>(a, st, pdl, act_int, gm);
+  } else {
+    switch (shape) {
+      case 1: return launch_rows_act<M, 4, 1, 2, GS>(a, st, pdl, act_int, gm);
+      case 3: return launch_rows_act<M, 2, 2, 2, GS>(a, st, pdl, act_int, gm);
+      case 4: return launch_rows_act<M, 4, 1, 3, GS>(a, st, pdl, act_int, gm);
+      default: return launch_rows_act<M, 4, 2, 2, GS>(a, st, pdl, act_int, gm);
+    }
   }
 }
 
 // 3-bit rows: 64 channels per lane (six words, three 8-byte loads), shape 2
-// or 3, offset sums only.
-template <int M>
+// or 3, offset sums only; groups of 64 or 128 channels.
+template <int M, int GS>
 static cudaError_t launch_rows3(const RowsArgs& a, cudaStream_t st, bool pdl, int shape, int gm) {
-  return shape == 3 ? launch_rows<M, 2, 2, 2, 3, ActHalf3>(a, st, pdl, gm)
-                    : launch_rows<M, 4, 2, 2, 3, ActHalf3>(a, st, pdl, gm);
+  return shape == 3 ? launch_rows<M, 2, 2, 2, 3, ActHalf3, GS>(a, st, pdl, gm)
+                    : launch_rows<M, 4, 2, 2, 3, ActHalf3, GS>(a, st, pdl, gm);
+}
+
+bool gemv_rows_supported(int bits, int group, int64_t M, int64_t K) {
+  if (!((bits == 4 || bits == 3) && M <= 2 && K <= 16384)) return false;
+  return group == kGroup || group == 64 || (group == 32 && bits == 4 && K <= 8192);
 }
 
 cudaError_t launch_gemv_rows(const void* X, const uint32_t* packed, const void* steps, const void* zeros, int64_t M,
-                             int64_t N, int64_t K, int bits, void* Y, cudaStream_t st, int shape, bool act_int,
-                             int grid_mode, bool pdl) {
+                             int64_t N, int64_t K, int bits, int group, void* Y, cudaStream_t st, int shape,
+                             bool act_int, int grid_mode, bool pdl) {
   RowsArgs a;
   a.X = static_cast<const __half*>(X);
   a.P = packed;
@@ -693,8 +710,12 @@ cudaError_t launch_gemv_rows(const void* X, const uint32_t* packed, const void* 
   a.Y = static_cast<__half*>(Y);
   a.N = (int)N;
   a.K = (int)K;
-  if (bits == 3)
-    return M == 1 ? launch_rows3<1>(a, st, pdl, shape, grid_mode) : launch_rows3<2>(a, st, pdl, shape, grid_mode);
+  if (bits == 3) {
+    if (group == 64)
+      return M == 1 ? launch_rows3<1, 64>(a, st, pdl, shape, grid_mode) : launch_rows3<2, 64>(a, st, pdl, shape, grid_mode);
+    return M == 1 ? launch_rows3<1, kGroup>(a, st, pdl, shape, grid_mode)
+                  : launch_rows3<2, kGroup>(a, st, pdl, shape, grid_mode);
+  }
   // measured fastest: at M = 1, (4, 32, 2) under an 85-register cap for
   // 4096-channel rows and for 8192-channel rows of at most 2^27 weights (more
   // CTAs per SM), else (4, 64, 2) (fewer cross-warp sums per weight); at
@@ -704,8 +725,14 @@ cudaError_t launch_gemv_rows(const void* X, const uint32_t* packed, const void* 
     else shape = K <= 4096 ? 4 : 2;
   }
   if (K > 8192 && (shape == 1 || shape == 4)) shape = 2;  // at most 8 warps
-  return M == 1 ? launch_rows_shape<1>(a, st, pdl, act_int, shape, grid_mode)
-                : launch_rows_shape<2>(a, st, pdl, act_int, shape, grid_mode);
+  if (group == 32)
+    return M == 1 ? launch_rows_shape<1, 32>(a, st, pdl, act_int, shape, grid_mode)
+                  : launch_rows_shape<2, 32>(a, st, pdl, act_int, shape, grid_mode);
+  if (group == 64)
+    return M == 1 ? launch_rows_shape<1, 64>(a, st, pdl, act_int, shape, grid_mode)
+                  : launch_rows_shape<2, 64>(a, st, pdl, act_int, shape, grid_mode);
+  return M == 1 ? launch_rows_shape<1, kGroup>(a, st, pdl, act_int, shape, grid_mode)
+                : launch_rows_shape<2, kGroup>(a, st, pdl, act_int, shape, grid_mode);
 }
 
 }  // namespace wq

@@ -8,20 +8,20 @@
 #include <stdint.h>
 
 namespace wq {
-cudaError_t launch_quantize_pack(const void* W, const void* s, int64_t N, int64_t K, int bits, bool sym,
+cudaError_t launch_quantize_pack(const void* W, const void* s, int64_t N, int64_t K, int bits, int group, bool sym,
                                  uint32_t* packed, void* steps, void* zeros, int* err, cudaStream_t st);
 cudaError_t launch_unpack_dequant(const uint32_t* packed, const void* steps, const void* zeros, int64_t N,
-                                  int64_t K, int bits, void* out, cudaStream_t st);
+                                  int64_t K, int bits, int group, void* out, cudaStream_t st);
 cudaError_t launch_gemv(const void* X, const uint32_t* packed, const void* steps, const void* zeros, int64_t M,
                         int64_t N, int64_t K, int bits, void* Y, cudaStream_t st, int variant, bool pdl);
 size_t gemv_smem_bytes(int bits, int variant, int M, int N, int K);
-bool gemv_rows_supported(int bits, int64_t M, int64_t K);
+bool gemv_rows_supported(int bits, int group, int64_t M, int64_t K);
 cudaError_t launch_gemv_rows(const void* X, const uint32_t* packed, const void* steps, const void* zeros, int64_t M,
-                             int64_t N, int64_t K, int bits, void* Y, cudaStream_t st, int shape, bool act_int,
-                             int grid_mode, bool pdl);
+                             int64_t N, int64_t K, int bits, int group, void* Y, cudaStream_t st, int shape,
+                             bool act_int, int grid_mode, bool pdl);
 cudaError_t launch_gemm_tc(const void* X, const uint32_t* packed, const void* steps, const void* zeros, int64_t M,
-                           int64_t N, int64_t K, void* Y, int* err, cudaStream_t st, int stages_opt, int bk_opt,
-                           int dw_opt, int wait_ms, bool stall, bool a_smem);
+                           int64_t N, int64_t K, int bits, int group, void* Y, int* err, cudaStream_t st,
+                           int stages_opt, int bk_opt, int dw_opt, int ksplit_opt, int wait_ms, bool stall);
 // Workspace layout of the AWQ search (wq_awq.cu): mu, the candidate scales,
 // the per-tile partial losses, and (two-kernel loss path only) the error
 // matrices of one batch of alphas.
@@ -44,5 +44,13 @@ cudaError_t launch_awq_search_noalloc(const void* X, int64_t T, int64_t K, const
                                       int* err, bool fused, cudaStream_t st);
 // AWQ scale folding (wq_fold.cu): out = in / s along rows (s[R]) or columns (s[C]).
 cudaError_t launch_fold(const void* in, const void* s, void* out, int64_t R, int64_t C, bool row_axis, int* err,
+                        cudaStream_t st);
+// GPTQ (wq_gptq.cu): workspace layout and the launch sequence.
+struct GptqPlan {
+  size_t off_H, off_G, off_W, off_Err, off_dead, total;
+};
+GptqPlan plan_gptq(int64_t N, int64_t K);
+cudaError_t launch_gptq(const void* X, int64_t T, const void* W, int64_t N, int64_t K, int bits, int group, bool sym,
+                        double damp, uint32_t* packed, void* steps, void* zeros, void* workspace, int* err,
                         cudaStream_t st);
 }  // namespace wq

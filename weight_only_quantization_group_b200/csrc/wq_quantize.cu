@@ -17,6 +17,8 @@
 // the 1.5 * 2^23 addition (both on packed fp32 pairs, two channels per
 // instruction), and one integer multiply-add into the packed word.
 // 2 B/weight in, 0.5 (0.375) B/weight out.
+#include <type_traits>
+
 #include "wq_quant_core.cuh"
 #include "wq_launch.h"
 
@@ -36,10 +38,11 @@ __device__ __forceinline__ void pack_lane(F level, int zero, uint32_t (&o)[4]) {
   }
 }
 
-// One lane unit u: channels [32u, 32u + 32) of the row-major weight, a
-// quarter of group u / 4. The group's decision (shared by its 4 lanes), then
-// the lane's 32 codes, packed and stored. sk: the unit's 32 AWQ scales.
-template <int BITS, bool SYM, bool HAS_S>
+// One lane unit u: channels [32u, 32u + 32) of the row-major weight, 1/LPG of
+// group u / LPG (LPG = group size / 32 lanes per group: 4, 2 or 1). The
+// group's decision (shared by its LPG lanes), then the lane's 32 codes,
+// packed and stored. sk: the unit's 32 AWQ scales.
+template <int BITS, bool SYM, bool HAS_S, int LPG>
 __device__ __forceinline__ void quantize_unit(const uint4 (&raw)[4], const __half* __restrict__ sk, int64_t u,
                                               bool valid, uint32_t* __restrict__ packed,
                                               __half* __restrict__ steps, __half* __restrict__ zeros, int* err) {
@@ -59,14 +62,14 @@ __device__ __forceinline__ void quantize_unit(const uint4 (&raw)[4], const __hal
       ws[2 * i + 1] = 0.f;
       fma2_f16_f32(ws[2 * i], ws[2 * i + 1], (&raw[i >> 2].x)[i & 3], (&sr[i >> 2].x)[i & 3]);
     }
-    gq = group_quant_decide<BITS, SYM, 32, 4>(ws);
+    gq = group_quant_decide<BITS, SYM, 32, LPG>(ws);
   } else {
-    gq = group_quant_decide_h<BITS, SYM, 4>(raw);
+    gq = group_quant_decide_h<BITS, SYM, LPG>(raw);
   }
-  if (valid && (u & 3) == 0) {
+  if (valid && (u % LPG) == 0) {
     if (!isfinite(gq.sf)) latch_error(err, WQ_ERR_RANGE);
-    steps[u >> 2] = gq.step_h;
-    zeros[u >> 2] = __int2half_rn(gq.zero);
+    steps[u / LPG] = gq.step_h;
+    zeros[u / LPG] = __int2half_rn(gq.zero);
   }
   auto value = [&](int i) -> float {
     if constexpr (HAS_S) return ws[i]; else return lane_half(raw, i);
@@ -97,7 +100,7 @@ __device__ __forceinline__ void quantize_unit(const uint4 (&raw)[4], const __hal
   }
 }
 
-template <int BITS, bool SYM, bool HAS_S>
+template <int BITS, bool SYM, bool HAS_S, int LPG>
 __global__ void __launch_bounds__(256)
 quantize_pack_kernel(const __half* __restrict__ W, const __half* __restrict__ s, int64_t N, int64_t K,
                      uint32_t* __restrict__ packed, __half* __restrict__ steps,
@@ -132,15 +135,16 @@ quantize_pack_kernel(const __half* __restrict__ W, const __half* __restrict__ s,
       if (col >= kunits) col -= kunits;
     }
     load(next);
-    quantize_unit<BITS, SYM, HAS_S>(raw, sk, cur, cur < units, packed, steps, zeros, err);
+    quantize_unit<BITS, SYM, HAS_S, LPG>(raw, sk, cur, cur < units, packed, steps, zeros, err);
   }
 }
 
-// Inverse: one thread per 8 (4-bit) or 32 (3-bit) weights.
+// Inverse: one thread per 8 (4-bit) or 32 (3-bit) weights (never across a
+// group: groups are 32, 64 or 128 channels).
 template <int BITS>
 __global__ void __launch_bounds__(256)
 unpack_dequant_kernel(const uint32_t* __restrict__ packed, const __half* __restrict__ steps,
-                      const __half* __restrict__ zeros, int64_t N, int64_t K, __half* __restrict__ out) {
+                      const __half* __restrict__ zeros, int64_t N, int64_t K, int group, __half* __restrict__ out) {
   constexpr int PER = BITS == 4 ? 8 : 32;
   const int64_t units = N * K / PER;
   const int64_t u = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
@@ -148,7 +152,7 @@ unpack_dequant_kernel(const uint32_t* __restrict__ packed, const __half* __restr
   const int64_t e0 = u * PER;  // first element (row-major)
   const int64_t n = e0 / K;
   const int64_t k = e0 % K;
-  const int64_t gidx = n * (K / kGroup) + k / kGroup;
+  const int64_t gidx = n * (K / group) + k / group;
   const float sf = __half2float(steps[gidx]);
   const float z = __half2float(zeros[gidx]);
   int q[PER];
@@ -181,9 +185,9 @@ unpack_dequant_kernel(const uint32_t* __restrict__ packed, const __half* __restr
   }
 }
 
-cudaError_t launch_quantize_pack(const void* W, const void* s, int64_t N, int64_t K, int bits, bool sym,
+cudaError_t launch_quantize_pack(const void* W, const void* s, int64_t N, int64_t K, int bits, int group, bool sym,
                                  uint32_t* packed, void* steps, void* zeros, int* err, cudaStream_t st) {
-  const int64_t units = N * (K / kGroup) * 4;  // 4 lanes per group
+  const int64_t units = N * K / 32;  // lane units of 32 channels
   const dim3 block(256);
   auto Wp = static_cast<const __half*>(W);
   auto sp = static_cast<const __half*>(s);
@@ -202,30 +206,39 @@ cudaError_t launch_quantize_pack(const void* W, const void* s, int64_t N, int64_
     const dim3 grid((unsigned)(need < resident ? need : resident));
     kern<<<grid, block, 0, st>>>(Wp, sp, N, K, packed, stp, zp, err);
   };
-#define WQ_QP(B, S, H) launch(quantize_pack_kernel<B, S, H>)
+  auto by_group = [&](auto bits_c, auto sym_c, auto s_c) {
+    constexpr int B = decltype(bits_c)::value;
+    constexpr bool S = decltype(sym_c)::value, H = decltype(s_c)::value;
+    if (group == 32) launch(quantize_pack_kernel<B, S, H, 1>);
+    else if (group == 64) launch(quantize_pack_kernel<B, S, H, 2>);
+    else launch(quantize_pack_kernel<B, S, H, 4>);
+  };
+  using T = std::true_type;
+  using F = std::false_type;
+  using B4 = std::integral_constant<int, 4>;
+  using B3 = std::integral_constant<int, 3>;
   if (bits == 4) {
-    if (sym) { if (s) WQ_QP(4, true, true); else WQ_QP(4, true, false); }
-    else     { if (s) WQ_QP(4, false, true); else WQ_QP(4, false, false); }
+    if (sym) { if (s) by_group(B4{}, T{}, T{}); else by_group(B4{}, T{}, F{}); }
+    else     { if (s) by_group(B4{}, F{}, T{}); else by_group(B4{}, F{}, F{}); }
   } else {
-    if (sym) { if (s) WQ_QP(3, true, true); else WQ_QP(3, true, false); }
-    else     { if (s) WQ_QP(3, false, true); else WQ_QP(3, false, false); }
+    if (sym) { if (s) by_group(B3{}, T{}, T{}); else by_group(B3{}, T{}, F{}); }
+    else     { if (s) by_group(B3{}, F{}, T{}); else by_group(B3{}, F{}, F{}); }
   }
-#undef WQ_QP
   return cudaGetLastError();
 }
 
 cudaError_t launch_unpack_dequant(const uint32_t* packed, const void* steps, const void* zeros, int64_t N,
-                                  int64_t K, int bits, void* out, cudaStream_t st) {
+                                  int64_t K, int bits, int group, void* out, cudaStream_t st) {
   const int per = bits == 4 ? 8 : 32;
   const int64_t units = N * K / per;
   const dim3 grid((unsigned)((units + 255) / 256));
   if (bits == 4)
     unpack_dequant_kernel<4><<<grid, 256, 0, st>>>(packed, static_cast<const __half*>(steps),
-                                                   static_cast<const __half*>(zeros), N, K,
+                                                   static_cast<const __half*>(zeros), N, K, group,
                                                    static_cast<__half*>(out));
   else
     unpack_dequant_kernel<3><<<grid, 256, 0, st>>>(packed, static_cast<const __half*>(steps),
-                                                   static_cast<const __half*>(zeros), N, K,
+                                                   static_cast<const __half*>(zeros), N, K, group,
                                                    static_cast<__half*>(out));
   return cudaGetLastError();
 }
