@@ -59,6 +59,8 @@ __all__ = [
     "awq_fold_into_linear_rows",
     "decoder_block_ref",
     "awq_fold_block",
+    "act_quantize_int8_groups",
+    "w4a8_gemm_ref",
     "gptq_hessian",
     "gptq_quantize",
     "GPTQ_DAMP",
@@ -568,3 +570,43 @@ def _code_of(w32: np.ndarray, step_h: np.ndarray, zero_h: np.ndarray, bits: int,
     Q = (1 << bits) - 1
     q = np.rint(w32 / sf).astype(np.int32) + zero_h.astype(np.int32)
     return np.clip(q, 0, Q).astype(np.uint8)
+
+
+# ---------------------------------------------------------------------------
+# W4A8: 4-bit weights and 8-bit activations, both per group of channels
+# ([MIT-Lab4/5] "The five implementation files and grading": the Lab 5 linear
+# is W4A8 with group size 32; the int8 absmax form of [CMU-L19/20] "absmax
+# and zero-point" applied to each group of activations)
+# ---------------------------------------------------------------------------
+
+def act_quantize_int8_groups(X16: np.ndarray, group: int = 32):
+    """Per row m and group g of ``group`` consecutive channels: multiplier
+    mult = 127 / max|x| (1 for an all-zero group), code = round(mult * x)
+    (ties to even), clipped to [-127, 127]. fp32 arithmetic on the fp16
+    inputs (one IEEE division, one multiply, rint), as on the GPU.
+    Returns (codes int8 [M][K], mult fp32 [M][K/group])."""
+    X = np.asarray(X16)
+    assert X.dtype == np.float16 and X.ndim == 2
+    M, K = X.shape
+    assert K % group == 0
+    x = X.astype(np.float32).reshape(M, K // group, group)
+    amax = np.abs(x).max(axis=2)
+    mult = np.where(amax == 0, np.float32(1.0), np.float32(127.0) / np.where(amax == 0, np.float32(1.0), amax))
+    mult = mult.astype(np.float32)
+    q = np.clip(np.rint(x * mult[:, :, None]), -127, 127).astype(np.int8)
+    return q.reshape(M, K), mult
+
+
+def w4a8_gemm_ref(qx: np.ndarray, mult: np.ndarray, codes: np.ndarray, steps: np.ndarray, zeros: np.ndarray,
+                  group: int) -> np.ndarray:
+    """Y[m][n] = sum_g (step[n][g] / mult[m][g]) * sum_{k in g} (q[n][k] - zero[n][g]) * qx[m][k]:
+    the integer dot product of each group, scaled by the weight's step and
+    the activation's 1/multiplier, summed over groups in fp64."""
+    M, K = qx.shape
+    N = codes.shape[0]
+    G = K // group
+    qw = codes.astype(np.int64).reshape(N, G, group) - zeros.astype(np.int64)[:, :, None]
+    qa = qx.astype(np.int64).reshape(M, G, group)
+    dots = np.einsum("mgk,ngk->mng", qa, qw)  # exact integers
+    scale = steps.astype(np.float64)[None, :, :] / mult.astype(np.float64)[:, None, :]
+    return np.sum(dots.astype(np.float64) * scale, axis=2)

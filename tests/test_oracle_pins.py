@@ -586,3 +586,58 @@ def test_gptq_beats_rtn_on_correlated_inputs():
 
     for bits in (3, 4):
         assert loss(*O.gptq_quantize(W, X, bits, 128, False)) < 0.8 * loss(*O.quantize_groups(W, bits, 128, False))
+
+
+# ---------------------------------------------------------------------------
+# W4A8 ("MIT 6.5940 Lab 4 + Lab 5", W4A8 with group size 32; int8 absmax of
+# "CMU 11-868 L19-L20", "absmax and zero-point")
+# ---------------------------------------------------------------------------
+
+def test_act_int8_groups_hand_values_and_bounds():
+    """The group's largest magnitude maps to +-127; ties round to even; an
+    all-zero group keeps multiplier 1; every value is within half a code step
+    of its dequantized code."""
+    x = np.zeros((1, 64), np.float16)
+    x[0, :4] = [2.0, -1.0, 0.5, 1.0 / 127.0 * 2.0]      # mult = 63.5: 127, -63.5 -> -64 (even), 31.75 -> 32
+    q, m = O.act_quantize_int8_groups(x, 32)
+    assert m[0, 0] == np.float32(63.5) and m[0, 1] == 1.0
+    assert list(q[0, :3]) == [127, -64, 32]
+    assert np.all(q[0, 32:] == 0)
+    g = np.random.default_rng(71)
+    X = (g.standard_normal((5, 256)) * np.exp(g.normal(0, 2, 256))).astype(np.float16)
+    q, m = O.act_quantize_int8_groups(X, 32)
+    back = q.astype(np.float64).reshape(5, 8, 32) / m.astype(np.float64)[:, :, None]
+    err = np.abs(back - X.astype(np.float64).reshape(5, 8, 32))
+    assert np.all(err <= (0.5 + 1e-6) / m.astype(np.float64)[:, :, None])
+    assert np.all(np.abs(q.reshape(5, 8, 32)).max(axis=2) == 127)
+
+
+def test_w4a8_ref_reduces_to_the_exact_matmul():
+    """With activations that are integers of magnitude <= 127 and a group
+    maximum of 127 (multiplier 1), quantizing them changes nothing, and the
+    W4A8 reference equals the fp64 matmul of the dequantized weight; the
+    integer group sums keep every product exact."""
+    g = np.random.default_rng(72)
+    K, N, M = 128, 20, 3
+    X = g.integers(-127, 128, (M, K)).astype(np.float16)
+    X[:, ::32] = 127
+    codes, st, z = O.quantize_groups((0.02 * g.standard_normal((N, K))).astype(np.float16), 4, 32, False)
+    qx, mult = O.act_quantize_int8_groups(X, 32)
+    assert np.all(mult == 1.0) and np.array_equal(qx.astype(np.float16), X)
+    assert np.allclose(O.w4a8_gemm_ref(qx, mult, codes, st, z, 32), O.gemm_ref(X, codes, st, z, 32),
+                       rtol=1e-14, atol=1e-12)
+
+
+def test_w4a8_ref_brute_force_loops():
+    g = np.random.default_rng(73)
+    K, N, M = 64, 3, 2
+    codes, st, z = O.quantize_groups((0.02 * g.standard_normal((N, K))).astype(np.float16), 4, 32, True)
+    qx, mult = O.act_quantize_int8_groups((g.standard_normal((M, K))).astype(np.float16), 32)
+    Y = O.w4a8_gemm_ref(qx, mult, codes, st, z, 32)
+    for m in range(M):
+        for n in range(N):
+            t = Fraction(0)
+            for gi in range(2):
+                dot = sum((int(codes[n, k]) - int(z[n, gi])) * int(qx[m, k]) for k in range(32 * gi, 32 * gi + 32))
+                t += Fraction(dot) * Fraction(float(st[n, gi])) / Fraction(float(mult[m, gi]))
+            assert abs(float(t) - Y[m, n]) <= 1e-12 * max(1.0, abs(float(t)))
