@@ -687,6 +687,24 @@ def measure_rows(wq, torch, synth, dev, block, peaks):
         "best_alpha": {g: int(o["best"].item()) / 20 for (g, _, _, _), o in zip(prepared, outs)}}
     del prepared, outs, packs
 
+    # GPTQ (fp64 Hessian, factorizations, column loop with error feedback)
+    # on LLaMA-2-7B-shaped linears with 512 calibration tokens, 4-bit g128
+    for name, N, K in (("q_proj", 4096, 4096), ("gate_proj", 11008, 4096)):
+        g0 = synth.rng(90)
+        Wg = dt(synth.weight(g0, N, K, 0.02))
+        Xg = dt(synth.activations(g0, 512, K, channel_frac=0.01, channel_mult=20.0))
+        wsg = torch.empty(wq.wq_gptq_workspace_bytes(N, K), dtype=torch.uint8, device=dev)
+        wq.wq_gptq_quantize_pack(Wg, Xg, workspace=wsg)
+        torch.cuda.synchronize()
+        a.record()
+        wq.wq_gptq_quantize_pack(Wg, Xg, workspace=wsg)
+        b.record()
+        torch.cuda.synchronize()
+        assert wq.wq_get_last_device_error() == 0
+        rows[f"gptq_llama7b_{name}_T512_w4"] = {"ms": a.elapsed_time(b), "N": N, "K": K,
+                                                "workspace_MB": wsg.numel() / 1e6}
+        del wsg
+
     # AWQ scale folding over the block: s_qkv into the first norm's weight,
     # s_o into v_proj's rows, s_gate_up into the second norm's weight,
     # s_down into up_proj's rows (fp16 in, fp16 out: 4 bytes per element)

@@ -205,6 +205,29 @@ int32_t wq_awq_scale_search_noalloc(const void* X_dev, int64_t T, int64_t K, con
                                     double* mu_out_dev, double* loss_out_dev, int32_t* best_out_dev,
                                     void* stream);
 
+/* W4A8 -- 4-bit weights and 8-bit activations, one scale per group of
+ * channels for each ("MIT 6.5940 Lab 4 + Lab 5", section "The five
+ * implementation files and grading": the Lab 5 linear is W4A8 with group size
+ * 32; the activation codes are the int8 absmax form of "CMU 11-868 L19-L20
+ * Model Quantization", section "absmax and zero-point", per group).
+ *   wq_quantize_act_int8  X_dev fp16 [M][K] -> q_dev int8 [M][K] and mult_dev
+ *       fp32 [M][K/group]: per row and group, mult = 127 / max|x| (fp32
+ *       division; 1 for an all-zero group), q = rint(x * mult) (fp32, ties to
+ *       even) clipped to [-127, 127]. group in {32, 64, 128}, K % group == 0.
+ *   wq_w4a8_gemm  Y[m][n] = sum_g (step[n][g] / mult[m][g]) *
+ *       sum_{k in g} (q_w[n][k] - zero[n][g]) * q[m][k]: exact integer dot
+ *       products per group (dp4a), scaled and summed in fp32, Y fp16 [M][N].
+ *       The weight is wq_quantize_pack's 4-bit layout with cfg->group_size
+ *       equal to the activations' group; K <= 16384 (else
+ *       WQ_ERR_UNSUPPORTED); q_dev 16-byte aligned.
+ * Asynchronous on `stream`, one launch each (wq_w4a8_gemm: one per 4 rows of
+ * M). */
+int32_t wq_quantize_act_int8(const void* X_dev, int64_t M, int64_t K, int32_t group, int8_t* q_dev,
+                             float* mult_dev, void* stream);
+int32_t wq_w4a8_gemm(const int8_t* q_dev, const float* mult_dev, const uint32_t* packed_dev,
+                     const void* steps_dev, const void* zeros_dev, int64_t M, int64_t N, int64_t K,
+                     const wq_quant_cfg* cfg, void* Y_dev, void* stream);
+
 /* GPTQ -- quantize + pack with error feedback ("CMU 11-868 L19-L20 Model
  * Quantization", sections "The algorithm in four steps" and "Why it can
  * actually run: from OBS to GPTQ"), writing the same packed layout, steps

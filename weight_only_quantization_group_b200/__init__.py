@@ -39,6 +39,8 @@ __all__ = [
     "wq_awq_fold_linear_rows",
     "wq_gptq_workspace_bytes",
     "wq_gptq_quantize_pack",
+    "wq_quantize_act_int8",
+    "wq_w4a8_gemm",
     "EXPORTED_SYMBOLS",
 ]
 
@@ -65,6 +67,8 @@ EXPORTED_SYMBOLS = (
     "wq_awq_fold_linear_rows",
     "wq_gptq_workspace_bytes",
     "wq_gptq_quantize_pack",
+    "wq_quantize_act_int8",
+    "wq_w4a8_gemm",
 )
 
 WQ_OK = 0
@@ -139,6 +143,8 @@ def _load() -> ctypes.CDLL:
                                               ctypes.POINTER(ctypes.c_double), i32, vp, vp, vp, vp, vp]),
         "wq_awq_fold_norm": (i32, [vp, vp, i64, vp, vp]),
         "wq_gptq_workspace_bytes": (sz, [i64, i64, cfgp]),
+        "wq_quantize_act_int8": (i32, [vp, i64, i64, i32, vp, vp, vp]),
+        "wq_w4a8_gemm": (i32, [vp, vp, vp, vp, vp, i64, i64, i64, cfgp, vp, vp]),
         "wq_gptq_quantize_pack": (i32, [vp, i64, vp, i64, i64, cfgp, ctypes.c_double, vp, vp, vp, vp, sz, vp]),
         "wq_awq_fold_linear_rows": (i32, [vp, vp, vp, i64, i64, vp, vp, vp]),
     }
@@ -588,3 +594,47 @@ def wq_gptq_quantize_pack(W: torch.Tensor, X: torch.Tensor, *, bits: int = 4, gr
                                         workspace.numel() * workspace.element_size(), _stream(stream, W.device.index))
     _raise(st, "wq_gptq_quantize_pack")
     return packed, steps, zeros
+
+
+def wq_quantize_act_int8(X: torch.Tensor, *, group_size: int = 32, out=None, stream=None):
+    """int8 codes and fp32 multipliers of fp16 activations X [M][K], one
+    multiplier per row and group; returns (q int8 [M][K], mult fp32 [M][K/group])."""
+    _check(X, torch.float16, "X")
+    if X.dim() != 2:
+        raise ValueError(f"X must be [M][K], got shape {tuple(X.shape)}")
+    M, K = X.shape
+    if out is None:
+        q = torch.empty((M, K), dtype=torch.int8, device=X.device)
+        mult = torch.empty((M, K // group_size if group_size > 0 else 0), dtype=torch.float32, device=X.device)
+    else:
+        q, mult = out
+        _need(q, "q", torch.int8, M * K)
+        _need(mult, "mult", torch.float32, 4 * M * (K // group_size))
+    _on_device_of(X, q=q, mult=mult)
+    with _device_of(X):
+        st = _lib.wq_quantize_act_int8(_ptr(X), M, K, group_size, _ptr(q), _ptr(mult), _stream(stream, X.device.index))
+    _raise(st, "wq_quantize_act_int8")
+    return q, mult
+
+
+def wq_w4a8_gemm(q: torch.Tensor, mult: torch.Tensor, packed: torch.Tensor, steps: torch.Tensor,
+                 zeros: torch.Tensor, N: int, *, group_size: int = 32, symmetric: bool = False, out=None,
+                 stream=None):
+    """Y [M][N] fp16 from int8 activation codes (wq_quantize_act_int8) and a
+    4-bit packed weight of the same group size."""
+    _check(q, torch.int8, "q")
+    if q.dim() != 2:
+        raise ValueError(f"q must be [M][K], got shape {tuple(q.shape)}")
+    M, K = q.shape
+    c = _cfg(4, group_size, symmetric)
+    _quant_operands(N, K, c, packed, steps, zeros)
+    _need(mult, "mult", torch.float32, 4 * M * (K // group_size))
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.float16, device=q.device)
+    _need(out, "out", torch.float16, 2 * M * N)
+    _on_device_of(q, mult=mult, packed=packed, steps=steps, zeros=zeros, out=out)
+    with _device_of(q):
+        st = _lib.wq_w4a8_gemm(_ptr(q), _ptr(mult), _ptr(packed), _ptr(steps), _ptr(zeros), M, N, K,
+                               ctypes.byref(c), _ptr(out), _stream(stream, q.device.index))
+    _raise(st, "wq_w4a8_gemm")
+    return out

@@ -255,6 +255,34 @@ int32_t wq_awq_scale_search_noalloc(const void* X, int64_t T, int64_t K, const v
                                                    static_cast<cudaStream_t>(stream)));
 }
 
+int32_t wq_quantize_act_int8(const void* X, int64_t M, int64_t K, int32_t group, int8_t* q, float* mult,
+                             void* stream) {
+  NvtxRange nvtx_range("wq_quantize_act_int8");
+  if (group != 32 && group != 64 && group != wq::kGroup) return WQ_ERR_INVALID_ARG;
+  if (M < 1 || K < group || K % group != 0 || M > (int64_t)INT32_MAX / 2 || K > (int64_t)INT32_MAX / 2)
+    return WQ_ERR_INVALID_ARG;
+  if (!X || !q || !mult) return WQ_ERR_INVALID_ARG;
+  if (!aligned(X, 2) || !aligned(q, 4) || !aligned(mult, 4)) return WQ_ERR_ALIGNMENT;
+  return cuda_status(wq::launch_act_int8(X, M, K, group, q, mult, static_cast<cudaStream_t>(stream)));
+}
+
+int32_t wq_w4a8_gemm(const int8_t* q, const float* mult, const uint32_t* packed, const void* steps, const void* zeros,
+                     int64_t M, int64_t N, int64_t K, const wq_quant_cfg* cfg, void* Y, void* stream) {
+  NvtxRange nvtx_range("wq_w4a8_gemm");
+  int32_t st = check_cfg(cfg);
+  if (st != WQ_OK) return st;
+  if (cfg->bits != 4) return WQ_ERR_UNSUPPORTED;
+  if ((st = check_shape(N, K)) != WQ_OK) return st;
+  if (M < 1 || M > (int64_t)INT32_MAX / 2) return WQ_ERR_INVALID_ARG;
+  if (K > 16384) return WQ_ERR_UNSUPPORTED;  // the activation codes of 4 rows in one CTA's shared memory
+  if (!q || !mult || !packed || !steps || !zeros || !Y) return WQ_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(mult, 4) || !aligned(packed, 16) || !aligned(steps, 2) || !aligned(zeros, 2) ||
+      !aligned(Y, 2))
+    return WQ_ERR_ALIGNMENT;
+  return cuda_status(wq::launch_w4a8_gemv(q, mult, packed, steps, zeros, M, N, K, cfg->group_size, Y,
+                                          static_cast<cudaStream_t>(stream)));
+}
+
 size_t wq_gptq_workspace_bytes(int64_t N, int64_t K, const wq_quant_cfg* cfg) {
   if (check_cfg(cfg) != WQ_OK || check_shape(N, K) != WQ_OK) return 0;
   return wq::plan_gptq(N, K).total;

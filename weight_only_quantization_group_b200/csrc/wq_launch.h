@@ -45,6 +45,12 @@ cudaError_t launch_awq_search_noalloc(const void* X, int64_t T, int64_t K, const
 // AWQ scale folding (wq_fold.cu): out = in / s along rows (s[R]) or columns (s[C]).
 cudaError_t launch_fold(const void* in, const void* s, void* out, int64_t R, int64_t C, bool row_axis, int* err,
                         cudaStream_t st);
+// W4A8 (wq_w4a8.cu): int8 activations per group, and the dp4a GEMV.
+cudaError_t launch_act_int8(const void* X, int64_t M, int64_t K, int group, int8_t* q, float* mult,
+                            cudaStream_t st);
+size_t w4a8_smem_bytes(int M, int64_t K);
+cudaError_t launch_w4a8_gemv(const int8_t* qx, const float* mult, const uint32_t* packed, const void* steps,
+                             const void* zeros, int64_t M, int64_t N, int64_t K, int group, void* Y, cudaStream_t st);
 // GPTQ (wq_gptq.cu): workspace layout and the launch sequence.
 struct GptqPlan {
   size_t off_H, off_G, off_W, off_Err, off_dead, total;

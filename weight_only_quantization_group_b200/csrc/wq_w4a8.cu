@@ -1,0 +1,172 @@
+// W4A8: 4-bit weights and 8-bit activations, each with one scale per group
+// of channels ("MIT 6.5940 Lab 4 + Lab 5", section "The five implementation
+// files and grading": the Lab 5 linear is W4A8 with group size 32; the
+// activations use the int8 absmax form of "CMU 11-868 L19-L20 Model
+// Quantization", section "absmax and zero-point", per group).
+//
+//   act_int8_kernel   per row and group: mult = 127 / max|x| (1 for a zero
+//                     group), code = rint(x * mult) clipped to +-127 -- fp32,
+//                     the oracle's operation order
+//   w4a8_gemv_kernel  y[m][n] = sum_g (step[n][g] / mult[m][g]) *
+//                     sum_{k in g} (q[n][k] - zero[n][g]) * code[m][k]
+//
+// The group sums are integer dot products: a packed word's 8 codes are two
+// words of 4 unsigned bytes after one AND and one shift-AND (byte order of
+// the 4-bit layout: k0 k4 k1 k5 | k2 k6 k3 k7), and dp4a multiplies them by
+// the activation bytes permuted the same way once per lane (two PRMT per 8
+// channels, outside the row loop). The zero point leaves the integer sum as
+// zero * (sum of the group's codes), also an integer. The per-(row, group)
+// scale cannot ride inside a tensor-core accumulator (both operands change
+// scale every group), so this path is the CUDA cores' int8 dot product.
+//
+// Mapping: each CTA stages the M rows of activation codes (permuted) with
+// their per-32-channel code sums and 1 / mult in shared memory; a warp takes
+// one output row at a time (rows grid-strided over the warps), lane l
+// channels 32 l + 1024 j of it (one 32-channel group fragment per
+// 1024-channel slice), one 16-byte load of packed weight per slice.
+#include "wq_common.cuh"
+#include "wq_launch.h"
+
+namespace wq {
+
+__global__ void __launch_bounds__(256) act_int8_kernel(const __half* __restrict__ X, int64_t n_groups, int group,
+                                                       int8_t* __restrict__ q, float* __restrict__ mult) {
+  for (int64_t gi = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; gi < n_groups;
+       gi += (int64_t)gridDim.x * blockDim.x) {
+    const __half* x = X + gi * group;
+    float amax = 0.0f;
+    for (int i = 0; i < group; ++i) amax = fmaxf(amax, fabsf(__half2float(x[i])));
+    const float m = amax == 0.0f ? 1.0f : __fdiv_rn(127.0f, amax);
+    mult[gi] = m;
+    for (int i = 0; i < group; i += 4) {
+      char4 c;
+      c.x = (signed char)fminf(fmaxf(rintf(__fmul_rn(__half2float(x[i]), m)), -127.f), 127.f);
+      c.y = (signed char)fminf(fmaxf(rintf(__fmul_rn(__half2float(x[i + 1]), m)), -127.f), 127.f);
+      c.z = (signed char)fminf(fmaxf(rintf(__fmul_rn(__half2float(x[i + 2]), m)), -127.f), 127.f);
+      c.w = (signed char)fminf(fmaxf(rintf(__fmul_rn(__half2float(x[i + 3]), m)), -127.f), 127.f);
+      *reinterpret_cast<char4*>(q + gi * group + i) = c;
+    }
+  }
+}
+
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+  uint32_t d;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+  return d;
+}
+
+template <int M>
+__global__ void __launch_bounds__(256) w4a8_gemv_kernel(const int8_t* __restrict__ qx, const float* __restrict__ mult,
+                                                        const uint32_t* __restrict__ P, const __half* __restrict__ steps,
+                                                        const __half* __restrict__ zeros, int N, int K, int group,
+                                                        __half* __restrict__ Y) {
+  extern __shared__ uint32_t xsm[];                       // [M][K/4] permuted codes
+  int* xsum = reinterpret_cast<int*>(xsm + M * (K / 4));  // [M][K/32] code sum of each 32 channels
+  float* rmul = reinterpret_cast<float*>(xsum + M * (K / 32));  // [M][K/32] 1 / mult of their group
+  const int G = K / group;
+  for (int e = threadIdx.x; e < M * (K / 32); e += blockDim.x) {
+    const int m = e / (K / 32), c32 = e % (K / 32);
+    const uint4* src = reinterpret_cast<const uint4*>(qx + (size_t)m * K + 32 * c32);
+    const uint4 v0 = src[0], v1 = src[1];
+    const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+    uint32_t* dst = xsm + (size_t)m * (K / 4) + 8 * c32;
+    int sum = 0;
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {  // channels 8c .. 8c + 7: words w[2c] (x0..x3), w[2c+1] (x4..x7)
+      dst[2 * c] = prmt(w[2 * c], w[2 * c + 1], 0x5140);      // x0 x4 x1 x5
+      dst[2 * c + 1] = prmt(w[2 * c], w[2 * c + 1], 0x7362);  // x2 x6 x3 x7
+      sum = __dp4a((int)w[2 * c], 0x01010101, sum);
+      sum = __dp4a((int)w[2 * c + 1], 0x01010101, sum);
+    }
+    xsum[e] = sum;
+    rmul[e] = 1.0f / mult[(size_t)m * G + (32 * c32) / group];
+  }
+  __syncthreads();
+  const int lane = threadIdx.x & 31;
+  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int nwarps = (gridDim.x * blockDim.x) >> 5;
+  const int slices = (K + 1023) / 1024;
+  const size_t row_words = (size_t)K / 8;
+  for (int n = warp; n < N; n += nwarps) {
+    float acc[M];
+#pragma unroll
+    for (int m = 0; m < M; ++m) acc[m] = 0.0f;
+    for (int j = 0; j < slices; ++j) {
+      const int c32 = 32 * j + lane;  // this lane's 32-channel chunk
+      if (32 * c32 < K) {
+        const uint4 wv = ld_stream_v4(P + (size_t)n * row_words + 4 * c32);
+        const float st = __half2float(steps[(size_t)n * G + (32 * c32) / group]);
+        const int z = (int)__half2float(zeros[(size_t)n * G + (32 * c32) / group]);
+        const uint32_t ws[4] = {wv.x, wv.y, wv.z, wv.w};
+#pragma unroll
+        for (int m = 0; m < M; ++m) {
+          const uint4* xa = reinterpret_cast<const uint4*>(xsm + (size_t)m * (K / 4) + 8 * c32);
+          const uint4 a0 = xa[0], a1 = xa[1];
+          const uint32_t av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+          int d = 0;
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            d = __dp4a((int)(ws[c] & 0x0F0F0F0Fu), (int)av[2 * c], d);
+            d = __dp4a((int)((ws[c] >> 4) & 0x0F0F0F0Fu), (int)av[2 * c + 1], d);
+          }
+          const int e = m * (K / 32) + c32;
+          acc[m] = fmaf((float)(d - z * xsum[e]), st * rmul[e], acc[m]);
+        }
+      }
+    }
+#pragma unroll
+    for (int m = 0; m < M; ++m) {
+      float v = acc[m];
+#pragma unroll
+      for (int o = 16; o >= 1; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+      if (lane == 0) Y[(size_t)m * N + n] = __float2half_rn(v);
+    }
+  }
+}
+
+size_t w4a8_smem_bytes(int M, int64_t K) { return (size_t)M * K + (size_t)M * (K / 32) * 8; }
+
+cudaError_t launch_act_int8(const void* X, int64_t M, int64_t K, int group, int8_t* q, float* mult,
+                            cudaStream_t st) {
+  const int64_t ng = M * (K / group);
+  const int64_t blocks = (ng + 255) / 256;
+  act_int8_kernel<<<(unsigned)(blocks < 4096 ? blocks : 4096), 256, 0, st>>>(static_cast<const __half*>(X), ng,
+                                                                             group, q, mult);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_w4a8_gemv(const int8_t* qx, const float* mult, const uint32_t* packed, const void* steps,
+                             const void* zeros, int64_t M, int64_t N, int64_t K, int group, void* Y, cudaStream_t st) {
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  auto s = static_cast<const __half*>(steps);
+  auto z = static_cast<const __half*>(zeros);
+  for (int64_t m0 = 0; m0 < M; m0 += 4) {
+    const int mc = (int)(M - m0 < 4 ? M - m0 : 4);
+    const int8_t* q = qx + m0 * K;
+    const float* mu = mult + m0 * (K / group);
+    __half* y = static_cast<__half*>(Y) + m0 * N;
+    const size_t smem = w4a8_smem_bytes(mc, K);
+    // one CTA of 8 warps per SM (at most one per 8 rows)
+    const int64_t want = (N + 7) / 8;
+    const unsigned blocks = (unsigned)(want < sms ? want : sms);
+    auto go = [&](auto kern) {
+      cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      if (e != cudaSuccess) return e;
+      kern<<<blocks, 256, smem, st>>>(q, mu, packed, s, z, (int)N, (int)K, group, y);
+      return cudaGetLastError();
+    };
+    cudaError_t e;
+    switch (mc) {
+      case 1: e = go(w4a8_gemv_kernel<1>); break;
+      case 2: e = go(w4a8_gemv_kernel<2>); break;
+      case 3: e = go(w4a8_gemv_kernel<3>); break;
+      default: e = go(w4a8_gemv_kernel<4>); break;
+    }
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
+
+}  // namespace wq
