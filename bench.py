@@ -572,9 +572,16 @@ def measure_rows(wq, torch, synth, dev, block, peaks):
                 wq.wq_set_option(wq.WQ_OPT_TC_STAGES, 0)
                 wq.wq_set_option(wq.WQ_OPT_TC_BK, 0)
                 wq.wq_set_option(wq.WQ_OPT_TC_DEQUANT_WARPS, 0)
+    c4 = synth.config_llama65b_decode(4)
     # the other kernel on each side of the crossover, for the record
     for M in (2, 3, 4, 8, 16):
         path = wq.WQ_PATH_TENSOR_CORE if M < 3 else wq.WQ_PATH_GEMV
+        if M in (3, 4):  # the row kernel's M = 4 instance on the 8192 x 8192 shape too
+            wq.wq_set_option(wq.WQ_OPT_GEMM_PATH, path)
+            try:
+                gemv_row(f"smallm4_M{M}_8192x8192_w4_gemv", 8192, 8192, 4, c4.W, synth.smallm_activations(M), M=M)
+            finally:
+                wq.wq_set_option(wq.WQ_OPT_GEMM_PATH, wq.WQ_PATH_AUTO)
         wq.wq_set_option(wq.WQ_OPT_GEMM_PATH, path)
         try:
             tag = "tc" if path == wq.WQ_PATH_TENSOR_CORE else "gemv"
@@ -588,7 +595,6 @@ def measure_rows(wq, torch, synth, dev, block, peaks):
         for M in synth.SMALLM_SWEEP:
             gemv_row(f"smallm{bits}_M{M}_8192x8192_w{bits}", 8192, 8192, bits, cb.W, synth.smallm_activations(M), M=M)
     # the K split forced, M = 16, 8192 x 8192 4-bit
-    c4 = synth.config_llama65b_decode(4)
     for ks in (1, 2, 4, 8):
         wq.wq_set_option(wq.WQ_OPT_TC_KSPLIT, ks)
         try:
@@ -686,6 +692,21 @@ def measure_rows(wq, torch, synth, dev, block, peaks):
         "note": "decode step: the block's 7 linears once (weights L2-resident after packing, not rotated)",
         "best_alpha": {g: int(o["best"].item()) / 20 for (g, _, _, _), o in zip(prepared, outs)}}
     del prepared, outs, packs
+
+    # W4A8 (Lab 5's linear): int8 activation codes per group of 32, dp4a
+    # group dot products, 8192 x 28672 (weights rotated through > 4x L2)
+    for M in (1, 4):
+        packed, steps, zeros = wq.wq_quantize_pack(dt(big.W), bits=4, group_size=32)
+        nc = max(2, math.ceil(4 * L2_BYTES / (28672 * 8192 // 2)))
+        qs = [(packed, steps, zeros)] + [tuple(t.clone() for t in (packed, steps, zeros)) for _ in range(nc - 1)]
+        qx, mult = wq.wq_quantize_act_int8(dt(synth.smallm_activations(M)), group_size=32)
+        Y = torch.empty((M, 28672), dtype=torch.float16, device=dev)
+        fns = [lambda q=q: wq.wq_w4a8_gemm(qx, mult, *q, 28672, group_size=32, out=Y) for q in qs]
+        ms = _time_graph(torch, fns) / nc
+        by = 28672 * 8192 // 2 + 28672 * (8192 // 32) * 4 + M * 8192 * 5 + M * 28672 * 2
+        rows[f"w4a8_g32_M{M}_8192x28672"] = {"us": ms * 1e3, "GB/s": by / (ms * 1e-3) / 1e9,
+                                             "frac_hbm": by / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"]}
+        del qs
 
     # GPTQ (fp64 Hessian, factorizations, column loop with error feedback)
     # on LLaMA-2-7B-shaped linears with 512 calibration tokens, 4-bit g128

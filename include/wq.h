@@ -191,8 +191,13 @@ int32_t wq_awq_scale_search(const void* X_dev, int64_t T, int64_t K, const void*
  * Scratch: one 24 MiB array in the library's own device memory (a file-scope
  * static device variable). Every GPU that loads the library holds it until
  * the process exits. The first call on a device looks up the array's device
- * address with that device current; make that first call before any stream
- * capture. All calls share the array, which keeps the last call's contents
+ * address with that device current and keeps it for the life of the
+ * process; make that first call before any stream capture, and do not use
+ * the library on a device after cudaDeviceReset (or any teardown of its
+ * primary context) -- the kept address would no longer be valid. With the
+ * default fused loss path only the per-tile partial losses live in the
+ * array; the two-kernel path also builds the error matrix there, one alpha
+ * and at most 16 MiB of rows at a time. All calls share the array, which keeps the last call's contents
  * (nothing in it has to start at zero), so calls that overlap on the GPU --
  * from other streams or threads -- race and must be serialized by the caller.
  * Limits: K <= 16384, n_alpha <= 64 and
@@ -305,8 +310,14 @@ int32_t wq_awq_fold_linear_rows(const void* W_dev, const void* b_dev, const void
  *                       memory, warps split rows, cluster split-K).
  *                       WQ_GEMV_KERNEL_TILED forces the tiled kernel.
  *  WQ_OPT_PDL           1 (default): GEMV launches allow programmatic dependent
- *                       launch (the kernel fetches its first weights before
- *                       waiting for the previous kernel in the stream); 0: off.
+ *                       launch (the kernel fetches its first weights, steps
+ *                       and zeros before waiting for the previous kernel in
+ *                       the stream); 0: off. So with it on, the kernel just
+ *                       before a GEMV in the stream must not write that
+ *                       GEMV's packed weights, steps or zeros (this library's
+ *                       own kernels never do: they release their dependents
+ *                       only at their end or after their last such write);
+ *                       set 0 when a caller's kernel does.
  *  WQ_OPT_GEMV_ROWS_SHAPE  rows per batch R, input channels per lane C and
  *                       register stages S of the row-streaming kernel:
  *                       0 default (M = 1: shape 1 for K <= 4096 and for
@@ -331,7 +342,7 @@ int32_t wq_awq_fold_linear_rows(const void* W_dev, const void* b_dev, const void
  *                       tile of the tensor-core kernel along K (their fp32
  *                       partial tiles are added in rank order in the first
  *                       CTA's shared memory): 0 default (library choice: the
- *                       largest of 1, 2, 4, 8 with all CTAs resident at once
+ *                       largest of 1, 2, 4, 8 with at most one CTA per SM
  *                       and at least 4 stages each), 1, 2, 4 or 8 (the call
  *                       fails with WQ_ERR_CUDA when the first CTA's ring
  *                       cannot hold the other partial tiles or K has fewer

@@ -309,8 +309,9 @@ def _gemv_error_bound(X, steps):
 @pytest.fixture(params=["rows_int", "rows_half", "tiled", "tiled_exact"])
 def gemv_variant(wq, request):
     """GEMV kernel choice: the row-streaming kernel where it applies, with
-    integer digit products (default) or fp32 offset sums; the tiled kernel
-    with offset sums; the tiled kernel with exact fp16 (q - zero) products."""
+    integer digit products or fp32 offset sums (the default); the tiled
+    kernel with offset sums; the tiled kernel with exact fp16 (q - zero)
+    products."""
     kern = wq.WQ_GEMV_KERNEL_TILED if request.param.startswith("tiled") else wq.WQ_GEMV_KERNEL_AUTO
     var = {"rows_int": wq.WQ_GEMV_INT_DIGITS, "rows_half": wq.WQ_GEMV_OFFSET_SUMS,
            "tiled": wq.WQ_GEMV_OFFSET_SUMS, "tiled_exact": wq.WQ_GEMV_EXACT}[request.param]
@@ -745,3 +746,23 @@ def test_tc_gemm_split_k_refused_when_partials_do_not_fit(wq, tc_path):
     finally:
         wq.wq_set_option(wq.WQ_OPT_TC_KSPLIT, 0)
         wq.wq_set_option(wq.WQ_OPT_TC_STAGES, 0)
+
+
+@pytest.mark.parametrize("group", [128, 64, 32])
+@pytest.mark.parametrize("M", [3, 4])
+@pytest.mark.parametrize("NK", [(333, 1152), (4096, 4096), (100, 8192)])
+def test_gemv_rows_m3_m4(wq, group, M, NK):
+    """The row-streaming kernel's M = 4 instance (M = 3 with a zero fourth row)
+    forced for K <= 8192, against the oracle."""
+    N, K = NK
+    g = synth.rng(2300 + M + group + N)
+    W = synth.weight(g, N, K, 0.02, channel_frac=0.01, channel_mult=10.0)
+    X = synth.activations(g, M, K, channel_frac=0.01, channel_mult=20.0)
+    (codes, st, z), qg = assert_quant_parity(wq, W, None, 4, False, group)
+    wq.wq_set_option(wq.WQ_OPT_GEMM_PATH, wq.WQ_PATH_GEMV)
+    try:
+        Y = run_gemm(wq, X, qg, N, 4, group=group)
+    finally:
+        wq.wq_set_option(wq.WQ_OPT_GEMM_PATH, wq.WQ_PATH_AUTO)
+    assert_close(Y, O.gemm_ref(X, codes, st, z, group))
+

@@ -1,4 +1,5 @@
-// S5 for M <= 2 (4- and 3-bit): row-streaming decode GEMV with activations in registers.
+// S5 for M <= 2 (4- and 3-bit) and M <= 4 (4-bit, K <= 8192): row-streaming
+// decode GEMV with activations in registers.
 //
 // The decode GEMV streams the packed weight once ("MIT 6.5940 Lab 4 + Lab 5",
 // "Starting point and setup"; "CMU 11-868 L19-L20", "where does the speed
@@ -21,7 +22,7 @@
 //     32/(R*M) batches, so the CTA meets at a barrier only that often.
 //
 // Two ways to form a lane's sum_k x_k (q_k - zero) over its channels:
-//   ActInt (default): the lane's activations become one 24-bit fixed-point
+//   ActInt (WQ_GEMV_INT_DIGITS): the lane's activations become one 24-bit fixed-point
 //     image x_k ~ X_k 2^-F (F per lane and row of X, |X_k| < 2^22, so every
 //     fp16 value within 2^-13 of the lane's largest is exact and the others
 //     are rounded by at most 2^-23 of it), split into three base-256 digits.
@@ -31,7 +32,7 @@
 //     integer; the zero point is removed per digit in integers, and the only
 //     roundings are the fixed-point image and the final fp32 combination of
 //     three digit sums per row and lane.
-//   ActHalf: one LOP3 with 0x6400 in both fp16 lanes gives (1024 + q,
+//   ActHalf (default, WQ_GEMV_OFFSET_SUMS): one LOP3 with 0x6400 in both fp16 lanes gives (1024 + q,
 //     1024 + q') or (1024 + 16q, 1024 + 16q'); a mixed fp16 x fp16 -> fp32
 //     FMA multiplies it by the activation pair (exact products, fp32 sums).
 //     The offsets and the zero point are removed per row with the lane's
@@ -48,6 +49,7 @@ struct RowsArgs {
   const __half* zeros;
   __half* Y;
   int N, K;
+  int Mv;  // rows of X present (<= the kernel's M; the rest read as zeros and are not stored)
 };
 
 // One row batch of this lane: WPR packed words per row (4-bit: 4 per 32
@@ -127,7 +129,7 @@ __device__ __forceinline__ void load_lane_x(uint32_t (&xh)[M][16 * CPL], const R
 #pragma unroll
     for (int j = 0; j < 4 * CPL; ++j) {
       uint4 v = make_uint4(0, 0, 0, 0);
-      if (active) v = *reinterpret_cast<const uint4*>(a.X + (size_t)m * a.K + k0 + 8 * j);
+      if (active && m < a.Mv) v = *reinterpret_cast<const uint4*>(a.X + (size_t)m * a.K + k0 + 8 * j);
       xh[m][4 * j] = v.x; xh[m][4 * j + 1] = v.y; xh[m][4 * j + 2] = v.z; xh[m][4 * j + 3] = v.w;
     }
   }
@@ -158,9 +160,8 @@ __device__ __forceinline__ void group_totals(const float (&c1)[M], const float (
 template <int M>
 __device__ __forceinline__ float group_epilogue(const float (&c1g)[M], const float (&xg)[M], int m, float t,
                                                 __half sc, __half zh) {
-  const float c = (M == 1 || m == 0) ? c1g[0] : c1g[M - 1];
-  const float x = (M == 1 || m == 0) ? xg[0] : xg[M - 1];
-  return __half2float(sc) * fmaf(-__half2float(zh), x, t - c);
+  // m is a compile-time index wherever this is inlined (unrolled value loops)
+  return __half2float(sc) * fmaf(-__half2float(zh), xg[m], t - c1g[m]);
 }
 
 template <int M, int CPL>
@@ -572,7 +573,7 @@ gemv_rows_kernel(RowsArgs a) {
       for (int w = 0; w < nseg; ++w) t += red[((half * NB + sl) * nseg + w) * NV + idx];
       const int row0 = (blockIdx.x + (first + sl) * gridDim.x) * R;
       const int r = idx / M, m = idx % M;
-      if (row0 + r < a.N) a.Y[(size_t)m * a.N + row0 + r] = __float2half_rn(t);
+      if (row0 + r < a.N && m < a.Mv) a.Y[(size_t)m * a.N + row0 + r] = __float2half_rn(t);
     }
     half ^= 1;
     first += nslots;
@@ -694,8 +695,11 @@ static cudaError_t launch_rows3(const RowsArgs& a, cudaStream_t st, bool pdl, in
                     : launch_rows<M, 4, 2, 2, 3, ActHalf3, GS>(a, st, pdl, gm);
 }
 
+// M = 3 and 4 (4-bit, K <= 8192, fp32 offset sums) run the M = 4 instance of
+// the (4, 32, 2) shape, a missing fourth row reading as zeros.
 bool gemv_rows_supported(int bits, int group, int64_t M, int64_t K) {
-  if (!((bits == 4 || bits == 3) && M <= 2 && K <= 16384)) return false;
+  if (M > 2 && !(bits == 4 && M <= 4 && K <= 8192)) return false;
+  if (!((bits == 4 || bits == 3) && K <= 16384)) return false;
   return group == kGroup || group == 64 || (group == 32 && bits == 4 && K <= 8192);
 }
 
@@ -710,6 +714,12 @@ cudaError_t launch_gemv_rows(const void* X, const uint32_t* packed, const void* 
   a.Y = static_cast<__half*>(Y);
   a.N = (int)N;
   a.K = (int)K;
+  a.Mv = (int)M;
+  if (M > 2) {  // 4-bit, K <= 8192: (4, 32, 2) with fp32 offset sums
+    if (group == 32) return launch_rows<4, 4, 1, 2, 4, ActHalf, 32>(a, st, pdl, grid_mode);
+    if (group == 64) return launch_rows<4, 4, 1, 2, 4, ActHalf, 64>(a, st, pdl, grid_mode);
+    return launch_rows<4, 4, 1, 2, 4, ActHalf, kGroup>(a, st, pdl, grid_mode);
+  }
   if (bits == 3) {
     if (group == 64)
       return M == 1 ? launch_rows3<1, 64>(a, st, pdl, shape, grid_mode) : launch_rows3<2, 64>(a, st, pdl, shape, grid_mode);
