@@ -847,6 +847,88 @@ def cpu_baseline(cases, seconds: float):
                               "sample": f"{sample}, {reps} passes in {el:.1f} s, one thread"}}
 
 
+def _oracle_gemv_task(task):
+    """Oracle GEMV of one block of output rows, `reps` times (one thread)."""
+    import oracle as O
+    from threadpoolctl import threadpool_limits
+    X, words, st, z, K, bits, reps = task
+    with threadpool_limits(limits=1):
+        for _ in range(reps):
+            O.gemm_ref(X, O.unpack_codes(words, bits, K), st, z, 128)
+    return reps
+
+
+def oracle_table(path: str):
+    """The oracle, as it stands, timed on the host cores for each workload of
+    the result table: one thread, and over output rows on every core (one
+    single-threaded spawned process per core; the AWQ search over numpy's own
+    BLAS threads). Each cell runs on a sample of output rows and is scaled to
+    the whole workload by the sampled fraction (every step is linear in the
+    rows). Writes milliseconds per workload to `path`."""
+    import multiprocessing as mp
+
+    import oracle as O
+    import synth
+    from threadpoolctl import threadpool_limits
+    cores = os.cpu_count() or 1
+    pool = mp.get_context("spawn").Pool(cores)
+    out = {"cores": cores, "unit": "ms per workload (scaled from the sampled rows)", "cells": {}}
+
+    def gemv_cell(name, cases, bits, frac):
+        prepared = []
+        for X, W in cases:
+            N, K = W.shape
+            rows = max(1, N // frac)
+            codes, st, z = O.quantize_groups(W[:rows], bits, 128, False)
+            prepared.append((X, O.pack_codes(codes, bits), st, z, rows, K))
+        with threadpool_limits(limits=1):
+            t0 = time.perf_counter()
+            for X, words, st, z, rows, K in prepared:
+                O.gemm_ref(X, O.unpack_codes(words, bits, K), st, z, 128)
+            one = time.perf_counter() - t0
+        tasks = []
+        for X, words, st, z, rows, K in prepared:
+            b = np.linspace(0, rows, cores + 1).astype(int)
+            tasks += [(X, words[i:j], st[i:j], z[i:j], K, bits, 1) for i, j in zip(b[:-1], b[1:]) if j > i]
+        pool.map(_oracle_gemv_task, tasks, chunksize=1)  # workers warm
+        t0 = time.perf_counter()
+        pool.map(_oracle_gemv_task, tasks, chunksize=1)
+        allc = time.perf_counter() - t0
+        out["cells"][name] = {"one_core_ms": one * frac * 1e3, "all_cores_ms": allc * frac * 1e3,
+                              "sample": f"1/{frac} of the output rows"}
+        print(name, out["cells"][name], flush=True)
+
+    try:
+        c1 = synth.config_small_linear(0)
+        gemv_cell("small_linear_K256_N128_M1_w4", [(c1.X, c1.W)], 4, 1)
+        gemv_cell("llama2_7b_block_M1_w4", [(c.X, c.W) for c in synth.config_llama7b_decode(1)], 4, 16)
+        for bits in (4, 3):
+            c = synth.config_llama65b_decode(bits)
+            gemv_cell(f"llama65b_8192x8192_M1_w{bits}", [(c.X, c.W)], bits, 32)
+        W = synth.config_smallm_sweep(1).W
+        for M in (1, 16, 128):
+            gemv_cell(f"smallm_8192x28672_M{M}_w4", [(synth.smallm_activations(M), W)], 4, 64)
+        # AWQ search over the block: every search place on 1/16 of its rows
+        frac = 16
+        places = [(X, [Wl[: max(1, Wl.shape[0] // frac)] for _, Wl in named])
+                  for _, X, named in synth.config_awq_block(5)]
+        cell = {}
+        for label, lim in (("one_core_ms", 1), ("all_cores_ms", None)):
+            with threadpool_limits(limits=lim):
+                t0 = time.perf_counter()
+                for X, Ws in places:
+                    O.awq_search(X, Ws, 4, 128, False)
+                cell[label] = (time.perf_counter() - t0) * frac * 1e3
+        cell["sample"] = f"1/{frac} of the output rows of every search place; all cores = numpy's BLAS threads"
+        out["cells"]["awq_search_llama7b_block_w4"] = cell
+        print("awq_search_llama7b_block_w4", cell, flush=True)
+    finally:
+        pool.close()
+        pool.join()
+    with open(path, "w") as f:
+        json.dump(out, f, indent=1)
+
+
 # ---------------------------------------------------------------------------
 # reference arm: the oracle on the host cores
 # ---------------------------------------------------------------------------
@@ -979,7 +1061,13 @@ def main():
     ap.add_argument("--path", choices=["auto", "gemv", "tc"], default="auto")
     ap.add_argument("--gemv-variant", choices=["int", "offset", "exact", "tiled"], default="offset")
     ap.add_argument("--rows-shape", type=int, default=0, choices=list(range(5)))
+    ap.add_argument("--oracle-table", default=None,
+                    help="only time the oracle on the host cores for each workload of the result table "
+                         "and write the milliseconds to this JSON file")
     args = ap.parse_args()
+    if args.oracle_table:
+        oracle_table(args.oracle_table)
+        return
     if args.case:
         run_case(args)
         return

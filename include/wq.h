@@ -225,6 +225,10 @@ int32_t wq_awq_scale_search_noalloc(const void* X_dev, int64_t T, int64_t K, con
  *       The weight is wq_quantize_pack's 4-bit layout with cfg->group_size
  *       equal to the activations' group; K <= 16384 (else
  *       WQ_ERR_UNSUPPORTED); q_dev 16-byte aligned.
+ *       K <= 8192 runs the row-streaming GEMV (each lane's 32 codes of every
+ *       row of X in registers; with WQ_OPT_PDL on, the same rule on the
+ *       weight's writer as wq_w4a16_gemm), larger K a kernel that holds the
+ *       codes in shared memory.
  * Asynchronous on `stream`, one launch each (wq_w4a8_gemm: one per 4 rows of
  * M). */
 int32_t wq_quantize_act_int8(const void* X_dev, int64_t M, int64_t K, int32_t group, int8_t* q_dev,

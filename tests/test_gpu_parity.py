@@ -510,6 +510,27 @@ def test_tc_gemm_stage_width(wq, tc_path, dw, bk, M, NK):
     assert_close(Y, O.gemm_ref(X, codes, st, z, 128))
 
 
+@pytest.mark.parametrize("dw", [4, 8])
+@pytest.mark.parametrize("bits,group", [(3, 128), (3, 32), (4, 32), (4, 64)])
+@pytest.mark.parametrize("M", [3, 40, 130])
+def test_tc_gemm_dequant_quartets_bits_groups(wq, tc_path, dw, bits, group, M):
+    """One and two dequantizing warp quartets (the second takes every other
+    stage) for 3-bit tiles and groups smaller than a stage."""
+    N, K = 333, 1152
+    g = synth.rng(760 + M + bits + group)
+    W = synth.weight(g, N, K, 0.02, channel_frac=0.01, channel_mult=10.0)
+    X = synth.activations(g, M, K, channel_frac=0.01, channel_mult=20.0)
+    codes, st, z = O.quantize_groups(W, bits, group, False)
+    qg = (dev(O.pack_codes(codes, bits).reshape(-1).view(np.int32)), dev(st), dev(z))
+    wq.wq_set_option(wq.WQ_OPT_TC_DEQUANT_WARPS, dw)
+    try:
+        Y = wq.wq_w4a16_gemm(dev(X), *qg, N, bits=bits, group_size=group).cpu().numpy()
+        assert wq.wq_get_last_device_error() == 0
+    finally:
+        wq.wq_set_option(wq.WQ_OPT_TC_DEQUANT_WARPS, 0)
+    assert_close(Y, O.gemm_ref(X, codes, st, z, group))
+
+
 def test_tc_gemm_symmetric_and_closed_form(wq, tc_path):
     N, K, M = 256, 1024, 32
     g = np.random.default_rng(21)

@@ -279,6 +279,11 @@ int32_t wq_w4a8_gemm(const int8_t* q, const float* mult, const uint32_t* packed,
   if (!aligned(q, 16) || !aligned(mult, 4) || !aligned(packed, 16) || !aligned(steps, 2) || !aligned(zeros, 2) ||
       !aligned(Y, 2))
     return WQ_ERR_ALIGNMENT;
+  // K <= 8192: the row-streaming GEMV (32 channels per lane); above, the
+  // slice kernel with the codes in shared memory
+  if (K <= 8192)
+    return cuda_status(wq::launch_w4a8_rows(q, mult, packed, steps, zeros, M, N, K, cfg->group_size, Y,
+                                            static_cast<cudaStream_t>(stream), g_opt_pdl != 0));
   return cuda_status(wq::launch_w4a8_gemv(q, mult, packed, steps, zeros, M, N, K, cfg->group_size, Y,
                                           static_cast<cudaStream_t>(stream)));
 }

@@ -18,11 +18,11 @@
 //             tile (BK/64 128-byte-swizzled 64-channel boxes)
 //   warp 1    TMEM owner and single-thread tcgen05.mma issuer (BK/16 MMAs
 //             per stage)
-//   warps 2.. 4 (default) or 8 warps dequantize the packed tile into one of
-//             two tensor-memory A buffers (warp w: output channels
-//             32*(w%4)..+31 -- the TMEM lane quarter it may access -- and all
-//             or half of the stage's channels), then run the epilogue
-//             (tcgen05.ld -> fp16 -> Y).
+//   warps 2.. NH quartets of 4 warps dequantize the packed tile into a ring
+//             of tensor-memory A buffers (warp w: output channels
+//             32*(w%4)..+31 -- the TMEM lane quarter it may access; quartet h
+//             takes the stages kt = h mod NH, so NH stages are dequantized at
+//             once), then run the epilogue (tcgen05.ld -> fp16 -> Y).
 // The shared-memory ring and the TMEM A ring are separate, so the TMA runs as
 // far ahead as shared memory allows while only two A buffers occupy TMEM.
 // Split K: when the row tiles cannot fill the GPU (N = 8192 gives 64 tiles
@@ -109,27 +109,27 @@ __device__ __forceinline__ void dequant_chunk3(const uint32_t* w3, __half2 zz, _
 // 16-byte reads at a 48-byte row pitch already fall on distinct banks).
 // BK: input channels per stage, 128 (one group) or 64 (half a group; shallower
 // shared-memory stages, so a deeper ring fits when M is large; 4-bit only).
-// NH: dequantizing warp quartets; each of the NH owns 1/NH of a stage's words
-// of every row (more warps hide more latency, fewer amortize the per-stage
-// waits over more weights).
+// NH: dequantizing warp quartets; quartet h owns the stages kt = h mod NH
+// whole (every row, every channel), so the per-stage chain of one quartet
+// (wait for the tile, dequantize, store to tensor memory, publish) overlaps
+// with the other quartets' stages.
 // NA: depth of the TMEM A ring (2, or 3 when the tile leaves room).
 // GS: quantization group (128, or 32 / 64 channels: then every stage holds
 // BK / GS groups, and each dequantizing thread applies the step and zero of
 // the NGT groups of its part of the stage).
 template <int BITS, int BK, int NH, int NA, int GS>
-__global__ void __launch_bounds__(64 + 128 * NH, 1)
+__global__ void __launch_bounds__(64 + 128 * NH, NH == 2 ? 2 : 1)
 w4a16_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmP,
                      TcArgs a) {
-  static_assert(BITS == 4 || (BITS == 3 && BK == 128 && NH == 1), "3-bit tiles: 128-channel stages, 4 warps");
-  static_assert(GS >= BK || GS <= BK / NH, "small groups: whole groups in every thread's part");
-  constexpr int NGT = GS < BK ? BK / NH / GS : 1;  // groups in one thread's part of a stage
+  static_assert(BITS == 4 || (BITS == 3 && BK == 128), "3-bit tiles: 128-channel stages");
+  constexpr int NGT = GS < BK ? BK / GS : 1;      // groups in one stage
   constexpr int kRowBytes = BK * BITS / 8;        // packed bytes of one row and stage
   constexpr int kPackedStage = kTcRows * kRowBytes;  // bytes of the packed tile
   constexpr int kACols = BK / 2;                  // TMEM columns per A buffer
   constexpr int kXBoxes = BK / 64;                // 64-channel X boxes per stage
-  constexpr int kWords = BK * BITS / 32 / NH;     // packed words per dequant thread and stage
+  constexpr int kWords = BK * BITS / 32;          // packed words per dequant thread and stage
   constexpr int kChunks = kWords / 4;             // 16-byte chunks per dequant thread and stage
-  constexpr int kRegs = BK / 2 / NH;              // fp16 pairs per dequant thread and stage
+  constexpr int kRegs = BK / 2;                   // fp16 pairs per dequant thread and stage
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int S = a.stages;
@@ -162,7 +162,7 @@ w4a16_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
       mbar_init(&sempty[s], 1);
     }
     for (int b = 0; b < NA; ++b) {
-      mbar_init(&afull[b], 128 * NH);
+      mbar_init(&afull[b], 128);
       mbar_init(&aempty[b], 1);
     }
     mbar_init(accum, 1);
@@ -228,49 +228,40 @@ w4a16_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
   } else {
     // ---------------------------------------------------------- dequant + epilogue
     const int q = warp & 3;             // TMEM lane quarter this warp may access
-    const int h = (warp - 2) >> 2;      // which 1/NH of the stage's packed words of a row
+    const int h = (warp - 2) >> 2;      // quartet: stages kt = h mod NH
     const int r = 32 * q + lane;        // output channel within the tile
     const int n = n0 + r;
     const bool row_ok = n < a.N;
-    // step and zero of the current group(s), and of the next, fetched a
-    // group (or, for groups smaller than a stage, a stage) ahead of their use
+    // step and zero of the NGT groups of this quartet's current stage, and of
+    // its next stage, fetched one stage ahead of their use
     __half st_cur[NGT], zr_cur[NGT], st_next[NGT], zr_next[NGT];
-    // first group of this thread's part of stage kt (small groups)
-    auto part_group = [&](int kt) { return ((kt0 + kt) * BK + h * (BK / NH)) / GS; };
+    auto first_group = [&](int kt) { return ((kt0 + kt) * BK) / GS; };
 #pragma unroll
     for (int i = 0; i < NGT; ++i) {
-      const int g0 = GS < BK ? part_group(0) + i : (kt0 * BK) / GS;
-      st_cur[i] = zr_cur[i] = __float2half(0.f);
-      st_next[i] = row_ok ? a.steps[(size_t)n * G + g0] : __float2half(0.f);
-      zr_next[i] = row_ok ? a.zeros[(size_t)n * G + g0] : __float2half(0.f);
+      st_cur[i] = zr_cur[i] = st_next[i] = zr_next[i] = __float2half(0.f);
+      if (row_ok && h < KT) {
+        st_next[i] = a.steps[(size_t)n * G + first_group(h) + i];
+        zr_next[i] = a.zeros[(size_t)n * G + first_group(h) + i];
+      }
     }
     // Software pipeline: stage kt is dequantized into registers while the
-    // tensor-memory stores of stage kt-1 complete; then kt-1 is published to
-    // the MMA issuer and kt's stores are issued (tcgen05.st reads its source
-    // registers when it issues, so they need no copy).
+    // tensor-memory stores of this quartet's previous stage complete; then that
+    // stage is published to the MMA issuer and kt's stores are issued
+    // (tcgen05.st reads its source registers when it issues, so they need no
+    // copy).
     int pend_b = -1;  // A buffer whose stores are in flight (-1: none)
-    for (int kt = 0, s = 0, u = 0, b = 0, ub = 0; kt < KT; ++kt) {
+    // s = kt mod S, u = kt / S, b = kt mod NA, ub = kt / NA (NH <= S, NA)
+    for (int kt = h, s = h, u = 0, b = h, ub = 0; kt < KT; kt += NH) {
       if (__any_sync(0xffffffffu, *abort_flag != 0)) break;
-      if constexpr (GS < BK) {  // every stage: this part's groups, and the next stage's fetched
+      // (the next stage's group may be this one: half-group stages)
+      const bool new_group = first_group(kt + NH) != first_group(kt);
 #pragma unroll
-        for (int i = 0; i < NGT; ++i) {
-          st_cur[i] = st_next[i];
-          zr_cur[i] = zr_next[i];
-          const int gn = part_group(kt + 1) + i;
-          if (row_ok && kt + 1 < KT) {
-            st_next[i] = a.steps[(size_t)n * G + gn];
-            zr_next[i] = a.zeros[(size_t)n * G + gn];
-          }
-        }
-      } else {
-        const int g = ((kt0 + kt) * BK) / GS;
-        if (kt == 0 || ((kt0 + kt) * BK) % GS == 0) {  // a new group: take its prefetched scales, fetch the next
-          st_cur[0] = st_next[0];
-          zr_cur[0] = zr_next[0];
-          if (row_ok && g + 1 < G) {
-            st_next[0] = a.steps[(size_t)n * G + g + 1];
-            zr_next[0] = a.zeros[(size_t)n * G + g + 1];
-          }
+      for (int i = 0; i < NGT; ++i) {
+        st_cur[i] = st_next[i];
+        zr_cur[i] = zr_next[i];
+        if (row_ok && kt + NH < KT && new_group) {
+          st_next[i] = a.steps[(size_t)n * G + first_group(kt + NH) + i];
+          zr_next[i] = a.zeros[(size_t)n * G + first_group(kt + NH) + i];
         }
       }
       __half2 s2[NGT], zz[NGT], zz16n[NGT];
@@ -293,14 +284,14 @@ w4a16_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
       const int sw = BITS == 3 ? 0 : BK == 128 ? (r >> 1) & 3 : (r >> 2) & 1;
 #pragma unroll
       for (int i = 0; i < kChunks; ++i) {
-        const uint4 v = *reinterpret_cast<const uint4*>(prow + (((h * kChunks + i) ^ sw) << 4));
+        const uint4 v = *reinterpret_cast<const uint4*>(prow + ((i ^ sw) << 4));
         words[4 * i] = v.x; words[4 * i + 1] = v.y; words[4 * i + 2] = v.z; words[4 * i + 3] = v.w;
       }
       uint32_t nv[kRegs / 16][16];
       if constexpr (BITS == 4) {
 #pragma unroll
         for (int j = 0; j < kWords; ++j) {
-          const int gi = 8 * j / (GS < BK ? GS : 8 * kWords);  // word j's group within the part
+          const int gi = 8 * j / (GS < BK ? GS : BK);  // word j's group within the stage
           const uint4 d = dequant_word4(words[j], zz[gi], zz16n[gi], s2[gi]);
           nv[j >> 2][4 * (j & 3)] = d.x; nv[j >> 2][4 * (j & 3) + 1] = d.y;
           nv[j >> 2][4 * (j & 3) + 2] = d.z; nv[j >> 2][4 * (j & 3) + 3] = d.w;
@@ -308,14 +299,14 @@ w4a16_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
       } else {
 #pragma unroll
         for (int c = 0; c < kRegs / 16; ++c) {  // 32 channels from three words
-          const int gi = 32 * c / (GS < BK ? GS : 32 * (kRegs / 16));
+          const int gi = 32 * c / (GS < BK ? GS : BK);
           const __half z128n = __hneg(__hadd(zr_cur[gi], __float2half(128.f)));
           const __half z16n = __hneg(__hadd(zr_cur[gi], __float2half(16.f)));
           dequant_chunk3(&words[3 * c], zz[gi], __halves2half2(z128n, z128n), __halves2half2(z16n, z16n), s2[gi],
                          nv[c]);
         }
       }
-      if (pend_b >= 0) {  // publish the previous stage
+      if (pend_b >= 0) {  // publish this quartet's previous stage
         tmem_st_wait();
         tc_fence_before();
         mbar_arrive(&afull[pend_b]);
@@ -323,12 +314,12 @@ w4a16_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
       bool ok = true;
       if (kt >= NA) ok = mbar_wait(&aempty[b], (ub - 1) & 1, a.err, a.spin_limit);
       if (!__all_sync(0xffffffffu, ok)) { *abort_flag = 1; break; }
-      const uint32_t ta = tmem_a + ((uint32_t)(32 * q) << 16) + (uint32_t)(b * kACols + (kACols / NH) * h);
+      const uint32_t ta = tmem_a + ((uint32_t)(32 * q) << 16) + (uint32_t)(b * kACols);
 #pragma unroll
       for (int i = 0; i < kRegs / 16; ++i) tmem_st16(ta + 16 * i, nv[i]);
       pend_b = b;
-      if (++s == S) { s = 0; ++u; }
-      if (++b == NA) { b = 0; ++ub; }
+      if ((s += NH) >= S) { s -= S; ++u; }
+      if ((b += NH) >= NA) { b -= NA; ++ub; }
     }
     if (pend_b >= 0) {
       tmem_st_wait();
@@ -536,31 +527,38 @@ cudaError_t launch_gemm_tc(const void* X, const uint32_t* packed, const void* st
     // 1/(cps+1) of the SM's shared memory.
     const size_t smem_floor = (size_t)(228 * 1024) / (size_t)(cps + 1) + 1024;
     if (smem < smem_floor) smem = smem_floor;
-    // 4 dequantizing warps unless asked for 8 (4-bit, 128-channel groups only)
-    const int NH = dw_opt == 8 && bits == 4 && group == kGroup ? 2 : 1;
+    // Dequantizing warp quartets: 1, or 2 when asked for 8 warps (stages
+    // alternate between them; measured no faster) and the ring has at least 3
+    // stages. A quartet
+    // publishes stage kt only once it holds stage kt + NH, which needs the
+    // shared-memory slot that stage kt - S + NH frees: the ring must be deeper
+    // than NH.
+    const int NH = (dw_opt != 8 || S < 3) ? 1 : 2;
     using I1 = std::integral_constant<int, 1>;
     using I2 = std::integral_constant<int, 2>;
     using I32 = std::integral_constant<int, 32>;
     using I64 = std::integral_constant<int, 64>;
     using I128 = std::integral_constant<int, 128>;
-    auto pick = [&](auto bits_c, auto bk, auto nh, auto gs) {
+    auto pick_na = [&](auto bits_c, auto bk, auto nh, auto gs) {
       constexpr int B = decltype(bits_c)::value, K_ = decltype(bk)::value, H = decltype(nh)::value,
                     S_ = decltype(gs)::value;
       return NA == 3 ? w4a16_gemm_tc_kernel<B, K_, H, 3, S_> : w4a16_gemm_tc_kernel<B, K_, H, 2, S_>;
     };
+    auto pick = [&](auto bits_c, auto bk, auto gs) {
+      return NH == 1 ? pick_na(bits_c, bk, I1{}, gs) : pick_na(bits_c, bk, I2{}, gs);
+    };
     using B3 = std::integral_constant<int, 3>;
     using B4 = std::integral_constant<int, 4>;
-    decltype(pick(B4{}, I128{}, I1{}, I128{})) kern;
+    decltype(pick(B4{}, I128{}, I128{})) kern;
     if (bits == 3)
-      kern = group == 32 ? pick(B3{}, I128{}, I1{}, I32{}) : group == 64 ? pick(B3{}, I128{}, I1{}, I64{})
-                                                                         : pick(B3{}, I128{}, I1{}, I128{});
+      kern = group == 32 ? pick(B3{}, I128{}, I32{}) : group == 64 ? pick(B3{}, I128{}, I64{})
+                                                                   : pick(B3{}, I128{}, I128{});
     else if (group == 32)
-      kern = BK == 128 ? pick(B4{}, I128{}, I1{}, I32{}) : pick(B4{}, I64{}, I1{}, I32{});
+      kern = BK == 128 ? pick(B4{}, I128{}, I32{}) : pick(B4{}, I64{}, I32{});
     else if (group == 64)
-      kern = BK == 128 ? pick(B4{}, I128{}, I1{}, I64{}) : pick(B4{}, I64{}, I1{}, I64{});
+      kern = BK == 128 ? pick(B4{}, I128{}, I64{}) : pick(B4{}, I64{}, I64{});
     else
-      kern = BK == 128 ? (NH == 1 ? pick(B4{}, I128{}, I1{}, I128{}) : pick(B4{}, I128{}, I2{}, I128{}))
-                       : (NH == 1 ? pick(B4{}, I64{}, I1{}, I128{}) : pick(B4{}, I64{}, I2{}, I128{}));
+      kern = BK == 128 ? pick(B4{}, I128{}, I128{}) : pick(B4{}, I64{}, I128{});
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     // Split K over a cluster while the row tiles leave SMs idle: double it

@@ -37,6 +37,8 @@
 //     FMA multiplies it by the activation pair (exact products, fp32 sums).
 //     The offsets and the zero point are removed per row with the lane's
 //     activation class sums.
+#include <type_traits>
+
 #include "wq_common.cuh"
 #include "wq_launch.h"
 
@@ -50,6 +52,8 @@ struct RowsArgs {
   __half* Y;
   int N, K;
   int Mv;  // rows of X present (<= the kernel's M; the rest read as zeros and are not stored)
+  const int8_t* Xq;   // W4A8: int8 activation codes [M][K] (X unused)
+  const float* mult;  // W4A8: their multipliers [M][K / group]
 };
 
 // One row batch of this lane: WPR packed words per row (4-bit: 4 per 32
@@ -430,6 +434,91 @@ struct ActInt {
   }
 };
 
+// ---------------------------------------------------------------- ActW4A8
+// W4A8 ("MIT 6.5940 Lab 4 + Lab 5", "The five implementation files and
+// grading"): the activations are int8 codes with one fp32 multiplier per row
+// of X and group of channels. A lane's 32 codes of each row sit in eight
+// words permuted into the byte order of the masked code words (lo: channels
+// 8c + 0, 4, 1, 5, the low nibbles of a word's bytes; hi: 8c + 2, 6, 3, 7),
+// so dp4a multiplies four weights by four codes at once and the lane's dot
+// product is an exact integer. The zero point leaves zero * (sum of the
+// lane's codes), an integer too; the lane then scales by step / multiplier
+// in fp32 (its 32 channels lie in one weight group and one activation group).
+__device__ __forceinline__ uint32_t prmt_b32(uint32_t a, uint32_t b, uint32_t sel) {
+  uint32_t d;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+  return d;
+}
+
+template <int M, int CPL>
+struct ActW4A8 {
+  static_assert(CPL == 1, "W4A8 rows: 32 channels per lane");
+  static constexpr bool kGroupFirst = false;  // step / multiplier applied per lane
+  uint32_t lo[M][4], hi[M][4];
+  int xs[M];    // sum of the lane's codes
+  float rm[M];  // 1 / multiplier of the lane's activation group
+
+  template <int LPG>
+  __device__ __forceinline__ void load(const RowsArgs& a, int k0, bool active) {
+    const int gsz = 32 * LPG;  // group size
+#pragma unroll
+    for (int m = 0; m < M; ++m) {
+      uint4 v0 = make_uint4(0, 0, 0, 0), v1 = v0;
+      float mu = 1.0f;
+      if (active && m < a.Mv) {
+        const uint4* src = reinterpret_cast<const uint4*>(a.Xq + (size_t)m * a.K + k0);
+        v0 = src[0];
+        v1 = src[1];
+        mu = a.mult[(size_t)m * (a.K / gsz) + k0 / gsz];
+      }
+      const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+      int sum = 0;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {  // channels 8c .. 8c + 7: w[2c] = codes 0..3, w[2c + 1] = codes 4..7
+        lo[m][c] = prmt_b32(w[2 * c], w[2 * c + 1], 0x5140u);  // codes 0 4 1 5
+        hi[m][c] = prmt_b32(w[2 * c], w[2 * c + 1], 0x7362u);  // codes 2 6 3 7
+        sum = __dp4a((int)w[2 * c], 0x01010101, sum);
+        sum = __dp4a((int)w[2 * c + 1], 0x01010101, sum);
+      }
+      xs[m] = sum;
+      rm[m] = 1.0f / mu;
+    }
+  }
+
+  __device__ __forceinline__ float epilogue(int, float t, __half, __half) const { return t; }
+
+  template <int R, int RL>
+  __device__ __forceinline__ void compute(const RowsStage<R, 4 * CPL, RL>& s, float (&acc)[R * M]) const {
+    static_assert(RL == R, "the W4A8 path applies every row's step per lane");
+    int d[R][M];
+#pragma unroll
+    for (int r = 0; r < R; ++r)
+#pragma unroll
+      for (int m = 0; m < M; ++m) d[r][m] = 0;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+#pragma unroll
+      for (int r = 0; r < R; ++r) {
+        const uint32_t w = s.w[r][j];
+        const uint32_t ql = w & 0x0F0F0F0Fu;         // q of channels 0, 4, 1, 5
+        const uint32_t qh = (w >> 4) & 0x0F0F0F0Fu;  // q of channels 2, 6, 3, 7
+#pragma unroll
+        for (int m = 0; m < M; ++m) {
+          d[r][m] = dp4a_us(ql, lo[m][j], d[r][m]);
+          d[r][m] = dp4a_us(qh, hi[m][j], d[r][m]);
+        }
+      }
+    }
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      const int z = __half2int_rn(s.zh[r]);
+      const float sc = __half2float(s.sc[r]);
+#pragma unroll
+      for (int m = 0; m < M; ++m) acc[r * M + m] = (float)(d[r][m] - z * xs[m]) * (sc * rm[m]);
+    }
+  }
+};
+
 // Sum over the 32 lanes of v[idx] for every idx: afterwards lanes whose low
 // (5 - log2 NV) bits are zero hold one total each, for value `index`.
 template <int NV>
@@ -743,6 +832,38 @@ cudaError_t launch_gemv_rows(const void* X, const uint32_t* packed, const void* 
                   : launch_rows_shape<2, 64>(a, st, pdl, act_int, shape, grid_mode);
   return M == 1 ? launch_rows_shape<1, kGroup>(a, st, pdl, act_int, shape, grid_mode)
                 : launch_rows_shape<2, kGroup>(a, st, pdl, act_int, shape, grid_mode);
+}
+
+// W4A8 rows (K <= 8192, 32 channels per lane; the (4, 32, 2) shape): X in
+// chunks of up to 4 rows, a missing row reading as zeros.
+cudaError_t launch_w4a8_rows(const int8_t* qx, const float* mult, const uint32_t* packed, const void* steps,
+                             const void* zeros, int64_t M, int64_t N, int64_t K, int group, void* Y, cudaStream_t st,
+                             bool pdl) {
+  for (int64_t m0 = 0; m0 < M; m0 += 4) {
+    const int mc = (int)(M - m0 < 4 ? M - m0 : 4);
+    RowsArgs a;
+    a.X = nullptr;
+    a.Xq = qx + m0 * K;
+    a.mult = mult + m0 * (K / group);
+    a.P = packed;
+    a.steps = static_cast<const __half*>(steps);
+    a.zeros = static_cast<const __half*>(zeros);
+    a.Y = static_cast<__half*>(Y) + m0 * N;
+    a.N = (int)N;
+    a.K = (int)K;
+    a.Mv = mc;
+    auto go = [&](auto gs) -> cudaError_t {
+      constexpr int GS = decltype(gs)::value;
+      if (mc == 1) return launch_rows<1, 4, 1, 2, 4, ActW4A8, GS>(a, st, pdl, 1);
+      if (mc == 2) return launch_rows<2, 4, 1, 2, 4, ActW4A8, GS>(a, st, pdl, 1);
+      return launch_rows<4, 4, 1, 2, 4, ActW4A8, GS>(a, st, pdl, 1);
+    };
+    cudaError_t e = group == 32   ? go(std::integral_constant<int, 32>{})
+                    : group == 64 ? go(std::integral_constant<int, 64>{})
+                                  : go(std::integral_constant<int, kGroup>{});
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
 }
 
 }  // namespace wq

@@ -51,6 +51,10 @@ cudaError_t launch_act_int8(const void* X, int64_t M, int64_t K, int group, int8
 size_t w4a8_smem_bytes(int M, int64_t K);
 cudaError_t launch_w4a8_gemv(const int8_t* qx, const float* mult, const uint32_t* packed, const void* steps,
                              const void* zeros, int64_t M, int64_t N, int64_t K, int group, void* Y, cudaStream_t st);
+// W4A8 on the row-streaming GEMV (wq_gemv_rows.cu), K <= 8192.
+cudaError_t launch_w4a8_rows(const int8_t* qx, const float* mult, const uint32_t* packed, const void* steps,
+                             const void* zeros, int64_t M, int64_t N, int64_t K, int group, void* Y, cudaStream_t st,
+                             bool pdl);
 // GPTQ (wq_gptq.cu): workspace layout and the launch sequence.
 struct GptqPlan {
   size_t off_H, off_G, off_W, off_Err, off_dead, total;

@@ -19,11 +19,12 @@
 // scale cannot ride inside a tensor-core accumulator (both operands change
 // scale every group), so this path is the CUDA cores' int8 dot product.
 //
-// Mapping: each CTA stages the M rows of activation codes (permuted) with
-// their per-32-channel code sums and 1 / mult in shared memory; a warp takes
-// one output row at a time (rows grid-strided over the warps), lane l
-// channels 32 l + 1024 j of it (one 32-channel group fragment per
-// 1024-channel slice), one 16-byte load of packed weight per slice.
+// Mapping: every resident CTA slot gets a CTA; each stages the M rows of
+// activation codes (permuted) with their per-32-channel code sums and
+// 1 / mult in shared memory; a warp takes one output row at a time (rows
+// grid-strided over the warps), lane l channels 32 l + 1024 j of it (one
+// 32-channel group fragment per 1024-channel slice), one 16-byte load of
+// packed weight per slice, eight slices' loads issued together.
 #include "wq_common.cuh"
 #include "wq_launch.h"
 
@@ -54,6 +55,8 @@ __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
   asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
   return d;
 }
+
+constexpr int kSlicesInFlight = 8;  // 1024-channel slices whose loads a warp issues together
 
 template <int M>
 __global__ void __launch_bounds__(256) w4a8_gemv_kernel(const int8_t* __restrict__ qx, const float* __restrict__ mult,
@@ -91,26 +94,43 @@ __global__ void __launch_bounds__(256) w4a8_gemv_kernel(const int8_t* __restrict
     float acc[M];
 #pragma unroll
     for (int m = 0; m < M; ++m) acc[m] = 0.0f;
-    for (int j = 0; j < slices; ++j) {
-      const int c32 = 32 * j + lane;  // this lane's 32-channel chunk
-      if (32 * c32 < K) {
-        const uint4 wv = ld_stream_v4(P + (size_t)n * row_words + 4 * c32);
-        const float st = __half2float(steps[(size_t)n * G + (32 * c32) / group]);
-        const int z = (int)__half2float(zeros[(size_t)n * G + (32 * c32) / group]);
-        const uint32_t ws[4] = {wv.x, wv.y, wv.z, wv.w};
+    // eight slices of the row at a time: their weight, step and zero loads
+    // are all issued before the first dot product
+    for (int j0 = 0; j0 < slices; j0 += kSlicesInFlight) {
+      uint4 wv[kSlicesInFlight];
+      float st[kSlicesInFlight];
+      int zr[kSlicesInFlight];
 #pragma unroll
-        for (int m = 0; m < M; ++m) {
-          const uint4* xa = reinterpret_cast<const uint4*>(xsm + (size_t)m * (K / 4) + 8 * c32);
-          const uint4 a0 = xa[0], a1 = xa[1];
-          const uint32_t av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
-          int d = 0;
+      for (int jj = 0; jj < kSlicesInFlight; ++jj) {
+        const int c32 = 32 * (j0 + jj) + lane;  // this lane's 32-channel chunk of slice j0 + jj
+        wv[jj] = make_uint4(0u, 0u, 0u, 0u);
+        st[jj] = 0.0f;
+        zr[jj] = 0;
+        if (32 * c32 < K) {
+          wv[jj] = ld_stream_v4(P + (size_t)n * row_words + 4 * c32);
+          st[jj] = __half2float(steps[(size_t)n * G + (32 * c32) / group]);
+          zr[jj] = (int)__half2float(zeros[(size_t)n * G + (32 * c32) / group]);
+        }
+      }
 #pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            d = __dp4a((int)(ws[c] & 0x0F0F0F0Fu), (int)av[2 * c], d);
-            d = __dp4a((int)((ws[c] >> 4) & 0x0F0F0F0Fu), (int)av[2 * c + 1], d);
+      for (int jj = 0; jj < kSlicesInFlight; ++jj) {
+        const int c32 = 32 * (j0 + jj) + lane;
+        if (32 * c32 < K) {
+          const uint32_t ws[4] = {wv[jj].x, wv[jj].y, wv[jj].z, wv[jj].w};
+#pragma unroll
+          for (int m = 0; m < M; ++m) {
+            const uint4* xa = reinterpret_cast<const uint4*>(xsm + (size_t)m * (K / 4) + 8 * c32);
+            const uint4 a0 = xa[0], a1 = xa[1];
+            const uint32_t av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+            int d = 0;
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+              d = __dp4a((int)(ws[c] & 0x0F0F0F0Fu), (int)av[2 * c], d);
+              d = __dp4a((int)((ws[c] >> 4) & 0x0F0F0F0Fu), (int)av[2 * c + 1], d);
+            }
+            const int e = m * (K / 32) + c32;
+            acc[m] = fmaf((float)(d - zr[jj] * xsum[e]), st[jj] * rmul[e], acc[m]);
           }
-          const int e = m * (K / 32) + c32;
-          acc[m] = fmaf((float)(d - z * xsum[e]), st * rmul[e], acc[m]);
         }
       }
     }
@@ -148,12 +168,15 @@ cudaError_t launch_w4a8_gemv(const int8_t* qx, const float* mult, const uint32_t
     const float* mu = mult + m0 * (K / group);
     __half* y = static_cast<__half*>(Y) + m0 * N;
     const size_t smem = w4a8_smem_bytes(mc, K);
-    // one CTA of 8 warps per SM (at most one per 8 rows)
-    const int64_t want = (N + 7) / 8;
-    const unsigned blocks = (unsigned)(want < sms ? want : sms);
     auto go = [&](auto kern) {
       cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
       if (e != cudaSuccess) return e;
+      // every resident slot gets a CTA of 8 warps (at most one CTA per 8 rows)
+      int per_sm = 1;
+      if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, 256, smem) != cudaSuccess || per_sm < 1)
+        per_sm = 1;
+      const int64_t want = (N + 7) / 8, slots = (int64_t)sms * per_sm;
+      const unsigned blocks = (unsigned)(want < slots ? want : slots);
       kern<<<blocks, 256, smem, st>>>(q, mu, packed, s, z, (int)N, (int)K, group, y);
       return cudaGetLastError();
     };
