@@ -448,6 +448,13 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         "clocks": clocks,
         "rows_line": "printed on the line before this one" if rows else "not measured (--no-rows)",
     }
+    if "block_step_fused_4_launches" in rows:
+        f = rows["block_step_fused_4_launches"]
+        line["packed_4_launches"] = {
+            "value": round(f["GB/s"], 2), "unit": "GB/s", "ms_per_step": f["us"] / 1e3,
+            "frac": round(f["frac_hbm"], 4),
+            "note": "the same 7 linears and bytes, q|k|v and gate|up each packed as one weight (they share an "
+                    "input): 4 launches per step"}
     if not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(cases, args.cpu_seconds)
     return line, rows
@@ -557,6 +564,19 @@ def measure_rows(wq, torch, synth, dev, block, peaks):
             wq.wq_set_option(wq.WQ_OPT_GEMV_GRID, 1)
     for M in synth.SMALLM_SWEEP:
         gemv_row(f"smallm_M{M}_8192x28672_w4", 28672, 8192, 4, big.W, synth.smallm_activations(M), M=M)
+    # context: the dense fp16 matmul of the same shape (cuBLAS through torch),
+    # reading the 470 MB fp16 weight
+    Wd16 = dt(big.W)
+    for M in (1, 16, 128):
+        Xd = dt(synth.smallm_activations(M))
+        Yd = torch.empty((M, 28672), dtype=torch.float16, device=dev)
+        ms = _time_graph(torch, [lambda: torch.matmul(Xd, Wd16.t(), out=Yd)])
+        fl = 2.0 * M * 28672 * 8192
+        by = 28672 * 8192 * 2 + M * 8192 * 2 + M * 28672 * 2
+        rows[f"torch_fp16_dense_M{M}_8192x28672"] = {
+            "us": ms * 1e3, "TFLOP/s": fl / (ms * 1e-3) / 1e12, "frac_bf16_peak": fl / (ms * 1e-3) / 1e12 /
+            peaks["bf16_tflops"], "GB/s": by / (ms * 1e-3) / 1e9, "note": "torch.matmul, dense fp16 weight (context)"}
+    del Wd16
     # tensor-core kernel: dequantizing warps, channels per stage, ring depth (0 = library choice)
     for M in (4, 16, 64, 128):
         for dw, bk, S in ((8, 128, 0), (4, 128, 0), (4, 128, 5), (4, 64, 0), (8, 64, 5), (8, 128, 5)):
@@ -576,12 +596,18 @@ def measure_rows(wq, torch, synth, dev, block, peaks):
     # the other kernel on each side of the crossover, for the record
     for M in (2, 3, 4, 8, 16):
         path = wq.WQ_PATH_TENSOR_CORE if M < 3 else wq.WQ_PATH_GEMV
-        if M in (3, 4):  # the row kernel's M = 4 instance on the 8192 x 8192 shape too
-            wq.wq_set_option(wq.WQ_OPT_GEMM_PATH, path)
-            try:
-                gemv_row(f"smallm4_M{M}_8192x8192_w4_gemv", 8192, 8192, 4, c4.W, synth.smallm_activations(M), M=M)
-            finally:
-                wq.wq_set_option(wq.WQ_OPT_GEMM_PATH, wq.WQ_PATH_AUTO)
+        if M in (3, 4):  # both kernels at M = 3, 4 on the narrower weights (the default picks the row kernel)
+            for p2, t2 in ((wq.WQ_PATH_GEMV, "gemv"), (wq.WQ_PATH_TENSOR_CORE, "tc")):
+                wq.wq_set_option(wq.WQ_OPT_GEMM_PATH, p2)
+                try:
+                    gemv_row(f"smallm4_M{M}_8192x8192_w4_{t2}", 8192, 8192, 4, c4.W, synth.smallm_activations(M),
+                             M=M)
+                    for b in (block[0], block[4], block[6]):
+                        Xm = synth.activations(synth.rng(77 + M), M, b["K"])
+                        gemv_row(f"M{M}_{b['name'].replace('_M1', '')}_{t2}", b["N"], b["K"], 4,
+                                 b["W"].cpu().numpy(), Xm, M=M)
+                finally:
+                    wq.wq_set_option(wq.WQ_OPT_GEMM_PATH, wq.WQ_PATH_AUTO)
         wq.wq_set_option(wq.WQ_OPT_GEMM_PATH, path)
         try:
             tag = "tc" if path == wq.WQ_PATH_TENSOR_CORE else "gemv"
@@ -906,7 +932,7 @@ def oracle_table(path: str):
             c = synth.config_llama65b_decode(bits)
             gemv_cell(f"llama65b_8192x8192_M1_w{bits}", [(c.X, c.W)], bits, 32)
         W = synth.config_smallm_sweep(1).W
-        for M in (1, 16, 128):
+        for M in synth.SMALLM_SWEEP:
             gemv_cell(f"smallm_8192x28672_M{M}_w4", [(synth.smallm_activations(M), W)], 4, 64)
         # AWQ search over the block: every search place on 1/16 of its rows
         frac = 16
@@ -1011,11 +1037,19 @@ def run_case(args):
     wq.wq_set_option(wq.WQ_OPT_GEMV_KERNEL, wq.WQ_GEMV_KERNEL_TILED if args.gemv_variant == "tiled"
                      else wq.WQ_GEMV_KERNEL_AUTO)
     wq.wq_set_option(wq.WQ_OPT_GEMV_ROWS_SHAPE, args.rows_shape)
-    q = wq.wq_quantize_pack(W, bits=args.bits)
+    q = wq.wq_quantize_pack(W, bits=args.bits, group_size=args.group)
     Y = torch.empty((args.M, args.N), dtype=torch.float16, device=dev)
     if args.case == "awq":  # M calibration rows, one linear of N outputs, 20 alphas
         ws = torch.empty(wq.wq_awq_workspace_bytes(args.M, args.K, [args.N], 20, bits=args.bits),
                          dtype=torch.uint8, device=dev)
+    if args.case == "gptq":  # M calibration rows
+        ws = torch.empty(wq.wq_gptq_workspace_bytes(args.N, args.K, bits=args.bits, group_size=args.group),
+                         dtype=torch.uint8, device=dev)
+    if args.case == "w4a8":
+        qx, mult = wq.wq_quantize_act_int8(X, group_size=args.group)
+    if args.case == "fold":
+        sv = torch.from_numpy(synth.activations(g, 1, args.N, std=0.2).reshape(-1)).abs().add_(0.5).to(dev)
+        Wo = torch.empty_like(W)
     torch.cuda.synchronize()
     times = []
     for _ in range(args.reps):
@@ -1025,6 +1059,12 @@ def run_case(args):
             wq.wq_w4a16_gemm(X, *q, args.N, bits=args.bits, out=Y)
         elif args.case == "awq":
             wq.wq_awq_scale_search(X, [W], bits=args.bits, workspace=ws)
+        elif args.case == "gptq":
+            wq.wq_gptq_quantize_pack(W, X, bits=args.bits, group_size=args.group, workspace=ws, out=q)
+        elif args.case == "w4a8":
+            wq.wq_w4a8_gemm(qx, mult, *q, args.N, group_size=args.group, out=Y)
+        elif args.case == "fold":
+            wq.wq_awq_fold_linear_rows(W, sv, out=(Wo, None))
         else:
             wq.wq_quantize_pack(W, bits=args.bits, out=q)
         b.record()
@@ -1051,12 +1091,13 @@ def main():
     ap.add_argument("--eager", action="store_true", help="launch eagerly instead of replaying CUDA graphs")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--ref-seconds", type=float, default=60.0)
-    ap.add_argument("--case", choices=["gemm", "quantize", "awq"], default=None,
+    ap.add_argument("--case", choices=["gemm", "quantize", "awq", "gptq", "w4a8", "fold"], default=None,
                     help="run one small kernel configuration --reps times (for profiling)")
     ap.add_argument("--M", type=int, default=1)
     ap.add_argument("--N", type=int, default=8192)
     ap.add_argument("--K", type=int, default=8192)
     ap.add_argument("--bits", type=int, default=4)
+    ap.add_argument("--group", type=int, default=128)
     ap.add_argument("--reps", type=int, default=3)
     ap.add_argument("--path", choices=["auto", "gemv", "tc"], default="auto")
     ap.add_argument("--gemv-variant", choices=["int", "offset", "exact", "tiled"], default="offset")

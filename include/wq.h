@@ -291,7 +291,10 @@ int32_t wq_awq_fold_linear_rows(const void* W_dev, const void* b_dev, const void
  *  WQ_OPT_GEMM_PATH     WQ_PATH_AUTO (default): GEMV kernel below the
  *                       crossover M, tensor-core kernel at or above it;
  *                       WQ_PATH_GEMV / WQ_PATH_TENSOR_CORE force one kernel.
- *  WQ_OPT_CROSSOVER_M   smallest M sent to the tensor-core kernel (default 3).
+ *  WQ_OPT_CROSSOVER_M   smallest M sent to the tensor-core kernel (default 3;
+ *                       with WQ_PATH_AUTO, M = 3 and 4 at 4 bits with
+ *                       K <= 8192 stay on the row GEMV when the weight has
+ *                       fewer 128-row tiles than the device has SMs).
  *  WQ_OPT_GEMV_VARIANT  how the GEMV kernel forms sum_k x_k (q_k - zero):
  *                       WQ_GEMV_OFFSET_SUMS (default) multiplies x by the
  *                       unpacked (1024 + q) in fp32 (exact products) and

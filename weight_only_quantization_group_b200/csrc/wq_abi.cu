@@ -134,6 +134,19 @@ size_t wq_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, const wq_quant_c
   return 0;
 }
 
+// SMs of the current device (cached per process; one device type per process).
+static int num_sms() {
+  static std::atomic<int> sms{0};
+  int v = sms.load();
+  if (v == 0) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0)
+      v = 148;
+    sms.store(v);
+  }
+  return v;
+}
+
 int32_t wq_w4a16_gemm(const void* X, const uint32_t* packed, const void* steps, const void* zeros, int64_t M,
                       int64_t N, int64_t K, const wq_quant_cfg* cfg, void* Y, void* workspace,
                       size_t workspace_bytes, void* stream) {
@@ -152,6 +165,12 @@ int32_t wq_w4a16_gemm(const void* X, const uint32_t* packed, const void* steps, 
   const bool rows_ok = g_opt_gemv_kernel != WQ_GEMV_KERNEL_TILED && variant != WQ_GEMV_EXACT &&
                        wq::gemv_rows_supported(cfg->bits, group, M, K);
   bool tensor_core = M >= g_opt_crossover_m;
+  // M = 3, 4 (4-bit, K <= 8192) stay on the row GEMV when the weight has
+  // fewer 128-row tiles than the GPU has SMs: there the tensor-core kernel
+  // leaves SMs idle or splits K over clusters (8192 x 8192, M = 4: 21 us on
+  // the row kernel against 31 us), while wider weights keep every SM's
+  // tensor pipe busy (8192 x 28672, M = 4: 56 us against 67 us).
+  if (path == WQ_PATH_AUTO && tensor_core && M <= 4 && rows_ok && (N + 127) / 128 < num_sms()) tensor_core = false;
   if (path == WQ_PATH_GEMV) tensor_core = false;
   if (path == WQ_PATH_TENSOR_CORE) tensor_core = true;
   // groups of 32 or 64 channels that the row-streaming kernel does not take
