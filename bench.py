@@ -500,14 +500,18 @@ def measure_rows(wq, torch, synth, dev, block, peaks):
                                       "weights": sum(b["N"] * b["K"] for b in block)}
 
     # single-shape GEMVs, rotating copies >= 4x L2
-    def gemv_row(name, N, K, bits, W16, X16, M=1):
+    def gemv_row(name, N, K, bits, W16, X16, M=1, ws=True):
+        """ws: pass the GEMM workspace (the tensor-core kernel's stream-K
+        schedule where it applies), as a caller that has one would."""
         packed, steps, zeros = wq.wq_quantize_pack(dt(W16), bits=bits)
         wbytes = N * K * bits // 8
         nc = max(2, math.ceil(4 * L2_BYTES / wbytes))
         qs = [(packed, steps, zeros)] + [tuple(t.clone() for t in (packed, steps, zeros)) for _ in range(nc - 1)]
         X = dt(X16)
         Y = torch.empty((M, N), dtype=torch.float16, device=dev)
-        fns = [lambda q=q: wq.wq_w4a16_gemm(X, *q, N, bits=bits, out=Y) for q in qs]
+        nws = wq.wq_gemm_workspace_bytes(M, N, K, bits=bits) if ws else 0
+        W = torch.zeros(nws, dtype=torch.uint8, device=dev) if nws else None  # zero-filled once
+        fns = [lambda q=q: wq.wq_w4a16_gemm(X, *q, N, bits=bits, out=Y, workspace=W) for q in qs]
         ms = _time_graph(torch, fns) / nc
         by = gemm_bytes(M, N, K, bits)
         fl = 2.0 * M * N * K
@@ -564,6 +568,9 @@ def measure_rows(wq, torch, synth, dev, block, peaks):
             wq.wq_set_option(wq.WQ_OPT_GEMV_GRID, 1)
     for M in synth.SMALLM_SWEEP:
         gemv_row(f"smallm_M{M}_8192x28672_w4", 28672, 8192, 4, big.W, synth.smallm_activations(M), M=M)
+        if M >= 3:  # the same call without a workspace: one CTA per row tile
+            gemv_row(f"smallm_M{M}_8192x28672_w4_nows", 28672, 8192, 4, big.W, synth.smallm_activations(M), M=M,
+                     ws=False)
     # context: the dense fp16 matmul of the same shape (cuBLAS through torch),
     # reading the 470 MB fp16 weight
     Wd16 = dt(big.W)
@@ -1039,6 +1046,10 @@ def run_case(args):
     wq.wq_set_option(wq.WQ_OPT_GEMV_ROWS_SHAPE, args.rows_shape)
     q = wq.wq_quantize_pack(W, bits=args.bits, group_size=args.group)
     Y = torch.empty((args.M, args.N), dtype=torch.float16, device=dev)
+    ws = None
+    if args.case == "gemm" and args.workspace:
+        n = wq.wq_gemm_workspace_bytes(args.M, args.N, args.K, bits=args.bits, group_size=args.group)
+        ws = torch.zeros(max(n, 1), dtype=torch.uint8, device=dev) if n else None
     if args.case == "awq":  # M calibration rows, one linear of N outputs, 20 alphas
         ws = torch.empty(wq.wq_awq_workspace_bytes(args.M, args.K, [args.N], 20, bits=args.bits),
                          dtype=torch.uint8, device=dev)
@@ -1056,7 +1067,7 @@ def run_case(args):
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record()
         if args.case == "gemm":
-            wq.wq_w4a16_gemm(X, *q, args.N, bits=args.bits, out=Y)
+            wq.wq_w4a16_gemm(X, *q, args.N, bits=args.bits, group_size=args.group, out=Y, workspace=ws)
         elif args.case == "awq":
             wq.wq_awq_scale_search(X, [W], bits=args.bits, workspace=ws)
         elif args.case == "gptq":
@@ -1098,6 +1109,7 @@ def main():
     ap.add_argument("--K", type=int, default=8192)
     ap.add_argument("--bits", type=int, default=4)
     ap.add_argument("--group", type=int, default=128)
+    ap.add_argument("--workspace", action="store_true", help="--case gemm: pass the GEMM workspace")
     ap.add_argument("--reps", type=int, default=3)
     ap.add_argument("--path", choices=["auto", "gemv", "tc"], default="auto")
     ap.add_argument("--gemv-variant", choices=["int", "offset", "exact", "tiled"], default="offset")

@@ -138,9 +138,21 @@ size_t wq_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, const wq_quant_c
  * dequantized on the fly inside the matmul; "TinyChat (AWQ on-device
  * runtime)", "Notable features": fused dequant + GEMM). Small M runs a
  * bandwidth-bound GEMV kernel that streams the packed weights once; larger M
- * (3- and 4-bit) runs a tcgen05 tensor-core kernel. workspace_dev may be NULL when
- * wq_gemm_workspace_bytes() is 0. X must already be multiplied by
- * diag(s)^-1 when the weight was packed with AWQ scales s. */
+ * (3- and 4-bit) runs a tcgen05 tensor-core kernel. X must already be
+ * multiplied by diag(s)^-1 when the weight was packed with AWQ scales s.
+ * workspace_dev is optional: NULL, or device memory of at least
+ * wq_gemm_workspace_bytes(M, N, K, cfg) bytes, 256-byte aligned and
+ * zero-filled before its first use. Given it, the tensor-core kernel balances
+ * its work over all SMs (stream-K: every CTA of a persistent grid takes the
+ * same number of K stages, at most one row tile's worth; a tile split between
+ * CTAs is summed from their fp32 partial tiles in CTA order, so the result
+ * does not depend on timing) for M <= 16 (WQ_OPT_TC_STREAMK). Its first 64 KB hold
+ * arrival counters that every completed call leaves at zero, so calls of any
+ * shape may share one workspace as long as they do not overlap in time (same
+ * stream); after a call that ended in WQ_ERR_TIMEOUT, zero-fill it again.
+ * Without a workspace: one CTA per row tile (and K split over thread-block
+ * clusters when the tiles leave SMs idle). The same weight, X and workspace
+ * size give the same Y on every call. wq_gemm_workspace_bytes is 0 for M < 3. */
 int32_t wq_w4a16_gemm(const void* X_dev, const uint32_t* packed_dev, const void* steps_dev,
                       const void* zeros_dev, int64_t M, int64_t N, int64_t K,
                       const wq_quant_cfg* cfg, void* Y_dev, void* workspace_dev,
@@ -345,6 +357,12 @@ int32_t wq_awq_fold_linear_rows(const void* W_dev, const void* b_dev, const void
  *                       else 128), 64 or 128.
  *  WQ_OPT_TC_DEQUANT_WARPS  warps that dequantize in the tensor-core kernel:
  *                       0 default (4), 4 or 8.
+ *  WQ_OPT_TC_STREAMK    the tensor-core kernel's stream-K schedule (needs the
+ *                       workspace): 0 default (for M <= 16 per launch), 1
+ *                       off, 2 whenever the workspace is given. Off when 8
+ *                       dequantizing warps or a cluster split are asked for,
+ *                       or when two accumulators do not fit the tensor
+ *                       memory beside the A buffers (M > 96).
  *  WQ_OPT_TC_KSPLIT     CTAs of a thread-block cluster that share one 128-row
  *                       tile of the tensor-core kernel along K (their fp32
  *                       partial tiles are added in rank order in the first
@@ -396,6 +414,7 @@ int32_t wq_awq_fold_linear_rows(const void* W_dev, const void* b_dev, const void
 #define WQ_OPT_TEST_STALL 14
 #define WQ_OPT_AWQ_LOSS 15
 #define WQ_OPT_TC_KSPLIT 16
+#define WQ_OPT_TC_STREAMK 17
 
 #define WQ_AWQ_LOSS_TWO_KERNELS 0
 #define WQ_AWQ_LOSS_FUSED 1

@@ -110,6 +110,7 @@ def test_option_values_are_validated(wq):
         wq.WQ_OPT_TEST_STALL: ([1, 0], [2, -1]),
         wq.WQ_OPT_AWQ_LOSS: ([1, 0], [2, -1]),
         wq.WQ_OPT_TC_KSPLIT: ([0, 1, 2, 4, 8], [3, 16, -1]),
+        wq.WQ_OPT_TC_STREAMK: ([1, 2, 0], [3, -1]),
     }
     for opt, (good, bad) in cases.items():
         old = wq.wq_get_option(opt)

@@ -265,9 +265,16 @@ def test_unpack_dequant_bit_exact(wq, bits):
 # S5 GEMV (small M)
 # ---------------------------------------------------------------------------
 
-def run_gemm(wq, X, quant_gpu, N, bits, sym=False, group=128):
+def gemm_workspace(wq, M, N, K, bits, group=128):
+    n = wq.wq_gemm_workspace_bytes(M, N, K, bits=bits, group_size=group)
+    assert n > 0
+    return torch.zeros(n, dtype=torch.uint8, device="cuda")  # zero-filled before its first use
+
+
+def run_gemm(wq, X, quant_gpu, N, bits, sym=False, group=128, workspace=None):
     packed, steps, zeros = quant_gpu
-    Y = wq.wq_w4a16_gemm(dev(X), packed, steps, zeros, N, bits=bits, symmetric=sym, group_size=group)
+    Y = wq.wq_w4a16_gemm(dev(X), packed, steps, zeros, N, bits=bits, symmetric=sym, group_size=group,
+                         workspace=workspace)
     assert wq.wq_get_last_device_error() == 0
     return Y.cpu().numpy()
 
@@ -389,14 +396,23 @@ def test_gemv_llama65b_full(wq, gemv_variant, bits):
 
 
 def test_smallm_sweep_full_weight(wq):
-    """K=8192, N=28672 at every M of the sweep, against the fp64 oracle."""
+    """K=8192, N=28672 at every M of the sweep, against the fp64 oracle; M >= 3
+    both without a workspace (one CTA per row tile) and with one (the stream-K
+    schedule: 224 row tiles for 148 SMs), the latter twice (same result)."""
     c = synth.config_smallm_sweep(1)
     (codes, st, z), qg = assert_quant_parity(wq, c.W, None, 4, False)
     D = O.dequantize(codes, st, z, 128)
     for M in synth.SMALLM_SWEEP:
         X = synth.smallm_activations(M)
+        ref = X.astype(np.float64) @ D.T
         Y = run_gemm(wq, X, qg, 28672, 4)
-        assert_close(Y, X.astype(np.float64) @ D.T)
+        assert_close(Y, ref)
+        if M >= 3:
+            ws = gemm_workspace(wq, M, 28672, 8192, 4)
+            Y1 = run_gemm(wq, X, qg, 28672, 4, workspace=ws)
+            Y2 = run_gemm(wq, X, qg, 28672, 4, workspace=ws)
+            assert_close(Y1, ref)
+            assert np.array_equal(Y1.view(np.uint16), Y2.view(np.uint16))
 
 
 # ---------------------------------------------------------------------------
@@ -529,6 +545,74 @@ def test_tc_gemm_dequant_quartets_bits_groups(wq, tc_path, dw, bits, group, M):
     finally:
         wq.wq_set_option(wq.WQ_OPT_TC_DEQUANT_WARPS, 0)
     assert_close(Y, O.gemm_ref(X, codes, st, z, group))
+
+
+@pytest.fixture
+def streamk_forced(wq):
+    wq.wq_set_option(wq.WQ_OPT_TC_STREAMK, 2)
+    yield
+    wq.wq_set_option(wq.WQ_OPT_TC_STREAMK, 0)
+
+
+@pytest.mark.parametrize("bits,group", [(4, 128), (3, 128), (4, 32), (3, 64)])
+@pytest.mark.parametrize("M", [3, 16, 100, 200, 300])
+@pytest.mark.parametrize("NK", [(333, 1152), (1000, 4096), (2000, 2048)])
+def test_tc_gemm_streamk(wq, tc_path, streamk_forced, bits, group, M, NK):
+    """The stream-K schedule forced on small weights: CTAs whose stage ranges
+    start and end inside row tiles (one, two or three contributors per tile),
+    a ragged last tile, two M chunks; the same result on a second call."""
+    N, K = NK
+    g = synth.rng(800 + M + bits + group + N)
+    W = synth.weight(g, N, K, 0.02, channel_frac=0.01, channel_mult=10.0)
+    X = synth.activations(g, M, K, channel_frac=0.01, channel_mult=20.0)
+    codes, st, z = O.quantize_groups(W, bits, group, False)
+    qg = (dev(O.pack_codes(codes, bits).reshape(-1).view(np.int32)), dev(st), dev(z))
+    ws = gemm_workspace(wq, M, N, K, bits, group)
+    Y1 = run_gemm(wq, X, qg, N, bits, group=group, workspace=ws)
+    Y2 = run_gemm(wq, X, qg, N, bits, group=group, workspace=ws)
+    assert_close(Y1, O.gemm_ref(X, codes, st, z, group))
+    assert np.array_equal(Y1.view(np.uint16), Y2.view(np.uint16))
+    assert int(ws[:65536].count_nonzero()) == 0  # the arrival counters are left at zero
+
+
+def test_tc_gemm_streamk_workspace_shared_across_shapes(wq, tc_path, streamk_forced):
+    """One zero-filled workspace serves calls of different shapes in turn: the
+    arrival counters live in a fixed region that each call leaves at zero,
+    away from the partial tiles of any shape."""
+    g = synth.rng(870)
+    shapes = [(16, 2000, 4096), (200, 333, 1152), (64, 4096, 2048), (16, 2000, 4096)]
+    n = max(wq.wq_gemm_workspace_bytes(M, N, K) for M, N, K in shapes)
+    ws = torch.zeros(n, dtype=torch.uint8, device="cuda")
+    for M, N, K in shapes:
+        W = synth.weight(g, N, K, 0.02)
+        X = synth.activations(g, M, K)
+        codes, st, z = O.quantize_groups(W, 4, 128, False)
+        qg = (dev(O.pack_codes(codes, 4).reshape(-1).view(np.int32)), dev(st), dev(z))
+        assert_close(run_gemm(wq, X, qg, N, 4, workspace=ws), O.gemm_ref(X, codes, st, z, 128))
+        assert int(ws[:65536].count_nonzero()) == 0
+
+
+def test_tc_gemm_workspace_rules(wq, tc_path):
+    """A workspace smaller than wq_gemm_workspace_bytes is not used (the
+    per-tile schedule runs); an unaligned one is refused; M < 3 needs none."""
+    N, K, M = 1000, 4096, 16
+    g = synth.rng(850)
+    W = synth.weight(g, N, K, 0.02)
+    X = synth.activations(g, M, K)
+    codes, st, z = O.quantize_groups(W, 4, 128, False)
+    qg = (dev(O.pack_codes(codes, 4).reshape(-1).view(np.int32)), dev(st), dev(z))
+    assert wq.wq_gemm_workspace_bytes(2, N, K) == 0
+    need = wq.wq_gemm_workspace_bytes(M, N, K)
+    small = torch.zeros(need - 256, dtype=torch.uint8, device="cuda")
+    wq.wq_set_option(wq.WQ_OPT_TC_STREAMK, 2)
+    try:
+        assert_close(run_gemm(wq, X, qg, N, 4, workspace=small), O.gemm_ref(X, codes, st, z, 128))
+        big = torch.zeros(need + 512, dtype=torch.uint8, device="cuda")
+        with pytest.raises(wq.WQError) as e:
+            wq.wq_w4a16_gemm(dev(X), *qg, N, bits=4, workspace=big[1:])
+        assert e.value.status == wq.WQ_ERR_ALIGNMENT
+    finally:
+        wq.wq_set_option(wq.WQ_OPT_TC_STREAMK, 0)
 
 
 def test_tc_gemm_symmetric_and_closed_form(wq, tc_path):

@@ -102,6 +102,7 @@ WQ_OPT_WAIT_LIMIT_MS = 13
 WQ_OPT_TEST_STALL = 14
 WQ_OPT_AWQ_LOSS = 15
 WQ_OPT_TC_KSPLIT = 16
+WQ_OPT_TC_STREAMK = 17
 WQ_AWQ_LOSS_TWO_KERNELS = 0
 WQ_AWQ_LOSS_FUSED = 1
 

@@ -69,6 +69,7 @@ std::atomic<int64_t> g_opt_tc_stages{0};
 std::atomic<int64_t> g_opt_gemv_grid{1};
 std::atomic<int64_t> g_opt_tc_bk{0};
 std::atomic<int64_t> g_opt_tc_dequant_warps{0};
+std::atomic<int64_t> g_opt_tc_streamk{0};
 std::atomic<int64_t> g_opt_wait_limit_ms{2000};
 std::atomic<int64_t> g_opt_test_stall{0};
 std::atomic<int64_t> g_opt_awq_loss{WQ_AWQ_LOSS_FUSED};
@@ -130,8 +131,8 @@ int32_t wq_unpack_dequant(const uint32_t* packed, const void* steps, const void*
 }
 
 size_t wq_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, const wq_quant_cfg* cfg) {
-  (void)M; (void)N; (void)K; (void)cfg;
-  return 0;
+  if (check_cfg(cfg) != WQ_OK || check_shape(N, K) != WQ_OK || M < 3) return 0;
+  return wq::gemm_tc_workspace_bytes(M, N, K, cfg->bits);
 }
 
 // SMs of the current device (cached per process; one device type per process).
@@ -151,13 +152,13 @@ int32_t wq_w4a16_gemm(const void* X, const uint32_t* packed, const void* steps, 
                       int64_t N, int64_t K, const wq_quant_cfg* cfg, void* Y, void* workspace,
                       size_t workspace_bytes, void* stream) {
   NvtxRange nvtx_range("wq_w4a16_gemm");
-  (void)workspace; (void)workspace_bytes;
   int32_t st = check_cfg(cfg);
   if (st != WQ_OK) return st;
   if ((st = check_shape(N, K)) != WQ_OK) return st;
   if (M < 1 || M > (int64_t)INT32_MAX / 2) return WQ_ERR_INVALID_ARG;
   if (!X || !packed || !steps || !zeros || !Y) return WQ_ERR_INVALID_ARG;
-  if (!aligned(X, 16) || !aligned(packed, 16) || !aligned(steps, 2) || !aligned(zeros, 2) || !aligned(Y, 2))
+  if (!aligned(X, 16) || !aligned(packed, 16) || !aligned(steps, 2) || !aligned(zeros, 2) || !aligned(Y, 2) ||
+      (workspace && !aligned(workspace, 256)))
     return WQ_ERR_ALIGNMENT;
   // one reading of every option this call uses
   const int64_t path = g_opt_gemm_path, variant = g_opt_gemv_variant, pdl = g_opt_pdl;
@@ -183,6 +184,7 @@ int32_t wq_w4a16_gemm(const void* X, const uint32_t* packed, const void* steps, 
     return cuda_status(wq::launch_gemm_tc(X, packed, steps, zeros, M, N, K, cfg->bits, group, Y, flag,
                                           static_cast<cudaStream_t>(stream), (int)g_opt_tc_stages,
                                           (int)g_opt_tc_bk, (int)g_opt_tc_dequant_warps, (int)g_opt_tc_ksplit,
+                                          (int)g_opt_tc_streamk, workspace, workspace ? workspace_bytes : 0,
                                           (int)g_opt_wait_limit_ms, g_opt_test_stall != 0));
   }
   if (rows_ok)
@@ -394,6 +396,10 @@ int32_t wq_set_option(int32_t option, int64_t value) {
       if (value != 0 && value != 1 && value != 2 && value != 4 && value != 8) return WQ_ERR_INVALID_ARG;
       g_opt_tc_ksplit = value;
       return WQ_OK;
+    case WQ_OPT_TC_STREAMK:
+      if (value != 0 && value != 1 && value != 2) return WQ_ERR_INVALID_ARG;
+      g_opt_tc_streamk = value;
+      return WQ_OK;
     case WQ_OPT_TC_DEQUANT_WARPS:
       if (value != 0 && value != 4 && value != 8) return WQ_ERR_INVALID_ARG;
       g_opt_tc_dequant_warps = value;
@@ -435,6 +441,7 @@ int64_t wq_get_option(int32_t option) {
     case WQ_OPT_PDL: return g_opt_pdl;
     case WQ_OPT_AWQ_LOSS: return g_opt_awq_loss;
     case WQ_OPT_TC_KSPLIT: return g_opt_tc_ksplit;
+    case WQ_OPT_TC_STREAMK: return g_opt_tc_streamk;
   }
   return -1;
 }

@@ -21,7 +21,10 @@ cudaError_t launch_gemv_rows(const void* X, const uint32_t* packed, const void* 
                              bool act_int, int grid_mode, bool pdl);
 cudaError_t launch_gemm_tc(const void* X, const uint32_t* packed, const void* steps, const void* zeros, int64_t M,
                            int64_t N, int64_t K, int bits, int group, void* Y, int* err, cudaStream_t st,
-                           int stages_opt, int bk_opt, int dw_opt, int ksplit_opt, int wait_ms, bool stall);
+                           int stages_opt, int bk_opt, int dw_opt, int ksplit_opt, int streamk_opt, void* workspace,
+                           size_t workspace_bytes, int wait_ms, bool stall);
+// Workspace for the tensor-core kernel's stream-K schedule (M rows of X).
+size_t gemm_tc_workspace_bytes(int64_t M, int64_t N, int64_t K, int bits);
 // Workspace layout of the AWQ search (wq_awq.cu): mu, the candidate scales,
 // the per-tile partial losses, and (two-kernel loss path only) the error
 // matrices of one batch of alphas.
