@@ -727,7 +727,10 @@ static long rows_grid(long nbatch, int occ, int mode) {
 template <int M, int R, int CPL, int S, int BITS, template <int, int> class Act, int GS>
 static cudaError_t launch_rows(const RowsArgs& a, cudaStream_t st, bool pdl, int grid_mode) {
   const int nseg = (a.K + 1024 * CPL - 1) / (1024 * CPL);
-  auto kern = gemv_rows_kernel<M, R, CPL, S, BITS, Act, M == 1 ? (CPL == 1 && S == 2 ? 3 : 2) : 1, GS>;
+  // W4A8 with several rows of X: capped at 128 registers (two CTAs per SM);
+  // W4A16 at M > 1 would spill under a cap
+  constexpr bool kW4A8 = std::is_same<Act<M, CPL>, ActW4A8<M, CPL>>::value;
+  auto kern = gemv_rows_kernel<M, R, CPL, S, BITS, Act, M == 1 ? (CPL == 1 && S == 2 ? 3 : 2) : (kW4A8 ? 2 : 1), GS>;
   const int threads = 32 * nseg;
   const size_t smem = 2 * (size_t)32 * nseg * sizeof(float);  // [2][32/NV][nseg][NV]
   int occ = 0;
