@@ -727,10 +727,13 @@ static long rows_grid(long nbatch, int occ, int mode) {
 template <int M, int R, int CPL, int S, int BITS, template <int, int> class Act, int GS>
 static cudaError_t launch_rows(const RowsArgs& a, cudaStream_t st, bool pdl, int grid_mode) {
   const int nseg = (a.K + 1024 * CPL - 1) / (1024 * CPL);
-  // W4A8 with several rows of X: capped at 128 registers (two CTAs per SM);
-  // W4A16 at M > 1 would spill under a cap
+  // W4A8 with several rows of X, and the fp32-offset-sum kernel at M = 2 with
+  // 32 channels per lane and two stages: capped at 128 registers (two CTAs per
+  // SM, no spills); the other M > 1 instances would spill under the cap
   constexpr bool kW4A8 = std::is_same<Act<M, CPL>, ActW4A8<M, CPL>>::value;
-  auto kern = gemv_rows_kernel<M, R, CPL, S, BITS, Act, M == 1 ? (CPL == 1 && S == 2 ? 3 : 2) : (kW4A8 ? 2 : 1), GS>;
+  constexpr bool kHalf2x32 = std::is_same<Act<M, CPL>, ActHalf<M, CPL>>::value && M == 2 && CPL == 1 && S == 2;
+  constexpr int kMinB = M == 1 ? (CPL == 1 && S == 2 ? 3 : 2) : (kW4A8 || kHalf2x32) ? 2 : 1;
+  auto kern = gemv_rows_kernel<M, R, CPL, S, BITS, Act, kMinB, GS>;
   const int threads = 32 * nseg;
   const size_t smem = 2 * (size_t)32 * nseg * sizeof(float);  // [2][32/NV][nseg][NV]
   int occ = 0;
@@ -821,10 +824,12 @@ cudaError_t launch_gemv_rows(const void* X, const uint32_t* packed, const void* 
   // measured fastest: at M = 1, (4, 32, 2) under an 85-register cap for
   // 4096-channel rows and for 8192-channel rows of at most 2^27 weights (more
   // CTAs per SM), else (4, 64, 2) (fewer cross-warp sums per weight); at
-  // M = 2, (4, 32, 3) for 4096-channel rows, else (4, 64, 2)
+  // M = 2, (4, 32, 2) under a 128-register cap up to 8192-channel rows
+  // (8192 x 28672: 39.5 us against 41.3 with (4, 64, 2); 11008 x 4096: 9.8
+  // against 12.3), else (4, 64, 2)
   if (shape == 0) {
     if (M == 1) shape = (K <= 4096 || (K <= 8192 && N * K <= (int64_t(1) << 27))) ? 1 : 2;
-    else shape = K <= 4096 ? 4 : 2;
+    else shape = K <= 8192 ? 1 : 2;
   }
   if (K > 8192 && (shape == 1 || shape == 4)) shape = 2;  // at most 8 warps
   if (group == 32)
