@@ -83,6 +83,9 @@ def test_argument_validation_without_gpu(wq):
     assert L.wq_w4a16_gemm(good, good, good, good, 1, 8, 256, by(c), None, None, 0, None) == wq.WQ_ERR_INVALID_ARG
     assert L.wq_unpack_dequant(good, good, good, 8, 256, by(_cfg(wq, bits=6)), good, None) == wq.WQ_ERR_UNSUPPORTED
     assert wq.wq_gemm_workspace_bytes(1, 4096, 4096) == 0
+    # an unaligned workspace is refused before anything is launched
+    assert L.wq_w4a16_gemm(good, good, good, good, 16, 8, 256, by(c), good, good + 8, 1 << 20, None) == \
+        wq.WQ_ERR_ALIGNMENT
     # scale folding
     assert L.wq_awq_fold_norm(None, good, 8, good, None) == wq.WQ_ERR_INVALID_ARG
     assert L.wq_awq_fold_norm(good, good, 0, good, None) == wq.WQ_ERR_INVALID_ARG
@@ -279,3 +282,18 @@ def test_awq_workspace_follows_the_loss_path(wq):
     batch = min(20, (1 << 30) // (sum(Ns) * K * 2))
     assert two - fused == batch * sum(Ns) * K * 2
     assert 0 < fused < 8 << 20
+
+
+def test_gemm_workspace_size_is_its_layout(wq):
+    """The tensor-core kernel's stream-K workspace: 64 KB of arrival counters,
+    then two fp32 partial tiles (128 rows x M rounded up to 16) per CTA of the
+    persistent grid (two CTAs per SM on 148 SMs, at most half the stage
+    units); none for M < 3 (the row GEMV)."""
+    sms = 148
+    for M, N, K, cps in ((16, 28672, 8192, 2), (4, 8192, 8192, 2), (16, 1000, 4096, 2)):
+        BN = (M + 15) // 16 * 16
+        units = (N + 127) // 128 * (K // 128)
+        P = min(cps * sms, units // 2)
+        assert wq.wq_gemm_workspace_bytes(M, N, K) == 65536 + P * 2 * 128 * BN * 4
+    assert wq.wq_gemm_workspace_bytes(2, 28672, 8192) == 0
+    assert wq.wq_gemm_workspace_bytes(16, 28672, 8192, group_size=48) == 0  # invalid configuration

@@ -24,12 +24,23 @@
 //             takes the stages kt = h mod NH, so NH stages are dequantized at
 //             once), then run the epilogue (tcgen05.ld -> fp16 -> Y).
 // The shared-memory ring and the TMEM A ring are separate, so the TMA runs as
-// far ahead as shared memory allows while only two A buffers occupy TMEM.
-// Split K: when the row tiles cannot fill the GPU (N = 8192 gives 64 tiles
-// for 148 SMs), the KS CTAs of a thread-block cluster take consecutive K
-// ranges of the same tile; ranks 1.. send their fp32 partial tiles to rank 0's
-// shared memory (its idle ring) over distributed shared memory, and rank 0
-// adds them in rank order (deterministic) and writes Y.
+// far ahead as shared memory allows while only two or three A buffers occupy
+// TMEM.
+// Schedules:
+//   per tile  one CTA per 128-row tile; when the row tiles cannot fill the
+//             GPU (N = 8192 gives 64 tiles for 148 SMs), the KS CTAs of a
+//             thread-block cluster take consecutive K ranges of the same
+//             tile; ranks 1.. send their fp32 partial tiles to rank 0's
+//             shared memory (its idle ring) over distributed shared memory,
+//             and rank 0 adds them in rank order (deterministic) and writes Y.
+//   stream-K  (SK, with a caller workspace) a persistent grid; CTA c takes the
+//             (tile, stage) units [c U / P, (c + 1) U / P), at most one
+//             tile's worth: the end of one tile and the start of the next,
+//             each accumulated in its own TMEM columns. Partial tiles go to
+//             the workspace; per tile and lane quarter, the warp that arrives
+//             last at a counter adds all contributors' tiles in CTA order
+//             (deterministic), writes Y and zeroes the counter. No CTA waits
+//             for another.
 // Every mbarrier wait is bounded; on a timeout the kernel latches
 // WQ_ERR_TIMEOUT, drains its own copies, frees its tensor memory and returns.
 #include <cooperative_groups.h>
