@@ -164,3 +164,26 @@ def test_dequant_as_one_fma_is_exact():
     want = offs[:, None] * steps[None, :]
     assert np.array_equal(fused, want)
     assert np.array_equal(want.astype(np.float32).astype(np.float64), want)
+
+
+def _fp16_finite_nonzero():
+    v = np.arange(0, 0x10000, dtype=np.uint32).astype(np.uint16).view(np.float16).astype(np.float64)
+    return v[np.isfinite(v) & (v != 0)]
+
+
+def test_corrected_quotient_fold_operands():
+    """AWQ scale folding divides an fp16 weight (norm weight, linear row or
+    bias) by an fp16 scale with the same correction: any finite nonzero fp16
+    divisor of either sign (subnormals included) and any finite fp16 dividend
+    must give RN(w / s) exactly."""
+    rng = random.Random(13)
+    vals = _fp16_finite_nonzero()
+    small = vals[np.abs(vals) < 2.0 ** -14]  # the subnormals
+    for i in range(4000):
+        s = float(rng.choice(small if i % 5 == 0 else vals))
+        w = float(rng.choice(small if i % 7 == 0 else vals))
+        assert corrected_quotient_ok(w, s), (w, s)
+    # the extreme magnitudes
+    for w in (65504.0, -65504.0, 2.0 ** -24, -(2.0 ** -24), 1.0):
+        for s in (2.0 ** -24, -(2.0 ** -24), 65504.0, -65504.0, 3.0, 2.0 ** -14):
+            assert corrected_quotient_ok(w, s), (w, s)

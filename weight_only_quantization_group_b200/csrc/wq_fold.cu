@@ -6,20 +6,34 @@
 //   fold into a linear's rows      W'[n][k] = W[n][k] / s_n,       (s along rows)
 //                                  b'_n = b_n / s_n
 //
-// Stored form: fp16_rn(fp32 quotient) -- one IEEE fp32 division (__fdiv_rn)
-// and one rounding to fp16, the contract the oracle restates. A result that is
-// not finite in fp16 latches WQ_ERR_RANGE. HBM-bound: 2 B read + 2 B written
-// per element (+ the scale, from L1/L2); one wave of resident CTAs walks
-// 16-byte chunks grid-stride.
+// Stored form: fp16_rn(fp32 quotient) -- the correctly rounded fp32 quotient
+// and one rounding to fp16, the contract the oracle restates. The quotient is
+// formed without a division instruction: q0 = fl(w y) with y = rcp_refined(s),
+// r = w - s q0 (exact), q = fl(q0 + r y), Markstein's correction, exact for an
+// fp16 divisor (11 significant bits) and any fp32 dividend in this range (the
+// argument at group_quotient; checked in exact rational arithmetic for fp16
+// weights and scales of both signs, subnormals included). r = 0 keeps q0
+// itself, so a zero quotient keeps the sign of w / s; infinite or NaN operands
+// and a zero divisor take the IEEE division. A result that is not finite in
+// fp16 latches WQ_ERR_RANGE. HBM-bound: 2 B read + 2 B written per element
+// (+ the scale, from L1/L2); one wave of resident CTAs walks 16-byte chunks
+// grid-stride.
 #include "wq_common.cuh"
 #include "wq_launch.h"
+#include "wq_quant_core.cuh"
 
 namespace wq {
 
-__device__ __forceinline__ __half fold_one(__half w, float s, bool& bad) {
-  const __half q = __float2half_rn(__fdiv_rn(__half2float(w), s));
-  bad |= __hisinf(q) || __hisnan(q);
-  return q;
+// y: rcp_refined(s)
+__device__ __forceinline__ __half fold_one(__half wh, float s, float y, bool& bad) {
+  const float w = __half2float(wh);
+  const float q0 = __fmul_rn(w, y);
+  const float r = __fmaf_rn(-q0, s, w);
+  float q = r == 0.0f ? q0 : __fmaf_rn(r, y, q0);
+  if (!isfinite(q)) q = __fdiv_rn(w, s);  // infinite or NaN operands, zero divisor
+  const __half h = __float2half_rn(q);
+  bad |= __hisinf(h) || __hisnan(h);
+  return h;
 }
 
 // out[r][c] = in[r][c] / s[ROW_AXIS ? r : c] for an [R][C] fp16 matrix; C % 8
@@ -39,13 +53,17 @@ __global__ void __launch_bounds__(256) fold_vec_kernel(const __half* in, const _
     __half* oh = reinterpret_cast<__half*>(&o);
     if constexpr (ROW_AXIS) {
       const float sv = __half2float(s[i / cpr]);
+      const float y = rcp_refined(sv);
 #pragma unroll
-      for (int j = 0; j < 8; ++j) oh[j] = fold_one(h[j], sv, bad);
+      for (int j = 0; j < 8; ++j) oh[j] = fold_one(h[j], sv, y, bad);
     } else {
       const uint4 sr = *reinterpret_cast<const uint4*>(s + 8 * (i % cpr));
       const __half* sh = reinterpret_cast<const __half*>(&sr);
 #pragma unroll
-      for (int j = 0; j < 8; ++j) oh[j] = fold_one(h[j], __half2float(sh[j]), bad);
+      for (int j = 0; j < 8; ++j) {
+        const float sv = __half2float(sh[j]);
+        oh[j] = fold_one(h[j], sv, rcp_refined(sv), bad);
+      }
     }
     *reinterpret_cast<uint4*>(out + 8 * i) = o;
   }
@@ -58,7 +76,10 @@ __global__ void __launch_bounds__(256) fold_scalar_kernel(const __half* in, cons
                                                           __half* out, int64_t R, int64_t C, int* err) {
   bool bad = false;
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < R * C; i += (int64_t)gridDim.x * blockDim.x)
-    out[i] = fold_one(in[i], __half2float(s[ROW_AXIS ? i / C : i % C]), bad);
+  {
+    const float sv = __half2float(s[ROW_AXIS ? i / C : i % C]);
+    out[i] = fold_one(in[i], sv, rcp_refined(sv), bad);
+  }
   if (bad) latch_error(err, WQ_ERR_RANGE);
 }
 
