@@ -340,8 +340,8 @@ int32_t wq_awq_fold_linear_rows(const void* W_dev, const void* b_dev, const void
  *  WQ_OPT_GEMV_ROWS_SHAPE  rows per batch R, input channels per lane C and
  *                       register stages S of the row-streaming kernel:
  *                       0 default (M = 1: shape 1 for K <= 4096 and for
- *                       K <= 8192 with N*K <= 2^27, else 2; M = 2: shape 4 for
- *                       K <= 4096, else 2), 1 (4, 32, 2),
+ *                       K <= 8192 with N*K <= 2^27, else 2; M = 2: shape 1
+ *                       for K <= 8192, else 2; M = 3, 4: shape 1), 1 (4, 32, 2),
  *                       2 (4, 64, 2), 3 (2, 64, 2), 4 (4, 32, 3). Shapes with
  *                       C = 32 apply for K <= 8192; above it shape 2 runs.
  *  WQ_OPT_GEMV_GRID     grid of the row-streaming kernel (all CTAs resident, CTA c
