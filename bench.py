@@ -1052,6 +1052,8 @@ def run_case(args):
     wq.wq_set_option(wq.WQ_OPT_GEMV_KERNEL, wq.WQ_GEMV_KERNEL_TILED if args.gemv_variant == "tiled"
                      else wq.WQ_GEMV_KERNEL_AUTO)
     wq.wq_set_option(wq.WQ_OPT_GEMV_ROWS_SHAPE, args.rows_shape)
+    wq.wq_set_option(wq.WQ_OPT_AWQ_LOSS, wq.WQ_AWQ_LOSS_TWO_KERNELS if args.awq_loss == "two"
+                     else wq.WQ_AWQ_LOSS_FUSED)
     q = wq.wq_quantize_pack(W, bits=args.bits, group_size=args.group)
     Y = torch.empty((args.M, args.N), dtype=torch.float16, device=dev)
     ws = None
@@ -1122,6 +1124,8 @@ def main():
     ap.add_argument("--path", choices=["auto", "gemv", "tc"], default="auto")
     ap.add_argument("--gemv-variant", choices=["int", "offset", "exact", "tiled"], default="offset")
     ap.add_argument("--rows-shape", type=int, default=0, choices=list(range(5)))
+    ap.add_argument("--awq-loss", choices=["fused", "two"], default="fused",
+                    help="--case awq: loss GEMM with on-chip error tiles, or error matrix + loss GEMM")
     ap.add_argument("--oracle-table", default=None,
                     help="only time the oracle on the host cores for each workload of the result table "
                          "and write the milliseconds to this JSON file")
