@@ -108,6 +108,16 @@ def profiled_traffic(kernel: str):
     return e.get("dram_bytes_per_launch")
 
 
+def gpu_uuid(index: int) -> str | None:
+    """The CUDA device's UUID (to find the same GPU through NVML), or None."""
+    try:
+        import torch
+        u = getattr(torch.cuda.get_device_properties(index), "uuid", None)
+        return str(u) if u is not None else None
+    except Exception:
+        return None
+
+
 def max_over_ranks(ms: float, world: int, device) -> float:
     """The slowest rank's time: every rank reports its own device time and all
     take the maximum (the same collective on every rank, in the same order)."""
@@ -121,16 +131,32 @@ def max_over_ranks(ms: float, world: int, device) -> float:
 
 
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons sampled every 200 ms."""
+    """SM clocks and throttle reasons while the timed steps run: nvidia-smi
+    every 200 ms, one nvidia-smi reading on each side of the region, and an
+    NVML thread reading the clock and the active event reasons every 100 us
+    (a timed region of a millisecond sees no periodic nvidia-smi sample).
+    Read-only: nothing here changes a setting of the GPU."""
 
     QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    # NVML clocks-event reason bits (nvml.h, nvmlClocksEventReason*), by the
+    # names the summary reports
+    NVML_REASONS = {"sw_power_cap": 0x4, "hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20,
+                    "hw_thermal_slowdown": 0x40, "hw_power_brake_slowdown": 0x80}
 
-    def __init__(self, gpu_index: int):
+    def __init__(self, gpu_index: int, uuid: str | None = None, nvml=None, period_s: float = 100e-6):
         self.gpu = gpu_index
+        self.uuid = uuid
         self.proc = None
         self.lines = []
+        self.nvml = nvml            # the pynvml module (injected by tests), else imported on entry
+        self.period = period_s
+        self.nvml_sm = []           # SM MHz per NVML sample
+        self.nvml_reasons = set()
+        self.nvml_max = None
+        self._thread = None
+        self._stop = None
 
     def _once(self):
         """One immediate sample (a short timed region may see no periodic one)."""
@@ -141,6 +167,48 @@ class ClockSampler:
         except (OSError, subprocess.SubprocessError):
             pass
 
+    def _nvml_handle(self, nv):
+        """The NVML device of this rank's CUDA device: matched by UUID (NVML
+        does not follow CUDA_VISIBLE_DEVICES), else by index."""
+        if self.uuid:
+            want = self.uuid.lower().removeprefix("gpu-")
+            for i in range(nv.nvmlDeviceGetCount()):
+                h = nv.nvmlDeviceGetHandleByIndex(i)
+                u = nv.nvmlDeviceGetUUID(h)
+                u = (u.decode() if isinstance(u, bytes) else u).lower().removeprefix("gpu-")
+                if u == want:
+                    return h
+        return nv.nvmlDeviceGetHandleByIndex(self.gpu)
+
+    def _poll(self, nv, h):
+        while not self._stop.is_set():
+            try:
+                sm = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+                bits = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+            except Exception:
+                return
+            self.nvml_sm.append(float(sm))
+            for nm, b in self.NVML_REASONS.items():
+                if bits & b:
+                    self.nvml_reasons.add(nm)
+            time.sleep(self.period)
+
+    def _start_nvml(self):
+        import threading
+        nv = self.nvml
+        try:
+            if nv is None:
+                import pynvml as nv
+            nv.nvmlInit()
+            h = self._nvml_handle(nv)
+            self.nvml_max = float(nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM))
+        except Exception:
+            return
+        self.nvml = nv
+        self._stop = threading.Event()
+        self._thread = threading.Thread(target=self._poll, args=(nv, h), daemon=True)
+        self._thread.start()
+
     def __enter__(self):
         self._once()
         try:
@@ -149,9 +217,17 @@ class ClockSampler:
                  "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except OSError:
             self.proc = None
+        self._start_nvml()
         return self
 
     def __exit__(self, *exc):
+        if self._thread is not None:
+            self._stop.set()
+            self._thread.join(timeout=5)
+            try:
+                self.nvml.nvmlShutdown()
+            except Exception:
+                pass
         if self.proc is not None:
             self.proc.terminate()
             try:
@@ -178,10 +254,16 @@ class ClockSampler:
             for nm, v in zip(names, f[5:9]):
                 if v.lower() == "active":
                     reasons.add(nm)
-        if not sm:
-            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": 0}
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
-                "samples": len(sm)}
+        smi_samples = len(sm)
+        sm += self.nvml_sm
+        reasons |= self.nvml_reasons
+        if mx is None:
+            mx = self.nvml_max
+        out = {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx, "reasons": sorted(reasons),
+               "samples": len(sm), "nvml_samples": len(self.nvml_sm), "smi_samples": smi_samples}
+        if self.nvml_sm:
+            out["sm_mhz_min"] = min(self.nvml_sm)
+        return out
 
 
 # ---------------------------------------------------------------------------
@@ -257,7 +339,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     barrier()
     torch.cuda.synchronize()
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with ClockSampler(local_rank) as clk:
+    with ClockSampler(local_rank, gpu_uuid(local_rank)) as clk:
         ev0.record(stream)
         for i in range(args.steps):
             run_step(i)
