@@ -11,10 +11,11 @@
  * ---------------------------------------
  *  - W is an nn.Linear weight: [N][K] row-major fp16 (N output channels, K
  *    input channels). X is [M][K] row-major fp16, Y is [M][N] row-major fp16.
- *  - A group is `group_size` (= 128) consecutive input channels of one
- *    output row ("Quantising Large Language Models for Efficient Inference",
- *    section "Post-training methods for 4-bit weights": one scale and zero
- *    point per group of 64-128 weights within a row).
+ *  - A group is `group_size` (32, 64 or 128) consecutive input channels of
+ *    one output row ("Quantising Large Language Models for Efficient
+ *    Inference", section "Post-training methods for 4-bit weights": one scale
+ *    and zero point per group of 64-128 weights within a row; the Lab 5 linear
+ *    of "MIT 6.5940 Lab 4 + Lab 5" uses 32).
  *  - Pointers named *_dev are device pointers the caller allocated (e.g. torch
  *    tensors' data_ptr()). The library never frees or retains them.
  *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default
@@ -59,9 +60,15 @@
  *         and bit b of k = 31 is bit 31 of word b. Exactly 3 bits per weight.
  *  steps, zeros: fp16 [N][K/group_size] row-major.
  *
- * Supported: bits in {3, 4}; group_size == 128; K % 128 == 0; N >= 1;
- * M >= 1. Device pointers must be 16-byte aligned (weights, X, packed words)
- * or 4-byte aligned (steps, zeros, Y, s, mu). Inputs must be finite.
+ * Rows are independent: linears that read the same input (q|k|v, gate|up)
+ * can be packed as one weight by concatenating their packed rows, steps and
+ * zeros along N; one wq_w4a16_gemm call then writes all their outputs, in the
+ * same column order, with fewer launches than one call per linear.
+ *
+ * Supported: bits in {3, 4}; group_size in {32, 64, 128} (the AWQ search:
+ * 128); K % 128 == 0; N >= 1; M >= 1. Device pointers must be 16-byte aligned
+ * (weights, X, packed words) or 4-byte aligned (steps, zeros, Y, s, mu).
+ * Inputs must be finite.
  */
 #ifndef WQ_H_
 #define WQ_H_
@@ -78,7 +85,7 @@ extern "C" {
 typedef enum wq_status {
   WQ_OK = 0,
   WQ_ERR_INVALID_ARG = 1,  /* null pointer, non-positive size, bad config  */
-  WQ_ERR_UNSUPPORTED = 2,  /* valid but not implemented (e.g. group != 128) */
+  WQ_ERR_UNSUPPORTED = 2,  /* valid but not implemented (e.g. 2 or 8 bits)  */
   WQ_ERR_ALIGNMENT = 3,    /* a pointer is not aligned as required          */
   WQ_ERR_CUDA = 4,         /* a CUDA runtime call or launch failed          */
   WQ_ERR_TIMEOUT = 5,      /* device: a bounded wait gave up                */
@@ -88,7 +95,7 @@ typedef enum wq_status {
 
 typedef struct wq_quant_cfg {
   int32_t bits;        /* 3 or 4                                   */
-  int32_t group_size;  /* 128                                      */
+  int32_t group_size;  /* 32, 64 or 128                            */
   int32_t symmetric;   /* 0: asymmetric zero point, 1: symmetric   */
 } wq_quant_cfg;
 
@@ -174,8 +181,9 @@ int32_t wq_w4a16_gemm(const void* X_dev, const uint32_t* packed_dev, const void*
  * squares are summed in fp64 in a fixed order, so results are deterministic.
  * Against fp64 the losses come out low by about 2e-9 * K relative -- the
  * accumulator rounds toward zero -- nearly the same for every alpha).
- * Writes s_out_dev (fp16 [K]) = s_best with best = the first index of the
- * smallest L_j; optionally mu_out_dev (fp64 [K]), loss_out_dev (fp64
+ * cfg->group_size must be 128 (the pages' AWQ setting; else
+ * WQ_ERR_UNSUPPORTED). Writes s_out_dev (fp16 [K]) = s_best with best = the
+ * first index of the smallest L_j; optionally mu_out_dev (fp64 [K]), loss_out_dev (fp64
  * [n_alpha]) and best_out_dev (int32, device). Quantize the weights with
  * wq_quantize_pack(W, s_out) and feed the matmul X * diag(s)^-1 afterwards.
  * workspace_dev: >= wq_awq_workspace_bytes(...) bytes, 256-byte aligned, no
