@@ -16,27 +16,38 @@
 //     is computed (two register stages); the first batch is requested before
 //     the programmatic-dependent-launch wait, since only X depends on the
 //     previous kernel.
-//   * Per batch the R x M partials are reduced across lanes with a butterfly
-//     that halves the value count at each exchange. Across warps they are
-//     summed through shared memory in warp order (deterministic), once per
-//     32/(R*M) batches, so the CTA meets at a barrier only that often.
+//   * Per batch the R x M partials are reduced across lanes with butterflies
+//     that halve the value count at each exchange. For ActHalf and ActHalf3
+//     the halvings run over the lanes of one quantization group first, so the
+//     step, the zero point and the 1024 offsets are applied once per group
+//     total (group-first reduction); the remaining lane bits finish the sum.
+//     ActInt and ActW4A8 scale per lane (their scales are per lane) before
+//     the reduction.
+//     Across warps the totals meet in shared memory in warp order
+//     (deterministic), once per 32/(R*M) batches, so the CTA meets at a
+//     barrier only that often.
 //
-// Two ways to form a lane's sum_k x_k (q_k - zero) over its channels:
-//   ActInt (WQ_GEMV_INT_DIGITS): the lane's activations become one 24-bit fixed-point
-//     image x_k ~ X_k 2^-F (F per lane and row of X, |X_k| < 2^22, so every
-//     fp16 value within 2^-13 of the lane's largest is exact and the others
-//     are rounded by at most 2^-23 of it), split into three base-256 digits.
-//     A packed code word masked with 0xF0F0F0F0 -- before and after a 4-bit
-//     shift -- holds 16 q of four channels in its bytes, and dp4a multiplies
-//     them by four digits at once. Every product and sum is an exact
-//     integer; the zero point is removed per digit in integers, and the only
-//     roundings are the fixed-point image and the final fp32 combination of
-//     three digit sums per row and lane.
-//   ActHalf (default, WQ_GEMV_OFFSET_SUMS): one LOP3 with 0x6400 in both fp16 lanes gives (1024 + q,
-//     1024 + q') or (1024 + 16q, 1024 + 16q'); a mixed fp16 x fp16 -> fp32
-//     FMA multiplies it by the activation pair (exact products, fp32 sums).
-//     The offsets and the zero point are removed per row with the lane's
-//     activation class sums.
+// Activation classes (how a lane forms its sum over its channels):
+//   ActHalf (4-bit, default, WQ_GEMV_OFFSET_SUMS): one LOP3 with 0x6400 in
+//     both fp16 lanes gives (1024 + q, 1024 + q') or (1024 + 16q,
+//     1024 + 16q'); a mixed fp16 x fp16 -> fp32 FMA multiplies it by the
+//     activation pair (exact products, fp32 sums). The offsets and the zero
+//     point are removed per group total with the lane's activation class
+//     sums.
+//   ActHalf3 (3-bit): the same with pairs (1024 + q * {1, 8, 64}) taken from
+//     three words per 32 channels.
+//   ActInt (4-bit, WQ_GEMV_INT_DIGITS): the lane's activations become one
+//     24-bit fixed-point image x_k ~ X_k 2^-F (F per lane and row of X,
+//     |X_k| < 2^22, so every fp16 value within 2^-13 of the lane's largest is
+//     exact and the others are rounded by at most 2^-23 of it), split into
+//     three base-256 digits. A packed code word masked with 0xF0F0F0F0 --
+//     before and after a 4-bit shift -- holds 16 q of four channels in its
+//     bytes, and dp4a multiplies them by four digits at once. Every product
+//     and sum is an exact integer; the zero point is removed per digit in
+//     integers, and the only roundings are the fixed-point image and the
+//     final fp32 combination of three digit sums per row and lane.
+//   ActW4A8 (W4A8): int8 activation codes permuted to the packed byte order,
+//     exact dp4a group dot products, scaled by step / multiplier per lane.
 #include <type_traits>
 
 #include "wq_common.cuh"
