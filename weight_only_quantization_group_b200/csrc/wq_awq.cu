@@ -11,14 +11,15 @@
 // Pipeline, all on the caller's stream:
 //   absmean      mu_k = sum_t |x_tk| / T        (fp64; the sum is exact)
 //   candidates   s_j,k = fp16_rn(max(mu_k, 2^-14) ^ alpha_j)
-//   per batch of alphas:
-//     awq_error  E_j = W - Q(W diag s_j) diag(s_j)^-1, fp16, every linear of
-//                the group stacked row-wise (same decision code as the packer)
+//   loss (default): one launch of awq_loss_fused, a tcgen05 GEMM that builds
+//                each tile of E_j = W - Q(W diag s_j) diag(s_j)^-1 in shared
+//                memory (same decision code as the packer) and sums the
+//                squares of D = E_j X^T in fp64: no E in global memory, one
+//                partial per (alpha, row tile, 512-token chunk)
+//   loss (two-kernel option, WQ_OPT_AWQ_LOSS), per batch of alphas:
+//     awq_error  E_j in fp16, every linear of the group stacked row-wise
 //     awq_loss   tcgen05 GEMM D = E_j X^T per 128x128 tile, epilogue sums D^2
 //                in fp64 -> one partial per (alpha, tile)
-//   (or, with the fused loss option, one launch of awq_loss_fused, which
-//    builds each E tile in shared memory inside the GEMM: no E in global
-//    memory, one partial per (alpha, row tile, 512-token chunk))
 //   finalize     L_j = sum of the partials, one warp per alpha in a fixed
 //                order (deterministic), first argmin, s_out = s_best
 #include <cstring>

@@ -1,4 +1,8 @@
-// S5: W4A16 / W3A16 decode GEMV for small M (1..8 rows of X per launch).
+// S5': W4A16 / W3A16 decode GEMV for small M (1..8 rows of X per launch),
+// the fallback behind the row-streaming kernel (wq_gemv_rows.cu): taken when
+// the GEMV path runs a call that kernel does not take (K > 16384,
+// WQ_GEMV_EXACT, more rows of X than its instances hold) or when forced with
+// WQ_GEMV_KERNEL_TILED; groups of 128.
 //
 // Single-batch decode is a GEMV and is bound by the bytes of weight it must
 // stream ("MIT 6.5940 Lab 4 + Lab 5", "Starting point and setup": the

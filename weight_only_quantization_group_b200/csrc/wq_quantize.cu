@@ -3,15 +3,16 @@
 // Quantizer: "LLM Quantization: 160GB Model on a Laptop", sections "Symmetric
 // Quantization" and "Asymmetric Quantization"; integer zero point as in "CMU
 // 11-868 L19-L20 Model Quantization", section "absmax and zero-point"; one
-// step and zero per 128 input channels of a row ("Quantising Large Language
-// Models for Efficient Inference", "Post-training methods for 4-bit weights").
+// step and zero per group of 32, 64 or 128 input channels of a row
+// ("Quantising Large Language Models for Efficient Inference", "Post-training
+// methods for 4-bit weights").
 // Optional AWQ input-channel scaling W * diag(s) first ("MIT 6.5940 Lab 4 +
 // Lab 5", "Question 2").
 //
-// Mapping: a lane unit is 32 consecutive input channels of one group, four
+// Mapping: a lane unit is 32 consecutive input channels of one group, g / 32
 // lanes per group (four 16-byte loads of W; one 16-byte store of 4-bit codes,
-// or the three words of a 3-bit chunk); the group's range is reduced with two
-// xor-shuffles. One wave of resident CTAs walks the units grid-stride, the
+// or the three words of a 3-bit chunk); the group's range is reduced with
+// log2(g / 32) xor-shuffles (none for g = 32). One wave of resident CTAs walks the units grid-stride, the
 // next unit's loads in flight while the current one is quantized. Per weight:
 // the correctly rounded quotient without a division (group_quotient), rint by
 // the 1.5 * 2^23 addition (both on packed fp32 pairs, two channels per

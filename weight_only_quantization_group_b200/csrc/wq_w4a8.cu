@@ -9,6 +9,9 @@
 //                     the oracle's operation order
 //   w4a8_gemv_kernel  y[m][n] = sum_g (step[n][g] / mult[m][g]) *
 //                     sum_{k in g} (q[n][k] - zero[n][g]) * code[m][k]
+//                     for K > 8192; up to K = 8192 the row-streaming GEMV
+//                     computes the same sums with its ActW4A8 class
+//                     (wq_gemv_rows.cu)
 //
 // The group sums are integer dot products: a packed word's 8 codes are two
 // words of 4 unsigned bytes after one AND and one shift-AND (byte order of
@@ -19,9 +22,9 @@
 // scale cannot ride inside a tensor-core accumulator (both operands change
 // scale every group), so this path is the CUDA cores' int8 dot product.
 //
-// Mapping: every resident CTA slot gets a CTA; each stages the M rows of
-// activation codes (permuted) with their per-32-channel code sums and
-// 1 / mult in shared memory; a warp takes one output row at a time (rows
+// Mapping (w4a8_gemv_kernel): every resident CTA slot gets a CTA; each
+// stages the M rows of activation codes (permuted) with their per-32-channel
+// code sums and 1 / mult in shared memory; a warp takes one output row at a time (rows
 // grid-strided over the warps), lane l channels 32 l + 1024 j of it (one
 // 32-channel group fragment per 1024-channel slice), one 16-byte load of
 // packed weight per slice, eight slices' loads issued together.
