@@ -118,7 +118,7 @@ size_t wq_packed_words(int64_t N, int64_t K, const wq_quant_cfg* cfg);
  * optional AWQ scaling W * diag(s) (s_dev: fp16 [K], or NULL for none;
  * "MIT 6.5940 Lab 4 + Lab 5", section "Question 2"), and writes packed_dev
  * (uint32, wq_packed_words(N,K,cfg) words), steps_dev and zeros_dev (fp16
- * [N][K/128] each). One kernel launch. A step that is not finite in fp16
+ * [N][K/group_size] each). One kernel launch. A step that is not finite in fp16
  * (a group holding an infinite or NaN weight, or a range too large for fp16)
  * latches WQ_ERR_RANGE in the device flag; that group's codes are then
  * unspecified. */
@@ -132,9 +132,11 @@ int32_t wq_unpack_dequant(const uint32_t* packed_dev, const void* steps_dev,
                           const void* zeros_dev, int64_t N, int64_t K,
                           const wq_quant_cfg* cfg, void* W_out_dev, void* stream);
 
-/* Workspace the matmul needs for (M, N, K, cfg), in bytes (currently 0:
- * split-K partial sums are reduced on chip through thread-block-cluster
- * shared memory). */
+/* Size in bytes of the optional matmul workspace for (M, N, K, cfg): the
+ * tensor-core kernel's stream-K schedule (64 KB of arrival counters, then two
+ * fp32 partial tiles of 128 x M rounded up to 16 per CTA of the persistent
+ * grid); 0 when M < 3 (the GEMV kernels take none) or the config is
+ * invalid. The matmul runs without it as well. */
 size_t wq_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, const wq_quant_cfg* cfg);
 
 /* S5/S6 -- weight-only matmul Y = X * deq(W)^T.

@@ -390,6 +390,8 @@ def wq_unpack_dequant(packed: torch.Tensor, steps: torch.Tensor, zeros: torch.Te
 
 def wq_gemm_workspace_bytes(M: int, N: int, K: int, *, bits: int = 4, group_size: int = 128,
                             symmetric: bool = False) -> int:
+    """Bytes of the optional matmul workspace (the tensor-core kernel's stream-K
+    schedule); 0 when M < 3. Allocate it zero-filled once and reuse it."""
     c = _cfg(bits, group_size, symmetric)
     return int(_lib.wq_gemm_workspace_bytes(M, N, K, ctypes.byref(c)))
 
@@ -397,7 +399,12 @@ def wq_gemm_workspace_bytes(M: int, N: int, K: int, *, bits: int = 4, group_size
 def wq_w4a16_gemm(X: torch.Tensor, packed: torch.Tensor, steps: torch.Tensor, zeros: torch.Tensor, N: int, *,
                   bits: int = 4, group_size: int = 128, symmetric: bool = False, out=None, workspace=None,
                   stream=None):
-    """Y[M][N] = X[M][K] * deq(W)^T with fp32 accumulation; returns Y (fp16)."""
+    """Y[M][N] = X[M][K] * deq(W)^T with fp32 accumulation; returns Y (fp16).
+
+    `workspace` (optional): a zero-filled uint8 CUDA tensor of at least
+    wq_gemm_workspace_bytes(M, N, K, ...) bytes, reusable across calls on one
+    stream; with it the tensor-core kernel spreads its stages evenly over the
+    SMs (stream-K) for M <= 16."""
     _check(X, torch.float16, "X")
     c = _cfg(bits, group_size, symmetric)
     _gemm_operands(X, packed, steps, zeros, N, c, out)
