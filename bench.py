@@ -9,10 +9,16 @@ cache, so every step streams its weights from HBM. Each block copy's seven
 launches are one CUDA graph.
 
 The headline `value` is the effective bandwidth of the step: algorithmic bytes
-(packed weights + fp16 steps + fp16 zeros + X + Y) / device time. `rows`
-carries the other hot-path rows measured in the same run (quantize + pack,
-single-shape GEMVs incl. the 3-bit and 8192x28672 cases, the small-M sweep,
-the AWQ search). `roofline` divides by the measured HBM copy bandwidth.
+(packed weights + fp16 steps + fp16 zeros + X + Y) / device time. The last
+stdout line is that headline with `roofline` (against the measured HBM copy
+bandwidth, with the DRAM traffic ncu recorded for the kernel's current
+source), `e2e` (the public calls from pinned host buffers), `cpu_baseline`
+(the oracle on 1 and all host cores), `clocks` and `gpu_launches`. The line
+before it carries `rows`, the other hot-path rows measured in the same run:
+quantize + pack, the block with q|k|v and gate|up packed, single-shape GEMVs
+(3-bit, groups of 32/64, 8192x28672), the small-M sweep with and without the
+GEMM workspace, dense fp16 matmuls for context, W4A8, the AWQ search (fused,
+two-kernel, 3-bit pipeline), the scale fold and GPTQ.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
