@@ -608,8 +608,9 @@ __device__ __forceinline__ float group_first_reduce(float (&v)[NV], int lane, in
 // At most 8 warps: K <= 8192 with 32 channels per lane, K <= 16384 with 64.
 // MINB: minimum CTAs per SM for the register allocation: 3 (85 registers)
 // for the M = 1, 32-channel, two-stage instance, 2 (128 registers) for the
-// other M = 1 instances (each measured faster, more CTAs per SM), 1 for M = 2
-// (a cap would spill).
+// other M = 1 instances (each measured faster, more CTAs per SM), for W4A8
+// with 2-4 rows of X and for the M = 2, 32-channel, two-stage offset-sum
+// instance; 1 for the other M > 1 instances (a cap would spill).
 template <int M, int R, int CPL, int S, int BITS, template <int, int> class Act, int MINB = 1, int GS = kGroup>
 __global__ void __launch_bounds__(256, MINB)
 gemv_rows_kernel(RowsArgs a) {
