@@ -15,7 +15,11 @@ import pytest
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
-# (what the mistake is, exact text in oracle/wq_oracle.py, replacement)
+# (what the mistake is, exact text in oracle/wq_oracle.py, replacement).
+# Not listed, because it is no mistake: computing the stored fold's quotient
+# in fp64 instead of fp32 before the fp16 rounding gives the same fp16 value
+# for every pair of fp16 operands (test_fold_fp16_is_the_correctly_rounded_
+# quotient_exhaustive), so no pin can tell the two apart.
 MUTANTS = [
     ("symmetric codes rounded down instead of to nearest",
      "qs = np.clip(np.rint(wg / sf), -qmax - 1, qmax)", "qs = np.clip(np.floor(wg / sf), -qmax - 1, qmax)"),
@@ -75,6 +79,36 @@ MUTANTS = [
     ("W4A8 scale multiplies by the activation multiplier",
      "scale = steps.astype(np.float64)[None, :, :] / mult.astype(np.float64)[:, None, :]",
      "scale = steps.astype(np.float64)[None, :, :] * mult.astype(np.float64)[:, None, :]"),
+    ("asymmetric codes subtract the zero point",
+     "q = np.rint(wg / sf32[:, :, None]).astype(np.int32) + zero[:, :, None]",
+     "q = np.rint(wg / sf32[:, :, None]).astype(np.int32) - zero[:, :, None]"),
+    ("asymmetric Q off by one", "        Q = (1 << bits) - 1\n        mn", "        Q = (1 << bits)\n        mn"),
+    ("asymmetric all-zero group without the step-1 rule",
+     "step_h = np.where(r == 0, np.float16(1.0), step_h)", "step_h = step_h"),
+    ("symmetric all-zero group without the step-1 rule",
+     "step_h = np.where(amax == 0, np.float16(1.0), step_h)", "step_h = step_h"),
+    ("4-bit unpack keeps 3 bits",
+     "out[:, :, 2 * j] = (w >> np.uint32(4 * j)) & 0xF", "out[:, :, 2 * j] = (w >> np.uint32(4 * j)) & 0x7"),
+    ("alpha grid divided by n - 1",
+     "return np.arange(n_alpha, dtype=np.float64) / float(n_alpha)",
+     "return np.arange(n_alpha, dtype=np.float64) / float(n_alpha - 1)"),
+    ("no floor on mu", "m = np.maximum(np.asarray(mu, dtype=np.float64), MU_FLOOR)",
+     "m = np.asarray(mu, dtype=np.float64)"),
+    ("AWQ loss over the first linear only",
+     "        total += float(np.sum(P * P))\n    return total",
+     "        total += float(np.sum(P * P))\n        break\n    return total"),
+    ("linear fold leaves the bias", "bf = None if b is None else np.asarray(b, dtype=np.float64) / s64",
+     "bf = None if b is None else np.asarray(b, dtype=np.float64)"),
+    ("GPTQ code with the zero point's sign flipped",
+     "q = np.rint(w32 / sf).astype(np.int32) + zero_h.astype(np.int32)",
+     "q = np.rint(w32 / sf).astype(np.int32) - zero_h.astype(np.int32)"),
+    ("GPTQ group parameters from the original weights",
+     "gc, gs, gz = quantize_groups_f32(W[:, i:i + group].astype(np.float32), bits, group, symmetric)",
+     "gc, gs, gz = quantize_groups_f32(np.asarray(W16)[:, i:i + group].astype(np.float32), bits, group, symmetric)"),
+    ("GPTQ keeps the weights of dead channels", "    W[:, dead] = 0.0\n", "    pass\n"),
+    ("W4A8 all-zero activation group with multiplier 0",
+     "mult = np.where(amax == 0, np.float32(1.0), np.float32(127.0)",
+     "mult = np.where(amax == 0, np.float32(0.0), np.float32(127.0)"),
     ("W4A8 without the zero point",
      "qw = codes.astype(np.int64).reshape(N, G, group) - zeros.astype(np.int64)[:, :, None]",
      "qw = codes.astype(np.int64).reshape(N, G, group)"),

@@ -153,6 +153,10 @@ def test_quantizer_error_bound_and_code_range(bits, symmetric):
     err = np.abs(deq - w.astype(np.float64))
     assert np.all(err <= stepk * (0.5 + 2.0 ** -20))
     assert np.all(deq[-1, :128] == 0)
+    # the all-zero group: step 1 (the reading of [CMU]'s range := 1), its
+    # codes at the zero point (0 asymmetric, 2^(b-1) symmetric)
+    zp = (1 << (bits - 1)) if symmetric else 0
+    assert steps[-1, 0] == 1 and zeros[-1, 0] == zp and np.all(codes[-1, :128] == zp)
 
 
 @pytest.mark.parametrize("symmetric", [False, True])
@@ -463,6 +467,45 @@ def test_fold_fp16_within_half_ulp_of_exact_quotient():
                 Fraction(_fp16_half_ulp(float(exact))) * (1 + Fraction(1, 2 ** 12))
         exact = Fraction(float(b[n])) / Fraction(float(sr[n]))
         assert abs(Fraction(float(bf[n])) - exact) <= Fraction(_fp16_half_ulp(float(exact))) * (1 + Fraction(1, 2 ** 12))
+
+
+def test_fold_fp16_is_the_correctly_rounded_quotient_exhaustive():
+    """The stored fold fp16_rn(fp32_rn(gamma / s)) is the correctly rounded
+    fp16 quotient for every positive finite fp16 dividend and every fp16
+    divisor in [1, 2) (other divisors differ by a power of two). Reference:
+    the fp64 quotient rounded to fp16, which is correctly rounded because a
+    quotient of two fp16 values lies about 2^-23 (relative) or more from any
+    fp16 rounding midpoint, far beyond fp64's rounding error; a sample of
+    it is checked against exact fractions."""
+    allw = np.arange(1, 0x7C00, dtype=np.uint16).view(np.float16)
+    s = (np.arange(1024, 2048) / 1024).astype(np.float16)
+    for k in range(0, len(allw), 4096):
+        w = allw[k:k + 4096]
+        Wv, Sv = np.repeat(w, len(s)), np.tile(s, len(w))
+        got = O.awq_fold_into_norm(Wv, Sv)
+        want = (Wv.astype(np.float64) / Sv.astype(np.float64)).astype(np.float16)
+        assert np.array_equal(got.view(np.uint16), want.view(np.uint16))
+    rng = np.random.default_rng(5)
+    for _ in range(300):
+        w, sv = allw[rng.integers(len(allw))], s[rng.integers(len(s))]
+        exact = Fraction(float(w)) / Fraction(float(sv))
+        r = np.float16(np.float64(w) / np.float64(sv))
+        for nb in (np.nextafter(r, np.float16(np.inf)), np.nextafter(r, np.float16(0))):
+            assert abs(Fraction(float(r)) - exact) <= abs(Fraction(float(nb)) - exact)
+
+
+def test_fold_linear_rows_with_bias_restores_the_consumers_input_fp64():
+    """A linear y = x W^T + b whose output rows absorb diag(s)^-1 feeds a
+    consumer that now reads y' diag(s): y' * s must equal y (fp64, to
+    rounding), bias included; leaving the bias unfolded breaks it."""
+    g = np.random.default_rng(34)
+    W, b = g.normal(0, 0.1, (24, 40)), g.normal(0, 0.5, 24)
+    sv = np.exp(g.normal(0, 1, 24))
+    x = g.normal(0, 1, (9, 40))
+    y = x @ W.T + b
+    Wf, bf = O.awq_fold_into_linear_rows(W, sv, b)
+    assert np.max(np.abs((x @ Wf.T + bf) * sv[None, :] - y)) <= 1e-13 * np.max(np.abs(y))
+    assert np.max(np.abs((x @ Wf.T + b) * sv[None, :] - y)) > 1e-2 * np.max(np.abs(y))
 
 
 def test_fold_fp16_hand_values():
