@@ -155,8 +155,9 @@ size_t wq_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, const wq_quant_c
  * its work over all SMs (stream-K: every CTA of a persistent grid takes the
  * same number of K stages, at most one row tile's worth; a tile split between
  * CTAs is summed from their fp32 partial tiles in CTA order, so the result
- * does not depend on timing) for M <= 16 (WQ_OPT_TC_STREAMK). Its first 64 KB hold
- * arrival counters that every completed call leaves at zero, so calls of any
+ * does not depend on timing) for M <= 16 (WQ_OPT_TC_STREAMK). Its first
+ * 64 KB hold arrival counters that every completed call leaves at zero, so
+ * calls of any
  * shape may share one workspace as long as they do not overlap in time (same
  * stream); after a call that ended in WQ_ERR_TIMEOUT, zero-fill it again.
  * Without a workspace: one CTA per row tile (and K split over thread-block
@@ -192,8 +193,8 @@ int32_t wq_w4a16_gemm(const void* X_dev, const uint32_t* packed_dev, const void*
  * initial contents required. The size depends on WQ_OPT_AWQ_LOSS when it is
  * asked for: the two-kernel path keeps the error matrices of a batch of
  * alphas (up to 1 GiB), the fused path none; a workspace too small for the
- * path selected at the call returns WQ_ERR_WORKSPACE. A non-finite candidate or loss latches
- * WQ_ERR_RANGE in the device flag. */
+ * path selected at the call returns WQ_ERR_WORKSPACE. A non-finite
+ * candidate or loss latches WQ_ERR_RANGE in the device flag. */
 size_t wq_awq_workspace_bytes(int64_t T, int64_t K, const int64_t* N_i, int32_t n_lin, int32_t n_alpha,
                               const wq_quant_cfg* cfg);
 int32_t wq_awq_scale_search(const void* X_dev, int64_t T, int64_t K, const void* const* W_dev,
@@ -219,8 +220,9 @@ int32_t wq_awq_scale_search(const void* X_dev, int64_t T, int64_t K, const void*
  * primary context) -- the kept address would no longer be valid. With the
  * default fused loss path only the per-tile partial losses live in the
  * array; the two-kernel path also builds the error matrix there, one alpha
- * and at most 16 MiB of rows at a time. All calls share the array, which keeps the last call's contents
- * (nothing in it has to start at zero), so calls that overlap on the GPU --
+ * and at most 16 MiB of rows at a time. All calls share the array, which
+ * keeps the last call's contents (nothing in it has to start at zero), so
+ * calls that overlap on the GPU --
  * from other streams or threads -- race and must be serialized by the caller.
  * Limits: K <= 16384, n_alpha <= 64 and
  * n_alpha * ceil(T/128) * ceil(sum_i N_i / 128) <= 786432; a larger problem
