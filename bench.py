@@ -421,7 +421,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
 
     rows = {}
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    if rank == 0 and not args.no_rows:
+    if rank == 0 and world == 1 and not args.no_rows:
         # the same graphs' step time with programmatic dependent launch off
         wq.wq_set_option(wq.WQ_OPT_PDL, 0)
         try:
@@ -532,9 +532,10 @@ def run_ours(args, rank: int, world: int, local_rank: int):
                          "out, stream sync per step"),
                 "eager_value": round(world * step_bytes * e2e_steps / (e2e_eager_ms * 1e-3) / 1e9, 2),
                 "eager_ms_per_step": e2e_eager_ms / e2e_steps},
-        "gpu_launches": 7 * args.steps,
+        "gpu_launches": 7 * args.steps * world,  # all ranks' launches in the timed region
         "clocks": clocks,
-        "rows_line": "printed on the line before this one" if rows else "not measured (--no-rows)",
+        "rows_line": ("printed on the line before this one" if rows else
+                      "measured at N = 1 only" if world > 1 else "not measured (--no-rows)"),
     }
     if "block_step_fused_4_launches" in rows:
         f = rows["block_step_fused_4_launches"]
@@ -543,7 +544,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
             "frac": round(f["frac_hbm"], 4),
             "note": "the same 7 linears and bytes, q|k|v and gate|up each packed as one weight (they share an "
                     "input): 4 launches per step"}
-    if not args.no_cpu_baseline:
+    if not args.no_cpu_baseline and world == 1:  # the host baseline: rank 0 at N = 1 only
         line["cpu_baseline"] = cpu_baseline(cases, args.cpu_seconds)
     return line, rows
 
