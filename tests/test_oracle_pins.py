@@ -397,6 +397,23 @@ def test_awq_search_picks_minimum_and_beats_rtn():
 # AWQ scale folding ("MIT 6.5940 Lab 4 + Lab 5", "Question 2")
 # ---------------------------------------------------------------------------
 
+
+def test_awq_loss_falls_then_rises_over_alpha():
+    """Too large a scale inflates the group maximum, so the loss over alpha
+    falls and then rises ("MIT 6.5940 Lab 4 + Lab 5", "How to self-study it":
+    the turning point of the scale sweep): with a few outlier input channels
+    the best alpha is interior and the largest alpha loses to alpha = 0."""
+    g = np.random.default_rng(3)
+    K, N, T = 256, 64, 64
+    X = g.normal(0, 1, (T, K))
+    X[:, g.choice(K, 3, replace=False)] *= 20
+    W = g.normal(0, 0.02, (N, K))
+    r = O.awq_search(X.astype(np.float16), [W.astype(np.float16)], 4, 128, False)
+    L, best = r["losses"], r["best"]
+    assert 0 < best < len(L) - 1
+    assert L[0] > 1.5 * L[best] and L[-1] > 3.0 * L[best] and L[-1] > L[0]
+    assert np.all(np.diff(L[best:]) > 0)      # rises steadily past the turning point
+
 def _block_params(g, D=64, H=96):
     return {"gamma1": 1.0 + 0.1 * g.standard_normal(D), "wq": g.normal(0, 0.1, (D, D)),
             "wk": g.normal(0, 0.1, (D, D)), "wv": g.normal(0, 0.1, (D, D)), "wo": g.normal(0, 0.1, (D, D)),
