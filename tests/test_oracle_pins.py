@@ -393,11 +393,6 @@ def test_awq_search_picks_minimum_and_beats_rtn():
     assert r["losses"][r["best"]] == O.awq_loss(X, Ws, r["s"], 4, 128, False)
 
 
-# ---------------------------------------------------------------------------
-# AWQ scale folding ("MIT 6.5940 Lab 4 + Lab 5", "Question 2")
-# ---------------------------------------------------------------------------
-
-
 def test_awq_loss_falls_then_rises_over_alpha():
     """Too large a scale inflates the group maximum, so the loss over alpha
     falls and then rises ("MIT 6.5940 Lab 4 + Lab 5", "How to self-study it":
@@ -413,6 +408,12 @@ def test_awq_loss_falls_then_rises_over_alpha():
     assert 0 < best < len(L) - 1
     assert L[0] > 1.5 * L[best] and L[-1] > 3.0 * L[best] and L[-1] > L[0]
     assert np.all(np.diff(L[best:]) > 0)      # rises steadily past the turning point
+
+
+# ---------------------------------------------------------------------------
+# AWQ scale folding ("MIT 6.5940 Lab 4 + Lab 5", "Question 2")
+# ---------------------------------------------------------------------------
+
 
 def _block_params(g, D=64, H=96):
     return {"gamma1": 1.0 + 0.1 * g.standard_normal(D), "wq": g.normal(0, 0.1, (D, D)),
