@@ -57,6 +57,21 @@ def _cfg(wq, bits=4, group=128, sym=0):
     return wq._Cfg(bits, group, sym)
 
 
+def _cuda_device_present():
+    try:
+        import torch
+        return torch.cuda.is_available()
+    except Exception:
+        return False
+
+
+# The validation tests pass fake device addresses that every call must reject
+# before it touches CUDA; on a machine with a GPU they do not run, so that a
+# check that wrongly passed could never launch a kernel on them.
+fake_pointers = pytest.mark.skipif(_cuda_device_present(), reason="fake device addresses: host-only")
+
+
+@fake_pointers
 def test_argument_validation_without_gpu(wq):
     L = wq.lib()
     good = 0x10000  # a fake, 16-byte aligned address; validation fails before any use
@@ -93,6 +108,77 @@ def test_argument_validation_without_gpu(wq):
     assert L.wq_awq_fold_linear_rows(good, good, good, 4, 8, good, None, None) == wq.WQ_ERR_INVALID_ARG
     assert L.wq_awq_fold_linear_rows(good, None, good, 0, 8, good, None, None) == wq.WQ_ERR_INVALID_ARG
     assert L.wq_awq_fold_linear_rows(good, None, good + 1, 4, 8, good, None, None) == wq.WQ_ERR_ALIGNMENT
+
+
+@fake_pointers
+def test_search_gptq_and_w4a8_validation_without_gpu(wq):
+    """AWQ search, GPTQ, int8 activations and W4A8: every argument check
+    returns its status before anything touches CUDA."""
+    L = wq.lib()
+    good = 0x10000
+    by = ctypes.byref
+    c = _cfg(wq)
+    VP = ctypes.c_void_p
+    # AWQ search: W_dev is a host array of device pointers
+    W2 = (VP * 2)(good, good)
+    N2 = (ctypes.c_int64 * 2)(128, 256)
+    al = (ctypes.c_double * 3)(0.0, 0.05, 0.1)
+
+    def search(X=good, T=64, K=256, W=W2, N=N2, n_lin=2, cfg=c, alpha=al, n_alpha=3, s_out=good,
+               mu=None, loss=None, best=None, ws=good, ws_bytes=1 << 30):
+        return L.wq_awq_scale_search(X, T, K, W, N, n_lin, by(cfg) if cfg is not None else None, alpha, n_alpha,
+                                     s_out, mu, loss, best, ws, ws_bytes, None)
+
+    assert search(cfg=_cfg(wq, group=64)) == wq.WQ_ERR_UNSUPPORTED        # AWQ: groups of 128
+    assert search(cfg=None) == wq.WQ_ERR_INVALID_ARG
+    assert search(T=0) == wq.WQ_ERR_INVALID_ARG
+    assert search(K=200) == wq.WQ_ERR_INVALID_ARG
+    assert search(n_lin=0) == wq.WQ_ERR_INVALID_ARG and search(n_lin=9) == wq.WQ_ERR_INVALID_ARG
+    assert search(n_alpha=0) == wq.WQ_ERR_INVALID_ARG and search(n_alpha=65) == wq.WQ_ERR_INVALID_ARG
+    assert search(N=(ctypes.c_int64 * 2)(128, 0)) == wq.WQ_ERR_INVALID_ARG
+    assert search(X=None) == wq.WQ_ERR_INVALID_ARG and search(s_out=None) == wq.WQ_ERR_INVALID_ARG
+    assert search(W=(VP * 2)(good, None)) == wq.WQ_ERR_INVALID_ARG
+    assert search(W=(VP * 2)(good, good + 8)) == wq.WQ_ERR_ALIGNMENT
+    assert search(alpha=(ctypes.c_double * 3)(0.0, float("nan"), 0.1)) == wq.WQ_ERR_INVALID_ARG
+    assert search(X=good + 8) == wq.WQ_ERR_ALIGNMENT
+    assert search(loss=good + 4) == wq.WQ_ERR_ALIGNMENT and search(best=good + 2) == wq.WQ_ERR_ALIGNMENT
+    assert search(ws=None) == wq.WQ_ERR_WORKSPACE
+    need = L.wq_awq_workspace_bytes(64, 256, N2, 2, 3, by(c))
+    assert need > 0 and search(ws_bytes=need - 1) == wq.WQ_ERR_WORKSPACE
+    assert search(ws=good + 128, ws_bytes=need) == wq.WQ_ERR_ALIGNMENT
+    assert L.wq_awq_scale_search_noalloc(good, 64, 32768, W2, N2, 2, by(c), al, 3, good, None, None, None,
+                                         None) == wq.WQ_ERR_WORKSPACE       # K beyond the fixed scratch
+
+    # GPTQ
+    def gptq(X=good, T=64, W=good, N=8, K=256, cfg=c, damp=0.01, packed=good, ws=good, ws_bytes=1 << 30):
+        return L.wq_gptq_quantize_pack(X, T, W, N, K, by(cfg), damp, packed, good, good, ws, ws_bytes, None)
+
+    assert gptq(cfg=_cfg(wq, bits=5)) == wq.WQ_ERR_UNSUPPORTED
+    assert gptq(T=0) == wq.WQ_ERR_INVALID_ARG and gptq(K=100) == wq.WQ_ERR_INVALID_ARG
+    assert gptq(damp=-0.1) == wq.WQ_ERR_INVALID_ARG and gptq(damp=float("nan")) == wq.WQ_ERR_INVALID_ARG
+    assert gptq(X=None) == wq.WQ_ERR_INVALID_ARG
+    assert gptq(packed=good + 4) == wq.WQ_ERR_ALIGNMENT and gptq(W=good + 1) == wq.WQ_ERR_ALIGNMENT
+    need = L.wq_gptq_workspace_bytes(8, 256, by(c))
+    assert need > 0 and gptq(ws_bytes=need - 1) == wq.WQ_ERR_WORKSPACE and gptq(ws=None) == wq.WQ_ERR_WORKSPACE
+    assert gptq(ws=good + 64, ws_bytes=need) == wq.WQ_ERR_ALIGNMENT
+
+    # int8 activations
+    assert L.wq_quantize_act_int8(good, 2, 256, 48, good, good, None) == wq.WQ_ERR_INVALID_ARG
+    assert L.wq_quantize_act_int8(good, 0, 256, 32, good, good, None) == wq.WQ_ERR_INVALID_ARG
+    assert L.wq_quantize_act_int8(good, 2, 80, 32, good, good, None) == wq.WQ_ERR_INVALID_ARG
+    assert L.wq_quantize_act_int8(good, 2, 256, 32, None, good, None) == wq.WQ_ERR_INVALID_ARG
+    assert L.wq_quantize_act_int8(good, 2, 256, 32, good + 2, good, None) == wq.WQ_ERR_ALIGNMENT
+
+    # W4A8
+    c32 = _cfg(wq, group=32)
+
+    def w4a8(q=good, M=2, N=8, K=256, cfg=c32, Y=good):
+        return L.wq_w4a8_gemm(q, good, good, good, good, M, N, K, by(cfg), Y, None)
+
+    assert w4a8(cfg=_cfg(wq, bits=3, group=32)) == wq.WQ_ERR_UNSUPPORTED
+    assert w4a8(K=32768) == wq.WQ_ERR_UNSUPPORTED
+    assert w4a8(M=0) == wq.WQ_ERR_INVALID_ARG and w4a8(Y=None) == wq.WQ_ERR_INVALID_ARG
+    assert w4a8(q=good + 4) == wq.WQ_ERR_ALIGNMENT
 
 
 def test_option_values_are_validated(wq):
