@@ -9,7 +9,9 @@ arguments the quantizer relies on, independent of any CUDA code:
   representable in fp32, and the cases include exact ties and near-ties;
 * rint by adding 1.5 * 2^23 rounds to nearest with ties to even for |x| < 2^22;
 * the dequantized value (level - zero) * step is one exact fma of the offset
-  level with the step and the constant -(1.5 * 2^23) * step.
+  level with the step and the constant -(1.5 * 2^23) * step;
+* GPTQ's factor Cholesky(H^-1)^T is the inverse of the "UL" factor of H,
+  the route the GPU takes without forming H^-1 (fp64).
 """
 import random
 from fractions import Fraction as F
@@ -187,3 +189,32 @@ def test_corrected_quotient_fold_operands():
     for w in (65504.0, -65504.0, 2.0 ** -24, -(2.0 ** -24), 1.0):
         for s in (2.0 ** -24, -(2.0 ** -24), 65504.0, -65504.0, 3.0, 2.0 ** -14):
             assert corrected_quotient_ok(w, s), (w, s)
+
+
+def test_gptq_factor_from_the_ul_factorization():
+    """The GPU's route to GPTQ's factor: the "UL" factorization H = U U^T
+    with U upper triangular (computed from the bottom-right corner), then
+    G = U^-1. G is upper triangular with a positive diagonal and
+    G^T G = U^-T U^-1 = H^-1, so by the uniqueness of the Cholesky factor it
+    is the page's Cholesky(H^-1)^T, reached without forming H^-1 (fp64)."""
+    g = np.random.default_rng(9)
+    K = 48
+    X = g.normal(0, 1, (200, K)) @ (np.eye(K) + 0.3 * g.normal(0, 1, (K, K)))
+    H = 2.0 * X.T @ X
+    H += 0.01 * np.mean(np.diag(H)) * np.eye(K)
+    # UL by columns from the last: U[j][j] = sqrt(H[j][j] - sum_{k>j} U[j][k]^2),
+    # U[i][j] = (H[i][j] - sum_{k>j} U[i][k] U[j][k]) / U[j][j] for i < j
+    U = np.zeros((K, K))
+    for j in range(K - 1, -1, -1):
+        U[j, j] = np.sqrt(H[j, j] - U[j, j + 1:] @ U[j, j + 1:])
+        for i in range(j):
+            U[i, j] = (H[i, j] - U[i, j + 1:] @ U[j, j + 1:]) / U[j, j]
+    assert np.allclose(np.triu(U), U) and np.all(np.diag(U) > 0)
+    assert np.max(np.abs(U @ U.T - H)) <= 1e-12 * np.max(np.abs(H))
+    G = np.linalg.solve(U, np.eye(K))               # U^-1, upper triangular
+    ref = np.linalg.cholesky(np.linalg.inv(H)).T     # the page's factor
+    assert np.allclose(np.triu(G), G, atol=1e-14 * np.max(np.abs(G)))
+    assert np.max(np.abs(G - ref)) <= 1e-9 * np.max(np.abs(ref))
+    # the ordinary (LU-order) Cholesky factor of H does not give it
+    L = np.linalg.cholesky(H)
+    assert np.max(np.abs(np.linalg.inv(L).T - ref)) > 1e-3 * np.max(np.abs(ref))
