@@ -1,5 +1,5 @@
-"""Exact-arithmetic checks (CPU, rational numbers) of the two rounding
-arguments the quantizer relies on, independent of any CUDA code:
+"""Arithmetic checks (CPU; exact rational numbers where rounding decides) of
+the arguments the CUDA path relies on, independent of any CUDA code:
 
 * the quotient w / step is formed without a division as
   q0 = RN(w y), r = w - step q0, q = RN(q0 + r y) (Markstein's correction),
