@@ -299,6 +299,7 @@ def _raise(st: int, where: str):
 
 
 def wq_layout_version() -> int:
+    """Version of the packed layout (codes, steps, zeros) this library writes and reads."""
     return int(lib().wq_layout_version())
 
 
@@ -330,14 +331,17 @@ def load_packed(path, device=None):
 
 
 def wq_abi_version() -> int:
+    """ABI version of the loaded libwq.so."""
     return int(_lib.wq_abi_version())
 
 
 def wq_status_string(status: int) -> str:
+    """Name and meaning of a status code."""
     return _lib.wq_status_string(int(status)).decode()
 
 
 def wq_packed_words(N: int, K: int, bits: int = 4, group_size: int = 128, symmetric: bool = False) -> int:
+    """uint32 words of the packed [N][K] weight (N*K/8 at 4 bits, 3*N*K/32 at 3); 0 if invalid."""
     c = _cfg(bits, group_size, symmetric)
     return int(_lib.wq_packed_words(N, K, ctypes.byref(c)))
 
@@ -433,11 +437,14 @@ def wq_set_option(option: int, value: int) -> None:
 
 
 def wq_get_option(option: int) -> int:
+    """Current value of a process-wide option (WQ_OPT_*)."""
     return int(_lib.wq_get_option(int(option)))
 
 
 def wq_awq_workspace_bytes(T: int, K: int, Ns, n_alpha: int = 20, *, bits: int = 4, group_size: int = 128,
                            symmetric: bool = False) -> int:
+    """Workspace bytes of wq_awq_scale_search for T calibration rows, K input channels and
+    the linears' output sizes Ns (for the loss path WQ_OPT_AWQ_LOSS selects now); 0 if invalid."""
     c = _cfg(bits, group_size, symmetric)
     arr = (ctypes.c_int64 * len(Ns))(*[int(n) for n in Ns])
     return int(_lib.wq_awq_workspace_bytes(T, K, arr, len(Ns), n_alpha, ctypes.byref(c)))
@@ -563,6 +570,7 @@ def wq_awq_fold_linear_rows(W: torch.Tensor, s: torch.Tensor, b: torch.Tensor | 
 
 
 def wq_gptq_workspace_bytes(N: int, K: int, *, bits: int = 4, group_size: int = 128, symmetric: bool = False) -> int:
+    """Workspace bytes of wq_gptq_quantize_pack for an [N][K] weight; 0 if invalid."""
     c = _cfg(bits, group_size, symmetric)
     return int(_lib.wq_gptq_workspace_bytes(N, K, ctypes.byref(c)))
 
